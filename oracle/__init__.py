@@ -1,0 +1,167 @@
+"""Double-precision CPU oracle for the VQ decode linear (test infrastructure).
+
+Only the test suite, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the CUDA library and
+its Python binding) never imports, links or calls it.
+
+The arithmetic lives in ``eva_oracle.c`` (plain C, double); this module only
+compiles it with gcc and marshals numpy arrays through ctypes.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "eva_oracle.c")
+_LIB = os.path.join(_HERE, "libeva_oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile eva_oracle.c into libeva_oracle.so next to it (gcc, -fopenmp)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
+               "-o", _LIB + ".tmp", _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(_LIB + ".tmp", _LIB)
+    return _LIB
+
+
+class _Desc(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int), ("K", ctypes.c_int), ("d", ctypes.c_int),
+                ("ncent", ctypes.c_int), ("codebook_rows", ctypes.c_int),
+                ("residual_group", ctypes.c_int), ("hadamard_block", ctypes.c_int)]
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        lib.vq_oracle_f16_to_f64.argtypes = [ctypes.c_uint16]
+        lib.vq_oracle_f16_to_f64.restype = ctypes.c_double
+        lib.vq_oracle_f16_array_to_f64.argtypes = [P, ctypes.c_int64, P]
+        lib.vq_oracle_f16_array_to_f64.restype = None
+        lib.vq_oracle_hadamard.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, P]
+        lib.vq_oracle_hadamard.restype = ctypes.c_int
+        lib.vq_oracle_linear.argtypes = [ctypes.POINTER(_Desc), P, P, P, P, P, P,
+                                         ctypes.c_int, P, ctypes.c_int]
+        lib.vq_oracle_linear.restype = ctypes.c_int
+        lib.vq_oracle_lookup_form.argtypes = [ctypes.POINTER(_Desc), P, P, P, P, P, P,
+                                              ctypes.c_int, P, P]
+        lib.vq_oracle_lookup_form.restype = ctypes.c_int
+        lib.vq_oracle_optimal_alpha.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int, P]
+        lib.vq_oracle_optimal_alpha.restype = ctypes.c_int
+        lib.vq_oracle_max_threads.argtypes = []
+        lib.vq_oracle_max_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c16(a):
+    return None if a is None else np.ascontiguousarray(a, dtype=np.float16).view(np.uint16)
+
+
+def f16_to_f64(h) -> np.ndarray:
+    """Decode fp16 values (array of float16 or uint16 bit patterns) into float64."""
+    h = np.ascontiguousarray(h)
+    bits = h.view(np.uint16) if h.dtype == np.float16 else h.astype(np.uint16)
+    bits = np.ascontiguousarray(bits)
+    out = np.empty(bits.shape, np.float64)
+    _load().vq_oracle_f16_array_to_f64(_ptr(bits), bits.size, _ptr(out))
+    return out
+
+
+def hadamard(x, hsign, b: int) -> np.ndarray:
+    """x~ = hsign * (H_b x) / sqrt(b) per block; x fp16 [B][K] -> float64 [B][K]."""
+    x16 = _c16(np.atleast_2d(x))
+    B, K = x16.shape
+    hs = None if hsign is None else np.ascontiguousarray(hsign, dtype=np.int8)
+    out = np.empty((B, K), np.float64)
+    rc = _load().vq_oracle_hadamard(_ptr(x16), _ptr(hs), B, K, int(b), _ptr(out))
+    if rc:
+        raise ValueError(f"vq_oracle_hadamard: {rc}")
+    return out
+
+
+def _desc(N, K, d, ncent, codebook_rows, residual_group, hadamard_block):
+    return _Desc(int(N), int(K), int(d), int(ncent), int(codebook_rows),
+                 int(residual_group), int(hadamard_block))
+
+
+def _prep(wc, wi, signs, alpha, hsign, x, codebook_rows, residual_group, hadamard_block):
+    wc16 = _c16(wc)
+    if wc16.ndim == 2:
+        wc16 = wc16[None]
+    G, ncent, d = wc16.shape
+    wi8 = np.ascontiguousarray(wi, dtype=np.uint8)
+    N, J = wi8.shape
+    x16 = _c16(np.atleast_2d(x))
+    B, K = x16.shape
+    if J * d != K:
+        raise ValueError("WI width times d must equal K")
+    if (N // codebook_rows if codebook_rows else 1) != G:
+        raise ValueError("codebook count does not match codebook_rows")
+    sg = None if signs is None else np.ascontiguousarray(signs, dtype=np.uint8)
+    al = _c16(alpha)
+    hs = None if hsign is None else np.ascontiguousarray(hsign, dtype=np.int8)
+    desc = _desc(N, K, d, ncent, codebook_rows, residual_group, hadamard_block)
+    return desc, wc16, wi8, sg, al, hs, x16, B, N
+
+
+def linear(wc, wi, x, *, signs=None, alpha=None, hsign=None, codebook_rows=0,
+           residual_group=0, hadamard_block=0, nthreads=1) -> np.ndarray:
+    """y [B][N] float64: the dequantised-weight product (the plain definition)."""
+    desc, wc16, wi8, sg, al, hs, x16, B, N = _prep(
+        wc, wi, signs, alpha, hsign, x, codebook_rows, residual_group, hadamard_block)
+    y = np.empty((B, N), np.float64)
+    rc = _load().vq_oracle_linear(ctypes.byref(desc), _ptr(wc16), _ptr(wi8), _ptr(sg), _ptr(al),
+                                  _ptr(hs), _ptr(x16), B, _ptr(y), int(nthreads))
+    if rc:
+        raise ValueError(f"vq_oracle_linear: {rc}")
+    return y
+
+
+def lookup_form(wc, wi, x, *, signs=None, alpha=None, hsign=None, codebook_rows=0,
+                residual_group=0, hadamard_block=0):
+    """(y, sum|W x~|) [B][N] float64 via the output-codebook two-step form."""
+    desc, wc16, wi8, sg, al, hs, x16, B, N = _prep(
+        wc, wi, signs, alpha, hsign, x, codebook_rows, residual_group, hadamard_block)
+    y = np.empty((B, N), np.float64)
+    absy = np.empty((B, N), np.float64)
+    rc = _load().vq_oracle_lookup_form(ctypes.byref(desc), _ptr(wc16), _ptr(wi8), _ptr(sg),
+                                       _ptr(al), _ptr(hs), _ptr(x16), B, _ptr(y), _ptr(absy))
+    if rc:
+        raise ValueError(f"vq_oracle_lookup_form: {rc}")
+    return y, absy
+
+
+def optimal_alpha(r, group: int) -> np.ndarray:
+    """argmin_alpha ||r - alpha sign(r)||^2 per row and group of `group` columns."""
+    r = np.ascontiguousarray(r, dtype=np.float64)
+    rows, cols = r.shape
+    out = np.empty((rows, cols // group), np.float64)
+    rc = _load().vq_oracle_optimal_alpha(_ptr(r), rows, cols, int(group), _ptr(out))
+    if rc:
+        raise ValueError(f"vq_oracle_optimal_alpha: {rc}")
+    return out
+
+
+def max_threads() -> int:
+    return int(_load().vq_oracle_max_threads())
+
+
+def layer_linear(layer, x, nthreads=1) -> np.ndarray:
+    """Oracle output for a synth.LayerData and activations x."""
+    s = layer.shape
+    return linear(layer.wc, layer.wi, x, signs=layer.signs, alpha=layer.alpha, hsign=layer.hsign,
+                  codebook_rows=s.codebook_rows, residual_group=s.residual_group,
+                  hadamard_block=s.hadamard_block, nthreads=nthreads)

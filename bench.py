@@ -1,0 +1,370 @@
+#!/usr/bin/env python3
+"""Benchmark of the VQ decode linear on B200: microseconds per layer and the
+achieved HBM bandwidth of the algorithmic weight stream.
+
+A step is one call of the layer (one pass of the whole path, x[B,K] -> y[B,N])
+on one batch of synthetic input.  To keep the weights out of L2 the steps walk
+a ring of distinct layer instances whose index bytes total more than twice the
+L2 size; the ring is captured once in a CUDA graph and replayed.  Steps are
+timed with CUDA events on the launching stream between two barriers.
+
+Default workload: the Llama-2-7B-shaped 4096x4096 2-bit layer at batch 1.
+Multi-GPU (torchrun): every rank runs its own ring (replicas, weak scaling);
+the elapsed time is the maximum over ranks and the value is the total
+work of all ranks divided by it.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                  [--config llama7b_layer] [--layer 0] [--batch 1]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+FALLBACK_HBM_GBS = 6650.0
+METRIC = "µs/layer and achieved HBM GB/s (% of B200 peak), 2-bit VQ linear"
+KERNEL_SOURCES = ("vector_quantized_weight_b200/csrc/eva_vq.cu",
+                  "vector_quantized_weight_b200/csrc/eva_vq_kernels.cuh",
+                  "vector_quantized_weight_b200/csrc/eva_vq_layout.cuh")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=None)
+    ap.add_argument("--impl", default="eva", choices=["eva", "reference"])
+    ap.add_argument("--config", default="llama7b_layer")
+    ap.add_argument("--layer", type=int, default=0)
+    ap.add_argument("--batch", type=int, default=None)
+    ap.add_argument("--ring", type=int, default=0, help="ring length (0: > 2x L2)")
+    ap.add_argument("--path", type=int, default=0)
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    return ap.parse_args()
+
+
+def source_sha() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def load_traffic(workload: str):
+    """dram bytes per launch of the lookup kernel from a committed ncu summary,
+    or None when the kernel sources changed since it was captured."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        e = d.get(workload)
+        if e and e.get("source_sha") == source_sha():
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu = gpu_id
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.15)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm, mx, reasons = [], [], set()
+        for line in (self.out or "").splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def cpu_baseline(shape, B, seed, seconds):
+    """The oracle, as written, on the host cores: whole layers, repeated for
+    about `seconds` of CPU time."""
+    import numpy as np
+    import oracle
+    from vector_quantized_weight_b200 import synth
+    layer = synth.make_layer(shape, seed)
+    x = synth.make_x(shape.K, B, seed)
+    nthreads = os.cpu_count() or 1
+    oracle.layer_linear(layer, x, nthreads=nthreads)     # load + page in
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.layer_linear(layer, x, nthreads=nthreads)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or (reps >= 1 and el * (reps + 1) / reps > 3 * seconds):
+            break
+    us = el / reps * 1e6
+    return us, reps, nthreads
+
+
+def stream_bytes(shape, B):
+    wi = shape.N * shape.J
+    sg = shape.N * shape.K // 8 if shape.residual_group else 0
+    al = shape.N * (shape.K // shape.residual_group) * 2 if shape.residual_group else 0
+    return wi + sg + al + 2 * B * shape.K
+
+
+def run_reference(args, shape, B, seed, world, rank):
+    if rank != 0:
+        return
+    us, reps, threads = cpu_baseline(shape, B, seed, args.cpu_seconds)
+    gbs = stream_bytes(shape, B) / (us * 1e-6) / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s",
+        "us_per_layer": round(us, 3), "n_gpus": args.gpus, "steps": reps, "warmup": 1,
+        "ms_per_step": round(us / 1e3, 6), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{args.config}:{shape.name}", "N": shape.N, "K": shape.K, "batch": B},
+        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{reps} whole-layer oracle calls (dequantise + fp64 GEMV), "
+                                   f"{threads} OpenMP threads over output rows"},
+        "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    world, rank, local = dist_setup()
+    from vector_quantized_weight_b200 import synth
+    cfg = synth.CONFIGS[args.config]
+    shape = cfg.layers[args.layer]
+    B = args.batch or cfg.batches[0]
+    seed = synth.layer_seed(cfg.index, args.layer)
+
+    if args.impl == "reference":
+        run_reference(args, shape, B, seed, world, rank)
+        return
+
+    import numpy as np
+    import torch
+    from vector_quantized_weight_b200 import eva_vq
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist
+
+    props = torch.cuda.get_device_properties(dev)
+    l2 = int(getattr(props, "L2_cache_size", 126 * 2**20) or 126 * 2**20)
+    wi_bytes = shape.N * shape.J
+    ring = args.ring or max(2, math.ceil(2 * l2 / wi_bytes) + 1)
+    steps = args.steps if args.steps is not None else ring * max(1, 400_000 // ring)
+    warmup = max(3, args.warmup if args.warmup is not None else 2 * ring)
+
+    # Ring of distinct layers: each replica draws its own weights (seeded).
+    stream = torch.cuda.Stream(device=dev)
+    layers, xs, ys = [], [], []
+    with torch.cuda.stream(stream):
+        for r in range(ring):
+            lay = synth.make_layer(shape, seed + 1000 * (r + 1) + 7919 * rank)
+            layers.append(eva_vq.from_layer(lay, max_batch=B, path=args.path, device=dev))
+            xs.append(torch.from_numpy(synth.make_x(shape.K, B, seed + r)).to(dev))
+            ys.append(torch.empty((B, shape.N), dtype=torch.float16, device=dev))
+    torch.cuda.synchronize(dev)
+    info = layers[0].info()
+
+    def sweep(n, start=0):
+        for i in range(n):
+            r = (start + i) % ring
+            layers[r](xs[r], out=ys[r], stream=stream)
+
+    # Warm-up (eager), then capture one full ring and a remainder graph.
+    with torch.cuda.stream(stream):
+        sweep(warmup)
+    torch.cuda.synchronize(dev)
+    full, rem = divmod(steps, ring)
+    g_full = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_full, stream=stream):
+        sweep(ring)
+    g_rem = None
+    if rem:
+        g_rem = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_rem, stream=stream):
+            sweep(rem)
+    with torch.cuda.stream(stream):
+        g_full.replay()
+    torch.cuda.synchronize(dev)
+
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    uuid = getattr(props, "uuid", None)
+    gpu_id = f"GPU-{uuid}" if uuid is not None else str(local)
+    with ClockSampler(gpu_id) as clk:
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(full):
+                g_full.replay()
+            if g_rem is not None:
+                g_rem.replay()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1)
+    if pg:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms = float(t.item())
+    del g_full, g_rem
+
+    # End to end through the public host-buffer call: x copied in from
+    # pinned memory and y read back every step.
+    e2e = None
+    if not args.no_e2e:
+        n_e2e = min(steps, 2000)
+        xh = [torch.from_numpy(synth.make_x(shape.K, B, seed + r)).pin_memory() for r in range(ring)]
+        yh = torch.empty((B, shape.N), dtype=torch.float16).pin_memory()
+        for i in range(8):
+            layers[i % ring].run_host(xh[i % ring], yh, stream=stream)
+        if pg:
+            pg.barrier()
+        torch.cuda.synchronize(dev)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for i in range(n_e2e):
+            r = i % ring
+            layers[r].run_host(xh[r], yh, stream=stream)
+        a1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_e2e = a0.elapsed_time(a1)
+        if pg:
+            t = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        sb = stream_bytes(shape, B)
+        e2e = {"value": round(world * n_e2e * sb / (ms_e2e * 1e-3) / 1e9, 4), "unit": "GB/s",
+               "us_per_layer": round(ms_e2e * 1e3 / n_e2e, 3),
+               "h2d_bytes_per_step": 2 * B * shape.K, "d2h_bytes_per_step": 2 * B * shape.N,
+               "steps": n_e2e}
+
+    for lay in layers:
+        lay.close()
+    if pg:
+        pg.destroy_process_group()
+    if rank != 0:
+        return
+
+    sb = stream_bytes(shape, B)
+    us_layer = ms * 1e3 / steps
+    gbs = world * steps * sb / (ms * 1e-3) / 1e9
+    peak, peak_kind = load_peaks()
+    workload = f"{args.config}:{shape.name}:B{B}"
+    # Dominant kernel: the fused lookup kernel, one launch per step; its
+    # average launch duration is the timed region over the launches.
+    lookup_us = us_layer
+    achieved = sb / (lookup_us * 1e-6) / 1e9
+    line = {
+        "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s",
+        "us_per_layer": round(us_layer, 4),
+        "pct_of_8tbs": round(100 * gbs / world / 8000.0, 2),
+        "pct_of_measured_hbm": round(100 * gbs / world / peak, 2),
+        "n_gpus": world, "steps": steps, "warmup": warmup, "ms_per_step": round(ms / steps, 7),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+        "data": "synthetic",
+        "config": {"workload": workload, "N": shape.N, "K": shape.K, "d": shape.d, "index_bits": 8,
+                   "batch": B, "codebook_rows": shape.codebook_rows,
+                   "residual_group": shape.residual_group, "hadamard_block": shape.hadamard_block,
+                   "ring_layers": ring, "ring_index_bytes": ring * wi_bytes,
+                   "l2_bytes": l2, "l2_policy": "inputs larger than L2: ring of distinct layers > 2x L2",
+                   "graph": "one CUDA graph per ring sweep", "parallelism": f"replicas x{world}",
+                   "grid": info.grid, "kernels_per_step": info.kernels_per_run},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 3), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": load_traffic(workload),
+                     "peak_kind": peak_kind, "kernel": "eva_lookup_kernel",
+                     "algorithmic_bytes_per_launch": sb},
+        "gpu_launches": steps * info.kernels_per_run,
+        "clocks": clk.summary(),
+    }
+    if e2e:
+        line["e2e"] = e2e
+    if not args.no_cpu:
+        us_cpu, reps, threads = cpu_baseline(shape, B, seed, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": round(sb / (us_cpu * 1e-6) / 1e9, 4), "unit": "GB/s",
+                                "us_per_layer": round(us_cpu, 2), "cores": threads, "kind": "oracle",
+                                "sample": f"{reps} whole-layer oracle calls of {shape.name} B={B} "
+                                          f"(dequantise + fp64 GEMV), OpenMP over output rows"}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

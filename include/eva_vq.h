@@ -1,0 +1,155 @@
+/*
+ * eva_vq.h -- C ABI of the B200 (sm_100a) decode-phase linear layer with
+ * vector-quantized weights.
+ *
+ * The operation (EVA: Accelerating LLM Decoding via an Efficient Vector
+ * Quantization Architecture, technical summary section 2.A):
+ *   - the input x of one decode step is cut into J = K/d sub-vectors x_j of
+ *     length d (d = 4);
+ *   - the weight codebook WC holds 2^n centroids of length d (n = 8, so 256
+ *     centroids and one index byte per 4 weights: 2 bits per weight);
+ *   - the output codebook OC[j][c] = <x_j, WC[c]> turns the matrix-vector
+ *     product into a small matrix-matrix product;
+ *   - the output is gathered through the weight-index matrix WI and summed:
+ *     y[o] = sum_j OC[j][WI[o][j]].
+ * The 3.125-bit variant (Replacing MatMul with SRAM lookup: a 3-bit edge
+ * inference architecture, section details and its quantize() sample) adds a
+ * randomized Hadamard rotation of the input and a 1-bit residual sign per
+ * weight with one fp16 scale alpha per group of 128 inputs:
+ *   y[o] = sum_j OC~[j][WI[o][j]] + sum_q alpha[o][q] sum_{k in q} sigma[o][k] x~[k],
+ * with x~ = s (.) (H_b x) / sqrt(b) blockwise (Sylvester H_b, s = hsign).
+ *
+ * All entry points return a status code and never abort or trap.  No entry
+ * point throws.  Device pointers must be 16-byte aligned.
+ */
+#ifndef EVA_VQ_H
+#define EVA_VQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define EVA_API __attribute__((visibility("default")))
+#else
+#define EVA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st *eva_stream_t;
+
+typedef enum {
+    EVA_OK = 0,
+    EVA_ERR_INVALID_ARG = 1,     /* bad pointer, size, alignment or handle      */
+    EVA_ERR_UNSUPPORTED = 2,     /* valid but not implemented (d != 4, n != 8)   */
+    EVA_ERR_CUDA = 3,            /* a CUDA runtime call failed                   */
+    EVA_ERR_OOM = 4,             /* device allocation failed in create           */
+    EVA_ERR_DEVICE_TIMEOUT = 5,  /* a bounded device wait gave up                */
+    EVA_ERR_NO_DEVICE = 6        /* no sm_100 device is current                  */
+} eva_status_t;
+
+typedef enum { EVA_F16 = 0, EVA_F32 = 1 } eva_dtype_t;
+
+/* Kernel family used by run(). */
+typedef enum {
+    EVA_PATH_AUTO = 0,        /* pick per call from B and the codebook layout   */
+    EVA_PATH_OC_LOOKUP = 1,   /* output codebook in shared memory + lookups     */
+    EVA_PATH_DEQUANT_MMA = 2  /* codebook gather into tensor-core operands      */
+} eva_path_t;
+
+typedef struct {
+    int32_t N;               /* output features, >= 1                                   */
+    int32_t K;               /* input features, multiple of d (and of 128 with residual) */
+    int32_t d;               /* sub-vector length; 4 is the only supported value        */
+    int32_t index_bits;      /* n; 8 is the only supported value (256 centroids)        */
+    int32_t codebook_rows;   /* 0: one shared codebook; R > 0: codebook g serves rows
+                                [R g, R g + R); R must be a multiple of 16 dividing N    */
+    int32_t residual_group;  /* 0: no sign residual; 128: signs + one alpha per 128 k   */
+    int32_t hadamard_block;  /* 0: no rotation; b: power of two in [8, 4096] dividing K */
+    int32_t max_batch;       /* largest B passed to run(), 1..64; sizes the workspace   */
+    eva_dtype_t out_dtype;   /* dtype of y                                               */
+    eva_path_t path;         /* EVA_PATH_AUTO unless a test or benchmark forces one     */
+} eva_vq_desc;
+
+typedef struct eva_vq_linear *eva_vq_linear_t;
+
+/*
+ * Create a layer.  Copies and repacks the weights into library-owned device
+ * memory; the copies are enqueued on `stream`, and the caller's buffers may
+ * be released once `stream` has passed this call.  All pointers are device
+ * pointers (16-byte aligned):
+ *   wc     fp16 [G][256][d], G = codebook_rows ? N / codebook_rows : 1
+ *   wi     u8   [N][K/d], canonical row-major, WI[o][j] = centroid of row o, sub-vector j
+ *   signs  u8   [N][K/8], bit i of byte m is sigma[o][8m+i] (1: +1, 0: -1); NULL unless residual
+ *   alpha  fp16 [N][K/residual_group]; NULL unless residual
+ *   hsign  int8 [K], entries +1 or -1; NULL unless hadamard_block
+ * Returns EVA_ERR_INVALID_ARG / EVA_ERR_UNSUPPORTED before touching the
+ * device when the descriptor or pointers are unusable, EVA_ERR_OOM when an
+ * allocation fails (nothing is leaked), EVA_ERR_CUDA on a failed launch.
+ */
+EVA_API eva_status_t eva_vq_linear_create(eva_vq_linear_t *out, const eva_vq_desc *desc,
+                                  const void *wc, const uint8_t *wi, const uint8_t *signs,
+                                  const void *alpha, const int8_t *hsign, eva_stream_t stream);
+
+/*
+ * y = layer(x) for B tokens, asynchronous on `stream`; no host sync and no
+ * allocation.  x: device fp16 [B][K]; y: device [B][N] of desc.out_dtype.
+ * Both are caller-owned and must not overlap.  One handle must not run on
+ * two streams at once (its workspace is shared); distinct handles are
+ * independent.  Kernels are launched with programmatic dependent launch: a
+ * kernel of this call may start loading weights while the previous kernel
+ * on the stream is finishing, but reads x only after it has completed.
+ * Rejects B < 1 or B > max_batch, null or misaligned x / y.
+ */
+EVA_API eva_status_t eva_vq_linear_run(eva_vq_linear_t h, const void *x, int32_t B, void *y,
+                               eva_stream_t stream);
+
+/*
+ * The same call with HOST buffers: copies x (host fp16 [B][K]) to the
+ * handle's staging buffer, runs, copies y back to y_host ([B][N] of
+ * out_dtype) and waits for `stream`.  Pinned host memory makes the copies
+ * asynchronous; pageable memory works but is slower.
+ */
+EVA_API eva_status_t eva_vq_linear_run_host(eva_vq_linear_t h, const void *x_host, int32_t B,
+                                    void *y_host, eva_stream_t stream);
+
+/* Free the handle's device memory.  The caller must have synchronised every
+ * stream the handle ran on.  NULL is accepted. */
+EVA_API eva_status_t eva_vq_linear_destroy(eva_vq_linear_t h);
+
+/*
+ * Test hook: decode the handle's repacked index stream with the same
+ * position functions the lookup kernels use, writing canonical WI
+ * [N][K/d] u8 to device memory `wi_out`.  Bit-exact inverse of create().
+ */
+EVA_API eva_status_t eva_vq_unpack_indices(eva_vq_linear_t h, uint8_t *wi_out, eva_stream_t stream);
+
+/* Synchronises the device and reports a device-side error word set by a
+ * kernel (EVA_ERR_DEVICE_TIMEOUT for a bounded wait that gave up). */
+EVA_API eva_status_t eva_vq_sync_status(eva_vq_linear_t h);
+
+/* Static string for a status code. */
+EVA_API const char *eva_vq_status_string(eva_status_t s);
+
+typedef struct {
+    int64_t stream_bytes;     /* algorithmic bytes per token-batch: WI + signs + alpha + x */
+    int64_t wi_bytes, sign_bytes, alpha_bytes, codebook_bytes;
+    int64_t workspace_bytes;  /* device memory owned by the handle beyond the weights */
+    int32_t slices;           /* K-slices of 64 sub-vectors                             */
+    int32_t row_tiles;        /* row tiles of 16 outputs                                */
+    int32_t grid;             /* CTAs of the lookup kernel for the last run             */
+    int32_t kernels_per_run;  /* kernel launches per run() for the last run            */
+    int32_t path;             /* eva_path_t used by the last run                       */
+    int32_t sm_count;
+} eva_vq_info;
+
+/* Sizes and launch shape of a handle (host only, no device work). */
+EVA_API eva_status_t eva_vq_linear_info(eva_vq_linear_t h, eva_vq_info *info);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* EVA_VQ_H */

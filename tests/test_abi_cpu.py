@@ -1,0 +1,101 @@
+"""The C-ABI library on a machine without a GPU: it builds, loads, exports
+every function include/eva_vq.h declares, and rejects bad arguments on the
+host before any device work."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from vector_quantized_weight_b200 import build, eva_vq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "eva_vq.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"EVA_API\s+[\w\s\*]*?\b(eva_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_binding_functions():
+    assert declared_functions() == sorted(eva_vq.ABI_FUNCTIONS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = eva_vq.load()
+    out = subprocess.run(["nm", "-D", "--defined-only", build.LIB], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    for fn in declared_functions():
+        assert fn in exported, fn
+        assert getattr(lib, fn) is not None
+    # nothing beyond the ABI leaks out of the library
+    assert exported == set(declared_functions())
+
+
+def test_status_strings():
+    for s in range(7):
+        assert eva_vq.eva_vq_status_string(s)
+    assert eva_vq.eva_vq_status_string(99) == "unknown status"
+
+
+def _desc(**kw):
+    base = dict(N=256, K=512, d=4, index_bits=8, codebook_rows=0, residual_group=0,
+                hadamard_block=0, max_batch=1, out_dtype=0, path=0)
+    base.update(kw)
+    return eva_vq.eva_vq_desc(*[base[f] for f, _ in eva_vq.eva_vq_desc._fields_])
+
+
+def _create(desc, wc=0x1000, wi=0x2000, signs=None, alpha=None, hsign=None):
+    lib = eva_vq.load()
+    h = ctypes.c_void_p()
+    return lib.eva_vq_linear_create(ctypes.byref(h), ctypes.byref(desc), wc, wi, signs, alpha, hsign, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(d=3), eva_vq.EVA_ERR_UNSUPPORTED),
+    (dict(index_bits=4), eva_vq.EVA_ERR_UNSUPPORTED),
+    (dict(N=0), eva_vq.EVA_ERR_INVALID_ARG),
+    (dict(K=510), eva_vq.EVA_ERR_INVALID_ARG),
+    (dict(codebook_rows=100), eva_vq.EVA_ERR_INVALID_ARG),
+    (dict(codebook_rows=48), eva_vq.EVA_ERR_INVALID_ARG),     # does not divide N=256
+    (dict(residual_group=64), eva_vq.EVA_ERR_UNSUPPORTED),
+    (dict(hadamard_block=384), eva_vq.EVA_ERR_INVALID_ARG),
+    (dict(hadamard_block=1024), eva_vq.EVA_ERR_INVALID_ARG),  # does not divide K=512
+    (dict(max_batch=0), eva_vq.EVA_ERR_INVALID_ARG),
+    (dict(max_batch=65), eva_vq.EVA_ERR_INVALID_ARG),
+    (dict(out_dtype=7), eva_vq.EVA_ERR_INVALID_ARG),
+])
+def test_create_rejects_bad_descriptor(kw, expect):
+    assert _create(_desc(**kw)) == expect
+
+
+def test_create_rejects_bad_pointers():
+    assert _create(_desc(), wc=None) == eva_vq.EVA_ERR_INVALID_ARG
+    assert _create(_desc(), wi=None) == eva_vq.EVA_ERR_INVALID_ARG
+    assert _create(_desc(), wc=0x1004) == eva_vq.EVA_ERR_INVALID_ARG           # misaligned
+    assert _create(_desc(residual_group=128)) == eva_vq.EVA_ERR_INVALID_ARG     # residual without signs
+    assert _create(_desc(), signs=0x3000, alpha=0x4000) == eva_vq.EVA_ERR_INVALID_ARG  # signs without residual
+    assert _create(_desc(hadamard_block=64)) == eva_vq.EVA_ERR_INVALID_ARG      # rotation without signs s
+    lib = eva_vq.load()
+    assert lib.eva_vq_linear_create(None, ctypes.byref(_desc()), 0x1000, 0x2000, None, None, None,
+                                    None) == eva_vq.EVA_ERR_INVALID_ARG
+
+
+def test_calls_on_null_handle():
+    lib = eva_vq.load()
+    assert lib.eva_vq_linear_run(None, 0x1000, 1, 0x2000, None) == eva_vq.EVA_ERR_INVALID_ARG
+    assert lib.eva_vq_linear_run_host(None, 0x1000, 1, 0x2000, None) == eva_vq.EVA_ERR_INVALID_ARG
+    assert lib.eva_vq_unpack_indices(None, 0x1000, None) == eva_vq.EVA_ERR_INVALID_ARG
+    assert lib.eva_vq_sync_status(None) == eva_vq.EVA_ERR_INVALID_ARG
+    assert lib.eva_vq_linear_info(None, None) == eva_vq.EVA_ERR_INVALID_ARG
+    assert lib.eva_vq_linear_destroy(None) == eva_vq.EVA_OK
+
+
+def test_create_without_device_reports_no_device():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    assert _create(_desc()) == eva_vq.EVA_ERR_NO_DEVICE

@@ -1,0 +1,147 @@
+"""CUDA path against the double-precision oracle, through the C ABI.
+
+Every configuration of the decode workloads (tiny, Llama-2-7B layer and
+block at batch 1/4/16, Gemma-2-9B-shaped 3.125-bit layers, Llama-2-70B-shaped
+layers with one codebook per 128 rows at batch 1/8/32) runs at full size in
+the launch configuration the benchmark uses; the oracle checks a sample of
+output rows (all rows where it is cheap).  Indices are checked bit-exactly,
+integer-valued problems exactly, everything else within the norm-relative
+tolerance TOL.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from tests.conftest import cuda_available
+from tests.gpu_helpers import TOL, norm_rel_err, run_gpu, sample_rows, sub_layer_oracle
+from vector_quantized_weight_b200 import synth
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not cuda_available(), reason="needs a CUDA device")]
+
+
+def _layers_and_batches():
+    out = []
+    for key, cfg in synth.CONFIGS.items():
+        for li, shape in enumerate(cfg.layers):
+            for B in cfg.batches:
+                out.append(pytest.param(key, li, B, id=f"{key}-{shape.name}-B{B}"))
+    return out
+
+
+@pytest.mark.parametrize("key,li,B", _layers_and_batches())
+def test_config_parity(key, li, B):
+    cfg = synth.CONFIGS[key]
+    shape = cfg.layers[li]
+    seed = synth.layer_seed(cfg.index, li)
+    layer = synth.make_layer(shape, seed)
+    x = synth.make_x(shape.K, B, seed)
+    y = run_gpu(layer, x)
+    rows = sample_rows(shape.N, shape.codebook_rows, n=192, seed=seed) if shape.N * shape.K * B > 2**26 \
+        else np.arange(shape.N)
+    ref = sub_layer_oracle(layer, x, rows)
+    err = norm_rel_err(y[:, rows], ref)
+    assert np.all(err <= TOL), (err.max(), TOL)
+
+
+@pytest.mark.parametrize("N,K,pattern", [
+    (256, 512, "random"), (4096, 4096, "random"), (100, 300, "ramp"), (17, 260, "rowcol"),
+    (11008, 4096, "a5"), (4096, 11008, "ones"), (48, 1024, "zeros"), (3584, 14336, "random"),
+])
+def test_index_roundtrip_bit_exact(N, K, pattern):
+    import torch
+    from vector_quantized_weight_b200 import eva_vq
+    wi = synth.adversarial_wi(N, K // 4, pattern, seed=N + K)
+    wc = torch.zeros((1, 256, 4), dtype=torch.float16, device="cuda")
+    lin = eva_vq.VQLinear(wc, torch.from_numpy(wi).cuda())
+    back = lin.unpack_indices().cpu().numpy()
+    torch.cuda.synchronize()
+    lin.close()
+    assert np.array_equal(back, wi)
+
+
+@pytest.mark.parametrize("B", [1, 2, 3])
+@pytest.mark.parametrize("N,K,cbr", [(256, 512, 0), (128, 1024, 16), (40, 264, 0)])
+def test_integer_inputs_exact(N, K, cbr, B):
+    """Small-integer codebooks and inputs: every product and sum is exact in
+    fp16 / fp32, so the GPU must reproduce the oracle exactly."""
+    rng = np.random.default_rng(N + K + B)
+    G = N // cbr if cbr else 1
+    layer = synth.LayerData(synth.LayerShape("int", N, K, codebook_rows=cbr),
+                            rng.integers(-2, 3, size=(G, 256, 4)).astype(np.float16),
+                            rng.integers(0, 256, size=(N, K // 4)).astype(np.uint8), None, None, None)
+    x = rng.integers(-3, 4, size=(B, K)).astype(np.float16)
+    y = run_gpu(layer, x, out_dtype="float32")
+    ref = oracle.layer_linear(layer, x)
+    assert np.array_equal(y, ref)
+
+
+@pytest.mark.parametrize("N,K,B,cbr,resid,had", [
+    (17, 260, 1, 0, 0, 0),          # ragged rows and a partial last K-slice
+    (100, 132, 2, 0, 0, 0),
+    (33, 384, 3, 0, 128, 0),        # odd batch, residual without rotation
+    (64, 640, 1, 0, 128, 128),      # rotation block 128, residual
+    (272, 1024, 5, 16, 0, 0),       # 17 codebooks of 16 rows, odd batch
+    (3584, 3584, 1, 0, 128, 512),   # Gemma block structure
+    (8, 8192, 64, 0, 0, 0),         # maximum batch
+])
+def test_edge_cases(N, K, B, cbr, resid, had):
+    shape = synth.LayerShape("edge", N, K, codebook_rows=cbr, residual_group=resid, hadamard_block=had)
+    layer = synth.make_layer(shape, 1234 + N, alpha_signed=True)
+    x = synth.make_x(K, B, 99)
+    for dt in ("float16", "float32"):
+        y = run_gpu(layer, x, out_dtype=dt)
+        ref = oracle.layer_linear(layer, x, nthreads=8)
+        err = norm_rel_err(y, ref)
+        assert np.all(err <= TOL), (dt, err.max())
+
+
+def test_residual_only_changes_with_signs():
+    """Flipping every sign bit of one row changes only that row, by
+    -2 * sum_q alpha_q sum_k sigma_k x~_k (twice its residual)."""
+    shape = synth.LayerShape("flip", 64, 512, residual_group=128)
+    layer = synth.make_layer(shape, 77)
+    x = synth.make_x(512, 1, 5)
+    y0 = run_gpu(layer, x, out_dtype="float32")
+    layer.signs[5] ^= 0xFF
+    y1 = run_gpu(layer, x, out_dtype="float32")
+    diff = np.abs(y1 - y0)[0]
+    assert diff[5] > 0 and np.all(np.delete(diff, 5) == 0)
+
+
+def test_deterministic_and_host_path():
+    import torch
+    from vector_quantized_weight_b200 import eva_vq
+    shape = synth.CONFIGS["llama7b_layer"].layers[0]
+    layer = synth.make_layer(shape, 5)
+    x = synth.make_x(shape.K, 1, 5)
+    lin = eva_vq.from_layer(layer, max_batch=1)
+    xt = torch.from_numpy(x).cuda()
+    y1 = lin(xt).cpu()
+    y2 = lin(xt).cpu()
+    assert torch.equal(y1, y2)
+    xh = torch.from_numpy(x).pin_memory()
+    yh = torch.empty((1, shape.N), dtype=torch.float16).pin_memory()
+    lin.run_host(xh, yh)
+    assert torch.equal(yh, y1)
+    assert eva_vq.eva_vq_sync_status(lin.handle) == eva_vq.EVA_OK
+    lin.close()
+
+
+def test_run_rejects_bad_arguments():
+    import ctypes
+    import torch
+    from vector_quantized_weight_b200 import eva_vq
+    shape = synth.LayerShape("err", 64, 256)
+    layer = synth.make_layer(shape, 3)
+    lin = eva_vq.from_layer(layer, max_batch=2)
+    lib = eva_vq.load()
+    x = torch.zeros((4, 256), dtype=torch.float16, device="cuda")
+    y = torch.zeros((4, 64), dtype=torch.float16, device="cuda")
+    h = lin.handle
+    assert lib.eva_vq_linear_run(h, x.data_ptr(), 0, y.data_ptr(), None) == eva_vq.EVA_ERR_INVALID_ARG
+    assert lib.eva_vq_linear_run(h, x.data_ptr(), 3, y.data_ptr(), None) == eva_vq.EVA_ERR_INVALID_ARG
+    assert lib.eva_vq_linear_run(h, x.data_ptr() + 2, 1, y.data_ptr(), None) == eva_vq.EVA_ERR_INVALID_ARG
+    assert lib.eva_vq_linear_run(h, None, 1, y.data_ptr(), None) == eva_vq.EVA_ERR_INVALID_ARG
+    torch.cuda.synchronize()
+    lin.close()

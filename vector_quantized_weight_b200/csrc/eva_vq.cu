@@ -1,0 +1,377 @@
+// eva_vq.cu -- C ABI of the VQ decode linear (see include/eva_vq.h).
+//
+// Host side only: argument validation, device memory owned by a handle, the
+// create-time repack, and the launch sequence of run():
+//   [Hadamard rotation of x]  ->  fused OC build + lookup + accumulate
+// Every launch goes to the caller's stream with programmatic dependent launch
+// so a kernel's weight prefetch overlaps the tail of the one before it.
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <new>
+
+#include "../../include/eva_vq.h"
+#include "eva_vq_kernels.cuh"
+
+using namespace eva;
+
+struct eva_vq_linear {
+    eva_vq_desc desc;
+    int device = 0, sm_count = 0;
+    int J = 0, S = 0, T = 0, Npad = 0, G = 1, tiles_per_cb = 0;
+    int Gs = 1, Gt = 1;                 // lookup grid (slice groups x row groups)
+    uint8_t *wi = nullptr;              // repacked indices
+    uint8_t *sg = nullptr;              // repacked signs
+    __half *al = nullptr;               // repacked alpha
+    __half *wc = nullptr;               // codebooks [G][256][4]
+    int8_t *hsign = nullptr;            // Hadamard signs [K]
+    float *partial = nullptr;           // [max_batch][Gs][Npad]
+    unsigned *counters = nullptr;       // [Gt]
+    float *xt = nullptr;                // rotated input [max_batch][K]
+    int *status = nullptr;              // device error word
+    void *x_stage = nullptr, *y_stage = nullptr;
+    int64_t workspace_bytes = 0;
+    int last_grid = 0, last_kernels = 0, last_path = 0;
+};
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+eva_status_t cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return EVA_OK;
+    if (e == cudaErrorMemoryAllocation) return EVA_ERR_OOM;
+    return EVA_ERR_CUDA;
+}
+
+bool is_pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
+
+eva_status_t validate_desc(const eva_vq_desc *d) {
+    if (!d) return EVA_ERR_INVALID_ARG;
+    if (d->N < 1 || d->K < 1 || d->N > (1 << 24) || d->K > (1 << 22)) return EVA_ERR_INVALID_ARG;
+    if (d->d != kD || d->index_bits != 8) return EVA_ERR_UNSUPPORTED;
+    if (d->K % kD) return EVA_ERR_INVALID_ARG;
+    if (d->codebook_rows < 0) return EVA_ERR_INVALID_ARG;
+    if (d->codebook_rows && (d->codebook_rows % kTileRows || d->N % d->codebook_rows))
+        return EVA_ERR_INVALID_ARG;
+    if (d->residual_group != 0 && d->residual_group != 128) return EVA_ERR_UNSUPPORTED;
+    if (d->residual_group && d->K % d->residual_group) return EVA_ERR_INVALID_ARG;
+    if (d->hadamard_block) {
+        if (!is_pow2(d->hadamard_block) || d->hadamard_block < 8 || d->hadamard_block > 4096 ||
+            d->K % d->hadamard_block)
+            return EVA_ERR_INVALID_ARG;
+    }
+    if (d->max_batch < 1 || d->max_batch > 64) return EVA_ERR_INVALID_ARG;
+    if (d->out_dtype != EVA_F16 && d->out_dtype != EVA_F32) return EVA_ERR_INVALID_ARG;
+    if (d->path != EVA_PATH_AUTO && d->path != EVA_PATH_OC_LOOKUP && d->path != EVA_PATH_DEQUANT_MMA)
+        return EVA_ERR_INVALID_ARG;
+    if (d->path == EVA_PATH_DEQUANT_MMA) return EVA_ERR_UNSUPPORTED;
+    return EVA_OK;
+}
+
+// Pick the CTA rectangle (Gs slice groups x Gt row groups, Gs*Gt <= SMs) that
+// minimises the per-SM shared-memory-pipe time: lookups (32 warp-wide loads
+// per unit), output-codebook stores (256 per build, one build per slice and
+// codebook spanned) and the split-K epilogue.
+void plan_grid(eva_vq_linear *h) {
+    const int S = h->S, T = h->T, P = h->sm_count;
+    double best = 1e300;
+    int bs = 1, bt = std::min(T, P);
+    for (int gs = 1; gs <= std::min(S, P); ++gs) {
+        for (int gt = 1; gt <= std::min(T, P / gs); ++gt) {
+            const int tiles = (T + gt - 1) / gt, slices = (S + gs - 1) / gs;
+            if ((tiles + kWarps - 1) / kWarps > kMaxTilesPerWarp) continue;
+            int builds = 1;
+            if (h->tiles_per_cb) builds = (tiles + h->tiles_per_cb - 1) / h->tiles_per_cb + 1;
+            double cost = (double)slices * (builds * 320.0 + tiles * 32.0);
+            cost += (gs > 1) ? 400.0 : 0.0;             // partials + fence + finalize
+            cost += 2000.0 * (double)(gs * gt) / (P * 64.0);  // mild preference for fewer CTAs
+            if (cost < best) { best = cost; bs = gs; bt = gt; }
+        }
+    }
+    h->Gs = bs;
+    h->Gt = bt;
+}
+
+template <typename K, typename... Args>
+cudaError_t launch_pdl(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+size_t lookup_smem(bool pair_t, bool resid) {
+    return (size_t)kOcBytes + ((pair_t && resid) ? (size_t)kOcBytes : 0);
+}
+
+cudaError_t set_smem_attrs() {
+    cudaError_t e;
+    e = cudaFuncSetAttribute(eva_lookup_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lookup_smem(false, false));
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(eva_lookup_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lookup_smem(false, true));
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(eva_lookup_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lookup_smem(true, false));
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(eva_lookup_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lookup_smem(true, true));
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(eva_hadamard_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 4096 * 4);
+}
+
+void free_handle(eva_vq_linear *h) {
+    if (!h) return;
+    void *ptrs[] = {h->wi, h->sg, h->al, h->wc, h->hsign, h->partial, h->counters, h->xt,
+                    h->status, h->x_stage, h->y_stage};
+    for (void *p : ptrs)
+        if (p) cudaFree(p);
+    delete h;
+}
+
+template <typename T>
+cudaError_t dalloc(T **p, size_t bytes, int64_t *acc) {
+    *p = nullptr;
+    if (bytes == 0) return cudaSuccess;
+    cudaError_t e = cudaMalloc(reinterpret_cast<void **>(p), bytes);
+    if (e == cudaSuccess && acc) *acc += (int64_t)bytes;
+    return e;
+}
+
+unsigned blocks_for(long long total, int threads) { return (unsigned)((total + threads - 1) / threads); }
+
+}  // namespace
+
+extern "C" {
+
+const char *eva_vq_status_string(eva_status_t s) {
+    switch (s) {
+        case EVA_OK: return "ok";
+        case EVA_ERR_INVALID_ARG: return "invalid argument";
+        case EVA_ERR_UNSUPPORTED: return "unsupported configuration";
+        case EVA_ERR_CUDA: return "CUDA runtime error";
+        case EVA_ERR_OOM: return "device allocation failed";
+        case EVA_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+        case EVA_ERR_NO_DEVICE: return "no sm_100 device";
+    }
+    return "unknown status";
+}
+
+eva_status_t eva_vq_linear_create(eva_vq_linear_t *out, const eva_vq_desc *desc, const void *wc,
+                                  const uint8_t *wi, const uint8_t *signs, const void *alpha,
+                                  const int8_t *hsign, eva_stream_t stream) {
+    if (!out) return EVA_ERR_INVALID_ARG;
+    *out = nullptr;
+    eva_status_t st = validate_desc(desc);
+    if (st != EVA_OK) return st;
+    if (!wc || !wi || !aligned16(wc) || !aligned16(wi)) return EVA_ERR_INVALID_ARG;
+    if (desc->residual_group) {
+        if (!signs || !alpha || !aligned16(signs) || !aligned16(alpha)) return EVA_ERR_INVALID_ARG;
+    } else if (signs || alpha) {
+        return EVA_ERR_INVALID_ARG;
+    }
+    if (desc->hadamard_block) {
+        if (!hsign || !aligned16(hsign)) return EVA_ERR_INVALID_ARG;
+    } else if (hsign) {
+        return EVA_ERR_INVALID_ARG;
+    }
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return EVA_ERR_NO_DEVICE;
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return EVA_ERR_NO_DEVICE;
+    if (prop.major != 10) return EVA_ERR_NO_DEVICE;
+
+    eva_vq_linear *h = new (std::nothrow) eva_vq_linear();
+    if (!h) return EVA_ERR_OOM;
+    h->desc = *desc;
+    h->device = dev;
+    h->sm_count = prop.multiProcessorCount;
+    const int N = desc->N, K = desc->K;
+    h->J = K / kD;
+    h->S = (h->J + kSliceJ - 1) / kSliceJ;
+    h->T = (N + kTileRows - 1) / kTileRows;
+    h->Npad = h->T * kTileRows;
+    h->G = desc->codebook_rows ? N / desc->codebook_rows : 1;
+    h->tiles_per_cb = desc->codebook_rows ? desc->codebook_rows / kTileRows : 0;
+    plan_grid(h);
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const long long units = (long long)h->S * h->T;
+    int64_t ws = 0;
+    cudaError_t e = cudaSuccess;
+    auto chk = [&](cudaError_t r) { if (e == cudaSuccess) e = r; };
+    chk(set_smem_attrs());
+    chk(dalloc(&h->wi, (size_t)units * kUnitBytes, nullptr));
+    chk(dalloc(&h->wc, (size_t)h->G * kCent * kD * sizeof(__half), nullptr));
+    if (desc->residual_group) {
+        chk(dalloc(&h->sg, (size_t)units * kSignUnitBytes, nullptr));
+        chk(dalloc(&h->al, (size_t)units * kAlphaUnitHalves * sizeof(__half), nullptr));
+    }
+    if (desc->hadamard_block) {
+        chk(dalloc(&h->hsign, (size_t)K, nullptr));
+        chk(dalloc(&h->xt, (size_t)desc->max_batch * K * sizeof(float), &ws));
+    }
+    chk(dalloc(&h->partial, h->Gs > 1 ? (size_t)desc->max_batch * h->Gs * h->Npad * sizeof(float) : 0, &ws));
+    chk(dalloc(&h->counters, (size_t)h->Gt * sizeof(unsigned), &ws));
+    chk(dalloc(&h->status, sizeof(int), &ws));
+    const size_t ybytes = (size_t)desc->max_batch * N * (desc->out_dtype == EVA_F32 ? 4 : 2);
+    chk(dalloc(&h->x_stage, (size_t)desc->max_batch * K * sizeof(__half), &ws));
+    chk(dalloc(&h->y_stage, ybytes, &ws));
+    h->workspace_bytes = ws;
+    if (e != cudaSuccess) {
+        free_handle(h);
+        return cuda_status(e);
+    }
+
+    const int thr = 256;
+    const long long wib = units * kUnitBytes;
+    eva_repack_wi_kernel<<<blocks_for(wib, thr), thr, 0, s>>>(wi, h->wi, N, h->J, h->T, wib);
+    chk(cudaGetLastError());
+    chk(cudaMemcpyAsync(h->wc, wc, (size_t)h->G * kCent * kD * sizeof(__half), cudaMemcpyDeviceToDevice, s));
+    if (desc->residual_group) {
+        const long long sb = units * kSignUnitBytes, ab = units * kAlphaUnitHalves;
+        eva_repack_signs_kernel<<<blocks_for(sb, thr), thr, 0, s>>>(signs, h->sg, N, K / 8, h->T, sb);
+        chk(cudaGetLastError());
+        eva_repack_alpha_kernel<<<blocks_for(ab, thr), thr, 0, s>>>(
+            reinterpret_cast<const __half *>(alpha), h->al, N, K / desc->residual_group, h->T, ab);
+        chk(cudaGetLastError());
+    }
+    if (desc->hadamard_block) chk(cudaMemcpyAsync(h->hsign, hsign, (size_t)K, cudaMemcpyDeviceToDevice, s));
+    chk(cudaMemsetAsync(h->counters, 0, (size_t)h->Gt * sizeof(unsigned), s));
+    chk(cudaMemsetAsync(h->status, 0, sizeof(int), s));
+    if (e != cudaSuccess) {
+        cudaStreamSynchronize(s);
+        free_handle(h);
+        return cuda_status(e);
+    }
+    *out = h;
+    return EVA_OK;
+}
+
+eva_status_t eva_vq_linear_run(eva_vq_linear_t h, const void *x, int32_t B, void *y, eva_stream_t stream) {
+    if (!h || !x || !y || !aligned16(x) || !aligned16(y)) return EVA_ERR_INVALID_ARG;
+    if (B < 1 || B > h->desc.max_batch) return EVA_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const eva_vq_desc &d = h->desc;
+    int kernels = 0;
+    cudaError_t e = cudaSuccess;
+
+    LookupParams p;
+    p.wi = h->wi;
+    p.sg = h->sg;
+    p.al = h->al;
+    p.wc = h->wc;
+    p.x = x;
+    p.x_f32 = 0;
+    p.partial = h->partial;
+    p.counters = h->counters;
+    p.y = y;
+    p.N = d.N;
+    p.Npad = h->Npad;
+    p.K = d.K;
+    p.S = h->S;
+    p.T = h->T;
+    p.B = B;
+    p.Gs = h->Gs;
+    p.Gt = h->Gt;
+    p.tiles_per_cb = h->tiles_per_cb;
+    p.out_f32 = d.out_dtype == EVA_F32 ? 1 : 0;
+
+    if (d.hadamard_block) {
+        const int b = d.hadamard_block;
+        const int thr = std::min(b / 2, 1024);
+        e = launch_pdl(eva_hadamard_kernel, dim3(d.K / b, B), dim3(thr), (size_t)b * sizeof(float), s,
+                       reinterpret_cast<const __half *>(x), (const int8_t *)h->hsign, h->xt, d.K, b,
+                       (float)(1.0 / std::sqrt((double)b)));
+        if (e != cudaSuccess) return cuda_status(e);
+        ++kernels;
+        p.x = h->xt;
+        p.x_f32 = 1;
+    }
+
+    const bool pair_t = B > 1;
+    const bool resid = d.residual_group != 0;
+    const dim3 grid(h->Gs * h->Gt), block(kThreads);
+    const size_t smem = lookup_smem(pair_t, resid);
+    if (!pair_t && !resid) e = launch_pdl(eva_lookup_kernel<false, false>, grid, block, smem, s, p);
+    else if (!pair_t && resid) e = launch_pdl(eva_lookup_kernel<false, true>, grid, block, smem, s, p);
+    else if (pair_t && !resid) e = launch_pdl(eva_lookup_kernel<true, false>, grid, block, smem, s, p);
+    else e = launch_pdl(eva_lookup_kernel<true, true>, grid, block, smem, s, p);
+    if (e != cudaSuccess) return cuda_status(e);
+    ++kernels;
+    h->last_grid = (int)grid.x;
+    h->last_kernels = kernels;
+    h->last_path = EVA_PATH_OC_LOOKUP;
+    return EVA_OK;
+}
+
+eva_status_t eva_vq_linear_run_host(eva_vq_linear_t h, const void *x_host, int32_t B, void *y_host,
+                                    eva_stream_t stream) {
+    if (!h || !x_host || !y_host) return EVA_ERR_INVALID_ARG;
+    if (B < 1 || B > h->desc.max_batch) return EVA_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const size_t xb = (size_t)B * h->desc.K * sizeof(__half);
+    const size_t yb = (size_t)B * h->desc.N * (h->desc.out_dtype == EVA_F32 ? 4 : 2);
+    cudaError_t e = cudaMemcpyAsync(h->x_stage, x_host, xb, cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return cuda_status(e);
+    eva_status_t st = eva_vq_linear_run(h, h->x_stage, B, h->y_stage, stream);
+    if (st != EVA_OK) return st;
+    e = cudaMemcpyAsync(y_host, h->y_stage, yb, cudaMemcpyDeviceToHost, s);
+    if (e != cudaSuccess) return cuda_status(e);
+    return cuda_status(cudaStreamSynchronize(s));
+}
+
+eva_status_t eva_vq_linear_destroy(eva_vq_linear_t h) {
+    free_handle(h);
+    return EVA_OK;
+}
+
+eva_status_t eva_vq_unpack_indices(eva_vq_linear_t h, uint8_t *wi_out, eva_stream_t stream) {
+    if (!h || !wi_out) return EVA_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const long long total = (long long)h->S * h->T * kUnitBytes;
+    eva_unpack_wi_kernel<<<blocks_for(total, 256), 256, 0, s>>>(h->wi, wi_out, h->desc.N, h->J, h->T, total);
+    return cuda_status(cudaGetLastError());
+}
+
+eva_status_t eva_vq_sync_status(eva_vq_linear_t h) {
+    if (!h) return EVA_ERR_INVALID_ARG;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_status(e);
+    int word = 0;
+    e = cudaMemcpy(&word, h->status, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_status(e);
+    return word ? EVA_ERR_DEVICE_TIMEOUT : EVA_OK;
+}
+
+eva_status_t eva_vq_linear_info(eva_vq_linear_t h, eva_vq_info *info) {
+    if (!h || !info) return EVA_ERR_INVALID_ARG;
+    const eva_vq_desc &d = h->desc;
+    std::memset(info, 0, sizeof(*info));
+    info->wi_bytes = (int64_t)d.N * (d.K / kD);
+    info->sign_bytes = d.residual_group ? (int64_t)d.N * (d.K / 8) : 0;
+    info->alpha_bytes = d.residual_group ? (int64_t)d.N * (d.K / d.residual_group) * 2 : 0;
+    info->codebook_bytes = (int64_t)h->G * kCent * kD * 2;
+    info->stream_bytes = info->wi_bytes + info->sign_bytes + info->alpha_bytes + (int64_t)d.K * 2;
+    info->workspace_bytes = h->workspace_bytes;
+    info->slices = h->S;
+    info->row_tiles = h->T;
+    info->grid = h->last_grid ? h->last_grid : h->Gs * h->Gt;
+    info->kernels_per_run = h->last_kernels ? h->last_kernels : (d.hadamard_block ? 2 : 1);
+    info->path = h->last_path ? h->last_path : EVA_PATH_OC_LOOKUP;
+    info->sm_count = h->sm_count;
+    return EVA_OK;
+}
+
+}  // extern "C"

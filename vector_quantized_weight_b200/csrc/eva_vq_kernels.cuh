@@ -1,0 +1,513 @@
+// eva_vq_kernels.cuh -- sm_100a kernels of the VQ decode linear.
+//
+//  eva_lookup_kernel   fused output-codebook build + conflict-free lookup +
+//                      accumulation (EVA summary section 2.A, both steps; the
+//                      Epilogue Unit of section 2.B that overlaps lookups with
+//                      the codebook product is played here by one CTA doing
+//                      both on one slice), with the optional 1-bit sign
+//                      residual of the 3-bit SRAM-lookup article.
+//  eva_hadamard_kernel randomized block Hadamard rotation of x (3-bit article,
+//                      quantize() sample: W_rot = W Q, so x~ = Q^T x).
+//  eva_repack_*        create-time repack of WI / signs / alpha into the
+//                      unit-major lane order the lookup kernel streams.
+//
+// Accumulation: the looked-up fp16 OC entries are summed by tensor-core MMAs
+// against a constant 0/1 "routing" matrix (f16 inputs, fp32 accumulation).
+// That is the adder tree: the MMA sums across the 16 k-columns supplied by
+// the four lanes of a row, so no warp shuffles are needed and the shared-
+// memory pipe carries only the lookups.
+#pragma once
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "eva_vq_layout.cuh"
+
+namespace eva {
+
+constexpr int kThreads = 512;
+constexpr int kWarps = kThreads / 32;
+constexpr int kMaxTilesPerWarp = 8;
+
+extern __shared__ __align__(1024) uint8_t eva_smem[];
+
+struct LookupParams {
+    const uint8_t *wi;       // repacked index units, [S][T] x 1024 B
+    const uint8_t *sg;       // repacked sign units, [S][T] x 512 B (residual only)
+    const __half *al;        // repacked alpha units, [S][T] x 32 halves (residual only)
+    const __half *wc;        // codebooks [G][256][4]
+    const void *x;           // activations [B][K]: fp16, or fp32 when x_f32
+    float *partial;          // split-K partial sums [B][Gs][Npad]
+    unsigned *counters;      // per row group, self-resetting
+    void *y;                 // output [B][N]
+    int N, Npad, K, S, T, B;
+    int Gs, Gt;              // CTA grid: blockIdx.x = tt * Gs + ts
+    int tiles_per_cb;        // 0: shared codebook; else row tiles per codebook
+    int x_f32, out_f32;
+};
+
+// ------------------------------------------------------------------ helpers
+
+__device__ __forceinline__ uint32_t lds32(uint32_t off) {
+    return *reinterpret_cast<const uint32_t *>(eva_smem + off);
+}
+__device__ __forceinline__ void sts32(uint32_t off, uint32_t v) {
+    *reinterpret_cast<uint32_t *>(eva_smem + off) = v;
+}
+
+// Streamed read-only 16-byte load that does not allocate in L1.
+__device__ __forceinline__ uint4 ldg_stream(const void *p) {
+    uint4 r;
+    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+        : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+        : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ void prefetch_l2_bulk(const void *p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// Programmatic dependent launch: wait for the preceding kernel's writes /
+// allow the next kernel to start its prologue.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+__device__ __forceinline__ uint32_t to_tf32(float f) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(f));
+    return r;
+}
+
+// D = A(16x4, tf32) * B(4x8, tf32), fp32 accumulate from zero.
+__device__ __forceinline__ void mma_tf32_k4(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
+    asm("mma.sync.aligned.m16n8k4.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, "
+        "{%7,%7,%7,%7};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(b0), "f"(0.f));
+}
+
+// D += A(16x16, f16) * B(16x8, f16), fp32 accumulate.
+__device__ __forceinline__ void mma_f16_k16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                            uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+__device__ __forceinline__ uint32_t half2_bits(float lo, float hi) { return pack_half2(lo, hi); }
+
+__device__ __forceinline__ void swap_if(bool c, uint32_t &a, uint32_t &b) {
+    uint32_t ta = c ? b : a, tb = c ? a : b;
+    a = ta;
+    b = tb;
+}
+
+// After the call v[r] holds the input v[r ^ q] (q in 0..3): lane q stores its
+// bank class r ^ q in round r, so the 32 lanes of a store hit 32 banks.
+__device__ __forceinline__ void xor_permute(uint32_t (&v)[4], int q) {
+    swap_if(q & 1, v[0], v[1]);
+    swap_if(q & 1, v[2], v[3]);
+    swap_if(q & 2, v[0], v[2]);
+    swap_if(q & 2, v[1], v[3]);
+}
+
+// x~[tok][k], zero outside [0, B) x [0, K).  Read through L2 (x may have
+// been written by the kernel this one waited for).
+__device__ __forceinline__ float load_x(const LookupParams &p, int tok, int k) {
+    if (tok >= p.B || k >= p.K) return 0.f;
+    size_t i = (size_t)tok * p.K + k;
+    if (p.x_f32) return __ldcg(reinterpret_cast<const float *>(p.x) + i);
+    unsigned short b = __ldcg(reinterpret_cast<const unsigned short *>(p.x) + i);
+    return __half2float(__ushort_as_half(b));
+}
+
+// --------------------------------------------------- output-codebook build
+//
+// OC[j][c] = sum_{u<4} x~[256 s + 4 j + u] * WC[cb][c][u] for the 64 sub-vectors
+// of slice s: a 64 x 4 by 4 x 256 product on tensor cores (m16n8k4, tf32; the
+// fp16 inputs are exact in tf32 and their products exact in fp32), rounded to
+// fp16 and stored in the conflict-free image.  Warp w builds centroid columns
+// 8 nt .. 8 nt + 7 for nt = w and w + 16.
+template <bool PAIR_T>
+__device__ __forceinline__ void build_oc(const LookupParams &p, int s, int cb, int pr, int warp,
+                                         int g, int q) {
+    constexpr int NTOK = PAIR_T ? 2 : 1;
+    uint32_t ax[NTOK][4][2];
+#pragma unroll
+    for (int tk = 0; tk < NTOK; ++tk) {
+        const int tok = PAIR_T ? 2 * pr + tk : 0;
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt) {
+            const int k = s * kSliceK + kD * (16 * mt + g) + q;
+            ax[tk][mt][0] = to_tf32(load_x(p, tok, k));
+            ax[tk][mt][1] = to_tf32(load_x(p, tok, k + 8 * kD));
+        }
+    }
+    const __half *wcb = p.wc + (size_t)cb * kCent * kD;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        const int nt = warp + 16 * half;
+        const uint32_t b0 = to_tf32(__half2float(wcb[(8 * nt + g) * kD + q]));
+        float D[NTOK][4][4];
+#pragma unroll
+        for (int tk = 0; tk < NTOK; ++tk)
+#pragma unroll
+            for (int mt = 0; mt < 4; ++mt) mma_tf32_k4(D[tk][mt], ax[tk][mt][0], ax[tk][mt][1], b0);
+        // D[tk][mt][2h + cc] = OC[16 mt + g + 8 h][8 nt + 2 q + cc]
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+            const uint32_t row = (uint32_t)(8 * nt + 2 * q + cc) * kOcRowBytes;
+            if (!PAIR_T) {
+                uint32_t W[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)  // class i: sub-vector g + 8 i (lo) and +32 (hi)
+                    W[i] = pack_half2(D[0][i >> 1][2 * (i & 1) + cc], D[0][(i >> 1) + 2][2 * (i & 1) + cc]);
+                xor_permute(W, q);
+#pragma unroll
+                for (int r = 0; r < 4; ++r) sts32(row + 4u * (g + 8 * (r ^ q)), W[r]);
+            } else {
+#pragma unroll
+                for (int hi = 0; hi < 2; ++hi) {
+                    uint32_t W[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int mt = (i >> 1) + 2 * hi, e = 2 * (i & 1) + cc;
+                        W[i] = pack_half2(D[0][mt][e], D[1][mt][e]);
+                    }
+                    xor_permute(W, q);
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) sts32(row + 4u * (g + 8 * (r ^ q) + 32 * hi), W[r]);
+                }
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------ sign-residual table
+//
+// The residual of a sign byte v at position m of the slice is
+// T[v][m] = sum_{i<8} sigma_i(v) x~[256 s + 8 m + i], sigma_i(v) = +1 if bit i
+// of v is set, else -1 -- the LUT of "input block x codebook" dot products of
+// the 3-bit SRAM-lookup article with the 256 sign patterns as codebook.
+// Warp w writes v = 16 w .. 16 w + 15; lane = position m, so every store hits
+// its own bank.  T = P_lo[v & 15] + P_hi[v >> 4] with 4-input partial sums.
+template <bool PAIR_T>
+__device__ __forceinline__ void build_sign_table(const LookupParams &p, int s, int pr, int warp,
+                                                 int lane, uint32_t t_off) {
+    constexpr int NTOK = PAIR_T ? 2 : 1;
+    float tv[NTOK][16];
+#pragma unroll
+    for (int tk = 0; tk < NTOK; ++tk) {
+        const int tok = PAIR_T ? 2 * pr + tk : 0;
+        float xv[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) xv[i] = load_x(p, tok, s * kSliceK + 8 * lane + i);
+        float phi = 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) phi += ((warp >> i) & 1) ? xv[4 + i] : -xv[4 + i];
+#pragma unroll
+        for (int a = 0; a < 16; ++a) {
+            float plo = 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) plo += ((a >> i) & 1) ? xv[i] : -xv[i];
+            tv[tk][a] = plo + phi;
+        }
+    }
+#pragma unroll
+    for (int a = 0; a < 16; ++a) {
+        const uint32_t w = PAIR_T ? pack_half2(tv[0][a], tv[NTOK - 1][a]) : pack_half2(tv[0][a], 0.f);
+        sts32(t_off + (uint32_t)(16 * warp + a) * kOcRowBytes + 4u * lane, w);
+    }
+}
+
+// ------------------------------------------------------------ lookup kernel
+template <bool PAIR_T, bool RESID>
+__global__ void __launch_bounds__(kThreads, 1) eva_lookup_kernel(const LookupParams p) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = lane >> 2, q = lane & 3;
+    const int ts = blockIdx.x % p.Gs, tt = blockIdx.x / p.Gs;
+    const int s0 = (int)((long long)p.S * ts / p.Gs), s1 = (int)((long long)p.S * (ts + 1) / p.Gs);
+    const int t0 = (int)((long long)p.T * tt / p.Gt), t1 = (int)((long long)p.T * (tt + 1) / p.Gt);
+    const int ntw = (t1 - t0 - warp + kWarps - 1) / kWarps;  // tiles owned by this warp
+
+    constexpr uint32_t OC_OFF = 0;
+    constexpr uint32_t HI_OFF = PAIR_T ? 128u : 0u;                      // a2/a3 column offset
+    constexpr uint32_t T_OFF = PAIR_T ? (uint32_t)kOcBytes : 128u;       // residual table
+
+    // Weights do not depend on the preceding kernel: start streaming them
+    // into L2 before waiting for it.
+    if (tid < s1 - s0) {
+        const size_t u = (size_t)(s0 + tid) * p.T + t0;
+        prefetch_l2_bulk(p.wi + u * kUnitBytes, (uint32_t)(t1 - t0) * kUnitBytes);
+        if (RESID) {
+            prefetch_l2_bulk(p.sg + u * kSignUnitBytes, (uint32_t)(t1 - t0) * kSignUnitBytes);
+            prefetch_l2_bulk(p.al + u * kAlphaUnitHalves, (uint32_t)(t1 - t0) * kAlphaUnitHalves * 2);
+        }
+    }
+    pdl_launch();
+
+    // Routing matrices of the accumulating MMA (B operand, 16 x 8, 0/1).
+    // One token: column 0 sums the low half of a0/a1 and the high half of
+    // a2/a3.  Token pair: column 0 sums the low halves, column 1 the high.
+    const uint32_t ONE_LO = 0x00003C00u, ONE_HI = 0x3C000000u;
+    uint32_t bo0, bo1;
+    if (!PAIR_T) {
+        bo0 = g == 0 ? ONE_LO : 0u;
+        bo1 = g == 0 ? ONE_HI : 0u;
+    } else {
+        bo0 = bo1 = g == 0 ? ONE_LO : (g == 1 ? ONE_HI : 0u);
+    }
+    // Residual table routing: lanes q = 0,1 feed group 0, q = 2,3 group 1.
+    uint32_t bt = 0;
+    if (RESID) {
+        if (!PAIR_T) bt = (g == (q >> 1)) ? ONE_LO : 0u;
+        else bt = (g == 2 * (q >> 1)) ? ONE_LO : (g == 2 * (q >> 1) + 1 ? ONE_HI : 0u);
+    }
+    uint32_t colw4[8];
+#pragma unroll
+    for (int s8 = 0; s8 < 8; ++s8) colw4[s8] = 4u * oc_col(lane, s8);
+    uint32_t mcol4[4][2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        mcol4[i][0] = RESID ? 4u * sign_pos(lane, i, 0) : 0u;
+        mcol4[i][1] = RESID ? 4u * sign_pos(lane, i, 2) : 0u;
+    }
+
+    pdl_wait();
+
+    const int npairs = PAIR_T ? (p.B + 1) / 2 : 1;
+    const int cb_first = p.tiles_per_cb ? t0 / p.tiles_per_cb : 0;
+    const int cb_last = p.tiles_per_cb ? (t1 - 1) / p.tiles_per_cb : 0;
+
+    for (int pr = 0; pr < npairs; ++pr) {
+        float acc[kMaxTilesPerWarp][4];
+#pragma unroll
+        for (int i = 0; i < kMaxTilesPerWarp; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+
+        for (int s = s0; s < s1; ++s) {
+            for (int cb = cb_first; cb <= cb_last; ++cb) {
+                __syncthreads();  // previous image fully consumed
+                build_oc<PAIR_T>(p, s, cb, pr, warp, g, q);
+                if (RESID && cb == cb_first) build_sign_table<PAIR_T>(p, s, pr, warp, lane, T_OFF);
+                __syncthreads();
+#pragma unroll
+                for (int i = 0; i < kMaxTilesPerWarp; ++i) {
+                    const int t = t0 + warp + kWarps * i;
+                    if (i >= ntw) break;
+                    if (p.tiles_per_cb && t / p.tiles_per_cb != cb) continue;
+                    const size_t unit = (size_t)s * p.T + t;
+                    const uint8_t *up = p.wi + unit * kUnitBytes + lane * 32;
+                    const uint4 v0 = ldg_stream(up), v1 = ldg_stream(up + 16);
+                    const uint32_t wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+                    for (int s8 = 0; s8 < 8; ++s8) {
+                        const uint32_t a0 = lds32(OC_OFF + __byte_perm(wv[s8], colw4[s8], 0x5504));
+                        const uint32_t a1 = lds32(OC_OFF + __byte_perm(wv[s8], colw4[s8], 0x5514));
+                        const uint32_t a2 = lds32(OC_OFF + HI_OFF + __byte_perm(wv[s8], colw4[s8], 0x5524));
+                        const uint32_t a3 = lds32(OC_OFF + HI_OFF + __byte_perm(wv[s8], colw4[s8], 0x5534));
+                        mma_f16_k16(acc[i], a0, a1, a2, a3, bo0, bo1);
+                    }
+                    if (RESID) {
+                        const uint4 sv = ldg_stream(p.sg + unit * kSignUnitBytes + lane * 16);
+                        const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
+                        float dt[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                        for (int mi = 0; mi < 4; ++mi) {
+                            const uint32_t a0 = lds32(T_OFF + __byte_perm(sw[mi], mcol4[mi][0], 0x5504));
+                            const uint32_t a1 = lds32(T_OFF + __byte_perm(sw[mi], mcol4[mi][0], 0x5514));
+                            const uint32_t a2 = lds32(T_OFF + __byte_perm(sw[mi], mcol4[mi][1], 0x5524));
+                            const uint32_t a3 = lds32(T_OFF + __byte_perm(sw[mi], mcol4[mi][1], 0x5534));
+                            mma_f16_k16(dt, a0, a1, a2, a3, bt, bt);
+                        }
+                        float dt1[4] = {0.f, 0.f, 0.f, 0.f};
+                        if (PAIR_T) {  // group 1 of a token pair sits in lane q = 1
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) dt1[e] = __shfl_down_sync(0xffffffffu, dt[e], 1);
+                        }
+                        if (q == 0) {
+                            const uint2 araw = *reinterpret_cast<const uint2 *>(
+                                p.al + unit * kAlphaUnitHalves + 4 * g);
+                            const __half2 ag = *reinterpret_cast<const __half2 *>(&araw.x);   // row g: grp 0, 1
+                            const __half2 ag8 = *reinterpret_cast<const __half2 *>(&araw.y);  // row g+8
+                            const float a_g0 = __low2float(ag), a_g1 = __high2float(ag);
+                            const float a_h0 = __low2float(ag8), a_h1 = __high2float(ag8);
+                            if (!PAIR_T) {
+                                acc[i][0] += a_g0 * dt[0] + a_g1 * dt[1];
+                                acc[i][2] += a_h0 * dt[2] + a_h1 * dt[3];
+                            } else {
+                                acc[i][0] += a_g0 * dt[0] + a_g1 * dt1[0];
+                                acc[i][1] += a_g0 * dt[1] + a_g1 * dt1[1];
+                                acc[i][2] += a_h0 * dt[2] + a_h1 * dt1[2];
+                                acc[i][3] += a_h0 * dt[3] + a_h1 * dt1[3];
+                            }
+                        }
+                    }
+                }
+            }
+        }
+
+        // Epilogue of this token (pair): lanes q = 0 hold column 0 (and 1).
+        if (q == 0) {
+#pragma unroll
+            for (int i = 0; i < kMaxTilesPerWarp; ++i) {
+                if (i >= ntw) break;
+                const int t = t0 + warp + kWarps * i;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int o = kTileRows * t + g + 8 * h;
+#pragma unroll
+                    for (int e = 0; e < (PAIR_T ? 2 : 1); ++e) {
+                        const int tok = PAIR_T ? 2 * pr + e : 0;
+                        const float v = acc[i][2 * h + e];
+                        if (tok >= p.B) continue;
+                        if (p.Gs == 1) {
+                            if (o < p.N) {
+                                const size_t yi = (size_t)tok * p.N + o;
+                                if (p.out_f32) reinterpret_cast<float *>(p.y)[yi] = v;
+                                else reinterpret_cast<__half *>(p.y)[yi] = __float2half_rn(v);
+                            }
+                        } else {
+                            __stcg(p.partial + ((size_t)tok * p.Gs + ts) * p.Npad + o, v);
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    if (p.Gs == 1) return;
+
+    // Split-K reduction: the last CTA of this row group sums the partials of
+    // all slice groups in a fixed order (bitwise reproducible).
+    __shared__ unsigned s_last;
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+        const unsigned prev = atomicAdd(p.counters + tt, 1u);
+        s_last = (prev == (unsigned)(p.Gs - 1)) ? 1u : 0u;
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    const int r0 = kTileRows * t0, r1 = min(kTileRows * t1, p.N);
+    const int rows = r1 - r0;
+    for (int idx = tid; idx < rows * p.B; idx += kThreads) {
+        const int tok = idx / rows, o = r0 + idx % rows;
+        const float *pp = p.partial + (size_t)tok * p.Gs * p.Npad + o;
+        float sum = 0.f;
+        for (int k = 0; k < p.Gs; ++k) sum += __ldcg(pp + (size_t)k * p.Npad);
+        const size_t yi = (size_t)tok * p.N + o;
+        if (p.out_f32) reinterpret_cast<float *>(p.y)[yi] = sum;
+        else reinterpret_cast<__half *>(p.y)[yi] = __float2half_rn(sum);
+    }
+    if (tid == 0) p.counters[tt] = 0u;  // ready for the next call on this stream
+}
+
+// ----------------------------------------------------- Hadamard rotation
+//
+// x~ = hsign (.) (H_b x) / sqrt(b) per block of b inputs: the natural-order
+// (Sylvester) fast Walsh-Hadamard transform in shared memory, fp32.
+// Grid (K / b, B).
+__global__ void __launch_bounds__(1024) eva_hadamard_kernel(const __half *__restrict__ x,
+                                                            const int8_t *__restrict__ hs,
+                                                            float *__restrict__ xt, int K, int b,
+                                                            float scale) {
+    float *sb = reinterpret_cast<float *>(eva_smem);
+    const int blk = blockIdx.x, tok = blockIdx.y;
+    pdl_launch();
+    pdl_wait();  // x may be the output of the preceding kernel
+    const unsigned short *xb =
+        reinterpret_cast<const unsigned short *>(x) + (size_t)tok * K + (size_t)blk * b;
+    for (int i = threadIdx.x; i < b; i += blockDim.x) sb[i] = __half2float(__ushort_as_half(__ldcg(xb + i)));
+    for (int h = 1; h < b; h <<= 1) {
+        __syncthreads();
+        for (int i = threadIdx.x; i < b / 2; i += blockDim.x) {
+            const int lo = (i / h) * 2 * h + (i % h);
+            const float a = sb[lo], c = sb[lo + h];
+            sb[lo] = a + c;
+            sb[lo + h] = a - c;
+        }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < b; i += blockDim.x) {
+        const int k = blk * b + i;
+        xt[(size_t)tok * K + k] = (float)hs[k] * sb[i] * scale;
+    }
+}
+
+// ------------------------------------------------------- create-time repack
+
+// One thread per packed byte; padding (rows >= N, sub-vectors >= J) is 0.
+__global__ void eva_repack_wi_kernel(const uint8_t *__restrict__ wi, uint8_t *__restrict__ out,
+                                     int N, int J, int T, long long total) {
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= total) return;
+    const long long unit = idx / kUnitBytes;
+    const int b = (int)(idx % kUnitBytes);
+    const int s = (int)(unit / T), t = (int)(unit % T);
+    int row, jl;
+    wi_unit_pos(b, row, jl);
+    const int o = kTileRows * t + row, j = kSliceJ * s + jl;
+    out[idx] = (o < N && j < J) ? wi[(size_t)o * J + j] : (uint8_t)0;
+}
+
+// Inverse of the repack (test hook): canonical [N][J] from the packed stream.
+__global__ void eva_unpack_wi_kernel(const uint8_t *__restrict__ packed, uint8_t *__restrict__ wi,
+                                     int N, int J, int T, long long total) {
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= total) return;
+    const long long unit = idx / kUnitBytes;
+    const int b = (int)(idx % kUnitBytes);
+    const int s = (int)(unit / T), t = (int)(unit % T);
+    int row, jl;
+    wi_unit_pos(b, row, jl);
+    const int o = kTileRows * t + row, j = kSliceJ * s + jl;
+    if (o < N && j < J) wi[(size_t)o * J + j] = packed[idx];
+}
+
+__global__ void eva_repack_signs_kernel(const uint8_t *__restrict__ sg, uint8_t *__restrict__ out,
+                                        int N, int K8, int T, long long total) {
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= total) return;
+    const long long unit = idx / kSignUnitBytes;
+    const int b = (int)(idx % kSignUnitBytes);
+    const int s = (int)(unit / T), t = (int)(unit % T);
+    int row, m;
+    sign_unit_pos(b, row, m);
+    const int o = kTileRows * t + row, mm = (kSliceK / 8) * s + m;
+    out[idx] = (o < N && mm < K8) ? sg[(size_t)o * K8 + mm] : (uint8_t)0;
+}
+
+__global__ void eva_unpack_signs_kernel(const uint8_t *__restrict__ packed, uint8_t *__restrict__ sg,
+                                        int N, int K8, int T, long long total) {
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= total) return;
+    const long long unit = idx / kSignUnitBytes;
+    const int b = (int)(idx % kSignUnitBytes);
+    const int s = (int)(unit / T), t = (int)(unit % T);
+    int row, m;
+    sign_unit_pos(b, row, m);
+    const int o = kTileRows * t + row, mm = (kSliceK / 8) * s + m;
+    if (o < N && mm < K8) sg[(size_t)o * K8 + mm] = packed[idx];
+}
+
+__global__ void eva_repack_alpha_kernel(const __half *__restrict__ al, __half *__restrict__ out,
+                                        int N, int NG, int T, long long total) {
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= total) return;
+    const long long unit = idx / kAlphaUnitHalves;
+    const int e = (int)(idx % kAlphaUnitHalves);
+    const int s = (int)(unit / T), t = (int)(unit % T);
+    int row, grp;
+    alpha_unit_pos(e, row, grp);
+    const int o = kTileRows * t + row, gq = 2 * s + grp;
+    out[idx] = (o < N && gq < NG) ? al[(size_t)o * NG + gq] : __float2half(0.f);
+}
+
+}  // namespace eva

@@ -1,0 +1,74 @@
+// eva_vq_layout.cuh -- data layout of the repacked weights and the shared-memory
+// output-codebook image, shared by the create-time repack, the unpack test hook
+// and the lookup kernels.
+//
+// Work unit: one tile of 16 output rows (the M of one tensor-core MMA) times one
+// K-slice of 64 sub-vectors (256 inputs).  A unit holds 1024 index bytes.
+//
+// Output-codebook (OC) image in shared memory: 256 centroid rows of 256 bytes
+// (64 32-bit words).  The bank of a word depends only on its column, never on
+// the centroid, so 32 lanes reading 32 distinct columns never collide whatever
+// indices they look up -- the conflict-free lookup of the EVA summary, section
+// 2.A ("rows derived from different input vectors map to different banks").
+//   one token  (j-paired):   word(c, w) = half2(OC[w][c], OC[w+32][c]), w < 32
+//   two tokens (token-paired): word(c, j) = half2(OC_a[j][c], OC_b[j][c]), j < 64
+//
+// The lookup for lane L = 4g + q (g = L/4, q = L%4) at k-step s8 reads column
+// w = (L + 4 s8) mod 32.  Per k-step the lane supplies the four A registers of
+// an m16n8k16 MMA: a0 -> row g, a1 -> row g+8 (sub-vector w), a2 -> row g,
+// a3 -> row g+8 (sub-vector w + 32).  Over the 8 k-steps row g sees each of
+// the 64 sub-vectors exactly once.
+#pragma once
+#include <stdint.h>
+
+namespace eva {
+
+constexpr int kD = 4;             // sub-vector length d
+constexpr int kCent = 256;        // 2^n centroids, n = 8
+constexpr int kSliceJ = 64;       // sub-vectors per K-slice
+constexpr int kSliceK = kSliceJ * kD;   // 256 inputs per K-slice
+constexpr int kTileRows = 16;     // output rows per unit
+constexpr int kUnitBytes = kSliceJ * kTileRows;      // 1024 index bytes
+constexpr int kSignUnitBytes = kTileRows * kSliceK / 8;  // 512 sign bytes
+constexpr int kAlphaUnitHalves = kTileRows * 2;     // 2 groups of 128 per slice
+constexpr int kOcRowBytes = 256;
+constexpr int kOcBytes = kCent * kOcRowBytes;       // 64 KB image
+
+// OC column read by lane `lane` at k-step `s8`.
+__host__ __device__ __forceinline__ int oc_col(int lane, int s8) { return (lane + 4 * s8) & 31; }
+
+// Index byte `b` of a unit (0..1023) -> (row in tile, sub-vector in slice).
+// Byte b = 32*lane + 4*s8 + r, r selecting the A register a_r.
+__host__ __device__ __forceinline__ void wi_unit_pos(int b, int &row, int &jl) {
+    const int lane = b >> 5, s8 = (b >> 2) & 7, r = b & 3;
+    row = (lane >> 2) + ((r & 1) ? 8 : 0);
+    jl = oc_col(lane, s8) + ((r & 2) ? 32 : 0);
+}
+
+// Sign position read by lane (g, q) in residual MMA i (0..3), register r.
+// Lanes q = 0,1 cover the first 128-input group of the slice (positions
+// 0..15), lanes q = 2,3 the second (16..31); per register the 32 lanes read
+// 32 distinct positions, i.e. 32 distinct banks.
+__host__ __device__ __forceinline__ int sign_pos(int lane, int i, int r) {
+    const int g = lane >> 2, q = lane & 3;
+    const int st = 2 * i + (r >> 1);
+    return 16 * (q >> 1) + ((2 * g + (q & 1) + 2 * st) & 15);
+}
+
+// Sign byte `b` of a unit (0..511) -> (row in tile, sign-byte position in slice).
+// Byte b = 16*lane + 4*i + r.
+__host__ __device__ __forceinline__ void sign_unit_pos(int b, int &row, int &m) {
+    const int lane = b >> 4, i = (b >> 2) & 3, r = b & 3;
+    row = (lane >> 2) + ((r & 1) ? 8 : 0);
+    m = sign_pos(lane, i, r);
+}
+
+// Alpha half `e` of a unit (0..31) -> (row in tile, group in slice).
+// Lane g (q = 0) reads halves 4g..4g+3: (row g: grp 0, 1), (row g+8: grp 0, 1).
+__host__ __device__ __forceinline__ void alpha_unit_pos(int e, int &row, int &grp) {
+    const int g = e >> 2;
+    row = g + (((e >> 1) & 1) ? 8 : 0);
+    grp = e & 1;
+}
+
+}  // namespace eva

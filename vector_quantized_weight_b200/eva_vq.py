@@ -1,0 +1,215 @@
+"""Thin ctypes binding of the C ABI in include/eva_vq.h.
+
+Functions carry the C names and only marshal arguments: every step of the
+layer runs in the CUDA library.  PyTorch is used for device memory and
+streams only (``VQLinear``).  There is no CPU fallback: if the library cannot
+be loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+from . import build as _build
+
+EVA_OK, EVA_ERR_INVALID_ARG, EVA_ERR_UNSUPPORTED, EVA_ERR_CUDA, EVA_ERR_OOM, \
+    EVA_ERR_DEVICE_TIMEOUT, EVA_ERR_NO_DEVICE = range(7)
+EVA_F16, EVA_F32 = 0, 1
+EVA_PATH_AUTO, EVA_PATH_OC_LOOKUP, EVA_PATH_DEQUANT_MMA = 0, 1, 2
+
+# Every function the header declares; the CPU tests check the library exports them.
+ABI_FUNCTIONS = (
+    "eva_vq_linear_create", "eva_vq_linear_run", "eva_vq_linear_run_host",
+    "eva_vq_linear_destroy", "eva_vq_unpack_indices", "eva_vq_sync_status",
+    "eva_vq_status_string", "eva_vq_linear_info",
+)
+
+
+class EvaError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        msg = eva_vq_status_string(status) if _lib is not None else str(status)
+        super().__init__(f"{fn} failed: {msg} ({status})")
+
+
+class eva_vq_desc(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int32), ("K", ctypes.c_int32), ("d", ctypes.c_int32),
+                ("index_bits", ctypes.c_int32), ("codebook_rows", ctypes.c_int32),
+                ("residual_group", ctypes.c_int32), ("hadamard_block", ctypes.c_int32),
+                ("max_batch", ctypes.c_int32), ("out_dtype", ctypes.c_int),
+                ("path", ctypes.c_int)]
+
+
+class eva_vq_info(ctypes.Structure):
+    _fields_ = [("stream_bytes", ctypes.c_int64), ("wi_bytes", ctypes.c_int64),
+                ("sign_bytes", ctypes.c_int64), ("alpha_bytes", ctypes.c_int64),
+                ("codebook_bytes", ctypes.c_int64), ("workspace_bytes", ctypes.c_int64),
+                ("slices", ctypes.c_int32), ("row_tiles", ctypes.c_int32),
+                ("grid", ctypes.c_int32), ("kernels_per_run", ctypes.c_int32),
+                ("path", ctypes.c_int32), ("sm_count", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def load(build_if_missing: bool = True) -> ctypes.CDLL:
+    """Load libeva_vq.so (building it with nvcc if it is absent)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_build.LIB):
+        if not build_if_missing:
+            raise RuntimeError(f"{_build.LIB} is missing; build it with vector_quantized_weight_b200.build")
+        _build.build()
+    lib = ctypes.CDLL(_build.LIB)
+    P, I32, H = ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p
+    lib.eva_vq_linear_create.argtypes = [ctypes.POINTER(H), ctypes.POINTER(eva_vq_desc), P, P, P, P, P, P]
+    lib.eva_vq_linear_run.argtypes = [H, P, I32, P, P]
+    lib.eva_vq_linear_run_host.argtypes = [H, P, I32, P, P]
+    lib.eva_vq_linear_destroy.argtypes = [H]
+    lib.eva_vq_unpack_indices.argtypes = [H, P, P]
+    lib.eva_vq_sync_status.argtypes = [H]
+    lib.eva_vq_status_string.argtypes = [ctypes.c_int]
+    lib.eva_vq_status_string.restype = ctypes.c_char_p
+    lib.eva_vq_linear_info.argtypes = [H, ctypes.POINTER(eva_vq_info)]
+    for fn in ABI_FUNCTIONS:
+        if fn != "eva_vq_status_string":
+            getattr(lib, fn).restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def _check(fn: str, rc: int):
+    if rc != EVA_OK:
+        raise EvaError(fn, rc)
+
+
+# ------------------------------------------------------------ the C names
+
+def eva_vq_status_string(status: int) -> str:
+    return load().eva_vq_status_string(int(status)).decode()
+
+
+def eva_vq_linear_create(desc: eva_vq_desc, wc: int, wi: int, signs: int | None, alpha: int | None,
+                         hsign: int | None, stream: int | None) -> int:
+    h = ctypes.c_void_p()
+    rc = load().eva_vq_linear_create(ctypes.byref(h), ctypes.byref(desc), wc, wi, signs, alpha,
+                                     hsign, stream)
+    _check("eva_vq_linear_create", rc)
+    return h.value
+
+
+def eva_vq_linear_run(h: int, x: int, B: int, y: int, stream: int | None) -> None:
+    _check("eva_vq_linear_run", load().eva_vq_linear_run(h, x, int(B), y, stream))
+
+
+def eva_vq_linear_run_host(h: int, x_host: int, B: int, y_host: int, stream: int | None) -> None:
+    _check("eva_vq_linear_run_host", load().eva_vq_linear_run_host(h, x_host, int(B), y_host, stream))
+
+
+def eva_vq_linear_destroy(h: int | None) -> None:
+    _check("eva_vq_linear_destroy", load().eva_vq_linear_destroy(h))
+
+
+def eva_vq_unpack_indices(h: int, wi_out: int, stream: int | None) -> None:
+    _check("eva_vq_unpack_indices", load().eva_vq_unpack_indices(h, wi_out, stream))
+
+
+def eva_vq_sync_status(h: int) -> int:
+    return int(load().eva_vq_sync_status(h))
+
+
+def eva_vq_linear_info(h: int) -> eva_vq_info:
+    info = eva_vq_info()
+    _check("eva_vq_linear_info", load().eva_vq_linear_info(h, ctypes.byref(info)))
+    return info
+
+
+# ------------------------------------------------------- torch convenience
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream=None):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+class VQLinear:
+    """One layer held on the device.  Weights are torch CUDA tensors in the
+    canonical layouts (see synth.py); they are copied and repacked by the
+    library, so the caller may drop them after construction."""
+
+    def __init__(self, wc, wi, *, signs=None, alpha=None, hsign=None, codebook_rows=0,
+                 residual_group=0, hadamard_block=0, max_batch=1, out_dtype="float16",
+                 path=EVA_PATH_AUTO, stream=None):
+        import torch
+        N, J = wi.shape
+        self.N, self.K = int(N), int(J) * 4
+        self.out_dtype = torch.float32 if out_dtype in ("float32", torch.float32) else torch.float16
+        self.max_batch = int(max_batch)
+        self.desc = eva_vq_desc(self.N, self.K, 4, 8, int(codebook_rows), int(residual_group),
+                                int(hadamard_block), self.max_batch,
+                                EVA_F32 if self.out_dtype == torch.float32 else EVA_F16, int(path))
+        tensors = [wc, wi, signs, alpha, hsign]
+        for t in tensors:
+            if t is not None and (not t.is_cuda or not t.is_contiguous()):
+                raise ValueError("weights must be contiguous CUDA tensors")
+        self.handle = None
+        self.handle = eva_vq_linear_create(self.desc, _ptr(wc), _ptr(wi), _ptr(signs), _ptr(alpha),
+                                           _ptr(hsign), _stream_handle(stream))
+
+    def __call__(self, x, out=None, stream=None):
+        import torch
+        if x.dtype != torch.float16 or not x.is_cuda or not x.is_contiguous():
+            raise ValueError("x must be a contiguous CUDA float16 tensor [B, K]")
+        x2 = x.view(-1, self.K)
+        B = x2.shape[0]
+        y = out if out is not None else torch.empty((B, self.N), dtype=self.out_dtype, device=x.device)
+        eva_vq_linear_run(self.handle, _ptr(x2), B, _ptr(y), _stream_handle(stream))
+        return y
+
+    def run_host(self, x_host, y_host, stream=None):
+        """Host buffers in and out (torch CPU tensors, ideally pinned)."""
+        B = x_host.shape[0]
+        eva_vq_linear_run_host(self.handle, _ptr(x_host), B, _ptr(y_host), _stream_handle(stream))
+        return y_host
+
+    def unpack_indices(self, stream=None):
+        import torch
+        out = torch.empty((self.N, self.K // 4), dtype=torch.uint8, device="cuda")
+        eva_vq_unpack_indices(self.handle, _ptr(out), _stream_handle(stream))
+        return out
+
+    def info(self) -> eva_vq_info:
+        return eva_vq_linear_info(self.handle)
+
+    def close(self):
+        if self.handle is not None:
+            eva_vq_linear_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def from_layer(layer, *, max_batch=1, out_dtype="float16", path=EVA_PATH_AUTO, device="cuda"):
+    """Build a VQLinear from a synth.LayerData (numpy arrays)."""
+    import torch
+
+    def dev(a):
+        return None if a is None else torch.from_numpy(a).to(device)
+    s = layer.shape
+    return VQLinear(dev(layer.wc), dev(layer.wi), signs=dev(layer.signs), alpha=dev(layer.alpha),
+                    hsign=dev(layer.hsign), codebook_rows=s.codebook_rows,
+                    residual_group=s.residual_group, hadamard_block=s.hadamard_block,
+                    max_batch=max_batch, out_dtype=out_dtype, path=path)

@@ -48,7 +48,8 @@ typedef enum {
     EVA_ERR_CUDA = 3,            /* a CUDA runtime call failed                   */
     EVA_ERR_OOM = 4,             /* device allocation failed in create           */
     EVA_ERR_DEVICE_TIMEOUT = 5,  /* a bounded device wait gave up                */
-    EVA_ERR_NO_DEVICE = 6        /* no sm_100 device is current                  */
+    EVA_ERR_NO_DEVICE = 6,       /* no sm_100 device is current                  */
+    EVA_ERR_DEVICE_CHECK = 7     /* checked build: a kernel access was out of bounds */
 } eva_status_t;
 
 typedef enum { EVA_F16 = 0, EVA_F32 = 1 } eva_dtype_t;
@@ -130,6 +131,15 @@ EVA_API eva_status_t eva_vq_unpack_indices(eva_vq_linear_t h, uint8_t *wi_out, e
 /* Synchronises the device and reports a device-side error word set by a
  * kernel (EVA_ERR_DEVICE_TIMEOUT for a bounded wait that gave up). */
 EVA_API eva_status_t eva_vq_sync_status(eva_vq_linear_t h);
+
+/*
+ * Diagnostic hook of the checked build (compiled with EVA_DEVICE_CHECKS):
+ * synchronises the device and copies the handle's 8-word check record to
+ * host memory out8: [0] number of rejected accesses, then for the first one
+ * [1] source line, [2] buffer id, [3] block, [4] thread, [5..6] byte offset
+ * (low, high), [7] access size.  In the regular build the record stays zero.
+ */
+EVA_API eva_status_t eva_vq_device_check_record(eva_vq_linear_t h, int32_t *out8);
 
 /* Static string for a status code. */
 EVA_API const char *eva_vq_status_string(eva_status_t s);

@@ -99,3 +99,16 @@ def test_create_without_device_reports_no_device():
     if torch.cuda.is_available():
         pytest.skip("a device is present")
     assert _create(_desc()) == eva_vq.EVA_ERR_NO_DEVICE
+
+
+def test_lookup_kernels_do_not_spill():
+    """ptxas report of every lookup-kernel instance: no local-memory stack
+    frame and no spills (the hot loop keeps everything in registers)."""
+    cmd = [build._nvcc(), *[f for f in build.NVCC_FLAGS if f != "-shared"], "-Xptxas", "-v", "-c",
+           "-I", os.path.join(ROOT, "include"), "-o", os.devnull, *build.SOURCES]
+    out = subprocess.run(cmd, capture_output=True, text=True, check=True).stderr
+    blocks = re.findall(r"Function properties for (\S*eva_lookup_kernel\S*)\n\s*(\d+) bytes stack frame, "
+                        r"(\d+) bytes spill stores, (\d+) bytes spill loads", out)
+    assert len(blocks) == 4, out
+    for name, stack, st, ld in blocks:
+        assert (stack, st, ld) == ("0", "0", "0"), (name, stack, st, ld)

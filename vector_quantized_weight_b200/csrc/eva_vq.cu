@@ -163,6 +163,7 @@ const char *eva_vq_status_string(eva_status_t s) {
         case EVA_ERR_OOM: return "device allocation failed";
         case EVA_ERR_DEVICE_TIMEOUT: return "device wait timed out";
         case EVA_ERR_NO_DEVICE: return "no sm_100 device";
+        case EVA_ERR_DEVICE_CHECK: return "device-side bounds check failed (checked build)";
     }
     return "unknown status";
 }
@@ -224,7 +225,7 @@ eva_status_t eva_vq_linear_create(eva_vq_linear_t *out, const eva_vq_desc *desc,
     }
     chk(dalloc(&h->partial, h->Gs > 1 ? (size_t)desc->max_batch * h->Gs * h->Npad * sizeof(float) : 0, &ws));
     chk(dalloc(&h->counters, (size_t)h->Gt * sizeof(unsigned), &ws));
-    chk(dalloc(&h->status, sizeof(int), &ws));
+    chk(dalloc(&h->status, 8 * sizeof(int), &ws));
     const size_t ybytes = (size_t)desc->max_batch * N * (desc->out_dtype == EVA_F32 ? 4 : 2);
     chk(dalloc(&h->x_stage, (size_t)desc->max_batch * K * sizeof(__half), &ws));
     chk(dalloc(&h->y_stage, ybytes, &ws));
@@ -249,7 +250,7 @@ eva_status_t eva_vq_linear_create(eva_vq_linear_t *out, const eva_vq_desc *desc,
     }
     if (desc->hadamard_block) chk(cudaMemcpyAsync(h->hsign, hsign, (size_t)K, cudaMemcpyDeviceToDevice, s));
     chk(cudaMemsetAsync(h->counters, 0, (size_t)h->Gt * sizeof(unsigned), s));
-    chk(cudaMemsetAsync(h->status, 0, sizeof(int), s));
+    chk(cudaMemsetAsync(h->status, 0, 8 * sizeof(int), s));
     if (e != cudaSuccess) {
         cudaStreamSynchronize(s);
         free_handle(h);
@@ -304,6 +305,27 @@ eva_status_t eva_vq_linear_run(eva_vq_linear_t h, const void *x, int32_t B, void
     const bool resid = d.residual_group != 0;
     const dim3 grid(h->Gs * h->Gt), block(kThreads);
     const size_t smem = lookup_smem(pair_t, resid);
+#ifdef EVA_DEVICE_CHECKS
+    {
+        const long long units = (long long)h->S * h->T;
+        const void *base[8] = {h->wi, h->sg, h->al, h->wc, p.x, h->partial, h->counters, y};
+        const unsigned long long bytes[8] = {
+            (unsigned long long)units * kUnitBytes,
+            h->sg ? (unsigned long long)units * kSignUnitBytes : 0ull,
+            h->al ? (unsigned long long)units * kAlphaUnitHalves * 2 : 0ull,
+            (unsigned long long)h->G * kCent * kD * 2,
+            (unsigned long long)B * d.K * (p.x_f32 ? 4 : 2),
+            h->partial ? (unsigned long long)d.max_batch * h->Gs * h->Npad * 4 : 0ull,
+            (unsigned long long)h->Gt * 4,
+            (unsigned long long)B * d.N * (p.out_f32 ? 4 : 2)};
+        for (int i = 0; i < 8; ++i) {
+            p.chk_base[i] = base[i];
+            p.chk_bytes[i] = bytes[i];
+        }
+        p.smem_bytes = (unsigned)smem;
+        p.chk_record = h->status;
+    }
+#endif
     if (!pair_t && !resid) e = launch_pdl(eva_lookup_kernel<false, false>, grid, block, smem, s, p);
     else if (!pair_t && resid) e = launch_pdl(eva_lookup_kernel<false, true>, grid, block, smem, s, p);
     else if (pair_t && !resid) e = launch_pdl(eva_lookup_kernel<true, false>, grid, block, smem, s, p);
@@ -352,7 +374,18 @@ eva_status_t eva_vq_sync_status(eva_vq_linear_t h) {
     int word = 0;
     e = cudaMemcpy(&word, h->status, sizeof(int), cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) return cuda_status(e);
+#ifdef EVA_DEVICE_CHECKS
+    return word ? EVA_ERR_DEVICE_CHECK : EVA_OK;
+#else
     return word ? EVA_ERR_DEVICE_TIMEOUT : EVA_OK;
+#endif
+}
+
+eva_status_t eva_vq_device_check_record(eva_vq_linear_t h, int32_t *out8) {
+    if (!h || !out8) return EVA_ERR_INVALID_ARG;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_status(e);
+    return cuda_status(cudaMemcpy(out8, h->status, 8 * sizeof(int), cudaMemcpyDeviceToHost));
 }
 
 eva_status_t eva_vq_linear_info(eva_vq_linear_t h, eva_vq_info *info) {

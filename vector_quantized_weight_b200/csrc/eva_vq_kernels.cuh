@@ -24,9 +24,9 @@
 
 namespace eva {
 
-constexpr int kThreads = 512;
+constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kMaxTilesPerWarp = 8;
+constexpr int kMaxTilesPerWarp = 12;
 
 extern __shared__ __align__(1024) uint8_t eva_smem[];
 
@@ -43,7 +43,56 @@ struct LookupParams {
     int Gs, Gt;              // CTA grid: blockIdx.x = tt * Gs + ts
     int tiles_per_cb;        // 0: shared codebook; else row tiles per codebook
     int x_f32, out_f32;
+#ifdef EVA_DEVICE_CHECKS
+    // Debug build only: bounds of every buffer the kernel touches.  A
+    // violating access is skipped and the first one is recorded.
+    const void *chk_base[8];
+    unsigned long long chk_bytes[8];
+    unsigned smem_bytes;
+    int *chk_record;         // [0] count, [1] line, [2] buffer, [3] block, [4] thread,
+                             // [5] offset low, [6] offset high, [7] size
+#endif
 };
+
+enum { BUF_WI = 0, BUF_SG, BUF_AL, BUF_WC, BUF_X, BUF_PARTIAL, BUF_COUNTERS, BUF_Y, BUF_SMEM };
+
+#ifdef EVA_DEVICE_CHECKS
+__device__ __noinline__ bool eva_check_fail(const LookupParams &p, int line, int buf, long long off,
+                                            unsigned long long n) {
+    if (atomicAdd(p.chk_record, 1) == 0) {
+        p.chk_record[1] = line;
+        p.chk_record[2] = buf;
+        p.chk_record[3] = (int)blockIdx.x;
+        p.chk_record[4] = (int)threadIdx.x;
+        p.chk_record[5] = (int)(off & 0xffffffffll);
+        p.chk_record[6] = (int)(off >> 32);
+        p.chk_record[7] = (int)n;
+    }
+    return true;
+}
+// True when [ptr, ptr + n) is outside buffer `buf` or misaligned for an
+// n-byte access (n up to 16).
+__device__ __forceinline__ bool eva_bad_g(const LookupParams &p, int buf, const void *ptr,
+                                          unsigned long long n, int line) {
+    const char *b = static_cast<const char *>(p.chk_base[buf]);
+    const char *q = static_cast<const char *>(ptr);
+    const long long off = (long long)(q - b);
+    const unsigned long long al = n >= 16 ? 16 : (n >= 8 ? 8 : (n >= 4 ? 4 : (n >= 2 ? 2 : 1)));
+    if (b && off >= 0 && (unsigned long long)off + n <= p.chk_bytes[buf] &&
+        (reinterpret_cast<uintptr_t>(q) % al) == 0)
+        return false;
+    return eva_check_fail(p, line, buf, off, n);
+}
+__device__ __forceinline__ bool eva_bad_s(const LookupParams &p, uint32_t off, int line) {
+    if (off + 4u <= p.smem_bytes && (off & 3u) == 0) return false;
+    return eva_check_fail(p, line, BUF_SMEM, off, 4);
+}
+#define EVA_BAD_G(buf, ptr, n) eva_bad_g(p, buf, ptr, n, __LINE__)
+#define EVA_BAD_S(off) eva_bad_s(p, off, __LINE__)
+#else
+#define EVA_BAD_G(buf, ptr, n) false
+#define EVA_BAD_S(off) false
+#endif
 
 // ------------------------------------------------------------------ helpers
 
@@ -61,6 +110,18 @@ __device__ __forceinline__ uint4 ldg_stream(const void *p) {
         : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
         : "l"(p));
     return r;
+}
+
+// The 32 index bytes of one lane in one unit.  Volatile with a memory
+// clobber so the compiler keeps it where it is written: the tile loop issues
+// exactly one unit of lookahead instead of hoisting every tile's load.
+__device__ __forceinline__ void ldg_unit(const void *p, uint4 &a, uint4 &b) {
+    asm volatile(
+        "ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%8];\n\t"
+        "ld.global.nc.L1::no_allocate.v4.u32 {%4,%5,%6,%7}, [%8+16];"
+        : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
+        : "l"(p)
+        : "memory");
 }
 
 __device__ __forceinline__ void prefetch_l2_bulk(const void *p, uint32_t bytes) {
@@ -122,8 +183,13 @@ __device__ __forceinline__ void xor_permute(uint32_t (&v)[4], int q) {
 __device__ __forceinline__ float load_x(const LookupParams &p, int tok, int k) {
     if (tok >= p.B || k >= p.K) return 0.f;
     size_t i = (size_t)tok * p.K + k;
-    if (p.x_f32) return __ldcg(reinterpret_cast<const float *>(p.x) + i);
-    unsigned short b = __ldcg(reinterpret_cast<const unsigned short *>(p.x) + i);
+    if (p.x_f32) {
+        const float *xp = reinterpret_cast<const float *>(p.x) + i;
+        return EVA_BAD_G(BUF_X, xp, 4) ? 0.f : __ldcg(xp);
+    }
+    const unsigned short *xp = reinterpret_cast<const unsigned short *>(p.x) + i;
+    if (EVA_BAD_G(BUF_X, xp, 2)) return 0.f;
+    unsigned short b = __ldcg(xp);
     return __half2float(__ushort_as_half(b));
 }
 
@@ -132,8 +198,8 @@ __device__ __forceinline__ float load_x(const LookupParams &p, int tok, int k) {
 // OC[j][c] = sum_{u<4} x~[256 s + 4 j + u] * WC[cb][c][u] for the 64 sub-vectors
 // of slice s: a 64 x 4 by 4 x 256 product on tensor cores (m16n8k4, tf32; the
 // fp16 inputs are exact in tf32 and their products exact in fp32), rounded to
-// fp16 and stored in the conflict-free image.  Warp w builds centroid columns
-// 8 nt .. 8 nt + 7 for nt = w and w + 16.
+// fp16 and stored in the conflict-free image.  Warp w builds the centroid
+// columns 8 nt .. 8 nt + 7 of nt = w, w + kWarps, ...
 template <bool PAIR_T>
 __device__ __forceinline__ void build_oc(const LookupParams &p, int s, int cb, int pr, int warp,
                                          int g, int q) {
@@ -150,39 +216,55 @@ __device__ __forceinline__ void build_oc(const LookupParams &p, int s, int cb, i
         }
     }
     const __half *wcb = p.wc + (size_t)cb * kCent * kD;
+#pragma unroll 1
+    for (int nt = warp; nt < kCent / 8; nt += kWarps) {
+        const __half *wp = wcb + (8 * nt + g) * kD + q;
+        const uint32_t b0 = to_tf32(EVA_BAD_G(BUF_WC, wp, 2) ? 0.f : __half2float(*wp));
+        if (!PAIR_T) {
+            // D[mt][2h + cc] = OC[16 mt + g + 8 h][8 nt + 2 q + cc]; the word of
+            // class i pairs sub-vector g + 8 i (m-tile i/2) with +32 (m-tile i/2 + 2).
+            float D[4][4];
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-        const int nt = warp + 16 * half;
-        const uint32_t b0 = to_tf32(__half2float(wcb[(8 * nt + g) * kD + q]));
-        float D[NTOK][4][4];
+            for (int mt = 0; mt < 4; ++mt) mma_tf32_k4(D[mt], ax[0][mt][0], ax[0][mt][1], b0);
 #pragma unroll
-        for (int tk = 0; tk < NTOK; ++tk)
-#pragma unroll
-            for (int mt = 0; mt < 4; ++mt) mma_tf32_k4(D[tk][mt], ax[tk][mt][0], ax[tk][mt][1], b0);
-        // D[tk][mt][2h + cc] = OC[16 mt + g + 8 h][8 nt + 2 q + cc]
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-            const uint32_t row = (uint32_t)(8 * nt + 2 * q + cc) * kOcRowBytes;
-            if (!PAIR_T) {
+            for (int cc = 0; cc < 2; ++cc) {
+                const uint32_t row = (uint32_t)(8 * nt + 2 * q + cc) * kOcRowBytes;
                 uint32_t W[4];
 #pragma unroll
-                for (int i = 0; i < 4; ++i)  // class i: sub-vector g + 8 i (lo) and +32 (hi)
-                    W[i] = pack_half2(D[0][i >> 1][2 * (i & 1) + cc], D[0][(i >> 1) + 2][2 * (i & 1) + cc]);
+                for (int i = 0; i < 4; ++i)
+                    W[i] = pack_half2(D[i >> 1][2 * (i & 1) + cc], D[(i >> 1) + 2][2 * (i & 1) + cc]);
                 xor_permute(W, q);
 #pragma unroll
-                for (int r = 0; r < 4; ++r) sts32(row + 4u * (g + 8 * (r ^ q)), W[r]);
-            } else {
+                for (int r = 0; r < 4; ++r) {
+                    const uint32_t off = row + 4u * (g + 8 * (r ^ q));
+                    if (!EVA_BAD_S(off)) sts32(off, W[r]);
+                }
+            }
+        } else {
+            // Token pair: sub-vectors 0..31 (m-tiles 0,1) then 32..63 (m-tiles 2,3).
 #pragma unroll
-                for (int hi = 0; hi < 2; ++hi) {
+            for (int hi = 0; hi < 2; ++hi) {
+                float D[2][2][4];
+#pragma unroll
+                for (int tk = 0; tk < 2; ++tk)
+#pragma unroll
+                    for (int m = 0; m < 2; ++m)
+                        mma_tf32_k4(D[tk][m], ax[tk][2 * hi + m][0], ax[tk][2 * hi + m][1], b0);
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    const uint32_t row = (uint32_t)(8 * nt + 2 * q + cc) * kOcRowBytes;
                     uint32_t W[4];
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        const int mt = (i >> 1) + 2 * hi, e = 2 * (i & 1) + cc;
-                        W[i] = pack_half2(D[0][mt][e], D[1][mt][e]);
+                        const int e = 2 * (i & 1) + cc;
+                        W[i] = pack_half2(D[0][i >> 1][e], D[NTOK - 1][i >> 1][e]);
                     }
                     xor_permute(W, q);
 #pragma unroll
-                    for (int r = 0; r < 4; ++r) sts32(row + 4u * (g + 8 * (r ^ q) + 32 * hi), W[r]);
+                    for (int r = 0; r < 4; ++r) {
+                        const uint32_t off = row + 4u * (g + 8 * (r ^ q) + 32 * hi);
+                        if (!EVA_BAD_S(off)) sts32(off, W[r]);
+                    }
                 }
             }
         }
@@ -195,34 +277,43 @@ __device__ __forceinline__ void build_oc(const LookupParams &p, int s, int cb, i
 // T[v][m] = sum_{i<8} sigma_i(v) x~[256 s + 8 m + i], sigma_i(v) = +1 if bit i
 // of v is set, else -1 -- the LUT of "input block x codebook" dot products of
 // the 3-bit SRAM-lookup article with the 256 sign patterns as codebook.
-// Warp w writes v = 16 w .. 16 w + 15; lane = position m, so every store hits
-// its own bank.  T = P_lo[v & 15] + P_hi[v >> 4] with 4-input partial sums.
+// Warp w writes the rows v whose high nibble is w, w + kWarps, ...; lane =
+// position m, so every store hits its own bank.  T = P_lo[v & 15] +
+// P_hi[v >> 4] with 4-input partial sums.
 template <bool PAIR_T>
 __device__ __forceinline__ void build_sign_table(const LookupParams &p, int s, int pr, int warp,
                                                  int lane, uint32_t t_off) {
     constexpr int NTOK = PAIR_T ? 2 : 1;
-    float tv[NTOK][16];
+    float xv[NTOK][8];
 #pragma unroll
     for (int tk = 0; tk < NTOK; ++tk) {
         const int tok = PAIR_T ? 2 * pr + tk : 0;
-        float xv[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) xv[i] = load_x(p, tok, s * kSliceK + 8 * lane + i);
-        float phi = 0.f;
+        for (int i = 0; i < 8; ++i) xv[tk][i] = load_x(p, tok, s * kSliceK + 8 * lane + i);
+    }
+#pragma unroll 1
+    for (int hn = warp; hn < 16; hn += kWarps) {
+        float phi[NTOK];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) phi += ((warp >> i) & 1) ? xv[4 + i] : -xv[4 + i];
+        for (int tk = 0; tk < NTOK; ++tk) {
+            phi[tk] = 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) phi[tk] += ((hn >> i) & 1) ? xv[tk][4 + i] : -xv[tk][4 + i];
+        }
 #pragma unroll
         for (int a = 0; a < 16; ++a) {
-            float plo = 0.f;
+            float tv[NTOK];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) plo += ((a >> i) & 1) ? xv[i] : -xv[i];
-            tv[tk][a] = plo + phi;
+            for (int tk = 0; tk < NTOK; ++tk) {
+                float plo = 0.f;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) plo += ((a >> i) & 1) ? xv[tk][i] : -xv[tk][i];
+                tv[tk] = plo + phi[tk];
+            }
+            const uint32_t w = PAIR_T ? pack_half2(tv[0], tv[NTOK - 1]) : pack_half2(tv[0], 0.f);
+            const uint32_t off = t_off + (uint32_t)(16 * hn + a) * kOcRowBytes + 4u * lane;
+            if (!EVA_BAD_S(off)) sts32(off, w);
         }
-    }
-#pragma unroll
-    for (int a = 0; a < 16; ++a) {
-        const uint32_t w = PAIR_T ? pack_half2(tv[0][a], tv[NTOK - 1][a]) : pack_half2(tv[0][a], 0.f);
-        sts32(t_off + (uint32_t)(16 * warp + a) * kOcRowBytes + 4u * lane, w);
     }
 }
 
@@ -244,10 +335,14 @@ __global__ void __launch_bounds__(kThreads, 1) eva_lookup_kernel(const LookupPar
     // into L2 before waiting for it.
     if (tid < s1 - s0) {
         const size_t u = (size_t)(s0 + tid) * p.T + t0;
-        prefetch_l2_bulk(p.wi + u * kUnitBytes, (uint32_t)(t1 - t0) * kUnitBytes);
+        const uint32_t nt = (uint32_t)(t1 - t0);
+        if (!EVA_BAD_G(BUF_WI, p.wi + u * kUnitBytes, nt * kUnitBytes))
+            prefetch_l2_bulk(p.wi + u * kUnitBytes, nt * kUnitBytes);
         if (RESID) {
-            prefetch_l2_bulk(p.sg + u * kSignUnitBytes, (uint32_t)(t1 - t0) * kSignUnitBytes);
-            prefetch_l2_bulk(p.al + u * kAlphaUnitHalves, (uint32_t)(t1 - t0) * kAlphaUnitHalves * 2);
+            if (!EVA_BAD_G(BUF_SG, p.sg + u * kSignUnitBytes, nt * kSignUnitBytes))
+                prefetch_l2_bulk(p.sg + u * kSignUnitBytes, nt * kSignUnitBytes);
+            if (!EVA_BAD_G(BUF_AL, p.al + u * kAlphaUnitHalves, nt * kAlphaUnitHalves * 2))
+                prefetch_l2_bulk(p.al + u * kAlphaUnitHalves, nt * kAlphaUnitHalves * 2);
         }
     }
     pdl_launch();
@@ -269,9 +364,6 @@ __global__ void __launch_bounds__(kThreads, 1) eva_lookup_kernel(const LookupPar
         if (!PAIR_T) bt = (g == (q >> 1)) ? ONE_LO : 0u;
         else bt = (g == 2 * (q >> 1)) ? ONE_LO : (g == 2 * (q >> 1) + 1 ? ONE_HI : 0u);
     }
-    uint32_t colw4[8];
-#pragma unroll
-    for (int s8 = 0; s8 < 8; ++s8) colw4[s8] = 4u * oc_col(lane, s8);
     uint32_t mcol4[4][2];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -292,37 +384,63 @@ __global__ void __launch_bounds__(kThreads, 1) eva_lookup_kernel(const LookupPar
 
         for (int s = s0; s < s1; ++s) {
             for (int cb = cb_first; cb <= cb_last; ++cb) {
+                // This warp's tiles t0 + warp + kWarps i that use codebook cb
+                // form the index range [i0, i1).
+                int i0 = 0, i1 = ntw;
+                if (p.tiles_per_cb) {
+                    const int lo = max(cb * p.tiles_per_cb, t0), hi = (cb + 1) * p.tiles_per_cb;
+                    i0 = max(0, (lo - t0 - warp + kWarps - 1) / kWarps);
+                    i1 = min(ntw, max(0, (hi - t0 - warp + kWarps - 1) / kWarps));
+                }
+                // The first unit's indices load while the codebook image builds.
+                uint4 nx0 = make_uint4(0u, 0u, 0u, 0u), nx1 = nx0;
+                if (i0 < i1) {
+                    const uint8_t *up = p.wi + ((size_t)s * p.T + t0 + warp + kWarps * i0) * kUnitBytes + lane * 32;
+                    if (!EVA_BAD_G(BUF_WI, up, 32)) ldg_unit(up, nx0, nx1);
+                }
                 __syncthreads();  // previous image fully consumed
                 build_oc<PAIR_T>(p, s, cb, pr, warp, g, q);
                 if (RESID && cb == cb_first) build_sign_table<PAIR_T>(p, s, pr, warp, lane, T_OFF);
                 __syncthreads();
 #pragma unroll
                 for (int i = 0; i < kMaxTilesPerWarp; ++i) {
+                    if (i < i0 || i >= i1) continue;
                     const int t = t0 + warp + kWarps * i;
-                    if (i >= ntw) break;
-                    if (p.tiles_per_cb && t / p.tiles_per_cb != cb) continue;
                     const size_t unit = (size_t)s * p.T + t;
-                    const uint8_t *up = p.wi + unit * kUnitBytes + lane * 32;
-                    const uint4 v0 = ldg_stream(up), v1 = ldg_stream(up + 16);
+                    const uint4 v0 = nx0, v1 = nx1;
+                    if (i + 1 < i1) {  // one unit of lookahead
+                        const uint8_t *up = p.wi + (unit + kWarps) * kUnitBytes + lane * 32;
+                        if (!EVA_BAD_G(BUF_WI, up, 32)) ldg_unit(up, nx0, nx1);
+                    }
                     const uint32_t wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
                     for (int s8 = 0; s8 < 8; ++s8) {
-                        const uint32_t a0 = lds32(OC_OFF + __byte_perm(wv[s8], colw4[s8], 0x5504));
-                        const uint32_t a1 = lds32(OC_OFF + __byte_perm(wv[s8], colw4[s8], 0x5514));
-                        const uint32_t a2 = lds32(OC_OFF + HI_OFF + __byte_perm(wv[s8], colw4[s8], 0x5524));
-                        const uint32_t a3 = lds32(OC_OFF + HI_OFF + __byte_perm(wv[s8], colw4[s8], 0x5534));
+                        const uint32_t cw = (4u * lane + 16u * s8) & 127u;   // 4 * oc_col(lane, s8)
+                        const uint32_t o0 = OC_OFF + __byte_perm(wv[s8], cw, 0x5504);
+                        const uint32_t o1 = OC_OFF + __byte_perm(wv[s8], cw, 0x5514);
+                        const uint32_t o2 = OC_OFF + HI_OFF + __byte_perm(wv[s8], cw, 0x5524);
+                        const uint32_t o3 = OC_OFF + HI_OFF + __byte_perm(wv[s8], cw, 0x5534);
+                        const uint32_t a0 = EVA_BAD_S(o0) ? 0u : lds32(o0);
+                        const uint32_t a1 = EVA_BAD_S(o1) ? 0u : lds32(o1);
+                        const uint32_t a2 = EVA_BAD_S(o2) ? 0u : lds32(o2);
+                        const uint32_t a3 = EVA_BAD_S(o3) ? 0u : lds32(o3);
                         mma_f16_k16(acc[i], a0, a1, a2, a3, bo0, bo1);
                     }
                     if (RESID) {
-                        const uint4 sv = ldg_stream(p.sg + unit * kSignUnitBytes + lane * 16);
+                        const uint8_t *sp = p.sg + unit * kSignUnitBytes + lane * 16;
+                        const uint4 sv = EVA_BAD_G(BUF_SG, sp, 16) ? make_uint4(0u, 0u, 0u, 0u) : ldg_stream(sp);
                         const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
                         float dt[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                         for (int mi = 0; mi < 4; ++mi) {
-                            const uint32_t a0 = lds32(T_OFF + __byte_perm(sw[mi], mcol4[mi][0], 0x5504));
-                            const uint32_t a1 = lds32(T_OFF + __byte_perm(sw[mi], mcol4[mi][0], 0x5514));
-                            const uint32_t a2 = lds32(T_OFF + __byte_perm(sw[mi], mcol4[mi][1], 0x5524));
-                            const uint32_t a3 = lds32(T_OFF + __byte_perm(sw[mi], mcol4[mi][1], 0x5534));
+                            const uint32_t o0 = T_OFF + __byte_perm(sw[mi], mcol4[mi][0], 0x5504);
+                            const uint32_t o1 = T_OFF + __byte_perm(sw[mi], mcol4[mi][0], 0x5514);
+                            const uint32_t o2 = T_OFF + __byte_perm(sw[mi], mcol4[mi][1], 0x5524);
+                            const uint32_t o3 = T_OFF + __byte_perm(sw[mi], mcol4[mi][1], 0x5534);
+                            const uint32_t a0 = EVA_BAD_S(o0) ? 0u : lds32(o0);
+                            const uint32_t a1 = EVA_BAD_S(o1) ? 0u : lds32(o1);
+                            const uint32_t a2 = EVA_BAD_S(o2) ? 0u : lds32(o2);
+                            const uint32_t a3 = EVA_BAD_S(o3) ? 0u : lds32(o3);
                             mma_f16_k16(dt, a0, a1, a2, a3, bt, bt);
                         }
                         float dt1[4] = {0.f, 0.f, 0.f, 0.f};
@@ -331,8 +449,9 @@ __global__ void __launch_bounds__(kThreads, 1) eva_lookup_kernel(const LookupPar
                             for (int e = 0; e < 4; ++e) dt1[e] = __shfl_down_sync(0xffffffffu, dt[e], 1);
                         }
                         if (q == 0) {
-                            const uint2 araw = *reinterpret_cast<const uint2 *>(
-                                p.al + unit * kAlphaUnitHalves + 4 * g);
+                            const __half *ap = p.al + unit * kAlphaUnitHalves + 4 * g;
+                            const uint2 araw = EVA_BAD_G(BUF_AL, ap, 8) ? make_uint2(0u, 0u)
+                                                                         : *reinterpret_cast<const uint2 *>(ap);
                             const __half2 ag = *reinterpret_cast<const __half2 *>(&araw.x);   // row g: grp 0, 1
                             const __half2 ag8 = *reinterpret_cast<const __half2 *>(&araw.y);  // row g+8
                             const float a_g0 = __low2float(ag), a_g1 = __high2float(ag);
@@ -369,11 +488,17 @@ __global__ void __launch_bounds__(kThreads, 1) eva_lookup_kernel(const LookupPar
                         if (p.Gs == 1) {
                             if (o < p.N) {
                                 const size_t yi = (size_t)tok * p.N + o;
-                                if (p.out_f32) reinterpret_cast<float *>(p.y)[yi] = v;
-                                else reinterpret_cast<__half *>(p.y)[yi] = __float2half_rn(v);
+                                if (p.out_f32) {
+                                    float *yp = reinterpret_cast<float *>(p.y) + yi;
+                                    if (!EVA_BAD_G(BUF_Y, yp, 4)) *yp = v;
+                                } else {
+                                    __half *yp = reinterpret_cast<__half *>(p.y) + yi;
+                                    if (!EVA_BAD_G(BUF_Y, yp, 2)) *yp = __float2half_rn(v);
+                                }
                             }
                         } else {
-                            __stcg(p.partial + ((size_t)tok * p.Gs + ts) * p.Npad + o, v);
+                            float *pp = p.partial + ((size_t)tok * p.Gs + ts) * p.Npad + o;
+                            if (!EVA_BAD_G(BUF_PARTIAL, pp, 4)) __stcg(pp, v);
                         }
                     }
                 }
@@ -389,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1) eva_lookup_kernel(const LookupPar
     __threadfence();
     __syncthreads();
     if (tid == 0) {
-        const unsigned prev = atomicAdd(p.counters + tt, 1u);
+        const unsigned prev = EVA_BAD_G(BUF_COUNTERS, p.counters + tt, 4) ? 0u : atomicAdd(p.counters + tt, 1u);
         s_last = (prev == (unsigned)(p.Gs - 1)) ? 1u : 0u;
     }
     __syncthreads();
@@ -401,12 +526,21 @@ __global__ void __launch_bounds__(kThreads, 1) eva_lookup_kernel(const LookupPar
         const int tok = idx / rows, o = r0 + idx % rows;
         const float *pp = p.partial + (size_t)tok * p.Gs * p.Npad + o;
         float sum = 0.f;
-        for (int k = 0; k < p.Gs; ++k) sum += __ldcg(pp + (size_t)k * p.Npad);
+        for (int k = 0; k < p.Gs; ++k) {
+            const float *q = pp + (size_t)k * p.Npad;
+            sum += EVA_BAD_G(BUF_PARTIAL, q, 4) ? 0.f : __ldcg(q);
+        }
         const size_t yi = (size_t)tok * p.N + o;
-        if (p.out_f32) reinterpret_cast<float *>(p.y)[yi] = sum;
-        else reinterpret_cast<__half *>(p.y)[yi] = __float2half_rn(sum);
+        if (p.out_f32) {
+            float *yp = reinterpret_cast<float *>(p.y) + yi;
+            if (!EVA_BAD_G(BUF_Y, yp, 4)) *yp = sum;
+        } else {
+            __half *yp = reinterpret_cast<__half *>(p.y) + yi;
+            if (!EVA_BAD_G(BUF_Y, yp, 2)) *yp = __float2half_rn(sum);
+        }
     }
-    if (tid == 0) p.counters[tt] = 0u;  // ready for the next call on this stream
+    if (tid == 0 && !EVA_BAD_G(BUF_COUNTERS, p.counters + tt, 4))
+        p.counters[tt] = 0u;  // ready for the next call on this stream
 }
 
 // ----------------------------------------------------- Hadamard rotation

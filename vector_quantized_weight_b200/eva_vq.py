@@ -13,7 +13,7 @@ import os
 from . import build as _build
 
 EVA_OK, EVA_ERR_INVALID_ARG, EVA_ERR_UNSUPPORTED, EVA_ERR_CUDA, EVA_ERR_OOM, \
-    EVA_ERR_DEVICE_TIMEOUT, EVA_ERR_NO_DEVICE = range(7)
+    EVA_ERR_DEVICE_TIMEOUT, EVA_ERR_NO_DEVICE, EVA_ERR_DEVICE_CHECK = range(8)
 EVA_F16, EVA_F32 = 0, 1
 EVA_PATH_AUTO, EVA_PATH_OC_LOOKUP, EVA_PATH_DEQUANT_MMA = 0, 1, 2
 
@@ -21,7 +21,7 @@ EVA_PATH_AUTO, EVA_PATH_OC_LOOKUP, EVA_PATH_DEQUANT_MMA = 0, 1, 2
 ABI_FUNCTIONS = (
     "eva_vq_linear_create", "eva_vq_linear_run", "eva_vq_linear_run_host",
     "eva_vq_linear_destroy", "eva_vq_unpack_indices", "eva_vq_sync_status",
-    "eva_vq_status_string", "eva_vq_linear_info",
+    "eva_vq_status_string", "eva_vq_linear_info", "eva_vq_device_check_record",
 )
 
 
@@ -53,7 +53,8 @@ _lib = None
 
 
 def library_path() -> str:
-    return _build.LIB
+    """The regular library, or the checked build when EVA_VQ_CHECKED=1."""
+    return _build.CHECKED_LIB if os.environ.get("EVA_VQ_CHECKED") == "1" else _build.LIB
 
 
 def load(build_if_missing: bool = True) -> ctypes.CDLL:
@@ -61,11 +62,12 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     global _lib
     if _lib is not None:
         return _lib
-    if not os.path.exists(_build.LIB):
+    path = library_path()
+    if not os.path.exists(path):
         if not build_if_missing:
-            raise RuntimeError(f"{_build.LIB} is missing; build it with vector_quantized_weight_b200.build")
-        _build.build()
-    lib = ctypes.CDLL(_build.LIB)
+            raise RuntimeError(f"{path} is missing; build it with vector_quantized_weight_b200.build")
+        _build.build(checked=path == _build.CHECKED_LIB)
+    lib = ctypes.CDLL(path)
     P, I32, H = ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p
     lib.eva_vq_linear_create.argtypes = [ctypes.POINTER(H), ctypes.POINTER(eva_vq_desc), P, P, P, P, P, P]
     lib.eva_vq_linear_run.argtypes = [H, P, I32, P, P]
@@ -76,6 +78,7 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.eva_vq_status_string.argtypes = [ctypes.c_int]
     lib.eva_vq_status_string.restype = ctypes.c_char_p
     lib.eva_vq_linear_info.argtypes = [H, ctypes.POINTER(eva_vq_info)]
+    lib.eva_vq_device_check_record.argtypes = [H, P]
     for fn in ABI_FUNCTIONS:
         if fn != "eva_vq_status_string":
             getattr(lib, fn).restype = ctypes.c_int
@@ -121,6 +124,12 @@ def eva_vq_unpack_indices(h: int, wi_out: int, stream: int | None) -> None:
 
 def eva_vq_sync_status(h: int) -> int:
     return int(load().eva_vq_sync_status(h))
+
+
+def eva_vq_device_check_record(h: int) -> list:
+    rec = (ctypes.c_int32 * 8)()
+    _check("eva_vq_device_check_record", load().eva_vq_device_check_record(h, rec))
+    return list(rec)
 
 
 def eva_vq_linear_info(h: int) -> eva_vq_info:

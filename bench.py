@@ -49,6 +49,9 @@ def parse_args():
     ap.add_argument("--batch", type=int, default=None)
     ap.add_argument("--ring", type=int, default=0, help="ring length (0: > 2x L2)")
     ap.add_argument("--path", type=int, default=0)
+    ap.add_argument("--x-pool", type=int, default=4,
+                    help="distinct activation buffers cycled by the ring (activations stay in L2, "
+                         "as the output of the preceding op does in a decode step)")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -235,7 +238,8 @@ def main():
         for r in range(ring):
             lay = synth.make_layer(shape, seed + 1000 * (r + 1) + 7919 * rank)
             layers.append(eva_vq.from_layer(lay, max_batch=B, path=args.path, device=dev))
-            xs.append(torch.from_numpy(synth.make_x(shape.K, B, seed + r)).to(dev))
+            if r < max(1, args.x_pool):
+                xs.append(torch.from_numpy(synth.make_x(shape.K, B, seed + r)).to(dev))
             ys.append(torch.empty((B, shape.N), dtype=torch.float16, device=dev))
     torch.cuda.synchronize(dev)
     info = layers[0].info()
@@ -243,7 +247,7 @@ def main():
     def sweep(n, start=0):
         for i in range(n):
             r = (start + i) % ring
-            layers[r](xs[r], out=ys[r], stream=stream)
+            layers[r](xs[r % len(xs)], out=ys[r], stream=stream)
 
     # Warm-up (eager), then capture one full ring and a remainder graph.
     with torch.cuda.stream(stream):
@@ -346,6 +350,7 @@ def main():
                    "residual_group": shape.residual_group, "hadamard_block": shape.hadamard_block,
                    "ring_layers": ring, "ring_index_bytes": ring * wi_bytes,
                    "l2_bytes": l2, "l2_policy": "inputs larger than L2: ring of distinct layers > 2x L2",
+                   "x_pool": len(xs),
                    "graph": "one CUDA graph per ring sweep", "parallelism": f"replicas x{world}",
                    "grid": info.grid, "kernels_per_step": info.kernels_per_run},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 3), "peak": peak, "unit": "GB/s",

@@ -113,8 +113,11 @@ cudaError_t launch_pdl(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_
     return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
+// Dynamic shared memory of the lookup kernel: the OC image (with the residual
+// table in its unused half for one token, or a second image for a token
+// pair) and the staged x~ slice.
 size_t lookup_smem(bool pair_t, bool resid) {
-    return (size_t)kOcBytes + ((pair_t && resid) ? (size_t)kOcBytes : 0);
+    return (size_t)kOcBytes + ((pair_t && resid) ? (size_t)kOcBytes : 0) + kXStageBytes;
 }
 
 cudaError_t set_smem_attrs() {

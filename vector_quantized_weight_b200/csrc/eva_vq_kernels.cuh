@@ -26,7 +26,7 @@ namespace eva {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kMaxTilesPerWarp = 12;
+constexpr int kMaxTilesPerWarp = 8;
 
 extern __shared__ __align__(1024) uint8_t eva_smem[];
 
@@ -112,13 +112,14 @@ __device__ __forceinline__ uint4 ldg_stream(const void *p) {
     return r;
 }
 
-// The 32 index bytes of one lane in one unit.  Volatile with a memory
+// The 32 index bytes of one lane in one unit (two 16-byte halves 512 bytes
+// apart, see wi_unit_pos).  Volatile with a memory
 // clobber so the compiler keeps it where it is written: the tile loop issues
 // exactly one unit of lookahead instead of hoisting every tile's load.
 __device__ __forceinline__ void ldg_unit(const void *p, uint4 &a, uint4 &b) {
     asm volatile(
         "ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%8];\n\t"
-        "ld.global.nc.L1::no_allocate.v4.u32 {%4,%5,%6,%7}, [%8+16];"
+        "ld.global.nc.L1::no_allocate.v4.u32 {%4,%5,%6,%7}, [%8+512];"
         : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
         : "l"(p)
         : "memory");
@@ -193,33 +194,99 @@ __device__ __forceinline__ float load_x(const LookupParams &p, int tok, int k) {
     return __half2float(__ushort_as_half(b));
 }
 
+// ------------------------------------------------------------- x staging
+//
+// The x~ values of one K-slice (256 inputs per token, as fp32) are staged once
+// per CTA in shared memory: one warp per token, 8 consecutive inputs per lane
+// with 128-bit loads when aligned; zeros past K or past B.
+constexpr uint32_t kXStageBytes = 2u * kSliceK * 4u;   // room for a token pair
+
+template <bool PAIR_T>
+__device__ __forceinline__ void stage_x(const LookupParams &p, int s, int pr, int warp, int lane,
+                                        uint32_t x_off) {
+    constexpr int NTOK = PAIR_T ? 2 : 1;
+    if (warp >= NTOK) return;
+    const int tok = PAIR_T ? 2 * pr + warp : 0;
+    const int k0 = s * kSliceK + 8 * lane;
+    float v[8];
+    const size_t i = (size_t)tok * p.K + k0;
+    bool done = false;
+    if (tok < p.B && k0 + 8 <= p.K) {
+        if (p.x_f32 && (i & 3) == 0) {
+            const float4 *xp = reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(p.x) + i);
+            if (!EVA_BAD_G(BUF_X, xp, 32)) {
+                const float4 a = __ldcg(xp), b = __ldcg(xp + 1);
+                v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+                v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+                done = true;
+            }
+        } else if (!p.x_f32 && (i & 7) == 0) {
+            const uint4 *xp = reinterpret_cast<const uint4 *>(reinterpret_cast<const __half *>(p.x) + i);
+            if (!EVA_BAD_G(BUF_X, xp, 16)) {
+                const uint4 r = __ldcg(xp);
+                const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const __half2 h2 = *reinterpret_cast<const __half2 *>(&w[j]);
+                    v[2 * j] = __low2float(h2);
+                    v[2 * j + 1] = __high2float(h2);
+                }
+                done = true;
+            }
+        }
+    }
+    if (!done) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = load_x(p, tok, k0 + j);
+    }
+    const uint32_t off = x_off + (uint32_t)(warp * kSliceK + 8 * lane) * 4u;
+    if (!EVA_BAD_S(off) && !EVA_BAD_S(off + 28u)) {
+        *reinterpret_cast<float4 *>(eva_smem + off) = make_float4(v[0], v[1], v[2], v[3]);
+        *reinterpret_cast<float4 *>(eva_smem + off + 16) = make_float4(v[4], v[5], v[6], v[7]);
+    }
+}
+
+__device__ __forceinline__ float lds_x(const LookupParams &p, uint32_t x_off, int idx) {
+    const uint32_t off = x_off + 4u * (uint32_t)idx;
+    return EVA_BAD_S(off) ? 0.f : *reinterpret_cast<const float *>(eva_smem + off);
+}
+
+// B fragments of the codebook product for this warp's centroid tiles
+// nt = warp + kWarps j: lane (g, q) holds WC[cb][8 nt + g][q] as tf32.
+__device__ __forceinline__ void load_codebook_frag(const LookupParams &p, int cb, int warp, int g, int q,
+                                                   uint32_t (&bf)[4]) {
+    const __half *wcb = p.wc + (size_t)cb * kCent * kD;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const __half *wp = wcb + (8 * (warp + kWarps * j) + g) * kD + q;
+        bf[j] = to_tf32(EVA_BAD_G(BUF_WC, wp, 2) ? 0.f : __half2float(__ldg(wp)));
+    }
+}
+
 // --------------------------------------------------- output-codebook build
 //
 // OC[j][c] = sum_{u<4} x~[256 s + 4 j + u] * WC[cb][c][u] for the 64 sub-vectors
 // of slice s: a 64 x 4 by 4 x 256 product on tensor cores (m16n8k4, tf32; the
 // fp16 inputs are exact in tf32 and their products exact in fp32), rounded to
 // fp16 and stored in the conflict-free image.  Warp w builds the centroid
-// columns 8 nt .. 8 nt + 7 of nt = w, w + kWarps, ...
+// columns 8 nt .. 8 nt + 7 of nt = w + kWarps j, j = 0..3.
 template <bool PAIR_T>
-__device__ __forceinline__ void build_oc(const LookupParams &p, int s, int cb, int pr, int warp,
-                                         int g, int q) {
+__device__ __forceinline__ void build_oc(const LookupParams &p, int warp, int g, int q,
+                                         const uint32_t (&bf)[4], uint32_t x_off) {
     constexpr int NTOK = PAIR_T ? 2 : 1;
     uint32_t ax[NTOK][4][2];
 #pragma unroll
-    for (int tk = 0; tk < NTOK; ++tk) {
-        const int tok = PAIR_T ? 2 * pr + tk : 0;
+    for (int tk = 0; tk < NTOK; ++tk)
 #pragma unroll
         for (int mt = 0; mt < 4; ++mt) {
-            const int k = s * kSliceK + kD * (16 * mt + g) + q;
-            ax[tk][mt][0] = to_tf32(load_x(p, tok, k));
-            ax[tk][mt][1] = to_tf32(load_x(p, tok, k + 8 * kD));
+            const int idx = tk * kSliceK + kD * (16 * mt + g) + q;
+            ax[tk][mt][0] = to_tf32(lds_x(p, x_off, idx));
+            ax[tk][mt][1] = to_tf32(lds_x(p, x_off, idx + 8 * kD));
         }
-    }
-    const __half *wcb = p.wc + (size_t)cb * kCent * kD;
-#pragma unroll 1
-    for (int nt = warp; nt < kCent / 8; nt += kWarps) {
-        const __half *wp = wcb + (8 * nt + g) * kD + q;
-        const uint32_t b0 = to_tf32(EVA_BAD_G(BUF_WC, wp, 2) ? 0.f : __half2float(*wp));
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int nt = warp + kWarps * j;
+        const uint32_t b0 = bf[j];
         if (!PAIR_T) {
             // D[mt][2h + cc] = OC[16 mt + g + 8 h][8 nt + 2 q + cc]; the word of
             // class i pairs sub-vector g + 8 i (m-tile i/2) with +32 (m-tile i/2 + 2).
@@ -281,16 +348,14 @@ __device__ __forceinline__ void build_oc(const LookupParams &p, int s, int cb, i
 // position m, so every store hits its own bank.  T = P_lo[v & 15] +
 // P_hi[v >> 4] with 4-input partial sums.
 template <bool PAIR_T>
-__device__ __forceinline__ void build_sign_table(const LookupParams &p, int s, int pr, int warp,
-                                                 int lane, uint32_t t_off) {
+__device__ __forceinline__ void build_sign_table(const LookupParams &p, int warp, int lane,
+                                                 uint32_t t_off, uint32_t x_off) {
     constexpr int NTOK = PAIR_T ? 2 : 1;
     float xv[NTOK][8];
 #pragma unroll
-    for (int tk = 0; tk < NTOK; ++tk) {
-        const int tok = PAIR_T ? 2 * pr + tk : 0;
+    for (int tk = 0; tk < NTOK; ++tk)
 #pragma unroll
-        for (int i = 0; i < 8; ++i) xv[tk][i] = load_x(p, tok, s * kSliceK + 8 * lane + i);
-    }
+        for (int i = 0; i < 8; ++i) xv[tk][i] = lds_x(p, x_off, tk * kSliceK + 8 * lane + i);
 #pragma unroll 1
     for (int hn = warp; hn < 16; hn += kWarps) {
         float phi[NTOK];
@@ -318,8 +383,24 @@ __device__ __forceinline__ void build_sign_table(const LookupParams &p, int s, i
 }
 
 // ------------------------------------------------------------ lookup kernel
+//
+// Grid: Gs x Gt CTAs; CTA (ts, tt) owns K-slices [s0, s1) and row tiles
+// [t0, t1); warp w owns the tiles t0 + w + kWarps i.  Per slice (and per
+// codebook spanned): stage x~, build the OC image, then every warp streams
+// its units: unpack an index byte into a shared-memory address with one byte
+// permute, read the OC word, and feed four words per k-step into an MMA that
+// sums them (the adder tree).  Partial sums of a row group are combined by
+// the last of its Gs CTAs in a fixed order.
+//
+// Before the dependency wait the kernel only touches weights: the bulk L2
+// prefetch of its index range and the codebook fragments.  For one token
+// without residual the launch bounds of two CTAs per SM (128 registers) leave
+// room for the next layer's CTA to run that prologue while this one computes,
+// so the weight stream of layer l+1 overlaps the lookups of layer l; the
+// token-pair and residual variants need more registers and run one CTA per SM.
+
 template <bool PAIR_T, bool RESID>
-__global__ void __launch_bounds__(kThreads, 1) eva_lookup_kernel(const LookupParams p) {
+__global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_lookup_kernel(const LookupParams p) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, q = lane & 3;
     const int ts = blockIdx.x % p.Gs, tt = blockIdx.x / p.Gs;
@@ -330,9 +411,12 @@ __global__ void __launch_bounds__(kThreads, 1) eva_lookup_kernel(const LookupPar
     constexpr uint32_t OC_OFF = 0;
     constexpr uint32_t HI_OFF = PAIR_T ? 128u : 0u;                      // a2/a3 column offset
     constexpr uint32_t T_OFF = PAIR_T ? (uint32_t)kOcBytes : 128u;       // residual table
+    constexpr uint32_t X_OFF = (PAIR_T && RESID) ? 2u * kOcBytes : (uint32_t)kOcBytes;
+    const int cb_first = p.tiles_per_cb ? t0 / p.tiles_per_cb : 0;
+    const int cb_last = p.tiles_per_cb ? (t1 - 1) / p.tiles_per_cb : 0;
 
-    // Weights do not depend on the preceding kernel: start streaming them
-    // into L2 before waiting for it.
+    // ---- prologue: weights only ----
+    pdl_launch();
     if (tid < s1 - s0) {
         const size_t u = (size_t)(s0 + tid) * p.T + t0;
         const uint32_t nt = (uint32_t)(t1 - t0);
@@ -345,7 +429,9 @@ __global__ void __launch_bounds__(kThreads, 1) eva_lookup_kernel(const LookupPar
                 prefetch_l2_bulk(p.al + u * kAlphaUnitHalves, nt * kAlphaUnitHalves * 2);
         }
     }
-    pdl_launch();
+    uint32_t bfrag[4];
+    int cur_cb = cb_first;   // codebook whose fragments bfrag holds
+    load_codebook_frag(p, cb_first, warp, g, q, bfrag);
 
     // Routing matrices of the accumulating MMA (B operand, 16 x 8, 0/1).
     // One token: column 0 sums the low half of a0/a1 and the high half of
@@ -364,55 +450,55 @@ __global__ void __launch_bounds__(kThreads, 1) eva_lookup_kernel(const LookupPar
         if (!PAIR_T) bt = (g == (q >> 1)) ? ONE_LO : 0u;
         else bt = (g == 2 * (q >> 1)) ? ONE_LO : (g == 2 * (q >> 1) + 1 ? ONE_HI : 0u);
     }
-    uint32_t mcol4[4][2];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        mcol4[i][0] = RESID ? 4u * sign_pos(lane, i, 0) : 0u;
-        mcol4[i][1] = RESID ? 4u * sign_pos(lane, i, 2) : 0u;
-    }
 
-    pdl_wait();
+    pdl_wait();   // x (and y, partials, counters) belong to the stream order from here on
 
     const int npairs = PAIR_T ? (p.B + 1) / 2 : 1;
-    const int cb_first = p.tiles_per_cb ? t0 / p.tiles_per_cb : 0;
-    const int cb_last = p.tiles_per_cb ? (t1 - 1) / p.tiles_per_cb : 0;
-
     for (int pr = 0; pr < npairs; ++pr) {
         float acc[kMaxTilesPerWarp][4];
 #pragma unroll
         for (int i = 0; i < kMaxTilesPerWarp; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
 
         for (int s = s0; s < s1; ++s) {
+            stage_x<PAIR_T>(p, s, pr, warp, lane, X_OFF);
             for (int cb = cb_first; cb <= cb_last; ++cb) {
-                // This warp's tiles t0 + warp + kWarps i that use codebook cb
-                // form the index range [i0, i1).
+                // This warp's tiles that use codebook cb: the index range [i0, i1).
                 int i0 = 0, i1 = ntw;
                 if (p.tiles_per_cb) {
                     const int lo = max(cb * p.tiles_per_cb, t0), hi = (cb + 1) * p.tiles_per_cb;
                     i0 = max(0, (lo - t0 - warp + kWarps - 1) / kWarps);
                     i1 = min(ntw, max(0, (hi - t0 - warp + kWarps - 1) / kWarps));
+                    if (cb != cur_cb) {
+                        load_codebook_frag(p, cb, warp, g, q, bfrag);
+                        cur_cb = cb;
+                    }
                 }
-                // The first unit's indices load while the codebook image builds.
+                // Lookahead buffer: the first tile's indices load (from L2, where
+                // the prologue's bulk prefetch put them) while the image builds.
                 uint4 nx0 = make_uint4(0u, 0u, 0u, 0u), nx1 = nx0;
-                if (i0 < i1) {
-                    const uint8_t *up = p.wi + ((size_t)s * p.T + t0 + warp + kWarps * i0) * kUnitBytes + lane * 32;
-                    if (!EVA_BAD_G(BUF_WI, up, 32)) ldg_unit(up, nx0, nx1);
+                {
+                    const int la = i0;
+                    if (la < i1) {
+                        const uint8_t *up = p.wi + ((size_t)s * p.T + t0 + warp + kWarps * la) * kUnitBytes + 16 * lane;
+                        if (!EVA_BAD_G(BUF_WI, up, 16) && !EVA_BAD_G(BUF_WI, up + 512, 16)) ldg_unit(up, nx0, nx1);
+                    }
                 }
-                __syncthreads();  // previous image fully consumed
-                build_oc<PAIR_T>(p, s, cb, pr, warp, g, q);
-                if (RESID && cb == cb_first) build_sign_table<PAIR_T>(p, s, pr, warp, lane, T_OFF);
+                __syncthreads();  // x~ staged; previous image fully consumed
+                build_oc<PAIR_T>(p, warp, g, q, bfrag, X_OFF);
+                if (RESID && cb == cb_first) build_sign_table<PAIR_T>(p, warp, lane, T_OFF, X_OFF);
                 __syncthreads();
 #pragma unroll
                 for (int i = 0; i < kMaxTilesPerWarp; ++i) {
                     if (i < i0 || i >= i1) continue;
-                    const int t = t0 + warp + kWarps * i;
-                    const size_t unit = (size_t)s * p.T + t;
+                    const size_t unit = (size_t)s * p.T + t0 + warp + kWarps * i;
                     const uint4 v0 = nx0, v1 = nx1;
                     if (i + 1 < i1) {  // one unit of lookahead
-                        const uint8_t *up = p.wi + (unit + kWarps) * kUnitBytes + lane * 32;
-                        if (!EVA_BAD_G(BUF_WI, up, 32)) ldg_unit(up, nx0, nx1);
+                        const uint8_t *up = p.wi + (unit + kWarps) * kUnitBytes + 16 * lane;
+                        if (!EVA_BAD_G(BUF_WI, up, 16) && !EVA_BAD_G(BUF_WI, up + 512, 16)) ldg_unit(up, nx0, nx1);
                     }
                     const uint32_t wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+                    // Even and odd k-steps accumulate in two chains.
+                    float db[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int s8 = 0; s8 < 8; ++s8) {
                         const uint32_t cw = (4u * lane + 16u * s8) & 127u;   // 4 * oc_col(lane, s8)
@@ -424,8 +510,14 @@ __global__ void __launch_bounds__(kThreads, 1) eva_lookup_kernel(const LookupPar
                         const uint32_t a1 = EVA_BAD_S(o1) ? 0u : lds32(o1);
                         const uint32_t a2 = EVA_BAD_S(o2) ? 0u : lds32(o2);
                         const uint32_t a3 = EVA_BAD_S(o3) ? 0u : lds32(o3);
-                        mma_f16_k16(acc[i], a0, a1, a2, a3, bo0, bo1);
+                        if (s8 & 1) mma_f16_k16(db, a0, a1, a2, a3, bo0, bo1);
+                        else mma_f16_k16(acc[i], a0, a1, a2, a3, bo0, bo1);
+                        // Compiler-only fence (emits nothing): at most 16 lookups
+                        // in flight per warp, which keeps the kernel in 128 registers.
+                        if ((s8 & 3) == 3) asm volatile("" ::: "memory");
                     }
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) acc[i][e] += db[e];
                     if (RESID) {
                         const uint8_t *sp = p.sg + unit * kSignUnitBytes + lane * 16;
                         const uint4 sv = EVA_BAD_G(BUF_SG, sp, 16) ? make_uint4(0u, 0u, 0u, 0u) : ldg_stream(sp);
@@ -433,10 +525,11 @@ __global__ void __launch_bounds__(kThreads, 1) eva_lookup_kernel(const LookupPar
                         float dt[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                         for (int mi = 0; mi < 4; ++mi) {
-                            const uint32_t o0 = T_OFF + __byte_perm(sw[mi], mcol4[mi][0], 0x5504);
-                            const uint32_t o1 = T_OFF + __byte_perm(sw[mi], mcol4[mi][0], 0x5514);
-                            const uint32_t o2 = T_OFF + __byte_perm(sw[mi], mcol4[mi][1], 0x5524);
-                            const uint32_t o3 = T_OFF + __byte_perm(sw[mi], mcol4[mi][1], 0x5534);
+                            const uint32_t m0 = 4u * sign_pos(lane, mi, 0), m2 = 4u * sign_pos(lane, mi, 2);
+                            const uint32_t o0 = T_OFF + __byte_perm(sw[mi], m0, 0x5504);
+                            const uint32_t o1 = T_OFF + __byte_perm(sw[mi], m0, 0x5514);
+                            const uint32_t o2 = T_OFF + __byte_perm(sw[mi], m2, 0x5524);
+                            const uint32_t o3 = T_OFF + __byte_perm(sw[mi], m2, 0x5534);
                             const uint32_t a0 = EVA_BAD_S(o0) ? 0u : lds32(o0);
                             const uint32_t a1 = EVA_BAD_S(o1) ? 0u : lds32(o1);
                             const uint32_t a2 = EVA_BAD_S(o2) ? 0u : lds32(o2);
@@ -509,17 +602,22 @@ __global__ void __launch_bounds__(kThreads, 1) eva_lookup_kernel(const LookupPar
     if (p.Gs == 1) return;
 
     // Split-K reduction: the last CTA of this row group sums the partials of
-    // all slice groups in a fixed order (bitwise reproducible).
+    // all slice groups in a fixed order (bitwise reproducible).  One thread
+    // publishes the CTA's partials with a gpu-scope fence before counting in;
+    // the last one to count in fences again before reading them.
     __shared__ unsigned s_last;
-    __threadfence();
     __syncthreads();
     if (tid == 0) {
-        const unsigned prev = EVA_BAD_G(BUF_COUNTERS, p.counters + tt, 4) ? 0u : atomicAdd(p.counters + tt, 1u);
+        unsigned prev = 0;
+        if (!EVA_BAD_G(BUF_COUNTERS, p.counters + tt, 4)) {
+            asm volatile("fence.acq_rel.gpu;" ::: "memory");
+            prev = atomicAdd(p.counters + tt, 1u);
+        }
         s_last = (prev == (unsigned)(p.Gs - 1)) ? 1u : 0u;
+        if (s_last) asm volatile("fence.acq_rel.gpu;" ::: "memory");
     }
     __syncthreads();
     if (!s_last) return;
-    __threadfence();
     const int r0 = kTileRows * t0, r1 = min(kTileRows * t1, p.N);
     const int rows = r1 - r0;
     for (int idx = tid; idx < rows * p.B; idx += kThreads) {
@@ -527,8 +625,8 @@ __global__ void __launch_bounds__(kThreads, 1) eva_lookup_kernel(const LookupPar
         const float *pp = p.partial + (size_t)tok * p.Gs * p.Npad + o;
         float sum = 0.f;
         for (int k = 0; k < p.Gs; ++k) {
-            const float *q = pp + (size_t)k * p.Npad;
-            sum += EVA_BAD_G(BUF_PARTIAL, q, 4) ? 0.f : __ldcg(q);
+            const float *q2 = pp + (size_t)k * p.Npad;
+            sum += EVA_BAD_G(BUF_PARTIAL, q2, 4) ? 0.f : __ldcg(q2);
         }
         const size_t yi = (size_t)tok * p.N + o;
         if (p.out_f32) {

@@ -38,9 +38,12 @@ constexpr int kOcBytes = kCent * kOcRowBytes;       // 64 KB image
 __host__ __device__ __forceinline__ int oc_col(int lane, int s8) { return (lane + 4 * s8) & 31; }
 
 // Index byte `b` of a unit (0..1023) -> (row in tile, sub-vector in slice).
-// Byte b = 32*lane + 4*s8 + r, r selecting the A register a_r.
+// Byte b = 512*h + 16*lane + 4*(s8 - 4h) + r: the first 16 bytes of all 32
+// lanes (k-steps 0..3) come first, then the second 16 (k-steps 4..7), so each
+// 128-bit load of a warp reads 512 contiguous bytes (coalesced in global
+// memory, bank-conflict-free in shared memory).  r selects the A register a_r.
 __host__ __device__ __forceinline__ void wi_unit_pos(int b, int &row, int &jl) {
-    const int lane = b >> 5, s8 = (b >> 2) & 7, r = b & 3;
+    const int h = b >> 9, lane = (b >> 4) & 31, s8 = 4 * h + ((b >> 2) & 3), r = b & 3;
     row = (lane >> 2) + ((r & 1) ? 8 : 0);
     jl = oc_col(lane, s8) + ((r & 2) ? 32 : 0);
 }

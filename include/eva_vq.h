@@ -108,6 +108,22 @@ EVA_API eva_status_t eva_vq_linear_create(eva_vq_linear_t *out, const eva_vq_des
 EVA_API eva_status_t eva_vq_linear_run(eva_vq_linear_t h, const void *x, int32_t B, void *y,
                                eva_stream_t stream);
 
+/* Flags of eva_vq_linear_run_ex. */
+enum {
+    /* x was not written by the kernel that precedes this call on `stream`
+     * (for example it was produced earlier and already waited for, or it is
+     * the shared input of several independent layers).  The layer may then
+     * read x and do all of its lookups while the preceding kernel is still
+     * running; y and the handle's workspace are still written in stream
+     * order.  Passing it when x IS produced by the preceding kernel is a
+     * race. */
+    EVA_RUN_INPUT_READY = 1u
+};
+
+/* eva_vq_linear_run with flags (0 gives eva_vq_linear_run). */
+EVA_API eva_status_t eva_vq_linear_run_ex(eva_vq_linear_t h, const void *x, int32_t B, void *y,
+                                          eva_stream_t stream, uint32_t flags);
+
 /*
  * The same call with HOST buffers: copies x (host fp16 [B][K]) to the
  * handle's staging buffer, runs, copies y back to y_host ([B][N] of
@@ -140,6 +156,18 @@ EVA_API eva_status_t eva_vq_sync_status(eva_vq_linear_t h);
  * (low, high), [7] access size.  In the regular build the record stays zero.
  */
 EVA_API eva_status_t eva_vq_device_check_record(eva_vq_linear_t h, int32_t *out8);
+
+/*
+ * Diagnostic hook of the timeline build (compiled with EVA_TIMELINE):
+ * synchronises the device and copies up to max_entries %globaltimer stamps
+ * (ns) of the last lookup launch to host memory `out`, 8 per CTA: start,
+ * after the dependency wait, codebook image started, image built, lookups
+ * done, split-K handshake done, finalisation done (0 when a CTA skipped a
+ * phase).  *count receives the number copied.  The regular build returns
+ * EVA_ERR_UNSUPPORTED.
+ */
+EVA_API eva_status_t eva_vq_debug_timeline(eva_vq_linear_t h, uint64_t *out, int32_t max_entries,
+                                           int32_t *count);
 
 /* Static string for a status code. */
 EVA_API const char *eva_vq_status_string(eva_status_t s);

@@ -145,3 +145,27 @@ def test_run_rejects_bad_arguments():
     assert lib.eva_vq_linear_run(h, None, 1, y.data_ptr(), None) == eva_vq.EVA_ERR_INVALID_ARG
     torch.cuda.synchronize()
     lin.close()
+
+
+@pytest.mark.parametrize("key,li,B", [("llama7b_layer", 0, 1), ("llama7b_block", 6, 4), ("gemma_3bit", 0, 1),
+                                      ("llama70b", 0, 8)])
+def test_input_ready_flag_matches_plain_run(key, li, B):
+    """EVA_RUN_INPUT_READY only relaxes when x is read: results are bitwise
+    those of the plain call, also for back-to-back calls on one handle."""
+    import torch
+    from vector_quantized_weight_b200 import eva_vq
+    cfg = synth.CONFIGS[key]
+    shape = cfg.layers[li]
+    layer = synth.make_layer(shape, 31)
+    lin = eva_vq.from_layer(layer, max_batch=B)
+    xs = [torch.from_numpy(synth.make_x(shape.K, B, 40 + i)).cuda() for i in range(3)]
+    ref = [lin(x).clone() for x in xs]
+    outs = [lin(x, input_ready=True) for x in xs]      # back to back, same workspace
+    torch.cuda.synchronize()
+    for a, b in zip(ref, outs):
+        assert torch.equal(a, b)
+    lib = eva_vq.load()
+    y = torch.empty_like(ref[0])
+    assert lib.eva_vq_linear_run_ex(lin.handle, xs[0].data_ptr(), B, y.data_ptr(), None, 2) == \
+        eva_vq.EVA_ERR_INVALID_ARG
+    lin.close()

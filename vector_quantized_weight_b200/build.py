@@ -11,6 +11,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libeva_vq.so")
 CHECKED_LIB = os.path.join(HERE, "libeva_vq_checked.so")   # device-side bounds checks
+TIMELINE_LIB = os.path.join(HERE, "libeva_vq_timeline.so") # per-CTA phase timestamps
 SOURCES = [os.path.join(HERE, "csrc", "eva_vq.cu")]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
               "-shared", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden"]
@@ -35,13 +36,15 @@ def up_to_date(lib: str = LIB) -> bool:
     return all(os.path.getmtime(f) <= t for f in _inputs())
 
 
-def build(force: bool = False, verbose: bool = False, checked: bool = False) -> str:
+def build(force: bool = False, verbose: bool = False, checked: bool = False,
+          timeline: bool = False) -> str:
     """Compile the library; checked=True builds the variant with device-side
-    bounds checks (EVA_DEVICE_CHECKS) into libeva_vq_checked.so."""
-    lib = CHECKED_LIB if checked else LIB
+    bounds checks (EVA_DEVICE_CHECKS), timeline=True the one that stamps each
+    CTA's phases (EVA_TIMELINE).  Both are diagnostics builds."""
+    lib = CHECKED_LIB if checked else (TIMELINE_LIB if timeline else LIB)
     if not force and up_to_date(lib):
         return lib
-    extra = ["-DEVA_DEVICE_CHECKS"] if checked else []
+    extra = ["-DEVA_DEVICE_CHECKS"] if checked else (["-DEVA_TIMELINE"] if timeline else [])
     cmd = [_nvcc(), *NVCC_FLAGS, *extra, "-I", os.path.join(ROOT, "include"), "-o", lib + ".tmp", *SOURCES]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
@@ -52,4 +55,5 @@ def build(force: bool = False, verbose: bool = False, checked: bool = False) -> 
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, checked="--checked" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, checked="--checked" in sys.argv,
+                timeline="--timeline" in sys.argv))

@@ -34,6 +34,7 @@ struct eva_vq_linear {
     unsigned *counters = nullptr;       // [Gt]
     float *xt = nullptr;                // rotated input [max_batch][K]
     int *status = nullptr;              // device error word
+    unsigned long long *timeline = nullptr;  // timeline build: [grid][8] stamps
     void *x_stage = nullptr, *y_stage = nullptr;
     int64_t workspace_bytes = 0;
     int last_grid = 0, last_kernels = 0, last_path = 0;
@@ -85,7 +86,7 @@ void plan_grid(eva_vq_linear *h) {
     for (int gs = 1; gs <= std::min(S, P); ++gs) {
         for (int gt = 1; gt <= std::min(T, P / gs); ++gt) {
             const int tiles = (T + gt - 1) / gt, slices = (S + gs - 1) / gs;
-            if ((tiles + kWarps - 1) / kWarps > kMaxTilesPerWarp) continue;
+            if (tiles > kMaxCtaTiles) continue;
             int builds = 1;
             if (h->tiles_per_cb) builds = (tiles + h->tiles_per_cb - 1) / h->tiles_per_cb + 1;
             double cost = (double)slices * (builds * 320.0 + tiles * 32.0);
@@ -115,20 +116,21 @@ cudaError_t launch_pdl(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_
 
 // Dynamic shared memory of the lookup kernel: the OC image (with the residual
 // table in its unused half for one token, or a second image for a token
-// pair) and the staged x~ slice.
-size_t lookup_smem(bool pair_t, bool resid) {
-    return (size_t)kOcBytes + ((pair_t && resid) ? (size_t)kOcBytes : 0) + kXStageBytes;
+// pair), the staged x~ slice and the running sums of `tiles` row tiles.
+size_t lookup_smem(bool pair_t, bool resid, int tiles) {
+    return (size_t)kOcBytes + ((pair_t && resid) ? (size_t)kOcBytes : 0) + kXStageBytes +
+           (size_t)tiles * kTileRows * 2 * 4;
 }
 
 cudaError_t set_smem_attrs() {
     cudaError_t e;
-    e = cudaFuncSetAttribute(eva_lookup_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lookup_smem(false, false));
+    e = cudaFuncSetAttribute(eva_lookup_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lookup_smem(false, false, kMaxCtaTiles));
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(eva_lookup_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lookup_smem(false, true));
+    e = cudaFuncSetAttribute(eva_lookup_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lookup_smem(false, true, kMaxCtaTiles));
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(eva_lookup_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lookup_smem(true, false));
+    e = cudaFuncSetAttribute(eva_lookup_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lookup_smem(true, false, kMaxCtaTiles));
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(eva_lookup_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lookup_smem(true, true));
+    e = cudaFuncSetAttribute(eva_lookup_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lookup_smem(true, true, kMaxCtaTiles));
     if (e != cudaSuccess) return e;
     return cudaFuncSetAttribute(eva_hadamard_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 4096 * 4);
 }
@@ -136,7 +138,7 @@ cudaError_t set_smem_attrs() {
 void free_handle(eva_vq_linear *h) {
     if (!h) return;
     void *ptrs[] = {h->wi, h->sg, h->al, h->wc, h->hsign, h->partial, h->counters, h->xt,
-                    h->status, h->x_stage, h->y_stage};
+                    h->status, h->x_stage, h->y_stage, h->timeline};
     for (void *p : ptrs)
         if (p) cudaFree(p);
     delete h;
@@ -229,6 +231,10 @@ eva_status_t eva_vq_linear_create(eva_vq_linear_t *out, const eva_vq_desc *desc,
     chk(dalloc(&h->partial, h->Gs > 1 ? (size_t)desc->max_batch * h->Gs * h->Npad * sizeof(float) : 0, &ws));
     chk(dalloc(&h->counters, (size_t)h->Gt * sizeof(unsigned), &ws));
     chk(dalloc(&h->status, 8 * sizeof(int), &ws));
+#ifdef EVA_TIMELINE
+    chk(dalloc(&h->timeline, (size_t)h->Gs * h->Gt * 8 * sizeof(unsigned long long), &ws));
+    if (e == cudaSuccess) chk(cudaMemsetAsync(h->timeline, 0, (size_t)h->Gs * h->Gt * 8 * 8, s));
+#endif
     const size_t ybytes = (size_t)desc->max_batch * N * (desc->out_dtype == EVA_F32 ? 4 : 2);
     chk(dalloc(&h->x_stage, (size_t)desc->max_batch * K * sizeof(__half), &ws));
     chk(dalloc(&h->y_stage, ybytes, &ws));
@@ -264,7 +270,14 @@ eva_status_t eva_vq_linear_create(eva_vq_linear_t *out, const eva_vq_desc *desc,
 }
 
 eva_status_t eva_vq_linear_run(eva_vq_linear_t h, const void *x, int32_t B, void *y, eva_stream_t stream) {
+    return eva_vq_linear_run_ex(h, x, B, y, stream, 0u);
+}
+
+eva_status_t eva_vq_linear_run_ex(eva_vq_linear_t h, const void *x, int32_t B, void *y, eva_stream_t stream,
+                                  uint32_t flags) {
     if (!h || !x || !y || !aligned16(x) || !aligned16(y)) return EVA_ERR_INVALID_ARG;
+    if (flags & ~(uint32_t)EVA_RUN_INPUT_READY) return EVA_ERR_INVALID_ARG;
+    const int input_ready = (flags & EVA_RUN_INPUT_READY) ? 1 : 0;
     if (B < 1 || B > h->desc.max_batch) return EVA_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const eva_vq_desc &d = h->desc;
@@ -291,13 +304,14 @@ eva_status_t eva_vq_linear_run(eva_vq_linear_t h, const void *x, int32_t B, void
     p.Gt = h->Gt;
     p.tiles_per_cb = h->tiles_per_cb;
     p.out_f32 = d.out_dtype == EVA_F32 ? 1 : 0;
+    p.input_ready = d.hadamard_block ? 0 : input_ready;   // x~ comes from the rotation kernel
 
     if (d.hadamard_block) {
         const int b = d.hadamard_block;
         const int thr = std::min(b / 2, 1024);
         e = launch_pdl(eva_hadamard_kernel, dim3(d.K / b, B), dim3(thr), (size_t)b * sizeof(float), s,
                        reinterpret_cast<const __half *>(x), (const int8_t *)h->hsign, h->xt, d.K, b,
-                       (float)(1.0 / std::sqrt((double)b)));
+                       (float)(1.0 / std::sqrt((double)b)), input_ready);
         if (e != cudaSuccess) return cuda_status(e);
         ++kernels;
         p.x = h->xt;
@@ -307,7 +321,10 @@ eva_status_t eva_vq_linear_run(eva_vq_linear_t h, const void *x, int32_t B, void
     const bool pair_t = B > 1;
     const bool resid = d.residual_group != 0;
     const dim3 grid(h->Gs * h->Gt), block(kThreads);
-    const size_t smem = lookup_smem(pair_t, resid);
+    const size_t smem = lookup_smem(pair_t, resid, (h->T + h->Gt - 1) / h->Gt);
+#ifdef EVA_TIMELINE
+    p.timeline = h->timeline;
+#endif
 #ifdef EVA_DEVICE_CHECKS
     {
         const long long units = (long long)h->S * h->T;
@@ -389,6 +406,21 @@ eva_status_t eva_vq_device_check_record(eva_vq_linear_t h, int32_t *out8) {
     cudaError_t e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return cuda_status(e);
     return cuda_status(cudaMemcpy(out8, h->status, 8 * sizeof(int), cudaMemcpyDeviceToHost));
+}
+
+eva_status_t eva_vq_debug_timeline(eva_vq_linear_t h, uint64_t *out, int32_t max_entries, int32_t *count) {
+    if (!h || !out || !count || max_entries < 0) return EVA_ERR_INVALID_ARG;
+    *count = 0;
+#ifdef EVA_TIMELINE
+    const int n = std::min(max_entries, h->Gs * h->Gt * 8);
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e == cudaSuccess) e = cudaMemcpy(out, h->timeline, (size_t)n * 8, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_status(e);
+    *count = n;
+    return EVA_OK;
+#else
+    return EVA_ERR_UNSUPPORTED;
+#endif
 }
 
 eva_status_t eva_vq_linear_info(eva_vq_linear_t h, eva_vq_info *info) {

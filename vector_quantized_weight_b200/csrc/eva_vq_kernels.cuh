@@ -26,7 +26,9 @@ namespace eva {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kMaxTilesPerWarp = 8;
+constexpr int kMaxCtaTiles = 128;  // row tiles per CTA (shared-memory accumulator size)
+constexpr int kLookahead = 4;      // units of index bytes in flight per warp
+constexpr uint32_t kAccBytes = kMaxCtaTiles * kTileRows * 2 * 4;
 
 extern __shared__ __align__(1024) uint8_t eva_smem[];
 
@@ -43,6 +45,8 @@ struct LookupParams {
     int Gs, Gt;              // CTA grid: blockIdx.x = tt * Gs + ts
     int tiles_per_cb;        // 0: shared codebook; else row tiles per codebook
     int x_f32, out_f32;
+    int input_ready;         // x was not written by the preceding kernel: read it
+                             // before the dependency wait (outputs still wait)
 #ifdef EVA_DEVICE_CHECKS
     // Debug build only: bounds of every buffer the kernel touches.  A
     // violating access is skipped and the first one is recorded.
@@ -52,7 +56,22 @@ struct LookupParams {
     int *chk_record;         // [0] count, [1] line, [2] buffer, [3] block, [4] thread,
                              // [5] offset low, [6] offset high, [7] size
 #endif
+#ifdef EVA_TIMELINE
+    unsigned long long *timeline;   // [grid][8] %globaltimer stamps of the last run
+#endif
 };
+
+// Timeline build only: thread 0 of each CTA stamps phase boundaries.
+#ifdef EVA_TIMELINE
+__device__ __forceinline__ unsigned long long eva_globaltimer() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+#define EVA_STAMP(ph) do { if (threadIdx.x == 0) p.timeline[blockIdx.x * 8 + (ph)] = eva_globaltimer(); } while (0)
+#else
+#define EVA_STAMP(ph) do { } while (0)
+#endif
 
 enum { BUF_WI = 0, BUF_SG, BUF_AL, BUF_WC, BUF_X, BUF_PARTIAL, BUF_COUNTERS, BUF_Y, BUF_SMEM };
 
@@ -412,10 +431,12 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
     constexpr uint32_t HI_OFF = PAIR_T ? 128u : 0u;                      // a2/a3 column offset
     constexpr uint32_t T_OFF = PAIR_T ? (uint32_t)kOcBytes : 128u;       // residual table
     constexpr uint32_t X_OFF = (PAIR_T && RESID) ? 2u * kOcBytes : (uint32_t)kOcBytes;
+    constexpr uint32_t ACC_OFF = X_OFF + kXStageBytes;   // per-CTA running sums
     const int cb_first = p.tiles_per_cb ? t0 / p.tiles_per_cb : 0;
     const int cb_last = p.tiles_per_cb ? (t1 - 1) / p.tiles_per_cb : 0;
 
     // ---- prologue: weights only ----
+    EVA_STAMP(0);
     pdl_launch();
     if (tid < s1 - s0) {
         const size_t u = (size_t)(s0 + tid) * p.T + t0;
@@ -451,13 +472,17 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
         else bt = (g == 2 * (q >> 1)) ? ONE_LO : (g == 2 * (q >> 1) + 1 ? ONE_HI : 0u);
     }
 
-    pdl_wait();   // x (and y, partials, counters) belong to the stream order from here on
+    // x (unless the caller vouches it is ready), y, partials and counters
+    // belong to the stream order from here on.
+    if (!p.input_ready) pdl_wait();
+    EVA_STAMP(1);
 
     const int npairs = PAIR_T ? (p.B + 1) / 2 : 1;
+    constexpr int NTOK = PAIR_T ? 2 : 1;
+    const int ctiles = t1 - t0;
+    float *acc_s = reinterpret_cast<float *>(eva_smem + ACC_OFF);   // [ctiles][16 rows][2 tokens]
     for (int pr = 0; pr < npairs; ++pr) {
-        float acc[kMaxTilesPerWarp][4];
-#pragma unroll
-        for (int i = 0; i < kMaxTilesPerWarp; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+        for (int e = tid; e < ctiles * kTileRows * 2; e += kThreads) acc_s[e] = 0.f;
 
         for (int s = s0; s < s1; ++s) {
             stage_x<PAIR_T>(p, s, pr, warp, lane, X_OFF);
@@ -473,32 +498,42 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
                         cur_cb = cb;
                     }
                 }
-                // Lookahead buffer: the first tile's indices load (from L2, where
-                // the prologue's bulk prefetch put them) while the image builds.
-                uint4 nx0 = make_uint4(0u, 0u, 0u, 0u), nx1 = nx0;
-                {
-                    const int la = i0;
-                    if (la < i1) {
-                        const uint8_t *up = p.wi + ((size_t)s * p.T + t0 + warp + kWarps * la) * kUnitBytes + 16 * lane;
-                        if (!EVA_BAD_G(BUF_WI, up, 16) && !EVA_BAD_G(BUF_WI, up + 512, 16)) ldg_unit(up, nx0, nx1);
+                // Lookahead ring of kLookahead units: the first ones load (from
+                // L2, where the prologue's bulk prefetch put them) while the
+                // image builds; each processed tile refills the ring's tail.
+                uint4 nb[kLookahead][2];
+#pragma unroll
+                for (int d = 0; d < kLookahead; ++d) {
+                    nb[d][0] = nb[d][1] = make_uint4(0u, 0u, 0u, 0u);
+                    if (i0 + d < i1) {
+                        const uint8_t *up = p.wi + ((size_t)s * p.T + t0 + warp + kWarps * (i0 + d)) * kUnitBytes + 16 * lane;
+                        if (!EVA_BAD_G(BUF_WI, up, 16) && !EVA_BAD_G(BUF_WI, up + 512, 16)) ldg_unit(up, nb[d][0], nb[d][1]);
                     }
                 }
-                __syncthreads();  // x~ staged; previous image fully consumed
+                __syncthreads();  // x~ staged, accumulator cleared, previous image consumed
+                EVA_STAMP(2);
                 build_oc<PAIR_T>(p, warp, g, q, bfrag, X_OFF);
                 if (RESID && cb == cb_first) build_sign_table<PAIR_T>(p, warp, lane, T_OFF, X_OFF);
                 __syncthreads();
+                EVA_STAMP(3);
+#pragma unroll 1
+                for (int i = i0; i < i1; ++i) {
+                    const int tl = warp + kWarps * i;              // tile index within the CTA
+                    const size_t unit = (size_t)s * p.T + t0 + tl;
+                    const uint4 v0 = nb[0][0], v1 = nb[0][1];
 #pragma unroll
-                for (int i = 0; i < kMaxTilesPerWarp; ++i) {
-                    if (i < i0 || i >= i1) continue;
-                    const size_t unit = (size_t)s * p.T + t0 + warp + kWarps * i;
-                    const uint4 v0 = nx0, v1 = nx1;
-                    if (i + 1 < i1) {  // one unit of lookahead
-                        const uint8_t *up = p.wi + (unit + kWarps) * kUnitBytes + 16 * lane;
-                        if (!EVA_BAD_G(BUF_WI, up, 16) && !EVA_BAD_G(BUF_WI, up + 512, 16)) ldg_unit(up, nx0, nx1);
+                    for (int d = 0; d + 1 < kLookahead; ++d) {
+                        nb[d][0] = nb[d + 1][0];
+                        nb[d][1] = nb[d + 1][1];
+                    }
+                    if (i + kLookahead < i1) {
+                        const uint8_t *up = p.wi + (unit + (size_t)kWarps * kLookahead) * kUnitBytes + 16 * lane;
+                        if (!EVA_BAD_G(BUF_WI, up, 16) && !EVA_BAD_G(BUF_WI, up + 512, 16))
+                            ldg_unit(up, nb[kLookahead - 1][0], nb[kLookahead - 1][1]);
                     }
                     const uint32_t wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
                     // Even and odd k-steps accumulate in two chains.
-                    float db[4] = {0.f, 0.f, 0.f, 0.f};
+                    float da[4] = {0.f, 0.f, 0.f, 0.f}, db[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int s8 = 0; s8 < 8; ++s8) {
                         const uint32_t cw = (4u * lane + 16u * s8) & 127u;   // 4 * oc_col(lane, s8)
@@ -511,13 +546,10 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
                         const uint32_t a2 = EVA_BAD_S(o2) ? 0u : lds32(o2);
                         const uint32_t a3 = EVA_BAD_S(o3) ? 0u : lds32(o3);
                         if (s8 & 1) mma_f16_k16(db, a0, a1, a2, a3, bo0, bo1);
-                        else mma_f16_k16(acc[i], a0, a1, a2, a3, bo0, bo1);
-                        // Compiler-only fence (emits nothing): at most 16 lookups
-                        // in flight per warp, which keeps the kernel in 128 registers.
-                        if ((s8 & 3) == 3) asm volatile("" ::: "memory");
+                        else mma_f16_k16(da, a0, a1, a2, a3, bo0, bo1);
                     }
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) acc[i][e] += db[e];
+                    for (int e = 0; e < 4; ++e) da[e] += db[e];
                     if (RESID) {
                         const uint8_t *sp = p.sg + unit * kSignUnitBytes + lane * 16;
                         const uint4 sv = EVA_BAD_G(BUF_SG, sp, 16) ? make_uint4(0u, 0u, 0u, 0u) : ldg_stream(sp);
@@ -550,55 +582,60 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
                             const float a_g0 = __low2float(ag), a_g1 = __high2float(ag);
                             const float a_h0 = __low2float(ag8), a_h1 = __high2float(ag8);
                             if (!PAIR_T) {
-                                acc[i][0] += a_g0 * dt[0] + a_g1 * dt[1];
-                                acc[i][2] += a_h0 * dt[2] + a_h1 * dt[3];
+                                da[0] += a_g0 * dt[0] + a_g1 * dt[1];
+                                da[2] += a_h0 * dt[2] + a_h1 * dt[3];
                             } else {
-                                acc[i][0] += a_g0 * dt[0] + a_g1 * dt1[0];
-                                acc[i][1] += a_g0 * dt[1] + a_g1 * dt1[1];
-                                acc[i][2] += a_h0 * dt[2] + a_h1 * dt1[2];
-                                acc[i][3] += a_h0 * dt[3] + a_h1 * dt1[3];
+                                da[0] += a_g0 * dt[0] + a_g1 * dt1[0];
+                                da[1] += a_g0 * dt[1] + a_g1 * dt1[1];
+                                da[2] += a_h0 * dt[2] + a_h1 * dt1[2];
+                                da[3] += a_h0 * dt[3] + a_h1 * dt1[3];
                             }
                         }
+                    }
+                    // Lanes q = 0 hold column 0 (and 1): rows g and g + 8 of the tile.
+                    if (q == 0) {
+#pragma unroll
+                        for (int h = 0; h < 2; ++h)
+#pragma unroll
+                            for (int e = 0; e < NTOK; ++e) {
+                                const int ai = ((tl * kTileRows) + g + 8 * h) * 2 + e;
+                                if (!EVA_BAD_S(ACC_OFF + 4u * (uint32_t)ai)) acc_s[ai] += da[2 * h + e];
+                            }
                     }
                 }
             }
         }
 
-        // Epilogue of this token (pair): lanes q = 0 hold column 0 (and 1).
-        if (q == 0) {
-#pragma unroll
-            for (int i = 0; i < kMaxTilesPerWarp; ++i) {
-                if (i >= ntw) break;
-                const int t = t0 + warp + kWarps * i;
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int o = kTileRows * t + g + 8 * h;
-#pragma unroll
-                    for (int e = 0; e < (PAIR_T ? 2 : 1); ++e) {
-                        const int tok = PAIR_T ? 2 * pr + e : 0;
-                        const float v = acc[i][2 * h + e];
-                        if (tok >= p.B) continue;
-                        if (p.Gs == 1) {
-                            if (o < p.N) {
-                                const size_t yi = (size_t)tok * p.N + o;
-                                if (p.out_f32) {
-                                    float *yp = reinterpret_cast<float *>(p.y) + yi;
-                                    if (!EVA_BAD_G(BUF_Y, yp, 4)) *yp = v;
-                                } else {
-                                    __half *yp = reinterpret_cast<__half *>(p.y) + yi;
-                                    if (!EVA_BAD_G(BUF_Y, yp, 2)) *yp = __float2half_rn(v);
-                                }
-                            }
+        // Epilogue of this token (pair): coalesced stores of the accumulator.
+        __syncthreads();
+        if (pr == 0 && p.input_ready) pdl_wait();   // outputs follow the stream order
+        for (int e = 0; e < NTOK; ++e) {
+            const int tok = PAIR_T ? 2 * pr + e : 0;
+            if (tok >= p.B) break;
+            for (int r = tid; r < ctiles * kTileRows; r += kThreads) {
+                const int o = kTileRows * t0 + r;
+                const float v = acc_s[r * 2 + e];
+                if (p.Gs == 1) {
+                    if (o < p.N) {
+                        const size_t yi = (size_t)tok * p.N + o;
+                        if (p.out_f32) {
+                            float *yp = reinterpret_cast<float *>(p.y) + yi;
+                            if (!EVA_BAD_G(BUF_Y, yp, 4)) *yp = v;
                         } else {
-                            float *pp = p.partial + ((size_t)tok * p.Gs + ts) * p.Npad + o;
-                            if (!EVA_BAD_G(BUF_PARTIAL, pp, 4)) __stcg(pp, v);
+                            __half *yp = reinterpret_cast<__half *>(p.y) + yi;
+                            if (!EVA_BAD_G(BUF_Y, yp, 2)) *yp = __float2half_rn(v);
                         }
                     }
+                } else {
+                    float *pp = p.partial + ((size_t)tok * p.Gs + ts) * p.Npad + o;
+                    if (!EVA_BAD_G(BUF_PARTIAL, pp, 4)) __stcg(pp, v);
                 }
             }
         }
+        __syncthreads();   // accumulator read before the next pair clears it
     }
 
+    EVA_STAMP(4);
     if (p.Gs == 1) return;
 
     // Split-K reduction: the last CTA of this row group sums the partials of
@@ -617,16 +654,25 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
         if (s_last) asm volatile("fence.acq_rel.gpu;" ::: "memory");
     }
     __syncthreads();
+    EVA_STAMP(5);
     if (!s_last) return;
     const int r0 = kTileRows * t0, r1 = min(kTileRows * t1, p.N);
     const int rows = r1 - r0;
     for (int idx = tid; idx < rows * p.B; idx += kThreads) {
         const int tok = idx / rows, o = r0 + idx % rows;
         const float *pp = p.partial + (size_t)tok * p.Gs * p.Npad + o;
+        // All Gs loads of a chunk are issued before the (ordered) sum, so the
+        // finalisation costs one L2 round trip per 16 slice groups.
         float sum = 0.f;
-        for (int k = 0; k < p.Gs; ++k) {
-            const float *q2 = pp + (size_t)k * p.Npad;
-            sum += EVA_BAD_G(BUF_PARTIAL, q2, 4) ? 0.f : __ldcg(q2);
+        for (int k0 = 0; k0 < p.Gs; k0 += 16) {
+            float v[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const float *q2 = pp + (size_t)(k0 + k) * p.Npad;
+                v[k] = (k0 + k < p.Gs && !EVA_BAD_G(BUF_PARTIAL, q2, 4)) ? __ldcg(q2) : 0.f;
+            }
+#pragma unroll
+            for (int k = 0; k < 16; ++k) sum += v[k];
         }
         const size_t yi = (size_t)tok * p.N + o;
         if (p.out_f32) {
@@ -639,6 +685,7 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
     }
     if (tid == 0 && !EVA_BAD_G(BUF_COUNTERS, p.counters + tt, 4))
         p.counters[tt] = 0u;  // ready for the next call on this stream
+    EVA_STAMP(6);
 }
 
 // ----------------------------------------------------- Hadamard rotation
@@ -649,11 +696,11 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
 __global__ void __launch_bounds__(1024) eva_hadamard_kernel(const __half *__restrict__ x,
                                                             const int8_t *__restrict__ hs,
                                                             float *__restrict__ xt, int K, int b,
-                                                            float scale) {
+                                                            float scale, int input_ready) {
     float *sb = reinterpret_cast<float *>(eva_smem);
     const int blk = blockIdx.x, tok = blockIdx.y;
     pdl_launch();
-    pdl_wait();  // x may be the output of the preceding kernel
+    if (!input_ready) pdl_wait();  // x may be the output of the preceding kernel
     const unsigned short *xb =
         reinterpret_cast<const unsigned short *>(x) + (size_t)tok * K + (size_t)blk * b;
     for (int i = threadIdx.x; i < b; i += blockDim.x) sb[i] = __half2float(__ushort_as_half(__ldcg(xb + i)));
@@ -667,6 +714,7 @@ __global__ void __launch_bounds__(1024) eva_hadamard_kernel(const __half *__rest
         }
     }
     __syncthreads();
+    if (input_ready) pdl_wait();  // the rotated input is this handle's workspace
     for (int i = threadIdx.x; i < b; i += blockDim.x) {
         const int k = blk * b + i;
         xt[(size_t)tok * K + k] = (float)hs[k] * sb[i] * scale;

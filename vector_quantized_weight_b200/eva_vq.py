@@ -18,10 +18,13 @@ EVA_F16, EVA_F32 = 0, 1
 EVA_PATH_AUTO, EVA_PATH_OC_LOOKUP, EVA_PATH_DEQUANT_MMA = 0, 1, 2
 
 # Every function the header declares; the CPU tests check the library exports them.
+EVA_RUN_INPUT_READY = 1
+
 ABI_FUNCTIONS = (
-    "eva_vq_linear_create", "eva_vq_linear_run", "eva_vq_linear_run_host",
+    "eva_vq_linear_create", "eva_vq_linear_run", "eva_vq_linear_run_ex", "eva_vq_linear_run_host",
     "eva_vq_linear_destroy", "eva_vq_unpack_indices", "eva_vq_sync_status",
     "eva_vq_status_string", "eva_vq_linear_info", "eva_vq_device_check_record",
+    "eva_vq_debug_timeline",
 )
 
 
@@ -53,8 +56,13 @@ _lib = None
 
 
 def library_path() -> str:
-    """The regular library, or the checked build when EVA_VQ_CHECKED=1."""
-    return _build.CHECKED_LIB if os.environ.get("EVA_VQ_CHECKED") == "1" else _build.LIB
+    """The regular library; EVA_VQ_CHECKED=1 selects the device-check build and
+    EVA_VQ_TIMELINE=1 the phase-timeline build (diagnostics only)."""
+    if os.environ.get("EVA_VQ_CHECKED") == "1":
+        return _build.CHECKED_LIB
+    if os.environ.get("EVA_VQ_TIMELINE") == "1":
+        return _build.TIMELINE_LIB
+    return _build.LIB
 
 
 def load(build_if_missing: bool = True) -> ctypes.CDLL:
@@ -66,11 +74,12 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     if not os.path.exists(path):
         if not build_if_missing:
             raise RuntimeError(f"{path} is missing; build it with vector_quantized_weight_b200.build")
-        _build.build(checked=path == _build.CHECKED_LIB)
+        _build.build(checked=path == _build.CHECKED_LIB, timeline=path == _build.TIMELINE_LIB)
     lib = ctypes.CDLL(path)
     P, I32, H = ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p
     lib.eva_vq_linear_create.argtypes = [ctypes.POINTER(H), ctypes.POINTER(eva_vq_desc), P, P, P, P, P, P]
     lib.eva_vq_linear_run.argtypes = [H, P, I32, P, P]
+    lib.eva_vq_linear_run_ex.argtypes = [H, P, I32, P, P, ctypes.c_uint32]
     lib.eva_vq_linear_run_host.argtypes = [H, P, I32, P, P]
     lib.eva_vq_linear_destroy.argtypes = [H]
     lib.eva_vq_unpack_indices.argtypes = [H, P, P]
@@ -79,6 +88,7 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.eva_vq_status_string.restype = ctypes.c_char_p
     lib.eva_vq_linear_info.argtypes = [H, ctypes.POINTER(eva_vq_info)]
     lib.eva_vq_device_check_record.argtypes = [H, P]
+    lib.eva_vq_debug_timeline.argtypes = [H, P, I32, ctypes.POINTER(I32)]
     for fn in ABI_FUNCTIONS:
         if fn != "eva_vq_status_string":
             getattr(lib, fn).restype = ctypes.c_int
@@ -110,6 +120,10 @@ def eva_vq_linear_run(h: int, x: int, B: int, y: int, stream: int | None) -> Non
     _check("eva_vq_linear_run", load().eva_vq_linear_run(h, x, int(B), y, stream))
 
 
+def eva_vq_linear_run_ex(h: int, x: int, B: int, y: int, stream: int | None, flags: int) -> None:
+    _check("eva_vq_linear_run_ex", load().eva_vq_linear_run_ex(h, x, int(B), y, stream, int(flags)))
+
+
 def eva_vq_linear_run_host(h: int, x_host: int, B: int, y_host: int, stream: int | None) -> None:
     _check("eva_vq_linear_run_host", load().eva_vq_linear_run_host(h, x_host, int(B), y_host, stream))
 
@@ -130,6 +144,13 @@ def eva_vq_device_check_record(h: int) -> list:
     rec = (ctypes.c_int32 * 8)()
     _check("eva_vq_device_check_record", load().eva_vq_device_check_record(h, rec))
     return list(rec)
+
+
+def eva_vq_debug_timeline(h: int, max_entries: int = 1 << 16) -> list:
+    buf = (ctypes.c_uint64 * max_entries)()
+    n = ctypes.c_int32()
+    _check("eva_vq_debug_timeline", load().eva_vq_debug_timeline(h, buf, max_entries, ctypes.byref(n)))
+    return list(buf[:n.value])
 
 
 def eva_vq_linear_info(h: int) -> eva_vq_info:
@@ -174,14 +195,15 @@ class VQLinear:
         self.handle = eva_vq_linear_create(self.desc, _ptr(wc), _ptr(wi), _ptr(signs), _ptr(alpha),
                                            _ptr(hsign), _stream_handle(stream))
 
-    def __call__(self, x, out=None, stream=None):
+    def __call__(self, x, out=None, stream=None, input_ready=False):
         import torch
         if x.dtype != torch.float16 or not x.is_cuda or not x.is_contiguous():
             raise ValueError("x must be a contiguous CUDA float16 tensor [B, K]")
         x2 = x.view(-1, self.K)
         B = x2.shape[0]
         y = out if out is not None else torch.empty((B, self.N), dtype=self.out_dtype, device=x.device)
-        eva_vq_linear_run(self.handle, _ptr(x2), B, _ptr(y), _stream_handle(stream))
+        eva_vq_linear_run_ex(self.handle, _ptr(x2), B, _ptr(y), _stream_handle(stream),
+                             EVA_RUN_INPUT_READY if input_ready else 0)
         return y
 
     def run_host(self, x_host, y_host, stream=None):

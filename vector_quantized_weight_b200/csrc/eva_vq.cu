@@ -24,14 +24,14 @@ struct eva_vq_linear {
     eva_vq_desc desc;
     int device = 0, sm_count = 0;
     int J = 0, S = 0, T = 0, Npad = 0, G = 1, tiles_per_cb = 0;
-    int Gs = 1, Gt = 1;                 // lookup grid (slice groups x row groups)
+    // Lookup grid per variant (index: token pair or not): Gs slice groups
+    // (one cluster) x Gt row groups, and its dynamic shared memory.
+    struct Plan { int Gs = 1, Gt = 1; size_t smem = 0; } plan[2];
     uint8_t *wi = nullptr;              // repacked indices
     uint8_t *sg = nullptr;              // repacked signs
     __half *al = nullptr;               // repacked alpha
     __half *wc = nullptr;               // codebooks [G][256][4]
     int8_t *hsign = nullptr;            // Hadamard signs [K]
-    float *partial = nullptr;           // [max_batch][Gs][Npad]
-    unsigned *counters = nullptr;       // [Gt]
     float *xt = nullptr;                // rotated input [max_batch][K]
     int *status = nullptr;              // device error word
     unsigned long long *timeline = nullptr;  // timeline build: [grid][8] stamps
@@ -75,45 +75,6 @@ eva_status_t validate_desc(const eva_vq_desc *d) {
     return EVA_OK;
 }
 
-// Pick the CTA rectangle (Gs slice groups x Gt row groups, Gs*Gt <= SMs) that
-// minimises the per-SM shared-memory-pipe time: lookups (32 warp-wide loads
-// per unit), output-codebook stores (256 per build, one build per slice and
-// codebook spanned) and the split-K epilogue.
-void plan_grid(eva_vq_linear *h) {
-    const int S = h->S, T = h->T, P = h->sm_count;
-    double best = 1e300;
-    int bs = 1, bt = std::min(T, P);
-    for (int gs = 1; gs <= std::min(S, P); ++gs) {
-        for (int gt = 1; gt <= std::min(T, P / gs); ++gt) {
-            const int tiles = (T + gt - 1) / gt, slices = (S + gs - 1) / gs;
-            if (tiles > kMaxCtaTiles) continue;
-            int builds = 1;
-            if (h->tiles_per_cb) builds = (tiles + h->tiles_per_cb - 1) / h->tiles_per_cb + 1;
-            double cost = (double)slices * (builds * 320.0 + tiles * 32.0);
-            cost += (gs > 1) ? 400.0 : 0.0;             // partials + fence + finalize
-            cost += 2000.0 * (double)(gs * gt) / (P * 64.0);  // mild preference for fewer CTAs
-            if (cost < best) { best = cost; bs = gs; bt = gt; }
-        }
-    }
-    h->Gs = bs;
-    h->Gt = bt;
-}
-
-template <typename K, typename... Args>
-cudaError_t launch_pdl(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = block;
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kernel, args...);
-}
-
 // Dynamic shared memory of the lookup kernel: the OC image (with the residual
 // table in its unused half for one token, or a second image for a token
 // pair), the staged x~ slice and the running sums of `tiles` row tiles.
@@ -122,23 +83,125 @@ size_t lookup_smem(bool pair_t, bool resid, int tiles) {
            (size_t)tiles * kTileRows * 2 * 4;
 }
 
+using LookupFn = void (*)(LookupParams);
+LookupFn lookup_fn(bool pair_t, bool resid, bool grouped) {
+    if (grouped) {
+        if (!pair_t) return resid ? eva_lookup_kernel<false, true, true> : eva_lookup_kernel<false, false, true>;
+        return resid ? eva_lookup_kernel<true, true, true> : eva_lookup_kernel<true, false, true>;
+    }
+    if (!pair_t) return resid ? eva_lookup_kernel<false, true, false> : eva_lookup_kernel<false, false, false>;
+    return resid ? eva_lookup_kernel<true, true, false> : eva_lookup_kernel<true, false, false>;
+}
+
+// Largest number of clusters of `cs` CTAs of this kernel resident at once.
+int max_active_clusters(LookupFn fn, size_t smem, int cs) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(cs * 64);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute a[1];
+    a[0].id = cudaLaunchAttributeClusterDimension;
+    a[0].val.clusterDim.x = cs;
+    a[0].val.clusterDim.y = 1;
+    a[0].val.clusterDim.z = 1;
+    cfg.attrs = a;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, (const void *)fn, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return n;
+}
+
+// Pick the CTA rectangle: Gs slice groups (one thread-block cluster, Gs <=
+// 16) x Gt row groups, every cluster resident in one wave with at most one
+// CTA of this layer per SM (the second slot stays free for the next layer's
+// prologue), at most kMaxCtaTiles row tiles per CTA.  The cost model counts
+// the latency-bound phases of a CTA: per slice the x~ staging and the image
+// build, per unit of lookups a share of the warps' tile loop, and the
+// cluster reduction.
+void plan_grid(eva_vq_linear *h, int pair_t) {
+    const int S = h->S, T = h->T, P = h->sm_count;
+    const bool resid = h->desc.residual_group != 0;
+    const LookupFn fn = lookup_fn(pair_t != 0, resid, h->tiles_per_cb != 0);
+    double best = 1e300;
+    eva_vq_linear::Plan pl;
+    pl.Gs = 1;
+    pl.Gt = std::min(T, P);
+    for (int gs = 1; gs <= std::min(S, 16); ++gs) {
+        const int gt_min = (T + kMaxCtaTiles - 1) / kMaxCtaTiles;
+        // Capacity with one CTA per SM: the occupancy query counts CTA slots,
+        // so ask with a footprint that leaves room for a single CTA per SM.
+        const size_t smem_one = std::max(lookup_smem(pair_t, resid, (T + gt_min - 1) / gt_min),
+                                         (size_t)120 * 1024);
+        const int clusters = max_active_clusters(fn, smem_one, gs);
+        // One CTA of this layer per SM: no more clusters than P / gs either.
+        const int gt_max = std::min({T, clusters, P / gs});
+        for (int gt = gt_min; gt <= gt_max; ++gt) {
+            const int tiles = (T + gt - 1) / gt, slices = (S + gs - 1) / gs;
+            int builds = 1;
+            if (h->tiles_per_cb) builds = (tiles + h->tiles_per_cb - 1) / h->tiles_per_cb + 1;
+            double cost = (double)slices * (1300.0 + 900.0 * builds + 250.0 * ((tiles + kWarps - 1) / kWarps));
+            cost += (gs > 1) ? 600.0 + 40.0 * gs : 0.0;
+            if (cost < best) {
+                best = cost;
+                pl.Gs = gs;
+                pl.Gt = gt;
+            }
+        }
+    }
+    pl.smem = lookup_smem(pair_t, resid, (T + pl.Gt - 1) / pl.Gt);
+    h->plan[pair_t] = pl;
+}
+
+// Launch with programmatic dependent launch (and a cluster shape when
+// cluster > 0) on the caller's stream.
+template <typename K, typename... Args>
+cudaError_t launch_pdl(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t st, int cluster,
+                       Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    int n = 1;
+    if (cluster > 0) {
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = cluster;
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        n = 2;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+
 cudaError_t set_smem_attrs() {
     cudaError_t e;
-    e = cudaFuncSetAttribute(eva_lookup_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lookup_smem(false, false, kMaxCtaTiles));
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(eva_lookup_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lookup_smem(false, true, kMaxCtaTiles));
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(eva_lookup_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lookup_smem(true, false, kMaxCtaTiles));
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(eva_lookup_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lookup_smem(true, true, kMaxCtaTiles));
-    if (e != cudaSuccess) return e;
+    for (int v = 0; v < 8; ++v) {
+        const LookupFn fn = lookup_fn(v & 1, (v >> 1) & 1, (v >> 2) & 1);
+        e = cudaFuncSetAttribute((const void *)fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+        // The limit also covers the one-CTA-per-SM footprint the planner's
+        // occupancy query uses; launches request only what they need.
+        e = cudaFuncSetAttribute((const void *)fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)std::max(lookup_smem(v & 1, (v >> 1) & 1, kMaxCtaTiles),
+                                               (size_t)120 * 1024));
+        if (e != cudaSuccess) return e;
+    }
     return cudaFuncSetAttribute(eva_hadamard_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 4096 * 4);
 }
 
 void free_handle(eva_vq_linear *h) {
     if (!h) return;
-    void *ptrs[] = {h->wi, h->sg, h->al, h->wc, h->hsign, h->partial, h->counters, h->xt,
-                    h->status, h->x_stage, h->y_stage, h->timeline};
+    void *ptrs[] = {h->wi, h->sg, h->al, h->wc, h->hsign, h->xt, h->status, h->x_stage,
+                    h->y_stage, h->timeline};
     for (void *p : ptrs)
         if (p) cudaFree(p);
     delete h;
@@ -210,14 +273,15 @@ eva_status_t eva_vq_linear_create(eva_vq_linear_t *out, const eva_vq_desc *desc,
     h->Npad = h->T * kTileRows;
     h->G = desc->codebook_rows ? N / desc->codebook_rows : 1;
     h->tiles_per_cb = desc->codebook_rows ? desc->codebook_rows / kTileRows : 0;
-    plan_grid(h);
-
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const long long units = (long long)h->S * h->T;
     int64_t ws = 0;
     cudaError_t e = cudaSuccess;
     auto chk = [&](cudaError_t r) { if (e == cudaSuccess) e = r; };
     chk(set_smem_attrs());
+    plan_grid(h, 0);
+    if (desc->max_batch > 1) plan_grid(h, 1);
+    const int max_grid = std::max(h->plan[0].Gs * h->plan[0].Gt, h->plan[1].Gs * h->plan[1].Gt);
     chk(dalloc(&h->wi, (size_t)units * kUnitBytes, nullptr));
     chk(dalloc(&h->wc, (size_t)h->G * kCent * kD * sizeof(__half), nullptr));
     if (desc->residual_group) {
@@ -228,12 +292,10 @@ eva_status_t eva_vq_linear_create(eva_vq_linear_t *out, const eva_vq_desc *desc,
         chk(dalloc(&h->hsign, (size_t)K, nullptr));
         chk(dalloc(&h->xt, (size_t)desc->max_batch * K * sizeof(float), &ws));
     }
-    chk(dalloc(&h->partial, h->Gs > 1 ? (size_t)desc->max_batch * h->Gs * h->Npad * sizeof(float) : 0, &ws));
-    chk(dalloc(&h->counters, (size_t)h->Gt * sizeof(unsigned), &ws));
     chk(dalloc(&h->status, 8 * sizeof(int), &ws));
 #ifdef EVA_TIMELINE
-    chk(dalloc(&h->timeline, (size_t)h->Gs * h->Gt * 8 * sizeof(unsigned long long), &ws));
-    if (e == cudaSuccess) chk(cudaMemsetAsync(h->timeline, 0, (size_t)h->Gs * h->Gt * 8 * 8, s));
+    chk(dalloc(&h->timeline, (size_t)max_grid * 8 * sizeof(unsigned long long), &ws));
+    if (e == cudaSuccess) chk(cudaMemsetAsync(h->timeline, 0, (size_t)max_grid * 8 * 8, s));
 #endif
     const size_t ybytes = (size_t)desc->max_batch * N * (desc->out_dtype == EVA_F32 ? 4 : 2);
     chk(dalloc(&h->x_stage, (size_t)desc->max_batch * K * sizeof(__half), &ws));
@@ -258,7 +320,6 @@ eva_status_t eva_vq_linear_create(eva_vq_linear_t *out, const eva_vq_desc *desc,
         chk(cudaGetLastError());
     }
     if (desc->hadamard_block) chk(cudaMemcpyAsync(h->hsign, hsign, (size_t)K, cudaMemcpyDeviceToDevice, s));
-    chk(cudaMemsetAsync(h->counters, 0, (size_t)h->Gt * sizeof(unsigned), s));
     chk(cudaMemsetAsync(h->status, 0, 8 * sizeof(int), s));
     if (e != cudaSuccess) {
         cudaStreamSynchronize(s);
@@ -291,8 +352,6 @@ eva_status_t eva_vq_linear_run_ex(eva_vq_linear_t h, const void *x, int32_t B, v
     p.wc = h->wc;
     p.x = x;
     p.x_f32 = 0;
-    p.partial = h->partial;
-    p.counters = h->counters;
     p.y = y;
     p.N = d.N;
     p.Npad = h->Npad;
@@ -300,8 +359,10 @@ eva_status_t eva_vq_linear_run_ex(eva_vq_linear_t h, const void *x, int32_t B, v
     p.S = h->S;
     p.T = h->T;
     p.B = B;
-    p.Gs = h->Gs;
-    p.Gt = h->Gt;
+    const bool pair_t = B > 1;
+    const eva_vq_linear::Plan &pl = h->plan[pair_t ? 1 : 0];
+    p.Gs = pl.Gs;
+    p.Gt = pl.Gt;
     p.tiles_per_cb = h->tiles_per_cb;
     p.out_f32 = d.out_dtype == EVA_F32 ? 1 : 0;
     p.input_ready = d.hadamard_block ? 0 : input_ready;   // x~ comes from the rotation kernel
@@ -309,7 +370,7 @@ eva_status_t eva_vq_linear_run_ex(eva_vq_linear_t h, const void *x, int32_t B, v
     if (d.hadamard_block) {
         const int b = d.hadamard_block;
         const int thr = std::min(b / 2, 1024);
-        e = launch_pdl(eva_hadamard_kernel, dim3(d.K / b, B), dim3(thr), (size_t)b * sizeof(float), s,
+        e = launch_pdl(eva_hadamard_kernel, dim3(d.K / b, B), dim3(thr), (size_t)b * sizeof(float), s, 0,
                        reinterpret_cast<const __half *>(x), (const int8_t *)h->hsign, h->xt, d.K, b,
                        (float)(1.0 / std::sqrt((double)b)), input_ready);
         if (e != cudaSuccess) return cuda_status(e);
@@ -318,25 +379,24 @@ eva_status_t eva_vq_linear_run_ex(eva_vq_linear_t h, const void *x, int32_t B, v
         p.x_f32 = 1;
     }
 
-    const bool pair_t = B > 1;
     const bool resid = d.residual_group != 0;
-    const dim3 grid(h->Gs * h->Gt), block(kThreads);
-    const size_t smem = lookup_smem(pair_t, resid, (h->T + h->Gt - 1) / h->Gt);
+    const dim3 grid(pl.Gs * pl.Gt), block(kThreads);
+    const size_t smem = pl.smem;
 #ifdef EVA_TIMELINE
     p.timeline = h->timeline;
 #endif
 #ifdef EVA_DEVICE_CHECKS
     {
         const long long units = (long long)h->S * h->T;
-        const void *base[8] = {h->wi, h->sg, h->al, h->wc, p.x, h->partial, h->counters, y};
+        const void *base[8] = {h->wi, h->sg, h->al, h->wc, p.x, nullptr, nullptr, y};
         const unsigned long long bytes[8] = {
             (unsigned long long)units * kUnitBytes,
             h->sg ? (unsigned long long)units * kSignUnitBytes : 0ull,
             h->al ? (unsigned long long)units * kAlphaUnitHalves * 2 : 0ull,
             (unsigned long long)h->G * kCent * kD * 2,
             (unsigned long long)B * d.K * (p.x_f32 ? 4 : 2),
-            h->partial ? (unsigned long long)d.max_batch * h->Gs * h->Npad * 4 : 0ull,
-            (unsigned long long)h->Gt * 4,
+            0ull,
+            0ull,
             (unsigned long long)B * d.N * (p.out_f32 ? 4 : 2)};
         for (int i = 0; i < 8; ++i) {
             p.chk_base[i] = base[i];
@@ -346,10 +406,7 @@ eva_status_t eva_vq_linear_run_ex(eva_vq_linear_t h, const void *x, int32_t B, v
         p.chk_record = h->status;
     }
 #endif
-    if (!pair_t && !resid) e = launch_pdl(eva_lookup_kernel<false, false>, grid, block, smem, s, p);
-    else if (!pair_t && resid) e = launch_pdl(eva_lookup_kernel<false, true>, grid, block, smem, s, p);
-    else if (pair_t && !resid) e = launch_pdl(eva_lookup_kernel<true, false>, grid, block, smem, s, p);
-    else e = launch_pdl(eva_lookup_kernel<true, true>, grid, block, smem, s, p);
+    e = launch_pdl(lookup_fn(pair_t, resid, h->tiles_per_cb != 0), grid, block, smem, s, pl.Gs, p);
     if (e != cudaSuccess) return cuda_status(e);
     ++kernels;
     h->last_grid = (int)grid.x;
@@ -412,7 +469,7 @@ eva_status_t eva_vq_debug_timeline(eva_vq_linear_t h, uint64_t *out, int32_t max
     if (!h || !out || !count || max_entries < 0) return EVA_ERR_INVALID_ARG;
     *count = 0;
 #ifdef EVA_TIMELINE
-    const int n = std::min(max_entries, h->Gs * h->Gt * 8);
+    const int n = std::min(max_entries, h->last_grid * 8);
     cudaError_t e = cudaDeviceSynchronize();
     if (e == cudaSuccess) e = cudaMemcpy(out, h->timeline, (size_t)n * 8, cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) return cuda_status(e);
@@ -435,7 +492,7 @@ eva_status_t eva_vq_linear_info(eva_vq_linear_t h, eva_vq_info *info) {
     info->workspace_bytes = h->workspace_bytes;
     info->slices = h->S;
     info->row_tiles = h->T;
-    info->grid = h->last_grid ? h->last_grid : h->Gs * h->Gt;
+    info->grid = h->last_grid ? h->last_grid : h->plan[0].Gs * h->plan[0].Gt;
     info->kernels_per_run = h->last_kernels ? h->last_kernels : (d.hadamard_block ? 2 : 1);
     info->path = h->last_path ? h->last_path : EVA_PATH_OC_LOOKUP;
     info->sm_count = h->sm_count;

@@ -38,11 +38,9 @@ struct LookupParams {
     const __half *al;        // repacked alpha units, [S][T] x 32 halves (residual only)
     const __half *wc;        // codebooks [G][256][4]
     const void *x;           // activations [B][K]: fp16, or fp32 when x_f32
-    float *partial;          // split-K partial sums [B][Gs][Npad]
-    unsigned *counters;      // per row group, self-resetting
     void *y;                 // output [B][N]
     int N, Npad, K, S, T, B;
-    int Gs, Gt;              // CTA grid: blockIdx.x = tt * Gs + ts
+    int Gs, Gt;              // CTA grid: blockIdx.x = tt * Gs + ts; clusters of Gs CTAs
     int tiles_per_cb;        // 0: shared codebook; else row tiles per codebook
     int x_f32, out_f32;
     int input_ready;         // x was not written by the preceding kernel: read it
@@ -152,6 +150,23 @@ __device__ __forceinline__ void prefetch_l2_bulk(const void *p, uint32_t bytes) 
 // allow the next kernel to start its prologue.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Thread-block-cluster barrier (release/acquire): every CTA of the cluster
+// has arrived and its shared-memory writes are visible cluster-wide.
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+                 "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// fp32 load from the shared memory of cluster CTA `rank` at the address this
+// CTA uses for the same variable (distributed shared memory).
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t local_addr, uint32_t rank) {
+    uint32_t ra;
+    float v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(local_addr), "r"(rank));
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra) : "memory");
+    return v;
+}
 
 __device__ __forceinline__ uint32_t to_tf32(float f) {
     uint32_t r;
@@ -403,13 +418,13 @@ __device__ __forceinline__ void build_sign_table(const LookupParams &p, int warp
 
 // ------------------------------------------------------------ lookup kernel
 //
-// Grid: Gs x Gt CTAs; CTA (ts, tt) owns K-slices [s0, s1) and row tiles
-// [t0, t1); warp w owns the tiles t0 + w + kWarps i.  Per slice (and per
+// Grid: Gs x Gt CTAs in clusters of Gs; CTA (ts, tt) owns K-slices [s0, s1)
+// and row tiles [t0, t1); warp w owns the tiles t0 + w + kWarps i.  Per slice (and per
 // codebook spanned): stage x~, build the OC image, then every warp streams
 // its units: unpack an index byte into a shared-memory address with one byte
 // permute, read the OC word, and feed four words per k-step into an MMA that
-// sums them (the adder tree).  Partial sums of a row group are combined by
-// the last of its Gs CTAs in a fixed order.
+// sums them (the adder tree).  The Gs partial sums of a row group are combined
+// inside its cluster through distributed shared memory.
 //
 // Before the dependency wait the kernel only touches weights: the bulk L2
 // prefetch of its index range and the codebook fragments.  For one token
@@ -418,7 +433,7 @@ __device__ __forceinline__ void build_sign_table(const LookupParams &p, int warp
 // so the weight stream of layer l+1 overlaps the lookups of layer l; the
 // token-pair and residual variants need more registers and run one CTA per SM.
 
-template <bool PAIR_T, bool RESID>
+template <bool PAIR_T, bool RESID, bool GROUPED>
 __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_lookup_kernel(const LookupParams p) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, q = lane & 3;
@@ -432,8 +447,9 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
     constexpr uint32_t T_OFF = PAIR_T ? (uint32_t)kOcBytes : 128u;       // residual table
     constexpr uint32_t X_OFF = (PAIR_T && RESID) ? 2u * kOcBytes : (uint32_t)kOcBytes;
     constexpr uint32_t ACC_OFF = X_OFF + kXStageBytes;   // per-CTA running sums
-    const int cb_first = p.tiles_per_cb ? t0 / p.tiles_per_cb : 0;
-    const int cb_last = p.tiles_per_cb ? (t1 - 1) / p.tiles_per_cb : 0;
+    // GROUPED: one codebook per tiles_per_cb row tiles (else one shared codebook).
+    const int cb_first = GROUPED ? t0 / p.tiles_per_cb : 0;
+    const int cb_last = GROUPED ? (t1 - 1) / p.tiles_per_cb : 0;
 
     // ---- prologue: weights only ----
     EVA_STAMP(0);
@@ -472,8 +488,8 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
         else bt = (g == 2 * (q >> 1)) ? ONE_LO : (g == 2 * (q >> 1) + 1 ? ONE_HI : 0u);
     }
 
-    // x (unless the caller vouches it is ready), y, partials and counters
-    // belong to the stream order from here on.
+    // x (unless the caller vouches it is ready) and y belong to the stream
+    // order from here on.
     if (!p.input_ready) pdl_wait();
     EVA_STAMP(1);
 
@@ -489,7 +505,7 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
             for (int cb = cb_first; cb <= cb_last; ++cb) {
                 // This warp's tiles that use codebook cb: the index range [i0, i1).
                 int i0 = 0, i1 = ntw;
-                if (p.tiles_per_cb) {
+                if (GROUPED) {
                     const int lo = max(cb * p.tiles_per_cb, t0), hi = (cb + 1) * p.tiles_per_cb;
                     i0 = max(0, (lo - t0 - warp + kWarps - 1) / kWarps);
                     i1 = min(ntw, max(0, (hi - t0 - warp + kWarps - 1) / kWarps));
@@ -606,86 +622,54 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
             }
         }
 
-        // Epilogue of this token (pair): coalesced stores of the accumulator.
-        __syncthreads();
+        // Epilogue of this token (pair): the Gs CTAs of this row group form a
+        // thread-block cluster; after a cluster barrier each one sums a share
+        // of the rows over all Gs running-sum arrays (distributed shared
+        // memory, fixed order: bitwise reproducible) and stores y.
         if (pr == 0 && p.input_ready) pdl_wait();   // outputs follow the stream order
-        for (int e = 0; e < NTOK; ++e) {
-            const int tok = PAIR_T ? 2 * pr + e : 0;
-            if (tok >= p.B) break;
-            for (int r = tid; r < ctiles * kTileRows; r += kThreads) {
+        EVA_STAMP(4);
+        cluster_sync_all();
+        EVA_STAMP(5);
+        {
+            const int crow = ctiles * kTileRows;
+            const int rlo = crow * ts / p.Gs, rhi = crow * (ts + 1) / p.Gs, nrow = rhi - rlo;
+            const uint32_t acc_addr = (uint32_t)__cvta_generic_to_shared(acc_s);
+            for (int idx = tid; idx < nrow * NTOK; idx += kThreads) {
+                const int e = idx / nrow, r = rlo + idx % nrow;
+                const int tok = PAIR_T ? 2 * pr + e : 0;
                 const int o = kTileRows * t0 + r;
-                const float v = acc_s[r * 2 + e];
-                if (p.Gs == 1) {
-                    if (o < p.N) {
-                        const size_t yi = (size_t)tok * p.N + o;
-                        if (p.out_f32) {
-                            float *yp = reinterpret_cast<float *>(p.y) + yi;
-                            if (!EVA_BAD_G(BUF_Y, yp, 4)) *yp = v;
-                        } else {
-                            __half *yp = reinterpret_cast<__half *>(p.y) + yi;
-                            if (!EVA_BAD_G(BUF_Y, yp, 2)) *yp = __float2half_rn(v);
-                        }
-                    }
+                if (tok >= p.B || o >= p.N) continue;
+                const uint32_t la = acc_addr + 4u * (uint32_t)(r * 2 + e);
+                float sum = 0.f;
+                for (int k0 = 0; k0 < p.Gs; k0 += 8) {
+                    float v[8];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        v[k] = (k0 + k < p.Gs && !EVA_BAD_S(ACC_OFF + 4u * (uint32_t)(r * 2 + e)))
+                                   ? ld_dsmem_f32(la, (uint32_t)(k0 + k)) : 0.f;
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) sum += v[k];
+                }
+                const size_t yi = (size_t)tok * p.N + o;
+                if (p.out_f32) {
+                    float *yp = reinterpret_cast<float *>(p.y) + yi;
+                    if (!EVA_BAD_G(BUF_Y, yp, 4)) *yp = sum;
                 } else {
-                    float *pp = p.partial + ((size_t)tok * p.Gs + ts) * p.Npad + o;
-                    if (!EVA_BAD_G(BUF_PARTIAL, pp, 4)) __stcg(pp, v);
+                    __half *yp = reinterpret_cast<__half *>(p.y) + yi;
+                    if (!EVA_BAD_G(BUF_Y, yp, 2)) *yp = __float2half_rn(sum);
                 }
             }
         }
-        __syncthreads();   // accumulator read before the next pair clears it
+        cluster_sync_all();   // peers are done reading this CTA's sums
     }
-
-    EVA_STAMP(4);
-    if (p.Gs == 1) return;
-
-    // Split-K reduction: the last CTA of this row group sums the partials of
-    // all slice groups in a fixed order (bitwise reproducible).  One thread
-    // publishes the CTA's partials with a gpu-scope fence before counting in;
-    // the last one to count in fences again before reading them.
-    __shared__ unsigned s_last;
-    __syncthreads();
-    if (tid == 0) {
-        unsigned prev = 0;
-        if (!EVA_BAD_G(BUF_COUNTERS, p.counters + tt, 4)) {
-            asm volatile("fence.acq_rel.gpu;" ::: "memory");
-            prev = atomicAdd(p.counters + tt, 1u);
-        }
-        s_last = (prev == (unsigned)(p.Gs - 1)) ? 1u : 0u;
-        if (s_last) asm volatile("fence.acq_rel.gpu;" ::: "memory");
-    }
-    __syncthreads();
-    EVA_STAMP(5);
-    if (!s_last) return;
-    const int r0 = kTileRows * t0, r1 = min(kTileRows * t1, p.N);
-    const int rows = r1 - r0;
-    for (int idx = tid; idx < rows * p.B; idx += kThreads) {
-        const int tok = idx / rows, o = r0 + idx % rows;
-        const float *pp = p.partial + (size_t)tok * p.Gs * p.Npad + o;
-        // All Gs loads of a chunk are issued before the (ordered) sum, so the
-        // finalisation costs one L2 round trip per 16 slice groups.
-        float sum = 0.f;
-        for (int k0 = 0; k0 < p.Gs; k0 += 16) {
-            float v[16];
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const float *q2 = pp + (size_t)(k0 + k) * p.Npad;
-                v[k] = (k0 + k < p.Gs && !EVA_BAD_G(BUF_PARTIAL, q2, 4)) ? __ldcg(q2) : 0.f;
-            }
-#pragma unroll
-            for (int k = 0; k < 16; ++k) sum += v[k];
-        }
-        const size_t yi = (size_t)tok * p.N + o;
-        if (p.out_f32) {
-            float *yp = reinterpret_cast<float *>(p.y) + yi;
-            if (!EVA_BAD_G(BUF_Y, yp, 4)) *yp = sum;
-        } else {
-            __half *yp = reinterpret_cast<__half *>(p.y) + yi;
-            if (!EVA_BAD_G(BUF_Y, yp, 2)) *yp = __float2half_rn(sum);
-        }
-    }
-    if (tid == 0 && !EVA_BAD_G(BUF_COUNTERS, p.counters + tt, 4))
-        p.counters[tt] = 0u;  // ready for the next call on this stream
     EVA_STAMP(6);
+#ifdef EVA_TIMELINE
+    if (tid == 0) {
+        unsigned smid;
+        asm volatile("mov.u32 %0, %smid;" : "=r"(smid));
+        p.timeline[blockIdx.x * 8 + 7] = smid;
+    }
+#endif
 }
 
 // ----------------------------------------------------- Hadamard rotation

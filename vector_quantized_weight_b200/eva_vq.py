@@ -56,8 +56,11 @@ _lib = None
 
 
 def library_path() -> str:
-    """The regular library; EVA_VQ_CHECKED=1 selects the device-check build and
-    EVA_VQ_TIMELINE=1 the phase-timeline build (diagnostics only)."""
+    """The regular library; EVA_VQ_CHECKED=1 selects the device-check build,
+    EVA_VQ_TIMELINE=1 the phase-timeline build (diagnostics only), and
+    EVA_VQ_LIBRARY=<path> any other build of the same C ABI."""
+    if os.environ.get("EVA_VQ_LIBRARY"):
+        return os.environ["EVA_VQ_LIBRARY"]
     if os.environ.get("EVA_VQ_CHECKED") == "1":
         return _build.CHECKED_LIB
     if os.environ.get("EVA_VQ_TIMELINE") == "1":

@@ -110,14 +110,15 @@ EVA_API eva_status_t eva_vq_linear_run(eva_vq_linear_t h, const void *x, int32_t
 
 /* Flags of eva_vq_linear_run_ex. */
 enum {
-    /* x was not written by the kernel that precedes this call on `stream`
-     * (for example it was produced earlier and already waited for, or it is
-     * the shared input of several independent layers).  The layer may then
-     * read x and do all of its lookups while the preceding kernel is still
-     * running; y and the handle's workspace are still written in stream
-     * order.  Passing it when x IS produced by the preceding kernel is a
-     * race. */
-    EVA_RUN_INPUT_READY = 1u
+    /* Neither x nor y is accessed by the kernel that precedes this call on
+     * `stream` (for example several layers that read activations produced
+     * earlier and write distinct outputs).  The layer then runs without
+     * waiting for that kernel, so consecutive independent layers overlap;
+     * it still completes after it, so later calls keep the stream order.
+     * A layer with a Hadamard rotation only reads x early (its rotated-input
+     * workspace stays in stream order).  Passing it when x or y IS used by
+     * the preceding kernel is a race. */
+    EVA_RUN_INDEPENDENT = 1u
 };
 
 /* eva_vq_linear_run with flags (0 gives eva_vq_linear_run). */

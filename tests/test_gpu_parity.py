@@ -149,9 +149,9 @@ def test_run_rejects_bad_arguments():
 
 @pytest.mark.parametrize("key,li,B", [("llama7b_layer", 0, 1), ("llama7b_block", 6, 4), ("gemma_3bit", 0, 1),
                                       ("llama70b", 0, 8)])
-def test_input_ready_flag_matches_plain_run(key, li, B):
-    """EVA_RUN_INPUT_READY only relaxes when x is read: results are bitwise
-    those of the plain call, also for back-to-back calls on one handle."""
+def test_independent_flag_matches_plain_run(key, li, B):
+    """EVA_RUN_INDEPENDENT only relaxes ordering: results are bitwise those of
+    the plain call, also for back-to-back calls on one handle (distinct y)."""
     import torch
     from vector_quantized_weight_b200 import eva_vq
     cfg = synth.CONFIGS[key]
@@ -160,7 +160,7 @@ def test_input_ready_flag_matches_plain_run(key, li, B):
     lin = eva_vq.from_layer(layer, max_batch=B)
     xs = [torch.from_numpy(synth.make_x(shape.K, B, 40 + i)).cuda() for i in range(3)]
     ref = [lin(x).clone() for x in xs]
-    outs = [lin(x, input_ready=True) for x in xs]      # back to back, same workspace
+    outs = [lin(x, independent=True) for x in xs]      # back to back, same handle
     torch.cuda.synchronize()
     for a, b in zip(ref, outs):
         assert torch.equal(a, b)

@@ -77,10 +77,13 @@ eva_status_t validate_desc(const eva_vq_desc *d) {
 
 // Dynamic shared memory of the lookup kernel: the OC image (with the residual
 // table in its unused half for one token, or a second image for a token
-// pair), the staged x~ slice and the running sums of `tiles` row tiles.
-size_t lookup_smem(bool pair_t, bool resid, int tiles) {
+// pair), the staged x~ slice, the running sums of `tiles` row tiles and the
+// cluster reduction stage.
+size_t lookup_smem(bool pair_t, bool resid, int tiles, int gs) {
+    const size_t tile_bytes = (size_t)kTileRows * 2 * 4;
+    const size_t stage_tiles = (size_t)((tiles + gs - 1) / gs) * gs;   // reduction stage
     return (size_t)kOcBytes + ((pair_t && resid) ? (size_t)kOcBytes : 0) + kXStageBytes +
-           (size_t)tiles * kTileRows * 2 * 4;
+           (size_t)tiles * tile_bytes + stage_tiles * tile_bytes;
 }
 
 using LookupFn = void (*)(LookupParams);
@@ -133,7 +136,7 @@ void plan_grid(eva_vq_linear *h, int pair_t) {
         const int gt_min = (T + kMaxCtaTiles - 1) / kMaxCtaTiles;
         // Capacity with one CTA per SM: the occupancy query counts CTA slots,
         // so ask with a footprint that leaves room for a single CTA per SM.
-        const size_t smem_one = std::max(lookup_smem(pair_t, resid, (T + gt_min - 1) / gt_min),
+        const size_t smem_one = std::max(lookup_smem(pair_t, resid, (T + gt_min - 1) / gt_min, gs),
                                          (size_t)120 * 1024);
         const int clusters = max_active_clusters(fn, smem_one, gs);
         // One CTA of this layer per SM: no more clusters than P / gs either.
@@ -151,7 +154,7 @@ void plan_grid(eva_vq_linear *h, int pair_t) {
             }
         }
     }
-    pl.smem = lookup_smem(pair_t, resid, (T + pl.Gt - 1) / pl.Gt);
+    pl.smem = lookup_smem(pair_t, resid, (T + pl.Gt - 1) / pl.Gt, pl.Gs);
     h->plan[pair_t] = pl;
 }
 
@@ -191,7 +194,7 @@ cudaError_t set_smem_attrs() {
         // The limit also covers the one-CTA-per-SM footprint the planner's
         // occupancy query uses; launches request only what they need.
         e = cudaFuncSetAttribute((const void *)fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)std::max(lookup_smem(v & 1, (v >> 1) & 1, kMaxCtaTiles),
+                                 (int)std::max(lookup_smem(v & 1, (v >> 1) & 1, kMaxCtaTiles, 1),
                                                (size_t)120 * 1024));
         if (e != cudaSuccess) return e;
     }
@@ -337,8 +340,8 @@ eva_status_t eva_vq_linear_run(eva_vq_linear_t h, const void *x, int32_t B, void
 eva_status_t eva_vq_linear_run_ex(eva_vq_linear_t h, const void *x, int32_t B, void *y, eva_stream_t stream,
                                   uint32_t flags) {
     if (!h || !x || !y || !aligned16(x) || !aligned16(y)) return EVA_ERR_INVALID_ARG;
-    if (flags & ~(uint32_t)EVA_RUN_INPUT_READY) return EVA_ERR_INVALID_ARG;
-    const int input_ready = (flags & EVA_RUN_INPUT_READY) ? 1 : 0;
+    if (flags & ~(uint32_t)EVA_RUN_INDEPENDENT) return EVA_ERR_INVALID_ARG;
+    const int independent = (flags & EVA_RUN_INDEPENDENT) ? 1 : 0;
     if (B < 1 || B > h->desc.max_batch) return EVA_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const eva_vq_desc &d = h->desc;
@@ -363,16 +366,17 @@ eva_status_t eva_vq_linear_run_ex(eva_vq_linear_t h, const void *x, int32_t B, v
     const eva_vq_linear::Plan &pl = h->plan[pair_t ? 1 : 0];
     p.Gs = pl.Gs;
     p.Gt = pl.Gt;
+    p.acc_tiles = (h->T + pl.Gt - 1) / pl.Gt;
     p.tiles_per_cb = h->tiles_per_cb;
     p.out_f32 = d.out_dtype == EVA_F32 ? 1 : 0;
-    p.input_ready = d.hadamard_block ? 0 : input_ready;   // x~ comes from the rotation kernel
+    p.independent = d.hadamard_block ? 0 : independent;   // x~ comes from the rotation kernel
 
     if (d.hadamard_block) {
         const int b = d.hadamard_block;
         const int thr = std::min(b / 2, 1024);
         e = launch_pdl(eva_hadamard_kernel, dim3(d.K / b, B), dim3(thr), (size_t)b * sizeof(float), s, 0,
                        reinterpret_cast<const __half *>(x), (const int8_t *)h->hsign, h->xt, d.K, b,
-                       (float)(1.0 / std::sqrt((double)b)), input_ready);
+                       (float)(1.0 / std::sqrt((double)b)), independent);
         if (e != cudaSuccess) return cuda_status(e);
         ++kernels;
         p.x = h->xt;

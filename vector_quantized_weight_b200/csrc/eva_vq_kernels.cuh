@@ -43,8 +43,9 @@ struct LookupParams {
     int Gs, Gt;              // CTA grid: blockIdx.x = tt * Gs + ts; clusters of Gs CTAs
     int tiles_per_cb;        // 0: shared codebook; else row tiles per codebook
     int x_f32, out_f32;
-    int input_ready;         // x was not written by the preceding kernel: read it
-                             // before the dependency wait (outputs still wait)
+    int independent;         // neither x nor y is touched by the preceding kernel:
+                             // run without waiting for it (wait only before exit)
+    int acc_tiles;           // row tiles of the largest CTA (shared-memory layout)
 #ifdef EVA_DEVICE_CHECKS
     // Debug build only: bounds of every buffer the kernel touches.  A
     // violating access is skipped and the first one is recorded.
@@ -158,14 +159,12 @@ __device__ __forceinline__ void cluster_sync_all() {
                  "barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// fp32 load from the shared memory of cluster CTA `rank` at the address this
-// CTA uses for the same variable (distributed shared memory).
-__device__ __forceinline__ float ld_dsmem_f32(uint32_t local_addr, uint32_t rank) {
+// fp32 store into the shared memory of cluster CTA `rank`, at the address
+// this CTA uses for the same variable (distributed shared memory).
+__device__ __forceinline__ void st_dsmem_f32(uint32_t local_addr, uint32_t rank, float v) {
     uint32_t ra;
-    float v;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(local_addr), "r"(rank));
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra) : "memory");
-    return v;
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(ra), "f"(v) : "memory");
 }
 
 __device__ __forceinline__ uint32_t to_tf32(float f) {
@@ -454,6 +453,9 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
     // ---- prologue: weights only ----
     EVA_STAMP(0);
     pdl_launch();
+    // A CTA may write a peer's shared memory only once the peer runs: arrive
+    // now, wait (long satisfied) before the first remote store.
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
     if (tid < s1 - s0) {
         const size_t u = (size_t)(s0 + tid) * p.T + t0;
         const uint32_t nt = (uint32_t)(t1 - t0);
@@ -490,15 +492,23 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
 
     // x (unless the caller vouches it is ready) and y belong to the stream
     // order from here on.
-    if (!p.input_ready) pdl_wait();
+    if (!p.independent) pdl_wait();
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
     EVA_STAMP(1);
 
     const int npairs = PAIR_T ? (p.B + 1) / 2 : 1;
     constexpr int NTOK = PAIR_T ? 2 : 1;
     const int ctiles = t1 - t0;
-    float *acc_s = reinterpret_cast<float *>(eva_smem + ACC_OFF);   // [ctiles][16 rows][2 tokens]
+    // Running sums over this CTA's slices, [ctiles][16 rows][2 tokens], and the
+    // reduction stage of the tiles this CTA owns (tile tl belongs to cluster
+    // rank tl % Gs): [ceil(acc_tiles / Gs) slots][Gs sources][16 rows][2 tokens].
+    float *acc_s = reinterpret_cast<float *>(eva_smem + ACC_OFF);
+    const uint32_t STAGE_OFF = ACC_OFF + (uint32_t)p.acc_tiles * kTileRows * 2u * 4u;
+    const float *stage = reinterpret_cast<const float *>(eva_smem + STAGE_OFF);
+    const uint32_t stage_addr = (uint32_t)__cvta_generic_to_shared(eva_smem + STAGE_OFF);
     for (int pr = 0; pr < npairs; ++pr) {
-        for (int e = tid; e < ctiles * kTileRows * 2; e += kThreads) acc_s[e] = 0.f;
+        if (s1 - s0 > 1)
+            for (int e = tid; e < ctiles * kTileRows * 2; e += kThreads) acc_s[e] = 0.f;
 
         for (int s = s0; s < s1; ++s) {
             stage_x<PAIR_T>(p, s, pr, warp, lane, X_OFF);
@@ -609,46 +619,52 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
                         }
                     }
                     // Lanes q = 0 hold column 0 (and 1): rows g and g + 8 of the tile.
+                    // On the CTA's last slice the tile's sums go straight to the
+                    // shared memory of the cluster CTA that owns the tile.
                     if (q == 0) {
+                        const bool last = (s == s1 - 1);
+                        const uint32_t owner = (uint32_t)(tl % p.Gs);
+                        const int slot = tl / p.Gs;
 #pragma unroll
                         for (int h = 0; h < 2; ++h)
 #pragma unroll
                             for (int e = 0; e < NTOK; ++e) {
-                                const int ai = ((tl * kTileRows) + g + 8 * h) * 2 + e;
-                                if (!EVA_BAD_S(ACC_OFF + 4u * (uint32_t)ai)) acc_s[ai] += da[2 * h + e];
+                                const int row = g + 8 * h;
+                                const int ai = (tl * kTileRows + row) * 2 + e;
+                                float v = da[2 * h + e];
+                                if (s1 - s0 > 1 && !EVA_BAD_S(ACC_OFF + 4u * (uint32_t)ai)) {
+                                    if (!last) {
+                                        acc_s[ai] += v;
+                                        continue;
+                                    }
+                                    v += acc_s[ai];
+                                }
+                                const uint32_t si = (uint32_t)(((slot * p.Gs + ts) * kTileRows + row) * 2 + e);
+                                if (!EVA_BAD_S(STAGE_OFF + 4u * si)) st_dsmem_f32(stage_addr + 4u * si, owner, v);
                             }
                     }
                 }
             }
         }
 
-        // Epilogue of this token (pair): the Gs CTAs of this row group form a
-        // thread-block cluster; after a cluster barrier each one sums a share
-        // of the rows over all Gs running-sum arrays (distributed shared
-        // memory, fixed order: bitwise reproducible) and stores y.
-        if (pr == 0 && p.input_ready) pdl_wait();   // outputs follow the stream order
+        // Epilogue of this token (pair): once every CTA of the cluster has
+        // pushed its sums, each owner adds the Gs contributions of its tiles in
+        // a fixed order (bitwise reproducible) and stores y.
         EVA_STAMP(4);
         cluster_sync_all();
         EVA_STAMP(5);
         {
-            const int crow = ctiles * kTileRows;
-            const int rlo = crow * ts / p.Gs, rhi = crow * (ts + 1) / p.Gs, nrow = rhi - rlo;
-            const uint32_t acc_addr = (uint32_t)__cvta_generic_to_shared(acc_s);
-            for (int idx = tid; idx < nrow * NTOK; idx += kThreads) {
-                const int e = idx / nrow, r = rlo + idx % nrow;
+            const int my_tiles = (ctiles - ts + p.Gs - 1) / p.Gs;   // tiles tl = ts + Gs * slot
+            for (int idx = tid; idx < my_tiles * kTileRows * NTOK; idx += kThreads) {
+                const int e = idx % NTOK, row = (idx / NTOK) % kTileRows, slot = idx / (NTOK * kTileRows);
+                const int tl = ts + p.Gs * slot;
                 const int tok = PAIR_T ? 2 * pr + e : 0;
-                const int o = kTileRows * t0 + r;
+                const int o = kTileRows * (t0 + tl) + row;
                 if (tok >= p.B || o >= p.N) continue;
-                const uint32_t la = acc_addr + 4u * (uint32_t)(r * 2 + e);
                 float sum = 0.f;
-                for (int k0 = 0; k0 < p.Gs; k0 += 8) {
-                    float v[8];
-#pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        v[k] = (k0 + k < p.Gs && !EVA_BAD_S(ACC_OFF + 4u * (uint32_t)(r * 2 + e)))
-                                   ? ld_dsmem_f32(la, (uint32_t)(k0 + k)) : 0.f;
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) sum += v[k];
+                for (int k = 0; k < p.Gs; ++k) {
+                    const uint32_t si = (uint32_t)(((slot * p.Gs + k) * kTileRows + row) * 2 + e);
+                    sum += EVA_BAD_S(STAGE_OFF + 4u * si) ? 0.f : stage[si];
                 }
                 const size_t yi = (size_t)tok * p.N + o;
                 if (p.out_f32) {
@@ -660,8 +676,13 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
                 }
             }
         }
-        cluster_sync_all();   // peers are done reading this CTA's sums
+        // Before the next pair's sums are pushed, every owner must be done
+        // reading this pair's stage (and this CTA's warps done with acc_s).
+        if (pr + 1 < npairs) cluster_sync_all();
     }
+    // Independent calls still complete after the preceding kernel, so that
+    // later calls that wait on this one see the stream order.
+    if (p.independent) pdl_wait();
     EVA_STAMP(6);
 #ifdef EVA_TIMELINE
     if (tid == 0) {
@@ -680,11 +701,11 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
 __global__ void __launch_bounds__(1024) eva_hadamard_kernel(const __half *__restrict__ x,
                                                             const int8_t *__restrict__ hs,
                                                             float *__restrict__ xt, int K, int b,
-                                                            float scale, int input_ready) {
+                                                            float scale, int independent) {
     float *sb = reinterpret_cast<float *>(eva_smem);
     const int blk = blockIdx.x, tok = blockIdx.y;
     pdl_launch();
-    if (!input_ready) pdl_wait();  // x may be the output of the preceding kernel
+    if (!independent) pdl_wait();  // x may be the output of the preceding kernel
     const unsigned short *xb =
         reinterpret_cast<const unsigned short *>(x) + (size_t)tok * K + (size_t)blk * b;
     for (int i = threadIdx.x; i < b; i += blockDim.x) sb[i] = __half2float(__ushort_as_half(__ldcg(xb + i)));
@@ -698,7 +719,7 @@ __global__ void __launch_bounds__(1024) eva_hadamard_kernel(const __half *__rest
         }
     }
     __syncthreads();
-    if (input_ready) pdl_wait();  // the rotated input is this handle's workspace
+    if (independent) pdl_wait();  // the rotated input is this handle's workspace
     for (int i = threadIdx.x; i < b; i += blockDim.x) {
         const int k = blk * b + i;
         xt[(size_t)tok * K + k] = (float)hs[k] * sb[i] * scale;

@@ -18,7 +18,7 @@ EVA_F16, EVA_F32 = 0, 1
 EVA_PATH_AUTO, EVA_PATH_OC_LOOKUP, EVA_PATH_DEQUANT_MMA = 0, 1, 2
 
 # Every function the header declares; the CPU tests check the library exports them.
-EVA_RUN_INPUT_READY = 1
+EVA_RUN_INDEPENDENT = 1
 
 ABI_FUNCTIONS = (
     "eva_vq_linear_create", "eva_vq_linear_run", "eva_vq_linear_run_ex", "eva_vq_linear_run_host",
@@ -198,7 +198,7 @@ class VQLinear:
         self.handle = eva_vq_linear_create(self.desc, _ptr(wc), _ptr(wi), _ptr(signs), _ptr(alpha),
                                            _ptr(hsign), _stream_handle(stream))
 
-    def __call__(self, x, out=None, stream=None, input_ready=False):
+    def __call__(self, x, out=None, stream=None, independent=False):
         import torch
         if x.dtype != torch.float16 or not x.is_cuda or not x.is_contiguous():
             raise ValueError("x must be a contiguous CUDA float16 tensor [B, K]")
@@ -206,7 +206,7 @@ class VQLinear:
         B = x2.shape[0]
         y = out if out is not None else torch.empty((B, self.N), dtype=self.out_dtype, device=x.device)
         eva_vq_linear_run_ex(self.handle, _ptr(x2), B, _ptr(y), _stream_handle(stream),
-                             EVA_RUN_INPUT_READY if input_ready else 0)
+                             EVA_RUN_INDEPENDENT if independent else 0)
         return y
 
     def run_host(self, x_host, y_host, stream=None):

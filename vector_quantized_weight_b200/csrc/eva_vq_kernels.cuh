@@ -27,7 +27,7 @@ namespace eva {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxCtaTiles = 128;  // row tiles per CTA (shared-memory accumulator size)
-constexpr int kLookahead = 4;      // units of index bytes in flight per warp
+constexpr int kLookahead = 3;      // units of index bytes in flight per warp
 constexpr uint32_t kAccBytes = kMaxCtaTiles * kTileRows * 2 * 4;
 
 extern __shared__ __align__(1024) uint8_t eva_smem[];
@@ -159,12 +159,14 @@ __device__ __forceinline__ void cluster_sync_all() {
                  "barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// fp32 store into the shared memory of cluster CTA `rank`, at the address
+// 16-byte store into the shared memory of cluster CTA `rank`, at the address
 // this CTA uses for the same variable (distributed shared memory).
-__device__ __forceinline__ void st_dsmem_f32(uint32_t local_addr, uint32_t rank, float v) {
+__device__ __forceinline__ void st_dsmem_v4(uint32_t local_addr, uint32_t rank, float4 v) {
     uint32_t ra;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(local_addr), "r"(rank));
-    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(ra), "f"(v) : "memory");
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(ra), "f"(v.x), "f"(v.y),
+                 "f"(v.z), "f"(v.w)
+                 : "memory");
 }
 
 __device__ __forceinline__ uint32_t to_tf32(float f) {
@@ -434,6 +436,9 @@ __device__ __forceinline__ void build_sign_table(const LookupParams &p, int warp
 
 template <bool PAIR_T, bool RESID, bool GROUPED>
 __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_lookup_kernel(const LookupParams p) {
+    // Index units in flight per warp: with per-group codebooks a warp has at
+    // most one tile per codebook pass, so a short ring suffices.
+    constexpr int LA = GROUPED ? 2 : kLookahead;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, q = lane & 3;
     const int ts = blockIdx.x % p.Gs, tt = blockIdx.x / p.Gs;
@@ -499,16 +504,15 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
     const int npairs = PAIR_T ? (p.B + 1) / 2 : 1;
     constexpr int NTOK = PAIR_T ? 2 : 1;
     const int ctiles = t1 - t0;
-    // Running sums over this CTA's slices, [ctiles][16 rows][2 tokens], and the
-    // reduction stage of the tiles this CTA owns (tile tl belongs to cluster
-    // rank tl % Gs): [ceil(acc_tiles / Gs) slots][Gs sources][16 rows][2 tokens].
+    // Running sums over this CTA's slices, [ctiles][16 rows][2 tokens] (128
+    // bytes per tile), and the reduction stage of the tiles this CTA owns
+    // (tile tl belongs to cluster rank tl % Gs):
+    // [ceil(acc_tiles / Gs) slots][Gs sources][16 rows][2 tokens].
     float *acc_s = reinterpret_cast<float *>(eva_smem + ACC_OFF);
     const uint32_t STAGE_OFF = ACC_OFF + (uint32_t)p.acc_tiles * kTileRows * 2u * 4u;
     const float *stage = reinterpret_cast<const float *>(eva_smem + STAGE_OFF);
     const uint32_t stage_addr = (uint32_t)__cvta_generic_to_shared(eva_smem + STAGE_OFF);
     for (int pr = 0; pr < npairs; ++pr) {
-        if (s1 - s0 > 1)
-            for (int e = tid; e < ctiles * kTileRows * 2; e += kThreads) acc_s[e] = 0.f;
 
         for (int s = s0; s < s1; ++s) {
             stage_x<PAIR_T>(p, s, pr, warp, lane, X_OFF);
@@ -524,12 +528,12 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
                         cur_cb = cb;
                     }
                 }
-                // Lookahead ring of kLookahead units: the first ones load (from
+                // Lookahead ring of LA units: the first ones load (from
                 // L2, where the prologue's bulk prefetch put them) while the
                 // image builds; each processed tile refills the ring's tail.
-                uint4 nb[kLookahead][2];
+                uint4 nb[LA][2];
 #pragma unroll
-                for (int d = 0; d < kLookahead; ++d) {
+                for (int d = 0; d < LA; ++d) {
                     nb[d][0] = nb[d][1] = make_uint4(0u, 0u, 0u, 0u);
                     if (i0 + d < i1) {
                         const uint8_t *up = p.wi + ((size_t)s * p.T + t0 + warp + kWarps * (i0 + d)) * kUnitBytes + 16 * lane;
@@ -548,14 +552,14 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
                     const size_t unit = (size_t)s * p.T + t0 + tl;
                     const uint4 v0 = nb[0][0], v1 = nb[0][1];
 #pragma unroll
-                    for (int d = 0; d + 1 < kLookahead; ++d) {
+                    for (int d = 0; d + 1 < LA; ++d) {
                         nb[d][0] = nb[d + 1][0];
                         nb[d][1] = nb[d + 1][1];
                     }
-                    if (i + kLookahead < i1) {
-                        const uint8_t *up = p.wi + (unit + (size_t)kWarps * kLookahead) * kUnitBytes + 16 * lane;
+                    if (i + LA < i1) {
+                        const uint8_t *up = p.wi + (unit + (size_t)kWarps * LA) * kUnitBytes + 16 * lane;
                         if (!EVA_BAD_G(BUF_WI, up, 16) && !EVA_BAD_G(BUF_WI, up + 512, 16))
-                            ldg_unit(up, nb[kLookahead - 1][0], nb[kLookahead - 1][1]);
+                            ldg_unit(up, nb[LA - 1][0], nb[LA - 1][1]);
                     }
                     const uint32_t wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
                     // Even and odd k-steps accumulate in two chains.
@@ -619,38 +623,37 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
                         }
                     }
                     // Lanes q = 0 hold column 0 (and 1): rows g and g + 8 of the tile.
-                    // On the CTA's last slice the tile's sums go straight to the
-                    // shared memory of the cluster CTA that owns the tile.
+                    // A tile is visited once per slice: the first visit stores.
                     if (q == 0) {
-                        const bool last = (s == s1 - 1);
-                        const uint32_t owner = (uint32_t)(tl % p.Gs);
-                        const int slot = tl / p.Gs;
 #pragma unroll
                         for (int h = 0; h < 2; ++h)
 #pragma unroll
                             for (int e = 0; e < NTOK; ++e) {
-                                const int row = g + 8 * h;
-                                const int ai = (tl * kTileRows + row) * 2 + e;
-                                float v = da[2 * h + e];
-                                if (s1 - s0 > 1 && !EVA_BAD_S(ACC_OFF + 4u * (uint32_t)ai)) {
-                                    if (!last) {
-                                        acc_s[ai] += v;
-                                        continue;
-                                    }
-                                    v += acc_s[ai];
-                                }
-                                const uint32_t si = (uint32_t)(((slot * p.Gs + ts) * kTileRows + row) * 2 + e);
-                                if (!EVA_BAD_S(STAGE_OFF + 4u * si)) st_dsmem_f32(stage_addr + 4u * si, owner, v);
+                                const int ai = (tl * kTileRows + g + 8 * h) * 2 + e;
+                                if (!EVA_BAD_S(ACC_OFF + 4u * (uint32_t)ai))
+                                    acc_s[ai] = (s == s0) ? da[2 * h + e] : acc_s[ai] + da[2 * h + e];
                             }
                     }
                 }
             }
         }
 
-        // Epilogue of this token (pair): once every CTA of the cluster has
-        // pushed its sums, each owner adds the Gs contributions of its tiles in
-        // a fixed order (bitwise reproducible) and stores y.
+        // Epilogue of this token (pair): every CTA pushes the 128-byte sum
+        // block of each of its tiles into the shared memory of the cluster CTA
+        // that owns the tile (rank tl % Gs) with 16-byte remote stores; after
+        // the cluster barrier each owner adds the Gs contributions of its
+        // tiles in a fixed order (bitwise reproducible) and stores y.
         EVA_STAMP(4);
+        __syncthreads();
+        for (int i = tid; i < ctiles * 8; i += kThreads) {
+            const int tl = i >> 3, chunk = i & 7;
+            const uint32_t src = ACC_OFF + (uint32_t)(tl * 32 + chunk * 4) * 4u;
+            const uint32_t dst = (uint32_t)((((tl / p.Gs) * p.Gs + ts) * 32 + chunk * 4) * 4);
+            if (!EVA_BAD_S(src) && !EVA_BAD_S(src + 12u) && !EVA_BAD_S(STAGE_OFF + dst) && !EVA_BAD_S(STAGE_OFF + dst + 12u)) {
+                const float4 v = *reinterpret_cast<const float4 *>(eva_smem + src);
+                st_dsmem_v4(stage_addr + dst, (uint32_t)(tl % p.Gs), v);
+            }
+        }
         cluster_sync_all();
         EVA_STAMP(5);
         {

@@ -49,7 +49,8 @@ typedef enum {
     EVA_ERR_OOM = 4,             /* device allocation failed in create           */
     EVA_ERR_DEVICE_TIMEOUT = 5,  /* a bounded device wait gave up                */
     EVA_ERR_NO_DEVICE = 6,       /* no sm_100 device is current                  */
-    EVA_ERR_DEVICE_CHECK = 7     /* checked build: a kernel access was out of bounds */
+    EVA_ERR_DEVICE_CHECK = 7,    /* checked build: a kernel access was out of bounds */
+    EVA_ERR_SCRATCH_TOO_SMALL = 8 /* eva_vq_linear_run_noalloc: B * K * 4 > 4 MiB      */
 } eva_status_t;
 
 typedef enum { EVA_F16 = 0, EVA_F32 = 1 } eva_dtype_t;
@@ -124,6 +125,41 @@ enum {
 /* eva_vq_linear_run with flags (0 gives eva_vq_linear_run). */
 EVA_API eva_status_t eva_vq_linear_run_ex(eva_vq_linear_t h, const void *x, int32_t B, void *y,
                                           eva_stream_t stream, uint32_t flags);
+
+/*
+ * eva_vq_linear_run for callers that must not touch the device allocator.
+ * No counterpart in the EVA pages or the 3-bit SRAM-lookup article: it is a
+ * deployment convenience of this library.
+ *
+ * Who needs it: code that runs where cudaMalloc is off limits -- inside a
+ * stream capture that records a whole decode step into a CUDA graph (an
+ * allocation there either fails or breaks the capture), in real-time loops
+ * where cudaMalloc's implicit device synchronisation is not acceptable, or
+ * under an external memory manager that owns every byte of device memory.
+ * This call allocates nothing and frees nothing, and neither do its kernels.
+ *
+ * The only scratch memory the layer needs -- the rotated input x~ of a layer
+ * with hadamard_block != 0 -- comes from one library-wide device array of
+ * 4 MiB, `static __device__` in this library, so B * K * 4 must not exceed
+ * 4 MiB (EVA_ERR_SCRATCH_TOO_SMALL otherwise).  Every GPU that loads the
+ * library keeps those 4 MiB until the process exits.  Layers without a
+ * rotation use no scratch at all.
+ *
+ * Set-up: the first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture.  The device that is current must be the
+ * handle's.
+ *
+ * Sharing: every call on a device uses the same array and it keeps the last
+ * call's contents (nothing in it needs to start at zero: the rotation writes
+ * all of x~ before the lookups read it).  Two calls whose kernels overlap on
+ * the GPU -- on different streams, or with different handles at the same
+ * time -- race on the array; serialise them (one stream is enough).
+ *
+ * Arguments, layouts and results are those of eva_vq_linear_run.
+ */
+EVA_API eva_status_t eva_vq_linear_run_noalloc(eva_vq_linear_t h, const void *x, int32_t B, void *y,
+                                               eva_stream_t stream);
 
 /*
  * The same call with HOST buffers: copies x (host fp16 [B][K]) to the

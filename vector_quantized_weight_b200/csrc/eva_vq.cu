@@ -13,6 +13,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 #include <new>
 
 #include "../../include/eva_vq.h"
@@ -235,6 +236,8 @@ const char *eva_vq_status_string(eva_status_t s) {
         case EVA_ERR_DEVICE_TIMEOUT: return "device wait timed out";
         case EVA_ERR_NO_DEVICE: return "no sm_100 device";
         case EVA_ERR_DEVICE_CHECK: return "device-side bounds check failed (checked build)";
+        case EVA_ERR_SCRATCH_TOO_SMALL:
+            return "B * K * 4 bytes exceed the 4 MiB static scratch of eva_vq_linear_run_noalloc";
     }
     return "unknown status";
 }
@@ -417,6 +420,100 @@ eva_status_t eva_vq_linear_run_ex(eva_vq_linear_t h, const void *x, int32_t B, v
     h->last_kernels = kernels;
     h->last_path = EVA_PATH_OC_LOOKUP;
     return EVA_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free run.  The rotated input of a 3.125-bit layer normally lives
+// in a buffer the handle allocated with cudaMalloc.  This variant takes that
+// scratch from one file-scope device array instead, so the call never goes
+// near the device allocator.
+namespace {
+constexpr size_t kStaticScratchBytes = (size_t)4 << 20;   // 4 MiB: B * K * 4 bytes at most
+}
+static __device__ __align__(256) float eva_static_scratch[kStaticScratchBytes / sizeof(float)];
+
+namespace {
+std::mutex g_scratch_mu;
+float *g_scratch_dev[128] = {};   // device address of eva_static_scratch, per device ordinal
+
+// The host-side symbol is a stand-in, not a device address: look the real
+// address up once per device, with that device current.
+eva_status_t static_scratch(int dev, float **out) {
+    if (dev < 0 || dev >= 128) return EVA_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_dev[dev]) {
+        void *ptr = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&ptr, eva_static_scratch);
+        if (e != cudaSuccess || !ptr) return EVA_ERR_CUDA;
+        g_scratch_dev[dev] = static_cast<float *>(ptr);
+    }
+    *out = g_scratch_dev[dev];
+    return EVA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+eva_status_t eva_vq_linear_run_noalloc(eva_vq_linear_t h, const void *x, int32_t B, void *y,
+                                       eva_stream_t stream) {
+    if (!h || !x || !y || !aligned16(x) || !aligned16(y)) return EVA_ERR_INVALID_ARG;
+    if (B < 1 || B > h->desc.max_batch) return EVA_ERR_INVALID_ARG;
+    const eva_vq_desc &d = h->desc;
+    if ((size_t)B * d.K * sizeof(float) > kStaticScratchBytes) return EVA_ERR_SCRATCH_TOO_SMALL;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev != h->device) return EVA_ERR_INVALID_ARG;
+    float *scratch = nullptr;
+    if (d.hadamard_block) {
+        const eva_status_t st = static_scratch(dev, &scratch);
+        if (st != EVA_OK) return st;
+    }
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const bool pair_t = B > 1;
+    const eva_vq_linear::Plan &pl = h->plan[pair_t ? 1 : 0];
+    LookupParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.wi = h->wi;
+    p.sg = h->sg;
+    p.al = h->al;
+    p.wc = h->wc;
+    p.x = x;
+    p.x_f32 = 0;
+    p.y = y;
+    p.N = d.N;
+    p.Npad = h->Npad;
+    p.K = d.K;
+    p.S = h->S;
+    p.T = h->T;
+    p.B = B;
+    p.tiles_per_cb = h->tiles_per_cb;
+    p.out_f32 = d.out_dtype == EVA_F32 ? 1 : 0;
+    p.independent = 0;
+    p.Gs = pl.Gs;
+    p.Gt = pl.Gt;
+    p.acc_tiles = (h->T + pl.Gt - 1) / pl.Gt;
+#ifdef EVA_TIMELINE
+    p.timeline = h->timeline;
+#endif
+#ifdef EVA_DEVICE_CHECKS
+    return EVA_ERR_UNSUPPORTED;   // the checked build validates the handle path only
+#endif
+    cudaError_t e;
+    if (d.hadamard_block) {
+        const int b = d.hadamard_block;
+        const int thr = std::min(b / 2, 1024);
+        e = launch_pdl(eva_hadamard_kernel, dim3(d.K / b, B), dim3(thr), (size_t)b * sizeof(float), s, 0,
+                       reinterpret_cast<const __half *>(x), (const int8_t *)h->hsign, scratch, d.K, b,
+                       (float)(1.0 / std::sqrt((double)b)), 0);
+        if (e != cudaSuccess) return cuda_status(e);
+        p.x = scratch;
+        p.x_f32 = 1;
+    }
+    const bool resid = d.residual_group != 0;
+    e = launch_pdl(lookup_fn(pair_t, resid, h->tiles_per_cb != 0), dim3(pl.Gs * pl.Gt), dim3(kThreads),
+                   pl.smem, s, pl.Gs, p);
+    return cuda_status(e);
 }
 
 eva_status_t eva_vq_linear_run_host(eva_vq_linear_t h, const void *x_host, int32_t B, void *y_host,

@@ -13,7 +13,7 @@ import os
 from . import build as _build
 
 EVA_OK, EVA_ERR_INVALID_ARG, EVA_ERR_UNSUPPORTED, EVA_ERR_CUDA, EVA_ERR_OOM, \
-    EVA_ERR_DEVICE_TIMEOUT, EVA_ERR_NO_DEVICE, EVA_ERR_DEVICE_CHECK = range(8)
+    EVA_ERR_DEVICE_TIMEOUT, EVA_ERR_NO_DEVICE, EVA_ERR_DEVICE_CHECK, EVA_ERR_SCRATCH_TOO_SMALL = range(9)
 EVA_F16, EVA_F32 = 0, 1
 EVA_PATH_AUTO, EVA_PATH_OC_LOOKUP, EVA_PATH_DEQUANT_MMA = 0, 1, 2
 
@@ -24,7 +24,7 @@ ABI_FUNCTIONS = (
     "eva_vq_linear_create", "eva_vq_linear_run", "eva_vq_linear_run_ex", "eva_vq_linear_run_host",
     "eva_vq_linear_destroy", "eva_vq_unpack_indices", "eva_vq_sync_status",
     "eva_vq_status_string", "eva_vq_linear_info", "eva_vq_device_check_record",
-    "eva_vq_debug_timeline",
+    "eva_vq_debug_timeline", "eva_vq_linear_run_noalloc",
 )
 
 
@@ -83,6 +83,7 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.eva_vq_linear_create.argtypes = [ctypes.POINTER(H), ctypes.POINTER(eva_vq_desc), P, P, P, P, P, P]
     lib.eva_vq_linear_run.argtypes = [H, P, I32, P, P]
     lib.eva_vq_linear_run_ex.argtypes = [H, P, I32, P, P, ctypes.c_uint32]
+    lib.eva_vq_linear_run_noalloc.argtypes = [H, P, I32, P, P]
     lib.eva_vq_linear_run_host.argtypes = [H, P, I32, P, P]
     lib.eva_vq_linear_destroy.argtypes = [H]
     lib.eva_vq_unpack_indices.argtypes = [H, P, P]
@@ -125,6 +126,13 @@ def eva_vq_linear_run(h: int, x: int, B: int, y: int, stream: int | None) -> Non
 
 def eva_vq_linear_run_ex(h: int, x: int, B: int, y: int, stream: int | None, flags: int) -> None:
     _check("eva_vq_linear_run_ex", load().eva_vq_linear_run_ex(h, x, int(B), y, stream, int(flags)))
+
+
+def eva_vq_linear_run_noalloc(h: int, x: int, B: int, y: int, stream: int | None) -> None:
+    """eva_vq_linear_run without any device allocation: a rotated layer's
+    scratch comes from the library's 4 MiB static device array (see the
+    header for who needs this and the sharing rules)."""
+    _check("eva_vq_linear_run_noalloc", load().eva_vq_linear_run_noalloc(h, x, int(B), y, stream))
 
 
 def eva_vq_linear_run_host(h: int, x_host: int, B: int, y_host: int, stream: int | None) -> None:

@@ -49,6 +49,12 @@ def parse_args():
     ap.add_argument("--batch", type=int, default=None)
     ap.add_argument("--ring", type=int, default=0, help="ring length (0: > 2x L2)")
     ap.add_argument("--path", type=int, default=0)
+    ap.add_argument("--chain", default="independent", choices=["independent", "dependent"],
+                    help="independent: the ring's layers are declared independent "
+                         "(EVA_RUN_INDEPENDENT) and overlap; dependent: every call waits "
+                         "for the kernel before it, as when each layer feeds the next")
+    ap.add_argument("--no-dependent", action="store_true",
+                    help="skip the extra dependent-chain measurement")
     ap.add_argument("--x-pool", type=int, default=4,
                     help="distinct activation buffers cycled by the ring (activations stay in L2, "
                          "as the output of the preceding op does in a decode step)")
@@ -141,6 +147,21 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
                 "samples": len(sm)}
+
+
+def max_over_ranks(ms: float, pg, device) -> float:
+    """Elapsed time of a replicated measurement: the maximum over ranks."""
+    if pg is None:
+        return ms
+    import torch
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput_gbs(world: int, steps: int, bytes_per_step: int, ms: float) -> float:
+    """Whole-job GB/s: every rank streams `steps` layers of `bytes_per_step`."""
+    return world * steps * bytes_per_step / (ms * 1e-3) / 1e9
 
 
 def dist_setup():
@@ -244,35 +265,39 @@ def main():
     torch.cuda.synchronize(dev)
     info = layers[0].info()
 
-    def sweep(n, start=0):
+    def sweep(n, independent, start=0):
         for i in range(n):
             r = (start + i) % ring
-            layers[r](xs[r % len(xs)], out=ys[r], stream=stream)
+            layers[r](xs[r % len(xs)], out=ys[r], stream=stream, independent=independent)
 
-    # Warm-up (eager), then capture one full ring and a remainder graph.
-    with torch.cuda.stream(stream):
-        sweep(warmup)
-    torch.cuda.synchronize(dev)
-    full, rem = divmod(steps, ring)
-    g_full = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_full, stream=stream):
-        sweep(ring)
-    g_rem = None
-    if rem:
-        g_rem = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g_rem, stream=stream):
-            sweep(rem)
-    with torch.cuda.stream(stream):
-        g_full.replay()
-    torch.cuda.synchronize(dev)
-
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if pg:
-        pg.barrier()
-    torch.cuda.synchronize(dev)
     uuid = getattr(props, "uuid", None)
     gpu_id = f"GPU-{uuid}" if uuid is not None else str(local)
-    with ClockSampler(gpu_id) as clk:
+
+    def timed(independent, n_steps, sample_clocks):
+        """Warm up eagerly, capture one ring sweep (and a remainder) in CUDA
+        graphs, then time exactly n_steps calls between barriers."""
+        with torch.cuda.stream(stream):
+            sweep(warmup, independent)
+        torch.cuda.synchronize(dev)
+        full, rem = divmod(n_steps, ring)
+        g_full = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_full, stream=stream):
+            sweep(ring, independent)
+        g_rem = None
+        if rem:
+            g_rem = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_rem, stream=stream):
+                sweep(rem, independent)
+        with torch.cuda.stream(stream):
+            g_full.replay()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if pg:
+            pg.barrier()
+        torch.cuda.synchronize(dev)
+        clk = ClockSampler(gpu_id) if sample_clocks else None
+        if clk:
+            clk.__enter__()
         with torch.cuda.stream(stream):
             e0.record(stream)
             for _ in range(full):
@@ -281,15 +306,21 @@ def main():
                 g_rem.replay()
             e1.record(stream)
         torch.cuda.synchronize(dev)
-    if pg:
-        pg.barrier()
-    torch.cuda.synchronize(dev)
-    ms = e0.elapsed_time(e1)
-    if pg:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms = float(t.item())
-    del g_full, g_rem
+        if clk:
+            clk.__exit__(None, None, None)
+        if pg:
+            pg.barrier()
+        torch.cuda.synchronize(dev)
+        ms = max_over_ranks(e0.elapsed_time(e1), pg, dev)
+        del g_full, g_rem
+        return ms, clk
+
+    ms, clk = timed(args.chain == "independent", steps, True)
+    dep = None
+    if args.chain == "independent" and not args.no_dependent:
+        dep_steps = ring * max(1, min(steps, 200_000) // ring)
+        ms_dep, _ = timed(False, dep_steps, False)
+        dep = (dep_steps, ms_dep)
 
     # End to end through the public host-buffer call: x copied in from
     # pinned memory and y read back every step.
@@ -310,13 +341,9 @@ def main():
             layers[r].run_host(xh[r], yh, stream=stream)
         a1.record(stream)
         torch.cuda.synchronize(dev)
-        ms_e2e = a0.elapsed_time(a1)
-        if pg:
-            t = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            ms_e2e = float(t.item())
+        ms_e2e = max_over_ranks(a0.elapsed_time(a1), pg, dev)
         sb = stream_bytes(shape, B)
-        e2e = {"value": round(world * n_e2e * sb / (ms_e2e * 1e-3) / 1e9, 4), "unit": "GB/s",
+        e2e = {"value": round(job_throughput_gbs(world, n_e2e, sb, ms_e2e), 4), "unit": "GB/s",
                "us_per_layer": round(ms_e2e * 1e3 / n_e2e, 3),
                "h2d_bytes_per_step": 2 * B * shape.K, "d2h_bytes_per_step": 2 * B * shape.N,
                "steps": n_e2e}
@@ -330,7 +357,7 @@ def main():
 
     sb = stream_bytes(shape, B)
     us_layer = ms * 1e3 / steps
-    gbs = world * steps * sb / (ms * 1e-3) / 1e9
+    gbs = job_throughput_gbs(world, steps, sb, ms)
     peak, peak_kind = load_peaks()
     workload = f"{args.config}:{shape.name}:B{B}"
     # Dominant kernel: the fused lookup kernel, one launch per step; its
@@ -352,6 +379,9 @@ def main():
                    "l2_bytes": l2, "l2_policy": "inputs larger than L2: ring of distinct layers > 2x L2",
                    "x_pool": len(xs),
                    "graph": "one CUDA graph per ring sweep", "parallelism": f"replicas x{world}",
+                   "call": ("eva_vq_linear_run_ex(EVA_RUN_INDEPENDENT): the ring's layers read "
+                            "activations produced before the timed region and write distinct outputs"
+                            if args.chain == "independent" else "eva_vq_linear_run (stream-ordered)"),
                    "grid": info.grid, "kernels_per_step": info.kernels_per_run},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 3), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": load_traffic(workload),
@@ -360,6 +390,14 @@ def main():
         "gpu_launches": steps * info.kernels_per_run,
         "clocks": clk.summary(),
     }
+    if dep:
+        dep_steps, ms_dep = dep
+        us_dep = ms_dep * 1e3 / dep_steps
+        line["dependent_chain"] = {
+            "us_per_layer": round(us_dep, 4), "steps": dep_steps,
+            "value": round(job_throughput_gbs(world, dep_steps, sb, ms_dep), 4), "unit": "GB/s",
+            "note": "every call waits for the kernel before it (plain eva_vq_linear_run), as when each "
+                    "layer's output feeds the next"}
     if e2e:
         line["e2e"] = e2e
     if not args.no_cpu:

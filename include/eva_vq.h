@@ -116,9 +116,7 @@ enum {
      * earlier and write distinct outputs).  The layer then runs without
      * waiting for that kernel, so consecutive independent layers overlap;
      * it still completes after it, so later calls keep the stream order.
-     * A layer with a Hadamard rotation only reads x early (its rotated-input
-     * workspace stays in stream order).  Passing it when x or y IS used by
-     * the preceding kernel is a race. */
+     * Passing it when x or y IS used by the preceding kernel is a race. */
     EVA_RUN_INDEPENDENT = 1u
 };
 
@@ -138,12 +136,15 @@ EVA_API eva_status_t eva_vq_linear_run_ex(eva_vq_linear_t h, const void *x, int3
  * under an external memory manager that owns every byte of device memory.
  * This call allocates nothing and frees nothing, and neither do its kernels.
  *
- * The only scratch memory the layer needs -- the rotated input x~ of a layer
- * with hadamard_block != 0 -- comes from one library-wide device array of
- * 4 MiB, `static __device__` in this library, so B * K * 4 must not exceed
- * 4 MiB (EVA_ERR_SCRATCH_TOO_SMALL otherwise).  Every GPU that loads the
- * library keeps those 4 MiB until the process exits.  Layers without a
- * rotation use no scratch at all.
+ * For a layer with hadamard_block != 0 this call runs the rotation as a
+ * kernel of its own (eva_vq_linear_run fuses it into the lookup kernel) and
+ * the rotated input x~ goes through scratch memory: one library-wide device
+ * array of 4 MiB, `static __device__` in this library, so B * K * 4 must not
+ * exceed 4 MiB (EVA_ERR_SCRATCH_TOO_SMALL otherwise).  Every GPU that loads
+ * the library keeps those 4 MiB until the process exits.  Layers without a
+ * rotation use no scratch at all.  Results are bitwise those of
+ * eva_vq_linear_run: both rotations take the same butterflies in the same
+ * order.
  *
  * Set-up: the first call on a device looks up the array's device address
  * (cudaGetSymbolAddress, with that device current); make that first call

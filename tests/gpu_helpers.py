@@ -58,5 +58,8 @@ def run_gpu(layer, x, *, out_dtype="float16", path=0, max_batch=None):
     y = lin(xt)
     torch.cuda.synchronize()
     out = y.float().cpu().numpy().astype(np.float64)
+    # no bounded device wait gave up (and, in the bounds-checked build, no
+    # access fell outside its buffer)
+    assert eva_vq.eva_vq_sync_status(lin.handle) == eva_vq.EVA_OK
     lin.close()
     return out

@@ -109,6 +109,6 @@ def test_lookup_kernels_do_not_spill():
     out = subprocess.run(cmd, capture_output=True, text=True, check=True).stderr
     blocks = re.findall(r"Function properties for (\S*eva_lookup_kernel\S*)\n\s*(\d+) bytes stack frame, "
                         r"(\d+) bytes spill stores, (\d+) bytes spill loads", out)
-    assert len(blocks) == 8, out
+    assert len(blocks) == 16, out
     for name, stack, st, ld in blocks:
         assert (stack, st, ld) == ("0", "0", "0"), (name, stack, st, ld)

@@ -24,16 +24,19 @@ using namespace eva;
 struct eva_vq_linear {
     eva_vq_desc desc;
     int device = 0, sm_count = 0;
+    int smem_per_sm = 0, smem_reserved = 0, smem_optin = 0;   // shared memory, bytes
+    int regs_per_sm = 0;
     int J = 0, S = 0, T = 0, Npad = 0, G = 1, tiles_per_cb = 0;
     // Lookup grid per variant (index: token pair or not): Gs slice groups
     // (one cluster) x Gt row groups, and its dynamic shared memory.
-    struct Plan { int Gs = 1, Gt = 1; size_t smem = 0; } plan[2];
+    // `staged` index units per CTA are copied into shared memory up front
+    // (`smem`); calls flagged independent skip that copy (`smem_nostage`).
+    struct Plan { int Gs = 1, Gt = 1, staged = 0; size_t smem = 0, smem_nostage = 0; } plan[2];
     uint8_t *wi = nullptr;              // repacked indices
     uint8_t *sg = nullptr;              // repacked signs
     __half *al = nullptr;               // repacked alpha
     __half *wc = nullptr;               // codebooks [G][256][4]
     int8_t *hsign = nullptr;            // Hadamard signs [K]
-    float *xt = nullptr;                // rotated input [max_batch][K]
     int *status = nullptr;              // device error word
     unsigned long long *timeline = nullptr;  // timeline build: [grid][8] stamps
     void *x_stage = nullptr, *y_stage = nullptr;
@@ -78,23 +81,53 @@ eva_status_t validate_desc(const eva_vq_desc *d) {
 
 // Dynamic shared memory of the lookup kernel: the OC image (with the residual
 // table in its unused half for one token, or a second image for a token
-// pair), the staged x~ slice, the running sums of `tiles` row tiles and the
-// cluster reduction stage.
-size_t lookup_smem(bool pair_t, bool resid, int tiles, int gs) {
+// pair), the staged x~ slice of one or two tokens, the staging copy's
+// mbarrier, the running sums of `tiles` row tiles, the cluster reduction
+// stage and, 128-byte aligned, the fused rotation's scratch (rotation blocks
+// b > 256: b floats per token) and the `staged` index units of the first slice.
+size_t lookup_smem(bool pair_t, bool resid, int tiles, int gs, int rot_b, int staged = 0) {
     const size_t tile_bytes = (size_t)kTileRows * 2 * 4;
     const size_t stage_tiles = (size_t)((tiles + gs - 1) / gs) * gs;   // reduction stage
-    return (size_t)kOcBytes + ((pair_t && resid) ? (size_t)kOcBytes : 0) + kXStageBytes +
-           (size_t)tiles * tile_bytes + stage_tiles * tile_bytes;
+    const size_t base = (size_t)kOcBytes + ((pair_t && resid) ? (size_t)kOcBytes : 0) +
+                        (pair_t ? kXStageBytes : kXStageBytes / 2) + 128 + (size_t)tiles * tile_bytes +
+                        stage_tiles * tile_bytes;
+    const size_t rot = rot_b > kSliceK ? (size_t)(pair_t ? 2 : 1) * rot_b * 4 : 0;
+    return ((base + 127) & ~(size_t)127) + rot + (size_t)staged * kUnitBytes;
+}
+
+// Index units of the first slice a CTA copies into shared memory: as many of
+// its `tiles` as fit in what is left of the per-SM budget.  The budget keeps
+// two CTAs per SM (this layer's and the next layer's early-launched one)
+// wherever the registers and the rest of the footprint allow it, else one.
+int staged_tiles(const eva_vq_linear *h, const void *fn, bool pair_t, bool resid, int tiles, int gs) {
+    const size_t base = lookup_smem(pair_t, resid, tiles, gs, h->desc.hadamard_block, 0);
+    const size_t per_sm = (size_t)h->smem_per_sm, reserved = (size_t)h->smem_reserved;
+    const size_t two = per_sm / 2 - reserved;
+    const size_t one = std::min(per_sm - reserved, (size_t)h->smem_optin);
+    cudaFuncAttributes fa;
+    bool two_fit_regs = false;
+    if (cudaFuncGetAttributes(&fa, fn) == cudaSuccess)
+        two_fit_regs = 2 * fa.numRegs * kThreads <= h->regs_per_sm;
+    else
+        cudaGetLastError();
+    const size_t budget = (two_fit_regs && base <= two) ? two : one;
+    if (base >= budget) return 0;
+    return (int)std::min<size_t>((size_t)tiles, (budget - base) / kUnitBytes);
 }
 
 using LookupFn = void (*)(LookupParams);
-LookupFn lookup_fn(bool pair_t, bool resid, bool grouped) {
+template <bool ROT>
+LookupFn lookup_fn_r(bool pair_t, bool resid, bool grouped) {
     if (grouped) {
-        if (!pair_t) return resid ? eva_lookup_kernel<false, true, true> : eva_lookup_kernel<false, false, true>;
-        return resid ? eva_lookup_kernel<true, true, true> : eva_lookup_kernel<true, false, true>;
+        if (!pair_t) return resid ? eva_lookup_kernel<false, true, true, ROT> : eva_lookup_kernel<false, false, true, ROT>;
+        return resid ? eva_lookup_kernel<true, true, true, ROT> : eva_lookup_kernel<true, false, true, ROT>;
     }
-    if (!pair_t) return resid ? eva_lookup_kernel<false, true, false> : eva_lookup_kernel<false, false, false>;
-    return resid ? eva_lookup_kernel<true, true, false> : eva_lookup_kernel<true, false, false>;
+    if (!pair_t) return resid ? eva_lookup_kernel<false, true, false, ROT> : eva_lookup_kernel<false, false, false, ROT>;
+    return resid ? eva_lookup_kernel<true, true, false, ROT> : eva_lookup_kernel<true, false, false, ROT>;
+}
+// rot: the instance that computes the Hadamard rotation while staging x.
+LookupFn lookup_fn(bool pair_t, bool resid, bool grouped, bool rot) {
+    return rot ? lookup_fn_r<true>(pair_t, resid, grouped) : lookup_fn_r<false>(pair_t, resid, grouped);
 }
 
 // Largest number of clusters of `cs` CTAs of this kernel resident at once.
@@ -128,7 +161,7 @@ int max_active_clusters(LookupFn fn, size_t smem, int cs) {
 void plan_grid(eva_vq_linear *h, int pair_t) {
     const int S = h->S, T = h->T, P = h->sm_count;
     const bool resid = h->desc.residual_group != 0;
-    const LookupFn fn = lookup_fn(pair_t != 0, resid, h->tiles_per_cb != 0);
+    const LookupFn fn = lookup_fn(pair_t != 0, resid, h->tiles_per_cb != 0, h->desc.hadamard_block != 0);
     double best = 1e300;
     eva_vq_linear::Plan pl;
     pl.Gs = 1;
@@ -137,7 +170,8 @@ void plan_grid(eva_vq_linear *h, int pair_t) {
         const int gt_min = (T + kMaxCtaTiles - 1) / kMaxCtaTiles;
         // Capacity with one CTA per SM: the occupancy query counts CTA slots,
         // so ask with a footprint that leaves room for a single CTA per SM.
-        const size_t smem_one = std::max(lookup_smem(pair_t, resid, (T + gt_min - 1) / gt_min, gs),
+        const size_t smem_one = std::max(lookup_smem(pair_t, resid, (T + gt_min - 1) / gt_min, gs,
+                                                     h->desc.hadamard_block),
                                          (size_t)120 * 1024);
         const int clusters = max_active_clusters(fn, smem_one, gs);
         // One CTA of this layer per SM: no more clusters than P / gs either.
@@ -155,7 +189,10 @@ void plan_grid(eva_vq_linear *h, int pair_t) {
             }
         }
     }
-    pl.smem = lookup_smem(pair_t, resid, (T + pl.Gt - 1) / pl.Gt, pl.Gs);
+    const int tiles = (T + pl.Gt - 1) / pl.Gt;
+    pl.staged = staged_tiles(h, (const void *)fn, pair_t != 0, resid, tiles, pl.Gs);
+    pl.smem = lookup_smem(pair_t, resid, tiles, pl.Gs, h->desc.hadamard_block, pl.staged);
+    pl.smem_nostage = lookup_smem(pair_t, resid, tiles, pl.Gs, h->desc.hadamard_block, 0);
     h->plan[pair_t] = pl;
 }
 
@@ -186,17 +223,16 @@ cudaError_t launch_pdl(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_
 }
 
 
-cudaError_t set_smem_attrs() {
+cudaError_t set_smem_attrs(int smem_optin) {
     cudaError_t e;
-    for (int v = 0; v < 8; ++v) {
-        const LookupFn fn = lookup_fn(v & 1, (v >> 1) & 1, (v >> 2) & 1);
+    for (int v = 0; v < 16; ++v) {
+        const LookupFn fn = lookup_fn(v & 1, (v >> 1) & 1, (v >> 2) & 1, (v >> 3) & 1);
         e = cudaFuncSetAttribute((const void *)fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         if (e != cudaSuccess) return e;
-        // The limit also covers the one-CTA-per-SM footprint the planner's
-        // occupancy query uses; launches request only what they need.
-        e = cudaFuncSetAttribute((const void *)fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)std::max(lookup_smem(v & 1, (v >> 1) & 1, kMaxCtaTiles, 1),
-                                               (size_t)120 * 1024));
+        // The device's per-block limit: it covers the one-CTA-per-SM footprint
+        // the planner's occupancy query uses and any index staging; launches
+        // request only what they need.
+        e = cudaFuncSetAttribute((const void *)fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_optin);
         if (e != cudaSuccess) return e;
     }
     return cudaFuncSetAttribute(eva_hadamard_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 4096 * 4);
@@ -204,7 +240,7 @@ cudaError_t set_smem_attrs() {
 
 void free_handle(eva_vq_linear *h) {
     if (!h) return;
-    void *ptrs[] = {h->wi, h->sg, h->al, h->wc, h->hsign, h->xt, h->status, h->x_stage,
+    void *ptrs[] = {h->wi, h->sg, h->al, h->wc, h->hsign, h->status, h->x_stage,
                     h->y_stage, h->timeline};
     for (void *p : ptrs)
         if (p) cudaFree(p);
@@ -272,6 +308,10 @@ eva_status_t eva_vq_linear_create(eva_vq_linear_t *out, const eva_vq_desc *desc,
     h->desc = *desc;
     h->device = dev;
     h->sm_count = prop.multiProcessorCount;
+    h->smem_per_sm = (int)prop.sharedMemPerMultiprocessor;
+    h->smem_reserved = (int)prop.reservedSharedMemPerBlock;
+    h->smem_optin = (int)prop.sharedMemPerBlockOptin;
+    h->regs_per_sm = prop.regsPerMultiprocessor;
     const int N = desc->N, K = desc->K;
     h->J = K / kD;
     h->S = (h->J + kSliceJ - 1) / kSliceJ;
@@ -284,7 +324,7 @@ eva_status_t eva_vq_linear_create(eva_vq_linear_t *out, const eva_vq_desc *desc,
     int64_t ws = 0;
     cudaError_t e = cudaSuccess;
     auto chk = [&](cudaError_t r) { if (e == cudaSuccess) e = r; };
-    chk(set_smem_attrs());
+    chk(set_smem_attrs(h->smem_optin));
     plan_grid(h, 0);
     if (desc->max_batch > 1) plan_grid(h, 1);
     const int max_grid = std::max(h->plan[0].Gs * h->plan[0].Gt, h->plan[1].Gs * h->plan[1].Gt);
@@ -296,7 +336,6 @@ eva_status_t eva_vq_linear_create(eva_vq_linear_t *out, const eva_vq_desc *desc,
     }
     if (desc->hadamard_block) {
         chk(dalloc(&h->hsign, (size_t)K, nullptr));
-        chk(dalloc(&h->xt, (size_t)desc->max_batch * K * sizeof(float), &ws));
     }
     chk(dalloc(&h->status, 8 * sizeof(int), &ws));
 #ifdef EVA_TIMELINE
@@ -352,6 +391,7 @@ eva_status_t eva_vq_linear_run_ex(eva_vq_linear_t h, const void *x, int32_t B, v
     cudaError_t e = cudaSuccess;
 
     LookupParams p;
+    std::memset(&p, 0, sizeof(p));
     p.wi = h->wi;
     p.sg = h->sg;
     p.al = h->al;
@@ -370,25 +410,24 @@ eva_status_t eva_vq_linear_run_ex(eva_vq_linear_t h, const void *x, int32_t B, v
     p.Gs = pl.Gs;
     p.Gt = pl.Gt;
     p.acc_tiles = (h->T + pl.Gt - 1) / pl.Gt;
+    // A call that waits for its predecessor copies its first indices into
+    // shared memory while it waits.  An independent call starts at once and
+    // streams them through registers, leaving the shared-memory bandwidth to
+    // the lookups of the calls it overlaps with.
+    p.wi_staged = independent ? 0 : pl.staged;
+    p.status = h->status;
     p.tiles_per_cb = h->tiles_per_cb;
     p.out_f32 = d.out_dtype == EVA_F32 ? 1 : 0;
-    p.independent = d.hadamard_block ? 0 : independent;   // x~ comes from the rotation kernel
-
-    if (d.hadamard_block) {
-        const int b = d.hadamard_block;
-        const int thr = std::min(b / 2, 1024);
-        e = launch_pdl(eva_hadamard_kernel, dim3(d.K / b, B), dim3(thr), (size_t)b * sizeof(float), s, 0,
-                       reinterpret_cast<const __half *>(x), (const int8_t *)h->hsign, h->xt, d.K, b,
-                       (float)(1.0 / std::sqrt((double)b)), independent);
-        if (e != cudaSuccess) return cuda_status(e);
-        ++kernels;
-        p.x = h->xt;
-        p.x_f32 = 1;
+    p.independent = independent;
+    if (d.hadamard_block) {   // the rotation runs inside the lookup kernel
+        p.rot_b = d.hadamard_block;
+        p.hs = h->hsign;
+        p.rot_scale = (float)(1.0 / std::sqrt((double)d.hadamard_block));
     }
 
     const bool resid = d.residual_group != 0;
     const dim3 grid(pl.Gs * pl.Gt), block(kThreads);
-    const size_t smem = pl.smem;
+    const size_t smem = p.wi_staged ? pl.smem : pl.smem_nostage;
 #ifdef EVA_TIMELINE
     p.timeline = h->timeline;
 #endif
@@ -413,7 +452,7 @@ eva_status_t eva_vq_linear_run_ex(eva_vq_linear_t h, const void *x, int32_t B, v
         p.chk_record = h->status;
     }
 #endif
-    e = launch_pdl(lookup_fn(pair_t, resid, h->tiles_per_cb != 0), grid, block, smem, s, pl.Gs, p);
+    e = launch_pdl(lookup_fn(pair_t, resid, h->tiles_per_cb != 0, p.rot_b != 0), grid, block, smem, s, pl.Gs, p);
     if (e != cudaSuccess) return cuda_status(e);
     ++kernels;
     h->last_grid = (int)grid.x;
@@ -493,6 +532,8 @@ eva_status_t eva_vq_linear_run_noalloc(eva_vq_linear_t h, const void *x, int32_t
     p.Gs = pl.Gs;
     p.Gt = pl.Gt;
     p.acc_tiles = (h->T + pl.Gt - 1) / pl.Gt;
+    p.wi_staged = pl.staged;
+    p.status = h->status;
 #ifdef EVA_TIMELINE
     p.timeline = h->timeline;
 #endif
@@ -511,7 +552,7 @@ eva_status_t eva_vq_linear_run_noalloc(eva_vq_linear_t h, const void *x, int32_t
         p.x_f32 = 1;
     }
     const bool resid = d.residual_group != 0;
-    e = launch_pdl(lookup_fn(pair_t, resid, h->tiles_per_cb != 0), dim3(pl.Gs * pl.Gt), dim3(kThreads),
+    e = launch_pdl(lookup_fn(pair_t, resid, h->tiles_per_cb != 0, false), dim3(pl.Gs * pl.Gt), dim3(kThreads),
                    pl.smem, s, pl.Gs, p);
     return cuda_status(e);
 }
@@ -594,7 +635,7 @@ eva_status_t eva_vq_linear_info(eva_vq_linear_t h, eva_vq_info *info) {
     info->slices = h->S;
     info->row_tiles = h->T;
     info->grid = h->last_grid ? h->last_grid : h->plan[0].Gs * h->plan[0].Gt;
-    info->kernels_per_run = h->last_kernels ? h->last_kernels : (d.hadamard_block ? 2 : 1);
+    info->kernels_per_run = h->last_kernels ? h->last_kernels : 1;
     info->path = h->last_path ? h->last_path : EVA_PATH_OC_LOOKUP;
     info->sm_count = h->sm_count;
     return EVA_OK;

@@ -46,6 +46,13 @@ struct LookupParams {
     int independent;         // neither x nor y is touched by the preceding kernel:
                              // run without waiting for it (wait only before exit)
     int acc_tiles;           // row tiles of the largest CTA (shared-memory layout)
+    int wi_staged;           // leading row tiles whose first-slice indices are copied
+                             // into shared memory by one bulk copy in the prologue
+    int *status;             // device error word (bit 0: a bounded wait gave up)
+    const int8_t *hs;        // randomized Hadamard signs s [K] (fused rotation only)
+    int rot_b;               // 0, or the rotation block b: x~ = s . (H_b x) / sqrt(b) is
+                             // computed in the lookup kernel from fp16 x
+    float rot_scale;         // 1 / sqrt(b), rounded to fp32
 #ifdef EVA_DEVICE_CHECKS
     // Debug build only: bounds of every buffer the kernel touches.  A
     // violating access is skipped and the first one is recorded.
@@ -157,6 +164,43 @@ __device__ __forceinline__ void pdl_launch() { asm volatile("griddepcontrol.laun
 __device__ __forceinline__ void cluster_sync_all() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
                  "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// ---- one-shot mbarrier + bulk copy (global -> own shared memory, no multicast)
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+// Bounded wait for phase `parity` of the barrier: gives up (returns false)
+// after 2^20 tries (each try suspends for a short, hardware-chosen time).
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+    for (int it = 0; it < (1 << 20); ++it) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity)
+            : "memory");
+        if (ok) return true;
+    }
+    return false;
+}
+__device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ uint4 lds128(uint32_t off) {
+    return *reinterpret_cast<const uint4 *>(eva_smem + off);
 }
 
 // 16-byte store into the shared memory of cluster CTA `rank`, at the address
@@ -278,6 +322,133 @@ __device__ __forceinline__ void stage_x(const LookupParams &p, int s, int pr, in
     if (!EVA_BAD_S(off) && !EVA_BAD_S(off + 28u)) {
         *reinterpret_cast<float4 *>(eva_smem + off) = make_float4(v[0], v[1], v[2], v[3]);
         *reinterpret_cast<float4 *>(eva_smem + off + 16) = make_float4(v[4], v[5], v[6], v[7]);
+    }
+}
+
+// ------------------------------------------------- fused Hadamard rotation
+//
+// The randomized block rotation of the 3-bit article (x~ = Q^T x with
+// Q = blockdiag(H_b) diag(s) / sqrt(b)) computed while staging x: each CTA
+// transforms the whole b-block its slice falls in and keeps its 256 outputs.
+// The butterflies are those of the in-order fast Walsh-Hadamard transform
+// (stage h pairs positions lo and lo + h, lo with bit h clear, into
+// (a + c, a - c)), stage by stage, so every value is bitwise that of the
+// standalone rotation kernel below.
+
+// Eight consecutive fp16 inputs of token `tok` from k0 on, as fp32; zeros past
+// K or past B.
+__device__ __forceinline__ void load_x8_f16(const LookupParams &p, int tok, int k0, float (&v)[8]) {
+    const size_t i = (size_t)tok * p.K + k0;
+    if (tok < p.B && k0 + 8 <= p.K && (i & 7) == 0) {
+        const uint4 *xp = reinterpret_cast<const uint4 *>(reinterpret_cast<const __half *>(p.x) + i);
+        if (!EVA_BAD_G(BUF_X, xp, 16)) {
+            const uint4 r = __ldcg(xp);
+            const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const __half2 h2 = *reinterpret_cast<const __half2 *>(&w[j]);
+                v[2 * j] = __low2float(h2);
+                v[2 * j + 1] = __high2float(h2);
+            }
+            return;
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = load_x(p, tok, k0 + j);
+}
+
+// Stages h = 1 .. min(b, 256) / 2 over 256 consecutive inputs held by one
+// warp, eight per lane (lane L holds 8L .. 8L + 7).
+__device__ __forceinline__ void fwht_warp256(float (&v)[8], int lane, int b) {
+#pragma unroll
+    for (int h = 1; h < 8; h <<= 1) {
+        if (h >= b) break;
+#pragma unroll
+        for (int lo = 0; lo < 8; ++lo)
+            if (!(lo & h)) {
+                const float a = v[lo], c = v[lo + h];
+                v[lo] = a + c;
+                v[lo + h] = a - c;
+            }
+    }
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) {      // h = 8 m: partner lane L ^ m
+        if (8 * m >= b) break;
+        const bool hi = (lane & m) != 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float o = __shfl_xor_sync(0xffffffffu, v[j], m);
+            v[j] = hi ? o - v[j] : v[j] + o;
+        }
+    }
+}
+
+template <bool PAIR_T>
+__device__ __forceinline__ void stage_x_rot(const LookupParams &p, int s, int pr, int warp, int lane, int tid,
+                                            uint32_t x_off, uint32_t rot_off) {
+    constexpr int NTOK = PAIR_T ? 2 : 1;
+    const int b = p.rot_b, ks = s * kSliceK;
+    if (b <= kSliceK) {
+        // Whole blocks inside the slice: one warp per token.
+        if (warp >= NTOK) return;
+        const int tok = PAIR_T ? 2 * pr + warp : 0;
+        float v[8];
+        load_x8_f16(p, tok, ks + 8 * lane, v);
+        fwht_warp256(v, lane, b);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int k = ks + 8 * lane + j;
+            v[j] = (k < p.K ? (float)p.hs[k] : 0.f) * v[j] * p.rot_scale;
+        }
+        const uint32_t off = x_off + (uint32_t)(warp * kSliceK + 8 * lane) * 4u;
+        if (!EVA_BAD_S(off) && !EVA_BAD_S(off + 28u)) {
+            *reinterpret_cast<float4 *>(eva_smem + off) = make_float4(v[0], v[1], v[2], v[3]);
+            *reinterpret_cast<float4 *>(eva_smem + off + 16) = make_float4(v[4], v[5], v[6], v[7]);
+        }
+        return;
+    }
+    // b > 256 (K is a multiple of b): the slice is sub-block `a` of its block.
+    // Stages h < 256 run per sub-block in one warp each; h >= 256 combine the
+    // nsb = b / 256 sub-blocks through shared memory.
+    const int nsb = b / kSliceK, blk0 = (ks / b) * b, a = (ks - blk0) / kSliceK;
+    for (int w = warp; w < NTOK * nsb; w += kWarps) {
+        const int tk = w / nsb, sb = w - tk * nsb;
+        float v[8];
+        load_x8_f16(p, PAIR_T ? 2 * pr + tk : 0, blk0 + sb * kSliceK + 8 * lane, v);
+        fwht_warp256(v, lane, kSliceK);
+        const uint32_t off = rot_off + (uint32_t)(w * kSliceK + 8 * lane) * 4u;
+        if (!EVA_BAD_S(off) && !EVA_BAD_S(off + 28u)) {
+            *reinterpret_cast<float4 *>(eva_smem + off) = make_float4(v[0], v[1], v[2], v[3]);
+            *reinterpret_cast<float4 *>(eva_smem + off + 16) = make_float4(v[4], v[5], v[6], v[7]);
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < NTOK * kSliceK; e += kThreads) {
+        const int tk = e / kSliceK, i = e - tk * kSliceK;
+        float u[16];
+#pragma unroll
+        for (int sb = 0; sb < 16; ++sb) {
+            const uint32_t off = rot_off + (uint32_t)((tk * nsb + sb) * kSliceK + i) * 4u;
+            u[sb] = (sb < nsb && !EVA_BAD_S(off)) ? *reinterpret_cast<const float *>(eva_smem + off) : 0.f;
+        }
+#pragma unroll
+        for (int m = 1; m < 16; m <<= 1) {  // h = 256 m
+            if (m >= nsb) break;
+#pragma unroll
+            for (int lo = 0; lo < 16; ++lo)
+                if (!(lo & m)) {
+                    const float x0 = u[lo], x1 = u[lo + m];
+                    u[lo] = x0 + x1;
+                    u[lo + m] = x0 - x1;
+                }
+        }
+        float r = u[0];
+#pragma unroll
+        for (int sb = 1; sb < 16; ++sb)
+            if (sb == a) r = u[sb];
+        const int k = ks + i;
+        const uint32_t off = x_off + (uint32_t)(tk * kSliceK + i) * 4u;
+        if (!EVA_BAD_S(off)) *reinterpret_cast<float *>(eva_smem + off) = (float)p.hs[k] * r * p.rot_scale;
     }
 }
 
@@ -434,7 +605,7 @@ __device__ __forceinline__ void build_sign_table(const LookupParams &p, int warp
 // so the weight stream of layer l+1 overlaps the lookups of layer l; the
 // token-pair and residual variants need more registers and run one CTA per SM.
 
-template <bool PAIR_T, bool RESID, bool GROUPED>
+template <bool PAIR_T, bool RESID, bool GROUPED, bool ROT>
 __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_lookup_kernel(const LookupParams p) {
     // Index units in flight per warp: with per-group codebooks a warp has at
     // most one tile per codebook pass, so a short ring suffices.
@@ -450,7 +621,11 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
     constexpr uint32_t HI_OFF = PAIR_T ? 128u : 0u;                      // a2/a3 column offset
     constexpr uint32_t T_OFF = PAIR_T ? (uint32_t)kOcBytes : 128u;       // residual table
     constexpr uint32_t X_OFF = (PAIR_T && RESID) ? 2u * kOcBytes : (uint32_t)kOcBytes;
-    constexpr uint32_t ACC_OFF = X_OFF + kXStageBytes;   // per-CTA running sums
+    constexpr uint32_t XS_BYTES = PAIR_T ? kXStageBytes : kXStageBytes / 2;   // x~ of 1 or 2 tokens
+    constexpr uint32_t BAR_OFF = X_OFF + XS_BYTES;       // mbarrier of the index staging copy
+    constexpr uint32_t ACC_OFF = BAR_OFF + 128u;         // per-CTA running sums (128-byte
+                                                         // tile blocks stay 128-byte aligned)
+    constexpr int NTOK_C = PAIR_T ? 2 : 1;
     // GROUPED: one codebook per tiles_per_cb row tiles (else one shared codebook).
     const int cb_first = GROUPED ? t0 / p.tiles_per_cb : 0;
     const int cb_last = GROUPED ? (t1 - 1) / p.tiles_per_cb : 0;
@@ -461,16 +636,43 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
     // A CTA may write a peer's shared memory only once the peer runs: arrive
     // now, wait (long satisfied) before the first remote store.
     asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+    // The first slice's index bytes of the leading `staged` tiles: one bulk
+    // copy into shared memory, completing on an mbarrier.
+    const int staged = min(p.wi_staged, t1 - t0);
+    const uint32_t stage_bytes_c = (uint32_t)((p.acc_tiles + p.Gs - 1) / p.Gs) * p.Gs * kTileRows * 2u * 4u;
+    // Fused rotation scratch (b > 256): the b / 256 transformed sub-blocks of each token.
+    const uint32_t ROT_OFF = (ACC_OFF + (uint32_t)p.acc_tiles * kTileRows * 2u * 4u + stage_bytes_c + 127u) & ~127u;
+    const uint32_t rot_bytes = (ROT && p.rot_b > kSliceK) ? (uint32_t)NTOK_C * (uint32_t)p.rot_b * 4u : 0u;
+    const uint32_t WIS_OFF = ROT_OFF + rot_bytes;
+    const uint32_t bar = (uint32_t)__cvta_generic_to_shared(eva_smem + BAR_OFF);
+    if (tid == 0 && staged > 0) {
+        mbar_init(bar, 1);
+        const uint8_t *src = p.wi + ((size_t)s0 * p.T + t0) * kUnitBytes;
+        const uint32_t bytes = (uint32_t)staged * kUnitBytes;
+        if (staged > 0 && !EVA_BAD_G(BUF_WI, src, bytes) && !EVA_BAD_S(WIS_OFF) &&
+            !EVA_BAD_S(WIS_OFF + bytes - 4u)) {
+            mbar_arrive_expect_tx(bar, bytes);
+            const uint32_t dst = (uint32_t)__cvta_generic_to_shared(eva_smem + WIS_OFF);
+            for (uint32_t off = 0; off < bytes; off += 32768u)
+                bulk_copy_g2s(dst + off, src + off, min(32768u, bytes - off), bar);
+        } else {
+            mbar_arrive(bar);
+        }
+    }
     if (tid < s1 - s0) {
-        const size_t u = (size_t)(s0 + tid) * p.T + t0;
-        const uint32_t nt = (uint32_t)(t1 - t0);
-        if (!EVA_BAD_G(BUF_WI, p.wi + u * kUnitBytes, nt * kUnitBytes))
+        // Bulk L2 prefetch of this CTA's index range (the staged part excepted).
+        const int skip = (tid == 0) ? staged : 0;
+        const size_t u = (size_t)(s0 + tid) * p.T + t0 + skip;
+        const uint32_t nt = (uint32_t)(t1 - t0 - skip);
+        if (nt > 0 && !EVA_BAD_G(BUF_WI, p.wi + u * kUnitBytes, nt * kUnitBytes))
             prefetch_l2_bulk(p.wi + u * kUnitBytes, nt * kUnitBytes);
         if (RESID) {
-            if (!EVA_BAD_G(BUF_SG, p.sg + u * kSignUnitBytes, nt * kSignUnitBytes))
-                prefetch_l2_bulk(p.sg + u * kSignUnitBytes, nt * kSignUnitBytes);
-            if (!EVA_BAD_G(BUF_AL, p.al + u * kAlphaUnitHalves, nt * kAlphaUnitHalves * 2))
-                prefetch_l2_bulk(p.al + u * kAlphaUnitHalves, nt * kAlphaUnitHalves * 2);
+            const size_t ur = (size_t)(s0 + tid) * p.T + t0;
+            const uint32_t ntr = (uint32_t)(t1 - t0);
+            if (!EVA_BAD_G(BUF_SG, p.sg + ur * kSignUnitBytes, ntr * kSignUnitBytes))
+                prefetch_l2_bulk(p.sg + ur * kSignUnitBytes, ntr * kSignUnitBytes);
+            if (!EVA_BAD_G(BUF_AL, p.al + ur * kAlphaUnitHalves, ntr * kAlphaUnitHalves * 2))
+                prefetch_l2_bulk(p.al + ur * kAlphaUnitHalves, ntr * kAlphaUnitHalves * 2);
         }
     }
     uint32_t bfrag[4];
@@ -510,12 +712,14 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
     // [ceil(acc_tiles / Gs) slots][Gs sources][16 rows][2 tokens].
     float *acc_s = reinterpret_cast<float *>(eva_smem + ACC_OFF);
     const uint32_t STAGE_OFF = ACC_OFF + (uint32_t)p.acc_tiles * kTileRows * 2u * 4u;
+    bool wi_ready = false;   // the staging copy has landed (waited for once)
     const float *stage = reinterpret_cast<const float *>(eva_smem + STAGE_OFF);
     const uint32_t stage_addr = (uint32_t)__cvta_generic_to_shared(eva_smem + STAGE_OFF);
     for (int pr = 0; pr < npairs; ++pr) {
 
         for (int s = s0; s < s1; ++s) {
-            stage_x<PAIR_T>(p, s, pr, warp, lane, X_OFF);
+            if constexpr (ROT) stage_x_rot<PAIR_T>(p, s, pr, warp, lane, tid, X_OFF, ROT_OFF);
+            else stage_x<PAIR_T>(p, s, pr, warp, lane, X_OFF);
             for (int cb = cb_first; cb <= cb_last; ++cb) {
                 // This warp's tiles that use codebook cb: the index range [i0, i1).
                 int i0 = 0, i1 = ntw;
@@ -528,15 +732,18 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
                         cur_cb = cb;
                     }
                 }
-                // Lookahead ring of LA units: the first ones load (from
-                // L2, where the prologue's bulk prefetch put them) while the
-                // image builds; each processed tile refills the ring's tail.
+                // Tiles [i0, i_st) of the first slice read their indices from the
+                // shared-memory copy; the rest stream through a lookahead ring of
+                // LA units: the first ones load (from L2, where the prologue's
+                // bulk prefetch put them) while the image builds, and each
+                // processed tile refills the ring's tail.
+                const int i_st = (s == s0) ? min(i1, max(i0, (staged - warp + kWarps - 1) / kWarps)) : i0;
                 uint4 nb[LA][2];
 #pragma unroll
                 for (int d = 0; d < LA; ++d) {
                     nb[d][0] = nb[d][1] = make_uint4(0u, 0u, 0u, 0u);
-                    if (i0 + d < i1) {
-                        const uint8_t *up = p.wi + ((size_t)s * p.T + t0 + warp + kWarps * (i0 + d)) * kUnitBytes + 16 * lane;
+                    if (i_st + d < i1) {
+                        const uint8_t *up = p.wi + ((size_t)s * p.T + t0 + warp + kWarps * (i_st + d)) * kUnitBytes + 16 * lane;
                         if (!EVA_BAD_G(BUF_WI, up, 16) && !EVA_BAD_G(BUF_WI, up + 512, 16)) ldg_unit(up, nb[d][0], nb[d][1]);
                     }
                 }
@@ -546,21 +753,14 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
                 if (RESID && cb == cb_first) build_sign_table<PAIR_T>(p, warp, lane, T_OFF, X_OFF);
                 __syncthreads();
                 EVA_STAMP(3);
-#pragma unroll 1
-                for (int i = i0; i < i1; ++i) {
-                    const int tl = warp + kWarps * i;              // tile index within the CTA
-                    const size_t unit = (size_t)s * p.T + t0 + tl;
-                    const uint4 v0 = nb[0][0], v1 = nb[0][1];
-#pragma unroll
-                    for (int d = 0; d + 1 < LA; ++d) {
-                        nb[d][0] = nb[d + 1][0];
-                        nb[d][1] = nb[d + 1][1];
-                    }
-                    if (i + LA < i1) {
-                        const uint8_t *up = p.wi + (unit + (size_t)kWarps * LA) * kUnitBytes + 16 * lane;
-                        if (!EVA_BAD_G(BUF_WI, up, 16) && !EVA_BAD_G(BUF_WI, up + 512, 16))
-                            ldg_unit(up, nb[LA - 1][0], nb[LA - 1][1]);
-                    }
+                if (staged > 0 && !wi_ready) {
+                    // Bounded: if the copy never lands the CTA records it, skips
+                    // nothing else and still joins the cluster barrier below.
+                    wi_ready = true;
+                    if (!mbar_wait_bounded(bar, 0) && tid == 0 && p.status) atomicOr(p.status, 1);
+                }
+                // One tile: 32 lookups per lane, accumulated by 8 MMAs (+ the residual).
+                auto tile = [&](const int tl, const size_t unit, const uint4 v0, const uint4 v1) {
                     const uint32_t wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
                     // Even and odd k-steps accumulate in two chains.
                     float da[4] = {0.f, 0.f, 0.f, 0.f}, db[4] = {0.f, 0.f, 0.f, 0.f};
@@ -634,6 +834,34 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
                                     acc_s[ai] = (s == s0) ? da[2 * h + e] : acc_s[ai] + da[2 * h + e];
                             }
                     }
+                };
+                // Staged tiles first (indices from shared memory) ...
+#pragma unroll 1
+                for (int i = i0; i < i_st; ++i) {
+                    const int tl = warp + kWarps * i;              // tile index within the CTA
+                    const uint32_t wo = WIS_OFF + (uint32_t)tl * kUnitBytes + 16u * lane;
+                    const uint4 v0 = (EVA_BAD_S(wo) || EVA_BAD_S(wo + 12u)) ? make_uint4(0u, 0u, 0u, 0u) : lds128(wo);
+                    const uint4 v1 = (EVA_BAD_S(wo + 512u) || EVA_BAD_S(wo + 524u)) ? make_uint4(0u, 0u, 0u, 0u)
+                                                                                       : lds128(wo + 512u);
+                    tile(tl, (size_t)s * p.T + t0 + tl, v0, v1);
+                }
+                // ... then the streamed ones, through the lookahead ring.
+#pragma unroll 1
+                for (int i = i_st; i < i1; ++i) {
+                    const int tl = warp + kWarps * i;              // tile index within the CTA
+                    const size_t unit = (size_t)s * p.T + t0 + tl;
+                    const uint4 v0 = nb[0][0], v1 = nb[0][1];
+#pragma unroll
+                    for (int d = 0; d + 1 < LA; ++d) {
+                        nb[d][0] = nb[d + 1][0];
+                        nb[d][1] = nb[d + 1][1];
+                    }
+                    if (i + LA < i1) {
+                        const uint8_t *up = p.wi + (unit + (size_t)kWarps * LA) * kUnitBytes + 16 * lane;
+                        if (!EVA_BAD_G(BUF_WI, up, 16) && !EVA_BAD_G(BUF_WI, up + 512, 16))
+                            ldg_unit(up, nb[LA - 1][0], nb[LA - 1][1]);
+                    }
+                    tile(tl, unit, v0, v1);
                 }
             }
         }
@@ -683,6 +911,8 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
         // reading this pair's stage (and this CTA's warps done with acc_s).
         if (pr + 1 < npairs) cluster_sync_all();
     }
+    // No bulk copy may still be writing this CTA's shared memory at exit.
+    if (staged > 0 && !wi_ready) mbar_wait_bounded(bar, 0);
     // Independent calls still complete after the preceding kernel, so that
     // later calls that wait on this one see the stream order.
     if (p.independent) pdl_wait();

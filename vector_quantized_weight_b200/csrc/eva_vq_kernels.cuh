@@ -476,7 +476,18 @@ __device__ __forceinline__ void load_codebook_frag(const LookupParams &p, int cb
 // fp16 inputs are exact in tf32 and their products exact in fp32), rounded to
 // fp16 and stored in the conflict-free image.  Warp w builds the centroid
 // columns 8 nt .. 8 nt + 7 of nt = w + kWarps j, j = 0..3.
-template <bool PAIR_T>
+// Diagnostics build only (EVA_NAIVE_OC_LAYOUT): the one-token image of a
+// layer without residual is stored the naive way, word(c, w) at row w,
+// column c, so that a warp's 32 lookups land on banks chosen by the indices
+// (bank = c mod 32).  It exists to measure the bank conflicts the
+// column-per-sub-vector layout removes; results are the same.
+#ifdef EVA_NAIVE_OC_LAYOUT
+constexpr bool kNaiveOcBuild = true;
+#else
+constexpr bool kNaiveOcBuild = false;
+#endif
+
+template <bool PAIR_T, bool NAIVE = false>
 __device__ __forceinline__ void build_oc(const LookupParams &p, int warp, int g, int q,
                                          const uint32_t (&bf)[4], uint32_t x_off) {
     constexpr int NTOK = PAIR_T ? 2 : 1;
@@ -509,7 +520,8 @@ __device__ __forceinline__ void build_oc(const LookupParams &p, int warp, int g,
                 xor_permute(W, q);
 #pragma unroll
                 for (int r = 0; r < 4; ++r) {
-                    const uint32_t off = row + 4u * (g + 8 * (r ^ q));
+                    const uint32_t off = NAIVE ? 1024u * (uint32_t)(g + 8 * (r ^ q)) + 4u * (8 * nt + 2 * q + cc)
+                                               : row + 4u * (g + 8 * (r ^ q));
                     if (!EVA_BAD_S(off)) sts32(off, W[r]);
                 }
             }
@@ -626,6 +638,7 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
     constexpr uint32_t ACC_OFF = BAR_OFF + 128u;         // per-CTA running sums (128-byte
                                                          // tile blocks stay 128-byte aligned)
     constexpr int NTOK_C = PAIR_T ? 2 : 1;
+    constexpr bool NAIVE = kNaiveOcBuild && !PAIR_T && !RESID;
     // GROUPED: one codebook per tiles_per_cb row tiles (else one shared codebook).
     const int cb_first = GROUPED ? t0 / p.tiles_per_cb : 0;
     const int cb_last = GROUPED ? (t1 - 1) / p.tiles_per_cb : 0;
@@ -749,7 +762,7 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
                 }
                 __syncthreads();  // x~ staged, accumulator cleared, previous image consumed
                 EVA_STAMP(2);
-                build_oc<PAIR_T>(p, warp, g, q, bfrag, X_OFF);
+                build_oc<PAIR_T, NAIVE>(p, warp, g, q, bfrag, X_OFF);
                 if (RESID && cb == cb_first) build_sign_table<PAIR_T>(p, warp, lane, T_OFF, X_OFF);
                 __syncthreads();
                 EVA_STAMP(3);
@@ -767,10 +780,18 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
 #pragma unroll
                     for (int s8 = 0; s8 < 8; ++s8) {
                         const uint32_t cw = (4u * lane + 16u * s8) & 127u;   // 4 * oc_col(lane, s8)
-                        const uint32_t o0 = OC_OFF + __byte_perm(wv[s8], cw, 0x5504);
-                        const uint32_t o1 = OC_OFF + __byte_perm(wv[s8], cw, 0x5514);
-                        const uint32_t o2 = OC_OFF + HI_OFF + __byte_perm(wv[s8], cw, 0x5524);
-                        const uint32_t o3 = OC_OFF + HI_OFF + __byte_perm(wv[s8], cw, 0x5534);
+                        uint32_t o0, o1, o2, o3;
+                        if constexpr (NAIVE) {
+                            o0 = OC_OFF + (cw << 8) + ((wv[s8] & 0xFFu) << 2);
+                            o1 = OC_OFF + (cw << 8) + (((wv[s8] >> 8) & 0xFFu) << 2);
+                            o2 = OC_OFF + (cw << 8) + (((wv[s8] >> 16) & 0xFFu) << 2);
+                            o3 = OC_OFF + (cw << 8) + ((wv[s8] >> 24) << 2);
+                        } else {
+                            o0 = OC_OFF + __byte_perm(wv[s8], cw, 0x5504);
+                            o1 = OC_OFF + __byte_perm(wv[s8], cw, 0x5514);
+                            o2 = OC_OFF + HI_OFF + __byte_perm(wv[s8], cw, 0x5524);
+                            o3 = OC_OFF + HI_OFF + __byte_perm(wv[s8], cw, 0x5534);
+                        }
                         const uint32_t a0 = EVA_BAD_S(o0) ? 0u : lds32(o0);
                         const uint32_t a1 = EVA_BAD_S(o1) ? 0u : lds32(o1);
                         const uint32_t a2 = EVA_BAD_S(o2) ? 0u : lds32(o2);

@@ -57,7 +57,8 @@ _lib = None
 
 def library_path() -> str:
     """The regular library; EVA_VQ_CHECKED=1 selects the device-check build,
-    EVA_VQ_TIMELINE=1 the phase-timeline build (diagnostics only), and
+    EVA_VQ_TIMELINE=1 the phase-timeline build, EVA_VQ_NAIVE=1 the build with
+    the naive image layout (all three diagnostics only), and
     EVA_VQ_LIBRARY=<path> any other build of the same C ABI."""
     if os.environ.get("EVA_VQ_LIBRARY"):
         return os.environ["EVA_VQ_LIBRARY"]
@@ -65,6 +66,8 @@ def library_path() -> str:
         return _build.CHECKED_LIB
     if os.environ.get("EVA_VQ_TIMELINE") == "1":
         return _build.TIMELINE_LIB
+    if os.environ.get("EVA_VQ_NAIVE") == "1":
+        return _build.NAIVE_LIB
     return _build.LIB
 
 
@@ -77,7 +80,8 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     if not os.path.exists(path):
         if not build_if_missing:
             raise RuntimeError(f"{path} is missing; build it with vector_quantized_weight_b200.build")
-        _build.build(checked=path == _build.CHECKED_LIB, timeline=path == _build.TIMELINE_LIB)
+        _build.build(checked=path == _build.CHECKED_LIB, timeline=path == _build.TIMELINE_LIB,
+                     naive=path == _build.NAIVE_LIB)
     lib = ctypes.CDLL(path)
     P, I32, H = ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p
     lib.eva_vq_linear_create.argtypes = [ctypes.POINTER(H), ctypes.POINTER(eva_vq_desc), P, P, P, P, P, P]

@@ -24,7 +24,7 @@ _lib = None
 def build(force: bool = False) -> str:
     """Compile eva_oracle.c into libeva_oracle.so next to it (gcc, -fopenmp)."""
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
                "-o", _LIB + ".tmp", _SRC, "-lm"]
         subprocess.run(cmd, check=True)
         os.replace(_LIB + ".tmp", _LIB)
@@ -56,6 +56,14 @@ def _load():
         lib.vq_oracle_lookup_form.restype = ctypes.c_int
         lib.vq_oracle_optimal_alpha.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int, P]
         lib.vq_oracle_optimal_alpha.restype = ctypes.c_int
+        I64 = ctypes.c_int64
+        lib.vq_oracle_kmeans_assign.argtypes = [P, I64, ctypes.c_int, P, ctypes.c_int, I64, P]
+        lib.vq_oracle_kmeans_assign.restype = ctypes.c_int
+        lib.vq_oracle_kmeans_update.argtypes = [P, I64, ctypes.c_int, P, ctypes.c_int, I64, P, P, P]
+        lib.vq_oracle_kmeans_update.restype = ctypes.c_int
+        lib.vq_oracle_residual.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, ctypes.c_int,
+                                           P, ctypes.c_int, ctypes.c_int, P, P]
+        lib.vq_oracle_residual.restype = ctypes.c_int
         lib.vq_oracle_max_threads.argtypes = []
         lib.vq_oracle_max_threads.restype = ctypes.c_int
         _lib = lib
@@ -165,3 +173,86 @@ def layer_linear(layer, x, nthreads=1) -> np.ndarray:
     return linear(layer.wc, layer.wi, x, signs=layer.signs, alpha=layer.alpha, hsign=layer.hsign,
                   codebook_rows=s.codebook_rows, residual_group=s.residual_group,
                   hadamard_block=s.hadamard_block, nthreads=nthreads)
+
+
+# ------------------------------------------------------------------ quantizer
+
+def kmeans_assign(v, centroids, vecs_per_cb: int = 0) -> np.ndarray:
+    """Nearest centroid (fp32 squared distance, first minimum) of each vector.
+    v: [M][d] float32; centroids: [G][ncent][d] (or [ncent][d]) float32 -> int32 [M]."""
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    c = np.ascontiguousarray(centroids, dtype=np.float32)
+    if c.ndim == 2:
+        c = c[None]
+    M, d = v.shape
+    out = np.empty(M, np.int32)
+    rc = _load().vq_oracle_kmeans_assign(_ptr(v), M, d, _ptr(c), c.shape[1], int(vecs_per_cb), _ptr(out))
+    if rc:
+        raise ValueError(f"vq_oracle_kmeans_assign: {rc}")
+    return out
+
+
+def kmeans_update(v, idx, centroids, vecs_per_cb: int = 0):
+    """(new centroids float32 [G][ncent][d], counts int64 [G][ncent]): cluster means in double."""
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    c = np.ascontiguousarray(centroids, dtype=np.float32)
+    if c.ndim == 2:
+        c = c[None]
+    M, d = v.shape
+    new = np.empty_like(c)
+    counts = np.empty(c.shape[:2], np.int64)
+    rc = _load().vq_oracle_kmeans_update(_ptr(v), M, d, _ptr(idx), c.shape[1], int(vecs_per_cb), _ptr(c),
+                                         _ptr(new), _ptr(counts))
+    if rc:
+        raise ValueError(f"vq_oracle_kmeans_update: {rc}")
+    return new, counts
+
+
+def residual(wrot, wc, wi, *, codebook_rows: int = 0, group: int = 128):
+    """(packed signs u8 [N][K/8], alpha float64 [N][K/group]) of wrot - wc[wi]."""
+    wrot = np.ascontiguousarray(wrot, dtype=np.float32)
+    wc16 = _c16(wc)
+    if wc16.ndim == 2:
+        wc16 = wc16[None]
+    _, ncent, d = wc16.shape
+    wi8 = np.ascontiguousarray(wi, dtype=np.uint8)
+    N, K = wrot.shape
+    signs = np.empty((N, K // 8), np.uint8)
+    alpha = np.empty((N, K // group), np.float64)
+    rc = _load().vq_oracle_residual(_ptr(wrot), N, K, d, _ptr(wc16), ncent, _ptr(wi8), int(codebook_rows),
+                                    int(group), _ptr(signs), _ptr(alpha))
+    if rc:
+        raise ValueError(f"vq_oracle_residual: {rc}")
+    return signs, alpha
+
+
+def quantize(w, init_centroids, iters: int, *, hsign=None, hadamard_block: int = 0, codebook_rows: int = 0,
+             group: int = 128, d: int = 4):
+    """The 3-bit article's quantize() pipeline, step by step (plain K-means):
+    1. W_rot = W Q (rows rotated like x~, dense per-block product, then fp32);
+    2. blocks of d along each row; 3. `iters` Lloyd iterations from
+    init_centroids [G][ncent][d]; the codebook is stored in fp16 and the
+    pointers are the nearest fp16 centroids; 4.-7. residual, signs (packed),
+    alpha = mean |r| per group (rounded to fp16).
+    Returns (wc fp16 [G][ncent][d], wi u8 [N][K/d], signs u8 [N][K/8], alpha fp16 [N][K/group],
+    wrot float32 [N][K])."""
+    w16 = np.ascontiguousarray(w, dtype=np.float16)
+    N, K = w16.shape
+    if hadamard_block:
+        wrot = hadamard(w16, hsign, hadamard_block).astype(np.float32)
+    else:
+        wrot = f16_to_f64(w16).astype(np.float32)
+    v = wrot.reshape(N * (K // d), d)
+    vecs_per_cb = codebook_rows * (K // d) if codebook_rows else 0
+    cent = np.ascontiguousarray(init_centroids, dtype=np.float32)
+    if cent.ndim == 2:
+        cent = cent[None]
+    for _ in range(int(iters)):
+        idx = kmeans_assign(v, cent, vecs_per_cb)
+        cent, _counts = kmeans_update(v, idx, cent, vecs_per_cb)
+    wc = cent.astype(np.float16)
+    idx = kmeans_assign(v, wc.astype(np.float32), vecs_per_cb)
+    wi = idx.astype(np.uint8).reshape(N, K // d)
+    signs, alpha = residual(wrot, wc, wi, codebook_rows=codebook_rows, group=group)
+    return wc, wi, signs, alpha.astype(np.float16), wrot

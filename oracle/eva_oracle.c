@@ -39,6 +39,19 @@
  *    signs, the alpha minimising ||r - alpha*sign(r)||^2 over a group.
  *    (vq_oracle_optimal_alpha)
  *
+ *  - The same sample's quantize() pipeline, offline: rotate the weight rows
+ *    (W_rot = W Q, the same per-block transform as x~, row by row), cut them
+ *    into blocks of d, run K-means to get the codebook and the pointers,
+ *    take the residual W_rot - codebook[pointers], its 1-bit signs and the
+ *    optimal scale per group, and pack the signs into bytes.  Readings taken:
+ *    plain Lloyd K-means (the sample's sensitivity weights need calibration
+ *    data, which the pages do not give), started from centroids the caller
+ *    passes in, for a given number of iterations, an empty cluster keeping
+ *    its centroid; the nearest-centroid decision is made in fp32 (the
+ *    precision the GPU kernel decides in), distances summed in component
+ *    order, ties to the lower index; centroid means in double.
+ *    (vq_oracle_kmeans_assign, vq_oracle_kmeans_update, vq_oracle_residual)
+ *
  * Layouts are the canonical ones of the input generator:
  *   wc [G][2^n][d] fp16, wi [N][K/d] u8, signs [N][K/8] u8 LSB-first
  *   (bit set -> +1, clear -> -1), alpha [N][K/rg] fp16, hsign [K] int8,
@@ -334,6 +347,110 @@ int vq_oracle_optimal_alpha(const double *r, int rows, int cols, int group, doub
             }
             alpha_out[(size_t)i * (cols / group) + q] = num / den;
         }
+    return 0;
+}
+
+/*
+ * K-means assignment: for each of the M vectors of length d (fp32, [M][d]),
+ * the index of the nearest of the ncent centroids of its codebook (fp32,
+ * [G][ncent][d]); vector m uses codebook m / vecs_per_cb (0: one codebook).
+ * The squared distance is accumulated in float, one component at a time in
+ * order (each difference, square and sum rounded to float); the first
+ * minimum wins.  Compiled without floating-point contraction.
+ */
+int vq_oracle_kmeans_assign(const float *v, int64_t M, int d, const float *cent, int ncent,
+                            int64_t vecs_per_cb, int32_t *idx_out)
+{
+    if (!v || !cent || !idx_out || M < 0 || d <= 0 || ncent <= 0 || vecs_per_cb < 0) return -1;
+    for (int64_t m = 0; m < M; ++m) {
+        const int64_t g = vecs_per_cb ? m / vecs_per_cb : 0;
+        const float *cb = cent + (size_t)g * ncent * d;
+        int best = 0;
+        float best_d = 0.f;
+        for (int c = 0; c < ncent; ++c) {
+            float dist = 0.f;
+            for (int t = 0; t < d; ++t) {
+                const float diff = v[(size_t)m * d + t] - cb[(size_t)c * d + t];
+                const float sq = diff * diff;
+                dist = dist + sq;
+            }
+            if (c == 0 || dist < best_d) {
+                best = c;
+                best_d = dist;
+            }
+        }
+        idx_out[m] = best;
+    }
+    return 0;
+}
+
+/*
+ * K-means update: centroid c of codebook g becomes the mean (in double,
+ * rounded once to float) of the vectors assigned to it; a centroid with no
+ * vector keeps its old value.  counts_out[g][c] (optional) receives the
+ * cluster sizes.
+ */
+int vq_oracle_kmeans_update(const float *v, int64_t M, int d, const int32_t *idx, int ncent,
+                            int64_t vecs_per_cb, const float *old_cent, float *new_cent,
+                            int64_t *counts_out)
+{
+    if (!v || !idx || !old_cent || !new_cent || M < 0 || d <= 0 || ncent <= 0 || vecs_per_cb < 0)
+        return -1;
+    const int64_t G = vecs_per_cb ? (M + vecs_per_cb - 1) / vecs_per_cb : 1;
+    double *sum = calloc((size_t)G * ncent * d, sizeof(double));
+    int64_t *cnt = calloc((size_t)G * ncent, sizeof(int64_t));
+    if (!sum || !cnt) { free(sum); free(cnt); return -2; }
+    for (int64_t m = 0; m < M; ++m) {
+        const int64_t g = vecs_per_cb ? m / vecs_per_cb : 0;
+        const int c = idx[m];
+        if (c < 0 || c >= ncent) { free(sum); free(cnt); return -1; }
+        cnt[g * ncent + c] += 1;
+        for (int t = 0; t < d; ++t) sum[((size_t)g * ncent + c) * d + t] += (double)v[(size_t)m * d + t];
+    }
+    for (int64_t gc = 0; gc < G * ncent; ++gc) {
+        for (int t = 0; t < d; ++t)
+            new_cent[(size_t)gc * d + t] = cnt[gc] ? (float)(sum[(size_t)gc * d + t] / (double)cnt[gc])
+                                                   : old_cent[(size_t)gc * d + t];
+        if (counts_out) counts_out[gc] = cnt[gc];
+    }
+    free(sum); free(cnt);
+    return 0;
+}
+
+/*
+ * Residual, signs and scales of a quantized rotated weight.  wrot: fp32
+ * [N][K]; wc: fp16 [G][ncent][d]; wi: u8 [N][K/d]; row o uses codebook
+ * o / codebook_rows (0: one codebook).  The residual is
+ * r = wrot - codebook[pointer] evaluated in float (one rounding); its sign
+ * bit is set for r >= 0 (a zero residual counts as +1) and stored LSB-first
+ * along k (bit i of byte m is k = 8m + i, signs_out [N][K/8]).  alpha_out
+ * [N][K/group] (double) is the optimal scale of each group of `group`
+ * consecutive k: mean |r|, summed in double.
+ */
+int vq_oracle_residual(const float *wrot, int N, int K, int d, const uint16_t *wc, int ncent,
+                       const uint8_t *wi, int codebook_rows, int group, uint8_t *signs_out,
+                       double *alpha_out)
+{
+    if (!wrot || !wc || !wi || !signs_out || !alpha_out || N <= 0 || K <= 0 || d <= 0 || K % d ||
+        K % 8 || group <= 0 || K % group || (codebook_rows && N % codebook_rows))
+        return -1;
+    const int J = K / d;
+    memset(signs_out, 0, (size_t)N * (K / 8));
+    for (int o = 0; o < N; ++o) {
+        const int g = codebook_rows ? o / codebook_rows : 0;
+        for (int q = 0; q < K / group; ++q) {
+            double acc = 0.0;
+            for (int k = q * group; k < (q + 1) * group; ++k) {
+                const int c = wi[(size_t)o * J + k / d];
+                if (c >= ncent) return -1;
+                const float cv = (float)vq_oracle_f16_to_f64(wc[((size_t)g * ncent + c) * d + k % d]);
+                const float r = wrot[(size_t)o * K + k] - cv;
+                if (r >= 0.f) signs_out[(size_t)o * (K / 8) + k / 8] |= (uint8_t)(1u << (k % 8));
+                acc += fabs((double)r);
+            }
+            alpha_out[(size_t)o * (K / group) + q] = acc / (double)group;
+        }
+    }
     return 0;
 }
 

@@ -297,10 +297,106 @@ def pin_optimal_alpha(orc, seed=12):
         assert loss(a + eps) > base
 
 
+# ------------------------------------------------------------- quantizer
+
+def pin_kmeans_assign_scipy(orc, seed=13):
+    """Nearest-centroid indices against scipy.cluster.vq.vq, one shared and two
+    per-group codebooks; a duplicated centroid never wins over its first copy."""
+    import scipy.cluster.vq
+    rng = np.random.default_rng(seed)
+    v = rng.normal(size=(6000, 4)).astype(np.float32)
+    c = rng.normal(size=(64, 4)).astype(np.float32)
+    ref, _ = scipy.cluster.vq.vq(v, c)
+    assert np.array_equal(orc.kmeans_assign(v, c), ref)
+    c2 = rng.normal(size=(2, 64, 4)).astype(np.float32)
+    got = orc.kmeans_assign(v, c2, vecs_per_cb=3000)
+    assert np.array_equal(got[:3000], scipy.cluster.vq.vq(v[:3000], c2[0])[0])
+    assert np.array_equal(got[3000:], scipy.cluster.vq.vq(v[3000:], c2[1])[0])
+    cd = np.concatenate([c, c[:8]])                # centroids 64..71 repeat 0..7
+    assert orc.kmeans_assign(v, cd).max() < 64
+
+
+def pin_kmeans_sklearn(orc, seed=14):
+    """Lloyd iterations from the same start agree with scikit-learn's KMeans on
+    well-separated blobs (labels exactly, centroids to float rounding)."""
+    from sklearn.cluster import KMeans
+    rng = np.random.default_rng(seed)
+    centres = rng.uniform(-8, 8, size=(24, 4))
+    lab = rng.integers(0, 24, size=4000)
+    v = (centres[lab] + rng.normal(0, 0.6, size=(4000, 4))).astype(np.float32)
+    init = (centres + rng.normal(0, 0.8, size=centres.shape)).astype(np.float32)
+    cent = init[None]
+    for _ in range(6):
+        idx = orc.kmeans_assign(v, cent)
+        cent, counts = orc.kmeans_update(v, idx, cent)
+    assert counts.min() > 0
+    km = KMeans(n_clusters=24, init=init, n_init=1, max_iter=6, tol=0.0, algorithm="lloyd").fit(v)
+    assert np.allclose(cent[0], km.cluster_centers_, rtol=1e-5, atol=1e-5)
+    assert np.array_equal(orc.kmeans_assign(v, cent), km.predict(v))
+
+
+def pin_quantize_exact_recovery(orc, seed=15):
+    """A weight that IS a codebook reconstruction (fp16-exact, well-separated
+    centroids) comes back exactly: same codebook and pointers, zero residual
+    (every sign bit set: a zero residual counts as +1) and zero alpha.  A
+    centroid no vector is near keeps its start value."""
+    rng = np.random.default_rng(seed)
+    ncent, N, K = 16, 32, 256
+    wc_true = (rng.integers(-6, 7, size=(ncent, 4)) * 0.25).astype(np.float16)
+    wc_true[:, 0] = np.arange(ncent) * 0.5          # rows distinct, far apart
+    wi_true = rng.integers(0, ncent - 1, size=(N, K // 4)).astype(np.uint8)   # last centroid unused
+    w = wc_true[wi_true].reshape(N, K)
+    init = wc_true.astype(np.float32) + rng.uniform(-0.05, 0.05, size=wc_true.shape).astype(np.float32)
+    init[-1] = [100, 100, 100, 100]
+    wc, wi, signs, alpha, _ = orc.quantize(w, init, iters=3)
+    assert np.array_equal(wc[0, :-1], wc_true[:-1])
+    assert np.array_equal(wc[0, -1].astype(np.float32), init[-1])
+    assert np.array_equal(wi, wi_true)
+    assert np.all(signs == 0xFF) and np.all(alpha == 0)
+
+
+def pin_quantize_rotation(orc, seed=16):
+    """W_rot = W Q pairs with x~ = Q^T x: W_rot x~ = W x (Q orthogonal)."""
+    rng = np.random.default_rng(seed)
+    N, K, b = 8, 1024, 256
+    w = rng.normal(0, 0.5, size=(N, K)).astype(np.float16)
+    hs = rng.choice([-1, 1], size=K).astype(np.int8)
+    x = rng.normal(size=(1, K)).astype(np.float16)
+    init = rng.normal(0, 0.5, size=(256, 4)).astype(np.float32)
+    *_, wrot = orc.quantize(w, init, iters=1, hsign=hs, hadamard_block=b)
+    lhs = wrot.astype(np.float64) @ orc.hadamard(x, hs, b)[0]
+    rhs = w.astype(np.float64) @ x[0].astype(np.float64)
+    assert np.allclose(lhs, rhs, rtol=1e-5, atol=1e-4), np.abs(lhs - rhs).max()
+
+
+def pin_residual_identity(orc, seed=17):
+    """Per group, with alpha = mean|r| and the packed signs of r (bits decoded
+    by numpy, LSB first): ||r - alpha s||^2 = ||r||^2 - G alpha^2, which holds
+    only when s . r = sum |r|; also for per-group codebooks."""
+    rng = np.random.default_rng(seed)
+    N, K, G = 32, 512, 128
+    wrot = rng.normal(0, 0.05, size=(N, K)).astype(np.float32)
+    for cbr in (0, 16):
+        ncb = N // cbr if cbr else 1
+        wc = rng.normal(0, 0.05, size=(ncb, 256, 4)).astype(np.float16)
+        wi = rng.integers(0, 256, size=(N, K // 4)).astype(np.uint8)
+        signs, alpha = orc.residual(wrot, wc, wi, codebook_rows=cbr, group=G)
+        g = (np.arange(N) // cbr) if cbr else np.zeros(N, int)
+        rec = wc.astype(np.float64)[g[:, None], wi].reshape(N, K)
+        r = wrot.astype(np.float64) - rec
+        s = np.unpackbits(signs, axis=1, bitorder="little").astype(np.float64) * 2 - 1
+        a = np.repeat(alpha, G, axis=1)
+        lhs = ((r - a * s) ** 2).reshape(N, K // G, G).sum(axis=2)
+        rhs = (r ** 2).reshape(N, K // G, G).sum(axis=2) - G * alpha ** 2
+        assert np.allclose(lhs, rhs, rtol=1e-6, atol=1e-12), np.abs(lhs - rhs).max()
+        assert np.all(alpha >= 0)
+
+
 ALL_PINS = [
     pin_golden_vq, pin_golden_residual, pin_golden_hadamard, pin_f16_decode,
     pin_hadamard_scipy, pin_factorisation, pin_factorisation_residual, pin_rotation_composite,
     pin_unit_centroids, pin_all_equal_indices, pin_group_scaling, pin_residual_popcount,
     pin_residual_unit_inputs, pin_hadamard_orthogonal, pin_lookup_identity, pin_batch_rows,
-    pin_optimal_alpha,
+    pin_optimal_alpha, pin_kmeans_assign_scipy, pin_kmeans_sklearn, pin_quantize_exact_recovery,
+    pin_quantize_rotation, pin_residual_identity,
 ]

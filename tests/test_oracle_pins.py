@@ -64,6 +64,18 @@ MUTATIONS = {
     "f16_exponent_bias": ("expo - 25)", "expo - 24)"),
     "f16_subnormal_scale": ("ldexp((double)mant, -24)", "ldexp((double)mant, -25)"),
     "alpha_not_mean": ("num += v * s;", "num += v * v;"),
+    "kmeans_tie_to_last": ("if (c == 0 || dist < best_d) {", "if (c == 0 || dist <= best_d) {"),
+    "kmeans_component_dropped": ("            for (int t = 0; t < d; ++t) {\n                const float diff",
+                                 "            for (int t = 1; t < d; ++t) {\n                const float diff"),
+    "kmeans_mean_off_by_one": ("/ (double)cnt[gc])", "/ (double)(cnt[gc] + 1))"),
+    "kmeans_empty_zeroed": (": old_cent[(size_t)gc * d + t];", ": 0.f;"),
+    "kmeans_codebook_modulo": ("const int64_t g = vecs_per_cb ? m / vecs_per_cb : 0;\n        const float *cb",
+                               "const int64_t g = vecs_per_cb ? m % 2 : 0;\n        const float *cb"),
+    "residual_zero_negative": ("if (r >= 0.f)", "if (r > 0.f)"),
+    "residual_msb_first": ("(uint8_t)(1u << (k % 8))", "(uint8_t)(1u << (7 - k % 8))"),
+    "residual_alpha_rms": ("acc += fabs((double)r);", "acc += (double)r * (double)r;"),
+    "residual_codebook_modulo": ("const int g = codebook_rows ? o / codebook_rows : 0;\n        for (int q",
+                                 "const int g = codebook_rows ? o % (N / codebook_rows) : 0;\n        for (int q"),
 }
 
 

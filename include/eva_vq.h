@@ -225,6 +225,87 @@ typedef struct {
 /* Sizes and launch shape of a handle (host only, no device work). */
 EVA_API eva_status_t eva_vq_linear_info(eva_vq_linear_t h, eva_vq_info *info);
 
+/* ------------------------------------------------------------------------
+ * Offline quantizer: the quantize() sample of the 3-bit SRAM-lookup article
+ * ("section details"), run on the GPU.  Steps, in the sample's order:
+ *   1. W_rot = W Q, Q = blockdiag(H_b) diag(s) / sqrt(b) -- each row gets the
+ *      transform the layer applies to x (hadamard_block = 0: W_rot = W);
+ *   2. blocks of d = 4 along each row;
+ *   3. K-means: plain Lloyd iterations (the sample's sensitivity weighting
+ *      needs calibration data the pages do not give) from starting centroids
+ *      the caller chooses as blocks of W_rot; the codebook is stored in fp16
+ *      and the pointers are the nearest fp16 centroids;
+ *   4.-7. residual r = W_rot - codebook[pointer], its 1-bit signs packed
+ *      LSB-first along k (a zero residual counts as +1) and the optimal scale
+ *      per group, alpha = mean |r| (fp16).
+ * The outputs are exactly what eva_vq_linear_create takes (wc, wi, signs,
+ * alpha, with the same hsign and hadamard_block).
+ * ---------------------------------------------------------------------- */
+typedef struct {
+    int32_t N;               /* rows of W (output features), >= 1                      */
+    int32_t K;               /* columns of W, multiple of 4 (of 8 with a residual)     */
+    int32_t d;               /* block length; 4 is the only supported value            */
+    int32_t index_bits;      /* 1..8: 2^index_bits centroids per codebook              */
+    int32_t codebook_rows;   /* 0: one codebook; else rows per codebook (divides N)    */
+    int32_t residual_group;  /* 0: no residual; else a multiple of 8 dividing K (128)  */
+    int32_t hadamard_block;  /* 0: no rotation; b: power of two in [8, 4096] dividing K */
+    int32_t iters;           /* Lloyd iterations, >= 0                                 */
+} eva_quant_desc;
+
+/*
+ * Quantize W (device fp16 [N][K]).  hsign: device int8 [K] in {-1, +1}
+ * (required iff hadamard_block != 0).  init_index: device int32 [G][2^n]:
+ * codebook g's centroid c starts as block init_index[g][c] of the codebook's
+ * blocks (block m of codebook g is W_rot row g * codebook_rows + m / (K/4),
+ * inputs 4 (m mod K/4) ..; G = N / codebook_rows, or 1); an index out of
+ * range gives EVA_ERR_INVALID_ARG.  Outputs (device, caller-owned): wc_out fp16
+ * [G][2^n][4]; wi_out u8 [N][K/4]; signs_out u8 [N][K/8] and alpha_out fp16
+ * [N][K/residual_group] (required iff residual_group != 0).  Optional:
+ * wrot_out fp32 [N][K] (the rotated rows; also used as the working buffer
+ * when given) and cent_out fp32 [G][2^n][4] (the centroids after the last
+ * iteration, before rounding to fp16).  Work buffers are allocated on
+ * `stream` (stream-ordered) and freed before return; the call synchronises
+ * `stream` before it returns.
+ */
+EVA_API eva_status_t eva_vq_quantize(const eva_quant_desc *desc, const void *w, const int8_t *hsign,
+                                     const int32_t *init_index, void *wc_out, uint8_t *wi_out,
+                                     uint8_t *signs_out, void *alpha_out, float *wrot_out, float *cent_out,
+                                     eva_stream_t stream);
+
+/*
+ * The K-means steps on their own (asynchronous on `stream`).  v: device fp32
+ * [M][d] (16-byte aligned), d = 4; centroids: device fp32 [G][ncent][d],
+ * 1 <= ncent <= 256; block m belongs to codebook m / vecs_per_cb
+ * (vecs_per_cb = 0: one codebook, G = 1).
+ * assign: idx_out[m] = the nearest centroid, the squared distance summed in
+ * fp32 one component at a time (no fused multiply-add), the first minimum
+ * winning -- bit-exact with the decision rule the oracle states.
+ */
+EVA_API eva_status_t eva_vq_kmeans_assign(const float *v, int64_t M, int32_t d, const float *centroids,
+                                          int32_t ncent, int64_t vecs_per_cb, int32_t *idx_out,
+                                          eva_stream_t stream);
+
+/*
+ * update: new_out[g][c] = mean of the blocks assigned to c (double sums,
+ * one rounding to fp32); a centroid with no block keeps old[g][c].  new_out
+ * may equal old.  counts_out (optional) int64 [G][ncent].  Allocates its
+ * sums on `stream` (stream-ordered) and frees them before returning.
+ */
+EVA_API eva_status_t eva_vq_kmeans_update(const float *v, int64_t M, int32_t d, const int32_t *idx,
+                                          int32_t ncent, int64_t vecs_per_cb, const float *old,
+                                          float *new_out, int64_t *counts_out, eva_stream_t stream);
+
+/*
+ * residual: for wrot (device fp32 [N][K]), wc (device fp16 [G][ncent][4]) and
+ * wi (device u8 [N][K/4], row o using codebook o / codebook_rows): the packed
+ * signs of r = wrot - wc[wi] (fp32, bit set for r >= 0, LSB-first, device u8
+ * [N][K/8]) and alpha = mean |r| per group of `group` inputs (double sum,
+ * rounded to fp16, device [N][K/group]).  group: a multiple of 8 dividing K.
+ */
+EVA_API eva_status_t eva_vq_residual(const float *wrot, int32_t N, int32_t K, const void *wc, int32_t ncent,
+                                     const uint8_t *wi, int32_t codebook_rows, int32_t group,
+                                     uint8_t *signs_out, void *alpha_out, eva_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

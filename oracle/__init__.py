@@ -228,7 +228,7 @@ def residual(wrot, wc, wi, *, codebook_rows: int = 0, group: int = 128):
 
 
 def quantize(w, init_centroids, iters: int, *, hsign=None, hadamard_block: int = 0, codebook_rows: int = 0,
-             group: int = 128, d: int = 4):
+             group: int = 128, d: int = 4, init_index=None):
     """The 3-bit article's quantize() pipeline, step by step (plain K-means):
     1. W_rot = W Q (rows rotated like x~, dense per-block product, then fp32);
     2. blocks of d along each row; 3. `iters` Lloyd iterations from
@@ -245,7 +245,12 @@ def quantize(w, init_centroids, iters: int, *, hsign=None, hadamard_block: int =
         wrot = f16_to_f64(w16).astype(np.float32)
     v = wrot.reshape(N * (K // d), d)
     vecs_per_cb = codebook_rows * (K // d) if codebook_rows else 0
-    cent = np.ascontiguousarray(init_centroids, dtype=np.float32)
+    if init_index is not None:      # starting centroids = chosen blocks of each codebook's rows
+        ii = np.asarray(init_index, dtype=np.int64)
+        per = vecs_per_cb or v.shape[0]
+        cent = np.stack([v[g * per + ii[g]] for g in range(ii.shape[0])]).astype(np.float32)
+    else:
+        cent = np.ascontiguousarray(init_centroids, dtype=np.float32)
     if cent.ndim == 2:
         cent = cent[None]
     for _ in range(int(iters)):

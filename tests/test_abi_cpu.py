@@ -112,3 +112,43 @@ def test_lookup_kernels_do_not_spill():
     assert len(blocks) == 16, out
     for name, stack, st, ld in blocks:
         assert (stack, st, ld) == ("0", "0", "0"), (name, stack, st, ld)
+
+
+def _qdesc(**kw):
+    base = dict(N=64, K=256, d=4, index_bits=8, codebook_rows=0, residual_group=128, hadamard_block=0, iters=2)
+    base.update(kw)
+    return eva_vq.eva_quant_desc(*[base[f] for f, _ in eva_vq.eva_quant_desc._fields_])
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(d=8), eva_vq.EVA_ERR_UNSUPPORTED),
+    (dict(index_bits=9), eva_vq.EVA_ERR_UNSUPPORTED),
+    (dict(N=0), eva_vq.EVA_ERR_INVALID_ARG),
+    (dict(K=258), eva_vq.EVA_ERR_INVALID_ARG),
+    (dict(codebook_rows=48), eva_vq.EVA_ERR_INVALID_ARG),      # does not divide N
+    (dict(residual_group=100), eva_vq.EVA_ERR_INVALID_ARG),
+    (dict(hadamard_block=96), eva_vq.EVA_ERR_INVALID_ARG),     # not a power of two
+    (dict(iters=-1), eva_vq.EVA_ERR_INVALID_ARG),
+])
+def test_quantize_rejects_bad_descriptor(kw, expect):
+    lib = eva_vq.load()
+    d = _qdesc(**kw)
+    rc = lib.eva_vq_quantize(ctypes.byref(d), 0x1000, None, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, None, None, None)
+    assert rc == expect
+
+
+def test_quantize_and_steps_reject_bad_pointers():
+    lib = eva_vq.load()
+    d = _qdesc()
+    P = 0x1000
+    assert lib.eva_vq_quantize(None, P, None, P, P, P, P, P, None, None, None) == eva_vq.EVA_ERR_INVALID_ARG
+    assert lib.eva_vq_quantize(ctypes.byref(d), P, None, P, P, P, None, None, None, None, None) == \
+        eva_vq.EVA_ERR_INVALID_ARG                                   # residual without outputs
+    assert lib.eva_vq_quantize(ctypes.byref(d), P, 0x7000, P, P, P, P, P, None, None, None) == \
+        eva_vq.EVA_ERR_INVALID_ARG                                   # signs s without a rotation
+    assert lib.eva_vq_kmeans_assign(P, 10, 3, P, 256, 0, P, None) == eva_vq.EVA_ERR_UNSUPPORTED
+    assert lib.eva_vq_kmeans_assign(P + 4, 10, 4, P, 256, 0, P, None) == eva_vq.EVA_ERR_INVALID_ARG
+    assert lib.eva_vq_kmeans_assign(P, 10, 4, P, 257, 0, P, None) == eva_vq.EVA_ERR_INVALID_ARG
+    assert lib.eva_vq_kmeans_update(P, 10, 4, None, 256, 0, P, P, None, None) == eva_vq.EVA_ERR_INVALID_ARG
+    assert lib.eva_vq_residual(P, 4, 256, P, 256, P, 0, 100, P, P, None) == eva_vq.EVA_ERR_INVALID_ARG
+    assert lib.eva_vq_residual(P, 4, 256, P, 256, P, 3, 128, P, P, None) == eva_vq.EVA_ERR_INVALID_ARG

@@ -18,6 +18,7 @@
 
 #include "../../include/eva_vq.h"
 #include "eva_vq_kernels.cuh"
+#include "eva_vq_quant.cuh"
 
 using namespace eva;
 
@@ -639,6 +640,209 @@ eva_status_t eva_vq_linear_info(eva_vq_linear_t h, eva_vq_info *info) {
     info->path = h->last_path ? h->last_path : EVA_PATH_OC_LOOKUP;
     info->sm_count = h->sm_count;
     return EVA_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Offline quantizer (3-bit SRAM-lookup article, quantize() sample).
+namespace {
+
+bool aligned16c(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+eva_status_t kmeans_args(const float *v, int64_t M, int32_t d, const float *cent, int32_t ncent,
+                         int64_t vecs_per_cb) {
+    if (d != 4) return EVA_ERR_UNSUPPORTED;
+    if (!v || !cent || M < 0 || ncent < 1 || ncent > kMaxCent || vecs_per_cb < 0) return EVA_ERR_INVALID_ARG;
+    if (!aligned16c(v) || !aligned16c(cent)) return EVA_ERR_INVALID_ARG;
+    const int64_t G = vecs_per_cb ? (M + vecs_per_cb - 1) / vecs_per_cb : 1;
+    if (G > 65535) return EVA_ERR_INVALID_ARG;
+    return EVA_OK;
+}
+
+int64_t codebooks_of(int64_t M, int64_t vecs_per_cb) {
+    return vecs_per_cb ? std::max<int64_t>(1, (M + vecs_per_cb - 1) / vecs_per_cb) : 1;
+}
+
+template <typename IdxT>
+cudaError_t launch_assign(const float *v, int64_t M, const float *cent, int ncent, int64_t vecs_per_cb,
+                          IdxT *idx, cudaStream_t s) {
+    if (M == 0) return cudaSuccess;
+    const int64_t G = codebooks_of(M, vecs_per_cb);
+    const int64_t per = vecs_per_cb ? vecs_per_cb : M;
+    const int64_t bx = std::min<int64_t>(std::max<int64_t>(1, (per + 4 * kQThreads - 1) / (4 * kQThreads)), 2048);
+    eva_kmeans_assign_kernel<IdxT><<<dim3((unsigned)bx, (unsigned)G), kQThreads, 0, s>>>(
+        reinterpret_cast<const float4 *>(v), M, reinterpret_cast<const float4 *>(cent), ncent,
+        vecs_per_cb ? vecs_per_cb : M, idx);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_update(const float *v, int64_t M, const int32_t *idx, int ncent, int64_t vecs_per_cb,
+                          const float *old, float *out, int64_t *counts_out, double *sums,
+                          unsigned long long *counts, cudaStream_t s) {
+    const int64_t G = codebooks_of(M, vecs_per_cb);
+    const int n = (int)(G * ncent);
+    cudaError_t e = cudaMemsetAsync(sums, 0, (size_t)n * 4 * sizeof(double), s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(counts, 0, (size_t)n * sizeof(unsigned long long), s);
+    if (e != cudaSuccess) return e;
+    if (M > 0) {
+        const int64_t per = vecs_per_cb ? vecs_per_cb : M;
+        const int64_t bx = std::min<int64_t>(std::max<int64_t>(1, (per + kQThreads - 1) / kQThreads), 592);
+        eva_kmeans_accum_kernel<<<dim3((unsigned)bx, (unsigned)G), kQThreads, 0, s>>>(
+            reinterpret_cast<const float4 *>(v), M, idx, ncent, vecs_per_cb ? vecs_per_cb : M, sums, counts);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    eva_kmeans_finish_kernel<<<blocks_for(n, 256), 256, 0, s>>>(sums, counts, old, out,
+                                                                 reinterpret_cast<long long *>(counts_out), n);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_residual(const float *wrot, int N, int K, const __half *wc, int ncent, const uint8_t *wi,
+                            int codebook_rows, int group, uint8_t *signs, __half *alpha, cudaStream_t s) {
+    const long long warps = (long long)N * (K / group);
+    const long long threads = warps * 32;
+    eva_residual_kernel<<<(unsigned)((threads + kQThreads - 1) / kQThreads), kQThreads, 0, s>>>(
+        reinterpret_cast<const float4 *>(wrot), N, K, wc, ncent, wi, codebook_rows, group, signs, alpha);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+extern "C" {
+
+eva_status_t eva_vq_kmeans_assign(const float *v, int64_t M, int32_t d, const float *centroids, int32_t ncent,
+                                  int64_t vecs_per_cb, int32_t *idx_out, eva_stream_t stream) {
+    const eva_status_t st = kmeans_args(v, M, d, centroids, ncent, vecs_per_cb);
+    if (st != EVA_OK) return st;
+    if (!idx_out) return EVA_ERR_INVALID_ARG;
+    return cuda_status(launch_assign(v, M, centroids, ncent, vecs_per_cb, idx_out,
+                                     reinterpret_cast<cudaStream_t>(stream)));
+}
+
+eva_status_t eva_vq_kmeans_update(const float *v, int64_t M, int32_t d, const int32_t *idx, int32_t ncent,
+                                  int64_t vecs_per_cb, const float *old, float *new_out, int64_t *counts_out,
+                                  eva_stream_t stream) {
+    const eva_status_t st = kmeans_args(v, M, d, old, ncent, vecs_per_cb);
+    if (st != EVA_OK) return st;
+    if (!idx || !new_out) return EVA_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t n = codebooks_of(M, vecs_per_cb) * ncent;
+    double *sums = nullptr;
+    cudaError_t e = cudaMallocAsync(reinterpret_cast<void **>(&sums),
+                                    (size_t)n * (4 * sizeof(double) + sizeof(unsigned long long)), s);
+    if (e != cudaSuccess) return e == cudaErrorMemoryAllocation ? EVA_ERR_OOM : cuda_status(e);
+    e = launch_update(v, M, idx, ncent, vecs_per_cb, old, new_out, counts_out, sums,
+                      reinterpret_cast<unsigned long long *>(sums + 4 * n), s);
+    const cudaError_t ef = cudaFreeAsync(sums, s);
+    return cuda_status(e != cudaSuccess ? e : ef);
+}
+
+eva_status_t eva_vq_residual(const float *wrot, int32_t N, int32_t K, const void *wc, int32_t ncent,
+                             const uint8_t *wi, int32_t codebook_rows, int32_t group, uint8_t *signs_out,
+                             void *alpha_out, eva_stream_t stream) {
+    if (!wrot || !wc || !wi || !signs_out || !alpha_out || !aligned16c(wrot)) return EVA_ERR_INVALID_ARG;
+    if (N < 1 || K < 8 || K % 8 || ncent < 1 || ncent > kMaxCent || group < 8 || group % 8 || K % group)
+        return EVA_ERR_INVALID_ARG;
+    if (codebook_rows < 0 || (codebook_rows && N % codebook_rows)) return EVA_ERR_INVALID_ARG;
+    return cuda_status(launch_residual(wrot, N, K, reinterpret_cast<const __half *>(wc), ncent, wi, codebook_rows,
+                                       group, signs_out, reinterpret_cast<__half *>(alpha_out),
+                                       reinterpret_cast<cudaStream_t>(stream)));
+}
+
+eva_status_t eva_vq_quantize(const eva_quant_desc *desc, const void *w, const int8_t *hsign,
+                             const int32_t *init_index, void *wc_out, uint8_t *wi_out, uint8_t *signs_out,
+                             void *alpha_out, float *wrot_out, float *cent_out, eva_stream_t stream) {
+    if (!desc) return EVA_ERR_INVALID_ARG;
+    const eva_quant_desc &d = *desc;
+    if (d.d != 4) return EVA_ERR_UNSUPPORTED;
+    if (d.index_bits < 1 || d.index_bits > 8) return EVA_ERR_UNSUPPORTED;
+    if (d.N < 1 || d.K < 4 || d.K % 4 || d.iters < 0) return EVA_ERR_INVALID_ARG;
+    if (d.codebook_rows < 0 || (d.codebook_rows && d.N % d.codebook_rows)) return EVA_ERR_INVALID_ARG;
+    if (d.residual_group && (d.residual_group < 8 || d.residual_group % 8 || d.K % d.residual_group))
+        return EVA_ERR_INVALID_ARG;
+    if (d.hadamard_block) {
+        const int b = d.hadamard_block;
+        if (b < 8 || b > 4096 || (b & (b - 1)) || d.K % b || !hsign) return EVA_ERR_INVALID_ARG;
+    } else if (hsign) {
+        return EVA_ERR_INVALID_ARG;
+    }
+    if (!w || !init_index || !wc_out || !wi_out) return EVA_ERR_INVALID_ARG;
+    if (d.residual_group ? (!signs_out || !alpha_out) : (signs_out || alpha_out)) return EVA_ERR_INVALID_ARG;
+    if (wrot_out && !aligned16c(wrot_out)) return EVA_ERR_INVALID_ARG;
+    if (cent_out && !aligned16c(cent_out)) return EVA_ERR_INVALID_ARG;
+    const int ncent = 1 << d.index_bits;
+    const int64_t N = d.N, K = d.K, J = K / 4, M = N * J;
+    const int64_t vpc = d.codebook_rows ? (int64_t)d.codebook_rows * J : 0;
+    const int64_t G = d.codebook_rows ? N / d.codebook_rows : 1;
+    if (G > 65535) return EVA_ERR_INVALID_ARG;
+    const int64_t nc = G * ncent;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+    // Work buffers, one stream-ordered allocation: [wrot][cent][cent16][sums][counts][idx][err].
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    const size_t b_wrot = wrot_out ? 0 : up((size_t)M * 16), b_cent = up((size_t)nc * 16);
+    const size_t b_sums = up((size_t)nc * 32), b_cnt = up((size_t)nc * 8), b_idx = up((size_t)M * 4);
+    const size_t total = b_wrot + 2 * b_cent + b_sums + b_cnt + b_idx + 256;
+    uint8_t *ws = nullptr;
+    cudaError_t e = cudaMallocAsync(reinterpret_cast<void **>(&ws), total, s);
+    if (e != cudaSuccess) return e == cudaErrorMemoryAllocation ? EVA_ERR_OOM : cuda_status(e);
+    uint8_t *q = ws;
+    float *wrot = wrot_out ? wrot_out : reinterpret_cast<float *>(q);
+    q += b_wrot;
+    float *cent = reinterpret_cast<float *>(q);
+    q += b_cent;
+    float *cent16 = reinterpret_cast<float *>(q);
+    q += b_cent;
+    double *sums = reinterpret_cast<double *>(q);
+    q += b_sums;
+    unsigned long long *counts = reinterpret_cast<unsigned long long *>(q);
+    q += b_cnt;
+    int32_t *idx = reinterpret_cast<int32_t *>(q);
+    q += b_idx;
+    int *err = reinterpret_cast<int *>(q);
+    auto chk = [&](cudaError_t r) { if (e == cudaSuccess) e = r; };
+    chk(cudaMemsetAsync(err, 0, sizeof(int), s));
+
+    // 1. W_rot = W Q (rows rotated like x~), or W in fp32.
+    if (d.hadamard_block) {
+        const int b = d.hadamard_block, thr = std::min(b / 2, 1024);
+        for (int64_t r0 = 0; r0 < N && e == cudaSuccess; r0 += 65535) {
+            const int rows = (int)std::min<int64_t>(65535, N - r0);
+            eva_hadamard_kernel<<<dim3((unsigned)(K / b), (unsigned)rows), thr, (size_t)b * sizeof(float), s>>>(
+                reinterpret_cast<const __half *>(w) + r0 * K, hsign, wrot + r0 * K, (int)K, b,
+                (float)(1.0 / std::sqrt((double)b)), 1);
+            chk(cudaGetLastError());
+        }
+    } else {
+        eva_rows_to_f32_kernel<<<(unsigned)std::min<int64_t>(blocks_for(N * K, 256), 4096), 256, 0, s>>>(
+            reinterpret_cast<const __half *>(w), wrot, N * K);
+        chk(cudaGetLastError());
+    }
+    // 2.-3. blocks of 4, starting centroids, Lloyd iterations.
+    eva_gather_init_kernel<<<blocks_for(nc, 256), 256, 0, s>>>(
+        reinterpret_cast<const float4 *>(wrot), M, init_index, ncent, vpc ? vpc : M, (int)G,
+        reinterpret_cast<float4 *>(cent), err);
+    chk(cudaGetLastError());
+    for (int it = 0; it < d.iters && e == cudaSuccess; ++it) {
+        chk(launch_assign(wrot, M, cent, ncent, vpc, idx, s));
+        chk(launch_update(wrot, M, idx, ncent, vpc, cent, cent, nullptr, sums, counts, s));
+    }
+    if (cent_out) chk(cudaMemcpyAsync(cent_out, cent, (size_t)nc * 16, cudaMemcpyDeviceToDevice, s));
+    // fp16 codebook; pointers = nearest fp16 centroids.
+    eva_centroids_to_f16_kernel<<<blocks_for(nc * 4, 256), 256, 0, s>>>(cent, reinterpret_cast<__half *>(wc_out),
+                                                                        cent16, (int)(nc * 4));
+    chk(cudaGetLastError());
+    chk(launch_assign(wrot, M, cent16, ncent, vpc, wi_out, s));
+    // 4.-7. residual signs and scales.
+    if (d.residual_group)
+        chk(launch_residual(wrot, (int)N, (int)K, reinterpret_cast<const __half *>(wc_out), ncent, wi_out,
+                            d.codebook_rows, d.residual_group, signs_out, reinterpret_cast<__half *>(alpha_out), s));
+    int herr = 0;
+    chk(cudaMemcpyAsync(&herr, err, sizeof(int), cudaMemcpyDeviceToHost, s));
+    chk(cudaFreeAsync(ws, s));
+    chk(cudaStreamSynchronize(s));
+    if (e != cudaSuccess) return cuda_status(e);
+    return herr ? EVA_ERR_INVALID_ARG : EVA_OK;
 }
 
 }  // extern "C"

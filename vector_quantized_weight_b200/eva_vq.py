@@ -25,6 +25,7 @@ ABI_FUNCTIONS = (
     "eva_vq_linear_destroy", "eva_vq_unpack_indices", "eva_vq_sync_status",
     "eva_vq_status_string", "eva_vq_linear_info", "eva_vq_device_check_record",
     "eva_vq_debug_timeline", "eva_vq_linear_run_noalloc",
+    "eva_vq_quantize", "eva_vq_kmeans_assign", "eva_vq_kmeans_update", "eva_vq_residual",
 )
 
 
@@ -41,6 +42,13 @@ class eva_vq_desc(ctypes.Structure):
                 ("residual_group", ctypes.c_int32), ("hadamard_block", ctypes.c_int32),
                 ("max_batch", ctypes.c_int32), ("out_dtype", ctypes.c_int),
                 ("path", ctypes.c_int)]
+
+
+class eva_quant_desc(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int32), ("K", ctypes.c_int32), ("d", ctypes.c_int32),
+                ("index_bits", ctypes.c_int32), ("codebook_rows", ctypes.c_int32),
+                ("residual_group", ctypes.c_int32), ("hadamard_block", ctypes.c_int32),
+                ("iters", ctypes.c_int32)]
 
 
 class eva_vq_info(ctypes.Structure):
@@ -97,6 +105,11 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.eva_vq_linear_info.argtypes = [H, ctypes.POINTER(eva_vq_info)]
     lib.eva_vq_device_check_record.argtypes = [H, P]
     lib.eva_vq_debug_timeline.argtypes = [H, P, I32, ctypes.POINTER(I32)]
+    I64 = ctypes.c_int64
+    lib.eva_vq_quantize.argtypes = [ctypes.POINTER(eva_quant_desc), P, P, P, P, P, P, P, P, P, P]
+    lib.eva_vq_kmeans_assign.argtypes = [P, I64, I32, P, I32, I64, P, P]
+    lib.eva_vq_kmeans_update.argtypes = [P, I64, I32, P, I32, I64, P, P, P, P]
+    lib.eva_vq_residual.argtypes = [P, I32, I32, P, I32, P, I32, I32, P, P, P]
     for fn in ABI_FUNCTIONS:
         if fn != "eva_vq_status_string":
             getattr(lib, fn).restype = ctypes.c_int
@@ -172,6 +185,31 @@ def eva_vq_linear_info(h: int) -> eva_vq_info:
     info = eva_vq_info()
     _check("eva_vq_linear_info", load().eva_vq_linear_info(h, ctypes.byref(info)))
     return info
+
+
+def eva_vq_quantize(desc: eva_quant_desc, w: int, hsign: int | None, init_index: int, wc_out: int, wi_out: int,
+                    signs_out: int | None, alpha_out: int | None, wrot_out: int | None, cent_out: int | None,
+                    stream: int | None) -> None:
+    _check("eva_vq_quantize", load().eva_vq_quantize(ctypes.byref(desc), w, hsign, init_index, wc_out, wi_out,
+                                                     signs_out, alpha_out, wrot_out, cent_out, stream))
+
+
+def eva_vq_kmeans_assign(v: int, M: int, d: int, centroids: int, ncent: int, vecs_per_cb: int, idx_out: int,
+                         stream: int | None) -> None:
+    _check("eva_vq_kmeans_assign", load().eva_vq_kmeans_assign(v, int(M), int(d), centroids, int(ncent),
+                                                               int(vecs_per_cb), idx_out, stream))
+
+
+def eva_vq_kmeans_update(v: int, M: int, d: int, idx: int, ncent: int, vecs_per_cb: int, old: int, new_out: int,
+                         counts_out: int | None, stream: int | None) -> None:
+    _check("eva_vq_kmeans_update", load().eva_vq_kmeans_update(v, int(M), int(d), idx, int(ncent),
+                                                               int(vecs_per_cb), old, new_out, counts_out, stream))
+
+
+def eva_vq_residual(wrot: int, N: int, K: int, wc: int, ncent: int, wi: int, codebook_rows: int, group: int,
+                    signs_out: int, alpha_out: int, stream: int | None) -> None:
+    _check("eva_vq_residual", load().eva_vq_residual(wrot, int(N), int(K), wc, int(ncent), wi,
+                                                     int(codebook_rows), int(group), signs_out, alpha_out, stream))
 
 
 # ------------------------------------------------------- torch convenience
@@ -259,3 +297,31 @@ def from_layer(layer, *, max_batch=1, out_dtype="float16", path=EVA_PATH_AUTO, d
                     hsign=dev(layer.hsign), codebook_rows=s.codebook_rows,
                     residual_group=s.residual_group, hadamard_block=s.hadamard_block,
                     max_batch=max_batch, out_dtype=out_dtype, path=path)
+
+
+def quantize(w, init_index, iters: int, *, hsign=None, hadamard_block: int = 0, codebook_rows: int = 0,
+             residual_group: int = 128, index_bits: int = 8, keep_wrot: bool = False, keep_centroids: bool = False,
+             stream=None) -> dict:
+    """The offline quantizer on the GPU (eva_vq_quantize).  w: CUDA fp16
+    [N][K]; init_index: CUDA int32 [G][2^index_bits] starting blocks (see the
+    header).  Returns CUDA tensors wc, wi (and signs, alpha with a residual;
+    wrot, centroids on request) ready for VQLinear."""
+    import torch
+    N, K = w.shape
+    dev = w.device
+    G = N // codebook_rows if codebook_rows else 1
+    ncent = 1 << index_bits
+    out = {"wc": torch.empty((G, ncent, 4), dtype=torch.float16, device=dev),
+           "wi": torch.empty((N, K // 4), dtype=torch.uint8, device=dev)}
+    if residual_group:
+        out["signs"] = torch.empty((N, K // 8), dtype=torch.uint8, device=dev)
+        out["alpha"] = torch.empty((N, K // residual_group), dtype=torch.float16, device=dev)
+    if keep_wrot:
+        out["wrot"] = torch.empty((N, K), dtype=torch.float32, device=dev)
+    if keep_centroids:
+        out["centroids"] = torch.empty((G, ncent, 4), dtype=torch.float32, device=dev)
+    desc = eva_quant_desc(N, K, 4, index_bits, codebook_rows, residual_group, hadamard_block, iters)
+    eva_vq_quantize(desc, _ptr(w.contiguous()), _ptr(hsign), _ptr(init_index.contiguous()), _ptr(out["wc"]),
+                    _ptr(out["wi"]), _ptr(out.get("signs")), _ptr(out.get("alpha")), _ptr(out.get("wrot")),
+                    _ptr(out.get("centroids")), _stream_handle(stream))
+    return out

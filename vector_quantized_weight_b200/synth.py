@@ -156,3 +156,25 @@ def adversarial_wi(N: int, J: int, pattern: str, seed: int = 0) -> np.ndarray:
     if pattern == "random":
         return np.random.default_rng(seed).integers(0, 256, size=(N, J), dtype=np.uint8)
     raise ValueError(pattern)
+
+
+# ------------------------------------------------------- quantizer inputs
+
+def make_dense_weight(N: int, K: int, seed: int, std: float = 0.02) -> np.ndarray:
+    """A dense fp16 weight [N][K] ~ N(0, std^2) for the offline quantizer."""
+    rng = np.random.default_rng(seed + 9_000_000)
+    return rng.normal(0.0, std, size=(N, K)).astype(np.float16)
+
+
+def make_hsign(K: int, seed: int) -> np.ndarray:
+    """Rotation signs s [K] in {-1, +1} (int8)."""
+    rng = np.random.default_rng(seed + 8_000_000)
+    return rng.choice(np.array([-1, 1], np.int8), size=K)
+
+
+def kmeans_init_index(vecs_per_cb: int, G: int, ncent: int, seed: int) -> np.ndarray:
+    """Starting blocks of the K-means: for each of the G codebooks, ncent
+    distinct block indices in [0, vecs_per_cb), drawn without replacement
+    (int32 [G][ncent])."""
+    rng = np.random.default_rng(seed + 7_500_000)
+    return np.stack([rng.choice(vecs_per_cb, size=ncent, replace=False) for _ in range(G)]).astype(np.int32)

@@ -101,15 +101,18 @@ def test_create_without_device_reports_no_device():
     assert _create(_desc()) == eva_vq.EVA_ERR_NO_DEVICE
 
 
-def test_lookup_kernels_do_not_spill():
-    """ptxas report of every lookup-kernel instance: no local-memory stack
-    frame and no spills (the hot loop keeps everything in registers)."""
+def test_kernels_do_not_spill():
+    """ptxas report of every kernel (16 lookup instances, 4 dequantize
+    instances, the rotation, repack and quantizer kernels): no local-memory
+    stack frame and no spills (hot loops keep everything in registers)."""
     cmd = [build._nvcc(), *[f for f in build.NVCC_FLAGS if f != "-shared"], "-Xptxas", "-v", "-c",
            "-I", os.path.join(ROOT, "include"), "-o", os.devnull, *build.SOURCES]
     out = subprocess.run(cmd, capture_output=True, text=True, check=True).stderr
-    blocks = re.findall(r"Function properties for (\S*eva_lookup_kernel\S*)\n\s*(\d+) bytes stack frame, "
+    blocks = re.findall(r"Function properties for (\S*eva_\w+_kernel\S*)\n\s*(\d+) bytes stack frame, "
                         r"(\d+) bytes spill stores, (\d+) bytes spill loads", out)
-    assert len(blocks) == 16, out
+    assert sum("eva_lookup_kernel" in b[0] for b in blocks) == 16, out
+    assert sum("eva_dequant_kernel" in b[0] for b in blocks) == 4, out
+    assert sum("eva_kmeans_assign_kernel" in b[0] for b in blocks) == 2, out
     for name, stack, st, ld in blocks:
         assert (stack, st, ld) == ("0", "0", "0"), (name, stack, st, ld)
 

@@ -60,11 +60,12 @@ def test_index_roundtrip_bit_exact(N, K, pattern):
     assert np.array_equal(back, wi)
 
 
-@pytest.mark.parametrize("B", [1, 2, 3])
+@pytest.mark.parametrize("B", [1, 2, 3, 4, 8, 9, 16, 17])
 @pytest.mark.parametrize("N,K,cbr", [(256, 512, 0), (128, 1024, 16), (40, 264, 0)])
 def test_integer_inputs_exact(N, K, cbr, B):
     """Small-integer codebooks and inputs: every product and sum is exact in
-    fp16 / fp32, so the GPU must reproduce the oracle exactly."""
+    fp16 / fp32, so the GPU must reproduce the oracle exactly (B >= 4 takes
+    the dequantize path, B < 4 the lookup path)."""
     rng = np.random.default_rng(N + K + B)
     G = N // cbr if cbr else 1
     layer = synth.LayerData(synth.LayerShape("int", N, K, codebook_rows=cbr),
@@ -169,3 +170,37 @@ def test_independent_flag_matches_plain_run(key, li, B):
     assert lib.eva_vq_linear_run_ex(lin.handle, xs[0].data_ptr(), B, y.data_ptr(), None, 2) == \
         eva_vq.EVA_ERR_INVALID_ARG
     lin.close()
+
+
+@pytest.mark.parametrize("key,li,B", [("llama7b_layer", 0, 1), ("llama7b_layer", 0, 2), ("llama7b_block", 4, 4),
+                                      ("llama70b", 0, 8), ("tiny", 0, 1)])
+def test_both_paths_match_the_oracle(key, li, B):
+    """The lookup path and the dequantize path each meet the tolerance at any
+    batch size; the handle reports which one ran."""
+    import torch
+    from vector_quantized_weight_b200 import eva_vq
+    cfg = synth.CONFIGS[key]
+    shape = cfg.layers[li]
+    seed = synth.layer_seed(cfg.index, li)
+    layer = synth.make_layer(shape, seed)
+    x = synth.make_x(shape.K, B, seed)
+    rows = sample_rows(shape.N, shape.codebook_rows, n=128, seed=seed)
+    ref = sub_layer_oracle(layer, x, rows)
+    for path in (eva_vq.EVA_PATH_OC_LOOKUP, eva_vq.EVA_PATH_DEQUANT_MMA):
+        lin = eva_vq.from_layer(layer, max_batch=B, path=path)
+        y = lin(torch.from_numpy(x).cuda()).float().cpu().numpy()
+        torch.cuda.synchronize()
+        assert lin.info().path == path
+        assert eva_vq.eva_vq_sync_status(lin.handle) == eva_vq.EVA_OK
+        lin.close()
+        err = norm_rel_err(y[:, rows], ref)
+        assert np.all(err <= TOL), (path, err.max())
+
+
+def test_dequant_path_rejects_residual_layers():
+    from vector_quantized_weight_b200 import eva_vq
+    shape = synth.LayerShape("r", 64, 512, residual_group=128)
+    layer = synth.make_layer(shape, 1)
+    with pytest.raises(eva_vq.EvaError) as ei:
+        eva_vq.from_layer(layer, max_batch=8, path=eva_vq.EVA_PATH_DEQUANT_MMA)
+    assert ei.value.status == eva_vq.EVA_ERR_UNSUPPORTED

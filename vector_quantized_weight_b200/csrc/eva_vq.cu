@@ -19,6 +19,7 @@
 #include "../../include/eva_vq.h"
 #include "eva_vq_kernels.cuh"
 #include "eva_vq_quant.cuh"
+#include "eva_vq_dequant.cuh"
 
 using namespace eva;
 
@@ -33,6 +34,10 @@ struct eva_vq_linear {
     // `staged` index units per CTA are copied into shared memory up front
     // (`smem`); calls flagged independent skip that copy (`smem_nostage`).
     struct Plan { int Gs = 1, Gt = 1, staged = 0; size_t smem = 0, smem_nostage = 0; } plan[2];
+    // Dequantize-to-tensor-core path (no residual, no rotation): plans for 8
+    // and 16 tokens per pass.
+    bool dq_ok = false;
+    Plan dq[2];
     uint8_t *wi = nullptr;              // repacked indices
     uint8_t *sg = nullptr;              // repacked signs
     __half *al = nullptr;               // repacked alpha
@@ -76,7 +81,7 @@ eva_status_t validate_desc(const eva_vq_desc *d) {
     if (d->out_dtype != EVA_F16 && d->out_dtype != EVA_F32) return EVA_ERR_INVALID_ARG;
     if (d->path != EVA_PATH_AUTO && d->path != EVA_PATH_OC_LOOKUP && d->path != EVA_PATH_DEQUANT_MMA)
         return EVA_ERR_INVALID_ARG;
-    if (d->path == EVA_PATH_DEQUANT_MMA) return EVA_ERR_UNSUPPORTED;
+    if (d->path == EVA_PATH_DEQUANT_MMA && (d->residual_group || d->hadamard_block)) return EVA_ERR_UNSUPPORTED;
     return EVA_OK;
 }
 
@@ -224,8 +229,68 @@ cudaError_t launch_pdl(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_
 }
 
 
+using DequantFn = void (*)(LookupParams);
+DequantFn dequant_fn(bool grouped, int ntg) {
+    if (grouped) return ntg == 2 ? eva_dequant_kernel<true, 2> : eva_dequant_kernel<true, 1>;
+    return ntg == 2 ? eva_dequant_kernel<false, 2> : eva_dequant_kernel<false, 1>;
+}
+
+// Calls with at least this many tokens take the dequantize path (when the
+// layer allows it and the descriptor leaves the choice to the library).
+constexpr int kDequantMinBatch = 4;
+
+// Dynamic shared memory of the dequantize kernel: the replicated codebook,
+// the x stage of up to nsl slices, the running sums and the reduction stage.
+size_t dequant_smem(int nsl, int tiles, int gs, int ntg) {
+    const size_t blk = (size_t)kTileRows * 8 * ntg * 4;
+    const size_t xs = ((size_t)nsl * 8 * ntg * kXTokStride + 127) & ~(size_t)127;
+    const size_t nslot = (size_t)(tiles + gs - 1) / gs;
+    return (size_t)kTabBytes + xs + (size_t)tiles * blk + nslot * gs * blk;
+}
+
+// Same search as plan_grid, for the dequantize kernel (one CTA per SM, every
+// cluster in one wave when the shared memory allows it).
+void plan_dequant(eva_vq_linear *h, int ntg) {
+    const int S = h->S, T = h->T, P = h->sm_count;
+    const DequantFn fn = dequant_fn(h->tiles_per_cb != 0, ntg);
+    double best = 1e300;
+    eva_vq_linear::Plan pl;
+    pl.Gs = 0;
+    for (int gs = 1; gs <= std::min(S, 16); ++gs) {
+        const int nsl = (S + gs - 1) / gs;
+        const int gt_min = (T + kMaxCtaTiles - 1) / kMaxCtaTiles;
+        const int clusters = max_active_clusters((LookupFn)fn, (size_t)h->smem_optin, gs);
+        const int gt_max = std::min({T, std::max(clusters, gt_min), std::max(P / gs, gt_min)});
+        for (int gt = gt_min; gt <= gt_max; ++gt) {
+            const int tiles = (T + gt - 1) / gt;
+            if (dequant_smem(nsl, tiles, gs, ntg) > (size_t)h->smem_optin) continue;
+            int builds = 1;
+            if (h->tiles_per_cb) builds = (tiles + h->tiles_per_cb - 1) / h->tiles_per_cb + 1;
+            double cost = (double)nsl * (700.0 + (250.0 + 150.0 * ntg) * ((tiles + kWarps - 1) / kWarps)) +
+                          600.0 * builds + ((gs > 1) ? 600.0 + 40.0 * gs : 0.0);
+            if (gt > clusters) cost *= 2.0;   // beyond one wave
+            if (cost < best) {
+                best = cost;
+                pl.Gs = gs;
+                pl.Gt = gt;
+            }
+        }
+    }
+    if (pl.Gs == 0) return;   // nothing fits: the lookup path serves every batch
+    const int tiles = (T + pl.Gt - 1) / pl.Gt;
+    pl.smem = pl.smem_nostage = dequant_smem((S + pl.Gs - 1) / pl.Gs, tiles, pl.Gs, ntg);
+    h->dq[ntg - 1] = pl;
+}
+
 cudaError_t set_smem_attrs(int smem_optin) {
     cudaError_t e;
+    for (int v = 0; v < 4; ++v) {
+        const DequantFn fn = dequant_fn(v & 1, 1 + (v >> 1));
+        e = cudaFuncSetAttribute((const void *)fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute((const void *)fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_optin);
+        if (e != cudaSuccess) return e;
+    }
     for (int v = 0; v < 16; ++v) {
         const LookupFn fn = lookup_fn(v & 1, (v >> 1) & 1, (v >> 2) & 1, (v >> 3) & 1);
         e = cudaFuncSetAttribute((const void *)fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
@@ -237,6 +302,30 @@ cudaError_t set_smem_attrs(int smem_optin) {
         if (e != cudaSuccess) return e;
     }
     return cudaFuncSetAttribute(eva_hadamard_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 4096 * 4);
+}
+
+// Launch the dequantize kernel for a call whose common parameters are in p.
+cudaError_t launch_dequant(eva_vq_linear *h, LookupParams p, int B, cudaStream_t s, size_t *smem_out,
+                           int *grid_out) {
+    const int ntg = B > 8 ? 2 : 1;
+    const eva_vq_linear::Plan &pl = h->dq[ntg - 1];
+    p.Gs = pl.Gs;
+    p.Gt = pl.Gt;
+    p.acc_tiles = (h->T + pl.Gt - 1) / pl.Gt;
+    p.wi_staged = 0;
+    p.rot_b = 0;
+    *smem_out = pl.smem;
+    *grid_out = pl.Gs * pl.Gt;
+#ifdef EVA_DEVICE_CHECKS
+    p.smem_bytes = (unsigned)pl.smem;
+#endif
+    return launch_pdl(dequant_fn(h->tiles_per_cb != 0, ntg), dim3(pl.Gs * pl.Gt), dim3(kThreads), pl.smem, s,
+                      pl.Gs, p);
+}
+
+bool use_dequant(const eva_vq_linear *h, int B) {
+    if (!h->dq_ok) return false;
+    return h->desc.path == EVA_PATH_DEQUANT_MMA || (h->desc.path == EVA_PATH_AUTO && B >= kDequantMinBatch);
 }
 
 void free_handle(eva_vq_linear *h) {
@@ -328,7 +417,18 @@ eva_status_t eva_vq_linear_create(eva_vq_linear_t *out, const eva_vq_desc *desc,
     chk(set_smem_attrs(h->smem_optin));
     plan_grid(h, 0);
     if (desc->max_batch > 1) plan_grid(h, 1);
-    const int max_grid = std::max(h->plan[0].Gs * h->plan[0].Gt, h->plan[1].Gs * h->plan[1].Gt);
+    int max_grid = std::max(h->plan[0].Gs * h->plan[0].Gt, h->plan[1].Gs * h->plan[1].Gt);
+    if (!desc->residual_group && !desc->hadamard_block &&
+        (desc->path == EVA_PATH_DEQUANT_MMA || (desc->path == EVA_PATH_AUTO && desc->max_batch >= kDequantMinBatch))) {
+        plan_dequant(h, 1);
+        plan_dequant(h, 2);
+        h->dq_ok = h->dq[0].Gs > 0 && h->dq[1].Gs > 0;
+        if (h->dq_ok) max_grid = std::max({max_grid, h->dq[0].Gs * h->dq[0].Gt, h->dq[1].Gs * h->dq[1].Gt});
+        else if (desc->path == EVA_PATH_DEQUANT_MMA) {
+            free_handle(h);
+            return EVA_ERR_UNSUPPORTED;
+        }
+    }
     chk(dalloc(&h->wi, (size_t)units * kUnitBytes, nullptr));
     chk(dalloc(&h->wc, (size_t)h->G * kCent * kD * sizeof(__half), nullptr));
     if (desc->residual_group) {
@@ -453,6 +553,16 @@ eva_status_t eva_vq_linear_run_ex(eva_vq_linear_t h, const void *x, int32_t B, v
         p.chk_record = h->status;
     }
 #endif
+    if (use_dequant(h, B)) {
+        size_t dsmem = 0;
+        int dgrid = 0;
+        e = launch_dequant(h, p, B, s, &dsmem, &dgrid);
+        if (e != cudaSuccess) return cuda_status(e);
+        h->last_grid = dgrid;
+        h->last_kernels = kernels + 1;
+        h->last_path = EVA_PATH_DEQUANT_MMA;
+        return EVA_OK;
+    }
     e = launch_pdl(lookup_fn(pair_t, resid, h->tiles_per_cb != 0, p.rot_b != 0), grid, block, smem, s, pl.Gs, p);
     if (e != cudaSuccess) return cuda_status(e);
     ++kernels;
@@ -551,6 +661,11 @@ eva_status_t eva_vq_linear_run_noalloc(eva_vq_linear_t h, const void *x, int32_t
         if (e != cudaSuccess) return cuda_status(e);
         p.x = scratch;
         p.x_f32 = 1;
+    }
+    if (use_dequant(h, B)) {   // no rotation on this path, so no scratch either
+        size_t dsmem = 0;
+        int dgrid = 0;
+        return cuda_status(launch_dequant(h, p, B, s, &dsmem, &dgrid));
     }
     const bool resid = d.residual_group != 0;
     e = launch_pdl(lookup_fn(pair_t, resid, h->tiles_per_cb != 0, false), dim3(pl.Gs * pl.Gt), dim3(kThreads),

@@ -1,0 +1,258 @@
+// eva_vq_dequant.cuh -- the dequantize-to-tensor-core path for larger batches.
+//
+// The output-codebook lookups of the EVA summary (section 2.A) cost one
+// shared-memory read per index and token pair, so they grow with the batch.
+// The alternative the EVA summary's GEMM mode stands for: rebuild the weight
+// from the codebook (WC[WI], one 8-byte read per index whatever the batch)
+// and let tensor-core MMAs (m16n8k16, f16 in, fp32 accumulate) multiply it
+// with up to 16 tokens at a time.  Layers with a shared codebook or one
+// codebook per group of rows; no sign residual, no rotation (those keep the
+// lookup path).
+//
+// Same repacked index units and the same CTA grid as the lookup kernel
+// (clusters of Gs slice groups x Gt row groups, split-K sums combined in
+// distributed shared memory).  Per lane the index bytes of a unit are
+// rotated so that MMA block beta (16 inputs = 4 sub-vectors) reads, for lane
+// (g, q), sub-vector 4 beta + q (beta < 8) or 4 (beta - 8) + q + 32: the k
+// order inside a block is permuted identically in A (the weights) and B (x),
+// which leaves the product unchanged.  A fragment: the four fp16 components
+// of the lane's centroid for rows g and g + 8, read from a codebook table
+// replicated 16 times across the banks (conflict-free); B fragment: the same
+// sub-vector of token g, kept in registers for a whole slice.
+#pragma once
+#include "eva_vq_kernels.cuh"
+
+namespace eva {
+
+constexpr uint32_t kTabBytes = kCent * 16u * 8u;      // 256 centroids x 16 copies x 8 bytes
+constexpr uint32_t kXTokStride = 544u;                // bytes per staged token (512 + 32: conflict-free)
+
+// Sub-vector (within the slice) that lane quarter q reads in MMA block beta.
+__host__ __device__ __forceinline__ int dq_subvec(int beta, int q) {
+    return beta < 8 ? 4 * beta + q : 4 * (beta - 8) + q + 32;
+}
+
+__device__ __forceinline__ uint2 lds64(uint32_t off) { return *reinterpret_cast<const uint2 *>(eva_smem + off); }
+
+// Codebook cb replicated: entry c, copy r at c * 128 + 8 r (r = lane mod 16).
+__device__ __forceinline__ void build_codebook_table(const LookupParams &p, int cb, int tid) {
+    const uint2 *src = reinterpret_cast<const uint2 *>(p.wc + (size_t)cb * kCent * kD);
+    for (int i = tid; i < kCent * 16; i += kThreads) {
+        const int c = i >> 4, r = i & 15;
+        const uint32_t off = (uint32_t)c * 128u + 8u * (uint32_t)r;
+        if (!EVA_BAD_G(BUF_WC, src + c, 8) && !EVA_BAD_S(off) && !EVA_BAD_S(off + 4u))
+            *reinterpret_cast<uint2 *>(eva_smem + off) = __ldg(src + c);
+    }
+}
+
+template <bool GROUPED, int NTG>
+__global__ void __launch_bounds__(kThreads, 1) eva_dequant_kernel(const LookupParams p) {
+    constexpr int TT = 8 * NTG;                         // tokens per pass
+    constexpr uint32_t BLK = kTileRows * TT * 4u;       // bytes of one tile's sums
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = lane >> 2, q = lane & 3;
+    const int ts = blockIdx.x % p.Gs, tt = blockIdx.x / p.Gs;
+    const int s0 = (int)((long long)p.S * ts / p.Gs), s1 = (int)((long long)p.S * (ts + 1) / p.Gs);
+    const int t0 = (int)((long long)p.T * tt / p.Gt), t1 = (int)((long long)p.T * (tt + 1) / p.Gt);
+    const int ntw = (t1 - t0 - warp + kWarps - 1) / kWarps;
+    const int nsl = s1 - s0, ctiles = t1 - t0;
+    const int cb_first = GROUPED ? t0 / p.tiles_per_cb : 0;
+    const int cb_last = GROUPED ? (t1 - 1) / p.tiles_per_cb : 0;
+
+    // Shared memory: codebook table | x stage [slice][token] | running sums
+    // [tile][16][TT] | reduction stage [ceil(acc_tiles / Gs)][Gs][16][TT].
+    constexpr uint32_t TAB_OFF = 0, XS_OFF = kTabBytes;
+    // The layout must be the same in every CTA of a cluster (peers write into
+    // the reduction stage at this CTA's offsets): size the x stage for the
+    // largest slice count, ceil(S / Gs).
+    const int nsl_max = (p.S + p.Gs - 1) / p.Gs;
+    const uint32_t ACC_OFF = (XS_OFF + (uint32_t)(nsl_max * TT) * kXTokStride + 127u) & ~127u;
+    const uint32_t STAGE_OFF = ACC_OFF + (uint32_t)p.acc_tiles * BLK;
+    float *acc_s = reinterpret_cast<float *>(eva_smem + ACC_OFF);
+    const float *stage = reinterpret_cast<const float *>(eva_smem + STAGE_OFF);
+    const uint32_t stage_addr = (uint32_t)__cvta_generic_to_shared(eva_smem + STAGE_OFF);
+
+    // ---- prologue: weights only ----
+    EVA_STAMP(0);
+    pdl_launch();
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+    if (tid < nsl) {
+        const size_t u = (size_t)(s0 + tid) * p.T + t0;
+        const uint32_t nt = (uint32_t)ctiles;
+        if (!EVA_BAD_G(BUF_WI, p.wi + u * kUnitBytes, nt * kUnitBytes)) prefetch_l2_bulk(p.wi + u * kUnitBytes, nt * kUnitBytes);
+    }
+    build_codebook_table(p, cb_first, tid);
+    int built_cb = cb_first;
+
+    if (!p.independent) pdl_wait();
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+    EVA_STAMP(1);
+
+    const uint32_t lofs = 8u * (uint32_t)(lane & 15);   // this lane's copy in the table
+    for (int p0 = 0; p0 < p.B; p0 += TT) {
+        // x of this pass's tokens for all the CTA's slices, fp16, zeros past B / K.
+        for (int i = tid; i < nsl * TT * 32; i += kThreads) {
+            const int chunk = i & 31, n = (i >> 5) % TT, sl = i / (32 * TT);
+            const int tok = p0 + n, k0 = (s0 + sl) * kSliceK + 8 * chunk;
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (tok < p.B && k0 + 8 <= p.K && ((((size_t)tok * p.K + k0) & 7) == 0)) {
+                const uint4 *xp = reinterpret_cast<const uint4 *>(reinterpret_cast<const __half *>(p.x) +
+                                                                  (size_t)tok * p.K + k0);
+                if (!EVA_BAD_G(BUF_X, xp, 16)) v = __ldcg(xp);
+            } else if (tok < p.B && k0 < p.K) {
+                unsigned short h[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const unsigned short *xp = reinterpret_cast<const unsigned short *>(p.x) + (size_t)tok * p.K + k0 + e;
+                    h[e] = (k0 + e < p.K && !EVA_BAD_G(BUF_X, xp, 2)) ? __ldcg(xp) : (unsigned short)0;
+                }
+                v = make_uint4(h[0] | ((uint32_t)h[1] << 16), h[2] | ((uint32_t)h[3] << 16),
+                               h[4] | ((uint32_t)h[5] << 16), h[6] | ((uint32_t)h[7] << 16));
+            }
+            const uint32_t off = XS_OFF + (uint32_t)(sl * TT + n) * kXTokStride + 16u * (uint32_t)chunk;
+            if (!EVA_BAD_S(off) && !EVA_BAD_S(off + 12u)) *reinterpret_cast<uint4 *>(eva_smem + off) = v;
+        }
+        __syncthreads();
+        EVA_STAMP(2);
+
+        for (int cb = cb_first; cb <= cb_last; ++cb) {
+            int i0 = 0, i1 = ntw;
+            if (GROUPED) {
+                const int lo = max(cb * p.tiles_per_cb, t0), hi = (cb + 1) * p.tiles_per_cb;
+                i0 = max(0, (lo - t0 - warp + kWarps - 1) / kWarps);
+                i1 = min(ntw, max(0, (hi - t0 - warp + kWarps - 1) / kWarps));
+                if (cb != built_cb) {
+                    __syncthreads();               // every warp is done with the previous table
+                    build_codebook_table(p, cb, tid);
+                    __syncthreads();
+                    built_cb = cb;
+                }
+            }
+            for (int s = s0; s < s1; ++s) {
+                // B fragments of this slice: token 8t + g, sub-vector dq_subvec(beta, q).
+                uint2 xb[NTG][16];
+#pragma unroll
+                for (int t = 0; t < NTG; ++t)
+#pragma unroll
+                    for (int beta = 0; beta < 16; ++beta) {
+                        const uint32_t off = XS_OFF + (uint32_t)((s - s0) * TT + 8 * t + g) * kXTokStride +
+                                             8u * (uint32_t)dq_subvec(beta, q);
+                        xb[t][beta] = EVA_BAD_S(off) ? make_uint2(0u, 0u) : lds64(off);
+                    }
+                uint4 nb0 = make_uint4(0u, 0u, 0u, 0u), nb1 = nb0;
+                if (i0 < i1) {
+                    const uint8_t *up = p.wi + ((size_t)s * p.T + t0 + warp + kWarps * i0) * kUnitBytes + 16 * lane;
+                    if (!EVA_BAD_G(BUF_WI, up, 16) && !EVA_BAD_G(BUF_WI, up + 512, 16)) ldg_unit(up, nb0, nb1);
+                }
+#pragma unroll 1
+                for (int i = i0; i < i1; ++i) {
+                    const int tl = warp + kWarps * i;
+                    const uint32_t wv[8] = {nb0.x, nb0.y, nb0.z, nb0.w, nb1.x, nb1.y, nb1.z, nb1.w};
+                    if (i + 1 < i1) {
+                        const uint8_t *up = p.wi + ((size_t)s * p.T + t0 + tl + kWarps) * kUnitBytes + 16 * lane;
+                        if (!EVA_BAD_G(BUF_WI, up, 16) && !EVA_BAD_G(BUF_WI, up + 512, 16)) ldg_unit(up, nb0, nb1);
+                    }
+                    // rot[beta] = wv[(beta - g) mod 8]: the word holding sub-vectors 4 beta + q (+32).
+                    uint32_t rot[8];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) rot[k] = wv[k];
+#pragma unroll
+                    for (int bit = 1; bit < 8; bit <<= 1) {
+                        uint32_t nr[8];
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) nr[k] = (g & bit) ? rot[(k - bit) & 7] : rot[k];
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) rot[k] = nr[k];
+                    }
+                    float acc[NTG][2][4];
+#pragma unroll
+                    for (int t = 0; t < NTG; ++t)
+#pragma unroll
+                        for (int h = 0; h < 2; ++h)
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) acc[t][h][e] = 0.f;
+#pragma unroll
+                    for (int beta = 0; beta < 16; ++beta) {
+                        const uint32_t w = rot[beta & 7];
+                        const uint32_t cg = beta < 8 ? (w & 0xFFu) : ((w >> 16) & 0xFFu);
+                        const uint32_t ch = beta < 8 ? ((w >> 8) & 0xFFu) : (w >> 24);
+                        const uint32_t og = TAB_OFF + (cg << 7) + lofs, oh = TAB_OFF + (ch << 7) + lofs;
+                        const uint2 ag = EVA_BAD_S(og) ? make_uint2(0u, 0u) : lds64(og);
+                        const uint2 ah = EVA_BAD_S(oh) ? make_uint2(0u, 0u) : lds64(oh);
+#pragma unroll
+                        for (int t = 0; t < NTG; ++t)
+                            mma_f16_k16(acc[t][beta & 1], ag.x, ah.x, ag.y, ah.y, xb[t][beta].x, xb[t][beta].y);
+                    }
+                    // D: (row g, tokens 2q, 2q+1), (row g+8, tokens 2q, 2q+1) of each token group.
+#pragma unroll
+                    for (int t = 0; t < NTG; ++t)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int row = g + 8 * (e >> 1), tok = 8 * t + 2 * q + (e & 1);
+                            const int ai = (tl * kTileRows + row) * TT + tok;
+                            const float v = acc[t][0][e] + acc[t][1][e];
+                            if (!EVA_BAD_S(ACC_OFF + 4u * (uint32_t)ai)) acc_s[ai] = (s == s0) ? v : acc_s[ai] + v;
+                        }
+                }
+            }
+        }
+
+        // Split-K sums of this pass: push each tile's block to the owning
+        // cluster CTA (rank tl % Gs) with 16-byte remote stores, cluster
+        // barrier, owners add the Gs blocks in rank order and store y.
+        EVA_STAMP(4);
+        __syncthreads();
+        constexpr int CH = (int)(BLK / 16u);               // 16-byte chunks per tile block
+        for (int i = tid; i < ctiles * CH; i += kThreads) {
+            const int tl = i / CH, chunk = i % CH;
+            const uint32_t src = ACC_OFF + (uint32_t)tl * BLK + 16u * (uint32_t)chunk;
+            const uint32_t dst = (uint32_t)((tl / p.Gs) * p.Gs + ts) * BLK + 16u * (uint32_t)chunk;
+            if (!EVA_BAD_S(src) && !EVA_BAD_S(src + 12u) && !EVA_BAD_S(STAGE_OFF + dst) && !EVA_BAD_S(STAGE_OFF + dst + 12u)) {
+                const float4 v = *reinterpret_cast<const float4 *>(eva_smem + src);
+                st_dsmem_v4(stage_addr + dst, (uint32_t)(tl % p.Gs), v);
+            }
+        }
+        cluster_sync_all();
+        EVA_STAMP(5);
+        {
+            const int my_tiles = (ctiles - ts + p.Gs - 1) / p.Gs;
+            for (int idx = tid; idx < my_tiles * kTileRows * TT; idx += kThreads) {
+                const int row = idx % kTileRows, tok = (idx / kTileRows) % TT, slot = idx / (kTileRows * TT);
+                const int tl = ts + p.Gs * slot;
+                const int o = kTileRows * (t0 + tl) + row, b = p0 + tok;
+                if (b >= p.B || o >= p.N) continue;
+                float v[16];
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const uint32_t si = (uint32_t)((((slot * p.Gs + k) * kTileRows + row) * TT) + tok);
+                    v[k] = (k < p.Gs && !EVA_BAD_S(STAGE_OFF + 4u * si)) ? stage[si] : 0.f;
+                }
+                float sum = 0.f;
+#pragma unroll
+                for (int k = 0; k < 16; ++k)
+                    if (k < p.Gs) sum += v[k];
+                const size_t yi = (size_t)b * p.N + o;
+                if (p.out_f32) {
+                    float *yp = reinterpret_cast<float *>(p.y) + yi;
+                    if (!EVA_BAD_G(BUF_Y, yp, 4)) *yp = sum;
+                } else {
+                    __half *yp = reinterpret_cast<__half *>(p.y) + yi;
+                    if (!EVA_BAD_G(BUF_Y, yp, 2)) *yp = __float2half_rn(sum);
+                }
+            }
+        }
+        // The next pass rewrites the x stage, the sums and the owners' stages.
+        if (p0 + TT < p.B) cluster_sync_all();
+    }
+    if (p.independent) pdl_wait();
+    EVA_STAMP(6);
+#ifdef EVA_TIMELINE
+    if (tid == 0) {
+        unsigned smid;
+        asm volatile("mov.u32 %0, %smid;" : "=r"(smid));
+        p.timeline[blockIdx.x * 8 + 7] = smid;
+    }
+#endif
+}
+
+}  // namespace eva

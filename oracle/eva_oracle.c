@@ -104,8 +104,91 @@ static double sylvester(int p, int q)
 }
 
 /*
- * x~ = s (.) (H_b x) / sqrt(b), block by block, for one token.
- * xin and xout are K doubles; b must divide K (b = 0 copies x).
+ * Paley construction I of a Hadamard matrix of order 28 = 27 + 1, q = 27 = 3^3
+ * (q = 3 mod 4).  Reading taken (the pages give none): GF(27) is GF(3)[t]
+ * modulo t^3 + 2t + 2, element e = c0 + 3 c1 + 9 c2 is c0 + c1 t + c2 t^2;
+ * chi is the quadratic character (chi(a) = a^13, chi(0) = 0); the Jacobsthal
+ * matrix is Q[i][j] = chi(e_i - e_j); H28 = I + S with S = [0, 1^T; -1, Q].
+ */
+static int gf27_sub(int a, int b)
+{
+    int r = 0, w = 1;
+    for (int i = 0; i < 3; ++i) {
+        int d = ((a % 3) - (b % 3) + 3) % 3;
+        r += d * w;
+        w *= 3;
+        a /= 3;
+        b /= 3;
+    }
+    return r;
+}
+
+static int gf27_mul(int a, int b)
+{
+    int x[3], y[3], z[5] = {0, 0, 0, 0, 0};
+    for (int i = 0; i < 3; ++i) { x[i] = a % 3; a /= 3; y[i] = b % 3; b /= 3; }
+    for (int i = 0; i < 3; ++i)
+        for (int j = 0; j < 3; ++j) z[i + j] = (z[i + j] + x[i] * y[j]) % 3;
+    /* t^3 = t + 1 and t^4 = t^2 + t (mod 3, modulo t^3 + 2t + 2) */
+    z[1] = (z[1] + z[3]) % 3; z[0] = (z[0] + z[3]) % 3;
+    z[2] = (z[2] + z[4]) % 3; z[1] = (z[1] + z[4]) % 3;
+    return z[0] + 3 * z[1] + 9 * z[2];
+}
+
+static int gf27_chi(int a)
+{
+    if (a == 0) return 0;
+    int r = 1;
+    for (int i = 0; i < 13; ++i) r = gf27_mul(r, a);
+    return r == 1 ? 1 : -1;   /* a^13 is 1 or -1 (= element 2) */
+}
+
+static double paley28_entry(int i, int j)
+{
+    if (i == 0) return 1.0;
+    if (j == 0) return -1.0;
+    if (i == j) return 1.0;
+    return (double)gf27_chi(gf27_sub(i - 1, j - 1));
+}
+
+/* The 784 entries, computed once (the character is slow to evaluate). */
+static double paley28(int i, int j)
+{
+    static double tab[28][28];
+    static int ready = 0;
+    if (!ready) {
+#ifdef _OPENMP
+#pragma omp critical(vq_oracle_paley)
+#endif
+        {
+            if (!ready) {
+                for (int a = 0; a < 28; ++a)
+                    for (int b = 0; b < 28; ++b) tab[a][b] = paley28_entry(a, b);
+                ready = 1;
+            }
+        }
+    }
+    return tab[i][j];
+}
+
+static int is_pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
+
+/* Rotation blocks: a power of two b (Sylvester H_b), or b = 28 m with m a
+ * power of two (H_b = H28 (x) H_m, Kronecker, the order-28 factor outside). */
+static int valid_block(int b) { return is_pow2(b) || (b % 28 == 0 && is_pow2(b / 28)); }
+
+static double block_entry(int b, int p, int q)
+{
+    if (is_pow2(b)) return sylvester(p, q);
+    const int m = b / 28;
+    return paley28(p / m, q / m) * sylvester(p % m, q % m);
+}
+
+/*
+ * x~ = s (.) (H_b^T x) / sqrt(b), block by block, for one token (H_b^T = H_b
+ * for Sylvester blocks).  With Q = blockdiag(H_b) diag(s) / sqrt(b) this is
+ * x~ = Q^T x, the partner of W_rot = W Q.  xin and xout are K doubles; b must
+ * divide K (b = 0 copies x).
  */
 static void rotate_token(const double *xin, const int8_t *hsign, int K, int b, double *xout)
 {
@@ -119,7 +202,7 @@ static void rotate_token(const double *xin, const int8_t *hsign, int K, int b, d
         for (int p = 0; p < b; ++p) {
             double acc = 0.0;
             for (int q = 0; q < b; ++q)
-                acc += sylvester(p, q) * xb[q];
+                acc += block_entry(b, q, p) * xb[q];
             int k = blk * b + p;
             xout[k] = (double)hsign[k] * acc * inv;
         }
@@ -131,7 +214,7 @@ static void rotate_token(const double *xin, const int8_t *hsign, int K, int b, d
 int vq_oracle_hadamard(const uint16_t *x, const int8_t *hsign, int B, int K, int b, double *out)
 {
     if (!x || !out || B < 0 || K <= 0) return -1;
-    if (b > 0 && (!hsign || K % b != 0)) return -2;
+    if (b > 0 && (!hsign || K % b != 0 || !valid_block(b))) return -2;
     double *row = (double *)malloc(sizeof(double) * (size_t)K);
     if (!row) return -3;
     for (int t = 0; t < B; ++t) {

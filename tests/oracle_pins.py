@@ -392,11 +392,80 @@ def pin_residual_identity(orc, seed=17):
         assert np.all(alpha >= 0)
 
 
+# ------------------------------------------------- order-K (Paley) rotation
+
+def _rotation_matrix(orc, b):
+    """M = H_b / sqrt(b), read off the oracle's rotation of unit vectors:
+    rotating e_j gives H_b^T e_j / sqrt(b) = row j of M."""
+    eye = np.eye(b, dtype=np.float16)
+    return orc.hadamard(eye, np.ones(b, np.int8), b)
+
+
+def _gf27_squares():
+    """Nonzero squares of GF(27) = GF(3)[t] / (t^3 + 2t + 2), by enumeration;
+    element c0 + 3 c1 + 9 c2 is c0 + c1 t + c2 t^2."""
+    def mul(a, b):
+        x = [(a // 3 ** i) % 3 for i in range(3)]
+        y = [(b // 3 ** i) % 3 for i in range(3)]
+        z = np.convolve(x, y) % 3                       # degree <= 4
+        for d in (4, 3):                                # t^3 = -2t - 2 = t + 1 (mod 3)
+            c, z[d] = z[d], 0
+            z[d - 3] = (z[d - 3] + c) % 3
+            z[d - 2] = (z[d - 2] + c) % 3
+        return int(z[0] + 3 * z[1] + 9 * z[2])
+    return {mul(a, a) for a in range(1, 27)}
+
+
+def pin_paley_hadamard(orc):
+    """Order 28: entries +-1, H H^T = 28 I, skew (H + H^T = 2 I); the interior
+    is the quadratic character of GF(27) (squares found by enumeration)."""
+    H = np.rint(_rotation_matrix(orc, 28) * np.sqrt(28)).astype(int)
+    assert set(np.unique(H)) == {-1, 1}
+    assert np.array_equal(H @ H.T, 28 * np.eye(28, dtype=int))
+    assert np.array_equal(H + H.T, 2 * np.eye(28, dtype=int))
+    assert np.all(H[0] == 1) and np.all(H[1:, 0] == -1)
+    sq = _gf27_squares()
+    assert len(sq) == 13
+    def sub(a, b):
+        return sum((((a // 3 ** i) - (b // 3 ** i)) % 3) * 3 ** i for i in range(3))
+    for i in range(1, 28):
+        for j in range(1, 28):
+            if i != j:
+                assert H[i, j] == (1 if sub(i - 1, j - 1) in sq else -1), (i, j)
+
+
+def pin_paley_kronecker(orc):
+    """H_56 = H_28 (x) H_2 and H_224 = H_28 (x) H_8 (scipy's Sylvester
+    matrices), orthonormal after scaling."""
+    H28 = _rotation_matrix(orc, 28) * np.sqrt(28)
+    for m in (2, 8):
+        M = _rotation_matrix(orc, 28 * m)
+        ref = np.kron(H28, scipy.linalg.hadamard(m)) / np.sqrt(28 * m)
+        assert np.allclose(M, ref, atol=1e-12)
+        assert np.allclose(M @ M.T, np.eye(28 * m), atol=1e-12)
+
+
+def pin_paley_rotation_pairs(orc, seed=18):
+    """With a Paley block the weight rotation W_rot = W Q and the input
+    rotation x~ = Q^T x still pair up: W_rot x~ = W x."""
+    rng = np.random.default_rng(seed)
+    N, K, b = 4, 1792, 1792
+    w = rng.normal(0, 0.5, size=(N, K)).astype(np.float16)
+    hs = rng.choice([-1, 1], size=K).astype(np.int8)
+    x = rng.normal(size=(1, K)).astype(np.float16)
+    init = rng.normal(0, 0.5, size=(16, 4)).astype(np.float32)
+    *_, wrot = orc.quantize(w, init, iters=0, hsign=hs, hadamard_block=b)
+    lhs = wrot.astype(np.float64) @ orc.hadamard(x, hs, b)[0]
+    rhs = w.astype(np.float64) @ x[0].astype(np.float64)
+    assert np.allclose(lhs, rhs, rtol=1e-5, atol=1e-4), np.abs(lhs - rhs).max()
+
+
 ALL_PINS = [
     pin_golden_vq, pin_golden_residual, pin_golden_hadamard, pin_f16_decode,
     pin_hadamard_scipy, pin_factorisation, pin_factorisation_residual, pin_rotation_composite,
     pin_unit_centroids, pin_all_equal_indices, pin_group_scaling, pin_residual_popcount,
     pin_residual_unit_inputs, pin_hadamard_orthogonal, pin_lookup_identity, pin_batch_rows,
     pin_optimal_alpha, pin_kmeans_assign_scipy, pin_kmeans_sklearn, pin_quantize_exact_recovery,
-    pin_quantize_rotation, pin_residual_identity,
+    pin_quantize_rotation, pin_residual_identity, pin_paley_hadamard, pin_paley_kronecker,
+    pin_paley_rotation_pairs,
 ]

@@ -59,8 +59,15 @@ MUTATIONS = {
     "residual_dropped": ("wrow[k] += a * sign_of(d, signs, o, k);", "(void)a;"),
     "hadamard_sign_dropped": ("xout[k] = (double)hsign[k] * acc * inv;", "xout[k] = acc * inv;"),
     "hadamard_unnormalised": ("double inv = 1.0 / sqrt((double)b);", "double inv = 1.0;"),
-    "hadamard_transposed_block": ("acc += sylvester(p, q) * xb[q];",
-                                  "acc += sylvester(p, (q + 1) % b) * xb[q];"),
+    "hadamard_transposed_block": ("acc += block_entry(b, q, p) * xb[q];",
+                                  "acc += block_entry(b, (q + 1) % b, p) * xb[q];"),
+    "paley_not_transposed": ("acc += block_entry(b, q, p) * xb[q];", "acc += block_entry(b, p, q) * xb[q];"),
+    "paley_chi_flipped": ("return r == 1 ? 1 : -1;", "return r == 1 ? -1 : 1;"),
+    "paley_wrong_modulus": ("z[1] = (z[1] + z[3]) % 3; z[0] = (z[0] + z[3]) % 3;",
+                            "z[1] = (z[1] + z[3]) % 3; z[0] = (z[0] + 2 * z[3]) % 3;"),
+    "paley_kronecker_swapped": ("return paley28(p / m, q / m) * sylvester(p % m, q % m);",
+                                "return paley28(p % 28, q % 28) * sylvester(p / 28, q / 28);"),
+    "paley_border_sign": ("if (j == 0) return -1.0;", "if (j == 0) return 1.0;"),
     "f16_exponent_bias": ("expo - 25)", "expo - 24)"),
     "f16_subnormal_scale": ("ldexp((double)mant, -24)", "ldexp((double)mant, -25)"),
     "alpha_not_mean": ("num += v * s;", "num += v * v;"),

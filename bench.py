@@ -329,8 +329,8 @@ def main():
         n_e2e = min(steps, 2000)
         xh = [torch.from_numpy(synth.make_x(shape.K, B, seed + r)).pin_memory() for r in range(ring)]
         yh = torch.empty((B, shape.N), dtype=torch.float16).pin_memory()
-        for i in range(8):
-            layers[i % ring].run_host(xh[i % ring], yh, stream=stream)
+        for i in range(ring):        # every handle's first host call (captures its graph)
+            layers[i].run_host(xh[i], yh, stream=stream)
         if pg:
             pg.barrier()
         torch.cuda.synchronize(dev)

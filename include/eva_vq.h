@@ -17,7 +17,8 @@
  * randomized Hadamard rotation of the input and a 1-bit residual sign per
  * weight with one fp16 scale alpha per group of 128 inputs:
  *   y[o] = sum_j OC~[j][WI[o][j]] + sum_q alpha[o][q] sum_{k in q} sigma[o][k] x~[k],
- * with x~ = s (.) (H_b x) / sqrt(b) blockwise (Sylvester H_b, s = hsign).
+ * with x~ = s (.) (H_b^T x) / sqrt(b) blockwise (s = hsign; H_b a Sylvester
+ * matrix, or the Kronecker product of an order-28 Paley matrix with one).
  *
  * All entry points return a status code and never abort or trap.  No entry
  * point throws.  Device pointers must be 16-byte aligned.
@@ -70,7 +71,10 @@ typedef struct {
     int32_t codebook_rows;   /* 0: one shared codebook; R > 0: codebook g serves rows
                                 [R g, R g + R); R must be a multiple of 16 dividing N    */
     int32_t residual_group;  /* 0: no sign residual; 128: signs + one alpha per 128 k   */
-    int32_t hadamard_block;  /* 0: no rotation; b: power of two in [8, 4096] dividing K */
+    int32_t hadamard_block;  /* 0: no rotation; b dividing K: a power of two in [8, 4096]
+                                (Sylvester H_b), or 28 m with m a power of two in [64, 1024]
+                                (H_b = H28 (x) H_m, H28 from Paley's construction over GF(27)
+                                modulo t^3 + 2t + 2; b = K gives the order-K rotation)  */
     int32_t max_batch;       /* largest B passed to run(), 1..64; sizes the workspace   */
     eva_dtype_t out_dtype;   /* dtype of y                                               */
     eva_path_t path;         /* EVA_PATH_AUTO unless a test or benchmark forces one     */
@@ -165,8 +169,13 @@ EVA_API eva_status_t eva_vq_linear_run_noalloc(eva_vq_linear_t h, const void *x,
 /*
  * The same call with HOST buffers: copies x (host fp16 [B][K]) to the
  * handle's staging buffer, runs, copies y back to y_host ([B][N] of
- * out_dtype) and waits for `stream`.  Pinned host memory makes the copies
- * asynchronous; pageable memory works but is slower.
+ * out_dtype) and waits for `stream`.  With page-locked host buffers and x of
+ * at most 64 KB the kernels read x and write y in the mapped host memory
+ * directly (no copy operations); larger page-locked buffers go through one
+ * CUDA graph (copy in, run, copy out), captured on the first call for each B
+ * and replayed with its copy addresses updated; pageable memory works, one
+ * operation at a time, and is slower.  A handle keeps its graphs until it is
+ * destroyed.
  */
 EVA_API eva_status_t eva_vq_linear_run_host(eva_vq_linear_t h, const void *x_host, int32_t B,
                                     void *y_host, eva_stream_t stream);
@@ -248,7 +257,7 @@ typedef struct {
     int32_t index_bits;      /* 1..8: 2^index_bits centroids per codebook              */
     int32_t codebook_rows;   /* 0: one codebook; else rows per codebook (divides N)    */
     int32_t residual_group;  /* 0: no residual; else a multiple of 8 dividing K (128)  */
-    int32_t hadamard_block;  /* 0: no rotation; b: power of two in [8, 4096] dividing K */
+    int32_t hadamard_block;  /* 0: no rotation; else as in eva_vq_desc                 */
     int32_t iters;           /* Lloyd iterations, >= 0                                 */
 } eva_quant_desc;
 

@@ -64,6 +64,8 @@ def _create(desc, wc=0x1000, wi=0x2000, signs=None, alpha=None, hsign=None):
     (dict(residual_group=64), eva_vq.EVA_ERR_UNSUPPORTED),
     (dict(hadamard_block=384), eva_vq.EVA_ERR_INVALID_ARG),
     (dict(hadamard_block=1024), eva_vq.EVA_ERR_INVALID_ARG),  # does not divide K=512
+    (dict(K=896, hadamard_block=896), eva_vq.EVA_ERR_INVALID_ARG),    # 28 * 32: Paley factor m < 64
+    (dict(K=3584, hadamard_block=1792, residual_group=128), eva_vq.EVA_ERR_INVALID_ARG),  # no signs given
     (dict(max_batch=0), eva_vq.EVA_ERR_INVALID_ARG),
     (dict(max_batch=65), eva_vq.EVA_ERR_INVALID_ARG),
     (dict(out_dtype=7), eva_vq.EVA_ERR_INVALID_ARG),
@@ -155,3 +157,13 @@ def test_quantize_and_steps_reject_bad_pointers():
     assert lib.eva_vq_kmeans_update(P, 10, 4, None, 256, 0, P, P, None, None) == eva_vq.EVA_ERR_INVALID_ARG
     assert lib.eva_vq_residual(P, 4, 256, P, 256, P, 0, 100, P, P, None) == eva_vq.EVA_ERR_INVALID_ARG
     assert lib.eva_vq_residual(P, 4, 256, P, 256, P, 3, 128, P, P, None) == eva_vq.EVA_ERR_INVALID_ARG
+
+
+def test_create_accepts_order_k_rotation_descriptor():
+    """K = 3584 = 28 * 128 with b = K passes validation (the CPU machine then has
+    no device to create it on)."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    d = _desc(K=3584, hadamard_block=3584, residual_group=128)
+    assert _create(d, signs=0x3000, alpha=0x4000, hsign=0x5000) == eva_vq.EVA_ERR_NO_DEVICE

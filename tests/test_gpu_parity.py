@@ -85,6 +85,9 @@ def test_integer_inputs_exact(N, K, cbr, B):
     (272, 1024, 5, 16, 0, 0),       # 17 codebooks of 16 rows, odd batch
     (3584, 3584, 1, 0, 128, 512),   # Gemma block structure
     (8, 8192, 64, 0, 0, 0),         # maximum batch
+    (64, 1792, 3, 0, 128, 1792),    # order-28 Paley (x) Sylvester 64 rotation, token pairs
+    (32, 7168, 2, 0, 128, 7168),    # Paley (x) Sylvester 256: partial sums per warp
+    (48, 3584, 1, 0, 0, 1792),      # two Paley blocks, no residual
 ])
 def test_edge_cases(N, K, B, cbr, resid, had):
     shape = synth.LayerShape("edge", N, K, codebook_rows=cbr, residual_group=resid, hadamard_block=had)
@@ -204,3 +207,27 @@ def test_dequant_path_rejects_residual_layers():
     with pytest.raises(eva_vq.EvaError) as ei:
         eva_vq.from_layer(layer, max_batch=8, path=eva_vq.EVA_PATH_DEQUANT_MMA)
     assert ei.value.status == eva_vq.EVA_ERR_UNSUPPORTED
+
+
+def test_host_buffer_call_graph_and_pageable():
+    """eva_vq_linear_run_host with page-locked buffers (read and written in
+    place by the kernels for small x, else one replayed graph whose copy
+    addresses follow new buffers) and with pageable ones: all equal to the
+    device-buffer call."""
+    import torch
+    from vector_quantized_weight_b200 import eva_vq
+    shape = synth.CONFIGS["llama7b_layer"].layers[0]
+    layer = synth.make_layer(shape, 8)
+    lin = eva_vq.from_layer(layer, max_batch=16)
+    for B in (1, 16, 4, 16, 1):       # x of 8 and 32 KB: mapped host memory; 128 KB: the graph
+        for i in range(3):
+            x = synth.make_x(shape.K, B, 100 * B + i)
+            ref = lin(torch.from_numpy(x).cuda()).cpu()
+            xh = torch.from_numpy(x).pin_memory()
+            yh = torch.empty((B, shape.N), dtype=torch.float16).pin_memory()
+            lin.run_host(xh, yh)
+            assert torch.equal(yh, ref)
+            yp = torch.empty((B, shape.N), dtype=torch.float16)
+            lin.run_host(torch.from_numpy(x), yp)
+            assert torch.equal(yp, ref)
+    lin.close()

@@ -116,6 +116,7 @@ def _run_quantize(w, hsign, b, cbr, iters, init_index, index_bits=8, residual_gr
     (256, 512, 0, 0, 4),              # no rotation, one codebook
     (512, 1024, 256, 128, 3),         # rotation, one codebook per 128 rows
     (3584, 3584, 512, 0, 6),          # Gemma-2-9B-shaped 3.125-bit layer
+    (64, 1792, 1792, 0, 3),           # order-K rotation with a Paley factor
 ])
 def test_quantize_pipeline(N, K, b, cbr, iters):
     import torch

@@ -23,6 +23,7 @@ pytestmark = [pytest.mark.gpu,
     (synth.LayerShape("rot_3bit", 3584, 3584, residual_group=128, hadamard_block=512), 1),
     (synth.LayerShape("rot_pair", 512, 2048, residual_group=128, hadamard_block=2048), 3),
     (synth.LayerShape("plain_2bit", 4096, 4096), 1),
+    (synth.LayerShape("rot_paley", 256, 3584, residual_group=128, hadamard_block=3584), 1),
 ])
 def test_noalloc_run_matches_regular_run(shape, B):
     import torch

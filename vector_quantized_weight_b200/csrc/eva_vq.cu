@@ -43,9 +43,20 @@ struct eva_vq_linear {
     __half *al = nullptr;               // repacked alpha
     __half *wc = nullptr;               // codebooks [G][256][4]
     int8_t *hsign = nullptr;            // Hadamard signs [K]
+    int8_t *h28 = nullptr;              // order-28 Paley matrix (Paley rotation blocks)
     int *status = nullptr;              // device error word
     unsigned long long *timeline = nullptr;  // timeline build: [grid][8] stamps
     void *x_stage = nullptr, *y_stage = nullptr;
+    // Host-buffer calls: one captured graph (H2D copy, run, D2H copy) per
+    // batch size, replayed with the copies' host addresses updated.
+    struct HostGraph {
+        cudaGraphExec_t exec = nullptr;
+        cudaGraphNode_t h2d = nullptr, d2h = nullptr;
+        const void *x = nullptr;
+        void *y = nullptr;
+        bool failed = false;   // capture or instantiation refused: copies one by one
+    } host_graph[65];
+    cudaStream_t capture_stream = nullptr;
     int64_t workspace_bytes = 0;
     int last_grid = 0, last_kernels = 0, last_path = 0;
 };
@@ -62,6 +73,50 @@ eva_status_t cuda_status(cudaError_t e) {
 
 bool is_pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
 
+// Rotation blocks: a power of two in [8, 4096] (Sylvester), or b = 28 m with
+// m a power of two in [64, 1024] (Paley order 28 (x) Sylvester m; b is then a
+// multiple of 256, so every K-slice lies inside one block); b divides K.
+int paley_m(int b) { return (b % 28 == 0 && is_pow2(b / 28) && b / 28 >= 64 && b / 28 <= 1024) ? b / 28 : 0; }
+bool valid_rotation_block(int b, int K) {
+    if (b <= 0 || K % b) return false;
+    return (is_pow2(b) && b >= 8 && b <= 4096) || paley_m(b) != 0;
+}
+
+// The order-28 Hadamard matrix of Paley's first construction over GF(27):
+// GF(27) = GF(3)[t] / (t^3 + 2t + 2), element c0 + 3 c1 + 9 c2 = c0 + c1 t +
+// c2 t^2; chi(a) = +1 for a nonzero square, -1 for a non-square, 0 for 0;
+// Jacobsthal Q[i][j] = chi(e_i - e_j); H = I + [0, 1; -1, Q].
+void paley28_table(int8_t *out) {
+    auto mul = [](int a, int b) {
+        int x[3], y[3], z[5] = {0, 0, 0, 0, 0};
+        for (int i = 0; i < 3; ++i) { x[i] = a % 3; a /= 3; y[i] = b % 3; b /= 3; }
+        for (int i = 0; i < 3; ++i)
+            for (int j = 0; j < 3; ++j) z[i + j] = (z[i + j] + x[i] * y[j]) % 3;
+        for (int d = 4; d >= 3; --d) {          // t^3 = t + 1 (mod 3)
+            z[d - 3] = (z[d - 3] + z[d]) % 3;
+            z[d - 2] = (z[d - 2] + z[d]) % 3;
+            z[d] = 0;
+        }
+        return z[0] + 3 * z[1] + 9 * z[2];
+    };
+    bool square[27] = {};
+    for (int a = 1; a < 27; ++a) square[mul(a, a)] = true;
+    auto sub = [](int a, int b) {
+        int r = 0, w = 1;
+        for (int i = 0; i < 3; ++i, a /= 3, b /= 3, w *= 3) r += (((a % 3) - (b % 3) + 3) % 3) * w;
+        return r;
+    };
+    for (int i = 0; i < 28; ++i)
+        for (int j = 0; j < 28; ++j) {
+            int v;
+            if (i == 0) v = 1;
+            else if (j == 0) v = -1;
+            else if (i == j) v = 1;
+            else v = square[sub(i - 1, j - 1)] ? 1 : -1;
+            out[i * 28 + j] = (int8_t)v;
+        }
+}
+
 eva_status_t validate_desc(const eva_vq_desc *d) {
     if (!d) return EVA_ERR_INVALID_ARG;
     if (d->N < 1 || d->K < 1 || d->N > (1 << 24) || d->K > (1 << 22)) return EVA_ERR_INVALID_ARG;
@@ -72,11 +127,7 @@ eva_status_t validate_desc(const eva_vq_desc *d) {
         return EVA_ERR_INVALID_ARG;
     if (d->residual_group != 0 && d->residual_group != 128) return EVA_ERR_UNSUPPORTED;
     if (d->residual_group && d->K % d->residual_group) return EVA_ERR_INVALID_ARG;
-    if (d->hadamard_block) {
-        if (!is_pow2(d->hadamard_block) || d->hadamard_block < 8 || d->hadamard_block > 4096 ||
-            d->K % d->hadamard_block)
-            return EVA_ERR_INVALID_ARG;
-    }
+    if (d->hadamard_block && !valid_rotation_block(d->hadamard_block, d->K)) return EVA_ERR_INVALID_ARG;
     if (d->max_batch < 1 || d->max_batch > 64) return EVA_ERR_INVALID_ARG;
     if (d->out_dtype != EVA_F16 && d->out_dtype != EVA_F32) return EVA_ERR_INVALID_ARG;
     if (d->path != EVA_PATH_AUTO && d->path != EVA_PATH_OC_LOOKUP && d->path != EVA_PATH_DEQUANT_MMA)
@@ -97,7 +148,7 @@ size_t lookup_smem(bool pair_t, bool resid, int tiles, int gs, int rot_b, int st
     const size_t base = (size_t)kOcBytes + ((pair_t && resid) ? (size_t)kOcBytes : 0) +
                         (pair_t ? kXStageBytes : kXStageBytes / 2) + 128 + (size_t)tiles * tile_bytes +
                         stage_tiles * tile_bytes;
-    const size_t rot = rot_b > kSliceK ? (size_t)(pair_t ? 2 : 1) * rot_b * 4 : 0;
+    const size_t rot = rot_b ? (size_t)(pair_t ? 2 : 1) * rot_scratch_per_token(rot_b, paley_m(rot_b)) : 0;
     return ((base + 127) & ~(size_t)127) + rot + (size_t)staged * kUnitBytes;
 }
 
@@ -330,7 +381,10 @@ bool use_dequant(const eva_vq_linear *h, int B) {
 
 void free_handle(eva_vq_linear *h) {
     if (!h) return;
-    void *ptrs[] = {h->wi, h->sg, h->al, h->wc, h->hsign, h->status, h->x_stage,
+    for (auto &hg : h->host_graph)
+        if (hg.exec) cudaGraphExecDestroy(hg.exec);
+    if (h->capture_stream) cudaStreamDestroy(h->capture_stream);
+    void *ptrs[] = {h->wi, h->sg, h->al, h->wc, h->hsign, h->h28, h->status, h->x_stage,
                     h->y_stage, h->timeline};
     for (void *p : ptrs)
         if (p) cudaFree(p);
@@ -466,6 +520,12 @@ eva_status_t eva_vq_linear_create(eva_vq_linear_t *out, const eva_vq_desc *desc,
         chk(cudaGetLastError());
     }
     if (desc->hadamard_block) chk(cudaMemcpyAsync(h->hsign, hsign, (size_t)K, cudaMemcpyDeviceToDevice, s));
+    if (paley_m(desc->hadamard_block)) {
+        int8_t tab[28 * 28];
+        paley28_table(tab);
+        chk(dalloc(&h->h28, sizeof(tab), nullptr));
+        if (e == cudaSuccess) chk(cudaMemcpy(h->h28, tab, sizeof(tab), cudaMemcpyHostToDevice));
+    }
     chk(cudaMemsetAsync(h->status, 0, 8 * sizeof(int), s));
     if (e != cudaSuccess) {
         cudaStreamSynchronize(s);
@@ -522,6 +582,8 @@ eva_status_t eva_vq_linear_run_ex(eva_vq_linear_t h, const void *x, int32_t B, v
     p.independent = independent;
     if (d.hadamard_block) {   // the rotation runs inside the lookup kernel
         p.rot_b = d.hadamard_block;
+        p.rot_m = paley_m(d.hadamard_block);
+        p.h28 = h->h28;
         p.hs = h->hsign;
         p.rot_scale = (float)(1.0 / std::sqrt((double)d.hadamard_block));
     }
@@ -611,11 +673,15 @@ eva_status_t eva_vq_linear_run_noalloc(eva_vq_linear_t h, const void *x, int32_t
     if (!h || !x || !y || !aligned16(x) || !aligned16(y)) return EVA_ERR_INVALID_ARG;
     if (B < 1 || B > h->desc.max_batch) return EVA_ERR_INVALID_ARG;
     const eva_vq_desc &d = h->desc;
-    if ((size_t)B * d.K * sizeof(float) > kStaticScratchBytes) return EVA_ERR_SCRATCH_TOO_SMALL;
+    // A Paley rotation block has no standalone-kernel route that matches the
+    // fused rotation bit for bit at every size, so it stays fused (no scratch).
+    const bool fused_rot = paley_m(d.hadamard_block) != 0;
+    if (d.hadamard_block && !fused_rot && (size_t)B * d.K * sizeof(float) > kStaticScratchBytes)
+        return EVA_ERR_SCRATCH_TOO_SMALL;
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev != h->device) return EVA_ERR_INVALID_ARG;
     float *scratch = nullptr;
-    if (d.hadamard_block) {
+    if (d.hadamard_block && !fused_rot) {
         const eva_status_t st = static_scratch(dev, &scratch);
         if (st != EVA_OK) return st;
     }
@@ -652,7 +718,13 @@ eva_status_t eva_vq_linear_run_noalloc(eva_vq_linear_t h, const void *x, int32_t
     return EVA_ERR_UNSUPPORTED;   // the checked build validates the handle path only
 #endif
     cudaError_t e;
-    if (d.hadamard_block) {
+    if (fused_rot) {
+        p.rot_b = d.hadamard_block;
+        p.rot_m = paley_m(d.hadamard_block);
+        p.h28 = h->h28;
+        p.hs = h->hsign;
+        p.rot_scale = (float)(1.0 / std::sqrt((double)d.hadamard_block));
+    } else if (d.hadamard_block) {
         const int b = d.hadamard_block;
         const int thr = std::min(b / 2, 1024);
         e = launch_pdl(eva_hadamard_kernel, dim3(d.K / b, B), dim3(thr), (size_t)b * sizeof(float), s, 0,
@@ -668,10 +740,15 @@ eva_status_t eva_vq_linear_run_noalloc(eva_vq_linear_t h, const void *x, int32_t
         return cuda_status(launch_dequant(h, p, B, s, &dsmem, &dgrid));
     }
     const bool resid = d.residual_group != 0;
-    e = launch_pdl(lookup_fn(pair_t, resid, h->tiles_per_cb != 0, false), dim3(pl.Gs * pl.Gt), dim3(kThreads),
+    e = launch_pdl(lookup_fn(pair_t, resid, h->tiles_per_cb != 0, fused_rot), dim3(pl.Gs * pl.Gt), dim3(kThreads),
                    pl.smem, s, pl.Gs, p);
     return cuda_status(e);
 }
+
+// Inputs up to this size are read by the kernels straight from mapped host
+// memory in eva_vq_linear_run_host; larger ones are copied in first (every
+// row-group CTA reads x, so a large x would cross the bus several times).
+constexpr size_t kZeroCopyMaxBytes = 64 * 1024;
 
 eva_status_t eva_vq_linear_run_host(eva_vq_linear_t h, const void *x_host, int32_t B, void *y_host,
                                     eva_stream_t stream) {
@@ -680,6 +757,95 @@ eva_status_t eva_vq_linear_run_host(eva_vq_linear_t h, const void *x_host, int32
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const size_t xb = (size_t)B * h->desc.K * sizeof(__half);
     const size_t yb = (size_t)B * h->desc.N * (h->desc.out_dtype == EVA_F32 ? 4 : 2);
+    // Page-locked host buffers: one graph launch (copy in, run, copy out).
+    // Pageable ones: the three operations one by one.
+    cudaPointerAttributes ax, ay;
+    const bool pinned = cudaPointerGetAttributes(&ax, x_host) == cudaSuccess && ax.type == cudaMemoryTypeHost &&
+                        cudaPointerGetAttributes(&ay, y_host) == cudaSuccess && ay.type == cudaMemoryTypeHost;
+    cudaGetLastError();
+    // Small batches with page-locked buffers: no copies at all -- the kernel
+    // reads x from and writes y to the mapped host memory (the same bytes
+    // cross the bus, without two copy operations around the launch).
+    if (pinned && ax.devicePointer && ay.devicePointer && xb <= kZeroCopyMaxBytes &&
+        aligned16(ax.devicePointer) && aligned16(ay.devicePointer)) {
+        const eva_status_t st = eva_vq_linear_run(h, ax.devicePointer, B, ay.devicePointer, stream);
+        if (st != EVA_OK) return st;
+        return cuda_status(cudaStreamSynchronize(s));
+    }
+    if (pinned && !h->host_graph[B].failed) {
+        eva_vq_linear::HostGraph &hg = h->host_graph[B];
+        cudaError_t e = cudaSuccess;
+        if (!hg.exec) {
+            if (!h->capture_stream) {
+                e = cudaStreamCreateWithFlags(&h->capture_stream, cudaStreamNonBlocking);
+                if (e != cudaSuccess) return cuda_status(e);
+            }
+            cudaStream_t cs = h->capture_stream;
+            e = cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal);
+            if (e != cudaSuccess) return cuda_status(e);
+            cudaError_t e1 = cudaMemcpyAsync(h->x_stage, x_host, xb, cudaMemcpyHostToDevice, cs);
+            const eva_status_t st = e1 == cudaSuccess ? eva_vq_linear_run(h, h->x_stage, B, h->y_stage, cs)
+                                                      : EVA_ERR_CUDA;
+            cudaError_t e2 = st == EVA_OK ? cudaMemcpyAsync(y_host, h->y_stage, yb, cudaMemcpyDeviceToHost, cs)
+                                          : cudaSuccess;
+            cudaGraph_t graph = nullptr;
+            e = cudaStreamEndCapture(cs, &graph);
+            if (st == EVA_ERR_INVALID_ARG) {
+                if (graph) cudaGraphDestroy(graph);
+                return st;
+            }
+            if (st != EVA_OK || e1 != cudaSuccess || e2 != cudaSuccess || e != cudaSuccess) {
+                if (graph) cudaGraphDestroy(graph);
+                cudaGetLastError();
+                hg.failed = true;
+                return eva_vq_linear_run_host(h, x_host, B, y_host, stream);
+            }
+            // The two memcpy nodes: the first is the copy in, the last the copy out.
+            size_t n = 0;
+            cudaGraphGetNodes(graph, nullptr, &n);
+            cudaGraphNode_t nodes[16];
+            if (n > 16) n = 16;
+            cudaGraphGetNodes(graph, nodes, &n);
+            for (size_t i = 0; i < n; ++i) {
+                cudaGraphNodeType t;
+                cudaGraphNodeGetType(nodes[i], &t);
+                if (t != cudaGraphNodeTypeMemcpy) continue;
+                cudaMemcpy3DParms mp;
+                if (cudaGraphMemcpyNodeGetParams(nodes[i], &mp) != cudaSuccess) continue;
+                if (mp.srcPtr.ptr == x_host || mp.dstPtr.ptr == h->x_stage) hg.h2d = nodes[i];
+                else if (mp.dstPtr.ptr == y_host || mp.srcPtr.ptr == h->y_stage) hg.d2h = nodes[i];
+            }
+            e = cudaGraphInstantiate(&hg.exec, graph, 0);
+            cudaGraphDestroy(graph);
+            if (e != cudaSuccess || !hg.h2d || !hg.d2h) {
+                if (hg.exec) cudaGraphExecDestroy(hg.exec);
+                cudaGetLastError();
+                hg = eva_vq_linear::HostGraph();
+                hg.failed = true;
+                return eva_vq_linear_run_host(h, x_host, B, y_host, stream);
+            }
+            hg.x = x_host;
+            hg.y = y_host;
+        }
+        if (hg.x != x_host || hg.y != y_host) {
+            // New host buffers: update the two copies in place, or, where the
+            // runtime refuses that, capture the graph again for them.
+            e = cudaGraphExecMemcpyNodeSetParams1D(hg.exec, hg.h2d, h->x_stage, x_host, xb, cudaMemcpyHostToDevice);
+            if (e == cudaSuccess)
+                e = cudaGraphExecMemcpyNodeSetParams1D(hg.exec, hg.d2h, y_host, h->y_stage, yb, cudaMemcpyDeviceToHost);
+            if (e != cudaSuccess) {
+                cudaGetLastError();
+                cudaGraphExecDestroy(hg.exec);
+                hg = eva_vq_linear::HostGraph();
+                return eva_vq_linear_run_host(h, x_host, B, y_host, stream);
+            }
+            hg.x = x_host;
+            hg.y = y_host;
+        }
+        e = cudaGraphLaunch(hg.exec, s);
+        if (e != cudaSuccess) return cuda_status(e);
+        return cuda_status(cudaStreamSynchronize(s));
+    }
     cudaError_t e = cudaMemcpyAsync(h->x_stage, x_host, xb, cudaMemcpyHostToDevice, s);
     if (e != cudaSuccess) return cuda_status(e);
     eva_status_t st = eva_vq_linear_run(h, h->x_stage, B, h->y_stage, stream);
@@ -876,8 +1042,7 @@ eva_status_t eva_vq_quantize(const eva_quant_desc *desc, const void *w, const in
     if (d.residual_group && (d.residual_group < 8 || d.residual_group % 8 || d.K % d.residual_group))
         return EVA_ERR_INVALID_ARG;
     if (d.hadamard_block) {
-        const int b = d.hadamard_block;
-        if (b < 8 || b > 4096 || (b & (b - 1)) || d.K % b || !hsign) return EVA_ERR_INVALID_ARG;
+        if (!valid_rotation_block(d.hadamard_block, d.K) || !hsign) return EVA_ERR_INVALID_ARG;
     } else if (hsign) {
         return EVA_ERR_INVALID_ARG;
     }
@@ -919,16 +1084,30 @@ eva_status_t eva_vq_quantize(const eva_quant_desc *desc, const void *w, const in
     chk(cudaMemsetAsync(err, 0, sizeof(int), s));
 
     // 1. W_rot = W Q (rows rotated like x~), or W in fp32.
-    if (d.hadamard_block) {
-        const int b = d.hadamard_block, thr = std::min(b / 2, 1024);
+    int8_t *h28 = nullptr;
+    if (paley_m(d.hadamard_block)) {
+        int8_t tab[28 * 28];
+        paley28_table(tab);
+        chk(cudaMallocAsync(reinterpret_cast<void **>(&h28), sizeof(tab), s));
+        if (e == cudaSuccess) chk(cudaMemcpyAsync(h28, tab, sizeof(tab), cudaMemcpyHostToDevice, s));
+        if (e == cudaSuccess) chk(cudaStreamSynchronize(s));   // tab is on this stack frame
+    }
+    if (d.hadamard_block && e == cudaSuccess) {
+        const int b = d.hadamard_block, thr = std::min(b / 2, 1024), m = paley_m(b);
+        const float scale = (float)(1.0 / std::sqrt((double)b));
+        if (m) chk(cudaFuncSetAttribute(eva_paley_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)std::min<size_t>((size_t)b * sizeof(float), 232448)));
         for (int64_t r0 = 0; r0 < N && e == cudaSuccess; r0 += 65535) {
             const int rows = (int)std::min<int64_t>(65535, N - r0);
-            eva_hadamard_kernel<<<dim3((unsigned)(K / b), (unsigned)rows), thr, (size_t)b * sizeof(float), s>>>(
-                reinterpret_cast<const __half *>(w) + r0 * K, hsign, wrot + r0 * K, (int)K, b,
-                (float)(1.0 / std::sqrt((double)b)), 1);
+            if (m)
+                eva_paley_rows_kernel<<<dim3((unsigned)(K / b), (unsigned)rows), thr, (size_t)b * sizeof(float), s>>>(
+                    reinterpret_cast<const __half *>(w) + r0 * K, hsign, h28, wrot + r0 * K, (int)K, b, m, scale);
+            else
+                eva_hadamard_kernel<<<dim3((unsigned)(K / b), (unsigned)rows), thr, (size_t)b * sizeof(float), s>>>(
+                    reinterpret_cast<const __half *>(w) + r0 * K, hsign, wrot + r0 * K, (int)K, b, scale, 1);
             chk(cudaGetLastError());
         }
-    } else {
+    } else if (!d.hadamard_block) {
         eva_rows_to_f32_kernel<<<(unsigned)std::min<int64_t>(blocks_for(N * K, 256), 4096), 256, 0, s>>>(
             reinterpret_cast<const __half *>(w), wrot, N * K);
         chk(cudaGetLastError());
@@ -954,6 +1133,7 @@ eva_status_t eva_vq_quantize(const eva_quant_desc *desc, const void *w, const in
                             d.codebook_rows, d.residual_group, signs_out, reinterpret_cast<__half *>(alpha_out), s));
     int herr = 0;
     chk(cudaMemcpyAsync(&herr, err, sizeof(int), cudaMemcpyDeviceToHost, s));
+    if (h28) cudaFreeAsync(h28, s);
     chk(cudaFreeAsync(ws, s));
     chk(cudaStreamSynchronize(s));
     if (e != cudaSuccess) return cuda_status(e);

@@ -53,6 +53,8 @@ struct LookupParams {
     int rot_b;               // 0, or the rotation block b: x~ = s . (H_b x) / sqrt(b) is
                              // computed in the lookup kernel from fp16 x
     float rot_scale;         // 1 / sqrt(b), rounded to fp32
+    int rot_m;               // 0: Sylvester block; m: b = 28 m, H_b = H28 (x) H_m
+    const int8_t *h28;       // the order-28 Paley matrix [28][28] (rot_m != 0)
 #ifdef EVA_DEVICE_CHECKS
     // Debug build only: bounds of every buffer the kernel touches.  A
     // violating access is skipped and the first one is recorded.
@@ -383,10 +385,101 @@ __device__ __forceinline__ void fwht_warp256(float (&v)[8], int lane, int b) {
     }
 }
 
+// Rotation scratch in bytes per token: the b / 256 transformed sub-blocks of a
+// Sylvester block b > 256 or a Paley block with m <= 128; eight warps'
+// partial sums for a Paley block with m >= 256.
+__host__ __device__ __forceinline__ uint32_t rot_scratch_per_token(int b, int m) {
+    if (m >= 256) return 8u * kSliceK * 4u;
+    return (m > 0 || b > kSliceK) ? (uint32_t)b * 4u : 0u;
+}
+
+// Paley blocks b = 28 m (m a power of two >= 64, so every slice lies in one
+// block): x~ = s . (H_b^T x) / sqrt(b), H_b = H28 (x) H_m.  With k = a m + c
+// inside the block, (H_b^T x)[a m + c] = sum_a' H28[a'][a] (H_m x_a')[c].
+//  m <= 128: the H_m transforms of all 28 sub-blocks (warp FWHT stages below
+//    m over 256-input chunks) go to shared memory, then each output sums its
+//    28 terms in order a' = 0..27 -- the same operations, in the same order,
+//    as the standalone row kernel, so the values are bitwise equal;
+//  m >= 256: every 256-input chunk (a', c') is transformed by one warp and
+//    added with sign H28[a'][a] * sylvester(c', c) into that warp's partial
+//    sums of the slice's outputs; the eight partials are added in warp order.
+template <bool PAIR_T>
+__device__ __forceinline__ void stage_x_paley(const LookupParams &p, int s, int pr, int warp, int lane, int tid,
+                                              uint32_t x_off, uint32_t rot_off) {
+    constexpr int NTOK = PAIR_T ? 2 : 1;
+    const int b = p.rot_b, m = p.rot_m, ks = s * kSliceK;
+    const int blk0 = (ks / b) * b, kb = ks - blk0;       // block start, slice offset in the block
+    const uint32_t per_tok = rot_scratch_per_token(b, m);
+    if (m <= 128) {
+        const int nch = b / kSliceK;
+        for (int w = warp; w < NTOK * nch; w += kWarps) {
+            const int tk = w / nch, ch = w - tk * nch;
+            float v[8];
+            load_x8_f16(p, PAIR_T ? 2 * pr + tk : 0, blk0 + ch * kSliceK + 8 * lane, v);
+            fwht_warp256(v, lane, m);
+            const uint32_t off = rot_off + (uint32_t)tk * per_tok + (uint32_t)(ch * kSliceK + 8 * lane) * 4u;
+            if (!EVA_BAD_S(off) && !EVA_BAD_S(off + 28u)) {
+                *reinterpret_cast<float4 *>(eva_smem + off) = make_float4(v[0], v[1], v[2], v[3]);
+                *reinterpret_cast<float4 *>(eva_smem + off + 16) = make_float4(v[4], v[5], v[6], v[7]);
+            }
+        }
+        __syncthreads();
+        for (int e = tid; e < NTOK * kSliceK; e += kThreads) {
+            const int tk = e / kSliceK, i = e - tk * kSliceK;
+            const int a = (kb + i) / m, c = (kb + i) - a * m;
+            float acc = 0.f;
+            for (int a2 = 0; a2 < 28; ++a2) {
+                const uint32_t off = rot_off + (uint32_t)tk * per_tok + (uint32_t)(a2 * m + c) * 4u;
+                const float y = EVA_BAD_S(off) ? 0.f : *reinterpret_cast<const float *>(eva_smem + off);
+                acc = __ldg(p.h28 + a2 * 28 + a) > 0 ? acc + y : acc - y;
+            }
+            const uint32_t off = x_off + (uint32_t)(tk * kSliceK + i) * 4u;
+            if (!EVA_BAD_S(off)) *reinterpret_cast<float *>(eva_smem + off) = (float)p.hs[ks + i] * acc * p.rot_scale;
+        }
+        return;
+    }
+    const int a = kb / m, c = (kb - a * m) / kSliceK, cpm = m / kSliceK;   // 256-chunks per sub-block
+    const int nch = 28 * cpm;
+    for (int tk = 0; tk < NTOK; ++tk) {
+        float acc[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+        for (int ch = warp; ch < nch; ch += kWarps) {
+            const int a2 = ch / cpm, c2 = ch - a2 * cpm;
+            float v[8];
+            load_x8_f16(p, PAIR_T ? 2 * pr + tk : 0, blk0 + ch * kSliceK + 8 * lane, v);
+            fwht_warp256(v, lane, kSliceK);
+            const bool neg = (__ldg(p.h28 + a2 * 28 + a) < 0) != ((__popc((unsigned)(c2 & c)) & 1) != 0);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[j] = neg ? acc[j] - v[j] : acc[j] + v[j];
+        }
+        const uint32_t off = rot_off + (uint32_t)tk * per_tok + (uint32_t)(warp * kSliceK + 8 * lane) * 4u;
+        if (!EVA_BAD_S(off) && !EVA_BAD_S(off + 28u)) {
+            *reinterpret_cast<float4 *>(eva_smem + off) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            *reinterpret_cast<float4 *>(eva_smem + off + 16) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < NTOK * kSliceK; e += kThreads) {
+        const int tk = e / kSliceK, i = e - tk * kSliceK;
+        float acc = 0.f;
+        for (int w = 0; w < kWarps; ++w) {
+            const uint32_t off = rot_off + (uint32_t)tk * per_tok + (uint32_t)(w * kSliceK + i) * 4u;
+            acc += EVA_BAD_S(off) ? 0.f : *reinterpret_cast<const float *>(eva_smem + off);
+        }
+        const uint32_t off = x_off + (uint32_t)(tk * kSliceK + i) * 4u;
+        if (!EVA_BAD_S(off)) *reinterpret_cast<float *>(eva_smem + off) = (float)p.hs[ks + i] * acc * p.rot_scale;
+    }
+}
+
 template <bool PAIR_T>
 __device__ __forceinline__ void stage_x_rot(const LookupParams &p, int s, int pr, int warp, int lane, int tid,
                                             uint32_t x_off, uint32_t rot_off) {
     constexpr int NTOK = PAIR_T ? 2 : 1;
+    if (p.rot_m) {
+        stage_x_paley<PAIR_T>(p, s, pr, warp, lane, tid, x_off, rot_off);
+        return;
+    }
     const int b = p.rot_b, ks = s * kSliceK;
     if (b <= kSliceK) {
         // Whole blocks inside the slice: one warp per token.
@@ -655,7 +748,7 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
     const uint32_t stage_bytes_c = (uint32_t)((p.acc_tiles + p.Gs - 1) / p.Gs) * p.Gs * kTileRows * 2u * 4u;
     // Fused rotation scratch (b > 256): the b / 256 transformed sub-blocks of each token.
     const uint32_t ROT_OFF = (ACC_OFF + (uint32_t)p.acc_tiles * kTileRows * 2u * 4u + stage_bytes_c + 127u) & ~127u;
-    const uint32_t rot_bytes = (ROT && p.rot_b > kSliceK) ? (uint32_t)NTOK_C * (uint32_t)p.rot_b * 4u : 0u;
+    const uint32_t rot_bytes = ROT ? (uint32_t)NTOK_C * rot_scratch_per_token(p.rot_b, p.rot_m) : 0u;
     const uint32_t WIS_OFF = ROT_OFF + rot_bytes;
     const uint32_t bar = (uint32_t)__cvta_generic_to_shared(eva_smem + BAR_OFF);
     if (tid == 0 && staged > 0) {
@@ -977,6 +1070,43 @@ __global__ void __launch_bounds__(1024) eva_hadamard_kernel(const __half *__rest
     for (int i = threadIdx.x; i < b; i += blockDim.x) {
         const int k = blk * b + i;
         xt[(size_t)tok * K + k] = (float)hs[k] * sb[i] * scale;
+    }
+}
+
+// The Paley-block rotation of rows (weights in the quantizer; inputs in the
+// two-kernel route): grid (K / b, rows), b / 2 threads at most 1024, b floats
+// of shared memory.  Stages h < m of the fast transform inside every
+// m-sub-block, then out[a m + c] = sum_a' H28[a'][a] y[a' m + c] in order
+// a' = 0..27, times s / sqrt(b).
+__global__ void __launch_bounds__(1024) eva_paley_rows_kernel(const __half *__restrict__ x,
+                                                              const int8_t *__restrict__ hs,
+                                                              const int8_t *__restrict__ h28,
+                                                              float *__restrict__ xt, int K, int b, int m,
+                                                              float scale) {
+    float *sb = reinterpret_cast<float *>(eva_smem);
+    const int blk = blockIdx.x, tok = blockIdx.y;
+    const unsigned short *xb =
+        reinterpret_cast<const unsigned short *>(x) + (size_t)tok * K + (size_t)blk * b;
+    for (int i = threadIdx.x; i < b; i += blockDim.x) sb[i] = __half2float(__ushort_as_half(__ldcg(xb + i)));
+    for (int h = 1; h < m; h <<= 1) {
+        __syncthreads();
+        for (int i = threadIdx.x; i < b / 2; i += blockDim.x) {
+            const int lo = (i / h) * 2 * h + (i % h);
+            const float a = sb[lo], c = sb[lo + h];
+            sb[lo] = a + c;
+            sb[lo + h] = a - c;
+        }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < b; i += blockDim.x) {
+        const int a = i / m, c = i - a * m;
+        float acc = 0.f;
+        for (int a2 = 0; a2 < 28; ++a2) {
+            const float y = sb[a2 * m + c];
+            acc = h28[a2 * 28 + a] > 0 ? acc + y : acc - y;
+        }
+        const int k = blk * b + i;
+        xt[(size_t)tok * K + k] = (float)hs[k] * acc * scale;
     }
 }
 

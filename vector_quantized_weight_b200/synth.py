@@ -78,6 +78,16 @@ def _gemma_3bit():
     )
 
 
+def _gemma_3bit_order_k():
+    # The same layers with the rotation over the whole input dimension:
+    # 3584 = 28 * 128 and 14336 = 28 * 512, H_K = H28 (x) H_(K/28).
+    return (
+        LayerShape("gemma_3584x3584_rotK", 3584, 3584, residual_group=128, hadamard_block=3584),
+        LayerShape("gemma_14336x3584_rotK", 14336, 3584, residual_group=128, hadamard_block=3584),
+        LayerShape("gemma_3584x14336_rotK", 3584, 14336, residual_group=128, hadamard_block=14336),
+    )
+
+
 def _llama70b():
     return (
         LayerShape("l70b_8192x8192", 8192, 8192, codebook_rows=128),
@@ -97,6 +107,8 @@ CONFIGS = {
                          _gemma_3bit(), (1,), 3),
     "llama70b": Config("llama70b", "Llama-2-70B-shaped 2-bit linears, one codebook per 128 rows",
                        _llama70b(), (1, 8, 32), 4),
+    "gemma_3bit_rotK": Config("gemma_3bit_rotK", "Gemma-2-9B-shaped 3.125-bit linears, order-K (Paley x "
+                              "Sylvester) rotation", _gemma_3bit_order_k(), (1, 2), 5),
 }
 
 

@@ -142,13 +142,15 @@ eva_status_t validate_desc(const eva_vq_desc *d) {
 // mbarrier, the running sums of `tiles` row tiles, the cluster reduction
 // stage and, 128-byte aligned, the fused rotation's scratch (rotation blocks
 // b > 256: b floats per token) and the `staged` index units of the first slice.
-size_t lookup_smem(bool pair_t, bool resid, int tiles, int gs, int rot_b, int staged = 0) {
+size_t lookup_smem(bool pair_t, bool resid, int tiles, int gs, int rot_b, int s_total, int staged = 0) {
     const size_t tile_bytes = (size_t)kTileRows * 2 * 4;
     const size_t stage_tiles = (size_t)((tiles + gs - 1) / gs) * gs;   // reduction stage
     const size_t base = (size_t)kOcBytes + ((pair_t && resid) ? (size_t)kOcBytes : 0) +
                         (pair_t ? kXStageBytes : kXStageBytes / 2) + 128 + (size_t)tiles * tile_bytes +
                         stage_tiles * tile_bytes;
-    const size_t rot = rot_b ? (size_t)(pair_t ? 2 : 1) * rot_scratch_per_token(rot_b, paley_m(rot_b)) : 0;
+    const int ntok = pair_t ? 2 : 1;
+    const size_t xt = paley_m(rot_b) >= 256 ? (size_t)((s_total + gs - 1) / gs) * ntok * kSliceK * 4 : 0;
+    const size_t rot = rot_b ? xt + rot_scratch_bytes(rot_b, paley_m(rot_b), ntok) : 0;
     return ((base + 127) & ~(size_t)127) + rot + (size_t)staged * kUnitBytes;
 }
 
@@ -157,7 +159,7 @@ size_t lookup_smem(bool pair_t, bool resid, int tiles, int gs, int rot_b, int st
 // two CTAs per SM (this layer's and the next layer's early-launched one)
 // wherever the registers and the rest of the footprint allow it, else one.
 int staged_tiles(const eva_vq_linear *h, const void *fn, bool pair_t, bool resid, int tiles, int gs) {
-    const size_t base = lookup_smem(pair_t, resid, tiles, gs, h->desc.hadamard_block, 0);
+    const size_t base = lookup_smem(pair_t, resid, tiles, gs, h->desc.hadamard_block, h->S, 0);
     const size_t per_sm = (size_t)h->smem_per_sm, reserved = (size_t)h->smem_reserved;
     const size_t two = per_sm / 2 - reserved;
     const size_t one = std::min(per_sm - reserved, (size_t)h->smem_optin);
@@ -228,7 +230,7 @@ void plan_grid(eva_vq_linear *h, int pair_t) {
         // Capacity with one CTA per SM: the occupancy query counts CTA slots,
         // so ask with a footprint that leaves room for a single CTA per SM.
         const size_t smem_one = std::max(lookup_smem(pair_t, resid, (T + gt_min - 1) / gt_min, gs,
-                                                     h->desc.hadamard_block),
+                                                     h->desc.hadamard_block, S),
                                          (size_t)120 * 1024);
         const int clusters = max_active_clusters(fn, smem_one, gs);
         // One CTA of this layer per SM: no more clusters than P / gs either.
@@ -248,8 +250,8 @@ void plan_grid(eva_vq_linear *h, int pair_t) {
     }
     const int tiles = (T + pl.Gt - 1) / pl.Gt;
     pl.staged = staged_tiles(h, (const void *)fn, pair_t != 0, resid, tiles, pl.Gs);
-    pl.smem = lookup_smem(pair_t, resid, tiles, pl.Gs, h->desc.hadamard_block, pl.staged);
-    pl.smem_nostage = lookup_smem(pair_t, resid, tiles, pl.Gs, h->desc.hadamard_block, 0);
+    pl.smem = lookup_smem(pair_t, resid, tiles, pl.Gs, h->desc.hadamard_block, S, pl.staged);
+    pl.smem_nostage = lookup_smem(pair_t, resid, tiles, pl.Gs, h->desc.hadamard_block, S, 0);
     h->plan[pair_t] = pl;
 }
 

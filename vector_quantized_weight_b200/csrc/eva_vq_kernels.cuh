@@ -385,10 +385,98 @@ __device__ __forceinline__ void fwht_warp256(float (&v)[8], int lane, int b) {
     }
 }
 
+// Scratch of the fused rotation, in bytes: the transformed 256-input chunks of
+// one block for every token (Sylvester b > 256, Paley m <= 128), or eight
+// warps' partial sums of up to four slices (Paley m >= 256, one token at a
+// time).
+__host__ __device__ __forceinline__ uint32_t rot_scratch_bytes(int b, int m, int ntok) {
+    if (m >= 256) return 8u * 4u * kSliceK * 4u;
+    return (m > 0 || b > kSliceK) ? (uint32_t)ntok * (uint32_t)b * 4u : 0u;
+}
+
+// Paley blocks with m >= 256 (b >= 7168: a block holds 28 or more slices):
+// the rotated input x~ = s . (H_b^T x) / sqrt(b), H_b = H28 (x) H_m, of every
+// slice s0 .. s1-1 of this CTA, for the pair's tokens, into xt
+// [slice][token][256] (fp32).  With k = a m + c inside a block,
+// (H_b^T x)[a m + c] = sum_a' H28[a'][a] (H_m x_a')[c]; per group of up to
+// four slices of one block and per token, each warp transforms 256-input
+// chunks (a', c') once and adds them, with sign H28[a'][a] sylvester(c', c),
+// into partial sums of every slice of the group; the partials are added in
+// warp order.
+template <bool PAIR_T>
+__device__ __forceinline__ void stage_x_rot_all(const LookupParams &p, int s0, int s1, int pr, int warp, int lane,
+                                                int tid, uint32_t xt_off, uint32_t scr_off) {
+    constexpr int NTOK = PAIR_T ? 2 : 1;
+    const int b = p.rot_b, m = p.rot_m, nsl = s1 - s0;
+    auto finish = [&](int sl, int tk, int i, float acc) {
+        const int k = (s0 + sl) * kSliceK + i;
+        const uint32_t off = xt_off + (uint32_t)((sl * NTOK + tk) * kSliceK + i) * 4u;
+        if (!EVA_BAD_S(off)) *reinterpret_cast<float *>(eva_smem + off) = (k < p.K ? (float)p.hs[k] : 0.f) * acc * p.rot_scale;
+    };
+    auto tok_of = [&](int tk) { return PAIR_T ? 2 * pr + tk : 0; };
+    {
+        const int cpm = m / kSliceK, nch = 28 * cpm;
+        for (int g0 = 0; g0 < nsl;) {
+            // up to four consecutive slices inside one block
+            const int blk = (s0 + g0) * kSliceK / b;
+            int gn = 1;
+            while (gn < 4 && g0 + gn < nsl && (s0 + g0 + gn) * kSliceK / b == blk) ++gn;
+            const int blk0 = blk * b;
+            for (int tk = 0; tk < NTOK; ++tk) {
+                float acc[4][8];
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) acc[j][e] = 0.f;
+                for (int ch = warp; ch < nch; ch += kWarps) {
+                    const int a2 = ch / cpm, c2 = ch - a2 * cpm;
+                    float v[8];
+                    load_x8_f16(p, tok_of(tk), blk0 + ch * kSliceK + 8 * lane, v);
+                    fwht_warp256(v, lane, kSliceK);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        if (j >= gn) break;
+                        const int kb = (s0 + g0 + j) * kSliceK - blk0;
+                        const int a = kb / m, c = (kb - a * m) / kSliceK;
+                        const bool neg = (__ldg(p.h28 + a2 * 28 + a) < 0) != ((__popc((unsigned)(c2 & c)) & 1) != 0);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) acc[j][e] = neg ? acc[j][e] - v[e] : acc[j][e] + v[e];
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    if (j >= gn) break;
+                    const uint32_t off = scr_off + (uint32_t)((warp * 4 + j) * kSliceK + 8 * lane) * 4u;
+                    if (!EVA_BAD_S(off) && !EVA_BAD_S(off + 28u)) {
+                        *reinterpret_cast<float4 *>(eva_smem + off) = make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
+                        *reinterpret_cast<float4 *>(eva_smem + off + 16) = make_float4(acc[j][4], acc[j][5], acc[j][6], acc[j][7]);
+                    }
+                }
+                __syncthreads();
+                for (int e = tid; e < gn * kSliceK; e += kThreads) {
+                    const int j = e / kSliceK, i = e - j * kSliceK;
+                    float sum = 0.f;
+                    for (int w = 0; w < kWarps; ++w) {
+                        const uint32_t off = scr_off + (uint32_t)((w * 4 + j) * kSliceK + i) * 4u;
+                        sum += EVA_BAD_S(off) ? 0.f : *reinterpret_cast<const float *>(eva_smem + off);
+                    }
+                    finish(g0 + j, tk, i, sum);
+                }
+                __syncthreads();
+            }
+            g0 += gn;
+        }
+        return;
+    }
+}
+
+// Per-slice form of the rotation (one slice's outputs at a time): the
+// blocks' transforms are redone for every slice, which costs nothing extra
+// when a CTA has one slice or the blocks are small.
 // Rotation scratch in bytes per token: the b / 256 transformed sub-blocks of a
 // Sylvester block b > 256 or a Paley block with m <= 128; eight warps'
 // partial sums for a Paley block with m >= 256.
-__host__ __device__ __forceinline__ uint32_t rot_scratch_per_token(int b, int m) {
+__host__ __device__ __forceinline__ uint32_t rot_scratch_per_token_slice(int b, int m) {
     if (m >= 256) return 8u * kSliceK * 4u;
     return (m > 0 || b > kSliceK) ? (uint32_t)b * 4u : 0u;
 }
@@ -400,17 +488,15 @@ __host__ __device__ __forceinline__ uint32_t rot_scratch_per_token(int b, int m)
 //    m over 256-input chunks) go to shared memory, then each output sums its
 //    28 terms in order a' = 0..27 -- the same operations, in the same order,
 //    as the standalone row kernel, so the values are bitwise equal;
-//  m >= 256: every 256-input chunk (a', c') is transformed by one warp and
-//    added with sign H28[a'][a] * sylvester(c', c) into that warp's partial
-//    sums of the slice's outputs; the eight partials are added in warp order.
+//  (m >= 256 takes stage_x_rot_all, which serves all of a CTA's slices.)
 template <bool PAIR_T>
 __device__ __forceinline__ void stage_x_paley(const LookupParams &p, int s, int pr, int warp, int lane, int tid,
                                               uint32_t x_off, uint32_t rot_off) {
     constexpr int NTOK = PAIR_T ? 2 : 1;
     const int b = p.rot_b, m = p.rot_m, ks = s * kSliceK;
     const int blk0 = (ks / b) * b, kb = ks - blk0;       // block start, slice offset in the block
-    const uint32_t per_tok = rot_scratch_per_token(b, m);
-    if (m <= 128) {
+    const uint32_t per_tok = rot_scratch_per_token_slice(b, m);
+    {
         const int nch = b / kSliceK;
         for (int w = warp; w < NTOK * nch; w += kWarps) {
             const int tk = w / nch, ch = w - tk * nch;
@@ -437,38 +523,6 @@ __device__ __forceinline__ void stage_x_paley(const LookupParams &p, int s, int 
             if (!EVA_BAD_S(off)) *reinterpret_cast<float *>(eva_smem + off) = (float)p.hs[ks + i] * acc * p.rot_scale;
         }
         return;
-    }
-    const int a = kb / m, c = (kb - a * m) / kSliceK, cpm = m / kSliceK;   // 256-chunks per sub-block
-    const int nch = 28 * cpm;
-    for (int tk = 0; tk < NTOK; ++tk) {
-        float acc[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-        for (int ch = warp; ch < nch; ch += kWarps) {
-            const int a2 = ch / cpm, c2 = ch - a2 * cpm;
-            float v[8];
-            load_x8_f16(p, PAIR_T ? 2 * pr + tk : 0, blk0 + ch * kSliceK + 8 * lane, v);
-            fwht_warp256(v, lane, kSliceK);
-            const bool neg = (__ldg(p.h28 + a2 * 28 + a) < 0) != ((__popc((unsigned)(c2 & c)) & 1) != 0);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) acc[j] = neg ? acc[j] - v[j] : acc[j] + v[j];
-        }
-        const uint32_t off = rot_off + (uint32_t)tk * per_tok + (uint32_t)(warp * kSliceK + 8 * lane) * 4u;
-        if (!EVA_BAD_S(off) && !EVA_BAD_S(off + 28u)) {
-            *reinterpret_cast<float4 *>(eva_smem + off) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-            *reinterpret_cast<float4 *>(eva_smem + off + 16) = make_float4(acc[4], acc[5], acc[6], acc[7]);
-        }
-    }
-    __syncthreads();
-    for (int e = tid; e < NTOK * kSliceK; e += kThreads) {
-        const int tk = e / kSliceK, i = e - tk * kSliceK;
-        float acc = 0.f;
-        for (int w = 0; w < kWarps; ++w) {
-            const uint32_t off = rot_off + (uint32_t)tk * per_tok + (uint32_t)(w * kSliceK + i) * 4u;
-            acc += EVA_BAD_S(off) ? 0.f : *reinterpret_cast<const float *>(eva_smem + off);
-        }
-        const uint32_t off = x_off + (uint32_t)(tk * kSliceK + i) * 4u;
-        if (!EVA_BAD_S(off)) *reinterpret_cast<float *>(eva_smem + off) = (float)p.hs[ks + i] * acc * p.rot_scale;
     }
 }
 
@@ -746,9 +800,12 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
     // copy into shared memory, completing on an mbarrier.
     const int staged = min(p.wi_staged, t1 - t0);
     const uint32_t stage_bytes_c = (uint32_t)((p.acc_tiles + p.Gs - 1) / p.Gs) * p.Gs * kTileRows * 2u * 4u;
-    // Fused rotation scratch (b > 256): the b / 256 transformed sub-blocks of each token.
+    // Fused rotation: x~ of all this CTA's slices [ceil(S / Gs)][tokens][256]
+    // fp32, then the rotation's scratch.
     const uint32_t ROT_OFF = (ACC_OFF + (uint32_t)p.acc_tiles * kTileRows * 2u * 4u + stage_bytes_c + 127u) & ~127u;
-    const uint32_t rot_bytes = ROT ? (uint32_t)NTOK_C * rot_scratch_per_token(p.rot_b, p.rot_m) : 0u;
+    const bool rot_all = ROT && p.rot_m >= 256;   // Paley m >= 256: all slices at once
+    const uint32_t xt_bytes = rot_all ? (uint32_t)((p.S + p.Gs - 1) / p.Gs) * NTOK_C * kSliceK * 4u : 0u;
+    const uint32_t rot_bytes = ROT ? xt_bytes + rot_scratch_bytes(p.rot_b, p.rot_m, NTOK_C) : 0u;
     const uint32_t WIS_OFF = ROT_OFF + rot_bytes;
     const uint32_t bar = (uint32_t)__cvta_generic_to_shared(eva_smem + BAR_OFF);
     if (tid == 0 && staged > 0) {
@@ -822,10 +879,13 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
     const float *stage = reinterpret_cast<const float *>(eva_smem + STAGE_OFF);
     const uint32_t stage_addr = (uint32_t)__cvta_generic_to_shared(eva_smem + STAGE_OFF);
     for (int pr = 0; pr < npairs; ++pr) {
-
         for (int s = s0; s < s1; ++s) {
-            if constexpr (ROT) stage_x_rot<PAIR_T>(p, s, pr, warp, lane, tid, X_OFF, ROT_OFF);
-            else stage_x<PAIR_T>(p, s, pr, warp, lane, X_OFF);
+            const uint32_t x_off = rot_all ? ROT_OFF + (uint32_t)((s - s0) * NTOK_C) * kSliceK * 4u : X_OFF;
+            if constexpr (ROT) {
+                if (!rot_all) stage_x_rot<PAIR_T>(p, s, pr, warp, lane, tid, X_OFF, ROT_OFF);
+            } else {
+                stage_x<PAIR_T>(p, s, pr, warp, lane, X_OFF);
+            }
             for (int cb = cb_first; cb <= cb_last; ++cb) {
                 // This warp's tiles that use codebook cb: the index range [i0, i1).
                 int i0 = 0, i1 = ntw;
@@ -853,10 +913,17 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
                         if (!EVA_BAD_G(BUF_WI, up, 16) && !EVA_BAD_G(BUF_WI, up + 512, 16)) ldg_unit(up, nb[d][0], nb[d][1]);
                     }
                 }
+                // Paley blocks with m >= 256: x~ of every slice of this CTA at
+                // once (each chunk transformed once), after the first index
+                // loads are in flight; the slices then read their part of it.
+                if constexpr (ROT) {
+                    if (rot_all && s == s0 && cb == cb_first)
+                        stage_x_rot_all<PAIR_T>(p, s0, s1, pr, warp, lane, tid, ROT_OFF, ROT_OFF + xt_bytes);
+                }
                 __syncthreads();  // x~ staged, accumulator cleared, previous image consumed
                 EVA_STAMP(2);
-                build_oc<PAIR_T, NAIVE>(p, warp, g, q, bfrag, X_OFF);
-                if (RESID && cb == cb_first) build_sign_table<PAIR_T>(p, warp, lane, T_OFF, X_OFF);
+                build_oc<PAIR_T, NAIVE>(p, warp, g, q, bfrag, x_off);
+                if (RESID && cb == cb_first) build_sign_table<PAIR_T>(p, warp, lane, T_OFF, x_off);
                 __syncthreads();
                 EVA_STAMP(3);
                 if (staged > 0 && !wi_ready) {

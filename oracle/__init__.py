@@ -33,7 +33,7 @@ def build(force: bool = False) -> str:
 
 class _Desc(ctypes.Structure):
     _fields_ = [("N", ctypes.c_int), ("K", ctypes.c_int), ("d", ctypes.c_int),
-                ("ncent", ctypes.c_int), ("codebook_rows", ctypes.c_int),
+                ("ncent", ctypes.c_int), ("index_bits", ctypes.c_int), ("codebook_rows", ctypes.c_int),
                 ("residual_group", ctypes.c_int), ("hadamard_block", ctypes.c_int)]
 
 
@@ -100,18 +100,20 @@ def hadamard(x, hsign, b: int) -> np.ndarray:
     return out
 
 
-def _desc(N, K, d, ncent, codebook_rows, residual_group, hadamard_block):
-    return _Desc(int(N), int(K), int(d), int(ncent), int(codebook_rows),
+def _desc(N, K, d, ncent, codebook_rows, residual_group, hadamard_block, index_bits=8):
+    return _Desc(int(N), int(K), int(d), int(ncent), int(index_bits), int(codebook_rows),
                  int(residual_group), int(hadamard_block))
 
 
-def _prep(wc, wi, signs, alpha, hsign, x, codebook_rows, residual_group, hadamard_block):
+def _prep(wc, wi, signs, alpha, hsign, x, codebook_rows, residual_group, hadamard_block, index_bits=8):
     wc16 = _c16(wc)
     if wc16.ndim == 2:
         wc16 = wc16[None]
     G, ncent, d = wc16.shape
     wi8 = np.ascontiguousarray(wi, dtype=np.uint8)
     N, J = wi8.shape
+    if index_bits == 4:            # two indices per byte
+        J *= 2
     x16 = _c16(np.atleast_2d(x))
     B, K = x16.shape
     if J * d != K:
@@ -121,15 +123,16 @@ def _prep(wc, wi, signs, alpha, hsign, x, codebook_rows, residual_group, hadamar
     sg = None if signs is None else np.ascontiguousarray(signs, dtype=np.uint8)
     al = _c16(alpha)
     hs = None if hsign is None else np.ascontiguousarray(hsign, dtype=np.int8)
-    desc = _desc(N, K, d, ncent, codebook_rows, residual_group, hadamard_block)
+    desc = _desc(N, K, d, ncent, codebook_rows, residual_group, hadamard_block, index_bits)
     return desc, wc16, wi8, sg, al, hs, x16, B, N
 
 
 def linear(wc, wi, x, *, signs=None, alpha=None, hsign=None, codebook_rows=0,
-           residual_group=0, hadamard_block=0, nthreads=1) -> np.ndarray:
-    """y [B][N] float64: the dequantised-weight product (the plain definition)."""
+           residual_group=0, hadamard_block=0, nthreads=1, index_bits=8) -> np.ndarray:
+    """y [B][N] float64: the dequantised-weight product (the plain definition).
+    index_bits = 4: wi is packed two indices per byte ([N][K/8])."""
     desc, wc16, wi8, sg, al, hs, x16, B, N = _prep(
-        wc, wi, signs, alpha, hsign, x, codebook_rows, residual_group, hadamard_block)
+        wc, wi, signs, alpha, hsign, x, codebook_rows, residual_group, hadamard_block, index_bits)
     y = np.empty((B, N), np.float64)
     rc = _load().vq_oracle_linear(ctypes.byref(desc), _ptr(wc16), _ptr(wi8), _ptr(sg), _ptr(al),
                                   _ptr(hs), _ptr(x16), B, _ptr(y), int(nthreads))
@@ -139,10 +142,10 @@ def linear(wc, wi, x, *, signs=None, alpha=None, hsign=None, codebook_rows=0,
 
 
 def lookup_form(wc, wi, x, *, signs=None, alpha=None, hsign=None, codebook_rows=0,
-                residual_group=0, hadamard_block=0):
+                residual_group=0, hadamard_block=0, index_bits=8):
     """(y, sum|W x~|) [B][N] float64 via the output-codebook two-step form."""
     desc, wc16, wi8, sg, al, hs, x16, B, N = _prep(
-        wc, wi, signs, alpha, hsign, x, codebook_rows, residual_group, hadamard_block)
+        wc, wi, signs, alpha, hsign, x, codebook_rows, residual_group, hadamard_block, index_bits)
     y = np.empty((B, N), np.float64)
     absy = np.empty((B, N), np.float64)
     rc = _load().vq_oracle_lookup_form(ctypes.byref(desc), _ptr(wc16), _ptr(wi8), _ptr(sg),
@@ -172,7 +175,7 @@ def layer_linear(layer, x, nthreads=1) -> np.ndarray:
     s = layer.shape
     return linear(layer.wc, layer.wi, x, signs=layer.signs, alpha=layer.alpha, hsign=layer.hsign,
                   codebook_rows=s.codebook_rows, residual_group=s.residual_group,
-                  hadamard_block=s.hadamard_block, nthreads=nthreads)
+                  hadamard_block=s.hadamard_block, nthreads=nthreads, index_bits=s.index_bits)
 
 
 # ------------------------------------------------------------------ quantizer

@@ -226,7 +226,8 @@ int vq_oracle_hadamard(const uint16_t *x, const int8_t *hsign, int B, int K, int
 }
 
 typedef struct {
-    int N, K, d, ncent;          /* ncent = 2^n centroids per codebook */
+    int N, K, d, ncent;          /* ncent <= 2^n centroids per codebook */
+    int index_bits;              /* n: 8 (one byte per index) or 4 (two per byte) */
     int codebook_rows;           /* 0: one codebook; else rows per codebook */
     int residual_group;          /* 0: no residual */
     int hadamard_block;          /* 0: no rotation */
@@ -235,12 +236,25 @@ typedef struct {
 static int check_desc(const vq_oracle_desc *d)
 {
     if (!d || d->N <= 0 || d->K <= 0 || d->d <= 0 || d->K % d->d) return -1;
-    if (d->ncent <= 0 || d->ncent > 256) return -1;
+    if (d->index_bits != 8 && d->index_bits != 4) return -1;
+    if (d->ncent <= 0 || d->ncent > (1 << d->index_bits)) return -1;
+    if (d->index_bits == 4 && (d->K / d->d) % 2) return -1;
     if (d->codebook_rows < 0 || (d->codebook_rows && d->N % d->codebook_rows)) return -1;
     if (d->residual_group < 0 || (d->residual_group && (d->K % d->residual_group || d->K % 8)))
         return -1;
     if (d->hadamard_block < 0 || (d->hadamard_block && d->K % d->hadamard_block)) return -1;
     return 0;
+}
+
+/* Index WI[o][j].  n = 8: byte j of row o ([N][K/d]).  n = 4: the indices are
+ * packed two per byte ([N][K/(2d)]), sub-vector j in byte j/2, the even one in
+ * the low nibble (LSB first, like the sign bits). */
+static int index_of(const vq_oracle_desc *d, const uint8_t *wi, int o, int j)
+{
+    const int J = d->K / d->d;
+    if (d->index_bits == 8) return wi[(size_t)o * (size_t)J + (size_t)j];
+    const uint8_t byte = wi[(size_t)o * (size_t)(J / 2) + (size_t)(j / 2)];
+    return (byte >> (4 * (j & 1))) & 15;
 }
 
 /* Codebook index of output row o. */
@@ -265,7 +279,7 @@ static void dequant_row(const vq_oracle_desc *d, const uint16_t *wc, const uint8
     int g = group_of_row(d, o);
     const uint16_t *cb = wc + (size_t)g * (size_t)d->ncent * (size_t)d->d;
     for (int k = 0; k < d->K; ++k) {
-        int c = wi[(size_t)o * (size_t)J + (size_t)(k / d->d)];
+        int c = index_of(d, wi, o, k / d->d);
         wrow[k] = vq_oracle_f16_to_f64(cb[(size_t)c * (size_t)d->d + (size_t)(k % d->d)]);
     }
     if (d->residual_group) {
@@ -280,9 +294,9 @@ static void dequant_row(const vq_oracle_desc *d, const uint16_t *wc, const uint8
 
 static int check_indices(const vq_oracle_desc *d, const uint8_t *wi)
 {
-    int64_t n = (int64_t)d->N * (d->K / d->d);
-    for (int64_t i = 0; i < n; ++i)
-        if (wi[i] >= d->ncent) return -4;
+    for (int o = 0; o < d->N; ++o)
+        for (int j = 0; j < d->K / d->d; ++j)
+            if (index_of(d, wi, o, j) >= d->ncent) return -4;
     return 0;
 }
 
@@ -384,7 +398,7 @@ int vq_oracle_lookup_form(const vq_oracle_desc *desc, const uint16_t *wc, const 
         for (int t = 0; t < B; ++t) {
             double acc = 0.0;
             for (int j = 0; j < J; ++j) {
-                int c = wi[(size_t)o * J + j];
+                int c = index_of(desc, wi, o, j);
                 acc += oc[(((size_t)g * B + t) * J + j) * nc + c];
             }
             if (desc->residual_group) {

@@ -460,6 +460,36 @@ def pin_paley_rotation_pairs(orc, seed=18):
     assert np.allclose(lhs, rhs, rtol=1e-5, atol=1e-4), np.abs(lhs - rhs).max()
 
 
+# ------------------------------------------------- 4-bit (16-centroid) indices
+
+def pin_factorisation_4bit(orc, seed=19):
+    """16 centroids, indices packed two per byte (the even sub-vector in the
+    low nibble): a dense integer weight rebuilt from its codebook and packed
+    by plain integer arithmetic gives W x exactly, in both oracle forms, with
+    one shared codebook and with one per 8 rows; and a byte 0x21 holds the
+    indices (1, 2) in sub-vector order."""
+    rng = np.random.default_rng(seed)
+    N, K = 16, 64
+    for cbr in (0, 8):
+        G = N // cbr if cbr else 1
+        wc = rng.integers(-3, 4, size=(G, 16, 4)).astype(np.float16)
+        idx = rng.integers(0, 16, size=(N, K // 4))
+        g = (np.arange(N) // cbr) if cbr else np.zeros(N, int)
+        W = wc.astype(np.float64)[g[:, None], idx].reshape(N, K)
+        packed = (idx[:, 0::2] + 16 * idx[:, 1::2]).astype(np.uint8)
+        x = rng.integers(-3, 4, size=(2, K)).astype(np.float16)
+        ref = x.astype(np.float64) @ W.T
+        assert np.array_equal(orc.linear(wc, packed, x, codebook_rows=cbr, index_bits=4), ref)
+        yl, _ = orc.lookup_form(wc, packed, x, codebook_rows=cbr, index_bits=4)
+        assert np.array_equal(yl, ref)
+    wc = np.zeros((16, 4), np.float16)
+    wc[1] = [1, 0, 0, 0]
+    wc[2] = [0, 0, 0, 10]
+    x = np.arange(1, 9, dtype=np.float16)[None]          # K = 8: two sub-vectors
+    y = orc.linear(wc, np.array([[0x21]], np.uint8), x, index_bits=4)
+    assert y[0, 0] == 1 * 1 + 10 * 8                     # sub-vector 0 -> centroid 1, 1 -> 2
+
+
 ALL_PINS = [
     pin_golden_vq, pin_golden_residual, pin_golden_hadamard, pin_f16_decode,
     pin_hadamard_scipy, pin_factorisation, pin_factorisation_residual, pin_rotation_composite,
@@ -467,5 +497,5 @@ ALL_PINS = [
     pin_residual_unit_inputs, pin_hadamard_orthogonal, pin_lookup_identity, pin_batch_rows,
     pin_optimal_alpha, pin_kmeans_assign_scipy, pin_kmeans_sklearn, pin_quantize_exact_recovery,
     pin_quantize_rotation, pin_residual_identity, pin_paley_hadamard, pin_paley_kronecker,
-    pin_paley_rotation_pairs,
+    pin_paley_rotation_pairs, pin_factorisation_4bit,
 ]

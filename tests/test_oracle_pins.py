@@ -50,7 +50,9 @@ class _Mutant:
 MUTATIONS = {
     "sign_bit_msb_first": ("((byte >> (k % 8)) & 1)", "((byte >> (7 - k % 8)) & 1)"),
     "sign_polarity": ("? 1.0 : -1.0;\n}", "? -1.0 : 1.0;\n}"),
-    "subvector_strided": ("(size_t)(k / d->d)]", "(size_t)(k % J)]"),
+    "subvector_strided": ("int c = index_of(d, wi, o, k / d->d);", "int c = index_of(d, wi, o, k % (d->K / d->d));"),
+    "nibble_order_swapped": ("return (byte >> (4 * (j & 1))) & 15;", "return (byte >> (4 * (1 - (j & 1)))) & 15;"),
+    "nibble_byte_strided": ("(size_t)(J / 2) + (size_t)(j / 2)];", "(size_t)(J / 2) + (size_t)(j % (J / 2))];"),
     "centroid_component_reversed": ("(size_t)(k % d->d)]", "(size_t)(d->d - 1 - k % d->d)]"),
     "codebook_group_modulo": ("return d->codebook_rows ? o / d->codebook_rows : 0;",
                               "return d->codebook_rows ? o % (d->N / d->codebook_rows) : 0;"),

@@ -39,6 +39,7 @@ class LayerShape:
     codebook_rows: int = 0      # 0: one shared codebook; 128: one per 128 output rows
     residual_group: int = 0     # 0: no sign residual; 128: signs + alpha per 128 inputs
     hadamard_block: int = 0     # 0: no rotation; else block size b of the rotation
+    index_bits: int = 8         # 8: one index byte per sub-vector; 4: 16 centroids, two per byte
 
     @property
     def J(self) -> int:
@@ -47,6 +48,10 @@ class LayerShape:
     @property
     def G(self) -> int:
         return self.N // self.codebook_rows if self.codebook_rows else 1
+
+    @property
+    def ncent(self) -> int:
+        return 1 << self.index_bits
 
 
 @dataclass(frozen=True)
@@ -131,8 +136,10 @@ class LayerData:
 def make_layer(shape: LayerShape, seed: int, *, alpha_signed: bool = False) -> LayerData:
     """Draw the weights of one layer. Order: WC, WI, signs, alpha, hsign."""
     rng = np.random.default_rng(seed)
-    wc = rng.normal(0.0, 0.02, size=(shape.G, 256, shape.d)).astype(np.float16)
-    wi = rng.integers(0, 256, size=(shape.N, shape.J), dtype=np.uint8)
+    wc = rng.normal(0.0, 0.02, size=(shape.G, shape.ncent, shape.d)).astype(np.float16)
+    wi = rng.integers(0, shape.ncent, size=(shape.N, shape.J), dtype=np.uint8)
+    if shape.index_bits == 4:       # packed: sub-vector 2t in the low nibble of byte t
+        wi = pack_nibbles(wi)
     signs = alpha = hsign = None
     if shape.residual_group:
         signs = rng.integers(0, 256, size=(shape.N, shape.K // 8), dtype=np.uint8)
@@ -143,6 +150,12 @@ def make_layer(shape: LayerShape, seed: int, *, alpha_signed: bool = False) -> L
     if shape.hadamard_block:
         hsign = (rng.integers(0, 2, size=shape.K) * 2 - 1).astype(np.int8)
     return LayerData(shape, wc, wi, signs, alpha, hsign, seed)
+
+
+def pack_nibbles(idx: np.ndarray) -> np.ndarray:
+    """[N][J] indices < 16 -> [N][J/2] bytes, even sub-vector in the low nibble."""
+    idx = np.asarray(idx, dtype=np.uint8)
+    return (idx[:, 0::2] | (idx[:, 1::2] << 4)).astype(np.uint8)
 
 
 def make_x(K: int, B: int, seed: int) -> np.ndarray:

@@ -193,7 +193,7 @@ def cpu_baseline(shape, B, seed, seconds):
 
 
 def stream_bytes(shape, B):
-    wi = shape.N * shape.J
+    wi = shape.N * shape.J * shape.index_bits // 8
     sg = shape.N * shape.K // 8 if shape.residual_group else 0
     al = shape.N * (shape.K // shape.residual_group) * 2 if shape.residual_group else 0
     return wi + sg + al + 2 * B * shape.K

@@ -67,7 +67,10 @@ typedef struct {
     int32_t N;               /* output features, >= 1                                   */
     int32_t K;               /* input features, multiple of d (and of 128 with residual) */
     int32_t d;               /* sub-vector length; 4 is the only supported value        */
-    int32_t index_bits;      /* n; 8 is the only supported value (256 centroids)        */
+    int32_t index_bits;      /* n: 8 (256 centroids, one byte per index) or 4 (16
+                                centroids, two indices per byte: wi is [N][K/8], the even
+                                sub-vector in the low nibble; one shared codebook, no
+                                rotation, K a multiple of 8)                             */
     int32_t codebook_rows;   /* 0: one shared codebook; R > 0: codebook g serves rows
                                 [R g, R g + R); R must be a multiple of 16 dividing N    */
     int32_t residual_group;  /* 0: no sign residual; 128: signs + one alpha per 128 k   */
@@ -87,8 +90,9 @@ typedef struct eva_vq_linear *eva_vq_linear_t;
  * memory; the copies are enqueued on `stream`, and the caller's buffers may
  * be released once `stream` has passed this call.  All pointers are device
  * pointers (16-byte aligned):
- *   wc     fp16 [G][256][d], G = codebook_rows ? N / codebook_rows : 1
- *   wi     u8   [N][K/d], canonical row-major, WI[o][j] = centroid of row o, sub-vector j
+ *   wc     fp16 [G][2^n][d], G = codebook_rows ? N / codebook_rows : 1, n = index_bits
+ *   wi     u8   [N][K/d], canonical row-major, WI[o][j] = centroid of row o, sub-vector j;
+ *          4-bit indices: u8 [N][K/(2d)], WI[o][j] in byte j/2, bits 4 (j mod 2) .. +3
  *   signs  u8   [N][K/8], bit i of byte m is sigma[o][8m+i] (1: +1, 0: -1); NULL unless residual
  *   alpha  fp16 [N][K/residual_group]; NULL unless residual
  *   hsign  int8 [K], entries +1 or -1; NULL unless hadamard_block

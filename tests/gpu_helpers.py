@@ -28,7 +28,7 @@ def sub_layer_oracle(layer, x, rows, nthreads=8):
     alpha = None if layer.alpha is None else layer.alpha[rows]
     return oracle.linear(wc, wi, x, signs=signs, alpha=alpha, hsign=layer.hsign, codebook_rows=cbr,
                          residual_group=s.residual_group, hadamard_block=s.hadamard_block,
-                         nthreads=nthreads)
+                         nthreads=nthreads, index_bits=s.index_bits)
 
 
 def sample_rows(N, codebook_rows=0, n=256, seed=0):

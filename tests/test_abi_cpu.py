@@ -56,7 +56,9 @@ def _create(desc, wc=0x1000, wi=0x2000, signs=None, alpha=None, hsign=None):
 
 @pytest.mark.parametrize("kw,expect", [
     (dict(d=3), eva_vq.EVA_ERR_UNSUPPORTED),
-    (dict(index_bits=4), eva_vq.EVA_ERR_UNSUPPORTED),
+    (dict(index_bits=6), eva_vq.EVA_ERR_UNSUPPORTED),
+    (dict(index_bits=4, codebook_rows=16), eva_vq.EVA_ERR_UNSUPPORTED),   # 4-bit: one shared codebook
+    (dict(index_bits=4, K=516), eva_vq.EVA_ERR_INVALID_ARG),
     (dict(N=0), eva_vq.EVA_ERR_INVALID_ARG),
     (dict(K=510), eva_vq.EVA_ERR_INVALID_ARG),
     (dict(codebook_rows=100), eva_vq.EVA_ERR_INVALID_ARG),
@@ -112,7 +114,7 @@ def test_kernels_do_not_spill():
     out = subprocess.run(cmd, capture_output=True, text=True, check=True).stderr
     blocks = re.findall(r"Function properties for (\S*eva_\w+_kernel\S*)\n\s*(\d+) bytes stack frame, "
                         r"(\d+) bytes spill stores, (\d+) bytes spill loads", out)
-    assert sum("eva_lookup_kernel" in b[0] for b in blocks) == 16, out
+    assert sum("eva_lookup_kernel" in b[0] for b in blocks) == 20, out
     assert sum("eva_dequant_kernel" in b[0] for b in blocks) == 4, out
     assert sum("eva_kmeans_assign_kernel" in b[0] for b in blocks) == 2, out
     for name, stack, st, ld in blocks:
@@ -167,3 +169,36 @@ def test_create_accepts_order_k_rotation_descriptor():
         pytest.skip("a device is present")
     d = _desc(K=3584, hadamard_block=3584, residual_group=128)
     assert _create(d, signs=0x3000, alpha=0x4000, hsign=0x5000) == eva_vq.EVA_ERR_NO_DEVICE
+
+
+def test_unit_layouts_are_bijections():
+    """The repack layouts (host-compilable header): every (row, sub-vector) of
+    a unit appears exactly once, for byte indices and for 4-bit indices, and
+    the 4-bit inverse undoes the forward map."""
+    src = r"""
+#include <cstdio>
+#define __host__
+#define __device__
+#define __forceinline__ inline
+#include "eva_vq_layout.cuh"
+using namespace eva;
+int main() {
+    int bad = 0, seen8[16][64] = {{0}}, seen4[16][64] = {{0}};
+    for (int b = 0; b < kUnitBytes; ++b) { int r, j; wi_unit_pos(b, r, j); seen8[r][j]++; }
+    for (int n = 0; n < 2 * kUnitBytes4; ++n) {
+        int r, j; wi4_unit_pos(n, r, j); seen4[r][j]++;
+        if (wi4_unit_nibble(r, j) != n) ++bad;
+    }
+    for (int r = 0; r < 16; ++r) for (int j = 0; j < 64; ++j) bad += (seen8[r][j] != 1) + (seen4[r][j] != 1);
+    std::printf("%d\n", bad);
+    return 0;
+}
+"""
+    import tempfile
+    with tempfile.TemporaryDirectory() as d:
+        cpp = os.path.join(d, "t.cpp")
+        open(cpp, "w").write(src)
+        exe = os.path.join(d, "t")
+        subprocess.run(["g++", "-std=c++17", "-I", os.path.join(ROOT, "vector_quantized_weight_b200", "csrc"),
+                        "-o", exe, cpp], check=True)
+        assert subprocess.run([exe], capture_output=True, text=True, check=True).stdout.strip() == "0"

@@ -231,3 +231,38 @@ def test_host_buffer_call_graph_and_pageable():
             lin.run_host(torch.from_numpy(x), yp)
             assert torch.equal(yp, ref)
     lin.close()
+
+
+@pytest.mark.parametrize("N,K,B,resid", [(4096, 4096, 1, 0), (256, 512, 2, 0), (100, 264, 3, 0), (64, 512, 1, 128),
+                                         (48, 1024, 5, 128), (4096, 4096, 4, 0)])
+def test_four_bit_indices(N, K, B, resid):
+    """16-centroid codebooks with indices packed two per byte: against the
+    oracle (which reads the packed bytes itself), and the index round trip
+    is bit-exact."""
+    import torch
+    from vector_quantized_weight_b200 import eva_vq
+    shape = synth.LayerShape("idx4", N, K, residual_group=resid, index_bits=4)
+    layer = synth.make_layer(shape, N + K + B, alpha_signed=bool(resid))
+    x = synth.make_x(K, B, 7)
+    y = run_gpu(layer, x)
+    rows = sample_rows(N, 0, n=192, seed=3) if N * K * B > 2**24 else np.arange(N)
+    ref = sub_layer_oracle(layer, x, rows)
+    assert np.all(norm_rel_err(y[:, rows], ref) <= TOL)
+    lin = eva_vq.from_layer(layer, max_batch=B)
+    back = lin.unpack_indices().cpu().numpy()
+    torch.cuda.synchronize()
+    lin.close()
+    assert np.array_equal(back, layer.wi)
+
+
+def test_four_bit_integer_exact():
+    rng = np.random.default_rng(11)
+    N, K = 128, 512
+    wc = rng.integers(-2, 3, size=(1, 16, 4)).astype(np.float16)
+    idx = rng.integers(0, 16, size=(N, K // 4))
+    layer = synth.LayerData(synth.LayerShape("int4", N, K, index_bits=4), wc, synth.pack_nibbles(idx), None,
+                            None, None)
+    for B in (1, 2, 3):
+        x = rng.integers(-3, 4, size=(B, K)).astype(np.float16)
+        y = run_gpu(layer, x, out_dtype="float32")
+        assert np.array_equal(y, oracle.layer_linear(layer, x))

@@ -26,6 +26,7 @@ using namespace eva;
 struct eva_vq_linear {
     eva_vq_desc desc;
     int device = 0, sm_count = 0;
+    int ncent = kCent, unit_bytes = kUnitBytes;   // 16 and 512 for 4-bit indices
     int smem_per_sm = 0, smem_reserved = 0, smem_optin = 0;   // shared memory, bytes
     int regs_per_sm = 0;
     int J = 0, S = 0, T = 0, Npad = 0, G = 1, tiles_per_cb = 0;
@@ -120,7 +121,12 @@ void paley28_table(int8_t *out) {
 eva_status_t validate_desc(const eva_vq_desc *d) {
     if (!d) return EVA_ERR_INVALID_ARG;
     if (d->N < 1 || d->K < 1 || d->N > (1 << 24) || d->K > (1 << 22)) return EVA_ERR_INVALID_ARG;
-    if (d->d != kD || d->index_bits != 8) return EVA_ERR_UNSUPPORTED;
+    if (d->d != kD || (d->index_bits != 8 && d->index_bits != 4)) return EVA_ERR_UNSUPPORTED;
+    if (d->index_bits == 4) {
+        // 4-bit indices: one shared codebook, no rotation, whole index bytes.
+        if (d->codebook_rows || d->hadamard_block || d->path == EVA_PATH_DEQUANT_MMA) return EVA_ERR_UNSUPPORTED;
+        if (d->K % 8) return EVA_ERR_INVALID_ARG;
+    }
     if (d->K % kD) return EVA_ERR_INVALID_ARG;
     if (d->codebook_rows < 0) return EVA_ERR_INVALID_ARG;
     if (d->codebook_rows && (d->codebook_rows % kTileRows || d->N % d->codebook_rows))
@@ -142,7 +148,8 @@ eva_status_t validate_desc(const eva_vq_desc *d) {
 // mbarrier, the running sums of `tiles` row tiles, the cluster reduction
 // stage and, 128-byte aligned, the fused rotation's scratch (rotation blocks
 // b > 256: b floats per token) and the `staged` index units of the first slice.
-size_t lookup_smem(bool pair_t, bool resid, int tiles, int gs, int rot_b, int s_total, int staged = 0) {
+size_t lookup_smem(bool pair_t, bool resid, int tiles, int gs, int rot_b, int s_total, int staged = 0,
+                   size_t unit_bytes = kUnitBytes) {
     const size_t tile_bytes = (size_t)kTileRows * 2 * 4;
     const size_t stage_tiles = (size_t)((tiles + gs - 1) / gs) * gs;   // reduction stage
     const size_t base = (size_t)kOcBytes + ((pair_t && resid) ? (size_t)kOcBytes : 0) +
@@ -151,7 +158,7 @@ size_t lookup_smem(bool pair_t, bool resid, int tiles, int gs, int rot_b, int s_
     const int ntok = pair_t ? 2 : 1;
     const size_t xt = paley_m(rot_b) >= 256 ? (size_t)((s_total + gs - 1) / gs) * ntok * kSliceK * 4 : 0;
     const size_t rot = rot_b ? xt + rot_scratch_bytes(rot_b, paley_m(rot_b), ntok) : 0;
-    return ((base + 127) & ~(size_t)127) + rot + (size_t)staged * kUnitBytes;
+    return ((base + 127) & ~(size_t)127) + rot + (size_t)staged * unit_bytes;
 }
 
 // Index units of the first slice a CTA copies into shared memory: as many of
@@ -171,21 +178,29 @@ int staged_tiles(const eva_vq_linear *h, const void *fn, bool pair_t, bool resid
         cudaGetLastError();
     const size_t budget = (two_fit_regs && base <= two) ? two : one;
     if (base >= budget) return 0;
-    return (int)std::min<size_t>((size_t)tiles, (budget - base) / kUnitBytes);
+    return (int)std::min<size_t>((size_t)tiles, (budget - base) / h->unit_bytes);
 }
 
 using LookupFn = void (*)(LookupParams);
 template <bool ROT>
 LookupFn lookup_fn_r(bool pair_t, bool resid, bool grouped) {
     if (grouped) {
-        if (!pair_t) return resid ? eva_lookup_kernel<false, true, true, ROT> : eva_lookup_kernel<false, false, true, ROT>;
-        return resid ? eva_lookup_kernel<true, true, true, ROT> : eva_lookup_kernel<true, false, true, ROT>;
+        if (!pair_t)
+            return resid ? eva_lookup_kernel<false, true, true, ROT, false> : eva_lookup_kernel<false, false, true, ROT, false>;
+        return resid ? eva_lookup_kernel<true, true, true, ROT, false> : eva_lookup_kernel<true, false, true, ROT, false>;
     }
-    if (!pair_t) return resid ? eva_lookup_kernel<false, true, false, ROT> : eva_lookup_kernel<false, false, false, ROT>;
-    return resid ? eva_lookup_kernel<true, true, false, ROT> : eva_lookup_kernel<true, false, false, ROT>;
+    if (!pair_t)
+        return resid ? eva_lookup_kernel<false, true, false, ROT, false> : eva_lookup_kernel<false, false, false, ROT, false>;
+    return resid ? eva_lookup_kernel<true, true, false, ROT, false> : eva_lookup_kernel<true, false, false, ROT, false>;
 }
-// rot: the instance that computes the Hadamard rotation while staging x.
-LookupFn lookup_fn(bool pair_t, bool resid, bool grouped, bool rot) {
+// rot: the instance that computes the Hadamard rotation while staging x;
+// nib: 4-bit indices (shared codebook, no rotation).
+LookupFn lookup_fn(bool pair_t, bool resid, bool grouped, bool rot, bool nib = false) {
+    if (nib) {
+        if (!pair_t)
+            return resid ? eva_lookup_kernel<false, true, false, false, true> : eva_lookup_kernel<false, false, false, false, true>;
+        return resid ? eva_lookup_kernel<true, true, false, false, true> : eva_lookup_kernel<true, false, false, false, true>;
+    }
     return rot ? lookup_fn_r<true>(pair_t, resid, grouped) : lookup_fn_r<false>(pair_t, resid, grouped);
 }
 
@@ -220,7 +235,8 @@ int max_active_clusters(LookupFn fn, size_t smem, int cs) {
 void plan_grid(eva_vq_linear *h, int pair_t) {
     const int S = h->S, T = h->T, P = h->sm_count;
     const bool resid = h->desc.residual_group != 0;
-    const LookupFn fn = lookup_fn(pair_t != 0, resid, h->tiles_per_cb != 0, h->desc.hadamard_block != 0);
+    const LookupFn fn = lookup_fn(pair_t != 0, resid, h->tiles_per_cb != 0, h->desc.hadamard_block != 0,
+                                  h->desc.index_bits == 4);
     double best = 1e300;
     eva_vq_linear::Plan pl;
     pl.Gs = 1;
@@ -250,7 +266,7 @@ void plan_grid(eva_vq_linear *h, int pair_t) {
     }
     const int tiles = (T + pl.Gt - 1) / pl.Gt;
     pl.staged = staged_tiles(h, (const void *)fn, pair_t != 0, resid, tiles, pl.Gs);
-    pl.smem = lookup_smem(pair_t, resid, tiles, pl.Gs, h->desc.hadamard_block, S, pl.staged);
+    pl.smem = lookup_smem(pair_t, resid, tiles, pl.Gs, h->desc.hadamard_block, S, pl.staged, h->unit_bytes);
     pl.smem_nostage = lookup_smem(pair_t, resid, tiles, pl.Gs, h->desc.hadamard_block, S, 0);
     h->plan[pair_t] = pl;
 }
@@ -344,8 +360,9 @@ cudaError_t set_smem_attrs(int smem_optin) {
         e = cudaFuncSetAttribute((const void *)fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_optin);
         if (e != cudaSuccess) return e;
     }
-    for (int v = 0; v < 16; ++v) {
-        const LookupFn fn = lookup_fn(v & 1, (v >> 1) & 1, (v >> 2) & 1, (v >> 3) & 1);
+    for (int v = 0; v < 20; ++v) {
+        const LookupFn fn = v < 16 ? lookup_fn(v & 1, (v >> 1) & 1, (v >> 2) & 1, (v >> 3) & 1)
+                                   : lookup_fn(v & 1, (v >> 1) & 1, false, false, true);
         e = cudaFuncSetAttribute((const void *)fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         if (e != cudaSuccess) return e;
         // The device's per-block limit: it covers the one-CTA-per-SM footprint
@@ -465,6 +482,8 @@ eva_status_t eva_vq_linear_create(eva_vq_linear_t *out, const eva_vq_desc *desc,
     h->Npad = h->T * kTileRows;
     h->G = desc->codebook_rows ? N / desc->codebook_rows : 1;
     h->tiles_per_cb = desc->codebook_rows ? desc->codebook_rows / kTileRows : 0;
+    h->ncent = 1 << desc->index_bits;
+    h->unit_bytes = desc->index_bits == 4 ? kUnitBytes4 : kUnitBytes;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const long long units = (long long)h->S * h->T;
     int64_t ws = 0;
@@ -474,7 +493,7 @@ eva_status_t eva_vq_linear_create(eva_vq_linear_t *out, const eva_vq_desc *desc,
     plan_grid(h, 0);
     if (desc->max_batch > 1) plan_grid(h, 1);
     int max_grid = std::max(h->plan[0].Gs * h->plan[0].Gt, h->plan[1].Gs * h->plan[1].Gt);
-    if (!desc->residual_group && !desc->hadamard_block &&
+    if (!desc->residual_group && !desc->hadamard_block && desc->index_bits == 8 &&
         (desc->path == EVA_PATH_DEQUANT_MMA || (desc->path == EVA_PATH_AUTO && desc->max_batch >= kDequantMinBatch))) {
         plan_dequant(h, 1);
         plan_dequant(h, 2);
@@ -485,8 +504,8 @@ eva_status_t eva_vq_linear_create(eva_vq_linear_t *out, const eva_vq_desc *desc,
             return EVA_ERR_UNSUPPORTED;
         }
     }
-    chk(dalloc(&h->wi, (size_t)units * kUnitBytes, nullptr));
-    chk(dalloc(&h->wc, (size_t)h->G * kCent * kD * sizeof(__half), nullptr));
+    chk(dalloc(&h->wi, (size_t)units * h->unit_bytes, nullptr));
+    chk(dalloc(&h->wc, (size_t)h->G * h->ncent * kD * sizeof(__half), nullptr));
     if (desc->residual_group) {
         chk(dalloc(&h->sg, (size_t)units * kSignUnitBytes, nullptr));
         chk(dalloc(&h->al, (size_t)units * kAlphaUnitHalves * sizeof(__half), nullptr));
@@ -509,10 +528,13 @@ eva_status_t eva_vq_linear_create(eva_vq_linear_t *out, const eva_vq_desc *desc,
     }
 
     const int thr = 256;
-    const long long wib = units * kUnitBytes;
-    eva_repack_wi_kernel<<<blocks_for(wib, thr), thr, 0, s>>>(wi, h->wi, N, h->J, h->T, wib);
+    const long long wib = units * h->unit_bytes;
+    if (desc->index_bits == 4)
+        eva_repack_wi4_kernel<<<blocks_for(wib, thr), thr, 0, s>>>(wi, h->wi, N, h->J, h->T, wib);
+    else
+        eva_repack_wi_kernel<<<blocks_for(wib, thr), thr, 0, s>>>(wi, h->wi, N, h->J, h->T, wib);
     chk(cudaGetLastError());
-    chk(cudaMemcpyAsync(h->wc, wc, (size_t)h->G * kCent * kD * sizeof(__half), cudaMemcpyDeviceToDevice, s));
+    chk(cudaMemcpyAsync(h->wc, wc, (size_t)h->G * h->ncent * kD * sizeof(__half), cudaMemcpyDeviceToDevice, s));
     if (desc->residual_group) {
         const long long sb = units * kSignUnitBytes, ab = units * kAlphaUnitHalves;
         eva_repack_signs_kernel<<<blocks_for(sb, thr), thr, 0, s>>>(signs, h->sg, N, K / 8, h->T, sb);
@@ -580,6 +602,7 @@ eva_status_t eva_vq_linear_run_ex(eva_vq_linear_t h, const void *x, int32_t B, v
     p.wi_staged = independent ? 0 : pl.staged;
     p.status = h->status;
     p.tiles_per_cb = h->tiles_per_cb;
+    p.ncent = h->ncent;
     p.out_f32 = d.out_dtype == EVA_F32 ? 1 : 0;
     p.independent = independent;
     if (d.hadamard_block) {   // the rotation runs inside the lookup kernel
@@ -601,10 +624,10 @@ eva_status_t eva_vq_linear_run_ex(eva_vq_linear_t h, const void *x, int32_t B, v
         const long long units = (long long)h->S * h->T;
         const void *base[8] = {h->wi, h->sg, h->al, h->wc, p.x, nullptr, nullptr, y};
         const unsigned long long bytes[8] = {
-            (unsigned long long)units * kUnitBytes,
+            (unsigned long long)units * h->unit_bytes,
             h->sg ? (unsigned long long)units * kSignUnitBytes : 0ull,
             h->al ? (unsigned long long)units * kAlphaUnitHalves * 2 : 0ull,
-            (unsigned long long)h->G * kCent * kD * 2,
+            (unsigned long long)h->G * h->ncent * kD * 2,
             (unsigned long long)B * d.K * (p.x_f32 ? 4 : 2),
             0ull,
             0ull,
@@ -627,7 +650,8 @@ eva_status_t eva_vq_linear_run_ex(eva_vq_linear_t h, const void *x, int32_t B, v
         h->last_path = EVA_PATH_DEQUANT_MMA;
         return EVA_OK;
     }
-    e = launch_pdl(lookup_fn(pair_t, resid, h->tiles_per_cb != 0, p.rot_b != 0), grid, block, smem, s, pl.Gs, p);
+    e = launch_pdl(lookup_fn(pair_t, resid, h->tiles_per_cb != 0, p.rot_b != 0, d.index_bits == 4), grid, block, smem, s,
+                   pl.Gs, p);
     if (e != cudaSuccess) return cuda_status(e);
     ++kernels;
     h->last_grid = (int)grid.x;
@@ -706,6 +730,7 @@ eva_status_t eva_vq_linear_run_noalloc(eva_vq_linear_t h, const void *x, int32_t
     p.T = h->T;
     p.B = B;
     p.tiles_per_cb = h->tiles_per_cb;
+    p.ncent = h->ncent;
     p.out_f32 = d.out_dtype == EVA_F32 ? 1 : 0;
     p.independent = 0;
     p.Gs = pl.Gs;
@@ -742,7 +767,8 @@ eva_status_t eva_vq_linear_run_noalloc(eva_vq_linear_t h, const void *x, int32_t
         return cuda_status(launch_dequant(h, p, B, s, &dsmem, &dgrid));
     }
     const bool resid = d.residual_group != 0;
-    e = launch_pdl(lookup_fn(pair_t, resid, h->tiles_per_cb != 0, fused_rot), dim3(pl.Gs * pl.Gt), dim3(kThreads),
+    e = launch_pdl(lookup_fn(pair_t, resid, h->tiles_per_cb != 0, fused_rot, d.index_bits == 4), dim3(pl.Gs * pl.Gt),
+                   dim3(kThreads),
                    pl.smem, s, pl.Gs, p);
     return cuda_status(e);
 }
@@ -865,6 +891,11 @@ eva_status_t eva_vq_linear_destroy(eva_vq_linear_t h) {
 eva_status_t eva_vq_unpack_indices(eva_vq_linear_t h, uint8_t *wi_out, eva_stream_t stream) {
     if (!h || !wi_out) return EVA_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (h->desc.index_bits == 4) {   // canonical packed [N][J/2]
+        const long long total = (long long)h->desc.N * (h->J / 2);
+        eva_unpack_wi4_kernel<<<blocks_for(total, 256), 256, 0, s>>>(h->wi, wi_out, h->desc.N, h->J, h->T, total);
+        return cuda_status(cudaGetLastError());
+    }
     const long long total = (long long)h->S * h->T * kUnitBytes;
     eva_unpack_wi_kernel<<<blocks_for(total, 256), 256, 0, s>>>(h->wi, wi_out, h->desc.N, h->J, h->T, total);
     return cuda_status(cudaGetLastError());
@@ -910,10 +941,10 @@ eva_status_t eva_vq_linear_info(eva_vq_linear_t h, eva_vq_info *info) {
     if (!h || !info) return EVA_ERR_INVALID_ARG;
     const eva_vq_desc &d = h->desc;
     std::memset(info, 0, sizeof(*info));
-    info->wi_bytes = (int64_t)d.N * (d.K / kD);
+    info->wi_bytes = (int64_t)d.N * (d.K / kD) * d.index_bits / 8;
     info->sign_bytes = d.residual_group ? (int64_t)d.N * (d.K / 8) : 0;
     info->alpha_bytes = d.residual_group ? (int64_t)d.N * (d.K / d.residual_group) * 2 : 0;
-    info->codebook_bytes = (int64_t)h->G * kCent * kD * 2;
+    info->codebook_bytes = (int64_t)h->G * h->ncent * kD * 2;
     info->stream_bytes = info->wi_bytes + info->sign_bytes + info->alpha_bytes + (int64_t)d.K * 2;
     info->workspace_bytes = h->workspace_bytes;
     info->slices = h->S;

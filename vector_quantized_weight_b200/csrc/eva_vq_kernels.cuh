@@ -53,6 +53,7 @@ struct LookupParams {
     int rot_b;               // 0, or the rotation block b: x~ = s . (H_b x) / sqrt(b) is
                              // computed in the lookup kernel from fp16 x
     float rot_scale;         // 1 / sqrt(b), rounded to fp32
+    int ncent;               // centroids per codebook: 256, or 16 for 4-bit indices
     int rot_m;               // 0: Sylvester block; m: b = 28 m, H_b = H28 (x) H_m
     const int8_t *h28;       // the order-28 Paley matrix [28][28] (rot_m != 0)
 #ifdef EVA_DEVICE_CHECKS
@@ -608,11 +609,12 @@ __device__ __forceinline__ float lds_x(const LookupParams &p, uint32_t x_off, in
 // nt = warp + kWarps j: lane (g, q) holds WC[cb][8 nt + g][q] as tf32.
 __device__ __forceinline__ void load_codebook_frag(const LookupParams &p, int cb, int warp, int g, int q,
                                                    uint32_t (&bf)[4]) {
-    const __half *wcb = p.wc + (size_t)cb * kCent * kD;
+    const __half *wcb = p.wc + (size_t)cb * p.ncent * kD;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        const __half *wp = wcb + (8 * (warp + kWarps * j) + g) * kD + q;
-        bf[j] = to_tf32(EVA_BAD_G(BUF_WC, wp, 2) ? 0.f : __half2float(__ldg(wp)));
+        const int c = 8 * (warp + kWarps * j) + g;
+        const __half *wp = wcb + c * kD + q;
+        bf[j] = to_tf32((c >= p.ncent || EVA_BAD_G(BUF_WC, wp, 2)) ? 0.f : __half2float(__ldg(wp)));
     }
 }
 
@@ -650,6 +652,7 @@ __device__ __forceinline__ void build_oc(const LookupParams &p, int warp, int g,
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const int nt = warp + kWarps * j;
+        if (8 * nt >= p.ncent) continue;   // 16-centroid codebooks: two column tiles
         const uint32_t b0 = bf[j];
         if (!PAIR_T) {
             // D[mt][2h + cc] = OC[16 mt + g + 8 h][8 nt + 2 q + cc]; the word of
@@ -747,6 +750,17 @@ __device__ __forceinline__ void build_sign_table(const LookupParams &p, int warp
     }
 }
 
+// One unit's bytes for this lane: 8-bit indices, 16 bytes at p and 16 at
+// p + 512; 4-bit indices, the 16 bytes at p (b stays zero).
+template <bool NIB>
+__device__ __forceinline__ void load_unit(const LookupParams &p, const uint8_t *up, uint4 &a, uint4 &b) {
+    if constexpr (NIB) {
+        if (!EVA_BAD_G(BUF_WI, up, 16)) a = ldg_stream(up);
+    } else {
+        if (!EVA_BAD_G(BUF_WI, up, 16) && !EVA_BAD_G(BUF_WI, up + 512, 16)) ldg_unit(up, a, b);
+    }
+}
+
 // ------------------------------------------------------------ lookup kernel
 //
 // Grid: Gs x Gt CTAs in clusters of Gs; CTA (ts, tt) owns K-slices [s0, s1)
@@ -764,8 +778,10 @@ __device__ __forceinline__ void build_sign_table(const LookupParams &p, int warp
 // so the weight stream of layer l+1 overlaps the lookups of layer l; the
 // token-pair and residual variants need more registers and run one CTA per SM.
 
-template <bool PAIR_T, bool RESID, bool GROUPED, bool ROT>
+template <bool PAIR_T, bool RESID, bool GROUPED, bool ROT, bool NIB>
 __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_lookup_kernel(const LookupParams p) {
+    // NIB: 4-bit indices (16 centroids), units of 512 bytes (16 per lane).
+    constexpr uint32_t UB = NIB ? (uint32_t)kUnitBytes4 : (uint32_t)kUnitBytes;
     // Index units in flight per warp: with per-group codebooks a warp has at
     // most one tile per codebook pass, so a short ring suffices.
     constexpr int LA = GROUPED ? 2 : kLookahead;
@@ -785,7 +801,7 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
     constexpr uint32_t ACC_OFF = BAR_OFF + 128u;         // per-CTA running sums (128-byte
                                                          // tile blocks stay 128-byte aligned)
     constexpr int NTOK_C = PAIR_T ? 2 : 1;
-    constexpr bool NAIVE = kNaiveOcBuild && !PAIR_T && !RESID;
+    constexpr bool NAIVE = kNaiveOcBuild && !PAIR_T && !RESID && !NIB;
     // GROUPED: one codebook per tiles_per_cb row tiles (else one shared codebook).
     const int cb_first = GROUPED ? t0 / p.tiles_per_cb : 0;
     const int cb_last = GROUPED ? (t1 - 1) / p.tiles_per_cb : 0;
@@ -810,8 +826,8 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
     const uint32_t bar = (uint32_t)__cvta_generic_to_shared(eva_smem + BAR_OFF);
     if (tid == 0 && staged > 0) {
         mbar_init(bar, 1);
-        const uint8_t *src = p.wi + ((size_t)s0 * p.T + t0) * kUnitBytes;
-        const uint32_t bytes = (uint32_t)staged * kUnitBytes;
+        const uint8_t *src = p.wi + ((size_t)s0 * p.T + t0) * UB;
+        const uint32_t bytes = (uint32_t)staged * UB;
         if (staged > 0 && !EVA_BAD_G(BUF_WI, src, bytes) && !EVA_BAD_S(WIS_OFF) &&
             !EVA_BAD_S(WIS_OFF + bytes - 4u)) {
             mbar_arrive_expect_tx(bar, bytes);
@@ -827,8 +843,8 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
         const int skip = (tid == 0) ? staged : 0;
         const size_t u = (size_t)(s0 + tid) * p.T + t0 + skip;
         const uint32_t nt = (uint32_t)(t1 - t0 - skip);
-        if (nt > 0 && !EVA_BAD_G(BUF_WI, p.wi + u * kUnitBytes, nt * kUnitBytes))
-            prefetch_l2_bulk(p.wi + u * kUnitBytes, nt * kUnitBytes);
+        if (nt > 0 && !EVA_BAD_G(BUF_WI, p.wi + u * UB, nt * UB))
+            prefetch_l2_bulk(p.wi + u * UB, nt * UB);
         if (RESID) {
             const size_t ur = (size_t)(s0 + tid) * p.T + t0;
             const uint32_t ntr = (uint32_t)(t1 - t0);
@@ -909,8 +925,8 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
                 for (int d = 0; d < LA; ++d) {
                     nb[d][0] = nb[d][1] = make_uint4(0u, 0u, 0u, 0u);
                     if (i_st + d < i1) {
-                        const uint8_t *up = p.wi + ((size_t)s * p.T + t0 + warp + kWarps * (i_st + d)) * kUnitBytes + 16 * lane;
-                        if (!EVA_BAD_G(BUF_WI, up, 16) && !EVA_BAD_G(BUF_WI, up + 512, 16)) ldg_unit(up, nb[d][0], nb[d][1]);
+                        const uint8_t *up = p.wi + ((size_t)s * p.T + t0 + warp + kWarps * (i_st + d)) * UB + 16 * lane;
+                        load_unit<NIB>(p, up, nb[d][0], nb[d][1]);
                     }
                 }
                 // Paley blocks with m >= 256: x~ of every slice of this CTA at
@@ -941,7 +957,15 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
                     for (int s8 = 0; s8 < 8; ++s8) {
                         const uint32_t cw = (4u * lane + 16u * s8) & 127u;   // 4 * oc_col(lane, s8)
                         uint32_t o0, o1, o2, o3;
-                        if constexpr (NAIVE) {
+                        if constexpr (NIB) {
+                            // word s8 / 2, nibbles 4 (s8 & 1) + r: index c -> (c << 8) | cw
+                            const uint32_t w = wv[s8 >> 1];
+                            const int sh = 16 * (s8 & 1);
+                            o0 = OC_OFF + ((((w >> sh) << 8) & 0xF00u) | cw);
+                            o1 = OC_OFF + ((((w >> sh) << 4) & 0xF00u) | cw);
+                            o2 = OC_OFF + HI_OFF + (((w >> sh) & 0xF00u) | cw);
+                            o3 = OC_OFF + HI_OFF + (((w >> (sh + 4)) & 0xF00u) | cw);
+                        } else if constexpr (NAIVE) {
                             o0 = OC_OFF + (cw << 8) + ((wv[s8] & 0xFFu) << 2);
                             o1 = OC_OFF + (cw << 8) + (((wv[s8] >> 8) & 0xFFu) << 2);
                             o2 = OC_OFF + (cw << 8) + (((wv[s8] >> 16) & 0xFFu) << 2);
@@ -1020,10 +1044,10 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
 #pragma unroll 1
                 for (int i = i0; i < i_st; ++i) {
                     const int tl = warp + kWarps * i;              // tile index within the CTA
-                    const uint32_t wo = WIS_OFF + (uint32_t)tl * kUnitBytes + 16u * lane;
+                    const uint32_t wo = WIS_OFF + (uint32_t)tl * UB + 16u * lane;
                     const uint4 v0 = (EVA_BAD_S(wo) || EVA_BAD_S(wo + 12u)) ? make_uint4(0u, 0u, 0u, 0u) : lds128(wo);
-                    const uint4 v1 = (EVA_BAD_S(wo + 512u) || EVA_BAD_S(wo + 524u)) ? make_uint4(0u, 0u, 0u, 0u)
-                                                                                       : lds128(wo + 512u);
+                    const uint4 v1 = (NIB || EVA_BAD_S(wo + 512u) || EVA_BAD_S(wo + 524u)) ? make_uint4(0u, 0u, 0u, 0u)
+                                                                                              : lds128(wo + 512u);
                     tile(tl, (size_t)s * p.T + t0 + tl, v0, v1);
                 }
                 // ... then the streamed ones, through the lookahead ring.
@@ -1038,9 +1062,8 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
                         nb[d][1] = nb[d + 1][1];
                     }
                     if (i + LA < i1) {
-                        const uint8_t *up = p.wi + (unit + (size_t)kWarps * LA) * kUnitBytes + 16 * lane;
-                        if (!EVA_BAD_G(BUF_WI, up, 16) && !EVA_BAD_G(BUF_WI, up + 512, 16))
-                            ldg_unit(up, nb[LA - 1][0], nb[LA - 1][1]);
+                        const uint8_t *up = p.wi + (unit + (size_t)kWarps * LA) * UB + 16 * lane;
+                        load_unit<NIB>(p, up, nb[LA - 1][0], nb[LA - 1][1]);
                     }
                     tile(tl, unit, v0, v1);
                 }
@@ -1205,6 +1228,43 @@ __global__ void eva_unpack_wi_kernel(const uint8_t *__restrict__ packed, uint8_t
     wi_unit_pos(b, row, jl);
     const int o = kTileRows * t + row, j = kSliceJ * s + jl;
     if (o < N && j < J) wi[(size_t)o * J + j] = packed[idx];
+}
+
+// 4-bit indices: canonical [N][J/2] (sub-vector 2t in the low nibble of byte
+// t) -> units of 512 bytes; one thread per unit byte (two nibbles).
+__global__ void eva_repack_wi4_kernel(const uint8_t *__restrict__ wi, uint8_t *__restrict__ out, int N, int J,
+                                      int T, long long total) {
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= total) return;
+    const long long unit = idx / kUnitBytes4;
+    const int b = (int)(idx % kUnitBytes4);
+    const int s = (int)(unit / T), t = (int)(unit % T);
+    unsigned v = 0;
+    for (int h = 0; h < 2; ++h) {
+        int row, jl;
+        wi4_unit_pos(2 * b + h, row, jl);
+        const int o = kTileRows * t + row, j = kSliceJ * s + jl;
+        const unsigned c = (o < N && j < J) ? (wi[(size_t)o * (J / 2) + j / 2] >> (4 * (j & 1))) & 15u : 0u;
+        v |= c << (4 * h);
+    }
+    out[idx] = (uint8_t)v;
+}
+
+// Inverse (test hook): one thread per canonical byte.
+__global__ void eva_unpack_wi4_kernel(const uint8_t *__restrict__ packed, uint8_t *__restrict__ wi, int N, int J,
+                                      int T, long long total) {
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= total) return;
+    const int o = (int)(idx / (J / 2)), t2 = (int)(idx % (J / 2));
+    unsigned v = 0;
+    for (int h = 0; h < 2; ++h) {
+        const int j = 2 * t2 + h, s = j / kSliceJ, jl = j % kSliceJ;
+        const int n = wi4_unit_nibble(o % kTileRows, jl);
+        const long long unit = (long long)s * T + o / kTileRows;
+        const unsigned c = (packed[unit * kUnitBytes4 + (n >> 1)] >> (4 * (n & 1))) & 15u;
+        v |= c << (4 * h);
+    }
+    wi[idx] = (uint8_t)v;
 }
 
 __global__ void eva_repack_signs_kernel(const uint8_t *__restrict__ sg, uint8_t *__restrict__ out,

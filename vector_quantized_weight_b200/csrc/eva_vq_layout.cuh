@@ -48,6 +48,29 @@ __host__ __device__ __forceinline__ void wi_unit_pos(int b, int &row, int &jl) {
     jl = oc_col(lane, s8) + ((r & 2) ? 32 : 0);
 }
 
+// 4-bit indices (16 centroids): a unit is 512 bytes, 16 per lane; lane L's
+// word u (0..3) holds k-steps 2u and 2u + 1, nibble 4 (s8 & 1) + r of the
+// word being register r of k-step s8.  Nibble n = 32 L + 8 u + e of the unit
+// -> (row in tile, sub-vector in slice), with the same (lane, s8, r) meaning
+// as the byte layout.
+constexpr int kUnitBytes4 = kUnitBytes / 2;
+
+__host__ __device__ __forceinline__ void wi4_unit_pos(int n, int &row, int &jl) {
+    const int lane = n >> 5, u = (n >> 3) & 3, e = n & 7;
+    const int s8 = 2 * u + (e >> 2), r = e & 3;
+    row = (lane >> 2) + ((r & 1) ? 8 : 0);
+    jl = oc_col(lane, s8) + ((r & 2) ? 32 : 0);
+}
+
+// Inverse of wi4_unit_pos: the nibble of (row in tile, sub-vector in slice).
+__host__ __device__ __forceinline__ int wi4_unit_nibble(int row, int jl) {
+    const int r = ((row >= 8) ? 1 : 0) | ((jl >= 32) ? 2 : 0);
+    const int g = row & 7, w = jl & 31, q = w & 3;
+    const int s8 = (((w - q) >> 2) - g) & 7;
+    const int lane = 4 * g + q;
+    return 32 * lane + 8 * (s8 >> 1) + 4 * (s8 & 1) + r;
+}
+
 // Sign position read by lane (g, q) in residual MMA i (0..3), register r.
 // Lanes q = 0,1 cover the first 128-input group of the slice (positions
 // 0..15), lanes q = 2,3 the second (16..31); per register the 32 lanes read

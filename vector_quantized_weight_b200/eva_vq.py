@@ -231,13 +231,16 @@ class VQLinear:
 
     def __init__(self, wc, wi, *, signs=None, alpha=None, hsign=None, codebook_rows=0,
                  residual_group=0, hadamard_block=0, max_batch=1, out_dtype="float16",
-                 path=EVA_PATH_AUTO, stream=None):
+                 path=EVA_PATH_AUTO, index_bits=8, stream=None):
         import torch
         N, J = wi.shape
+        if index_bits == 4:          # two indices per byte
+            J *= 2
+        self.index_bits = int(index_bits)
         self.N, self.K = int(N), int(J) * 4
         self.out_dtype = torch.float32 if out_dtype in ("float32", torch.float32) else torch.float16
         self.max_batch = int(max_batch)
-        self.desc = eva_vq_desc(self.N, self.K, 4, 8, int(codebook_rows), int(residual_group),
+        self.desc = eva_vq_desc(self.N, self.K, 4, self.index_bits, int(codebook_rows), int(residual_group),
                                 int(hadamard_block), self.max_batch,
                                 EVA_F32 if self.out_dtype == torch.float32 else EVA_F16, int(path))
         tensors = [wc, wi, signs, alpha, hsign]
@@ -266,8 +269,10 @@ class VQLinear:
         return y_host
 
     def unpack_indices(self, stream=None):
+        """The canonical index matrix back: [N][K/4], or [N][K/8] packed for 4-bit indices."""
         import torch
-        out = torch.empty((self.N, self.K // 4), dtype=torch.uint8, device="cuda")
+        cols = self.K // 4 if self.index_bits == 8 else self.K // 8
+        out = torch.empty((self.N, cols), dtype=torch.uint8, device="cuda")
         eva_vq_unpack_indices(self.handle, _ptr(out), _stream_handle(stream))
         return out
 
@@ -296,7 +301,7 @@ def from_layer(layer, *, max_batch=1, out_dtype="float16", path=EVA_PATH_AUTO, d
     return VQLinear(dev(layer.wc), dev(layer.wi), signs=dev(layer.signs), alpha=dev(layer.alpha),
                     hsign=dev(layer.hsign), codebook_rows=s.codebook_rows,
                     residual_group=s.residual_group, hadamard_block=s.hadamard_block,
-                    max_batch=max_batch, out_dtype=out_dtype, path=path)
+                    max_batch=max_batch, out_dtype=out_dtype, path=path, index_bits=s.index_bits)
 
 
 def quantize(w, init_index, iters: int, *, hsign=None, hadamard_block: int = 0, codebook_rows: int = 0,

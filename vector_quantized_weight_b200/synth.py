@@ -112,6 +112,9 @@ CONFIGS = {
                          _gemma_3bit(), (1,), 3),
     "llama70b": Config("llama70b", "Llama-2-70B-shaped 2-bit linears, one codebook per 128 rows",
                        _llama70b(), (1, 8, 32), 4),
+    "llama7b_layer_4bit": Config("llama7b_layer_4bit", "Llama-2-7B-shaped 4096x4096 layer with 4-bit indices "
+                                 "(16 centroids, 1 bit per weight), batch 1 and 4",
+                                 (LayerShape("l7b_4096x4096_idx4", 4096, 4096, index_bits=4),), (1, 4), 6),
     "gemma_3bit_rotK": Config("gemma_3bit_rotK", "Gemma-2-9B-shaped 3.125-bit linears, order-K (Paley x "
                               "Sylvester) rotation", _gemma_3bit_order_k(), (1, 2), 5),
 }

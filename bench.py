@@ -61,6 +61,9 @@ def parse_args():
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--group", type=int, default=3,
+                    help="also time the ring as eva_vq_linear_run_group calls of this many independent "
+                         "layers (e.g. a block's q, k, v); 0 skips that leg")
     return ap.parse_args()
 
 
@@ -308,10 +311,20 @@ def main():
     torch.cuda.synchronize(dev)
     info = layers[0].info()
 
+    group = [1]   # layers per call in the sweep
+
     def sweep(n, independent, start=0):
-        for i in range(n):
-            r = (start + i) % ring
-            layers[r](xs[r % len(xs)], out=ys[r], stream=stream, independent=independent)
+        i = 0
+        while i < n:
+            k = min(group[0], n - i)
+            if k == 1:
+                r = (start + i) % ring
+                layers[r](xs[r % len(xs)], out=ys[r], stream=stream, independent=independent)
+            else:
+                rs = [(start + i + j) % ring for j in range(k)]
+                eva_vq.run_group([layers[r] for r in rs], [xs[r % len(xs)] for r in rs], [ys[r] for r in rs],
+                                 stream=stream, independent=independent)
+            i += k
 
     uuid = getattr(props, "uuid", None)
     gpu_id = f"GPU-{uuid}" if uuid is not None else str(local)
@@ -364,6 +377,15 @@ def main():
         dep_steps = ring * max(1, min(steps, 200_000) // ring)
         ms_dep, _ = timed(False, dep_steps, False)
         dep = (dep_steps, ms_dep)
+
+    # The same independent layers, `--group` of them per eva_vq_linear_run_group call.
+    grouped = None
+    if args.group > 1 and args.chain == "independent":
+        group[0] = args.group
+        g_steps = ring * max(1, min(steps, 200_000) // ring)
+        ms_g, _ = timed(True, g_steps, False)
+        grouped = (g_steps, ms_g)
+        group[0] = 1
 
     # End to end through the public host-buffer call: x copied in from
     # pinned memory and y read back every step.
@@ -432,6 +454,13 @@ def main():
         "gpu_launches": steps * info.kernels_per_run,
         "clocks": clk.summary(),
     }
+    if grouped:
+        gs_, gms = grouped
+        line["grouped_calls"] = {
+            "layers_per_call": args.group, "us_per_layer": round(gms * 1e3 / gs_, 4), "steps": gs_,
+            "value": round(job_throughput_gbs(world, gs_, sb, gms), 4), "unit": "GB/s",
+            "note": ("eva_vq_linear_run_group(EVA_RUN_INDEPENDENT) of consecutive ring layers, one launch "
+                     "each (as for a decoder block's q, k and v)")}
     if dep:
         dep_steps, ms_dep = dep
         us_dep = ms_dep * 1e3 / dep_steps

@@ -133,6 +133,22 @@ EVA_API eva_status_t eva_vq_linear_run_ex(eva_vq_linear_t h, const void *x, int3
                                           eva_stream_t stream, uint32_t flags);
 
 /*
+ * Several independent layers at once: layer i computes ys[i] = layer_i(xs[i])
+ * for the same B (1 <= count <= 16; all handles on the current device).  No
+ * layer may read another's output.  When every layer has the first one's
+ * N, K and format (8-bit indices, one shared codebook, no rotation, the same
+ * residual setting and output type) and takes the lookup path at this B,
+ * the layers run as ONE launch whose CTAs the hardware schedules as slots
+ * free -- e.g. the q, k and v projections of a decoder block, which share
+ * their input.  Otherwise it is one eva_vq_linear_run_ex per layer.  Results
+ * are bitwise those of separate calls.  `flags` as for eva_vq_linear_run_ex,
+ * for the group as a whole.  Not part of the pages' method: a launch-level
+ * convenience.
+ */
+EVA_API eva_status_t eva_vq_linear_run_group(const eva_vq_linear_t *hs, const void *const *xs, void *const *ys,
+                                             int32_t count, int32_t B, eva_stream_t stream, uint32_t flags);
+
+/*
  * eva_vq_linear_run for callers that must not touch the device allocator.
  * No counterpart in the EVA pages or the 3-bit SRAM-lookup article: it is a
  * deployment convenience of this library.

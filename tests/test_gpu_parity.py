@@ -266,3 +266,35 @@ def test_four_bit_integer_exact():
         x = rng.integers(-3, 4, size=(B, K)).astype(np.float16)
         y = run_gpu(layer, x, out_dtype="float32")
         assert np.array_equal(y, oracle.layer_linear(layer, x))
+
+
+@pytest.mark.parametrize("B", [1, 2])
+def test_grouped_call_matches_separate_calls(B):
+    """eva_vq_linear_run_group: one launch for layers of one shape and format
+    (bitwise equal to separate calls, also with the independent flag and with
+    the residual), separate launches for a mixed group."""
+    import torch
+    from vector_quantized_weight_b200 import eva_vq
+    for shape in (synth.LayerShape("g", 4096, 4096), synth.LayerShape("gr", 512, 1024, residual_group=128)):
+        lins = [eva_vq.from_layer(synth.make_layer(shape, 50 + i), max_batch=B) for i in range(3)]
+        xs = [torch.from_numpy(synth.make_x(shape.K, B, 60 + i)).cuda() for i in range(3)]
+        ref = [lin(x).clone() for lin, x in zip(lins, xs)]
+        for indep in (False, True):
+            outs = eva_vq.run_group(lins, xs, independent=indep)
+            torch.cuda.synchronize()
+            for a, b in zip(ref, outs):
+                assert torch.equal(a, b)
+        for lin in lins:
+            assert eva_vq.eva_vq_sync_status(lin.handle) == eva_vq.EVA_OK
+            lin.close()
+    mixed = [synth.LayerShape("m1", 256, 512), synth.LayerShape("m2", 128, 1024, codebook_rows=16),
+             synth.LayerShape("m3", 64, 512, residual_group=128, hadamard_block=128)]
+    lins = [eva_vq.from_layer(synth.make_layer(sh, 70), max_batch=B) for sh in mixed]
+    xs = [torch.from_numpy(synth.make_x(sh.K, B, 71)).cuda() for sh in mixed]
+    ref = [lin(x).clone() for lin, x in zip(lins, xs)]
+    outs = eva_vq.run_group(lins, xs)
+    torch.cuda.synchronize()
+    for a, b in zip(ref, outs):
+        assert torch.equal(a, b)
+    for lin in lins:
+        lin.close()

@@ -371,6 +371,16 @@ cudaError_t set_smem_attrs(int smem_optin) {
         e = cudaFuncSetAttribute((const void *)fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_optin);
         if (e != cudaSuccess) return e;
     }
+    for (int v = 0; v < 4; ++v) {
+        const void *fn = v == 0 ? (const void *)eva_lookup_group_kernel<false, false>
+                       : v == 1 ? (const void *)eva_lookup_group_kernel<false, true>
+                       : v == 2 ? (const void *)eva_lookup_group_kernel<true, false>
+                                : (const void *)eva_lookup_group_kernel<true, true>;
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_optin);
+        if (e != cudaSuccess) return e;
+    }
     return cudaFuncSetAttribute(eva_hadamard_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 4096 * 4);
 }
 
@@ -564,17 +574,12 @@ eva_status_t eva_vq_linear_run(eva_vq_linear_t h, const void *x, int32_t B, void
     return eva_vq_linear_run_ex(h, x, B, y, stream, 0u);
 }
 
-eva_status_t eva_vq_linear_run_ex(eva_vq_linear_t h, const void *x, int32_t B, void *y, eva_stream_t stream,
-                                  uint32_t flags) {
-    if (!h || !x || !y || !aligned16(x) || !aligned16(y)) return EVA_ERR_INVALID_ARG;
-    if (flags & ~(uint32_t)EVA_RUN_INDEPENDENT) return EVA_ERR_INVALID_ARG;
-    const int independent = (flags & EVA_RUN_INDEPENDENT) ? 1 : 0;
-    if (B < 1 || B > h->desc.max_batch) return EVA_ERR_INVALID_ARG;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const eva_vq_desc &d = h->desc;
-    int kernels = 0;
-    cudaError_t e = cudaSuccess;
+}  // extern "C"
 
+namespace {
+// Parameters of one call of the lookup kernel (arguments already checked).
+LookupParams call_params(eva_vq_linear *h, const void *x, int32_t B, void *y, int independent, size_t *smem) {
+    const eva_vq_desc &d = h->desc;
     LookupParams p;
     std::memset(&p, 0, sizeof(p));
     p.wi = h->wi;
@@ -590,8 +595,7 @@ eva_status_t eva_vq_linear_run_ex(eva_vq_linear_t h, const void *x, int32_t B, v
     p.S = h->S;
     p.T = h->T;
     p.B = B;
-    const bool pair_t = B > 1;
-    const eva_vq_linear::Plan &pl = h->plan[pair_t ? 1 : 0];
+    const eva_vq_linear::Plan &pl = h->plan[B > 1 ? 1 : 0];
     p.Gs = pl.Gs;
     p.Gt = pl.Gt;
     p.acc_tiles = (h->T + pl.Gt - 1) / pl.Gt;
@@ -612,10 +616,7 @@ eva_status_t eva_vq_linear_run_ex(eva_vq_linear_t h, const void *x, int32_t B, v
         p.hs = h->hsign;
         p.rot_scale = (float)(1.0 / std::sqrt((double)d.hadamard_block));
     }
-
-    const bool resid = d.residual_group != 0;
-    const dim3 grid(pl.Gs * pl.Gt), block(kThreads);
-    const size_t smem = p.wi_staged ? pl.smem : pl.smem_nostage;
+    *smem = p.wi_staged ? pl.smem : pl.smem_nostage;
 #ifdef EVA_TIMELINE
     p.timeline = h->timeline;
 #endif
@@ -636,27 +637,102 @@ eva_status_t eva_vq_linear_run_ex(eva_vq_linear_t h, const void *x, int32_t B, v
             p.chk_base[i] = base[i];
             p.chk_bytes[i] = bytes[i];
         }
-        p.smem_bytes = (unsigned)smem;
+        p.smem_bytes = (unsigned)*smem;
         p.chk_record = h->status;
     }
 #endif
+    return p;
+}
+
+// The layers a grouped launch can take: one lookup-kernel instance for all
+// (8-bit indices, shared codebook, no rotation, the lookup path at this B).
+bool groupable(const eva_vq_linear *h, int B) {
+    const eva_vq_desc &d = h->desc;
+    return d.index_bits == 8 && !d.codebook_rows && !d.hadamard_block && !use_dequant(h, B);
+}
+
+using GroupFn = void (*)(LookupGroup);
+GroupFn group_fn(bool pair_t, bool resid) {
+    if (pair_t) return resid ? eva_lookup_group_kernel<true, true> : eva_lookup_group_kernel<true, false>;
+    return resid ? eva_lookup_group_kernel<false, true> : eva_lookup_group_kernel<false, false>;
+}
+}  // namespace
+
+extern "C" {
+
+eva_status_t eva_vq_linear_run_ex(eva_vq_linear_t h, const void *x, int32_t B, void *y, eva_stream_t stream,
+                                  uint32_t flags) {
+    if (!h || !x || !y || !aligned16(x) || !aligned16(y)) return EVA_ERR_INVALID_ARG;
+    if (flags & ~(uint32_t)EVA_RUN_INDEPENDENT) return EVA_ERR_INVALID_ARG;
+    const int independent = (flags & EVA_RUN_INDEPENDENT) ? 1 : 0;
+    if (B < 1 || B > h->desc.max_batch) return EVA_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const eva_vq_desc &d = h->desc;
+    size_t smem = 0;
+    LookupParams p = call_params(h, x, B, y, independent, &smem);
+    cudaError_t e;
     if (use_dequant(h, B)) {
         size_t dsmem = 0;
         int dgrid = 0;
         e = launch_dequant(h, p, B, s, &dsmem, &dgrid);
         if (e != cudaSuccess) return cuda_status(e);
         h->last_grid = dgrid;
-        h->last_kernels = kernels + 1;
+        h->last_kernels = 1;
         h->last_path = EVA_PATH_DEQUANT_MMA;
         return EVA_OK;
     }
-    e = launch_pdl(lookup_fn(pair_t, resid, h->tiles_per_cb != 0, p.rot_b != 0, d.index_bits == 4), grid, block, smem, s,
-                   pl.Gs, p);
+    const bool pair_t = B > 1, resid = d.residual_group != 0;
+    const eva_vq_linear::Plan &pl = h->plan[pair_t ? 1 : 0];
+    e = launch_pdl(lookup_fn(pair_t, resid, h->tiles_per_cb != 0, p.rot_b != 0, d.index_bits == 4),
+                   dim3(pl.Gs * pl.Gt), dim3(kThreads), smem, s, pl.Gs, p);
     if (e != cudaSuccess) return cuda_status(e);
-    ++kernels;
-    h->last_grid = (int)grid.x;
-    h->last_kernels = kernels;
+    h->last_grid = pl.Gs * pl.Gt;
+    h->last_kernels = 1;
     h->last_path = EVA_PATH_OC_LOOKUP;
+    return EVA_OK;
+}
+
+eva_status_t eva_vq_linear_run_group(const eva_vq_linear_t *hs, const void *const *xs, void *const *ys,
+                                     int32_t count, int32_t B, eva_stream_t stream, uint32_t flags) {
+    if (!hs || !xs || !ys || count < 1 || count > kMaxGroup) return EVA_ERR_INVALID_ARG;
+    if (flags & ~(uint32_t)EVA_RUN_INDEPENDENT) return EVA_ERR_INVALID_ARG;
+    for (int i = 0; i < count; ++i) {
+        const eva_vq_linear_t h = hs[i];
+        if (!h || !xs[i] || !ys[i] || !aligned16(xs[i]) || !aligned16(ys[i])) return EVA_ERR_INVALID_ARG;
+        if (B < 1 || B > h->desc.max_batch || h->device != hs[0]->device) return EVA_ERR_INVALID_ARG;
+    }
+    // One launch when every layer has the first one's shape and format.
+    const eva_vq_desc &d0 = hs[0]->desc;
+    bool one = groupable(hs[0], B);
+    for (int i = 1; i < count && one; ++i) {
+        const eva_vq_desc &d = hs[i]->desc;
+        one = groupable(hs[i], B) && d.N == d0.N && d.K == d0.K && d.residual_group == d0.residual_group &&
+              d.out_dtype == d0.out_dtype;
+    }
+    if (!one) {
+        for (int i = 0; i < count; ++i) {
+            const eva_status_t st = eva_vq_linear_run_ex(hs[i], xs[i], B, ys[i], stream, flags);
+            if (st != EVA_OK) return st;
+        }
+        return EVA_OK;
+    }
+    const int independent = (flags & EVA_RUN_INDEPENDENT) ? 1 : 0;
+    LookupGroup g;
+    std::memset(&g, 0, sizeof(g));
+    size_t smem = 0;
+    for (int i = 0; i < count; ++i) g.p[i] = call_params(hs[i], xs[i], B, ys[i], independent, &smem);
+    const bool pair_t = B > 1;
+    const eva_vq_linear::Plan &pl = hs[0]->plan[pair_t ? 1 : 0];
+    g.count = count;
+    g.ctas_per_layer = pl.Gs * pl.Gt;
+    const cudaError_t e = launch_pdl(group_fn(pair_t, d0.residual_group != 0), dim3(count * pl.Gs * pl.Gt),
+                                     dim3(kThreads), smem, reinterpret_cast<cudaStream_t>(stream), pl.Gs, g);
+    if (e != cudaSuccess) return cuda_status(e);
+    for (int i = 0; i < count; ++i) {
+        hs[i]->last_grid = pl.Gs * pl.Gt;
+        hs[i]->last_kernels = 1;
+        hs[i]->last_path = EVA_PATH_OC_LOOKUP;
+    }
     return EVA_OK;
 }
 

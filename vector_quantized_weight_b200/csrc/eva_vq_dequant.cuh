@@ -51,7 +51,8 @@ __global__ void __launch_bounds__(kThreads, 1) eva_dequant_kernel(const LookupPa
     constexpr uint32_t BLK = kTileRows * TT * 4u;       // bytes of one tile's sums
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, q = lane & 3;
-    const int ts = blockIdx.x % p.Gs, tt = blockIdx.x / p.Gs;
+    const int eva_bid = blockIdx.x;
+    const int ts = eva_bid % p.Gs, tt = eva_bid / p.Gs;
     const int s0 = (int)((long long)p.S * ts / p.Gs), s1 = (int)((long long)p.S * (ts + 1) / p.Gs);
     const int t0 = (int)((long long)p.T * tt / p.Gt), t1 = (int)((long long)p.T * (tt + 1) / p.Gt);
     const int ntw = (t1 - t0 - warp + kWarps - 1) / kWarps;
@@ -250,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1) eva_dequant_kernel(const LookupPa
     if (tid == 0) {
         unsigned smid;
         asm volatile("mov.u32 %0, %smid;" : "=r"(smid));
-        p.timeline[blockIdx.x * 8 + 7] = smid;
+        p.timeline[eva_bid * 8 + 7] = smid;
     }
 #endif
 }

@@ -77,7 +77,7 @@ __device__ __forceinline__ unsigned long long eva_globaltimer() {
     asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
     return t;
 }
-#define EVA_STAMP(ph) do { if (threadIdx.x == 0) p.timeline[blockIdx.x * 8 + (ph)] = eva_globaltimer(); } while (0)
+#define EVA_STAMP(ph) do { if (threadIdx.x == 0) p.timeline[eva_bid * 8 + (ph)] = eva_globaltimer(); } while (0)
 #else
 #define EVA_STAMP(ph) do { } while (0)
 #endif
@@ -778,8 +778,9 @@ __device__ __forceinline__ void load_unit(const LookupParams &p, const uint8_t *
 // so the weight stream of layer l+1 overlaps the lookups of layer l; the
 // token-pair and residual variants need more registers and run one CTA per SM.
 
+// The whole per-CTA program; eva_bid is the CTA's index within its layer.
 template <bool PAIR_T, bool RESID, bool GROUPED, bool ROT, bool NIB>
-__global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_lookup_kernel(const LookupParams p) {
+__device__ __forceinline__ void lookup_body(const LookupParams &p, const int eva_bid) {
     // NIB: 4-bit indices (16 centroids), units of 512 bytes (16 per lane).
     constexpr uint32_t UB = NIB ? (uint32_t)kUnitBytes4 : (uint32_t)kUnitBytes;
     // Index units in flight per warp: with per-group codebooks a warp has at
@@ -787,7 +788,7 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
     constexpr int LA = GROUPED ? 2 : kLookahead;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, q = lane & 3;
-    const int ts = blockIdx.x % p.Gs, tt = blockIdx.x / p.Gs;
+    const int ts = eva_bid % p.Gs, tt = eva_bid / p.Gs;
     const int s0 = (int)((long long)p.S * ts / p.Gs), s1 = (int)((long long)p.S * (ts + 1) / p.Gs);
     const int t0 = (int)((long long)p.T * tt / p.Gt), t1 = (int)((long long)p.T * (tt + 1) / p.Gt);
     const int ntw = (t1 - t0 - warp + kWarps - 1) / kWarps;  // tiles owned by this warp
@@ -1125,9 +1126,30 @@ __global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_looku
     if (tid == 0) {
         unsigned smid;
         asm volatile("mov.u32 %0, %smid;" : "=r"(smid));
-        p.timeline[blockIdx.x * 8 + 7] = smid;
+        p.timeline[eva_bid * 8 + 7] = smid;
     }
 #endif
+}
+
+template <bool PAIR_T, bool RESID, bool GROUPED, bool ROT, bool NIB>
+__global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_lookup_kernel(const LookupParams p) {
+    lookup_body<PAIR_T, RESID, GROUPED, ROT, NIB>(p, blockIdx.x);
+}
+
+// Several independent layers of one shape and format in one launch: layer
+// blockIdx.x / ctas_per_layer, CTA blockIdx.x % ctas_per_layer of it (a
+// cluster never spans two layers: ctas_per_layer is a multiple of Gs).
+constexpr int kMaxGroup = 16;
+struct LookupGroup {
+    int count, ctas_per_layer;
+    LookupParams p[kMaxGroup];
+};
+
+template <bool PAIR_T, bool RESID>
+__global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_lookup_group_kernel(const LookupGroup g) {
+    const int li = blockIdx.x / g.ctas_per_layer;
+    if (li >= g.count) return;
+    lookup_body<PAIR_T, RESID, false, false, false>(g.p[li], blockIdx.x - li * g.ctas_per_layer);
 }
 
 // ----------------------------------------------------- Hadamard rotation

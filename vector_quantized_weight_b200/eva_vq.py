@@ -26,6 +26,7 @@ ABI_FUNCTIONS = (
     "eva_vq_status_string", "eva_vq_linear_info", "eva_vq_device_check_record",
     "eva_vq_debug_timeline", "eva_vq_linear_run_noalloc",
     "eva_vq_quantize", "eva_vq_kmeans_assign", "eva_vq_kmeans_update", "eva_vq_residual",
+    "eva_vq_linear_run_group",
 )
 
 
@@ -96,6 +97,7 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.eva_vq_linear_run.argtypes = [H, P, I32, P, P]
     lib.eva_vq_linear_run_ex.argtypes = [H, P, I32, P, P, ctypes.c_uint32]
     lib.eva_vq_linear_run_noalloc.argtypes = [H, P, I32, P, P]
+    lib.eva_vq_linear_run_group.argtypes = [P, P, P, I32, I32, P, ctypes.c_uint32]
     lib.eva_vq_linear_run_host.argtypes = [H, P, I32, P, P]
     lib.eva_vq_linear_destroy.argtypes = [H]
     lib.eva_vq_unpack_indices.argtypes = [H, P, P]
@@ -150,6 +152,16 @@ def eva_vq_linear_run_noalloc(h: int, x: int, B: int, y: int, stream: int | None
     scratch comes from the library's 4 MiB static device array (see the
     header for who needs this and the sharing rules)."""
     _check("eva_vq_linear_run_noalloc", load().eva_vq_linear_run_noalloc(h, x, int(B), y, stream))
+
+
+def eva_vq_linear_run_group(hs: list, xs: list, ys: list, B: int, stream: int | None, flags: int = 0) -> None:
+    """Independent layers in one launch where their shapes and formats allow
+    (see the header); hs, xs, ys are lists of handles and device pointers."""
+    n = len(hs)
+    ha = (ctypes.c_void_p * n)(*hs)
+    xa = (ctypes.c_void_p * n)(*xs)
+    ya = (ctypes.c_void_p * n)(*ys)
+    _check("eva_vq_linear_run_group", load().eva_vq_linear_run_group(ha, xa, ya, n, int(B), stream, int(flags)))
 
 
 def eva_vq_linear_run_host(h: int, x_host: int, B: int, y_host: int, stream: int | None) -> None:
@@ -330,3 +342,15 @@ def quantize(w, init_index, iters: int, *, hsign=None, hadamard_block: int = 0, 
                     _ptr(out["wi"]), _ptr(out.get("signs")), _ptr(out.get("alpha")), _ptr(out.get("wrot")),
                     _ptr(out.get("centroids")), _stream_handle(stream))
     return out
+
+
+def run_group(layers, xs, outs=None, stream=None, independent=False):
+    """Run VQLinear layers on their inputs (CUDA fp16 [B][K] tensors, one B)
+    as one grouped call; returns the outputs."""
+    import torch
+    B = xs[0].shape[0]
+    if outs is None:
+        outs = [torch.empty((B, l.N), dtype=l.out_dtype, device=x.device) for l, x in zip(layers, xs)]
+    eva_vq_linear_run_group([l.handle for l in layers], [x.data_ptr() for x in xs], [y.data_ptr() for y in outs],
+                            B, _stream_handle(stream), EVA_RUN_INDEPENDENT if independent else 0)
+    return outs

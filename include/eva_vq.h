@@ -6,8 +6,9 @@
  * Quantization Architecture, technical summary section 2.A):
  *   - the input x of one decode step is cut into J = K/d sub-vectors x_j of
  *     length d (d = 4);
- *   - the weight codebook WC holds 2^n centroids of length d (n = 8, so 256
- *     centroids and one index byte per 4 weights: 2 bits per weight);
+ *   - the weight codebook WC holds 2^n centroids of length d (n = 8: 256
+ *     centroids and one index byte per 4 weights, 2 bits per weight; or
+ *     n = 4: 16 centroids, two indices per byte, 1 bit per weight);
  *   - the output codebook OC[j][c] = <x_j, WC[c]> turns the matrix-vector
  *     product into a small matrix-matrix product;
  *   - the output is gathered through the weight-index matrix WI and summed:
@@ -45,7 +46,7 @@ typedef struct CUstream_st *eva_stream_t;
 typedef enum {
     EVA_OK = 0,
     EVA_ERR_INVALID_ARG = 1,     /* bad pointer, size, alignment or handle      */
-    EVA_ERR_UNSUPPORTED = 2,     /* valid but not implemented (d != 4, n != 8)   */
+    EVA_ERR_UNSUPPORTED = 2,     /* valid but not implemented (d != 4, n not 4/8) */
     EVA_ERR_CUDA = 3,            /* a CUDA runtime call failed                   */
     EVA_ERR_OOM = 4,             /* device allocation failed in create           */
     EVA_ERR_DEVICE_TIMEOUT = 5,  /* a bounded device wait gave up                */
@@ -60,7 +61,9 @@ typedef enum { EVA_F16 = 0, EVA_F32 = 1 } eva_dtype_t;
 typedef enum {
     EVA_PATH_AUTO = 0,        /* pick per call from B and the codebook layout   */
     EVA_PATH_OC_LOOKUP = 1,   /* output codebook in shared memory + lookups     */
-    EVA_PATH_DEQUANT_MMA = 2  /* codebook gather into tensor-core operands      */
+    EVA_PATH_DEQUANT_MMA = 2  /* codebook gather into tensor-core operands (8-bit
+                                 indices, no residual, no rotation); AUTO takes
+                                 it for B >= 4 when the layer allows it          */
 } eva_path_t;
 
 typedef struct {

@@ -106,7 +106,7 @@ def test_create_without_device_reports_no_device():
 
 
 def test_kernels_do_not_spill():
-    """ptxas report of every kernel (16 lookup instances, 4 dequantize
+    """ptxas report of every kernel (the lookup instances, the dequantize
     instances, the rotation, repack and quantizer kernels): no local-memory
     stack frame and no spills (hot loops keep everything in registers)."""
     cmd = [build._nvcc(), *[f for f in build.NVCC_FLAGS if f != "-shared"], "-Xptxas", "-v", "-c",
@@ -114,7 +114,8 @@ def test_kernels_do_not_spill():
     out = subprocess.run(cmd, capture_output=True, text=True, check=True).stderr
     blocks = re.findall(r"Function properties for (\S*eva_\w+_kernel\S*)\n\s*(\d+) bytes stack frame, "
                         r"(\d+) bytes spill stores, (\d+) bytes spill loads", out)
-    assert sum("eva_lookup_kernel" in b[0] for b in blocks) == 20, out
+    assert sum("eva_lookup_kernelI" in b[0] for b in blocks) == 20, out     # 16 + 4 with 4-bit indices
+    assert sum("eva_lookup_kernel3I" in b[0] for b in blocks) == 3, out     # three CTAs per SM
     assert sum("eva_dequant_kernel" in b[0] for b in blocks) == 4, out
     assert sum("eva_kmeans_assign_kernel" in b[0] for b in blocks) == 2, out
     for name, stack, st, ld in blocks:

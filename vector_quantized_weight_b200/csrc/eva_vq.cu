@@ -152,9 +152,13 @@ size_t lookup_smem(bool pair_t, bool resid, int tiles, int gs, int rot_b, int s_
                    size_t unit_bytes = kUnitBytes) {
     const size_t tile_bytes = (size_t)kTileRows * 2 * 4;
     const size_t stage_tiles = (size_t)((tiles + gs - 1) / gs) * gs;   // reduction stage
-    const size_t base = (size_t)kOcBytes + ((pair_t && resid) ? (size_t)kOcBytes : 0) +
-                        (pair_t ? kXStageBytes : kXStageBytes / 2) + 128 + (size_t)tiles * tile_bytes +
-                        stage_tiles * tile_bytes;
+    // One token without residual table or rotation: x~, mbarrier and running
+    // sums sit in the image rows' unused halves; only the stage follows.
+    const bool gaps = !pair_t && !resid && !rot_b && !kNaiveOcBuild;
+    const size_t base = gaps ? (size_t)kOcBytes + stage_tiles * tile_bytes
+                             : (size_t)kOcBytes + ((pair_t && resid) ? (size_t)kOcBytes : 0) +
+                                   (pair_t ? kXStageBytes : kXStageBytes / 2) + 128 + (size_t)tiles * tile_bytes +
+                                   stage_tiles * tile_bytes;
     const int ntok = pair_t ? 2 : 1;
     const size_t xt = paley_m(rot_b) >= 256 ? (size_t)((s_total + gs - 1) / gs) * ntok * kSliceK * 4 : 0;
     const size_t rot = rot_b ? xt + rot_scratch_bytes(rot_b, paley_m(rot_b), ntok) : 0;
@@ -202,6 +206,16 @@ LookupFn lookup_fn(bool pair_t, bool resid, bool grouped, bool rot, bool nib = f
         return resid ? eva_lookup_kernel<true, true, false, false, true> : eva_lookup_kernel<true, false, false, false, true>;
     }
     return rot ? lookup_fn_r<true>(pair_t, resid, grouped) : lookup_fn_r<false>(pair_t, resid, grouped);
+}
+
+// Three CTAs per SM (eva_lookup_kernel3): one token, no residual table, no
+// rotation, and few enough tiles per CTA that the tighter register budget
+// costs less than the third layer in flight gains (measured: 37 tiles of a
+// 4096 x 4096 layer gain, 77 tiles of 11008 x 4096 lose).
+constexpr int kThreePerSmMaxTiles = 48;
+LookupFn lookup_fn3(bool grouped, bool nib) {
+    if (nib) return eva_lookup_kernel3<false, true>;
+    return grouped ? eva_lookup_kernel3<true, false> : eva_lookup_kernel3<false, false>;
 }
 
 // Largest number of clusters of `cs` CTAs of this kernel resident at once.
@@ -371,6 +385,13 @@ cudaError_t set_smem_attrs(int smem_optin) {
         e = cudaFuncSetAttribute((const void *)fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_optin);
         if (e != cudaSuccess) return e;
     }
+    for (int v = 0; v < 3; ++v) {
+        const LookupFn fn = lookup_fn3(v == 1, v == 2);
+        e = cudaFuncSetAttribute((const void *)fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute((const void *)fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_optin);
+        if (e != cudaSuccess) return e;
+    }
     for (int v = 0; v < 4; ++v) {
         const void *fn = v == 0 ? (const void *)eva_lookup_group_kernel<false, false>
                        : v == 1 ? (const void *)eva_lookup_group_kernel<false, true>
@@ -401,6 +422,13 @@ cudaError_t launch_dequant(eva_vq_linear *h, LookupParams p, int B, cudaStream_t
 #endif
     return launch_pdl(dequant_fn(h->tiles_per_cb != 0, ntg), dim3(pl.Gs * pl.Gt), dim3(kThreads), pl.smem, s,
                       pl.Gs, p);
+}
+
+bool use_three_per_sm(const eva_vq_linear *h, int B) {
+    const eva_vq_desc &d = h->desc;
+    if (B > 1 || d.residual_group || d.hadamard_block || kNaiveOcBuild) return false;
+    const eva_vq_linear::Plan &pl = h->plan[0];
+    return (h->T + pl.Gt - 1) / pl.Gt <= kThreePerSmMaxTiles;
 }
 
 bool use_dequant(const eva_vq_linear *h, int B) {
@@ -683,8 +711,9 @@ eva_status_t eva_vq_linear_run_ex(eva_vq_linear_t h, const void *x, int32_t B, v
     }
     const bool pair_t = B > 1, resid = d.residual_group != 0;
     const eva_vq_linear::Plan &pl = h->plan[pair_t ? 1 : 0];
-    e = launch_pdl(lookup_fn(pair_t, resid, h->tiles_per_cb != 0, p.rot_b != 0, d.index_bits == 4),
-                   dim3(pl.Gs * pl.Gt), dim3(kThreads), smem, s, pl.Gs, p);
+    LookupFn fn = lookup_fn(pair_t, resid, h->tiles_per_cb != 0, p.rot_b != 0, d.index_bits == 4);
+    if (independent && use_three_per_sm(h, B)) fn = lookup_fn3(h->tiles_per_cb != 0, d.index_bits == 4);
+    e = launch_pdl(fn, dim3(pl.Gs * pl.Gt), dim3(kThreads), smem, s, pl.Gs, p);
     if (e != cudaSuccess) return cuda_status(e);
     h->last_grid = pl.Gs * pl.Gt;
     h->last_kernels = 1;

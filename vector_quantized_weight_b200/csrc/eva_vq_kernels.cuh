@@ -283,6 +283,17 @@ __device__ __forceinline__ float load_x(const LookupParams &p, int tok, int k) {
 // with 128-bit loads when aligned; zeros past K or past B.
 constexpr uint32_t kXStageBytes = 2u * kSliceK * 4u;   // room for a token pair
 
+// Layout of a one-token image without residual table: only columns 0..31 of
+// its 256-byte rows are lookups; the other 128 bytes of each row ("gaps")
+// hold the running sums (row tl: tile tl, tl < 248), the staging mbarrier
+// (row 247) and the x~ slice (rows 248..255, 32 floats each).  x_off ==
+// kXGaps selects that x~ layout.
+constexpr uint32_t kXGaps = 0xFFFF0000u;
+__host__ __device__ constexpr uint32_t gap_off(int row) { return (uint32_t)row * kOcRowBytes + 128u; }
+__device__ __forceinline__ uint32_t x_addr(uint32_t x_off, int idx) {
+    return x_off == kXGaps ? gap_off(248 + (idx >> 5)) + 4u * (uint32_t)(idx & 31) : x_off + 4u * (uint32_t)idx;
+}
+
 template <bool PAIR_T>
 __device__ __forceinline__ void stage_x(const LookupParams &p, int s, int pr, int warp, int lane,
                                         uint32_t x_off) {
@@ -321,7 +332,7 @@ __device__ __forceinline__ void stage_x(const LookupParams &p, int s, int pr, in
 #pragma unroll
         for (int j = 0; j < 8; ++j) v[j] = load_x(p, tok, k0 + j);
     }
-    const uint32_t off = x_off + (uint32_t)(warp * kSliceK + 8 * lane) * 4u;
+    const uint32_t off = x_addr(x_off, warp * kSliceK + 8 * lane);   // 8 floats, inside one gap
     if (!EVA_BAD_S(off) && !EVA_BAD_S(off + 28u)) {
         *reinterpret_cast<float4 *>(eva_smem + off) = make_float4(v[0], v[1], v[2], v[3]);
         *reinterpret_cast<float4 *>(eva_smem + off + 16) = make_float4(v[4], v[5], v[6], v[7]);
@@ -601,7 +612,7 @@ __device__ __forceinline__ void stage_x_rot(const LookupParams &p, int s, int pr
 }
 
 __device__ __forceinline__ float lds_x(const LookupParams &p, uint32_t x_off, int idx) {
-    const uint32_t off = x_off + 4u * (uint32_t)idx;
+    const uint32_t off = x_addr(x_off, idx);
     return EVA_BAD_S(off) ? 0.f : *reinterpret_cast<const float *>(eva_smem + off);
 }
 
@@ -778,6 +789,15 @@ __device__ __forceinline__ void load_unit(const LookupParams &p, const uint8_t *
 // so the weight stream of layer l+1 overlaps the lookups of layer l; the
 // token-pair and residual variants need more registers and run one CTA per SM.
 
+// Instances whose image rows lend their unused halves to x~, the mbarrier and
+// the running sums (one token, no residual table, no rotation; not the naive
+// diagnostics layout).  Their smaller footprint lets three CTAs share an SM
+// (eva_lookup_kernel3, compiled for that register budget).
+template <bool PAIR_T, bool RESID, bool ROT>
+constexpr bool kImageGaps = !PAIR_T && !RESID && !ROT && !kNaiveOcBuild;
+template <bool PAIR_T, bool RESID, bool ROT>
+constexpr int kLookupMinBlocks = (PAIR_T || RESID) ? 1 : 2;
+
 // The whole per-CTA program; eva_bid is the CTA's index within its layer.
 template <bool PAIR_T, bool RESID, bool GROUPED, bool ROT, bool NIB>
 __device__ __forceinline__ void lookup_body(const LookupParams &p, const int eva_bid) {
@@ -796,13 +816,22 @@ __device__ __forceinline__ void lookup_body(const LookupParams &p, const int eva
     constexpr uint32_t OC_OFF = 0;
     constexpr uint32_t HI_OFF = PAIR_T ? 128u : 0u;                      // a2/a3 column offset
     constexpr uint32_t T_OFF = PAIR_T ? (uint32_t)kOcBytes : 128u;       // residual table
-    constexpr uint32_t X_OFF = (PAIR_T && RESID) ? 2u * kOcBytes : (uint32_t)kOcBytes;
-    constexpr uint32_t XS_BYTES = PAIR_T ? kXStageBytes : kXStageBytes / 2;   // x~ of 1 or 2 tokens
-    constexpr uint32_t BAR_OFF = X_OFF + XS_BYTES;       // mbarrier of the index staging copy
-    constexpr uint32_t ACC_OFF = BAR_OFF + 128u;         // per-CTA running sums (128-byte
-                                                         // tile blocks stay 128-byte aligned)
     constexpr int NTOK_C = PAIR_T ? 2 : 1;
     constexpr bool NAIVE = kNaiveOcBuild && !PAIR_T && !RESID && !NIB;
+    // One token, no residual table, no rotation: x~, the mbarriers and the
+    // running sums live in the image rows' unused halves (kXGaps).
+    constexpr bool GAPS = kImageGaps<PAIR_T, RESID, ROT>;
+    constexpr uint32_t X_OFF = GAPS ? kXGaps : ((PAIR_T && RESID) ? 2u * kOcBytes : (uint32_t)kOcBytes);
+    constexpr uint32_t XS_BYTES = PAIR_T ? kXStageBytes : kXStageBytes / 2;   // x~ of 1 or 2 tokens
+    // mbarriers: index staging copy (+0), 8 bytes each
+    constexpr uint32_t BAR_OFF = GAPS ? gap_off(247) : X_OFF + XS_BYTES;
+    constexpr uint32_t ACC_OFF = GAPS ? (uint32_t)kOcBytes : BAR_OFF + 128u;   // (gaps: unused)
+    // Running sums of tile tl: 128 bytes [16 rows][2 tokens] fp32.
+    auto acc_off = [&](int tl) -> uint32_t {
+        return GAPS ? gap_off(tl) : ACC_OFF + (uint32_t)tl * kTileRows * 2u * 4u;
+    };
+    // The reduction stage starts after the image (gaps) or after the sums.
+    const uint32_t STAGE_OFF = GAPS ? (uint32_t)kOcBytes : ACC_OFF + (uint32_t)p.acc_tiles * kTileRows * 2u * 4u;
     // GROUPED: one codebook per tiles_per_cb row tiles (else one shared codebook).
     const int cb_first = GROUPED ? t0 / p.tiles_per_cb : 0;
     const int cb_last = GROUPED ? (t1 - 1) / p.tiles_per_cb : 0;
@@ -819,7 +848,7 @@ __device__ __forceinline__ void lookup_body(const LookupParams &p, const int eva
     const uint32_t stage_bytes_c = (uint32_t)((p.acc_tiles + p.Gs - 1) / p.Gs) * p.Gs * kTileRows * 2u * 4u;
     // Fused rotation: x~ of all this CTA's slices [ceil(S / Gs)][tokens][256]
     // fp32, then the rotation's scratch.
-    const uint32_t ROT_OFF = (ACC_OFF + (uint32_t)p.acc_tiles * kTileRows * 2u * 4u + stage_bytes_c + 127u) & ~127u;
+    const uint32_t ROT_OFF = (STAGE_OFF + stage_bytes_c + 127u) & ~127u;
     const bool rot_all = ROT && p.rot_m >= 256;   // Paley m >= 256: all slices at once
     const uint32_t xt_bytes = rot_all ? (uint32_t)((p.S + p.Gs - 1) / p.Gs) * NTOK_C * kSliceK * 4u : 0u;
     const uint32_t rot_bytes = ROT ? xt_bytes + rot_scratch_bytes(p.rot_b, p.rot_m, NTOK_C) : 0u;
@@ -890,8 +919,6 @@ __device__ __forceinline__ void lookup_body(const LookupParams &p, const int eva
     // bytes per tile), and the reduction stage of the tiles this CTA owns
     // (tile tl belongs to cluster rank tl % Gs):
     // [ceil(acc_tiles / Gs) slots][Gs sources][16 rows][2 tokens].
-    float *acc_s = reinterpret_cast<float *>(eva_smem + ACC_OFF);
-    const uint32_t STAGE_OFF = ACC_OFF + (uint32_t)p.acc_tiles * kTileRows * 2u * 4u;
     bool wi_ready = false;   // the staging copy has landed (waited for once)
     const float *stage = reinterpret_cast<const float *>(eva_smem + STAGE_OFF);
     const uint32_t stage_addr = (uint32_t)__cvta_generic_to_shared(eva_smem + STAGE_OFF);
@@ -1035,9 +1062,11 @@ __device__ __forceinline__ void lookup_body(const LookupParams &p, const int eva
                         for (int h = 0; h < 2; ++h)
 #pragma unroll
                             for (int e = 0; e < NTOK; ++e) {
-                                const int ai = (tl * kTileRows + g + 8 * h) * 2 + e;
-                                if (!EVA_BAD_S(ACC_OFF + 4u * (uint32_t)ai))
-                                    acc_s[ai] = (s == s0) ? da[2 * h + e] : acc_s[ai] + da[2 * h + e];
+                                const uint32_t ao = acc_off(tl) + (uint32_t)((g + 8 * h) * 2 + e) * 4u;
+                                if (!EVA_BAD_S(ao)) {
+                                    float *ap = reinterpret_cast<float *>(eva_smem + ao);
+                                    *ap = (s == s0) ? da[2 * h + e] : *ap + da[2 * h + e];
+                                }
                             }
                     }
                 };
@@ -1080,7 +1109,7 @@ __device__ __forceinline__ void lookup_body(const LookupParams &p, const int eva
         __syncthreads();
         for (int i = tid; i < ctiles * 8; i += kThreads) {
             const int tl = i >> 3, chunk = i & 7;
-            const uint32_t src = ACC_OFF + (uint32_t)(tl * 32 + chunk * 4) * 4u;
+            const uint32_t src = acc_off(tl) + (uint32_t)(chunk * 4) * 4u;
             const uint32_t dst = (uint32_t)((((tl / p.Gs) * p.Gs + ts) * 32 + chunk * 4) * 4);
             if (!EVA_BAD_S(src) && !EVA_BAD_S(src + 12u) && !EVA_BAD_S(STAGE_OFF + dst) && !EVA_BAD_S(STAGE_OFF + dst + 12u)) {
                 const float4 v = *reinterpret_cast<const float4 *>(eva_smem + src);
@@ -1132,8 +1161,16 @@ __device__ __forceinline__ void lookup_body(const LookupParams &p, const int eva
 }
 
 template <bool PAIR_T, bool RESID, bool GROUPED, bool ROT, bool NIB>
-__global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_lookup_kernel(const LookupParams p) {
+__global__ void __launch_bounds__(kThreads, (kLookupMinBlocks<PAIR_T, RESID, ROT>)) eva_lookup_kernel(const LookupParams p) {
     lookup_body<PAIR_T, RESID, GROUPED, ROT, NIB>(p, blockIdx.x);
+}
+
+// The one-token, no-residual, no-rotation program with the register budget of
+// three CTAs per SM: for independent calls of layers with few tiles per CTA,
+// where a third layer in flight outweighs the tighter registers.
+template <bool GROUPED, bool NIB>
+__global__ void __launch_bounds__(kThreads, 3) eva_lookup_kernel3(const LookupParams p) {
+    lookup_body<false, false, GROUPED, false, NIB>(p, blockIdx.x);
 }
 
 // Several independent layers of one shape and format in one launch: layer
@@ -1146,7 +1183,7 @@ struct LookupGroup {
 };
 
 template <bool PAIR_T, bool RESID>
-__global__ void __launch_bounds__(kThreads, (PAIR_T || RESID) ? 1 : 2) eva_lookup_group_kernel(const LookupGroup g) {
+__global__ void __launch_bounds__(kThreads, (kLookupMinBlocks<PAIR_T, RESID, false>)) eva_lookup_group_kernel(const LookupGroup g) {
     const int li = blockIdx.x / g.ctas_per_layer;
     if (li >= g.count) return;
     lookup_body<PAIR_T, RESID, false, false, false>(g.p[li], blockIdx.x - li * g.ctas_per_layer);

@@ -151,11 +151,14 @@ def test_run_rejects_bad_arguments():
     lin.close()
 
 
-@pytest.mark.parametrize("key,li,B", [("llama7b_layer", 0, 1), ("llama7b_block", 6, 4), ("gemma_3bit", 0, 1),
-                                      ("llama70b", 0, 8)])
+@pytest.mark.parametrize("key,li,B", [("llama7b_layer", 0, 1), ("llama7b_layer", 0, 2), ("llama7b_block", 4, 1),
+                                      ("llama7b_block", 6, 1), ("llama7b_block", 6, 4), ("gemma_3bit", 0, 1),
+                                      ("gemma_3bit", 1, 1), ("gemma_3bit_rotK", 0, 1), ("gemma_3bit_rotK", 0, 2),
+                                      ("llama70b", 0, 1), ("llama70b", 0, 8), ("llama7b_layer_4bit", 0, 1)])
 def test_independent_flag_matches_plain_run(key, li, B):
-    """EVA_RUN_INDEPENDENT only relaxes ordering: results are bitwise those of
-    the plain call, also for back-to-back calls on one handle (distinct y)."""
+    """EVA_RUN_INDEPENDENT relaxes ordering and takes a grid with fewer row
+    groups (the same slice split): results are bitwise those of the plain
+    call, also for back-to-back calls on one handle (distinct y)."""
     import torch
     from vector_quantized_weight_b200 import eva_vq
     cfg = synth.CONFIGS[key]

@@ -34,7 +34,11 @@ struct eva_vq_linear {
     // (one cluster) x Gt row groups, and its dynamic shared memory.
     // `staged` index units per CTA are copied into shared memory up front
     // (`smem`); calls flagged independent skip that copy (`smem_nostage`).
-    struct Plan { int Gs = 1, Gt = 1, staged = 0; size_t smem = 0, smem_nostage = 0; } plan[2];
+    struct Plan { int Gs = 1, Gt = 1, staged = 0; size_t smem = 0, smem_nostage = 0; };
+    // Lookup-path grids for one token and for token pairs: plan[] for calls
+    // that wait for their predecessor (one layer's latency), iplan[] for
+    // calls flagged independent (CTA-slot time per layer).
+    Plan plan[2], iplan[2];
     // Dequantize-to-tensor-core path (no residual, no rotation): plans for 8
     // and 16 tokens per pass.
     bool dq_ok = false;
@@ -283,6 +287,38 @@ void plan_grid(eva_vq_linear *h, int pair_t) {
     pl.smem = lookup_smem(pair_t, resid, tiles, pl.Gs, h->desc.hadamard_block, S, pl.staged, h->unit_bytes);
     pl.smem_nostage = lookup_smem(pair_t, resid, tiles, pl.Gs, h->desc.hadamard_block, S, 0);
     h->plan[pair_t] = pl;
+
+    // Independent calls overlap with their neighbours, so a layer costs the
+    // CTA slots it holds times how long it holds them, and every CTA pays the
+    // same fixed part (x~ staging, image build, cluster reduction) whatever
+    // its tile count.  Their grid therefore keeps the slice split and takes
+    // as few row groups as the per-CTA tile limit allows (the row-gap layout
+    // holds up to kMaxGapTiles running sums; with per-group codebooks more
+    // tiles per CTA also mean more image builds per CTA, so those stay at
+    // kMaxCtaTiles), without a larger footprint than two CTAs per SM (or the
+    // latency plan's own) permit.
+    eva_vq_linear::Plan ip = pl;
+    ip.staged = 0;
+    ip.smem = ip.smem_nostage = pl.smem_nostage;
+    const bool gaps = !pair_t && !resid && !h->desc.hadamard_block && !kNaiveOcBuild;
+    const int max_tiles = (gaps && !h->tiles_per_cb) ? kMaxGapTiles : kMaxCtaTiles;
+    const size_t two = (size_t)h->smem_per_sm / 2 - (size_t)h->smem_reserved;
+    const size_t fit = std::min(std::max(pl.smem_nostage, two), (size_t)h->smem_optin);
+    for (int gt = (T + max_tiles - 1) / max_tiles; gt < pl.Gt; ++gt) {
+        const size_t sm = lookup_smem(pair_t, resid, (T + gt - 1) / gt, pl.Gs, h->desc.hadamard_block, S, 0,
+                                      h->unit_bytes);
+        if (sm <= fit) {
+            ip.Gt = gt;
+            ip.smem = ip.smem_nostage = sm;
+            break;
+        }
+    }
+    h->iplan[pair_t] = ip;
+}
+
+// The grid of a lookup-path call.
+const eva_vq_linear::Plan &call_plan(const eva_vq_linear *h, int B, int independent) {
+    return independent ? h->iplan[B > 1 ? 1 : 0] : h->plan[B > 1 ? 1 : 0];
 }
 
 // Launch with programmatic dependent launch (and a cluster shape when
@@ -424,10 +460,10 @@ cudaError_t launch_dequant(eva_vq_linear *h, LookupParams p, int B, cudaStream_t
                       pl.Gs, p);
 }
 
-bool use_three_per_sm(const eva_vq_linear *h, int B) {
+bool use_three_per_sm(const eva_vq_linear *h, int B, int independent) {
     const eva_vq_desc &d = h->desc;
     if (B > 1 || d.residual_group || d.hadamard_block || kNaiveOcBuild) return false;
-    const eva_vq_linear::Plan &pl = h->plan[0];
+    const eva_vq_linear::Plan &pl = call_plan(h, B, independent);
     return (h->T + pl.Gt - 1) / pl.Gt <= kThreePerSmMaxTiles;
 }
 
@@ -623,7 +659,7 @@ LookupParams call_params(eva_vq_linear *h, const void *x, int32_t B, void *y, in
     p.S = h->S;
     p.T = h->T;
     p.B = B;
-    const eva_vq_linear::Plan &pl = h->plan[B > 1 ? 1 : 0];
+    const eva_vq_linear::Plan &pl = call_plan(h, B, independent);
     p.Gs = pl.Gs;
     p.Gt = pl.Gt;
     p.acc_tiles = (h->T + pl.Gt - 1) / pl.Gt;
@@ -710,9 +746,9 @@ eva_status_t eva_vq_linear_run_ex(eva_vq_linear_t h, const void *x, int32_t B, v
         return EVA_OK;
     }
     const bool pair_t = B > 1, resid = d.residual_group != 0;
-    const eva_vq_linear::Plan &pl = h->plan[pair_t ? 1 : 0];
+    const eva_vq_linear::Plan &pl = call_plan(h, B, independent);
     LookupFn fn = lookup_fn(pair_t, resid, h->tiles_per_cb != 0, p.rot_b != 0, d.index_bits == 4);
-    if (independent && use_three_per_sm(h, B)) fn = lookup_fn3(h->tiles_per_cb != 0, d.index_bits == 4);
+    if (independent && use_three_per_sm(h, B, independent)) fn = lookup_fn3(h->tiles_per_cb != 0, d.index_bits == 4);
     e = launch_pdl(fn, dim3(pl.Gs * pl.Gt), dim3(kThreads), smem, s, pl.Gs, p);
     if (e != cudaSuccess) return cuda_status(e);
     h->last_grid = pl.Gs * pl.Gt;
@@ -751,7 +787,7 @@ eva_status_t eva_vq_linear_run_group(const eva_vq_linear_t *hs, const void *cons
     size_t smem = 0;
     for (int i = 0; i < count; ++i) g.p[i] = call_params(hs[i], xs[i], B, ys[i], independent, &smem);
     const bool pair_t = B > 1;
-    const eva_vq_linear::Plan &pl = hs[0]->plan[pair_t ? 1 : 0];
+    const eva_vq_linear::Plan &pl = call_plan(hs[0], B, independent);
     g.count = count;
     g.ctas_per_layer = pl.Gs * pl.Gt;
     const cudaError_t e = launch_pdl(group_fn(pair_t, d0.residual_group != 0), dim3(count * pl.Gs * pl.Gt),

@@ -285,10 +285,11 @@ constexpr uint32_t kXStageBytes = 2u * kSliceK * 4u;   // room for a token pair
 
 // Layout of a one-token image without residual table: only columns 0..31 of
 // its 256-byte rows are lookups; the other 128 bytes of each row ("gaps")
-// hold the running sums (row tl: tile tl, tl < 248), the staging mbarrier
-// (row 247) and the x~ slice (rows 248..255, 32 floats each).  x_off ==
-// kXGaps selects that x~ layout.
+// hold the running sums (row tl: tile tl, tl < kMaxGapTiles), the staging
+// mbarrier (row 247) and the x~ slice (rows 248..255, 32 floats each).
+// x_off == kXGaps selects that x~ layout.
 constexpr uint32_t kXGaps = 0xFFFF0000u;
+constexpr int kMaxGapTiles = 247;   // row tiles per CTA in this layout
 __host__ __device__ constexpr uint32_t gap_off(int row) { return (uint32_t)row * kOcRowBytes + 128u; }
 __device__ __forceinline__ uint32_t x_addr(uint32_t x_off, int idx) {
     return x_off == kXGaps ? gap_off(248 + (idx >> 5)) + 4u * (uint32_t)(idx & 31) : x_off + 4u * (uint32_t)idx;
@@ -772,6 +773,19 @@ __device__ __forceinline__ void load_unit(const LookupParams &p, const uint8_t *
     }
 }
 
+// The residual operands of one unit: its sign bytes (16 per lane) and, in
+// lanes q = 0, the alpha halves of rows g and g + 8.
+__device__ __forceinline__ void load_resid(const LookupParams &p, size_t unit, int lane, int g, int q, uint4 &sv,
+                                           uint2 &av) {
+    const uint8_t *sp = p.sg + unit * kSignUnitBytes + lane * 16;
+    sv = EVA_BAD_G(BUF_SG, sp, 16) ? make_uint4(0u, 0u, 0u, 0u) : ldg_stream(sp);
+    av = make_uint2(0u, 0u);
+    if (q == 0) {
+        const __half *ap = p.al + unit * kAlphaUnitHalves + 4 * g;
+        if (!EVA_BAD_G(BUF_AL, ap, 8)) av = *reinterpret_cast<const uint2 *>(ap);
+    }
+}
+
 // ------------------------------------------------------------ lookup kernel
 //
 // Grid: Gs x Gt CTAs in clusters of Gs; CTA (ts, tt) owns K-slices [s0, s1)
@@ -783,11 +797,11 @@ __device__ __forceinline__ void load_unit(const LookupParams &p, const uint8_t *
 // inside its cluster through distributed shared memory.
 //
 // Before the dependency wait the kernel only touches weights: the bulk L2
-// prefetch of its index range and the codebook fragments.  For one token
-// without residual the launch bounds of two CTAs per SM (128 registers) leave
+// prefetch of its index range and the codebook fragments.  For one token the
+// launch bounds of two CTAs per SM (128 registers; no instance spills) leave
 // room for the next layer's CTA to run that prologue while this one computes,
 // so the weight stream of layer l+1 overlaps the lookups of layer l; the
-// token-pair and residual variants need more registers and run one CTA per SM.
+// token-pair variants need more registers and run one CTA per SM.
 
 // Instances whose image rows lend their unused halves to x~, the mbarrier and
 // the running sums (one token, no residual table, no rotation; not the naive
@@ -795,8 +809,8 @@ __device__ __forceinline__ void load_unit(const LookupParams &p, const uint8_t *
 // (eva_lookup_kernel3, compiled for that register budget).
 template <bool PAIR_T, bool RESID, bool ROT>
 constexpr bool kImageGaps = !PAIR_T && !RESID && !ROT && !kNaiveOcBuild;
-template <bool PAIR_T, bool RESID, bool ROT>
-constexpr int kLookupMinBlocks = (PAIR_T || RESID) ? 1 : 2;
+template <bool PAIR_T>
+constexpr int kLookupMinBlocks = PAIR_T ? 1 : 2;
 
 // The whole per-CTA program; eva_bid is the CTA's index within its layer.
 template <bool PAIR_T, bool RESID, bool GROUPED, bool ROT, bool NIB>
@@ -948,13 +962,26 @@ __device__ __forceinline__ void lookup_body(const LookupParams &p, const int eva
                 // bulk prefetch put them) while the image builds, and each
                 // processed tile refills the ring's tail.
                 const int i_st = (s == s0) ? min(i1, max(i0, (staged - warp + kWarps - 1) / kWarps)) : i0;
+                // With a residual the ring also carries each unit's signs and alpha.
+                constexpr int LR = RESID ? LA : 1;
                 uint4 nb[LA][2];
+                uint4 ns[LR];
+                uint2 na[LR];
+                if constexpr (!RESID) {
+                    ns[0] = make_uint4(0u, 0u, 0u, 0u);
+                    na[0] = make_uint2(0u, 0u);
+                }
 #pragma unroll
                 for (int d = 0; d < LA; ++d) {
                     nb[d][0] = nb[d][1] = make_uint4(0u, 0u, 0u, 0u);
+                    if constexpr (RESID) {
+                        ns[d] = make_uint4(0u, 0u, 0u, 0u);
+                        na[d] = make_uint2(0u, 0u);
+                    }
                     if (i_st + d < i1) {
-                        const uint8_t *up = p.wi + ((size_t)s * p.T + t0 + warp + kWarps * (i_st + d)) * UB + 16 * lane;
-                        load_unit<NIB>(p, up, nb[d][0], nb[d][1]);
+                        const size_t unit = (size_t)s * p.T + t0 + warp + kWarps * (i_st + d);
+                        load_unit<NIB>(p, p.wi + unit * UB + 16 * lane, nb[d][0], nb[d][1]);
+                        if constexpr (RESID) load_resid(p, unit, lane, g, q, ns[d], na[d]);
                     }
                 }
                 // Paley blocks with m >= 256: x~ of every slice of this CTA at
@@ -977,7 +1004,7 @@ __device__ __forceinline__ void lookup_body(const LookupParams &p, const int eva
                     if (!mbar_wait_bounded(bar, 0) && tid == 0 && p.status) atomicOr(p.status, 1);
                 }
                 // One tile: 32 lookups per lane, accumulated by 8 MMAs (+ the residual).
-                auto tile = [&](const int tl, const size_t unit, const uint4 v0, const uint4 v1) {
+                auto tile = [&](const int tl, const uint4 v0, const uint4 v1, const uint4 sv, const uint2 araw) {
                     const uint32_t wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
                     // Even and odd k-steps accumulate in two chains.
                     float da[4] = {0.f, 0.f, 0.f, 0.f}, db[4] = {0.f, 0.f, 0.f, 0.f};
@@ -1014,8 +1041,6 @@ __device__ __forceinline__ void lookup_body(const LookupParams &p, const int eva
 #pragma unroll
                     for (int e = 0; e < 4; ++e) da[e] += db[e];
                     if (RESID) {
-                        const uint8_t *sp = p.sg + unit * kSignUnitBytes + lane * 16;
-                        const uint4 sv = EVA_BAD_G(BUF_SG, sp, 16) ? make_uint4(0u, 0u, 0u, 0u) : ldg_stream(sp);
                         const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
                         float dt[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -1037,9 +1062,6 @@ __device__ __forceinline__ void lookup_body(const LookupParams &p, const int eva
                             for (int e = 0; e < 4; ++e) dt1[e] = __shfl_down_sync(0xffffffffu, dt[e], 1);
                         }
                         if (q == 0) {
-                            const __half *ap = p.al + unit * kAlphaUnitHalves + 4 * g;
-                            const uint2 araw = EVA_BAD_G(BUF_AL, ap, 8) ? make_uint2(0u, 0u)
-                                                                         : *reinterpret_cast<const uint2 *>(ap);
                             const __half2 ag = *reinterpret_cast<const __half2 *>(&araw.x);   // row g: grp 0, 1
                             const __half2 ag8 = *reinterpret_cast<const __half2 *>(&araw.y);  // row g+8
                             const float a_g0 = __low2float(ag), a_g1 = __high2float(ag);
@@ -1078,7 +1100,10 @@ __device__ __forceinline__ void lookup_body(const LookupParams &p, const int eva
                     const uint4 v0 = (EVA_BAD_S(wo) || EVA_BAD_S(wo + 12u)) ? make_uint4(0u, 0u, 0u, 0u) : lds128(wo);
                     const uint4 v1 = (NIB || EVA_BAD_S(wo + 512u) || EVA_BAD_S(wo + 524u)) ? make_uint4(0u, 0u, 0u, 0u)
                                                                                               : lds128(wo + 512u);
-                    tile(tl, (size_t)s * p.T + t0 + tl, v0, v1);
+                    uint4 sv = make_uint4(0u, 0u, 0u, 0u);
+                    uint2 av = make_uint2(0u, 0u);
+                    if (RESID) load_resid(p, (size_t)s * p.T + t0 + tl, lane, g, q, sv, av);
+                    tile(tl, v0, v1, sv, av);
                 }
                 // ... then the streamed ones, through the lookahead ring.
 #pragma unroll 1
@@ -1086,16 +1111,23 @@ __device__ __forceinline__ void lookup_body(const LookupParams &p, const int eva
                     const int tl = warp + kWarps * i;              // tile index within the CTA
                     const size_t unit = (size_t)s * p.T + t0 + tl;
                     const uint4 v0 = nb[0][0], v1 = nb[0][1];
+                    const uint4 sv = ns[0];
+                    const uint2 av = na[0];
 #pragma unroll
                     for (int d = 0; d + 1 < LA; ++d) {
                         nb[d][0] = nb[d + 1][0];
                         nb[d][1] = nb[d + 1][1];
+                        if constexpr (RESID) {
+                            ns[d] = ns[d + 1];
+                            na[d] = na[d + 1];
+                        }
                     }
                     if (i + LA < i1) {
-                        const uint8_t *up = p.wi + (unit + (size_t)kWarps * LA) * UB + 16 * lane;
-                        load_unit<NIB>(p, up, nb[LA - 1][0], nb[LA - 1][1]);
+                        const size_t un = unit + (size_t)kWarps * LA;
+                        load_unit<NIB>(p, p.wi + un * UB + 16 * lane, nb[LA - 1][0], nb[LA - 1][1]);
+                        if (RESID) load_resid(p, un, lane, g, q, ns[LR - 1], na[LR - 1]);
                     }
-                    tile(tl, unit, v0, v1);
+                    tile(tl, v0, v1, sv, av);
                 }
             }
         }
@@ -1161,7 +1193,7 @@ __device__ __forceinline__ void lookup_body(const LookupParams &p, const int eva
 }
 
 template <bool PAIR_T, bool RESID, bool GROUPED, bool ROT, bool NIB>
-__global__ void __launch_bounds__(kThreads, (kLookupMinBlocks<PAIR_T, RESID, ROT>)) eva_lookup_kernel(const LookupParams p) {
+__global__ void __launch_bounds__(kThreads, kLookupMinBlocks<PAIR_T>) eva_lookup_kernel(const LookupParams p) {
     lookup_body<PAIR_T, RESID, GROUPED, ROT, NIB>(p, blockIdx.x);
 }
 
@@ -1183,7 +1215,7 @@ struct LookupGroup {
 };
 
 template <bool PAIR_T, bool RESID>
-__global__ void __launch_bounds__(kThreads, (kLookupMinBlocks<PAIR_T, RESID, false>)) eva_lookup_group_kernel(const LookupGroup g) {
+__global__ void __launch_bounds__(kThreads, kLookupMinBlocks<PAIR_T>) eva_lookup_group_kernel(const LookupGroup g) {
     const int li = blockIdx.x / g.ctas_per_layer;
     if (li >= g.count) return;
     lookup_body<PAIR_T, RESID, false, false, false>(g.p[li], blockIdx.x - li * g.ctas_per_layer);

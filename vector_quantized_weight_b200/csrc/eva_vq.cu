@@ -291,26 +291,37 @@ void plan_grid(eva_vq_linear *h, int pair_t) {
     // Independent calls overlap with their neighbours, so a layer costs the
     // CTA slots it holds times how long it holds them, and every CTA pays the
     // same fixed part (x~ staging, image build, cluster reduction) whatever
-    // its tile count.  Their grid therefore keeps the slice split and takes
-    // as few row groups as the per-CTA tile limit allows (the row-gap layout
-    // holds up to kMaxGapTiles running sums; with per-group codebooks more
-    // tiles per CTA also mean more image builds per CTA, so those stay at
-    // kMaxCtaTiles), without a larger footprint than two CTAs per SM (or the
-    // latency plan's own) permit.
+    // its work.  Their grid therefore uses clusters of at most 8 CTAs (half
+    // the latency plan's slice groups when it has more: 8-CTA clusters fill
+    // 144 of the 148 SMs where 16-CTA ones fill 112) and as few row groups as
+    // a per-CTA tile limit allows: 128 tiles, 64 with per-group codebooks
+    // (there more tiles per CTA also mean more image builds per CTA).  It
+    // never has more CTAs than the latency plan, stays within what the
+    // running-sum layout holds (kMaxGapTiles in the row-gap layout,
+    // kMaxCtaTiles otherwise) and within a footprint of two CTAs per SM (or
+    // the latency plan's own); if nothing qualifies it is the latency plan.
     eva_vq_linear::Plan ip = pl;
     ip.staged = 0;
     ip.smem = ip.smem_nostage = pl.smem_nostage;
-    const bool gaps = !pair_t && !resid && !h->desc.hadamard_block && !kNaiveOcBuild;
-    const int max_tiles = (gaps && !h->tiles_per_cb) ? kMaxGapTiles : kMaxCtaTiles;
-    const size_t two = (size_t)h->smem_per_sm / 2 - (size_t)h->smem_reserved;
-    const size_t fit = std::min(std::max(pl.smem_nostage, two), (size_t)h->smem_optin);
-    for (int gt = (T + max_tiles - 1) / max_tiles; gt < pl.Gt; ++gt) {
-        const size_t sm = lookup_smem(pair_t, resid, (T + gt - 1) / gt, pl.Gs, h->desc.hadamard_block, S, 0,
-                                      h->unit_bytes);
-        if (sm <= fit) {
-            ip.Gt = gt;
-            ip.smem = ip.smem_nostage = sm;
-            break;
+    {
+        const int gs = pl.Gs > 8 ? (pl.Gs + 1) / 2 : pl.Gs;
+        const bool gaps = !pair_t && !resid && !h->desc.hadamard_block && !kNaiveOcBuild;
+        const int hard = gaps ? kMaxGapTiles : kMaxCtaTiles;
+        const int soft = h->tiles_per_cb ? kMaxCtaTiles / 2 : kMaxCtaTiles;
+        const int gt_hi = std::min(T, std::max(1, pl.Gs * pl.Gt / gs));
+        const size_t two = (size_t)h->smem_per_sm / 2 - (size_t)h->smem_reserved;
+        const size_t fit = std::min(std::max(pl.smem_nostage, two), (size_t)h->smem_optin);
+        int gt = std::max((T + soft - 1) / soft, (T + hard - 1) / hard);
+        if (gt > gt_hi) gt = std::max(gt_hi, (T + hard - 1) / hard);
+        for (; gt <= gt_hi; ++gt) {
+            const size_t sm = lookup_smem(pair_t, resid, (T + gt - 1) / gt, gs, h->desc.hadamard_block, S, 0,
+                                          h->unit_bytes);
+            if (sm <= fit) {
+                ip.Gs = gs;
+                ip.Gt = gt;
+                ip.smem = ip.smem_nostage = sm;
+                break;
+            }
         }
     }
     h->iplan[pair_t] = ip;

@@ -49,13 +49,15 @@ def norm_rel_err(y, ref):
     return np.abs(y - ref).max(axis=1) / den
 
 
-def run_gpu(layer, x, *, out_dtype="float16", path=0, max_batch=None):
+def run_gpu(layer, x, *, out_dtype="float16", path=0, max_batch=None, independent=False):
+    """One call through the C ABI; independent=True takes the EVA_RUN_INDEPENDENT
+    launch (its own grid) that the benchmark times."""
     import torch
     from vector_quantized_weight_b200 import eva_vq
     B = x.shape[0]
     lin = eva_vq.from_layer(layer, max_batch=max_batch or B, out_dtype=out_dtype, path=path)
     xt = torch.from_numpy(x).cuda()
-    y = lin(xt)
+    y = lin(xt, independent=independent)
     torch.cuda.synchronize()
     out = y.float().cpu().numpy().astype(np.float64)
     # no bounded device wait gave up (and, in the bounds-checked build, no

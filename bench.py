@@ -372,11 +372,12 @@ def main():
         return ms, clk
 
     ms, clk = timed(args.chain == "independent", steps, True)
+    info = layers[0].info()   # the grid and path of the timed calls
     dep = None
     if args.chain == "independent" and not args.no_dependent:
         dep_steps = ring * max(1, min(steps, 200_000) // ring)
         ms_dep, _ = timed(False, dep_steps, False)
-        dep = (dep_steps, ms_dep)
+        dep = (dep_steps, ms_dep, layers[0].info().grid)
 
     # The same independent layers, `--group` of them per eva_vq_linear_run_group call.
     grouped = None
@@ -462,10 +463,10 @@ def main():
             "note": ("eva_vq_linear_run_group(EVA_RUN_INDEPENDENT) of consecutive ring layers, one launch "
                      "each (as for a decoder block's q, k and v)")}
     if dep:
-        dep_steps, ms_dep = dep
+        dep_steps, ms_dep, dep_grid = dep
         us_dep = ms_dep * 1e3 / dep_steps
         line["dependent_chain"] = {
-            "us_per_layer": round(us_dep, 4), "steps": dep_steps,
+            "us_per_layer": round(us_dep, 4), "steps": dep_steps, "grid": dep_grid,
             "value": round(job_throughput_gbs(world, dep_steps, sb, ms_dep), 4), "unit": "GB/s",
             "note": "every call waits for the kernel before it (plain eva_vq_linear_run), as when each "
                     "layer's output feeds the next"}

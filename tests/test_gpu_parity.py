@@ -172,9 +172,11 @@ def test_independent_flag_matches_plain_run(key, li, B):
     xs_np = [synth.make_x(shape.K, B, 40 + i) for i in range(3)]
     xs = [torch.from_numpy(x).cuda() for x in xs_np]
     ref = [lin(x).clone() for x in xs]
+    plain_grid = lin.info().grid
     outs = [lin(x, independent=True).clone() for x in xs]      # back to back, same handle
     again = [lin(x, independent=True) for x in xs]
     torch.cuda.synchronize()
+    assert 0 < lin.info().grid <= plain_grid                   # never more CTAs than the plain call
     rows = sample_rows(shape.N, shape.codebook_rows, n=64, seed=li)
     for x, a, b, c in zip(xs_np, ref, outs, again):
         assert torch.equal(b, c)

@@ -127,7 +127,12 @@ enum {
      * earlier and write distinct outputs).  The layer then runs without
      * waiting for that kernel, so consecutive independent layers overlap;
      * it still completes after it, so later calls keep the stream order.
-     * Passing it when x or y IS used by the preceding kernel is a race. */
+     * Passing it when x or y IS used by the preceding kernel is a race.
+     * Such calls also take a grid made for overlap (fewer CTAs, each
+     * covering more K-slices and row tiles; never more CTAs than the plain
+     * call): y is then summed over the K-slices in another fp32 order, so
+     * it matches the plain call within the rounding tolerance, not bit for
+     * bit (repeated independent calls are bitwise equal to each other). */
     EVA_RUN_INDEPENDENT = 1u
 };
 
@@ -144,7 +149,7 @@ EVA_API eva_status_t eva_vq_linear_run_ex(eva_vq_linear_t h, const void *x, int3
  * the layers run as ONE launch whose CTAs the hardware schedules as slots
  * free -- e.g. the q, k and v projections of a decoder block, which share
  * their input.  Otherwise it is one eva_vq_linear_run_ex per layer.  Results
- * are bitwise those of separate calls.  `flags` as for eva_vq_linear_run_ex,
+ * are bitwise those of separate calls with the same flags.  `flags` as for eva_vq_linear_run_ex,
  * for the group as a whole.  Not part of the pages' method: a launch-level
  * convenience.
  */

@@ -264,6 +264,9 @@ class VQLinear:
                                            _ptr(hsign), _stream_handle(stream))
 
     def __call__(self, x, out=None, stream=None, independent=False):
+        """y = layer(x) on `stream`.  independent=True passes EVA_RUN_INDEPENDENT:
+        the caller promises the preceding kernel on the stream neither writes x
+        nor touches y; the call then overlaps it and takes the overlap grid."""
         import torch
         if x.dtype != torch.float16 or not x.is_cuda or not x.is_contiguous():
             raise ValueError("x must be a contiguous CUDA float16 tensor [B, K]")

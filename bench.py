@@ -35,7 +35,8 @@ FALLBACK_HBM_GBS = 6650.0
 METRIC = "µs/layer and achieved HBM GB/s (% of B200 peak), 2-bit VQ linear"
 KERNEL_SOURCES = ("vector_quantized_weight_b200/csrc/eva_vq.cu",
                   "vector_quantized_weight_b200/csrc/eva_vq_kernels.cuh",
-                  "vector_quantized_weight_b200/csrc/eva_vq_layout.cuh")
+                  "vector_quantized_weight_b200/csrc/eva_vq_layout.cuh",
+                  "vector_quantized_weight_b200/csrc/eva_vq_plan.h")
 
 
 def parse_args():

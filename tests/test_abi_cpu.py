@@ -203,3 +203,59 @@ int main() {
         subprocess.run(["g++", "-std=c++17", "-I", os.path.join(ROOT, "vector_quantized_weight_b200", "csrc"),
                         "-o", exe, cpp], check=True)
         assert subprocess.run([exe], capture_output=True, text=True, check=True).stdout.strip() == "0"
+
+
+def test_independent_grid_invariants():
+    """The grid of independent calls (host-compilable header), over every
+    latency plan of up to 148 CTAs and row-tile counts up to 2000, with a
+    footprint that grows with the tile count: clusters of at most 8 CTAs (the
+    latency plan's Gs when it is at most 8, else half of it), never more CTAs
+    than the latency plan, never more tiles per CTA than the layout holds,
+    within the footprint budget, and the fewest row groups that satisfy all
+    of that (no smaller Gt would do)."""
+    src = r"""
+#include <cstdio>
+#include <cstddef>
+#include "eva_vq_plan.h"
+using namespace eva;
+int main() {
+    long long bad = 0, found = 0;
+    const int hards[2] = {128, 247}, softs[2] = {64, 128};
+    const size_t fits[3] = {70000, 98304, 116736};
+    for (int T = 1; T <= 2000; T += (T < 300 ? 1 : 7))
+    for (int lgs = 1; lgs <= 16; ++lgs)
+    for (int lgt = 1; lgs * lgt <= 148 && lgt <= T; ++lgt)
+    for (int hi = 0; hi < 2; ++hi) for (int si = 0; si < 2; ++si) for (int fi = 0; fi < 3; ++fi) {
+        const int hard = hards[hi], soft = softs[si];
+        const size_t fit = fits[fi];
+        auto smem = [](int tiles, int gs) { return (size_t)65536 + 256 * (size_t)tiles + 8 * (size_t)gs; };
+        int gs = 0, gt = 0; size_t sm = 0;
+        if (!independent_grid(T, lgs, lgt, hard, soft, fit, smem, &gs, &gt, &sm)) continue;
+        ++found;
+        const int tiles = (T + gt - 1) / gt;
+        bad += gs != (lgs > 8 ? (lgs + 1) / 2 : lgs);
+        bad += gs > 8 || gt < 1 || gt > T;
+        bad += gs * gt > lgs * lgt;
+        bad += tiles > hard;
+        bad += sm != smem(tiles, gs) || sm > fit;
+        // minimal: no smaller row-group count meets the same constraints
+        // and the preferred tile count
+        for (int g2 = 1; g2 < gt; ++g2) {
+            const int t2 = (T + g2 - 1) / g2;
+            if (t2 <= hard && t2 <= soft && smem(t2, gs) <= fit) { ++bad; break; }
+        }
+    }
+    std::printf("%lld %lld\n", bad, found);
+    return 0;
+}
+"""
+    import tempfile
+    with tempfile.TemporaryDirectory() as d:
+        cpp = os.path.join(d, "t.cpp")
+        open(cpp, "w").write(src)
+        exe = os.path.join(d, "t")
+        subprocess.run(["g++", "-std=c++17", "-O2", "-I", os.path.join(ROOT, "vector_quantized_weight_b200", "csrc"),
+                        "-o", exe, cpp], check=True)
+        bad, found = map(int, subprocess.run([exe], capture_output=True, text=True, check=True).stdout.split())
+        assert bad == 0 and found > 100_000, (bad, found)
+

@@ -26,7 +26,7 @@ def _nvcc() -> str:
 
 
 def _inputs():
-    return SOURCES + glob.glob(os.path.join(HERE, "csrc", "*.cuh")) + \
+    return SOURCES + glob.glob(os.path.join(HERE, "csrc", "*.cuh")) + glob.glob(os.path.join(HERE, "csrc", "*.h")) + \
         [os.path.join(ROOT, "include", "eva_vq.h")]
 
 

@@ -18,6 +18,7 @@
 
 #include "../../include/eva_vq.h"
 #include "eva_vq_kernels.cuh"
+#include "eva_vq_plan.h"
 #include "eva_vq_quant.cuh"
 #include "eva_vq_dequant.cuh"
 
@@ -288,40 +289,30 @@ void plan_grid(eva_vq_linear *h, int pair_t) {
     pl.smem_nostage = lookup_smem(pair_t, resid, tiles, pl.Gs, h->desc.hadamard_block, S, 0);
     h->plan[pair_t] = pl;
 
-    // Independent calls overlap with their neighbours, so a layer costs the
-    // CTA slots it holds times how long it holds them, and every CTA pays the
-    // same fixed part (x~ staging, image build, cluster reduction) whatever
-    // its work.  Their grid therefore uses clusters of at most 8 CTAs (half
-    // the latency plan's slice groups when it has more: 8-CTA clusters fill
-    // 144 of the 148 SMs where 16-CTA ones fill 112) and as few row groups as
-    // a per-CTA tile limit allows: 128 tiles, 64 with per-group codebooks
-    // (there more tiles per CTA also mean more image builds per CTA).  It
-    // never has more CTAs than the latency plan, stays within what the
-    // running-sum layout holds (kMaxGapTiles in the row-gap layout,
-    // kMaxCtaTiles otherwise) and within a footprint of two CTAs per SM (or
-    // the latency plan's own); if nothing qualifies it is the latency plan.
+    // Calls flagged independent: their own grid (eva_vq_plan.h), preferring
+    // 128 row tiles per CTA, 64 with per-group codebooks (there more tiles per
+    // CTA also mean more image builds per CTA), at most what the running-sum
+    // layout holds (kMaxGapTiles in the row-gap layout, kMaxCtaTiles
+    // otherwise), within a footprint of two CTAs per SM (or the latency
+    // plan's own); if nothing qualifies it is the latency plan.
     eva_vq_linear::Plan ip = pl;
     ip.staged = 0;
     ip.smem = ip.smem_nostage = pl.smem_nostage;
     {
-        const int gs = pl.Gs > 8 ? (pl.Gs + 1) / 2 : pl.Gs;
         const bool gaps = !pair_t && !resid && !h->desc.hadamard_block && !kNaiveOcBuild;
         const int hard = gaps ? kMaxGapTiles : kMaxCtaTiles;
         const int soft = h->tiles_per_cb ? kMaxCtaTiles / 2 : kMaxCtaTiles;
-        const int gt_hi = std::min(T, std::max(1, pl.Gs * pl.Gt / gs));
         const size_t two = (size_t)h->smem_per_sm / 2 - (size_t)h->smem_reserved;
         const size_t fit = std::min(std::max(pl.smem_nostage, two), (size_t)h->smem_optin);
-        int gt = std::max((T + soft - 1) / soft, (T + hard - 1) / hard);
-        if (gt > gt_hi) gt = std::max(gt_hi, (T + hard - 1) / hard);
-        for (; gt <= gt_hi; ++gt) {
-            const size_t sm = lookup_smem(pair_t, resid, (T + gt - 1) / gt, gs, h->desc.hadamard_block, S, 0,
-                                          h->unit_bytes);
-            if (sm <= fit) {
-                ip.Gs = gs;
-                ip.Gt = gt;
-                ip.smem = ip.smem_nostage = sm;
-                break;
-            }
+        auto smem = [&](int tiles, int gs) {
+            return lookup_smem(pair_t, resid, tiles, gs, h->desc.hadamard_block, S, 0, h->unit_bytes);
+        };
+        int gs = 0, gt = 0;
+        size_t sm = 0;
+        if (independent_grid(T, pl.Gs, pl.Gt, hard, soft, fit, smem, &gs, &gt, &sm)) {
+            ip.Gs = gs;
+            ip.Gt = gt;
+            ip.smem = ip.smem_nostage = sm;
         }
     }
     h->iplan[pair_t] = ip;

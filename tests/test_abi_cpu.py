@@ -96,6 +96,26 @@ def test_calls_on_null_handle():
     assert lib.eva_vq_sync_status(None) == eva_vq.EVA_ERR_INVALID_ARG
     assert lib.eva_vq_linear_info(None, None) == eva_vq.EVA_ERR_INVALID_ARG
     assert lib.eva_vq_linear_destroy(None) == eva_vq.EVA_OK
+    assert lib.eva_vq_linear_run_ex(None, 0x1000, 1, 0x2000, None, 0) == eva_vq.EVA_ERR_INVALID_ARG
+    assert lib.eva_vq_linear_run_noalloc(None, 0x1000, 1, 0x2000, None) == eva_vq.EVA_ERR_INVALID_ARG
+
+
+def test_grouped_call_rejects_bad_arguments():
+    """eva_vq_linear_run_group: null arrays or handles, a count outside
+    1..16 and unknown flags are rejected before any device work."""
+    import ctypes
+    lib = eva_vq.load()
+    hs = (ctypes.c_void_p * 2)(None, None)
+    xs = (ctypes.c_void_p * 2)(0x1000, 0x1000)
+    ys = (ctypes.c_void_p * 2)(0x2000, 0x2000)
+    bad = eva_vq.EVA_ERR_INVALID_ARG
+    assert lib.eva_vq_linear_run_group(hs, xs, ys, 2, 1, None, 0) == bad
+    assert lib.eva_vq_linear_run_group(None, xs, ys, 2, 1, None, 0) == bad
+    assert lib.eva_vq_linear_run_group(hs, None, ys, 2, 1, None, 0) == bad
+    assert lib.eva_vq_linear_run_group(hs, xs, None, 2, 1, None, 0) == bad
+    assert lib.eva_vq_linear_run_group(hs, xs, ys, 0, 1, None, 0) == bad
+    assert lib.eva_vq_linear_run_group(hs, xs, ys, 17, 1, None, 0) == bad
+    assert lib.eva_vq_linear_run_group(hs, xs, ys, 2, 1, None, 4) == bad
 
 
 def test_create_without_device_reports_no_device():

@@ -5,10 +5,15 @@ achieved HBM bandwidth of the algorithmic weight stream.
 A step is one call of the layer (one pass of the whole path, x[B,K] -> y[B,N])
 on one batch of synthetic input.  To keep the weights out of L2 the steps walk
 a ring of distinct layer instances whose index bytes total more than twice the
-L2 size; the ring is captured once in a CUDA graph and replayed.  Steps are
-timed with CUDA events on the launching stream between two barriers.
+L2 size; the calls are captured in CUDA graphs and replayed.  Exactly --steps
+steps are timed with CUDA events that the graphs record themselves, between
+two barriers.
 
-Default workload: the Llama-2-7B-shaped 4096x4096 2-bit layer at batch 1.
+Default workload: the Llama-2-7B-shaped 4096x4096 2-bit layer at batch 1, as a
+chain of dependent calls (each call waits for the one before it and reads its
+output), the latency a decode step pays per layer.  The same line carries the
+ring as independent overlapping calls, as grouped calls of three layers, and
+the end-to-end host-buffer call.
 Multi-GPU (torchrun): every rank runs its own ring (replicas, weak scaling);
 the elapsed time is the maximum over ranks and the value is the total
 work of all ranks divided by it.
@@ -33,6 +38,13 @@ sys.path.insert(0, ROOT)
 
 FALLBACK_HBM_GBS = 6650.0
 METRIC = "µs/layer and achieved HBM GB/s (% of B200 peak), 2-bit VQ linear"
+# About 1 ms at 1.965 GHz: queued ahead of a timed region, long enough for the
+# host to enqueue every replay before the GPU reaches the start event.
+SPIN_CYCLES = 2_000_000
+# Untimed calls ahead of the start event (inside the same graph), and the
+# calls per replay of the middle graph of a long timed region.
+LEAD_IN = 8
+MID_GRAPH_CALLS = 512
 KERNEL_SOURCES = ("vector_quantized_weight_b200/csrc/eva_vq.cu",
                   "vector_quantized_weight_b200/csrc/eva_vq_kernels.cuh",
                   "vector_quantized_weight_b200/csrc/eva_vq_layout.cuh",
@@ -50,16 +62,21 @@ def parse_args():
     ap.add_argument("--batch", type=int, default=None)
     ap.add_argument("--ring", type=int, default=0, help="ring length (0: > 2x L2)")
     ap.add_argument("--path", type=int, default=0)
-    ap.add_argument("--chain", default="independent", choices=["independent", "dependent"],
-                    help="independent: the ring's layers are declared independent "
-                         "(EVA_RUN_INDEPENDENT) and overlap; dependent: every call waits "
-                         "for the kernel before it, as when each layer feeds the next")
+    ap.add_argument("--chain", default="dependent", choices=["independent", "dependent"],
+                    help="dependent (the headline): every call waits for the kernel before it "
+                         "and, for a square layer, reads its output, as when each layer feeds "
+                         "the next in a decode step; independent: the ring's layers are declared "
+                         "independent (EVA_RUN_INDEPENDENT) and overlap")
     ap.add_argument("--no-dependent", action="store_true",
-                    help="skip the extra dependent-chain measurement")
+                    help="with --chain independent: skip the extra dependent-chain measurement")
+    ap.add_argument("--no-independent", action="store_true",
+                    help="with --chain dependent: skip the extra independent-ring measurement")
     ap.add_argument("--x-pool", type=int, default=4,
                     help="distinct activation buffers cycled by the ring (activations stay in L2, "
                          "as the output of the preceding op does in a decode step)")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    ap.add_argument("--no-block", action="store_true",
+                    help="skip the Llama-2-7B decoder-block leg (seven linears with their dependencies)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--group", type=int, default=3,
@@ -314,41 +331,84 @@ def main():
 
     group = [1]   # layers per call in the sweep
 
+    # Dependent calls of a square layer form a true chain: call r reads the
+    # output of call r - 1 (the ring wraps around).  Otherwise every call
+    # reads one of the x-pool buffers, written before the timed region.
+    true_chain = shape.N == shape.K
+
+    def x_of(r, independent):
+        if not independent and true_chain:
+            return ys[(r - 1) % ring]
+        return xs[r % len(xs)]
+
     def sweep(n, independent, start=0):
         i = 0
         while i < n:
             k = min(group[0], n - i)
             if k == 1:
                 r = (start + i) % ring
-                layers[r](xs[r % len(xs)], out=ys[r], stream=stream, independent=independent)
+                layers[r](x_of(r, independent), out=ys[r], stream=stream, independent=independent)
             else:
                 rs = [(start + i + j) % ring for j in range(k)]
-                eva_vq.run_group([layers[r] for r in rs], [xs[r % len(xs)] for r in rs], [ys[r] for r in rs],
+                eva_vq.run_group([layers[r] for r in rs], [x_of(r, independent) for r in rs], [ys[r] for r in rs],
                                  stream=stream, independent=independent)
             i += k
 
     uuid = getattr(props, "uuid", None)
     gpu_id = f"GPU-{uuid}" if uuid is not None else str(local)
 
-    def timed(independent, n_steps, sample_clocks):
-        """Warm up eagerly, capture one ring sweep (and a remainder) in CUDA
-        graphs, then time exactly n_steps calls between barriers."""
+    # Written before every timed region: evicts the ring from L2, so the
+    # timed layers stream their weights from HBM even when the region covers
+    # fewer calls than one sweep of the ring.
+    flush = torch.empty(2 * l2 + (1 << 20), dtype=torch.uint8, device=dev)
+
+    def timed_units(emit, n_units, period, lead, sample_clocks=False):
+        """Time exactly n_units units on the device; emit(n, start) enqueues n
+        units starting at unit `start` (mod period) on `stream`.
+
+        The units are captured in CUDA graphs: a first graph holds a lead-in
+        of units (the period's last ones, untimed), the start event and the
+        first timed units; a middle graph of several periods is replayed as
+        often as needed; a last graph holds the remaining units and the stop
+        event.  The two events are recorded by the graphs themselves (external
+        event nodes), so the region holds the timed units alone: no graph
+        launch or host submission gap before its first unit.  Every graph is
+        replayed once untimed first; L2 is flushed and a spin kernel queued
+        before the timed replays, so the timed layers stream their weights
+        from HBM and the host has enqueued every replay before the GPU gets to
+        them."""
+        e0 = torch.cuda.Event(enable_timing=True, external=True)
+        e1 = torch.cuda.Event(enable_timing=True, external=True)
+        lead = min(lead, period)
+        first = min(n_units, period)
+        per_mid = period * max(1, MID_GRAPH_CALLS // period)
+        mids, last = divmod(n_units - first, per_mid)
+        graphs = []
+        g_first = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_first, stream=stream):
+            if lead:
+                emit(lead, period - lead)
+            e0.record(stream)
+            emit(first, 0)
+            if n_units == first:
+                e1.record(stream)
+        graphs.append((g_first, 1))
+        start = first % period
+        if mids:
+            g_mid = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_mid, stream=stream):
+                emit(per_mid, start)
+            graphs.append((g_mid, mids))
+        if n_units > first:
+            g_last = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_last, stream=stream):
+                emit(last, start)
+                e1.record(stream)
+            graphs.append((g_last, 1))
         with torch.cuda.stream(stream):
-            sweep(warmup, independent)
+            for g, _ in graphs:
+                g.replay()
         torch.cuda.synchronize(dev)
-        full, rem = divmod(n_steps, ring)
-        g_full = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g_full, stream=stream):
-            sweep(ring, independent)
-        g_rem = None
-        if rem:
-            g_rem = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g_rem, stream=stream):
-                sweep(rem, independent)
-        with torch.cuda.stream(stream):
-            g_full.replay()
-        torch.cuda.synchronize(dev)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         if pg:
             pg.barrier()
         torch.cuda.synchronize(dev)
@@ -356,12 +416,11 @@ def main():
         if clk:
             clk.__enter__()
         with torch.cuda.stream(stream):
-            e0.record(stream)
-            for _ in range(full):
-                g_full.replay()
-            if g_rem is not None:
-                g_rem.replay()
-            e1.record(stream)
+            flush.zero_()
+            torch.cuda._sleep(SPIN_CYCLES)
+            for g, n in graphs:
+                for _ in range(n):
+                    g.replay()
         torch.cuda.synchronize(dev)
         if clk:
             clk.__exit__(None, None, None)
@@ -369,25 +428,88 @@ def main():
             pg.barrier()
         torch.cuda.synchronize(dev)
         ms = max_over_ranks(e0.elapsed_time(e1), pg, dev)
-        del g_full, g_rem
+        del graphs
         return ms, clk
 
-    ms, clk = timed(args.chain == "independent", steps, True)
+    def timed(independent, n_steps, sample_clocks):
+        """Eager warm-up, then exactly n_steps calls of the ring, timed."""
+        with torch.cuda.stream(stream):
+            sweep(warmup, independent)
+        torch.cuda.synchronize(dev)
+        return timed_units(lambda n, st: sweep(n, independent, st), n_steps, ring, LEAD_IN, sample_clocks)
+
+    head_indep = args.chain == "independent"
+    ms, clk = timed(head_indep, steps, True)
     info = layers[0].info()   # the grid and path of the timed calls
+    # The extra legs run whole ring sweeps (at least ten: an overlapped leg
+    # fills and drains its pipeline once per timed region).
+    extra_steps = ring * max(10, min(steps, 200_000) // ring)
     dep = None
-    if args.chain == "independent" and not args.no_dependent:
-        dep_steps = ring * max(1, min(steps, 200_000) // ring)
-        ms_dep, _ = timed(False, dep_steps, False)
-        dep = (dep_steps, ms_dep, layers[0].info().grid)
+    if head_indep and not args.no_dependent:
+        ms_dep, _ = timed(False, extra_steps, False)
+        dep = (extra_steps, ms_dep, layers[0].info().grid)
+    indep = None
+    if not head_indep and not args.no_independent:
+        ms_ind, _ = timed(True, extra_steps, False)
+        indep = (extra_steps, ms_ind, layers[0].info().grid)
 
     # The same independent layers, `--group` of them per eva_vq_linear_run_group call.
     grouped = None
-    if args.group > 1 and args.chain == "independent":
+    if args.group > 1:
         group[0] = args.group
-        g_steps = ring * max(1, min(steps, 200_000) // ring)
-        ms_g, _ = timed(True, g_steps, False)
-        grouped = (g_steps, ms_g)
+        ms_g, _ = timed(True, extra_steps, False)
+        grouped = (extra_steps, ms_g)
         group[0] = 1
+
+    # A whole Llama-2-7B decoder block per unit (the workload's seven linears
+    # with their real dependencies): q, k and v in one grouped launch reading
+    # the block input; o reading q's output (standing in for the attention
+    # output); gate and up in one grouped launch reading o's output; down
+    # reading gate's output (standing in for act(gate) * up); the next block
+    # reads down's output.  Every launch waits for the one before it.
+    block = None
+    if not args.no_block:
+        bcfg = synth.CONFIGS["llama7b_block"]
+        bsh = bcfg.layers
+        block_wi = sum(sh.N * sh.J for sh in bsh)
+        nblk = max(2, math.ceil(2 * l2 / block_wi) + 1)
+        blayers, bys = [], []
+        with torch.cuda.stream(stream):
+            for b in range(nblk):
+                blayers.append([eva_vq.from_layer(synth.make_layer(sh, synth.layer_seed(bcfg.index, li) + 1000 * (b + 1)
+                                                                   + 7919 * rank), max_batch=B, device=dev)
+                                for li, sh in enumerate(bsh)])
+                bys.append([torch.zeros((B, sh.N), dtype=torch.float16, device=dev) for sh in bsh])
+            bys[-1][6].copy_(torch.from_numpy(synth.make_x(bsh[6].N, B, seed)).to(dev))
+        torch.cuda.synchronize(dev)
+
+        def emit_blocks(n, start):
+            for i in range(n):
+                b = (start + i) % nblk
+                L, Y, xin = blayers[b], bys[b], bys[(b - 1) % nblk][6]
+                eva_vq.run_group(L[0:3], [xin] * 3, Y[0:3], stream=stream)
+                L[3](Y[0], out=Y[3], stream=stream)
+                eva_vq.run_group(L[4:6], [Y[3]] * 2, Y[4:6], stream=stream)
+                L[6](Y[4], out=Y[6], stream=stream)
+
+        with torch.cuda.stream(stream):
+            emit_blocks(2 * nblk, 0)
+        torch.cuda.synchronize(dev)
+        n_blocks = nblk * max(10, min(steps, 200_000) // (7 * nblk))
+        ms_blk, _ = timed_units(emit_blocks, n_blocks, nblk, 1)
+        bbytes = sum(stream_bytes(sh, B) for sh in bsh)
+        us_blk = ms_blk * 1e3 / n_blocks
+        block = {"us_per_block": round(us_blk, 3), "us_per_layer": round(us_blk / len(bsh), 4),
+                 "blocks": n_blocks, "ring_blocks": nblk, "launches_per_block": 4,
+                 "value": round(job_throughput_gbs(world, n_blocks, bbytes, ms_blk), 4), "unit": "GB/s",
+                 "algorithmic_bytes_per_block": bbytes,
+                 "grids": [lay.info().grid for lay in blayers[0]],
+                 "note": ("Llama-2-7B decoder block, B=%d: q,k,v (one run_group) -> o -> gate,up (one run_group) "
+                          "-> down, each launch waiting for the one before it and reading its output" % B)}
+        for row in blayers:
+            for lay in row:
+                lay.close()
+        del blayers, bys
 
     # End to end through the public host-buffer call: x copied in from
     # pinned memory and y read back every step.
@@ -443,10 +565,18 @@ def main():
                    "ring_layers": ring, "ring_index_bytes": ring * wi_bytes,
                    "l2_bytes": l2, "l2_policy": "inputs larger than L2: ring of distinct layers > 2x L2",
                    "x_pool": len(xs),
-                   "graph": "one CUDA graph per ring sweep", "parallelism": f"replicas x{world}",
+                   "graph": "calls captured in CUDA graphs, the start and stop events recorded inside them",
+                   "parallelism": f"replicas x{world}",
                    "call": ("eva_vq_linear_run_ex(EVA_RUN_INDEPENDENT): the ring's layers read "
                             "activations produced before the timed region and write distinct outputs"
-                            if args.chain == "independent" else "eva_vq_linear_run (stream-ordered)"),
+                            if head_indep else
+                            ("eva_vq_linear_run: every call waits for the kernel before it and reads "
+                             "its output y as x (a chain of layers)" if true_chain else
+                             "eva_vq_linear_run: every call waits for the kernel before it (stream "
+                             "order) and reads an x-pool activation")),
+                   "timing": ("exactly `steps` calls between two CUDA events recorded by the graphs, after "
+                              f"{LEAD_IN} untimed lead-in calls; every graph replayed once before, L2 flushed "
+                              "and a spin kernel queued ahead of the replays"),
                    "grid": info.grid, "kernels_per_step": info.kernels_per_run},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 3), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": load_traffic(workload),
@@ -463,6 +593,13 @@ def main():
             "value": round(job_throughput_gbs(world, gs_, sb, gms), 4), "unit": "GB/s",
             "note": ("eva_vq_linear_run_group(EVA_RUN_INDEPENDENT) of consecutive ring layers, one launch "
                      "each (as for a decoder block's q, k and v)")}
+    if indep:
+        i_steps, ms_ind, i_grid = indep
+        line["independent_ring"] = {
+            "us_per_layer": round(ms_ind * 1e3 / i_steps, 4), "steps": i_steps, "grid": i_grid,
+            "value": round(job_throughput_gbs(world, i_steps, sb, ms_ind), 4), "unit": "GB/s",
+            "note": "eva_vq_linear_run_ex(EVA_RUN_INDEPENDENT) over the ring: layers that read activations "
+                    "produced earlier overlap (a throughput figure, not one layer's latency)"}
     if dep:
         dep_steps, ms_dep, dep_grid = dep
         us_dep = ms_dep * 1e3 / dep_steps
@@ -471,6 +608,8 @@ def main():
             "value": round(job_throughput_gbs(world, dep_steps, sb, ms_dep), 4), "unit": "GB/s",
             "note": "every call waits for the kernel before it (plain eva_vq_linear_run), as when each "
                     "layer's output feeds the next"}
+    if block:
+        line["decoder_block"] = block
     if e2e:
         line["e2e"] = e2e
     if not args.no_cpu:

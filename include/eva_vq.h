@@ -220,8 +220,24 @@ EVA_API eva_status_t eva_vq_linear_destroy(eva_vq_linear_t h);
 EVA_API eva_status_t eva_vq_unpack_indices(eva_vq_linear_t h, uint8_t *wi_out, eva_stream_t stream);
 
 /* Synchronises the device and reports a device-side error word set by a
- * kernel (EVA_ERR_DEVICE_TIMEOUT for a bounded wait that gave up). */
+ * kernel (EVA_ERR_DEVICE_TIMEOUT for a bounded wait that gave up).  The word
+ * belongs to the handle and stays set once a wait has given up. */
 EVA_API eva_status_t eva_vq_sync_status(eva_vq_linear_t h);
+
+/*
+ * Failure-detection test hook.  The only spin-wait of the kernels is the
+ * bounded wait of a waiting call (eva_vq_linear_run, or run_ex without
+ * EVA_RUN_INDEPENDENT) for the bulk copy that stages its first index units
+ * in shared memory; when it gives up, the CTA sets the handle's status word,
+ * still joins its cluster barriers and exits, and eva_vq_sync_status returns
+ * EVA_ERR_DEVICE_TIMEOUT.  After this hook the next such call on `h` that
+ * stages units issues neither that copy nor its arrival (so nothing is in
+ * flight and the wait cannot complete) and gives up after `rounds` try_wait
+ * rounds (1 .. 2^20; the regular limit is 2^20).  One-shot; y of that call
+ * is undefined.  No device fault, trap or hang is involved.
+ * EVA_ERR_INVALID_ARG for a null handle or rounds out of range.
+ */
+EVA_API eva_status_t eva_vq_debug_inject_wait_timeout(eva_vq_linear_t h, int32_t rounds);
 
 /*
  * Diagnostic hook of the checked build (compiled with EVA_DEVICE_CHECKS):
@@ -257,6 +273,8 @@ typedef struct {
     int32_t kernels_per_run;  /* kernel launches per run() for the last run            */
     int32_t path;             /* eva_path_t used by the last run                       */
     int32_t sm_count;
+    int32_t staged_units;     /* index units per CTA a waiting one-token call copies into
+                                 shared memory while it waits (0: none)                */
 } eva_vq_info;
 
 /* Sizes and launch shape of a handle (host only, no device work). */

@@ -98,6 +98,7 @@ def test_calls_on_null_handle():
     assert lib.eva_vq_linear_destroy(None) == eva_vq.EVA_OK
     assert lib.eva_vq_linear_run_ex(None, 0x1000, 1, 0x2000, None, 0) == eva_vq.EVA_ERR_INVALID_ARG
     assert lib.eva_vq_linear_run_noalloc(None, 0x1000, 1, 0x2000, None) == eva_vq.EVA_ERR_INVALID_ARG
+    assert lib.eva_vq_debug_inject_wait_timeout(None, 1024) == eva_vq.EVA_ERR_INVALID_ARG
 
 
 def test_grouped_call_rejects_bad_arguments():

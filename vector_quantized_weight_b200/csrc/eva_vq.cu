@@ -65,6 +65,9 @@ struct eva_vq_linear {
     cudaStream_t capture_stream = nullptr;
     int64_t workspace_bytes = 0;
     int last_grid = 0, last_kernels = 0, last_path = 0;
+    // Failure-detection test hook: > 0 makes the next staging call skip its
+    // index copy and give up its wait after this many rounds.
+    int inject_wait_rounds = 0;
 };
 
 namespace {
@@ -671,6 +674,12 @@ LookupParams call_params(eva_vq_linear *h, const void *x, int32_t B, void *y, in
     // the lookups of the calls it overlaps with.
     p.wi_staged = independent ? 0 : pl.staged;
     p.status = h->status;
+    p.wait_rounds = kWaitRounds;
+    if (h->inject_wait_rounds > 0 && p.wi_staged > 0) {   // one-shot test injection
+        p.skip_stage_copy = 1;
+        p.wait_rounds = h->inject_wait_rounds;
+        h->inject_wait_rounds = 0;
+    }
     p.tiles_per_cb = h->tiles_per_cb;
     p.ncent = h->ncent;
     p.out_f32 = d.out_dtype == EVA_F32 ? 1 : 0;
@@ -806,10 +815,11 @@ eva_status_t eva_vq_linear_run_group(const eva_vq_linear_t *hs, const void *cons
 }  // extern "C"
 
 // ---------------------------------------------------------------------------
-// Allocation-free run.  The rotated input of a 3.125-bit layer normally lives
-// in a buffer the handle allocated with cudaMalloc.  This variant takes that
-// scratch from one file-scope device array instead, so the call never goes
-// near the device allocator.
+// Allocation-free run.  eva_vq_linear_run computes the rotated input of a
+// 3.125-bit layer on chip, inside the lookup kernel; this variant keeps the
+// two-kernel route (a standalone rotation kernel, then the lookups), whose
+// rotated input goes through one file-scope device array rather than memory
+// anyone allocates, so the call never goes near the device allocator.
 namespace {
 constexpr size_t kStaticScratchBytes = (size_t)4 << 20;   // 4 MiB: B * K * 4 bytes at most
 }
@@ -881,6 +891,7 @@ eva_status_t eva_vq_linear_run_noalloc(eva_vq_linear_t h, const void *x, int32_t
     p.acc_tiles = (h->T + pl.Gt - 1) / pl.Gt;
     p.wi_staged = pl.staged;
     p.status = h->status;
+    p.wait_rounds = kWaitRounds;
 #ifdef EVA_TIMELINE
     p.timeline = h->timeline;
 #endif
@@ -907,13 +918,22 @@ eva_status_t eva_vq_linear_run_noalloc(eva_vq_linear_t h, const void *x, int32_t
     if (use_dequant(h, B)) {   // no rotation on this path, so no scratch either
         size_t dsmem = 0;
         int dgrid = 0;
-        return cuda_status(launch_dequant(h, p, B, s, &dsmem, &dgrid));
+        e = launch_dequant(h, p, B, s, &dsmem, &dgrid);
+        if (e != cudaSuccess) return cuda_status(e);
+        h->last_grid = dgrid;
+        h->last_kernels = 1;
+        h->last_path = EVA_PATH_DEQUANT_MMA;
+        return EVA_OK;
     }
     const bool resid = d.residual_group != 0;
     e = launch_pdl(lookup_fn(pair_t, resid, h->tiles_per_cb != 0, fused_rot, d.index_bits == 4), dim3(pl.Gs * pl.Gt),
                    dim3(kThreads),
                    pl.smem, s, pl.Gs, p);
-    return cuda_status(e);
+    if (e != cudaSuccess) return cuda_status(e);
+    h->last_grid = pl.Gs * pl.Gt;
+    h->last_kernels = (d.hadamard_block && !fused_rot) ? 2 : 1;   // standalone rotation, then the lookups
+    h->last_path = EVA_PATH_OC_LOOKUP;
+    return EVA_OK;
 }
 
 // Inputs up to this size are read by the kernels straight from mapped host
@@ -1058,6 +1078,12 @@ eva_status_t eva_vq_sync_status(eva_vq_linear_t h) {
 #endif
 }
 
+eva_status_t eva_vq_debug_inject_wait_timeout(eva_vq_linear_t h, int32_t rounds) {
+    if (!h || rounds < 1 || rounds > kWaitRounds) return EVA_ERR_INVALID_ARG;
+    h->inject_wait_rounds = rounds;
+    return EVA_OK;
+}
+
 eva_status_t eva_vq_device_check_record(eva_vq_linear_t h, int32_t *out8) {
     if (!h || !out8) return EVA_ERR_INVALID_ARG;
     cudaError_t e = cudaDeviceSynchronize();
@@ -1096,6 +1122,7 @@ eva_status_t eva_vq_linear_info(eva_vq_linear_t h, eva_vq_info *info) {
     info->kernels_per_run = h->last_kernels ? h->last_kernels : 1;
     info->path = h->last_path ? h->last_path : EVA_PATH_OC_LOOKUP;
     info->sm_count = h->sm_count;
+    info->staged_units = h->plan[0].staged;
     return EVA_OK;
 }
 

@@ -48,7 +48,11 @@ struct LookupParams {
     int acc_tiles;           // row tiles of the largest CTA (shared-memory layout)
     int wi_staged;           // leading row tiles whose first-slice indices are copied
                              // into shared memory by one bulk copy in the prologue
-    int *status;             // device error word (bit 0: a bounded wait gave up)
+    int *status;             // device error word (bit 0: the wait for the staged index
+                             // copy gave up; bit 1: the same wait at exit gave up)
+    int wait_rounds;         // try_wait rounds before a bounded wait gives up (> 0)
+    int skip_stage_copy;     // failure-detection test only: issue neither the staging
+                             // copy nor its arrival, so the bounded wait runs out
     const int8_t *hs;        // randomized Hadamard signs s [K] (fused rotation only)
     int rot_b;               // 0, or the rotation block b: x~ = s . (H_b x) / sqrt(b) is
                              // computed in the lookup kernel from fp16 x
@@ -181,9 +185,10 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 // Bounded wait for phase `parity` of the barrier: gives up (returns false)
-// after 2^20 tries (each try suspends for a short, hardware-chosen time).
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
-    for (int it = 0; it < (1 << 20); ++it) {
+// after `rounds` tries (each try suspends for a short, hardware-chosen time).
+constexpr int kWaitRounds = 1 << 20;
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, int rounds) {
+    for (int it = 0; it < rounds; ++it) {
         uint32_t ok;
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
@@ -633,10 +638,12 @@ __device__ __forceinline__ void load_codebook_frag(const LookupParams &p, int cb
 // --------------------------------------------------- output-codebook build
 //
 // OC[j][c] = sum_{u<4} x~[256 s + 4 j + u] * WC[cb][c][u] for the 64 sub-vectors
-// of slice s: a 64 x 4 by 4 x 256 product on tensor cores (m16n8k4, tf32; the
-// fp16 inputs are exact in tf32 and their products exact in fp32), rounded to
-// fp16 and stored in the conflict-free image.  Warp w builds the centroid
-// columns 8 nt .. 8 nt + 7 of nt = w + kWarps j, j = 0..3.
+// of slice s: a 64 x 4 by 4 x 256 product on tensor cores (m16n8k4, tf32),
+// rounded to fp16 and stored in the conflict-free image.  fp16 operands are
+// exact in tf32 and their products exact in fp32; the rotated input x~ of a
+// 3.125-bit layer is fp32 and is rounded to tf32 (11 significant bits, the
+// precision of the fp16 image entries themselves) before the product.  Warp
+// w builds the centroid columns 8 nt .. 8 nt + 7 of nt = w + kWarps j, j = 0..3.
 // Diagnostics build only (EVA_NAIVE_OC_LAYOUT): the one-token image of a
 // layer without residual is stored the naive way, word(c, w) at row w,
 // column c, so that a warp's 32 lookups land on banks chosen by the indices
@@ -872,7 +879,10 @@ __device__ __forceinline__ void lookup_body(const LookupParams &p, const int eva
         mbar_init(bar, 1);
         const uint8_t *src = p.wi + ((size_t)s0 * p.T + t0) * UB;
         const uint32_t bytes = (uint32_t)staged * UB;
-        if (staged > 0 && !EVA_BAD_G(BUF_WI, src, bytes) && !EVA_BAD_S(WIS_OFF) &&
+        if (p.skip_stage_copy) {
+            // Failure-detection test: nothing arrives and nothing is in flight;
+            // the bounded wait below gives up and records it.
+        } else if (staged > 0 && !EVA_BAD_G(BUF_WI, src, bytes) && !EVA_BAD_S(WIS_OFF) &&
             !EVA_BAD_S(WIS_OFF + bytes - 4u)) {
             mbar_arrive_expect_tx(bar, bytes);
             const uint32_t dst = (uint32_t)__cvta_generic_to_shared(eva_smem + WIS_OFF);
@@ -1001,7 +1011,7 @@ __device__ __forceinline__ void lookup_body(const LookupParams &p, const int eva
                     // Bounded: if the copy never lands the CTA records it, skips
                     // nothing else and still joins the cluster barrier below.
                     wi_ready = true;
-                    if (!mbar_wait_bounded(bar, 0) && tid == 0 && p.status) atomicOr(p.status, 1);
+                    if (!mbar_wait_bounded(bar, 0, p.wait_rounds) && tid == 0 && p.status) atomicOr(p.status, 1);
                 }
                 // One tile: 32 lookups per lane, accumulated by 8 MMAs (+ the residual).
                 auto tile = [&](const int tl, const uint4 v0, const uint4 v1, const uint4 sv, const uint2 araw) {
@@ -1178,7 +1188,8 @@ __device__ __forceinline__ void lookup_body(const LookupParams &p, const int eva
         if (pr + 1 < npairs) cluster_sync_all();
     }
     // No bulk copy may still be writing this CTA's shared memory at exit.
-    if (staged > 0 && !wi_ready) mbar_wait_bounded(bar, 0);
+    if (staged > 0 && !wi_ready && !mbar_wait_bounded(bar, 0, p.wait_rounds) && tid == 0 && p.status)
+        atomicOr(p.status, 2);
     // Independent calls still complete after the preceding kernel, so that
     // later calls that wait on this one see the stream order.
     if (p.independent) pdl_wait();

@@ -26,7 +26,7 @@ ABI_FUNCTIONS = (
     "eva_vq_status_string", "eva_vq_linear_info", "eva_vq_device_check_record",
     "eva_vq_debug_timeline", "eva_vq_linear_run_noalloc",
     "eva_vq_quantize", "eva_vq_kmeans_assign", "eva_vq_kmeans_update", "eva_vq_residual",
-    "eva_vq_linear_run_group",
+    "eva_vq_linear_run_group", "eva_vq_debug_inject_wait_timeout",
 )
 
 
@@ -58,7 +58,8 @@ class eva_vq_info(ctypes.Structure):
                 ("codebook_bytes", ctypes.c_int64), ("workspace_bytes", ctypes.c_int64),
                 ("slices", ctypes.c_int32), ("row_tiles", ctypes.c_int32),
                 ("grid", ctypes.c_int32), ("kernels_per_run", ctypes.c_int32),
-                ("path", ctypes.c_int32), ("sm_count", ctypes.c_int32)]
+                ("path", ctypes.c_int32), ("sm_count", ctypes.c_int32),
+                ("staged_units", ctypes.c_int32)]
 
 
 _lib = None
@@ -106,6 +107,7 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.eva_vq_status_string.restype = ctypes.c_char_p
     lib.eva_vq_linear_info.argtypes = [H, ctypes.POINTER(eva_vq_info)]
     lib.eva_vq_device_check_record.argtypes = [H, P]
+    lib.eva_vq_debug_inject_wait_timeout.argtypes = [H, I32]
     lib.eva_vq_debug_timeline.argtypes = [H, P, I32, ctypes.POINTER(I32)]
     I64 = ctypes.c_int64
     lib.eva_vq_quantize.argtypes = [ctypes.POINTER(eva_quant_desc), P, P, P, P, P, P, P, P, P, P]
@@ -178,6 +180,10 @@ def eva_vq_unpack_indices(h: int, wi_out: int, stream: int | None) -> None:
 
 def eva_vq_sync_status(h: int) -> int:
     return int(load().eva_vq_sync_status(h))
+
+
+def eva_vq_debug_inject_wait_timeout(h: int, rounds: int) -> None:
+    _check("eva_vq_debug_inject_wait_timeout", load().eva_vq_debug_inject_wait_timeout(h, rounds))
 
 
 def eva_vq_device_check_record(h: int) -> list:

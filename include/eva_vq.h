@@ -61,9 +61,21 @@ typedef enum { EVA_F16 = 0, EVA_F32 = 1 } eva_dtype_t;
 typedef enum {
     EVA_PATH_AUTO = 0,        /* pick per call from B and the codebook layout   */
     EVA_PATH_OC_LOOKUP = 1,   /* output codebook in shared memory + lookups     */
-    EVA_PATH_DEQUANT_MMA = 2  /* codebook gather into tensor-core operands (8-bit
-                                 indices, no residual, no rotation); AUTO takes
-                                 it for B >= 4 when the layer allows it          */
+    EVA_PATH_DEQUANT_MMA = 2, /* codebook gather into warp-level tensor-core
+                                 operands (mma.sync; 8-bit indices, no residual,
+                                 no rotation); AUTO takes it for B >= 4 when the
+                                 layer allows it and EVA_PATH_TCGEN05 does not  */
+    EVA_PATH_TCGEN05 = 3      /* weights rebuilt from the codebook into tensor
+                                 memory and multiplied by tcgen05.mma (fp32
+                                 accumulation in tensor memory), residual and
+                                 rotation included; 8-bit indices, K a multiple
+                                 of 64, codebook_rows 0 or a multiple of 128;
+                                 AUTO takes it for B >= 4 when the layer allows
+                                 it.  A rotated layer runs the standalone
+                                 rotation kernel first (x~ in a handle
+                                 workspace of max_batch * K * 4 bytes); the
+                                 handle keeps a second copy of the indices (and
+                                 signs) in 128-row blocks for this path.         */
 } eva_path_t;
 
 typedef struct {

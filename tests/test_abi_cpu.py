@@ -71,6 +71,10 @@ def _create(desc, wc=0x1000, wi=0x2000, signs=None, alpha=None, hsign=None):
     (dict(max_batch=0), eva_vq.EVA_ERR_INVALID_ARG),
     (dict(max_batch=65), eva_vq.EVA_ERR_INVALID_ARG),
     (dict(out_dtype=7), eva_vq.EVA_ERR_INVALID_ARG),
+    (dict(path=4), eva_vq.EVA_ERR_INVALID_ARG),
+    (dict(path=3, K=520), eva_vq.EVA_ERR_UNSUPPORTED),            # tcgen05 path: K a multiple of 64
+    (dict(path=3, codebook_rows=16), eva_vq.EVA_ERR_UNSUPPORTED),  # ... whole 128-row codebook blocks
+    (dict(path=3, index_bits=4), eva_vq.EVA_ERR_UNSUPPORTED),      # ... 8-bit indices
 ])
 def test_create_rejects_bad_descriptor(kw, expect):
     assert _create(_desc(**kw)) == expect

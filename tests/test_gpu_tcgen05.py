@@ -1,0 +1,97 @@
+"""The large-batch path on the fifth-generation tensor cores (tcgen05.mma,
+weights rebuilt from the codebook into tensor memory, fp32 accumulation in
+tensor memory) against the double-precision oracle, on every output row:
+shared and per-128-row codebooks, the Gemma-shaped 3.125-bit layers (sign
+residual and Hadamard rotation, Sylvester and Paley blocks), ragged batches
+(the MMA's N is the batch padded to 16) and the split-K cluster reduction."""
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from tests.conftest import cuda_available
+from tests.gpu_helpers import TOL, norm_rel_err
+from vector_quantized_weight_b200 import synth
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not cuda_available(), reason="needs a CUDA device")]
+
+NTHREADS = os.cpu_count() or 8
+
+
+def _run(layer, x, path, out_dtype="float16", independent=False):
+    import torch
+    from vector_quantized_weight_b200 import eva_vq
+    B = x.shape[0]
+    lin = eva_vq.from_layer(layer, max_batch=B, out_dtype=out_dtype, path=path)
+    y = lin(torch.from_numpy(x).cuda(), independent=independent).float().cpu().numpy().astype(np.float64)
+    torch.cuda.synchronize()
+    info = lin.info()
+    assert eva_vq.eva_vq_sync_status(lin.handle) == eva_vq.EVA_OK
+    lin.close()
+    return y, info
+
+
+@pytest.mark.parametrize("shape,B", [
+    (synth.LayerShape("tiny", 256, 512), 4),
+    (synth.LayerShape("l7b", 4096, 4096), 4),
+    (synth.LayerShape("l7b", 4096, 4096), 16),
+    (synth.LayerShape("l7b", 4096, 4096), 64),
+    (synth.LayerShape("l7b_gate", 11008, 4096), 16),
+    (synth.LayerShape("l7b_down", 4096, 11008), 16),
+    (synth.LayerShape("ragged", 200, 1088), 9),
+    (synth.LayerShape("ragged", 1000, 2048), 33),
+    (synth.LayerShape("l70b", 8192, 8192, codebook_rows=128), 8),
+    (synth.LayerShape("l70b", 8192, 8192, codebook_rows=128), 32),
+    (synth.LayerShape("cb256", 512, 1024, codebook_rows=256), 5),
+    (synth.LayerShape("gemma", 3584, 3584, residual_group=128, hadamard_block=512), 4),
+    (synth.LayerShape("gemma_up", 14336, 3584, residual_group=128, hadamard_block=512), 4),
+    (synth.LayerShape("gemma_down", 3584, 14336, residual_group=128, hadamard_block=2048), 4),
+    (synth.LayerShape("gemma_rotK", 3584, 3584, residual_group=128, hadamard_block=3584), 4),
+    (synth.LayerShape("resid_only", 384, 1024, residual_group=128), 7),
+])
+def test_tcgen05_path_matches_the_oracle(shape, B):
+    from vector_quantized_weight_b200 import eva_vq
+    layer = synth.make_layer(shape, 5000 + shape.N + B, alpha_signed=bool(shape.residual_group))
+    x = synth.make_x(shape.K, B, 17 + B)
+    ref = oracle.layer_linear(layer, x, nthreads=NTHREADS)
+    for independent in (False, True):
+        y, info = _run(layer, x, eva_vq.EVA_PATH_TCGEN05, independent=independent)
+        assert info.path == eva_vq.EVA_PATH_TCGEN05
+        err = norm_rel_err(y, ref)
+        assert np.all(err <= TOL), (independent, err.max())
+
+
+def test_tcgen05_integer_inputs_exact():
+    """Small-integer codebooks and inputs: every product and partial sum is
+    exact in fp16 / fp32, so the tensor-core path reproduces the oracle exactly."""
+    from vector_quantized_weight_b200 import eva_vq
+    rng = np.random.default_rng(3)
+    for N, K, cbr, B in ((256, 1024, 0, 16), (384, 2048, 128, 7)):
+        G = N // cbr if cbr else 1
+        layer = synth.LayerData(synth.LayerShape("int", N, K, codebook_rows=cbr),
+                                rng.integers(-2, 3, size=(G, 256, 4)).astype(np.float16),
+                                rng.integers(0, 256, size=(N, K // 4)).astype(np.uint8), None, None, None)
+        x = rng.integers(-3, 4, size=(B, K)).astype(np.float16)
+        y, _ = _run(layer, x, eva_vq.EVA_PATH_TCGEN05, out_dtype="float32")
+        assert np.array_equal(y, oracle.layer_linear(layer, x))
+
+
+def test_auto_takes_tcgen05_from_four_tokens():
+    from vector_quantized_weight_b200 import eva_vq
+    shape = synth.LayerShape("l7b", 4096, 4096)
+    layer = synth.make_layer(shape, 8)
+    for B, path in ((1, eva_vq.EVA_PATH_OC_LOOKUP), (3, eva_vq.EVA_PATH_OC_LOOKUP), (4, eva_vq.EVA_PATH_TCGEN05)):
+        x = synth.make_x(shape.K, B, 9)
+        _, info = _run(layer, x, eva_vq.EVA_PATH_AUTO)
+        assert info.path == path, (B, info.path)
+
+
+def test_tcgen05_rejects_layers_it_cannot_take():
+    from vector_quantized_weight_b200 import eva_vq
+    for shape in (synth.LayerShape("k_not_64", 256, 520), synth.LayerShape("cb16", 256, 512, codebook_rows=16),
+                  synth.LayerShape("idx4", 256, 512, index_bits=4)):
+        with pytest.raises(eva_vq.EvaError) as ei:
+            eva_vq.from_layer(synth.make_layer(shape, 1), max_batch=8, path=eva_vq.EVA_PATH_TCGEN05)
+        assert ei.value.status == eva_vq.EVA_ERR_UNSUPPORTED

@@ -21,6 +21,7 @@
 #include "eva_vq_plan.h"
 #include "eva_vq_quant.cuh"
 #include "eva_vq_dequant.cuh"
+#include "eva_vq_tcgen.cuh"
 
 using namespace eva;
 
@@ -44,6 +45,14 @@ struct eva_vq_linear {
     // and 16 tokens per pass.
     bool dq_ok = false;
     Plan dq[2];
+    // Fifth-generation tensor-core path (tcgen05): CTAs per 128-row block for
+    // 16, 32, 48 and 64 padded tokens, the row-block index / sign layouts, the
+    // canonical alpha and, for a rotated layer, the rotated-input workspace.
+    bool tc_ok = false;
+    int tc_gs[4] = {0, 0, 0, 0};
+    uint8_t *wib = nullptr, *sgb = nullptr;
+    __half *al_rm = nullptr;
+    float *xrot = nullptr;
     uint8_t *wi = nullptr;              // repacked indices
     uint8_t *sg = nullptr;              // repacked signs
     __half *al = nullptr;               // repacked alpha
@@ -126,6 +135,12 @@ void paley28_table(int8_t *out) {
         }
 }
 
+// Layers the tcgen05 path takes: 8-bit indices, K a multiple of 64 (whole
+// stages), codebooks shared or per whole 128-row blocks.
+bool tc_layer_ok(const eva_vq_desc &d) {
+    return d.index_bits == 8 && d.K % kTcStageK == 0 && (d.codebook_rows == 0 || d.codebook_rows % kTcRows == 0);
+}
+
 eva_status_t validate_desc(const eva_vq_desc *d) {
     if (!d) return EVA_ERR_INVALID_ARG;
     if (d->N < 1 || d->K < 1 || d->N > (1 << 24) || d->K > (1 << 22)) return EVA_ERR_INVALID_ARG;
@@ -144,9 +159,11 @@ eva_status_t validate_desc(const eva_vq_desc *d) {
     if (d->hadamard_block && !valid_rotation_block(d->hadamard_block, d->K)) return EVA_ERR_INVALID_ARG;
     if (d->max_batch < 1 || d->max_batch > 64) return EVA_ERR_INVALID_ARG;
     if (d->out_dtype != EVA_F16 && d->out_dtype != EVA_F32) return EVA_ERR_INVALID_ARG;
-    if (d->path != EVA_PATH_AUTO && d->path != EVA_PATH_OC_LOOKUP && d->path != EVA_PATH_DEQUANT_MMA)
+    if (d->path != EVA_PATH_AUTO && d->path != EVA_PATH_OC_LOOKUP && d->path != EVA_PATH_DEQUANT_MMA &&
+        d->path != EVA_PATH_TCGEN05)
         return EVA_ERR_INVALID_ARG;
     if (d->path == EVA_PATH_DEQUANT_MMA && (d->residual_group || d->hadamard_block)) return EVA_ERR_UNSUPPORTED;
+    if (d->path == EVA_PATH_TCGEN05 && !tc_layer_ok(*d)) return EVA_ERR_UNSUPPORTED;
     return EVA_OK;
 }
 
@@ -443,6 +460,15 @@ cudaError_t set_smem_attrs(int smem_optin) {
         e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_optin);
         if (e != cudaSuccess) return e;
     }
+    for (int v = 0; v < 2; ++v) {
+        const void *fn = v ? (const void *)eva_tc_kernel<true> : (const void *)eva_tc_kernel<false>;
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_optin);
+        if (e != cudaSuccess) return e;
+    }
+    e = cudaFuncSetAttribute(eva_paley_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 28 * 1024 * 4);
+    if (e != cudaSuccess) return e;
     return cudaFuncSetAttribute(eva_hadamard_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 4096 * 4);
 }
 
@@ -472,9 +498,61 @@ bool use_three_per_sm(const eva_vq_linear *h, int B, int independent) {
     return (h->T + pl.Gt - 1) / pl.Gt <= kThreePerSmMaxTiles;
 }
 
+// The tcgen05 path: forced, or AUTO from kDequantMinBatch tokens on.
+bool use_tc(const eva_vq_linear *h, int B) {
+    if (!h->tc_ok) return false;
+    return h->desc.path == EVA_PATH_TCGEN05 || (h->desc.path == EVA_PATH_AUTO && B >= kDequantMinBatch);
+}
+
 bool use_dequant(const eva_vq_linear *h, int B) {
-    if (!h->dq_ok) return false;
+    if (!h->dq_ok || use_tc(h, B)) return false;
     return h->desc.path == EVA_PATH_DEQUANT_MMA || (h->desc.path == EVA_PATH_AUTO && B >= kDequantMinBatch);
+}
+
+// Dynamic shared memory of a tcgen05-path CTA: at least kTcMinSmem, so no
+// more than two CTAs share an SM and their tensor-memory allocations (256
+// columns each) always fit in the SM's 512 -- an allocation never waits for
+// another CTA's.
+constexpr size_t kTcMinSmem = 80 * 1024;
+size_t tc_smem(const TcLayout &L) { return std::max((size_t)L.total, kTcMinSmem); }
+
+using TcFn = void (*)(TcParams);
+TcFn tc_fn(bool resid) { return resid ? eva_tc_kernel<true> : eva_tc_kernel<false>; }
+
+// CTAs per 128-row block (one cluster of Gs, consecutive K ranges) for Np
+// padded tokens: the fewest rounds of resident CTAs times the stages of the
+// longest K range, plus a share for the cluster reduction; 0 if nothing fits.
+int plan_tc(eva_vq_linear *h, int Np) {
+    const eva_vq_desc &d = h->desc;
+    const int R = (d.N + kTcRows - 1) / kTcRows, KB = d.K / kTcStageK;
+    const bool resid = d.residual_group != 0;
+    const TcFn fn = tc_fn(resid);
+    double best = 1e300;
+    int pick = 0;
+    for (int gs = 1; gs <= std::min(16, KB); ++gs) {
+        const TcLayout L = tc_layout(KB, gs, Np, resid ? 1 : 0);
+        if (tc_smem(L) > (size_t)h->smem_optin) continue;
+        int resident = 0;
+        if (gs > 1) {
+            resident = max_active_clusters((LookupFn)fn, tc_smem(L), gs) * gs;
+        } else {
+            int per_sm = 0;
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, (const void *)fn, kTcThreads, tc_smem(L)) !=
+                cudaSuccess) {
+                cudaGetLastError();
+                per_sm = 0;
+            }
+            resident = per_sm * h->sm_count;
+        }
+        if (resident <= 0) continue;
+        const int rounds = (R * gs + resident - 1) / resident;
+        const double cost = (double)rounds * (300.0 + 160.0 * ((KB + gs - 1) / gs)) + (gs > 1 ? 700.0 + 40.0 * gs : 0.0);
+        if (cost < best) {
+            best = cost;
+            pick = gs;
+        }
+    }
+    return pick;
 }
 
 void free_handle(eva_vq_linear *h) {
@@ -483,7 +561,7 @@ void free_handle(eva_vq_linear *h) {
         if (hg.exec) cudaGraphExecDestroy(hg.exec);
     if (h->capture_stream) cudaStreamDestroy(h->capture_stream);
     void *ptrs[] = {h->wi, h->sg, h->al, h->wc, h->hsign, h->h28, h->status, h->x_stage,
-                    h->y_stage, h->timeline};
+                    h->y_stage, h->timeline, h->wib, h->sgb, h->al_rm, h->xrot};
     for (void *p : ptrs)
         if (p) cudaFree(p);
     delete h;
@@ -583,7 +661,31 @@ eva_status_t eva_vq_linear_create(eva_vq_linear_t *out, const eva_vq_desc *desc,
             return EVA_ERR_UNSUPPORTED;
         }
     }
+    if (tc_layer_ok(*desc) &&
+        (desc->path == EVA_PATH_TCGEN05 || (desc->path == EVA_PATH_AUTO && desc->max_batch >= kDequantMinBatch))) {
+        // Plans for the padded batches up to max_batch; a batch whose padded
+        // size has no plan (its x range does not fit in shared memory) runs
+        // as several launches of the largest size that has one.
+        for (int i = 0; i < 4 && 16 * i < desc->max_batch; ++i) {
+            h->tc_gs[i] = plan_tc(h, 16 * (i + 1));
+            max_grid = std::max(max_grid, h->tc_gs[i] * ((N + kTcRows - 1) / kTcRows));
+        }
+        h->tc_ok = h->tc_gs[0] > 0;
+        if (!h->tc_ok && desc->path == EVA_PATH_TCGEN05) {
+            free_handle(h);
+            return EVA_ERR_UNSUPPORTED;
+        }
+    }
     chk(dalloc(&h->wi, (size_t)units * h->unit_bytes, nullptr));
+    const int R128 = (N + kTcRows - 1) / kTcRows;
+    if (h->tc_ok) {
+        chk(dalloc(&h->wib, (size_t)R128 * kTcRows * h->J, nullptr));
+        if (desc->residual_group) {
+            chk(dalloc(&h->sgb, (size_t)R128 * kTcRows * (K / 8), nullptr));
+            chk(dalloc(&h->al_rm, (size_t)N * (K / desc->residual_group) * sizeof(__half), nullptr));
+        }
+        if (desc->hadamard_block) chk(dalloc(&h->xrot, (size_t)desc->max_batch * K * sizeof(float), &ws));
+    }
     chk(dalloc(&h->wc, (size_t)h->G * h->ncent * kD * sizeof(__half), nullptr));
     if (desc->residual_group) {
         chk(dalloc(&h->sg, (size_t)units * kSignUnitBytes, nullptr));
@@ -621,6 +723,18 @@ eva_status_t eva_vq_linear_create(eva_vq_linear_t *out, const eva_vq_desc *desc,
         eva_repack_alpha_kernel<<<blocks_for(ab, thr), thr, 0, s>>>(
             reinterpret_cast<const __half *>(alpha), h->al, N, K / desc->residual_group, h->T, ab);
         chk(cudaGetLastError());
+    }
+    if (h->tc_ok) {
+        const long long nb = (long long)R128 * kTcRows * h->J;
+        eva_repack_wi_rowblock_kernel<<<blocks_for(nb, thr), thr, 0, s>>>(wi, h->wib, N, h->J, nb);
+        chk(cudaGetLastError());
+        if (desc->residual_group) {
+            const long long ns = (long long)R128 * kTcRows * (K / 8);
+            eva_repack_signs_rowblock_kernel<<<blocks_for(ns, thr), thr, 0, s>>>(signs, h->sgb, N, K / 8, ns);
+            chk(cudaGetLastError());
+            chk(cudaMemcpyAsync(h->al_rm, alpha, (size_t)N * (K / desc->residual_group) * sizeof(__half),
+                                cudaMemcpyDeviceToDevice, s));
+        }
     }
     if (desc->hadamard_block) chk(cudaMemcpyAsync(h->hsign, hsign, (size_t)K, cudaMemcpyDeviceToDevice, s));
     if (paley_m(desc->hadamard_block)) {
@@ -723,13 +837,90 @@ LookupParams call_params(eva_vq_linear *h, const void *x, int32_t B, void *y, in
 // (8-bit indices, shared codebook, no rotation, the lookup path at this B).
 bool groupable(const eva_vq_linear *h, int B) {
     const eva_vq_desc &d = h->desc;
-    return d.index_bits == 8 && !d.codebook_rows && !d.hadamard_block && !use_dequant(h, B);
+    return d.index_bits == 8 && !d.codebook_rows && !d.hadamard_block && !use_dequant(h, B) && !use_tc(h, B);
 }
 
 using GroupFn = void (*)(LookupGroup);
 GroupFn group_fn(bool pair_t, bool resid) {
     if (pair_t) return resid ? eva_lookup_group_kernel<true, true> : eva_lookup_group_kernel<true, false>;
     return resid ? eva_lookup_group_kernel<false, true> : eva_lookup_group_kernel<false, false>;
+}
+}  // namespace
+
+namespace {
+// One call on the tcgen05 path: for a rotated layer the standalone rotation
+// kernel first writes x~ (fp32) into `xrot`, then the tensor-core kernel.
+cudaError_t launch_tc(eva_vq_linear *h, const void *x, int B, void *y, cudaStream_t s, int independent,
+                      float *xrot) {
+    const eva_vq_desc &d = h->desc;
+    int kernels = 0;
+    cudaError_t e;
+    const void *xin = x;
+    int x_f32 = 0;
+    if (d.hadamard_block) {
+        const int b = d.hadamard_block, m = paley_m(b), thr = std::min(b / 2, 1024);
+        const float scale = (float)(1.0 / std::sqrt((double)b));
+        if (m) {
+            // Launched in plain stream order (it reads x as soon as it starts).
+            eva_paley_rows_kernel<<<dim3(d.K / b, B), thr, (size_t)b * sizeof(float), s>>>(
+                reinterpret_cast<const __half *>(x), h->hsign, h->h28, xrot, d.K, b, m, scale);
+            e = cudaGetLastError();
+        } else {
+            e = launch_pdl(eva_hadamard_kernel, dim3(d.K / b, B), dim3(thr), (size_t)b * sizeof(float), s, 0,
+                           reinterpret_cast<const __half *>(x), (const int8_t *)h->hsign, xrot, d.K, b, scale,
+                           independent);
+        }
+        if (e != cudaSuccess) return e;
+        xin = xrot;
+        x_f32 = 1;
+        independent = 0;    // the tensor-core kernel reads the rotation kernel's output
+        ++kernels;
+    }
+    // The largest padded batch with a plan takes the tokens in chunks.
+    int imax = 0;
+    for (int i = 0; i < 4; ++i)
+        if (h->tc_gs[i]) imax = i;
+    const int ybytes = d.out_dtype == EVA_F32 ? 4 : 2, xbytes = x_f32 ? 4 : 2;
+    int grid = 0;
+    for (int b0 = 0; b0 < B; b0 += 16 * (imax + 1)) {
+        const int nb = std::min(B - b0, 16 * (imax + 1));
+        const int Np = ((nb + 15) / 16) * 16;
+        const int gs = h->tc_gs[Np / 16 - 1];
+        TcParams p;
+        std::memset(&p, 0, sizeof(p));
+        p.wib = h->wib;
+        p.wc = h->wc;
+        p.sg = h->sgb;
+        p.al = h->al_rm;
+        p.x = static_cast<const char *>(xin) + (size_t)b0 * d.K * xbytes;
+        p.y = static_cast<char *>(y) + (size_t)b0 * d.N * ybytes;
+        p.N = d.N;
+        p.K = d.K;
+        p.B = nb;
+        p.Np = Np;
+        p.R = (d.N + kTcRows - 1) / kTcRows;
+        p.KB = d.K / kTcStageK;
+        p.Gs = gs;
+        p.rows_per_cb = d.codebook_rows;
+        p.x_f32 = x_f32;
+        p.out_f32 = d.out_dtype == EVA_F32 ? 1 : 0;
+        p.independent = independent;
+        p.resid = d.residual_group != 0;
+        p.status = h->status;
+        p.wait_rounds = kWaitRounds;
+#ifdef EVA_TIMELINE
+        p.timeline = h->timeline;
+#endif
+        const TcLayout L = tc_layout(p.KB, gs, Np, p.resid);
+        e = launch_pdl(tc_fn(p.resid != 0), dim3(p.R * gs), dim3(kTcThreads), tc_smem(L), s, gs > 1 ? gs : 0, p);
+        if (e != cudaSuccess) return e;
+        grid = p.R * gs;
+        ++kernels;
+    }
+    h->last_grid = grid;
+    h->last_kernels = kernels;
+    h->last_path = EVA_PATH_TCGEN05;
+    return cudaSuccess;
 }
 }  // namespace
 
@@ -744,8 +935,9 @@ eva_status_t eva_vq_linear_run_ex(eva_vq_linear_t h, const void *x, int32_t B, v
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const eva_vq_desc &d = h->desc;
     size_t smem = 0;
-    LookupParams p = call_params(h, x, B, y, independent, &smem);
     cudaError_t e;
+    if (use_tc(h, B)) return cuda_status(launch_tc(h, x, B, y, s, independent, h->xrot));
+    LookupParams p = call_params(h, x, B, y, independent, &smem);
     if (use_dequant(h, B)) {
         size_t dsmem = 0;
         int dgrid = 0;
@@ -852,6 +1044,20 @@ eva_status_t eva_vq_linear_run_noalloc(eva_vq_linear_t h, const void *x, int32_t
     if (!h || !x || !y || !aligned16(x) || !aligned16(y)) return EVA_ERR_INVALID_ARG;
     if (B < 1 || B > h->desc.max_batch) return EVA_ERR_INVALID_ARG;
     const eva_vq_desc &d = h->desc;
+    if (use_tc(h, B)) {
+        // The tensor-core path of a rotated layer always runs the standalone
+        // rotation first; its x~ goes through the static scratch.
+        if (d.hadamard_block && (size_t)B * d.K * sizeof(float) > kStaticScratchBytes)
+            return EVA_ERR_SCRATCH_TOO_SMALL;
+        int dev = -1;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev != h->device) return EVA_ERR_INVALID_ARG;
+        float *scratch = nullptr;
+        if (d.hadamard_block) {
+            const eva_status_t st = static_scratch(dev, &scratch);
+            if (st != EVA_OK) return st;
+        }
+        return cuda_status(launch_tc(h, x, B, y, reinterpret_cast<cudaStream_t>(stream), 0, scratch));
+    }
     // A Paley rotation block has no standalone-kernel route that matches the
     // fused rotation bit for bit at every size, so it stays fused (no scratch).
     const bool fused_rot = paley_m(d.hadamard_block) != 0;
@@ -1122,7 +1328,7 @@ eva_status_t eva_vq_linear_info(eva_vq_linear_t h, eva_vq_info *info) {
     info->kernels_per_run = h->last_kernels ? h->last_kernels : 1;
     info->path = h->last_path ? h->last_path : EVA_PATH_OC_LOOKUP;
     info->sm_count = h->sm_count;
-    info->staged_units = h->plan[0].staged;
+    info->staged_units = call_plan(h, 1, 0).staged;
     return EVA_OK;
 }
 

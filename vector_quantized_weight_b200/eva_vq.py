@@ -15,7 +15,7 @@ from . import build as _build
 EVA_OK, EVA_ERR_INVALID_ARG, EVA_ERR_UNSUPPORTED, EVA_ERR_CUDA, EVA_ERR_OOM, \
     EVA_ERR_DEVICE_TIMEOUT, EVA_ERR_NO_DEVICE, EVA_ERR_DEVICE_CHECK, EVA_ERR_SCRATCH_TOO_SMALL = range(9)
 EVA_F16, EVA_F32 = 0, 1
-EVA_PATH_AUTO, EVA_PATH_OC_LOOKUP, EVA_PATH_DEQUANT_MMA = 0, 1, 2
+EVA_PATH_AUTO, EVA_PATH_OC_LOOKUP, EVA_PATH_DEQUANT_MMA, EVA_PATH_TCGEN05 = 0, 1, 2, 3
 
 # Every function the header declares; the CPU tests check the library exports them.
 EVA_RUN_INDEPENDENT = 1

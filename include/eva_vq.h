@@ -84,8 +84,8 @@ typedef struct {
     int32_t d;               /* sub-vector length; 4 is the only supported value        */
     int32_t index_bits;      /* n: 8 (256 centroids, one byte per index) or 4 (16
                                 centroids, two indices per byte: wi is [N][K/8], the even
-                                sub-vector in the low nibble; one shared codebook, no
-                                rotation, K a multiple of 8)                             */
+                                sub-vector in the low nibble; K a multiple of 8; the
+                                lookup path at every batch size)                         */
     int32_t codebook_rows;   /* 0: one shared codebook; R > 0: codebook g serves rows
                                 [R g, R g + R); R must be a multiple of 16 dividing N    */
     int32_t residual_group;  /* 0: no sign residual; 128: signs + one alpha per 128 k   */
@@ -326,7 +326,9 @@ typedef struct {
  * blocks (block m of codebook g is W_rot row g * codebook_rows + m / (K/4),
  * inputs 4 (m mod K/4) ..; G = N / codebook_rows, or 1); an index out of
  * range gives EVA_ERR_INVALID_ARG.  Outputs (device, caller-owned): wc_out fp16
- * [G][2^n][4]; wi_out u8 [N][K/4]; signs_out u8 [N][K/8] and alpha_out fp16
+ * [G][2^n][4]; wi_out u8 [N][K/4] (index_bits = 4: packed two per byte,
+ * [N][K/8] with the even sub-vector in the low nibble -- the layout
+ * eva_vq_linear_create takes; K a multiple of 8); signs_out u8 [N][K/8] and alpha_out fp16
  * [N][K/residual_group] (required iff residual_group != 0).  Optional:
  * wrot_out fp32 [N][K] (the rotated rows; also used as the working buffer
  * when given) and cent_out fp32 [G][2^n][4] (the centroids after the last

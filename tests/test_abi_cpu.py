@@ -57,7 +57,7 @@ def _create(desc, wc=0x1000, wi=0x2000, signs=None, alpha=None, hsign=None):
 @pytest.mark.parametrize("kw,expect", [
     (dict(d=3), eva_vq.EVA_ERR_UNSUPPORTED),
     (dict(index_bits=6), eva_vq.EVA_ERR_UNSUPPORTED),
-    (dict(index_bits=4, codebook_rows=16), eva_vq.EVA_ERR_UNSUPPORTED),   # 4-bit: one shared codebook
+    (dict(index_bits=4, path=2), eva_vq.EVA_ERR_UNSUPPORTED),   # 4-bit: the lookup path only
     (dict(index_bits=4, K=516), eva_vq.EVA_ERR_INVALID_ARG),
     (dict(N=0), eva_vq.EVA_ERR_INVALID_ARG),
     (dict(K=510), eva_vq.EVA_ERR_INVALID_ARG),
@@ -131,17 +131,18 @@ def test_create_without_device_reports_no_device():
 
 
 def test_kernels_do_not_spill():
-    """ptxas report of every kernel (the lookup instances, the dequantize
-    instances, the rotation, repack and quantizer kernels): no local-memory
+    """ptxas report of every kernel (the lookup instances, the dequantize and
+    tcgen05 instances, the rotation, repack and quantizer kernels): no local-memory
     stack frame and no spills (hot loops keep everything in registers)."""
     cmd = [build._nvcc(), *[f for f in build.NVCC_FLAGS if f != "-shared"], "-Xptxas", "-v", "-c",
            "-I", os.path.join(ROOT, "include"), "-o", os.devnull, *build.SOURCES]
     out = subprocess.run(cmd, capture_output=True, text=True, check=True).stderr
     blocks = re.findall(r"Function properties for (\S*eva_\w+_kernel\S*)\n\s*(\d+) bytes stack frame, "
                         r"(\d+) bytes spill stores, (\d+) bytes spill loads", out)
-    assert sum("eva_lookup_kernelI" in b[0] for b in blocks) == 20, out     # 16 + 4 with 4-bit indices
-    assert sum("eva_lookup_kernel3I" in b[0] for b in blocks) == 3, out     # three CTAs per SM
+    assert sum("eva_lookup_kernelI" in b[0] for b in blocks) == 32, out     # 16 for 8-bit + 16 for 4-bit indices
+    assert sum("eva_lookup_kernel3I" in b[0] for b in blocks) == 4, out     # three CTAs per SM
     assert sum("eva_dequant_kernel" in b[0] for b in blocks) == 4, out
+    assert sum("eva_tc_kernel" in b[0] for b in blocks) == 2, out           # tcgen05 path, with / without residual
     assert sum("eva_kmeans_assign_kernel" in b[0] for b in blocks) == 2, out
     for name, stack, st, ld in blocks:
         assert (stack, st, ld) == ("0", "0", "0"), (name, stack, st, ld)

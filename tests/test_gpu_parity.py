@@ -248,20 +248,28 @@ def test_host_buffer_call_graph_and_pageable():
     lin.close()
 
 
-@pytest.mark.parametrize("N,K,B,resid", [(4096, 4096, 1, 0), (256, 512, 2, 0), (100, 264, 3, 0), (64, 512, 1, 128),
-                                         (48, 1024, 5, 128), (4096, 4096, 4, 0)])
-def test_four_bit_indices(N, K, B, resid):
-    """16-centroid codebooks with indices packed two per byte: against the
-    oracle (which reads the packed bytes itself), and the index round trip
-    is bit-exact."""
+@pytest.mark.parametrize("N,K,B,resid,cbr,had", [
+    (4096, 4096, 1, 0, 0, 0), (256, 512, 2, 0, 0, 0), (100, 264, 3, 0, 0, 0), (64, 512, 1, 128, 0, 0),
+    (48, 1024, 5, 128, 0, 0), (4096, 4096, 4, 0, 0, 0),
+    (8192, 8192, 1, 0, 128, 0), (1024, 2048, 3, 0, 128, 0), (272, 1024, 2, 0, 16, 0),   # per-group codebooks
+    (3584, 3584, 1, 128, 0, 512), (512, 1024, 2, 128, 0, 1024),                          # rotation + residual
+    (3584, 3584, 1, 128, 0, 3584), (128, 1792, 3, 128, 128, 1792),                       # Paley blocks
+])
+def test_four_bit_indices(N, K, B, resid, cbr, had):
+    """16-centroid codebooks with indices packed two per byte (shared or per
+    group of rows, with or without rotation and sign residual): against the
+    oracle (which reads the packed bytes itself) on every row, in both launch
+    configurations, and the index round trip is bit-exact."""
     import torch
     from vector_quantized_weight_b200 import eva_vq
-    shape = synth.LayerShape("idx4", N, K, residual_group=resid, index_bits=4)
+    shape = synth.LayerShape("idx4", N, K, residual_group=resid, index_bits=4, codebook_rows=cbr,
+                             hadamard_block=had)
     layer = synth.make_layer(shape, N + K + B, alpha_signed=bool(resid))
     x = synth.make_x(K, B, 7)
-    y = run_gpu(layer, x)
     ref = oracle.layer_linear(layer, x, nthreads=NTHREADS)
-    assert np.all(norm_rel_err(y, ref) <= TOL)
+    for independent in (False, True):
+        y = run_gpu(layer, x, independent=independent)
+        assert np.all(norm_rel_err(y, ref) <= TOL), independent
     lin = eva_vq.from_layer(layer, max_batch=B)
     back = lin.unpack_indices().cpu().numpy()
     torch.cuda.synchronize()

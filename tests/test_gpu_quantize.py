@@ -183,3 +183,37 @@ def test_quantize_rejects_out_of_range_start():
     with pytest.raises(eva_vq.EvaError) as ei:
         _run_quantize(w, None, 0, 0, 2, init)
     assert ei.value.status == eva_vq.EVA_ERR_INVALID_ARG
+
+
+def test_quantize_four_bit_packed():
+    """index_bits = 4: 16 centroids per codebook, the pointers packed two per
+    byte (the layout the layer takes); unpacked they are the oracle's nearest
+    fp16 centroids, the residual follows them, and the quantized layer (one
+    codebook per 128 rows, rotation, sign residual) runs through the lookup
+    path against the oracle."""
+    import torch
+    from vector_quantized_weight_b200 import eva_vq
+    N, K, b, cbr, iters = 512, 1024, 256, 128, 3
+    seed = 4242
+    w = synth.make_dense_weight(N, K, seed)
+    hs = synth.make_hsign(K, seed)
+    J, G = K // 4, N // cbr
+    vpc = cbr * J
+    init = synth.kmeans_init_index(vpc, G, 16, seed)
+    out, _ = _run_quantize(w, hs, b, cbr, iters, init, index_bits=4)
+    assert out["wi"].shape == (N, K // 8)
+    idx = np.stack([out["wi"] & 15, out["wi"] >> 4], axis=-1).reshape(N, J)
+    v = out["wrot"].reshape(N * J, 4)
+    assert np.array_equal(idx.reshape(-1), oracle.kmeans_assign(v, out["wc"].astype(np.float32), vpc))
+    signs_ref, _ = oracle.residual(out["wrot"], out["wc"], idx.astype(np.uint8), codebook_rows=cbr, group=128)
+    assert np.array_equal(out["signs"], signs_ref)
+    x = synth.make_x(K, 3, seed)
+    lin = eva_vq.VQLinear(_cuda(out["wc"]), _cuda(out["wi"]), signs=_cuda(out["signs"]), alpha=_cuda(out["alpha"]),
+                          hsign=_cuda(hs), codebook_rows=cbr, residual_group=128, hadamard_block=b, max_batch=3,
+                          index_bits=4)
+    y = lin(_cuda(x)).float().cpu().numpy().astype(np.float64)
+    torch.cuda.synchronize()
+    lin.close()
+    yq = oracle.linear(out["wc"], out["wi"], x, signs=out["signs"], alpha=out["alpha"], hsign=hs, codebook_rows=cbr,
+                       residual_group=128, hadamard_block=b, index_bits=4)
+    assert np.all(norm_rel_err(y, yq) <= TOL)

@@ -41,6 +41,10 @@ struct eva_vq_linear {
     // that wait for their predecessor (one layer's latency), iplan[] for
     // calls flagged independent (CTA-slot time per layer).
     Plan plan[2], iplan[2];
+    // Waiting one-token calls of 2..4 layers in one eva_vq_linear_run_group
+    // launch (a decoder block's q, k, v or gate, up): each layer's grid for
+    // its share of the SMs.
+    Plan gplan[5];
     // Dequantize-to-tensor-core path (no residual, no rotation): plans for 8
     // and 16 tokens per pass.
     bool dq_ok = false;
@@ -146,8 +150,8 @@ eva_status_t validate_desc(const eva_vq_desc *d) {
     if (d->N < 1 || d->K < 1 || d->N > (1 << 24) || d->K > (1 << 22)) return EVA_ERR_INVALID_ARG;
     if (d->d != kD || (d->index_bits != 8 && d->index_bits != 4)) return EVA_ERR_UNSUPPORTED;
     if (d->index_bits == 4) {
-        // 4-bit indices: one shared codebook, no rotation, whole index bytes.
-        if (d->codebook_rows || d->hadamard_block || d->path == EVA_PATH_DEQUANT_MMA) return EVA_ERR_UNSUPPORTED;
+        // 4-bit indices: the lookup path only, whole index bytes.
+        if (d->path == EVA_PATH_DEQUANT_MMA) return EVA_ERR_UNSUPPORTED;
         if (d->K % 8) return EVA_ERR_INVALID_ARG;
     }
     if (d->K % kD) return EVA_ERR_INVALID_ARG;
@@ -211,26 +215,22 @@ int staged_tiles(const eva_vq_linear *h, const void *fn, bool pair_t, bool resid
 }
 
 using LookupFn = void (*)(LookupParams);
-template <bool ROT>
+template <bool ROT, bool NIB>
 LookupFn lookup_fn_r(bool pair_t, bool resid, bool grouped) {
     if (grouped) {
         if (!pair_t)
-            return resid ? eva_lookup_kernel<false, true, true, ROT, false> : eva_lookup_kernel<false, false, true, ROT, false>;
-        return resid ? eva_lookup_kernel<true, true, true, ROT, false> : eva_lookup_kernel<true, false, true, ROT, false>;
+            return resid ? eva_lookup_kernel<false, true, true, ROT, NIB> : eva_lookup_kernel<false, false, true, ROT, NIB>;
+        return resid ? eva_lookup_kernel<true, true, true, ROT, NIB> : eva_lookup_kernel<true, false, true, ROT, NIB>;
     }
     if (!pair_t)
-        return resid ? eva_lookup_kernel<false, true, false, ROT, false> : eva_lookup_kernel<false, false, false, ROT, false>;
-    return resid ? eva_lookup_kernel<true, true, false, ROT, false> : eva_lookup_kernel<true, false, false, ROT, false>;
+        return resid ? eva_lookup_kernel<false, true, false, ROT, NIB> : eva_lookup_kernel<false, false, false, ROT, NIB>;
+    return resid ? eva_lookup_kernel<true, true, false, ROT, NIB> : eva_lookup_kernel<true, false, false, ROT, NIB>;
 }
 // rot: the instance that computes the Hadamard rotation while staging x;
-// nib: 4-bit indices (shared codebook, no rotation).
+// nib: 4-bit indices.
 LookupFn lookup_fn(bool pair_t, bool resid, bool grouped, bool rot, bool nib = false) {
-    if (nib) {
-        if (!pair_t)
-            return resid ? eva_lookup_kernel<false, true, false, false, true> : eva_lookup_kernel<false, false, false, false, true>;
-        return resid ? eva_lookup_kernel<true, true, false, false, true> : eva_lookup_kernel<true, false, false, false, true>;
-    }
-    return rot ? lookup_fn_r<true>(pair_t, resid, grouped) : lookup_fn_r<false>(pair_t, resid, grouped);
+    if (nib) return rot ? lookup_fn_r<true, true>(pair_t, resid, grouped) : lookup_fn_r<false, true>(pair_t, resid, grouped);
+    return rot ? lookup_fn_r<true, false>(pair_t, resid, grouped) : lookup_fn_r<false, false>(pair_t, resid, grouped);
 }
 
 // Three CTAs per SM (eva_lookup_kernel3): one token, no residual table, no
@@ -239,15 +239,15 @@ LookupFn lookup_fn(bool pair_t, bool resid, bool grouped, bool rot, bool nib = f
 // 4096 x 4096 layer gain, 77 tiles of 11008 x 4096 lose).
 constexpr int kThreePerSmMaxTiles = 48;
 LookupFn lookup_fn3(bool grouped, bool nib) {
-    if (nib) return eva_lookup_kernel3<false, true>;
+    if (nib) return grouped ? eva_lookup_kernel3<true, true> : eva_lookup_kernel3<false, true>;
     return grouped ? eva_lookup_kernel3<true, false> : eva_lookup_kernel3<false, false>;
 }
 
 // Largest number of clusters of `cs` CTAs of this kernel resident at once.
-int max_active_clusters(LookupFn fn, size_t smem, int cs) {
+int max_active_clusters(LookupFn fn, size_t smem, int cs, int threads = kThreads) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(cs * 64);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(threads);
     cfg.dynamicSmemBytes = smem;
     cudaLaunchAttribute a[1];
     a[0].id = cudaLaunchAttributeClusterDimension;
@@ -267,12 +267,13 @@ int max_active_clusters(LookupFn fn, size_t smem, int cs) {
 // Pick the CTA rectangle: Gs slice groups (one thread-block cluster, Gs <=
 // 16) x Gt row groups, every cluster resident in one wave with at most one
 // CTA of this layer per SM (the second slot stays free for the next layer's
-// prologue), at most kMaxCtaTiles row tiles per CTA.  The cost model counts
-// the latency-bound phases of a CTA: per slice the x~ staging and the image
-// build, per unit of lookups a share of the warps' tile loop, and the
-// cluster reduction.
-void plan_grid(eva_vq_linear *h, int pair_t) {
-    const int S = h->S, T = h->T, P = h->sm_count;
+// prologue), at most kMaxCtaTiles row tiles per CTA.  `share` layers launched
+// together (eva_vq_linear_run_group) split the SMs and cluster slots.  The
+// cost model counts the latency-bound phases of a CTA: per slice the x~
+// staging and the image build, per unit of lookups a share of the warps'
+// tile loop, and the cluster reduction.
+eva_vq_linear::Plan latency_plan(const eva_vq_linear *h, int pair_t, int share) {
+    const int S = h->S, T = h->T, P = h->sm_count / share;
     const bool resid = h->desc.residual_group != 0;
     const LookupFn fn = lookup_fn(pair_t != 0, resid, h->tiles_per_cb != 0, h->desc.hadamard_block != 0,
                                   h->desc.index_bits == 4);
@@ -287,7 +288,7 @@ void plan_grid(eva_vq_linear *h, int pair_t) {
         const size_t smem_one = std::max(lookup_smem(pair_t, resid, (T + gt_min - 1) / gt_min, gs,
                                                      h->desc.hadamard_block, S),
                                          (size_t)120 * 1024);
-        const int clusters = max_active_clusters(fn, smem_one, gs);
+        const int clusters = max_active_clusters(fn, smem_one, gs) / share;
         // One CTA of this layer per SM: no more clusters than P / gs either.
         const int gt_max = std::min({T, clusters, P / gs});
         for (int gt = gt_min; gt <= gt_max; ++gt) {
@@ -307,6 +308,13 @@ void plan_grid(eva_vq_linear *h, int pair_t) {
     pl.staged = staged_tiles(h, (const void *)fn, pair_t != 0, resid, tiles, pl.Gs);
     pl.smem = lookup_smem(pair_t, resid, tiles, pl.Gs, h->desc.hadamard_block, S, pl.staged, h->unit_bytes);
     pl.smem_nostage = lookup_smem(pair_t, resid, tiles, pl.Gs, h->desc.hadamard_block, S, 0);
+    return pl;
+}
+
+void plan_grid(eva_vq_linear *h, int pair_t) {
+    const int S = h->S, T = h->T;
+    const bool resid = h->desc.residual_group != 0;
+    const eva_vq_linear::Plan pl = latency_plan(h, pair_t, 1);
     h->plan[pair_t] = pl;
 
     // Calls flagged independent: their own grid (eva_vq_plan.h), preferring
@@ -339,7 +347,8 @@ void plan_grid(eva_vq_linear *h, int pair_t) {
 }
 
 // The grid of a lookup-path call.
-const eva_vq_linear::Plan &call_plan(const eva_vq_linear *h, int B, int independent) {
+const eva_vq_linear::Plan &call_plan(const eva_vq_linear *h, int B, int independent, int share = 1) {
+    if (share > 1) return h->gplan[share];
     return independent ? h->iplan[B > 1 ? 1 : 0] : h->plan[B > 1 ? 1 : 0];
 }
 
@@ -432,9 +441,8 @@ cudaError_t set_smem_attrs(int smem_optin) {
         e = cudaFuncSetAttribute((const void *)fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_optin);
         if (e != cudaSuccess) return e;
     }
-    for (int v = 0; v < 20; ++v) {
-        const LookupFn fn = v < 16 ? lookup_fn(v & 1, (v >> 1) & 1, (v >> 2) & 1, (v >> 3) & 1)
-                                   : lookup_fn(v & 1, (v >> 1) & 1, false, false, true);
+    for (int v = 0; v < 32; ++v) {
+        const LookupFn fn = lookup_fn(v & 1, (v >> 1) & 1, (v >> 2) & 1, (v >> 3) & 1, (v >> 4) & 1);
         e = cudaFuncSetAttribute((const void *)fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         if (e != cudaSuccess) return e;
         // The device's per-block limit: it covers the one-CTA-per-SM footprint
@@ -443,8 +451,8 @@ cudaError_t set_smem_attrs(int smem_optin) {
         e = cudaFuncSetAttribute((const void *)fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_optin);
         if (e != cudaSuccess) return e;
     }
-    for (int v = 0; v < 3; ++v) {
-        const LookupFn fn = lookup_fn3(v == 1, v == 2);
+    for (int v = 0; v < 4; ++v) {
+        const LookupFn fn = lookup_fn3(v & 1, (v >> 1) & 1);
         e = cudaFuncSetAttribute((const void *)fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute((const void *)fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_optin);
@@ -534,7 +542,7 @@ int plan_tc(eva_vq_linear *h, int Np) {
         if (tc_smem(L) > (size_t)h->smem_optin) continue;
         int resident = 0;
         if (gs > 1) {
-            resident = max_active_clusters((LookupFn)fn, tc_smem(L), gs) * gs;
+            resident = max_active_clusters((LookupFn)fn, tc_smem(L), gs, kTcThreads) * gs;
         } else {
             int per_sm = 0;
             if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, (const void *)fn, kTcThreads, tc_smem(L)) !=
@@ -649,6 +657,7 @@ eva_status_t eva_vq_linear_create(eva_vq_linear_t *out, const eva_vq_desc *desc,
     chk(set_smem_attrs(h->smem_optin));
     plan_grid(h, 0);
     if (desc->max_batch > 1) plan_grid(h, 1);
+    for (int c = 2; c <= 4; ++c) h->gplan[c] = latency_plan(h, 0, c);
     int max_grid = std::max(h->plan[0].Gs * h->plan[0].Gt, h->plan[1].Gs * h->plan[1].Gt);
     if (!desc->residual_group && !desc->hadamard_block && desc->index_bits == 8 &&
         (desc->path == EVA_PATH_DEQUANT_MMA || (desc->path == EVA_PATH_AUTO && desc->max_batch >= kDequantMinBatch))) {
@@ -761,7 +770,8 @@ eva_status_t eva_vq_linear_run(eva_vq_linear_t h, const void *x, int32_t B, void
 
 namespace {
 // Parameters of one call of the lookup kernel (arguments already checked).
-LookupParams call_params(eva_vq_linear *h, const void *x, int32_t B, void *y, int independent, size_t *smem) {
+LookupParams call_params(eva_vq_linear *h, const void *x, int32_t B, void *y, int independent, size_t *smem,
+                         int share = 1) {
     const eva_vq_desc &d = h->desc;
     LookupParams p;
     std::memset(&p, 0, sizeof(p));
@@ -778,7 +788,7 @@ LookupParams call_params(eva_vq_linear *h, const void *x, int32_t B, void *y, in
     p.S = h->S;
     p.T = h->T;
     p.B = B;
-    const eva_vq_linear::Plan &pl = call_plan(h, B, independent);
+    const eva_vq_linear::Plan &pl = call_plan(h, B, independent, share);
     p.Gs = pl.Gs;
     p.Gt = pl.Gt;
     p.acc_tiles = (h->T + pl.Gt - 1) / pl.Gt;
@@ -988,9 +998,11 @@ eva_status_t eva_vq_linear_run_group(const eva_vq_linear_t *hs, const void *cons
     LookupGroup g;
     std::memset(&g, 0, sizeof(g));
     size_t smem = 0;
-    for (int i = 0; i < count; ++i) g.p[i] = call_params(hs[i], xs[i], B, ys[i], independent, &smem);
+    // Waiting one-token groups of 2..4 layers: each layer on its share of the SMs.
+    const int share = (!independent && B == 1 && count >= 2 && count <= 4) ? count : 1;
+    for (int i = 0; i < count; ++i) g.p[i] = call_params(hs[i], xs[i], B, ys[i], independent, &smem, share);
     const bool pair_t = B > 1;
-    const eva_vq_linear::Plan &pl = call_plan(hs[0], B, independent);
+    const eva_vq_linear::Plan &pl = call_plan(hs[0], B, independent, share);
     g.count = count;
     g.ctas_per_layer = pl.Gs * pl.Gt;
     const cudaError_t e = launch_pdl(group_fn(pair_t, d0.residual_group != 0), dim3(count * pl.Gs * pl.Gt),
@@ -1447,6 +1459,7 @@ eva_status_t eva_vq_quantize(const eva_quant_desc *desc, const void *w, const in
     if (d.d != 4) return EVA_ERR_UNSUPPORTED;
     if (d.index_bits < 1 || d.index_bits > 8) return EVA_ERR_UNSUPPORTED;
     if (d.N < 1 || d.K < 4 || d.K % 4 || d.iters < 0) return EVA_ERR_INVALID_ARG;
+    if (d.index_bits == 4 && d.K % 8) return EVA_ERR_INVALID_ARG;   // whole packed bytes
     if (d.codebook_rows < 0 || (d.codebook_rows && d.N % d.codebook_rows)) return EVA_ERR_INVALID_ARG;
     if (d.residual_group && (d.residual_group < 8 || d.residual_group % 8 || d.K % d.residual_group))
         return EVA_ERR_INVALID_ARG;
@@ -1467,11 +1480,15 @@ eva_status_t eva_vq_quantize(const eva_quant_desc *desc, const void *w, const in
     const int64_t nc = G * ncent;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 
-    // Work buffers, one stream-ordered allocation: [wrot][cent][cent16][sums][counts][idx][err].
+    // Work buffers, one stream-ordered allocation:
+    // [wrot][cent][cent16][sums][counts][idx][wi8][err] (wi8: the byte-per-pointer
+    // indices when the output packs them two per byte).
     auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    const bool packed = d.index_bits == 4;
     const size_t b_wrot = wrot_out ? 0 : up((size_t)M * 16), b_cent = up((size_t)nc * 16);
     const size_t b_sums = up((size_t)nc * 32), b_cnt = up((size_t)nc * 8), b_idx = up((size_t)M * 4);
-    const size_t total = b_wrot + 2 * b_cent + b_sums + b_cnt + b_idx + 256;
+    const size_t b_wi8 = packed ? up((size_t)M) : 0;
+    const size_t total = b_wrot + 2 * b_cent + b_sums + b_cnt + b_idx + b_wi8 + 256;
     uint8_t *ws = nullptr;
     cudaError_t e = cudaMallocAsync(reinterpret_cast<void **>(&ws), total, s);
     if (e != cudaSuccess) return e == cudaErrorMemoryAllocation ? EVA_ERR_OOM : cuda_status(e);
@@ -1488,6 +1505,8 @@ eva_status_t eva_vq_quantize(const eva_quant_desc *desc, const void *w, const in
     q += b_cnt;
     int32_t *idx = reinterpret_cast<int32_t *>(q);
     q += b_idx;
+    uint8_t *wi8 = packed ? q : wi_out;
+    q += b_wi8;
     int *err = reinterpret_cast<int *>(q);
     auto chk = [&](cudaError_t r) { if (e == cudaSuccess) e = r; };
     chk(cudaMemsetAsync(err, 0, sizeof(int), s));
@@ -1535,11 +1554,15 @@ eva_status_t eva_vq_quantize(const eva_quant_desc *desc, const void *w, const in
     eva_centroids_to_f16_kernel<<<blocks_for(nc * 4, 256), 256, 0, s>>>(cent, reinterpret_cast<__half *>(wc_out),
                                                                         cent16, (int)(nc * 4));
     chk(cudaGetLastError());
-    chk(launch_assign(wrot, M, cent16, ncent, vpc, wi_out, s));
+    chk(launch_assign(wrot, M, cent16, ncent, vpc, wi8, s));
     // 4.-7. residual signs and scales.
     if (d.residual_group)
-        chk(launch_residual(wrot, (int)N, (int)K, reinterpret_cast<const __half *>(wc_out), ncent, wi_out,
+        chk(launch_residual(wrot, (int)N, (int)K, reinterpret_cast<const __half *>(wc_out), ncent, wi8,
                             d.codebook_rows, d.residual_group, signs_out, reinterpret_cast<__half *>(alpha_out), s));
+    if (packed) {   // two pointers per byte, the even sub-vector in the low nibble
+        eva_pack_nibbles_kernel<<<blocks_for(M / 2, 256), 256, 0, s>>>(wi8, wi_out, M / 2);
+        chk(cudaGetLastError());
+    }
     int herr = 0;
     chk(cudaMemcpyAsync(&herr, err, sizeof(int), cudaMemcpyDeviceToHost, s));
     if (h28) cudaFreeAsync(h28, s);

@@ -193,4 +193,12 @@ __global__ void __launch_bounds__(kQThreads) eva_residual_kernel(const float4 *_
     if (lane == 0) alpha[(long long)o * gpr + q] = __double2half(acc / (double)group);
 }
 
+// Pointers < 16, one per byte -> two per byte, sub-vector 2t in the low nibble
+// of byte t (the 4-bit index layout of the layer).
+__global__ void eva_pack_nibbles_kernel(const uint8_t *__restrict__ wi8, uint8_t *__restrict__ out, long long n) {
+    const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= n) return;
+    out[t] = (uint8_t)((wi8[2 * t] & 15u) | ((wi8[2 * t + 1] & 15u) << 4));
+}
+
 }  // namespace eva

@@ -33,7 +33,8 @@ constexpr int kTcBufs = 4;                      // A stages in tensor memory
 constexpr int kTcStageCols = kTcStageK / 2;     // 32 TMEM columns per A stage (two fp16 each)
 constexpr int kTcAccCols = 64;                  // accumulator columns: up to 64 tokens
 constexpr int kTcTmemCols = 256;                // allocation: accumulator + 4 A stages (+ spare)
-constexpr int kTcThreads = 256;
+constexpr int kTcProducerWarps = 8;             // rebuild the weights (two per TMEM lane quarter)
+constexpr int kTcThreads = (kTcProducerWarps + 1) * 32;   // + one warp that issues the MMAs
 constexpr uint32_t kTcIdxStageBytes = kTcRows * kTcStageSv;   // 2048 index bytes per stage
 constexpr uint32_t kTcTabBytes = 256u * 16u * 8u;           // codebook table, 16 copies
 
@@ -88,7 +89,7 @@ __host__ __device__ inline TcLayout tc_layout(int KB, int Gs, int Np, int resid)
     L.stage = (xs_end > acc_end ? xs_end : acc_end);
     L.bar = L.stage + (uint32_t)Gs * rpo * (uint32_t)Np * 4u;
     L.bar = (L.bar + 15u) & ~15u;
-    L.slot = L.bar + 8u * (2 + kTcBufs);
+    L.slot = L.bar + 8u * (2 + 2 * kTcBufs);
     L.total = L.slot + 16u;
     return L;
 }
@@ -96,7 +97,7 @@ __host__ __device__ inline TcLayout tc_layout(int KB, int Gs, int Np, int resid)
 template <bool RESID>
 __global__ void __launch_bounds__(kTcThreads, 1) eva_tc_kernel(const TcParams p) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int eva_bid = blockIdx.x;
+    [[maybe_unused]] const int eva_bid = blockIdx.x;   // timeline stamps
     const int rb = blockIdx.x / p.Gs, sg = blockIdx.x % p.Gs;
     const int kb0 = (int)((long long)p.KB * sg / p.Gs), kb1 = (int)((long long)p.KB * (sg + 1) / p.Gs);
     const int ns = kb1 - kb0;
@@ -104,13 +105,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) eva_tc_kernel(const TcParams p)
     const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(eva_smem);
     const uint32_t bar_idx = sbase + L.bar, bar_done = bar_idx + 8u;
     auto bar_free = [&](int b) { return bar_idx + 16u + 8u * (uint32_t)b; };
+    auto bar_full = [&](int b) { return bar_idx + 16u + 8u * (uint32_t)(kTcBufs + b); };
 
     // ---- prologue: weights only ----
     EVA_STAMP(0);
     if (tid == 0) {
         mbar_init(bar_idx, 1);
         mbar_init(bar_done, 1);
-        for (int b = 0; b < kTcBufs; ++b) mbar_init(bar_free(b), 1);
+        for (int b = 0; b < kTcBufs; ++b) {
+            mbar_init(bar_free(b), 1);
+            mbar_init(bar_full(b), kTcProducerWarps);
+        }
     }
     if (warp == 0) {
         tc::tmem_alloc(sbase + L.slot, kTcTmemCols);
@@ -191,48 +196,59 @@ __global__ void __launch_bounds__(kTcThreads, 1) eva_tc_kernel(const TcParams p)
     EVA_STAMP(2);
 
     const uint32_t idesc = tc::idesc_f16_f32(kTcRows, p.Np);
-    const int q4 = warp & 3, half = warp >> 2;   // TMEM lane quarter; sub-vectors 8 half .. + 7 of a stage
-    const int row = q4 * 32 + lane;              // this thread's row within the block
-    const uint32_t lofs = 8u * (uint32_t)(lane & 15);
     const uint32_t acc_col = 0, a_col = kTcAccCols;
-    for (int st = 0; st < ns; ++st) {
-        const int buf = st % kTcBufs;
-        if (st >= kTcBufs) ok &= mbar_wait_bounded(bar_free(buf), (uint32_t)((st / kTcBufs - 1) & 1), p.wait_rounds);
-        tc::fence_after_sync();
-        // Rebuild 8 sub-vectors (32 inputs) of this thread's row.
-        const uint4 iv = *reinterpret_cast<const uint4 *>(eva_smem + L.idx + (uint32_t)st * kTcIdxStageBytes +
-                                                           16u * (uint32_t)row);
-        const uint32_t w0 = half ? iv.z : iv.x, w1 = half ? iv.w : iv.y;
-        uint32_t a[16];
+    const int q4 = warp & 3, half = (warp >> 2) & 1;   // TMEM lane quarter; sub-vectors 8 half .. + 7 of a stage
+    const int row = q4 * 32 + lane;                    // this thread's row within the block (producers)
+    // Producers rebuild stage st into A buffer st % 4 and signal full[buf];
+    // the MMA thread waits for it, issues the stage's four MMAs and commits
+    // them to free[buf], which the producers wait for before the buffer's
+    // next use.  No block-wide barrier inside the loop.
+    if (warp < kTcProducerWarps) {
+        const uint32_t lofs = 8u * (uint32_t)(lane & 15);
+        for (int st = 0; st < ns; ++st) {
+            const int buf = st % kTcBufs;
+            if (st >= kTcBufs) ok &= mbar_wait_bounded(bar_free(buf), (uint32_t)((st / kTcBufs - 1) & 1), p.wait_rounds);
+            tc::fence_after_sync();
+            // Rebuild 8 sub-vectors (32 inputs) of this thread's row.
+            const uint4 iv = *reinterpret_cast<const uint4 *>(eva_smem + L.idx + (uint32_t)st * kTcIdxStageBytes +
+                                                               16u * (uint32_t)row);
+            const uint32_t w0 = half ? iv.z : iv.x, w1 = half ? iv.w : iv.y;
+            uint32_t a[16];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const uint32_t c = ((e < 4 ? w0 : w1) >> (8 * (e & 3))) & 0xFFu;
-            const uint2 cw = *reinterpret_cast<const uint2 *>(eva_smem + L.tab + (c << 7) + lofs);
-            a[2 * e] = cw.x;
-            a[2 * e + 1] = cw.y;
-        }
-        if (RESID) {
-            // sigma bits of the row's 32 inputs (LSB first), alpha of their 128-group.
-            const uint32_t sb = *reinterpret_cast<const uint32_t *>(eva_smem + L.sgn + (uint32_t)st * kTcRows * 8u +
-                                                                    8u * (uint32_t)row + 4u * (uint32_t)half);
-            const int k0 = (kb0 + st) * kTcStageK + 32 * half;
-            const __half al = reinterpret_cast<const __half *>(eva_smem + L.alp)[row * L.ngmax + k0 / 128 - g_lo];
-            const __half2 ap = __halves2half2(al, al), an = __hneg2(ap);
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                const uint32_t two = (sb >> (2 * e)) & 3u;
-                const __half2 sgn = __halves2half2((two & 1u) ? __low2half(ap) : __low2half(an),
-                                                   (two & 2u) ? __low2half(ap) : __low2half(an));
-                __half2 w = *reinterpret_cast<const __half2 *>(&a[e]);
-                w = __hadd2(w, sgn);
-                a[e] = *reinterpret_cast<const uint32_t *>(&w);
+            for (int e = 0; e < 8; ++e) {
+                const uint32_t c = ((e < 4 ? w0 : w1) >> (8 * (e & 3))) & 0xFFu;
+                const uint2 cw = *reinterpret_cast<const uint2 *>(eva_smem + L.tab + (c << 7) + lofs);
+                a[2 * e] = cw.x;
+                a[2 * e + 1] = cw.y;
             }
+            if (RESID) {
+                // sigma bits of the row's 32 inputs (LSB first), alpha of their 128-group.
+                const uint32_t sb = *reinterpret_cast<const uint32_t *>(eva_smem + L.sgn + (uint32_t)st * kTcRows * 8u +
+                                                                        8u * (uint32_t)row + 4u * (uint32_t)half);
+                const int k0 = (kb0 + st) * kTcStageK + 32 * half;
+                const __half al = reinterpret_cast<const __half *>(eva_smem + L.alp)[row * L.ngmax + k0 / 128 - g_lo];
+                const __half2 ap = __halves2half2(al, al), an = __hneg2(ap);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const uint32_t two = (sb >> (2 * e)) & 3u;
+                    const __half2 sgn = __halves2half2((two & 1u) ? __low2half(ap) : __low2half(an),
+                                                       (two & 2u) ? __low2half(ap) : __low2half(an));
+                    __half2 w = *reinterpret_cast<const __half2 *>(&a[e]);
+                    w = __hadd2(w, sgn);
+                    a[e] = *reinterpret_cast<const uint32_t *>(&w);
+                }
+            }
+            tc::tmem_st16(tc::taddr(tbase, (uint32_t)(q4 * 32), a_col + (uint32_t)buf * kTcStageCols + 16u * (uint32_t)half),
+                          a);
+            tc::tmem_st_wait();
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_full(buf));
         }
-        tc::tmem_st16(tc::taddr(tbase, (uint32_t)(q4 * 32), a_col + (uint32_t)buf * kTcStageCols + 16u * (uint32_t)half), a);
-        tc::tmem_st_wait();
-        tc::fence_before_sync();
-        __syncthreads();
-        if (tid == 0) {
+    } else if (lane == 0) {
+        for (int st = 0; st < ns; ++st) {
+            const int buf = st % kTcBufs;
+            ok &= mbar_wait_bounded(bar_full(buf), (uint32_t)((st / kTcBufs) & 1), p.wait_rounds);
             tc::fence_after_sync();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
@@ -243,9 +259,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) eva_tc_kernel(const TcParams p)
             }
             tc::commit(bar_free(buf));
         }
+        tc::commit(bar_done);
     }
     EVA_STAMP(3);
-    if (tid == 0) tc::commit(bar_done);
     ok &= mbar_wait_bounded(bar_done, 0, p.wait_rounds);
     tc::fence_after_sync();
     EVA_STAMP(4);
@@ -266,7 +282,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) eva_tc_kernel(const TcParams p)
         tc::fence_after_sync();
         tc::tmem_dealloc(tbase, kTcTmemCols);
     }
-    if (!ok && tid == 0 && p.status) atomicOr(p.status, 4);
+    if (!ok && p.status) atomicOr(p.status, 4);
 
     EVA_STAMP(5);
     // ---- split-K: rows [rpo r, rpo (r + 1)) belong to cluster rank r ----

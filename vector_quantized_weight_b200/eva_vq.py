@@ -337,8 +337,9 @@ def quantize(w, init_index, iters: int, *, hsign=None, hadamard_block: int = 0, 
     dev = w.device
     G = N // codebook_rows if codebook_rows else 1
     ncent = 1 << index_bits
+    # 4-bit pointers come packed two per byte (the layout VQLinear(index_bits=4) takes)
     out = {"wc": torch.empty((G, ncent, 4), dtype=torch.float16, device=dev),
-           "wi": torch.empty((N, K // 4), dtype=torch.uint8, device=dev)}
+           "wi": torch.empty((N, K // 8 if index_bits == 4 else K // 4), dtype=torch.uint8, device=dev)}
     if residual_group:
         out["signs"] = torch.empty((N, K // 8), dtype=torch.uint8, device=dev)
         out["alpha"] = torch.empty((N, K // residual_group), dtype=torch.float16, device=dev)

@@ -361,6 +361,7 @@ def main():
     # timed layers stream their weights from HBM even when the region covers
     # fewer calls than one sweep of the ring.
     flush = torch.empty(2 * l2 + (1 << 20), dtype=torch.uint8, device=dev)
+    side = torch.cuda.Stream(device=dev)
 
     def timed_units(emit, n_units, period, lead, sample_clocks=False):
         """Time exactly n_units units on the device; emit(n, start) enqueues n
@@ -371,8 +372,10 @@ def main():
         first timed units; a middle graph of several periods is replayed as
         often as needed; a last graph holds the remaining units and the stop
         event.  The two events are recorded by the graphs themselves (external
-        event nodes), so the region holds the timed units alone: no graph
-        launch or host submission gap before its first unit.  Every graph is
+        event nodes; the start event on a side branch that completes with the
+        last lead-in unit), so the region holds the timed units alone, in
+        steady state: no graph launch or host submission gap, and the first
+        timed unit overlaps the lead-in as any unit overlaps its predecessor.  Every graph is
         replayed once untimed first; L2 is flushed and a spin kernel queued
         before the timed replays, so the timed layers stream their weights
         from HBM and the host has enqueued every replay before the GPU gets to
@@ -388,10 +391,15 @@ def main():
         with torch.cuda.graph(g_first, stream=stream):
             if lead:
                 emit(lead, period - lead)
-            e0.record(stream)
+            # The start event on a branch of its own: it completes with the
+            # last lead-in call, and the first timed call still depends on
+            # that call alone (its programmatic launch overlap is kept).
+            side.wait_stream(stream)
+            e0.record(side)
             emit(first, 0)
             if n_units == first:
                 e1.record(stream)
+            stream.wait_stream(side)
         graphs.append((g_first, 1))
         start = first % period
         if mids:

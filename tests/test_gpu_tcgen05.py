@@ -78,14 +78,26 @@ def test_tcgen05_integer_inputs_exact():
         assert np.array_equal(y, oracle.layer_linear(layer, x))
 
 
-def test_auto_takes_tcgen05_from_four_tokens():
+def test_auto_path_by_batch():
+    """AUTO: lookups below four tokens; from four on the warp-level dequantize
+    path where the layer allows it, the tcgen05 path from 32 tokens with one
+    shared codebook; a residual / rotated layer keeps the lookup path below
+    eight tokens and takes tcgen05 from there."""
     from vector_quantized_weight_b200 import eva_vq
-    shape = synth.LayerShape("l7b", 4096, 4096)
-    layer = synth.make_layer(shape, 8)
-    for B, path in ((1, eva_vq.EVA_PATH_OC_LOOKUP), (3, eva_vq.EVA_PATH_OC_LOOKUP), (4, eva_vq.EVA_PATH_TCGEN05)):
-        x = synth.make_x(shape.K, B, 9)
-        _, info = _run(layer, x, eva_vq.EVA_PATH_AUTO)
-        assert info.path == path, (B, info.path)
+    plain = synth.LayerShape("l7b", 4096, 4096)
+    gemma = synth.LayerShape("gemma", 3584, 3584, residual_group=128, hadamard_block=512)
+    for shape, cases in ((plain, ((1, eva_vq.EVA_PATH_OC_LOOKUP), (3, eva_vq.EVA_PATH_OC_LOOKUP),
+                                  (4, eva_vq.EVA_PATH_DEQUANT_MMA), (16, eva_vq.EVA_PATH_DEQUANT_MMA),
+                                  (32, eva_vq.EVA_PATH_TCGEN05), (64, eva_vq.EVA_PATH_TCGEN05))),
+                         (gemma, ((1, eva_vq.EVA_PATH_OC_LOOKUP), (4, eva_vq.EVA_PATH_OC_LOOKUP),
+                                  (8, eva_vq.EVA_PATH_TCGEN05))),
+                         (synth.LayerShape("l70b", 8192, 8192, codebook_rows=128),
+                          ((8, eva_vq.EVA_PATH_DEQUANT_MMA), (32, eva_vq.EVA_PATH_DEQUANT_MMA)))):
+        layer = synth.make_layer(shape, 8)
+        for B, path in cases:
+            x = synth.make_x(shape.K, B, 9)
+            _, info = _run(layer, x, eva_vq.EVA_PATH_AUTO)
+            assert info.path == path, (shape.name, B, info.path)
 
 
 def test_tcgen05_rejects_layers_it_cannot_take():

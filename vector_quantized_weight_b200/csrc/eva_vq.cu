@@ -41,10 +41,6 @@ struct eva_vq_linear {
     // that wait for their predecessor (one layer's latency), iplan[] for
     // calls flagged independent (CTA-slot time per layer).
     Plan plan[2], iplan[2];
-    // Waiting one-token calls of 2..4 layers in one eva_vq_linear_run_group
-    // launch (a decoder block's q, k, v or gate, up): each layer's grid for
-    // its share of the SMs.
-    Plan gplan[5];
     // Dequantize-to-tensor-core path (no residual, no rotation): plans for 8
     // and 16 tokens per pass.
     bool dq_ok = false;
@@ -267,13 +263,12 @@ int max_active_clusters(LookupFn fn, size_t smem, int cs, int threads = kThreads
 // Pick the CTA rectangle: Gs slice groups (one thread-block cluster, Gs <=
 // 16) x Gt row groups, every cluster resident in one wave with at most one
 // CTA of this layer per SM (the second slot stays free for the next layer's
-// prologue), at most kMaxCtaTiles row tiles per CTA.  `share` layers launched
-// together (eva_vq_linear_run_group) split the SMs and cluster slots.  The
-// cost model counts the latency-bound phases of a CTA: per slice the x~
-// staging and the image build, per unit of lookups a share of the warps'
-// tile loop, and the cluster reduction.
-eva_vq_linear::Plan latency_plan(const eva_vq_linear *h, int pair_t, int share) {
-    const int S = h->S, T = h->T, P = h->sm_count / share;
+// prologue), at most kMaxCtaTiles row tiles per CTA.  The cost model counts
+// the latency-bound phases of a CTA: per slice the x~ staging and the image
+// build, per unit of lookups a share of the warps' tile loop, and the
+// cluster reduction.
+eva_vq_linear::Plan latency_plan(const eva_vq_linear *h, int pair_t) {
+    const int S = h->S, T = h->T, P = h->sm_count;
     const bool resid = h->desc.residual_group != 0;
     const LookupFn fn = lookup_fn(pair_t != 0, resid, h->tiles_per_cb != 0, h->desc.hadamard_block != 0,
                                   h->desc.index_bits == 4);
@@ -288,7 +283,7 @@ eva_vq_linear::Plan latency_plan(const eva_vq_linear *h, int pair_t, int share) 
         const size_t smem_one = std::max(lookup_smem(pair_t, resid, (T + gt_min - 1) / gt_min, gs,
                                                      h->desc.hadamard_block, S),
                                          (size_t)120 * 1024);
-        const int clusters = max_active_clusters(fn, smem_one, gs) / share;
+        const int clusters = max_active_clusters(fn, smem_one, gs);
         // One CTA of this layer per SM: no more clusters than P / gs either.
         const int gt_max = std::min({T, clusters, P / gs});
         for (int gt = gt_min; gt <= gt_max; ++gt) {
@@ -314,7 +309,7 @@ eva_vq_linear::Plan latency_plan(const eva_vq_linear *h, int pair_t, int share) 
 void plan_grid(eva_vq_linear *h, int pair_t) {
     const int S = h->S, T = h->T;
     const bool resid = h->desc.residual_group != 0;
-    const eva_vq_linear::Plan pl = latency_plan(h, pair_t, 1);
+    const eva_vq_linear::Plan pl = latency_plan(h, pair_t);
     h->plan[pair_t] = pl;
 
     // Calls flagged independent: their own grid (eva_vq_plan.h), preferring
@@ -347,8 +342,7 @@ void plan_grid(eva_vq_linear *h, int pair_t) {
 }
 
 // The grid of a lookup-path call.
-const eva_vq_linear::Plan &call_plan(const eva_vq_linear *h, int B, int independent, int share = 1) {
-    if (share > 1) return h->gplan[share];
+const eva_vq_linear::Plan &call_plan(const eva_vq_linear *h, int B, int independent) {
     return independent ? h->iplan[B > 1 ? 1 : 0] : h->plan[B > 1 ? 1 : 0];
 }
 
@@ -507,9 +501,28 @@ bool use_three_per_sm(const eva_vq_linear *h, int B, int independent) {
 }
 
 // The tcgen05 path: forced, or AUTO from kDequantMinBatch tokens on.
+// AUTO (measured per batch on B200, one layer waiting for the previous one):
+//  - layers the warp-level dequantize path takes (no residual, no rotation):
+//    that path from kDequantMinBatch tokens on, except one shared codebook
+//    from kTcMinBatch tokens on, where tcgen05 wins (4096 x 4096: 19.0 against
+//    22.3 us at 32 tokens, 25.4 against 40.2 at 64; with per-group codebooks
+//    the warp-level path stays ahead, 57.8 against 70.9 us at 32 tokens);
+//  - residual / rotated layers: the lookup path below kTcResidMinBatch tokens
+//    (3.125-bit 3584 x 3584: 15.4 against 22.0 us at 4 tokens), tcgen05 from
+//    there (24.7 against 55.5 us at 16).
+// A tcgen05.mma of M = 128 rows takes about as long for N = 16 tokens as for
+// N = 64 (about 100 cycles per instruction, measured), so the tensor-core
+// path pays off as the batch grows, while the warp-level MMA of 8 tokens
+// scales with the batch.
+constexpr int kTcMinBatch = 32;
+constexpr int kTcResidMinBatch = 8;
+
 bool use_tc(const eva_vq_linear *h, int B) {
     if (!h->tc_ok) return false;
-    return h->desc.path == EVA_PATH_TCGEN05 || (h->desc.path == EVA_PATH_AUTO && B >= kDequantMinBatch);
+    if (h->desc.path == EVA_PATH_TCGEN05) return true;
+    if (h->desc.path != EVA_PATH_AUTO || B < kDequantMinBatch) return false;
+    if (!h->dq_ok) return B >= kTcResidMinBatch;
+    return B >= kTcMinBatch && h->desc.codebook_rows == 0;
 }
 
 bool use_dequant(const eva_vq_linear *h, int B) {
@@ -517,12 +530,15 @@ bool use_dequant(const eva_vq_linear *h, int B) {
     return h->desc.path == EVA_PATH_DEQUANT_MMA || (h->desc.path == EVA_PATH_AUTO && B >= kDequantMinBatch);
 }
 
-// Dynamic shared memory of a tcgen05-path CTA: at least kTcMinSmem, so no
-// more than two CTAs share an SM and their tensor-memory allocations (256
-// columns each) always fit in the SM's 512 -- an allocation never waits for
-// another CTA's.
-constexpr size_t kTcMinSmem = 80 * 1024;
-size_t tc_smem(const TcLayout &L) { return std::max((size_t)L.total, kTcMinSmem); }
+// Tensor memory per tcgen05-path CTA (columns) and the dynamic shared memory
+// that goes with it: with 256 columns at least 80 KB, so no more than two
+// CTAs share an SM; with 512 at least 116 KB, so one CTA has the SM.  Either
+// way the allocations of the CTAs on an SM fit in its 512 columns together,
+// and an allocation never waits for another CTA's.
+constexpr int kTcTmemCols = 256;
+size_t tc_smem(const TcLayout &L, int tmem_cols = kTcTmemCols) {
+    return std::max((size_t)L.total, (size_t)(tmem_cols > 256 ? 116 : 80) * 1024);
+}
 
 using TcFn = void (*)(TcParams);
 TcFn tc_fn(bool resid) { return resid ? eva_tc_kernel<true> : eva_tc_kernel<false>; }
@@ -537,7 +553,7 @@ int plan_tc(eva_vq_linear *h, int Np) {
     const TcFn fn = tc_fn(resid);
     double best = 1e300;
     int pick = 0;
-    for (int gs = 1; gs <= std::min(16, KB); ++gs) {
+    for (int gs = 1; gs <= std::min(16, KB); gs *= 2) {   // a power of two: it divides the 128 rows
         const TcLayout L = tc_layout(KB, gs, Np, resid ? 1 : 0);
         if (tc_smem(L) > (size_t)h->smem_optin) continue;
         int resident = 0;
@@ -657,7 +673,6 @@ eva_status_t eva_vq_linear_create(eva_vq_linear_t *out, const eva_vq_desc *desc,
     chk(set_smem_attrs(h->smem_optin));
     plan_grid(h, 0);
     if (desc->max_batch > 1) plan_grid(h, 1);
-    for (int c = 2; c <= 4; ++c) h->gplan[c] = latency_plan(h, 0, c);
     int max_grid = std::max(h->plan[0].Gs * h->plan[0].Gt, h->plan[1].Gs * h->plan[1].Gt);
     if (!desc->residual_group && !desc->hadamard_block && desc->index_bits == 8 &&
         (desc->path == EVA_PATH_DEQUANT_MMA || (desc->path == EVA_PATH_AUTO && desc->max_batch >= kDequantMinBatch))) {
@@ -770,8 +785,7 @@ eva_status_t eva_vq_linear_run(eva_vq_linear_t h, const void *x, int32_t B, void
 
 namespace {
 // Parameters of one call of the lookup kernel (arguments already checked).
-LookupParams call_params(eva_vq_linear *h, const void *x, int32_t B, void *y, int independent, size_t *smem,
-                         int share = 1) {
+LookupParams call_params(eva_vq_linear *h, const void *x, int32_t B, void *y, int independent, size_t *smem) {
     const eva_vq_desc &d = h->desc;
     LookupParams p;
     std::memset(&p, 0, sizeof(p));
@@ -788,7 +802,7 @@ LookupParams call_params(eva_vq_linear *h, const void *x, int32_t B, void *y, in
     p.S = h->S;
     p.T = h->T;
     p.B = B;
-    const eva_vq_linear::Plan &pl = call_plan(h, B, independent, share);
+    const eva_vq_linear::Plan &pl = call_plan(h, B, independent);
     p.Gs = pl.Gs;
     p.Gt = pl.Gt;
     p.acc_tiles = (h->T + pl.Gt - 1) / pl.Gt;
@@ -918,11 +932,14 @@ cudaError_t launch_tc(eva_vq_linear *h, const void *x, int B, void *y, cudaStrea
         p.resid = d.residual_group != 0;
         p.status = h->status;
         p.wait_rounds = kWaitRounds;
+        p.tmem_cols = kTcTmemCols;
+        p.nbuf = std::min(kTcMaxBufs, (p.tmem_cols - ((Np + 31) & ~31)) / kTcStageCols);
 #ifdef EVA_TIMELINE
         p.timeline = h->timeline;
 #endif
         const TcLayout L = tc_layout(p.KB, gs, Np, p.resid);
-        e = launch_pdl(tc_fn(p.resid != 0), dim3(p.R * gs), dim3(kTcThreads), tc_smem(L), s, gs > 1 ? gs : 0, p);
+        e = launch_pdl(tc_fn(p.resid != 0), dim3(p.R * gs), dim3(kTcThreads), tc_smem(L, p.tmem_cols), s,
+                       gs > 1 ? gs : 0, p);
         if (e != cudaSuccess) return e;
         grid = p.R * gs;
         ++kernels;
@@ -998,11 +1015,9 @@ eva_status_t eva_vq_linear_run_group(const eva_vq_linear_t *hs, const void *cons
     LookupGroup g;
     std::memset(&g, 0, sizeof(g));
     size_t smem = 0;
-    // Waiting one-token groups of 2..4 layers: each layer on its share of the SMs.
-    const int share = (!independent && B == 1 && count >= 2 && count <= 4) ? count : 1;
-    for (int i = 0; i < count; ++i) g.p[i] = call_params(hs[i], xs[i], B, ys[i], independent, &smem, share);
+    for (int i = 0; i < count; ++i) g.p[i] = call_params(hs[i], xs[i], B, ys[i], independent, &smem);
     const bool pair_t = B > 1;
-    const eva_vq_linear::Plan &pl = call_plan(hs[0], B, independent, share);
+    const eva_vq_linear::Plan &pl = call_plan(hs[0], B, independent);
     g.count = count;
     g.ctas_per_layer = pl.Gs * pl.Gt;
     const cudaError_t e = launch_pdl(group_fn(pair_t, d0.residual_group != 0), dim3(count * pl.Gs * pl.Gt),

@@ -29,12 +29,11 @@ namespace eva {
 constexpr int kTcRows = 128;                    // rows per CTA: the MMA's M
 constexpr int kTcStageSv = 16;                  // sub-vectors per stage
 constexpr int kTcStageK = kTcStageSv * kD;      // 64 inputs per stage: four MMAs of K = 16
-constexpr int kTcBufs = 4;                      // A stages in tensor memory
+constexpr int kTcMaxBufs = 15;                  // A stages in tensor memory, at most
 constexpr int kTcStageCols = kTcStageK / 2;     // 32 TMEM columns per A stage (two fp16 each)
-constexpr int kTcAccCols = 64;                  // accumulator columns: up to 64 tokens
-constexpr int kTcTmemCols = 256;                // allocation: accumulator + 4 A stages (+ spare)
 constexpr int kTcProducerWarps = 8;             // rebuild the weights (two per TMEM lane quarter)
 constexpr int kTcThreads = (kTcProducerWarps + 1) * 32;   // + one warp that issues the MMAs
+constexpr int kTcXLoads = 8;                    // x chunks a thread has in flight while staging
 constexpr uint32_t kTcIdxStageBytes = kTcRows * kTcStageSv;   // 2048 index bytes per stage
 constexpr uint32_t kTcTabBytes = 256u * 16u * 8u;           // codebook table, 16 copies
 
@@ -47,12 +46,14 @@ struct TcParams {
     void *y;                 // [B][N]
     int N, K, B, Np;         // Np: tokens padded to a multiple of 16 (the MMA's N), <= 64
     int R, KB;               // row blocks, stages over K
-    int Gs;                  // CTAs per row block (one cluster); blockIdx.x = rb * Gs + sg
+    int Gs;                  // CTAs per row block (one cluster, Gs in 1, 2, 4, 8, 16); blockIdx.x = rb * Gs + sg
     int rows_per_cb;         // 0: one codebook; else rows per codebook (a multiple of 128)
     int x_f32, out_f32, independent;
     int resid;               // 1: add alpha * sigma to every rebuilt weight
     int *status;             // device error word (bit 2: a bounded wait of this kernel gave up)
     int wait_rounds;
+    int tmem_cols;           // tensor-memory allocation: 256 (two CTAs per SM) or 512 (one)
+    int nbuf;                // A stages in flight: (tmem_cols - a_col) / 32, a_col = Np rounded up to 32
 #ifdef EVA_TIMELINE
     unsigned long long *timeline;   // [grid][8] %globaltimer stamps of the last run
 #endif
@@ -85,11 +86,11 @@ __host__ __device__ inline TcLayout tc_layout(int KB, int Gs, int Np, int resid)
     L.acc = L.xs;
     const uint32_t xs_end = L.xs + (uint32_t)(Np / 8) * L.xs_sbo;
     const uint32_t acc_end = L.acc + (uint32_t)kTcRows * (uint32_t)Np * 4u;
-    const uint32_t rpo = (uint32_t)((kTcRows + Gs - 1) / Gs);          // rows owned per cluster rank
+    const uint32_t rpo = (uint32_t)(kTcRows / Gs);                     // rows owned per cluster rank
     L.stage = (xs_end > acc_end ? xs_end : acc_end);
     L.bar = L.stage + (uint32_t)Gs * rpo * (uint32_t)Np * 4u;
     L.bar = (L.bar + 15u) & ~15u;
-    L.slot = L.bar + 8u * (2 + 2 * kTcBufs);
+    L.slot = L.bar + 8u * (2 + 2 * kTcMaxBufs);
     L.total = L.slot + 16u;
     return L;
 }
@@ -105,20 +106,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) eva_tc_kernel(const TcParams p)
     const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(eva_smem);
     const uint32_t bar_idx = sbase + L.bar, bar_done = bar_idx + 8u;
     auto bar_free = [&](int b) { return bar_idx + 16u + 8u * (uint32_t)b; };
-    auto bar_full = [&](int b) { return bar_idx + 16u + 8u * (uint32_t)(kTcBufs + b); };
+    auto bar_full = [&](int b) { return bar_idx + 16u + 8u * (uint32_t)(kTcMaxBufs + b); };
+    const int nbuf = p.nbuf;
 
     // ---- prologue: weights only ----
     EVA_STAMP(0);
     if (tid == 0) {
         mbar_init(bar_idx, 1);
         mbar_init(bar_done, 1);
-        for (int b = 0; b < kTcBufs; ++b) {
+        for (int b = 0; b < nbuf; ++b) {
             mbar_init(bar_free(b), 1);
             mbar_init(bar_full(b), kTcProducerWarps);
         }
     }
     if (warp == 0) {
-        tc::tmem_alloc(sbase + L.slot, kTcTmemCols);
+        tc::tmem_alloc(sbase + L.slot, (uint32_t)p.tmem_cols);
         tc::tmem_relinquish();
     }
     tc::fence_before_sync();
@@ -166,27 +168,42 @@ __global__ void __launch_bounds__(kTcThreads, 1) eva_tc_kernel(const TcParams p)
     EVA_STAMP(1);
 
     // ---- x: the B operand, K-major core matrices of 8 tokens x 8 inputs ----
+    // A warp moves 8 tokens x 4 consecutive chunks of 8 inputs: lane l takes
+    // token 8 g8 + (l & 7), chunk 4 c4 + (l >> 3), so its global read is 64
+    // contiguous bytes per token and its shared-memory write 512 contiguous
+    // bytes (four core matrices, no bank conflict).  Every thread issues its
+    // loads (up to kTcXLoads) before it stores any: one round trip to L2.
     {
-        const int kbase = kb0 * kTcStageK, kc8 = ns * (kTcStageK / 8);
-        for (int i = tid; i < p.Np * kc8; i += kTcThreads) {
-            const int n = i / kc8, c8 = i - n * kc8;
-            const int k = kbase + 8 * c8;
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (n < p.B) {
-                if (p.x_f32) {
-                    const float4 *xp = reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(p.x) +
-                                                                        (size_t)n * p.K + k);
-                    const float4 a = __ldcg(xp), b = __ldcg(xp + 1);
-                    v.x = pack_half2(a.x, a.y);
-                    v.y = pack_half2(a.z, a.w);
-                    v.z = pack_half2(b.x, b.y);
-                    v.w = pack_half2(b.z, b.w);
-                } else {
-                    v = __ldcg(reinterpret_cast<const uint4 *>(reinterpret_cast<const __half *>(p.x) + (size_t)n * p.K + k));
+        const int kbase = kb0 * kTcStageK, kc8 = ns * (kTcStageK / 8), kc4 = kc8 / 4, total = p.Np * kc8;
+        for (int i0 = 0; i0 < total; i0 += kTcThreads * kTcXLoads) {
+            uint4 v[kTcXLoads];
+#pragma unroll
+            for (int u = 0; u < kTcXLoads; ++u) {
+                const int i = i0 + u * kTcThreads + tid;
+                const int q = i >> 5, g8 = q / kc4, c4 = q - g8 * kc4;
+                const int n = 8 * g8 + (lane & 7), c8 = 4 * c4 + (lane >> 3);
+                v[u] = make_uint4(0u, 0u, 0u, 0u);
+                if (i < total && n < p.B) {
+                    const size_t e = (size_t)n * p.K + kbase + 8 * c8;
+                    if (p.x_f32) {
+                        const float4 *xp = reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(p.x) + e);
+                        const float4 a = __ldcg(xp), b = __ldcg(xp + 1);
+                        v[u] = make_uint4(pack_half2(a.x, a.y), pack_half2(a.z, a.w), pack_half2(b.x, b.y),
+                                          pack_half2(b.z, b.w));
+                    } else {
+                        v[u] = __ldcg(reinterpret_cast<const uint4 *>(reinterpret_cast<const __half *>(p.x) + e));
+                    }
                 }
             }
-            *reinterpret_cast<uint4 *>(eva_smem + L.xs + (uint32_t)(n >> 3) * L.xs_sbo + (uint32_t)c8 * 128u +
-                                       (uint32_t)(n & 7) * 16u) = v;
+#pragma unroll
+            for (int u = 0; u < kTcXLoads; ++u) {
+                const int i = i0 + u * kTcThreads + tid;
+                if (i >= total) break;
+                const int q = i >> 5, g8 = q / kc4, c4 = q - g8 * kc4;
+                const int n = 8 * g8 + (lane & 7), c8 = 4 * c4 + (lane >> 3);
+                *reinterpret_cast<uint4 *>(eva_smem + L.xs + (uint32_t)(n >> 3) * L.xs_sbo + (uint32_t)c8 * 128u +
+                                           (uint32_t)(n & 7) * 16u) = v[u];
+            }
         }
     }
     // Make the x stage visible to the tensor cores (generic -> async proxy).
@@ -196,7 +213,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) eva_tc_kernel(const TcParams p)
     EVA_STAMP(2);
 
     const uint32_t idesc = tc::idesc_f16_f32(kTcRows, p.Np);
-    const uint32_t acc_col = 0, a_col = kTcAccCols;
+    const uint32_t acc_col = 0, a_col = (uint32_t)((p.Np + 31) & ~31);
     const int q4 = warp & 3, half = (warp >> 2) & 1;   // TMEM lane quarter; sub-vectors 8 half .. + 7 of a stage
     const int row = q4 * 32 + lane;                    // this thread's row within the block (producers)
     // Producers rebuild stage st into A buffer st % 4 and signal full[buf];
@@ -206,8 +223,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) eva_tc_kernel(const TcParams p)
     if (warp < kTcProducerWarps) {
         const uint32_t lofs = 8u * (uint32_t)(lane & 15);
         for (int st = 0; st < ns; ++st) {
-            const int buf = st % kTcBufs;
-            if (st >= kTcBufs) ok &= mbar_wait_bounded(bar_free(buf), (uint32_t)((st / kTcBufs - 1) & 1), p.wait_rounds);
+            const int buf = st % nbuf;
+            if (st >= nbuf) ok &= mbar_wait_bounded(bar_free(buf), (uint32_t)((st / nbuf - 1) & 1), p.wait_rounds);
             tc::fence_after_sync();
             // Rebuild 8 sub-vectors (32 inputs) of this thread's row.
             const uint4 iv = *reinterpret_cast<const uint4 *>(eva_smem + L.idx + (uint32_t)st * kTcIdxStageBytes +
@@ -247,8 +264,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) eva_tc_kernel(const TcParams p)
         }
     } else if (lane == 0) {
         for (int st = 0; st < ns; ++st) {
-            const int buf = st % kTcBufs;
-            ok &= mbar_wait_bounded(bar_full(buf), (uint32_t)((st / kTcBufs) & 1), p.wait_rounds);
+            const int buf = st % nbuf;
+            ok &= mbar_wait_bounded(bar_full(buf), (uint32_t)((st / nbuf) & 1), p.wait_rounds);
             tc::fence_after_sync();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
@@ -265,43 +282,44 @@ __global__ void __launch_bounds__(kTcThreads, 1) eva_tc_kernel(const TcParams p)
     ok &= mbar_wait_bounded(bar_done, 0, p.wait_rounds);
     tc::fence_after_sync();
     EVA_STAMP(4);
-    // ---- accumulator -> shared memory [row][Np] fp32 ----
+    // ---- accumulator -> shared memory, token-major [Np][128] fp32 ----
+    // (thread = row: consecutive threads write consecutive words)
+    float *acc = reinterpret_cast<float *>(eva_smem + L.acc);
     if (warp < 4) {
         for (int c0 = 0; c0 < p.Np; c0 += 8) {
             float v[8];
             tc::tmem_ld8(tc::taddr(tbase, (uint32_t)(warp * 32), acc_col + (uint32_t)c0), v);
             tc::tmem_ld_wait();
-            float *dst = reinterpret_cast<float *>(eva_smem + L.acc) + (size_t)row * p.Np + c0;
-            *reinterpret_cast<float4 *>(dst) = make_float4(v[0], v[1], v[2], v[3]);
-            *reinterpret_cast<float4 *>(dst + 4) = make_float4(v[4], v[5], v[6], v[7]);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[(c0 + e) * kTcRows + row] = v[e];
         }
     }
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 0) {
         tc::fence_after_sync();
-        tc::tmem_dealloc(tbase, kTcTmemCols);
+        tc::tmem_dealloc(tbase, (uint32_t)p.tmem_cols);
     }
     if (!ok && p.status) atomicOr(p.status, 4);
 
     EVA_STAMP(5);
-    // ---- split-K: rows [rpo r, rpo (r + 1)) belong to cluster rank r ----
-    const int rpo = (kTcRows + p.Gs - 1) / p.Gs;
-    const float *acc = reinterpret_cast<const float *>(eva_smem + L.acc);
+    // ---- split-K: rows [rpo r, rpo (r + 1)) belong to cluster rank r (Gs
+    // divides 128, so rpo is a multiple of 8); the owner's stage is
+    // [Gs sources][Np tokens][rpo rows] ----
+    const int rpo = kTcRows / p.Gs;
     if (p.Gs > 1) {
         const uint32_t stage_addr = sbase + L.stage;
-        const int n4 = p.Np / 4;
-        for (int i = tid; i < kTcRows * n4; i += kTcThreads) {
-            const int r = i / n4, c = (i - r * n4) * 4;
+        for (int i = tid; i < p.Np * (kTcRows / 4); i += kTcThreads) {
+            const int b = i / (kTcRows / 4), r = 4 * (i - b * (kTcRows / 4));
             const int owner = r / rpo, rl = r - owner * rpo;
-            const float4 v = *reinterpret_cast<const float4 *>(acc + (size_t)r * p.Np + c);
-            const uint32_t dst = (uint32_t)(((sg * rpo + rl) * p.Np + c) * 4);
+            const float4 v = *reinterpret_cast<const float4 *>(acc + b * kTcRows + r);
+            const uint32_t dst = (uint32_t)(((sg * p.Np + b) * rpo + rl) * 4);
             st_dsmem_v4(stage_addr + dst, (uint32_t)owner, v);
         }
         cluster_sync_all();
     }
     {
-        const int r0 = p.Gs > 1 ? sg * rpo : 0, nr = p.Gs > 1 ? min(rpo, kTcRows - r0) : kTcRows;
+        const int r0 = sg * rpo, nr = rpo;
         const float *stage = reinterpret_cast<const float *>(eva_smem + L.stage);
         for (int i = tid; i < nr * p.B; i += kTcThreads) {
             const int rl = i % nr, b = i / nr;
@@ -310,9 +328,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) eva_tc_kernel(const TcParams p)
             float sum;
             if (p.Gs > 1) {
                 sum = 0.f;
-                for (int k = 0; k < p.Gs; ++k) sum += stage[(k * rpo + rl) * p.Np + b];
+                for (int k = 0; k < p.Gs; ++k) sum += stage[(k * p.Np + b) * rpo + rl];
             } else {
-                sum = acc[(size_t)rl * p.Np + b];
+                sum = acc[b * kTcRows + rl];
             }
             const size_t yi = (size_t)b * p.N + o;
             if (p.out_f32) reinterpret_cast<float *>(p.y)[yi] = sum;

@@ -63,3 +63,27 @@ def test_inject_rejects_bad_round_counts():
         assert lib.eva_vq_debug_inject_wait_timeout(lin.handle, bad) == eva_vq.EVA_ERR_INVALID_ARG
     torch.cuda.synchronize()
     lin.close()
+
+
+def test_bounded_wait_gives_up_on_the_dequantize_path():
+    """The warp-level dequantize path (four tokens and more) stages its index
+    units the same way: the hook makes its wait run out too."""
+    import torch
+    from vector_quantized_weight_b200 import eva_vq
+    shape = synth.LayerShape("l7b_4096x4096", 4096, 4096)
+    layer = synth.make_layer(shape, 4244)
+    x_np = synth.make_x(shape.K, 4, 4245)
+    x = torch.from_numpy(x_np).cuda()
+    lin = eva_vq.from_layer(layer, max_batch=4)
+    eva_vq.eva_vq_debug_inject_wait_timeout(lin.handle, 1024)
+    lin(x)
+    torch.cuda.synchronize()
+    assert lin.info().path == eva_vq.EVA_PATH_DEQUANT_MMA
+    assert eva_vq.eva_vq_sync_status(lin.handle) == eva_vq.EVA_ERR_DEVICE_TIMEOUT
+    lin.close()
+    fresh = eva_vq.from_layer(layer, max_batch=4)
+    y = fresh(x).float().cpu().numpy()
+    torch.cuda.synchronize()
+    assert eva_vq.eva_vq_sync_status(fresh.handle) == eva_vq.EVA_OK
+    assert np.all(norm_rel_err(y, oracle.layer_linear(layer, x_np, nthreads=8)) <= TOL)
+    fresh.close()

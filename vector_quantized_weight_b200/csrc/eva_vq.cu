@@ -384,12 +384,14 @@ DequantFn dequant_fn(bool grouped, int ntg) {
 constexpr int kDequantMinBatch = 4;
 
 // Dynamic shared memory of the dequantize kernel: the replicated codebook,
-// the x stage of up to nsl slices, the running sums and the reduction stage.
-size_t dequant_smem(int nsl, int tiles, int gs, int ntg) {
+// the x stage of up to nsl slices, the running sums, the reduction stage, the
+// staging mbarrier and `staged` index units.
+size_t dequant_smem(int nsl, int tiles, int gs, int ntg, int staged = 0) {
     const size_t blk = (size_t)kTileRows * 8 * ntg * 4;
     const size_t xs = ((size_t)nsl * 8 * ntg * kXTokStride + 127) & ~(size_t)127;
     const size_t nslot = (size_t)(tiles + gs - 1) / gs;
-    return (size_t)kTabBytes + xs + (size_t)tiles * blk + nslot * gs * blk;
+    const size_t base = (size_t)kTabBytes + xs + (size_t)tiles * blk + nslot * gs * blk;
+    return ((base + 127) & ~(size_t)127) + 128 + (size_t)staged * kUnitBytes;
 }
 
 // Same search as plan_grid, for the dequantize kernel (one CTA per SM, every
@@ -421,8 +423,18 @@ void plan_dequant(eva_vq_linear *h, int ntg) {
         }
     }
     if (pl.Gs == 0) return;   // nothing fits: the lookup path serves every batch
-    const int tiles = (T + pl.Gt - 1) / pl.Gt;
-    pl.smem = pl.smem_nostage = dequant_smem((S + pl.Gs - 1) / pl.Gs, tiles, pl.Gs, ntg);
+    const int tiles = (T + pl.Gt - 1) / pl.Gt, nsl = (S + pl.Gs - 1) / pl.Gs;
+    // Index units copied into shared memory in the prologue: as many of the
+    // CTA's units as fit while the CTA still leaves half the SM to the next
+    // layer's early-launched CTA (whose prologue then overlaps this one);
+    // none when the rest of the footprint already takes more than half
+    // (measured: staging past that point costs the overlap, 6.1 -> 11.4 us
+    // for 4096^2 at 4 tokens).
+    const size_t base = dequant_smem(nsl, tiles, pl.Gs, ntg);
+    const size_t half = (size_t)h->smem_per_sm / 2 - (size_t)h->smem_reserved;
+    pl.staged = base < half ? (int)std::min<size_t>((size_t)nsl * tiles, (half - base) / kUnitBytes) : 0;
+    pl.smem = dequant_smem(nsl, tiles, pl.Gs, ntg, pl.staged);
+    pl.smem_nostage = dequant_smem(nsl, tiles, pl.Gs, ntg);
     h->dq[ntg - 1] = pl;
 }
 
@@ -474,6 +486,16 @@ cudaError_t set_smem_attrs(int smem_optin) {
     return cudaFuncSetAttribute(eva_hadamard_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 4096 * 4);
 }
 
+// Failure-detection test hook (eva_vq_debug_inject_wait_timeout): a launch
+// that stages index units skips their copy and gives up its wait early, once.
+void apply_injection(eva_vq_linear *h, LookupParams &p) {
+    if (h->inject_wait_rounds > 0 && p.wi_staged > 0) {
+        p.skip_stage_copy = 1;
+        p.wait_rounds = h->inject_wait_rounds;
+        h->inject_wait_rounds = 0;
+    }
+}
+
 // Launch the dequantize kernel for a call whose common parameters are in p.
 cudaError_t launch_dequant(eva_vq_linear *h, LookupParams p, int B, cudaStream_t s, size_t *smem_out,
                            int *grid_out) {
@@ -482,8 +504,9 @@ cudaError_t launch_dequant(eva_vq_linear *h, LookupParams p, int B, cudaStream_t
     p.Gs = pl.Gs;
     p.Gt = pl.Gt;
     p.acc_tiles = (h->T + pl.Gt - 1) / pl.Gt;
-    p.wi_staged = 0;
+    p.wi_staged = pl.staged;
     p.rot_b = 0;
+    apply_injection(h, p);
     *smem_out = pl.smem;
     *grid_out = pl.Gs * pl.Gt;
 #ifdef EVA_DEVICE_CHECKS
@@ -568,6 +591,10 @@ int plan_tc(eva_vq_linear *h, int Np) {
             }
             resident = per_sm * h->sm_count;
         }
+        // One CTA per SM of this layer at a time: in a chain of calls the next
+        // layer's early-launched CTAs (programmatic dependent launch) hold the
+        // other slot while they wait.
+        resident = std::min(resident, h->sm_count);
         if (resident <= 0) continue;
         const int rounds = (R * gs + resident - 1) / resident;
         const double cost = (double)rounds * (300.0 + 160.0 * ((KB + gs - 1) / gs)) + (gs > 1 ? 700.0 + 40.0 * gs : 0.0);
@@ -813,11 +840,6 @@ LookupParams call_params(eva_vq_linear *h, const void *x, int32_t B, void *y, in
     p.wi_staged = independent ? 0 : pl.staged;
     p.status = h->status;
     p.wait_rounds = kWaitRounds;
-    if (h->inject_wait_rounds > 0 && p.wi_staged > 0) {   // one-shot test injection
-        p.skip_stage_copy = 1;
-        p.wait_rounds = h->inject_wait_rounds;
-        h->inject_wait_rounds = 0;
-    }
     p.tiles_per_cb = h->tiles_per_cb;
     p.ncent = h->ncent;
     p.out_f32 = d.out_dtype == EVA_F32 ? 1 : 0;
@@ -979,6 +1001,7 @@ eva_status_t eva_vq_linear_run_ex(eva_vq_linear_t h, const void *x, int32_t B, v
     const eva_vq_linear::Plan &pl = call_plan(h, B, independent);
     LookupFn fn = lookup_fn(pair_t, resid, h->tiles_per_cb != 0, p.rot_b != 0, d.index_bits == 4);
     if (independent && use_three_per_sm(h, B, independent)) fn = lookup_fn3(h->tiles_per_cb != 0, d.index_bits == 4);
+    apply_injection(h, p);
     e = launch_pdl(fn, dim3(pl.Gs * pl.Gt), dim3(kThreads), smem, s, pl.Gs, p);
     if (e != cudaSuccess) return cuda_status(e);
     h->last_grid = pl.Gs * pl.Gt;

@@ -61,7 +61,9 @@ __global__ void __launch_bounds__(kThreads, 1) eva_dequant_kernel(const LookupPa
     const int cb_last = GROUPED ? (t1 - 1) / p.tiles_per_cb : 0;
 
     // Shared memory: codebook table | x stage [slice][token] | running sums
-    // [tile][16][TT] | reduction stage [ceil(acc_tiles / Gs)][Gs][16][TT].
+    // [tile][16][TT] | reduction stage [ceil(acc_tiles / Gs)][Gs][16][TT] |
+    // the staging mbarrier (128 bytes) | the staged index units (slice-major:
+    // unit sl * ctiles + tl).
     constexpr uint32_t TAB_OFF = 0, XS_OFF = kTabBytes;
     // The layout must be the same in every CTA of a cluster (peers write into
     // the reduction stage at this CTA's offsets): size the x stage for the
@@ -72,16 +74,44 @@ __global__ void __launch_bounds__(kThreads, 1) eva_dequant_kernel(const LookupPa
     float *acc_s = reinterpret_cast<float *>(eva_smem + ACC_OFF);
     const float *stage = reinterpret_cast<const float *>(eva_smem + STAGE_OFF);
     const uint32_t stage_addr = (uint32_t)__cvta_generic_to_shared(eva_smem + STAGE_OFF);
+    const uint32_t BAR_OFF = (STAGE_OFF + (uint32_t)((p.acc_tiles + p.Gs - 1) / p.Gs) * p.Gs * BLK + 127u) & ~127u;
+    const uint32_t UNITS_OFF = BAR_OFF + 128u;
+    const int nst = min(nsl * ctiles, p.wi_staged);   // units copied into shared memory
+    const uint32_t bar = (uint32_t)__cvta_generic_to_shared(eva_smem + BAR_OFF);
 
     // ---- prologue: weights only ----
     EVA_STAMP(0);
     pdl_launch();
     asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
-    if (tid < nsl) {
-        const size_t u = (size_t)(s0 + tid) * p.T + t0;
-        const uint32_t nt = (uint32_t)ctiles;
-        if (!EVA_BAD_G(BUF_WI, p.wi + u * kUnitBytes, nt * kUnitBytes)) prefetch_l2_bulk(p.wi + u * kUnitBytes, nt * kUnitBytes);
+    // The CTA's first nst index units: bulk copies into shared memory, one per
+    // slice (a slice's units of this CTA are contiguous), on one mbarrier.
+    if (tid == 0 && nst > 0) {
+        mbar_init(bar, 1);
+        if (!p.skip_stage_copy && !EVA_BAD_S(UNITS_OFF) && !EVA_BAD_S(UNITS_OFF + (uint32_t)nst * kUnitBytes - 4u)) {
+            mbar_arrive_expect_tx(bar, (uint32_t)nst * kUnitBytes);
+            for (int sl = 0; sl < nsl; ++sl) {
+                const int cnt = min(ctiles, nst - sl * ctiles);
+                if (cnt <= 0) break;
+                const uint8_t *src = p.wi + ((size_t)(s0 + sl) * p.T + t0) * kUnitBytes;
+                const uint32_t dst = (uint32_t)__cvta_generic_to_shared(eva_smem + UNITS_OFF) +
+                                     (uint32_t)(sl * ctiles) * kUnitBytes;
+                const uint32_t bytes = (uint32_t)cnt * kUnitBytes;
+                for (uint32_t off = 0; off < bytes; off += 32768u)
+                    bulk_copy_g2s(dst + off, src + off, min(32768u, bytes - off), bar);
+            }
+        } else if (!p.skip_stage_copy) {
+            mbar_arrive(bar);
+        }
     }
+    if (tid < nsl) {
+        // L2 prefetch of the slice's units that are not staged.
+        const int first = max(0, min(ctiles, nst - tid * ctiles));
+        const size_t u = (size_t)(s0 + tid) * p.T + t0 + first;
+        const uint32_t nt = (uint32_t)(ctiles - first);
+        if (nt > 0 && !EVA_BAD_G(BUF_WI, p.wi + u * kUnitBytes, nt * kUnitBytes))
+            prefetch_l2_bulk(p.wi + u * kUnitBytes, nt * kUnitBytes);
+    }
+    bool units_ready = nst == 0;
     build_codebook_table(p, cb_first, tid);
     int built_cb = cb_first;
 
@@ -140,19 +170,33 @@ __global__ void __launch_bounds__(kThreads, 1) eva_dequant_kernel(const LookupPa
                                              8u * (uint32_t)dq_subvec(beta, q);
                         xb[t][beta] = EVA_BAD_S(off) ? make_uint2(0u, 0u) : lds64(off);
                     }
-                uint4 nb0 = make_uint4(0u, 0u, 0u, 0u), nb1 = nb0;
-                if (i0 < i1) {
-                    const uint8_t *up = p.wi + ((size_t)s * p.T + t0 + warp + kWarps * i0) * kUnitBytes + 16 * lane;
-                    if (!EVA_BAD_G(BUF_WI, up, 16) && !EVA_BAD_G(BUF_WI, up + 512, 16)) ldg_unit(up, nb0, nb1);
+                if (!units_ready) {
+                    // Bounded: a give-up is recorded; the CTA still finishes.
+                    units_ready = true;
+                    if (!mbar_wait_bounded(bar, 0, p.wait_rounds) && tid == 0 && p.status) atomicOr(p.status, 1);
                 }
+                // Units [0, nst) of the CTA (slice-major) come from shared
+                // memory; the others stream from global memory one tile ahead.
+                const int ubase = (s - s0) * ctiles;
+                uint4 nb0 = make_uint4(0u, 0u, 0u, 0u), nb1 = nb0;
+                auto fetch = [&](int tl) {
+                    if (ubase + tl < nst) {
+                        const uint32_t wo = UNITS_OFF + (uint32_t)(ubase + tl) * kUnitBytes + 16u * (uint32_t)lane;
+                        if (!EVA_BAD_S(wo) && !EVA_BAD_S(wo + 524u)) {
+                            nb0 = lds128(wo);
+                            nb1 = lds128(wo + 512u);
+                        }
+                    } else {
+                        const uint8_t *up = p.wi + ((size_t)s * p.T + t0 + tl) * kUnitBytes + 16 * lane;
+                        if (!EVA_BAD_G(BUF_WI, up, 16) && !EVA_BAD_G(BUF_WI, up + 512, 16)) ldg_unit(up, nb0, nb1);
+                    }
+                };
+                if (i0 < i1) fetch(warp + kWarps * i0);
 #pragma unroll 1
                 for (int i = i0; i < i1; ++i) {
                     const int tl = warp + kWarps * i;
                     const uint32_t wv[8] = {nb0.x, nb0.y, nb0.z, nb0.w, nb1.x, nb1.y, nb1.z, nb1.w};
-                    if (i + 1 < i1) {
-                        const uint8_t *up = p.wi + ((size_t)s * p.T + t0 + tl + kWarps) * kUnitBytes + 16 * lane;
-                        if (!EVA_BAD_G(BUF_WI, up, 16) && !EVA_BAD_G(BUF_WI, up + 512, 16)) ldg_unit(up, nb0, nb1);
-                    }
+                    if (i + 1 < i1) fetch(tl + kWarps);
                     // rot[beta] = wv[(beta - g) mod 8]: the word holding sub-vectors 4 beta + q (+32).
                     uint32_t rot[8];
 #pragma unroll
@@ -245,6 +289,8 @@ __global__ void __launch_bounds__(kThreads, 1) eva_dequant_kernel(const LookupPa
         // The next pass rewrites the x stage, the sums and the owners' stages.
         if (p0 + TT < p.B) cluster_sync_all();
     }
+    // No bulk copy may still be writing this CTA's shared memory at exit.
+    if (!units_ready && !mbar_wait_bounded(bar, 0, p.wait_rounds) && tid == 0 && p.status) atomicOr(p.status, 2);
     if (p.independent) pdl_wait();
     EVA_STAMP(6);
 #ifdef EVA_TIMELINE

@@ -623,16 +623,31 @@ __device__ __forceinline__ float lds_x(const LookupParams &p, uint32_t x_off, in
 }
 
 // B fragments of the codebook product for this warp's centroid tiles
-// nt = warp + kWarps j: lane (g, q) holds WC[cb][8 nt + g][q] as tf32.
-__device__ __forceinline__ void load_codebook_frag(const LookupParams &p, int cb, int warp, int g, int q,
-                                                   uint32_t (&bf)[4]) {
+// nt = warp + kWarps j: lane (g, q) holds WC[cb][8 nt + g][q] as tf32.  The
+// raw fp16 bits are loaded first (load_codebook_raw) and converted when
+// used (frag_from_raw), so a later pass's codebook can be in flight while
+// the current one is used.
+__device__ __forceinline__ void load_codebook_raw(const LookupParams &p, int cb, int warp, int g, int q,
+                                                  uint32_t (&raw)[4]) {
     const __half *wcb = p.wc + (size_t)cb * p.ncent * kD;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const int c = 8 * (warp + kWarps * j) + g;
         const __half *wp = wcb + c * kD + q;
-        bf[j] = to_tf32((c >= p.ncent || EVA_BAD_G(BUF_WC, wp, 2)) ? 0.f : __half2float(__ldg(wp)));
+        raw[j] = (c >= p.ncent || EVA_BAD_G(BUF_WC, wp, 2))
+                     ? 0u
+                     : (uint32_t)__ldg(reinterpret_cast<const unsigned short *>(wp));
     }
+}
+__device__ __forceinline__ void frag_from_raw(const uint32_t (&raw)[4], uint32_t (&bf)[4]) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) bf[j] = to_tf32(__half2float(__ushort_as_half((unsigned short)raw[j])));
+}
+__device__ __forceinline__ void load_codebook_frag(const LookupParams &p, int cb, int warp, int g, int q,
+                                                   uint32_t (&bf)[4]) {
+    uint32_t raw[4];
+    load_codebook_raw(p, cb, warp, g, q, raw);
+    frag_from_raw(raw, bf);
 }
 
 // --------------------------------------------------- output-codebook build
@@ -911,6 +926,14 @@ __device__ __forceinline__ void lookup_body(const LookupParams &p, const int eva
     uint32_t bfrag[4];
     int cur_cb = cb_first;   // codebook whose fragments bfrag holds
     load_codebook_frag(p, cb_first, warp, g, q, bfrag);
+    // Per-group codebooks: the raw fragments of the codebook the next pass
+    // uses are loaded one pass ahead (the load then overlaps a whole pass).
+    uint32_t bnext[4] = {0u, 0u, 0u, 0u};
+    int next_cb = -1;
+    if (GROUPED && cb_last > cb_first) {
+        next_cb = cb_first + 1;
+        load_codebook_raw(p, next_cb, warp, g, q, bnext);
+    }
 
     // Routing matrices of the accumulating MMA (B operand, 16 x 8, 0/1).
     // One token: column 0 sums the low half of a0/a1 and the high half of
@@ -962,8 +985,15 @@ __device__ __forceinline__ void lookup_body(const LookupParams &p, const int eva
                     i0 = max(0, (lo - t0 - warp + kWarps - 1) / kWarps);
                     i1 = min(ntw, max(0, (hi - t0 - warp + kWarps - 1) / kWarps));
                     if (cb != cur_cb) {
-                        load_codebook_frag(p, cb, warp, g, q, bfrag);
+                        if (cb == next_cb) frag_from_raw(bnext, bfrag);
+                        else load_codebook_frag(p, cb, warp, g, q, bfrag);
                         cur_cb = cb;
+                        // the codebook of the pass after this one
+                        const int nxt = cb < cb_last ? cb + 1 : ((s + 1 < s1 || pr + 1 < npairs) ? cb_first : -1);
+                        if (nxt >= 0 && nxt != cb) {
+                            next_cb = nxt;
+                            load_codebook_raw(p, nxt, warp, g, q, bnext);
+                        }
                     }
                 }
                 // Tiles [i0, i_st) of the first slice read their indices from the
@@ -1161,18 +1191,30 @@ __device__ __forceinline__ void lookup_body(const LookupParams &p, const int eva
         cluster_sync_all();
         EVA_STAMP(5);
         {
+            // Four consecutive threads per output each add every fourth source
+            // (k = part, part + 4, ...), then two shuffles combine them: a
+            // fixed order, so y repeats bitwise.  The loop bound is the same
+            // for every thread (every lane takes part in the shuffles).
+            constexpr int SPL = 4;
             const int my_tiles = (ctiles - ts + p.Gs - 1) / p.Gs;   // tiles tl = ts + Gs * slot
-            for (int idx = tid; idx < my_tiles * kTileRows * NTOK; idx += kThreads) {
+            const int nout = my_tiles * kTileRows * NTOK;
+            for (int base = 0; base < nout * SPL; base += kThreads) {
+                const int idx = (base + tid) / SPL, part = (base + tid) % SPL;
                 const int e = idx % NTOK, row = (idx / NTOK) % kTileRows, slot = idx / (NTOK * kTileRows);
                 const int tl = ts + p.Gs * slot;
                 const int tok = PAIR_T ? 2 * pr + e : 0;
                 const int o = kTileRows * (t0 + tl) + row;
-                if (tok >= p.B || o >= p.N) continue;
+                const bool valid = idx < nout && tok < p.B && o < p.N;
                 float sum = 0.f;
-                for (int k = 0; k < p.Gs; ++k) {
-                    const uint32_t si = (uint32_t)(((slot * p.Gs + k) * kTileRows + row) * 2 + e);
-                    sum += EVA_BAD_S(STAGE_OFF + 4u * si) ? 0.f : stage[si];
+                if (valid) {
+                    for (int k = part; k < p.Gs; k += SPL) {
+                        const uint32_t si = (uint32_t)(((slot * p.Gs + k) * kTileRows + row) * 2 + e);
+                        sum += EVA_BAD_S(STAGE_OFF + 4u * si) ? 0.f : stage[si];
+                    }
                 }
+                sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+                sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+                if (!valid || part != 0) continue;
                 const size_t yi = (size_t)tok * p.N + o;
                 if (p.out_f32) {
                     float *yp = reinterpret_cast<float *>(p.y) + yi;

@@ -215,6 +215,31 @@ def test_both_paths_match_the_oracle(key, li, B):
         assert np.all(err <= TOL), (path, err.max())
 
 
+@pytest.mark.parametrize("N,K,cbr,B", [(8192, 8192, 128, 20), (4096, 4096, 0, 24), (8192, 8192, 128, 1),
+                                       (2064, 8192, 16, 9)])
+def test_dequant_path_large_layers(N, K, cbr, B):
+    """Layers whose index units do not all fit in shared memory next to the
+    rest of the dequantize kernel's footprint: the units past the staged ones
+    stream from global memory.  Two passes of 16 tokens, one token, and a
+    ragged row count with 16-row codebooks: every row against the oracle, and
+    a second call bitwise equal."""
+    import torch
+    from vector_quantized_weight_b200 import eva_vq
+    shape = synth.LayerShape("ring", N, K, codebook_rows=cbr)
+    layer = synth.make_layer(shape, 900 + B)
+    x = synth.make_x(K, B, 901 + B)
+    lin = eva_vq.from_layer(layer, max_batch=B, path=eva_vq.EVA_PATH_DEQUANT_MMA)
+    y = lin(torch.from_numpy(x).cuda())
+    again = lin(torch.from_numpy(x).cuda())
+    torch.cuda.synchronize()
+    assert lin.info().path == eva_vq.EVA_PATH_DEQUANT_MMA
+    assert eva_vq.eva_vq_sync_status(lin.handle) == eva_vq.EVA_OK
+    assert torch.equal(y, again)
+    lin.close()
+    err = norm_rel_err(y.float().cpu().numpy(), oracle.layer_linear(layer, x, nthreads=NTHREADS))
+    assert np.all(err <= TOL), err.max()
+
+
 def test_dequant_path_rejects_residual_layers():
     from vector_quantized_weight_b200 import eva_vq
     shape = synth.LayerShape("r", 64, 512, residual_group=128)

@@ -285,7 +285,12 @@ eva_vq_linear::Plan latency_plan(const eva_vq_linear *h, int pair_t) {
                                          (size_t)120 * 1024);
         const int clusters = max_active_clusters(fn, smem_one, gs);
         // One CTA of this layer per SM: no more clusters than P / gs either.
-        const int gt_max = std::min({T, clusters, P / gs});
+        // With per-group codebooks the image builds dominate and two CTAs of
+        // the layer per SM interleave them (measured, Llama-2-70B 8192^2 at
+        // one token: 24.1 us on 16 x 7, 21.3 on 16 x 13), at the cost of the
+        // next layer's early prologue.
+        const int per_sm = h->tiles_per_cb ? 2 : 1;
+        const int gt_max = std::min({T, per_sm * clusters, per_sm * (P / gs)});
         for (int gt = gt_min; gt <= gt_max; ++gt) {
             const int tiles = (T + gt - 1) / gt, slices = (S + gs - 1) / gs;
             int builds = 1;
@@ -374,9 +379,14 @@ cudaError_t launch_pdl(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_
 
 
 using DequantFn = void (*)(LookupParams);
-DequantFn dequant_fn(bool grouped, int ntg) {
-    if (grouped) return ntg == 2 ? eva_dequant_kernel<true, 2> : eva_dequant_kernel<true, 1>;
-    return ntg == 2 ? eva_dequant_kernel<false, 2> : eva_dequant_kernel<false, 1>;
+// `direct`: every CTA takes one K-slice (Gs = S), see eva_dequant_kernel.
+DequantFn dequant_fn(bool grouped, int ntg, bool direct) {
+    if (direct) {
+        if (grouped) return ntg == 2 ? eva_dequant_kernel<true, 2, true> : eva_dequant_kernel<true, 1, true>;
+        return ntg == 2 ? eva_dequant_kernel<false, 2, true> : eva_dequant_kernel<false, 1, true>;
+    }
+    if (grouped) return ntg == 2 ? eva_dequant_kernel<true, 2, false> : eva_dequant_kernel<true, 1, false>;
+    return ntg == 2 ? eva_dequant_kernel<false, 2, false> : eva_dequant_kernel<false, 1, false>;
 }
 
 // Calls with at least this many tokens take the dequantize path (when the
@@ -390,7 +400,9 @@ size_t dequant_smem(int nsl, int tiles, int gs, int ntg, int staged = 0) {
     const size_t blk = (size_t)kTileRows * 8 * ntg * 4;
     const size_t xs = ((size_t)nsl * 8 * ntg * kXTokStride + 127) & ~(size_t)127;
     const size_t nslot = (size_t)(tiles + gs - 1) / gs;
-    const size_t base = (size_t)kTabBytes + xs + (size_t)tiles * blk + nslot * gs * blk;
+    // With one slice per CTA the tiles' sums go straight to the owners' stages.
+    const size_t acc = nsl == 1 ? 0 : (size_t)tiles * blk;
+    const size_t base = (size_t)kTabBytes + xs + acc + nslot * gs * blk;
     return ((base + 127) & ~(size_t)127) + 128 + (size_t)staged * kUnitBytes;
 }
 
@@ -398,12 +410,12 @@ size_t dequant_smem(int nsl, int tiles, int gs, int ntg, int staged = 0) {
 // cluster in one wave when the shared memory allows it).
 void plan_dequant(eva_vq_linear *h, int ntg) {
     const int S = h->S, T = h->T, P = h->sm_count;
-    const DequantFn fn = dequant_fn(h->tiles_per_cb != 0, ntg);
     double best = 1e300;
     eva_vq_linear::Plan pl;
     pl.Gs = 0;
     for (int gs = 1; gs <= std::min(S, 16); ++gs) {
         const int nsl = (S + gs - 1) / gs;
+        const DequantFn fn = dequant_fn(h->tiles_per_cb != 0, ntg, nsl == 1);
         const int gt_min = (T + kMaxCtaTiles - 1) / kMaxCtaTiles;
         const int clusters = max_active_clusters((LookupFn)fn, (size_t)h->smem_optin, gs);
         const int gt_max = std::min({T, std::max(clusters, gt_min), std::max(P / gs, gt_min)});
@@ -440,8 +452,8 @@ void plan_dequant(eva_vq_linear *h, int ntg) {
 
 cudaError_t set_smem_attrs(int smem_optin) {
     cudaError_t e;
-    for (int v = 0; v < 4; ++v) {
-        const DequantFn fn = dequant_fn(v & 1, 1 + (v >> 1));
+    for (int v = 0; v < 8; ++v) {
+        const DequantFn fn = dequant_fn(v & 1, 1 + ((v >> 1) & 1), (v >> 2) & 1);
         e = cudaFuncSetAttribute((const void *)fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute((const void *)fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_optin);
@@ -512,8 +524,9 @@ cudaError_t launch_dequant(eva_vq_linear *h, LookupParams p, int B, cudaStream_t
 #ifdef EVA_DEVICE_CHECKS
     p.smem_bytes = (unsigned)pl.smem;
 #endif
-    return launch_pdl(dequant_fn(h->tiles_per_cb != 0, ntg), dim3(pl.Gs * pl.Gt), dim3(kThreads), pl.smem, s,
-                      pl.Gs, p);
+    const bool direct = (h->S + pl.Gs - 1) / pl.Gs == 1;   // the same rule as dequant_smem's
+    return launch_pdl(dequant_fn(h->tiles_per_cb != 0, ntg, direct), dim3(pl.Gs * pl.Gt), dim3(kThreads), pl.smem,
+                      s, pl.Gs, p);
 }
 
 bool use_three_per_sm(const eva_vq_linear *h, int B, int independent) {

@@ -45,8 +45,13 @@ __device__ __forceinline__ void build_codebook_table(const LookupParams &p, int 
     }
 }
 
-template <bool GROUPED, int NTG>
-__global__ void __launch_bounds__(kThreads, 1) eva_dequant_kernel(const LookupParams p) {
+// DIRECT: launched only when every CTA takes one K-slice (Gs = S), so a
+// tile's sums are final when its MMAs end and go straight from registers to
+// the owning cluster CTA's stage (no running sums in shared memory).
+// Two CTAs per SM where the registers allow it without spills (at most 128
+// a thread): then the next layer's CTA runs its prologue beside this one.
+template <bool GROUPED, int NTG, bool DIRECT>
+__global__ void __launch_bounds__(kThreads, (GROUPED && NTG == 2) ? 1 : 2) eva_dequant_kernel(const LookupParams p) {
     constexpr int TT = 8 * NTG;                         // tokens per pass
     constexpr uint32_t BLK = kTileRows * TT * 4u;       // bytes of one tile's sums
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -61,16 +66,17 @@ __global__ void __launch_bounds__(kThreads, 1) eva_dequant_kernel(const LookupPa
     const int cb_last = GROUPED ? (t1 - 1) / p.tiles_per_cb : 0;
 
     // Shared memory: codebook table | x stage [slice][token] | running sums
-    // [tile][16][TT] | reduction stage [ceil(acc_tiles / Gs)][Gs][16][TT] |
-    // the staging mbarrier (128 bytes) | the staged index units (slice-major:
-    // unit sl * ctiles + tl).
+    // [tile][16][TT] (only when a CTA takes several slices) | reduction stage
+    // [ceil(acc_tiles / Gs)][Gs][16][TT] | the staging mbarrier (128 bytes) |
+    // the staged index units (slice-major: unit sl * ctiles + tl).
     constexpr uint32_t TAB_OFF = 0, XS_OFF = kTabBytes;
     // The layout must be the same in every CTA of a cluster (peers write into
     // the reduction stage at this CTA's offsets): size the x stage for the
     // largest slice count, ceil(S / Gs).
     const int nsl_max = (p.S + p.Gs - 1) / p.Gs;
+    constexpr bool direct = DIRECT;
     const uint32_t ACC_OFF = (XS_OFF + (uint32_t)(nsl_max * TT) * kXTokStride + 127u) & ~127u;
-    const uint32_t STAGE_OFF = ACC_OFF + (uint32_t)p.acc_tiles * BLK;
+    const uint32_t STAGE_OFF = ACC_OFF + (direct ? 0u : (uint32_t)p.acc_tiles * BLK);
     float *acc_s = reinterpret_cast<float *>(eva_smem + ACC_OFF);
     const float *stage = reinterpret_cast<const float *>(eva_smem + STAGE_OFF);
     const uint32_t stage_addr = (uint32_t)__cvta_generic_to_shared(eva_smem + STAGE_OFF);
@@ -209,6 +215,10 @@ __global__ void __launch_bounds__(kThreads, 1) eva_dequant_kernel(const LookupPa
 #pragma unroll
                         for (int k = 0; k < 8; ++k) rot[k] = nr[k];
                     }
+                    // Two MMA accumulation chains per token group, one where the
+                    // registers of two CTAs per SM would not hold two (16 tokens,
+                    // sums pushed from registers).
+                    constexpr int kChains = (NTG == 2 && DIRECT) ? 1 : 2;
                     float acc[NTG][2][4];
 #pragma unroll
                     for (int t = 0; t < NTG; ++t)
@@ -226,18 +236,34 @@ __global__ void __launch_bounds__(kThreads, 1) eva_dequant_kernel(const LookupPa
                         const uint2 ah = EVA_BAD_S(oh) ? make_uint2(0u, 0u) : lds64(oh);
 #pragma unroll
                         for (int t = 0; t < NTG; ++t)
-                            mma_f16_k16(acc[t][beta & 1], ag.x, ah.x, ag.y, ah.y, xb[t][beta].x, xb[t][beta].y);
+                            mma_f16_k16(acc[t][kChains == 1 ? 0 : (beta & 1)], ag.x, ah.x, ag.y, ah.y, xb[t][beta].x, xb[t][beta].y);
                     }
                     // D: (row g, tokens 2q, 2q+1), (row g+8, tokens 2q, 2q+1) of each token group.
+                    if (direct) {
+                        // Into block ts of slot tl / Gs of the owner's (rank tl % Gs) stage.
+                        const uint32_t off = (uint32_t)((tl / p.Gs) * p.Gs + ts) * BLK + 4u * (uint32_t)(g * TT + 2 * q);
+                        const uint32_t ra = dsmem_map(stage_addr + off, (uint32_t)(tl % p.Gs));
 #pragma unroll
-                    for (int t = 0; t < NTG; ++t)
+                        for (int t = 0; t < NTG; ++t)
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int row = g + 8 * (e >> 1), tok = 8 * t + 2 * q + (e & 1);
-                            const int ai = (tl * kTileRows + row) * TT + tok;
-                            const float v = acc[t][0][e] + acc[t][1][e];
-                            if (!EVA_BAD_S(ACC_OFF + 4u * (uint32_t)ai)) acc_s[ai] = (s == s0) ? v : acc_s[ai] + v;
-                        }
+                            for (int h = 0; h < 2; ++h) {
+                                const uint32_t o = 4u * (uint32_t)(8 * h * TT + 8 * t);
+                                if (!EVA_BAD_S(STAGE_OFF + off + o) && !EVA_BAD_S(STAGE_OFF + off + o + 4u))
+                                    st_dsmem_v2(ra + o, acc[t][0][2 * h] + acc[t][1][2 * h],
+                                                acc[t][0][2 * h + 1] + acc[t][1][2 * h + 1]);
+                            }
+                    } else {
+#pragma unroll
+                        for (int t = 0; t < NTG; ++t)
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int row = g + 8 * (e >> 1), tok = 8 * t + 2 * q + (e & 1);
+                                const int ai = (tl * kTileRows + row) * TT + tok;
+                                const float v = acc[t][0][e] + acc[t][1][e];
+                                if (!EVA_BAD_S(ACC_OFF + 4u * (uint32_t)ai))
+                                    acc_s[ai] = (s == s0) ? v : acc_s[ai] + v;
+                            }
+                    }
                 }
             }
         }
@@ -248,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1) eva_dequant_kernel(const LookupPa
         EVA_STAMP(4);
         __syncthreads();
         constexpr int CH = (int)(BLK / 16u);               // 16-byte chunks per tile block
-        for (int i = tid; i < ctiles * CH; i += kThreads) {
+        for (int i = tid; !direct && i < ctiles * CH; i += kThreads) {
             const int tl = i / CH, chunk = i % CH;
             const uint32_t src = ACC_OFF + (uint32_t)tl * BLK + 16u * (uint32_t)chunk;
             const uint32_t dst = (uint32_t)((tl / p.Gs) * p.Gs + ts) * BLK + 16u * (uint32_t)chunk;

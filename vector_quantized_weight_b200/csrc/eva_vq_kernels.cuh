@@ -221,6 +221,17 @@ __device__ __forceinline__ void st_dsmem_v4(uint32_t local_addr, uint32_t rank, 
                  : "memory");
 }
 
+// The address of this CTA's shared-memory location `local_addr` in cluster
+// CTA `rank`, and an 8-byte store there.
+__device__ __forceinline__ uint32_t dsmem_map(uint32_t local_addr, uint32_t rank) {
+    uint32_t ra;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(local_addr), "r"(rank));
+    return ra;
+}
+__device__ __forceinline__ void st_dsmem_v2(uint32_t remote_addr, float x, float y) {
+    asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(remote_addr), "f"(x), "f"(y) : "memory");
+}
+
 __device__ __forceinline__ uint32_t to_tf32(float f) {
     uint32_t r;
     asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(f));

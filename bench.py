@@ -589,7 +589,8 @@ def main():
         "roofline": {"bound": "hbm", "achieved": round(achieved, 3), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": load_traffic(workload),
                      "peak_kind": peak_kind,
-                     "kernel": "eva_dequant_kernel" if info.path == eva_vq.EVA_PATH_DEQUANT_MMA else "eva_lookup_kernel",
+                     "kernel": {eva_vq.EVA_PATH_DEQUANT_MMA: "eva_dequant_kernel",
+                                eva_vq.EVA_PATH_TCGEN05: "eva_tc_kernel"}.get(info.path, "eva_lookup_kernel"),
                      "algorithmic_bytes_per_launch": sb},
         "gpu_launches": steps * info.kernels_per_run,
         "clocks": clk.summary(),

@@ -540,9 +540,11 @@ bool use_three_per_sm(const eva_vq_linear *h, int B, int independent) {
 // AUTO (measured per batch on B200, one layer waiting for the previous one):
 //  - layers the warp-level dequantize path takes (no residual, no rotation):
 //    that path from kDequantMinBatch tokens on, except one shared codebook
-//    from kTcMinBatch tokens on, where tcgen05 wins (4096 x 4096: 19.0 against
-//    22.3 us at 32 tokens, 25.4 against 40.2 at 64; with per-group codebooks
-//    the warp-level path stays ahead, 57.8 against 70.9 us at 32 tokens);
+//    past two 16-token passes (kTcMinBatch), where tcgen05 wins (4096 x 4096:
+//    16.3 against 17.0 us at 32 tokens, 19.1 against 24.2 at 48, 21.3 against
+//    32.0 at 64; 11008 x 4096: 35.0 against 49.0 at 32, 62.0 against 65.1 at
+//    64); with per-group codebooks the warp-level path stays ahead (8192 x
+//    8192: 62.3 against 85.2 us at 32 tokens);
 //  - residual / rotated layers: the lookup path below kTcResidMinBatch tokens
 //    (3.125-bit 3584 x 3584: 15.4 against 22.0 us at 4 tokens), tcgen05 from
 //    there (24.7 against 55.5 us at 16).
@@ -550,7 +552,7 @@ bool use_three_per_sm(const eva_vq_linear *h, int B, int independent) {
 // N = 64 (about 100 cycles per instruction, measured), so the tensor-core
 // path pays off as the batch grows, while the warp-level MMA of 8 tokens
 // scales with the batch.
-constexpr int kTcMinBatch = 32;
+constexpr int kTcMinBatch = 33;
 constexpr int kTcResidMinBatch = 8;
 
 bool use_tc(const eva_vq_linear *h, int B) {

@@ -400,9 +400,11 @@ size_t dequant_smem(int nsl, int tiles, int gs, int ntg, int staged = 0) {
     const size_t blk = (size_t)kTileRows * 8 * ntg * 4;
     const size_t xs = ((size_t)nsl * 8 * ntg * kXTokStride + 127) & ~(size_t)127;
     const size_t nslot = (size_t)(tiles + gs - 1) / gs;
-    // With one slice per CTA the tiles' sums go straight to the owners' stages.
+    // With one slice per CTA the tiles' sums go straight to the owners'
+    // stages, whose rows are then padded by two floats.
     const size_t acc = nsl == 1 ? 0 : (size_t)tiles * blk;
-    const size_t base = (size_t)kTabBytes + xs + acc + nslot * gs * blk;
+    const size_t blk_s = nsl == 1 ? (size_t)kTileRows * (8 * ntg + 2) * 4 : blk;
+    const size_t base = (size_t)kTabBytes + xs + acc + nslot * gs * blk_s;
     return ((base + 127) & ~(size_t)127) + 128 + (size_t)staged * kUnitBytes;
 }
 

@@ -53,7 +53,13 @@ __device__ __forceinline__ void build_codebook_table(const LookupParams &p, int 
 template <bool GROUPED, int NTG, bool DIRECT>
 __global__ void __launch_bounds__(kThreads, (GROUPED && NTG == 2) ? 1 : 2) eva_dequant_kernel(const LookupParams p) {
     constexpr int TT = 8 * NTG;                         // tokens per pass
-    constexpr uint32_t BLK = kTileRows * TT * 4u;       // bytes of one tile's sums
+    constexpr uint32_t BLK = kTileRows * TT * 4u;       // bytes of one tile's running sums
+    // A tile's block in the reduction stage.  Sums pushed from registers (8
+    // bytes a lane): rows TT + 2 floats apart, so the owners' reads (row
+    // fastest, for coalesced y stores) hit distinct banks; running-sum blocks
+    // copied 16 bytes at a time: rows TT floats apart, like the running sums.
+    constexpr int RS = DIRECT ? TT + 2 : TT;
+    constexpr uint32_t BLK_S = kTileRows * RS * 4u;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, q = lane & 3;
     const int eva_bid = blockIdx.x;
@@ -80,7 +86,7 @@ __global__ void __launch_bounds__(kThreads, (GROUPED && NTG == 2) ? 1 : 2) eva_d
     float *acc_s = reinterpret_cast<float *>(eva_smem + ACC_OFF);
     const float *stage = reinterpret_cast<const float *>(eva_smem + STAGE_OFF);
     const uint32_t stage_addr = (uint32_t)__cvta_generic_to_shared(eva_smem + STAGE_OFF);
-    const uint32_t BAR_OFF = (STAGE_OFF + (uint32_t)((p.acc_tiles + p.Gs - 1) / p.Gs) * p.Gs * BLK + 127u) & ~127u;
+    const uint32_t BAR_OFF = (STAGE_OFF + (uint32_t)((p.acc_tiles + p.Gs - 1) / p.Gs) * p.Gs * BLK_S + 127u) & ~127u;
     const uint32_t UNITS_OFF = BAR_OFF + 128u;
     const int nst = min(nsl * ctiles, p.wi_staged);   // units copied into shared memory
     const uint32_t bar = (uint32_t)__cvta_generic_to_shared(eva_smem + BAR_OFF);
@@ -241,13 +247,13 @@ __global__ void __launch_bounds__(kThreads, (GROUPED && NTG == 2) ? 1 : 2) eva_d
                     // D: (row g, tokens 2q, 2q+1), (row g+8, tokens 2q, 2q+1) of each token group.
                     if (direct) {
                         // Into block ts of slot tl / Gs of the owner's (rank tl % Gs) stage.
-                        const uint32_t off = (uint32_t)((tl / p.Gs) * p.Gs + ts) * BLK + 4u * (uint32_t)(g * TT + 2 * q);
+                        const uint32_t off = (uint32_t)((tl / p.Gs) * p.Gs + ts) * BLK_S + 4u * (uint32_t)(g * RS + 2 * q);
                         const uint32_t ra = dsmem_map(stage_addr + off, (uint32_t)(tl % p.Gs));
 #pragma unroll
                         for (int t = 0; t < NTG; ++t)
 #pragma unroll
                             for (int h = 0; h < 2; ++h) {
-                                const uint32_t o = 4u * (uint32_t)(8 * h * TT + 8 * t);
+                                const uint32_t o = 4u * (uint32_t)(8 * h * RS + 8 * t);
                                 if (!EVA_BAD_S(STAGE_OFF + off + o) && !EVA_BAD_S(STAGE_OFF + off + o + 4u))
                                     st_dsmem_v2(ra + o, acc[t][0][2 * h] + acc[t][1][2 * h],
                                                 acc[t][0][2 * h + 1] + acc[t][1][2 * h + 1]);
@@ -269,15 +275,17 @@ __global__ void __launch_bounds__(kThreads, (GROUPED && NTG == 2) ? 1 : 2) eva_d
         }
 
         // Split-K sums of this pass: push each tile's block to the owning
-        // cluster CTA (rank tl % Gs) with 16-byte remote stores, cluster
-        // barrier, owners add the Gs blocks in rank order and store y.
+        // cluster CTA (rank tl % Gs) with 16-byte remote stores (the direct
+        // kernel pushed them from the tile loop), cluster barrier, owners add
+        // the Gs blocks in rank order and store y.
         EVA_STAMP(4);
         __syncthreads();
+        static_assert(DIRECT || BLK_S == BLK, "running-sum blocks are copied as they are");
         constexpr int CH = (int)(BLK / 16u);               // 16-byte chunks per tile block
         for (int i = tid; !direct && i < ctiles * CH; i += kThreads) {
             const int tl = i / CH, chunk = i % CH;
             const uint32_t src = ACC_OFF + (uint32_t)tl * BLK + 16u * (uint32_t)chunk;
-            const uint32_t dst = (uint32_t)((tl / p.Gs) * p.Gs + ts) * BLK + 16u * (uint32_t)chunk;
+            const uint32_t dst = (uint32_t)((tl / p.Gs) * p.Gs + ts) * BLK_S + 16u * (uint32_t)chunk;
             if (!EVA_BAD_S(src) && !EVA_BAD_S(src + 12u) && !EVA_BAD_S(STAGE_OFF + dst) && !EVA_BAD_S(STAGE_OFF + dst + 12u)) {
                 const float4 v = *reinterpret_cast<const float4 *>(eva_smem + src);
                 st_dsmem_v4(stage_addr + dst, (uint32_t)(tl % p.Gs), v);
@@ -287,15 +295,16 @@ __global__ void __launch_bounds__(kThreads, (GROUPED && NTG == 2) ? 1 : 2) eva_d
         EVA_STAMP(5);
         {
             const int my_tiles = (ctiles - ts + p.Gs - 1) / p.Gs;
-            for (int idx = tid; idx < my_tiles * kTileRows * TT; idx += kThreads) {
-                const int row = idx % kTileRows, tok = (idx / kTileRows) % TT, slot = idx / (kTileRows * TT);
+            const int nb = min(TT, p.B - p0);               // tokens of this pass
+            for (int idx = tid; idx < my_tiles * kTileRows * nb; idx += kThreads) {
+                const int row = idx % kTileRows, tok = (idx / kTileRows) % nb, slot = idx / (kTileRows * nb);
                 const int tl = ts + p.Gs * slot;
                 const int o = kTileRows * (t0 + tl) + row, b = p0 + tok;
-                if (b >= p.B || o >= p.N) continue;
+                if (o >= p.N) continue;
                 float v[16];
 #pragma unroll
                 for (int k = 0; k < 16; ++k) {
-                    const uint32_t si = (uint32_t)((((slot * p.Gs + k) * kTileRows + row) * TT) + tok);
+                    const uint32_t si = (uint32_t)((((slot * p.Gs + k) * kTileRows + row) * RS) + tok);
                     v[k] = (k < p.Gs && !EVA_BAD_S(STAGE_OFF + 4u * si)) ? stage[si] : 0.f;
                 }
                 float sum = 0.f;

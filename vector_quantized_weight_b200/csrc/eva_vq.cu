@@ -436,7 +436,10 @@ void plan_dequant(eva_vq_linear *h, int ntg) {
             }
         }
     }
-    if (pl.Gs == 0) return;   // nothing fits: the lookup path serves every batch
+    if (pl.Gs == 0) {   // nothing fits: the lookup path serves every batch
+        h->dq[ntg - 1] = pl;
+        return;
+    }
     const int tiles = (T + pl.Gt - 1) / pl.Gt, nsl = (S + pl.Gs - 1) / pl.Gs;
     // Index units copied into shared memory in the prologue: as many of the
     // CTA's units as fit while the CTA still leaves half the SM to the next

@@ -50,8 +50,11 @@ __device__ __forceinline__ void build_codebook_table(const LookupParams &p, int 
 // the owning cluster CTA's stage (no running sums in shared memory).
 // Two CTAs per SM where the registers allow it without spills (at most 128
 // a thread): then the next layer's CTA runs its prologue beside this one.
+// The 16-token instances with running sums in shared memory take more than
+// half the SM's shared memory anyway, so they keep one CTA per SM and the
+// registers that go with it.
 template <bool GROUPED, int NTG, bool DIRECT>
-__global__ void __launch_bounds__(kThreads, (GROUPED && NTG == 2) ? 1 : 2) eva_dequant_kernel(const LookupParams p) {
+__global__ void __launch_bounds__(kThreads, (NTG == 2 && (GROUPED || !DIRECT)) ? 1 : 2) eva_dequant_kernel(const LookupParams p) {
     constexpr int TT = 8 * NTG;                         // tokens per pass
     constexpr uint32_t BLK = kTileRows * TT * 4u;       // bytes of one tile's running sums
     // A tile's block in the reduction stage.  Sums pushed from registers (8
@@ -158,12 +161,37 @@ __global__ void __launch_bounds__(kThreads, (GROUPED && NTG == 2) ? 1 : 2) eva_d
         __syncthreads();
         EVA_STAMP(2);
 
-        for (int cb = cb_first; cb <= cb_last; ++cb) {
-            int i0 = 0, i1 = ntw;
+        // This warp's tiles of codebook cb: warp + kWarps i for i in [i0, i1).
+        auto cb_tiles = [&](int cb, int &i0, int &i1) {
+            i0 = 0;
+            i1 = ntw;
             if (GROUPED) {
                 const int lo = max(cb * p.tiles_per_cb, t0), hi = (cb + 1) * p.tiles_per_cb;
                 i0 = max(0, (lo - t0 - warp + kWarps - 1) / kWarps);
                 i1 = min(ntw, max(0, (hi - t0 - warp + kWarps - 1) / kWarps));
+            }
+        };
+        // Units [0, nst) of the CTA (slice-major) come from shared memory; the
+        // others stream from global memory one unit ahead (nb0, nb1).
+        uint4 nb0 = make_uint4(0u, 0u, 0u, 0u), nb1 = nb0;
+        bool have_next = false;   // nb0, nb1 already hold the next (codebook, slice)'s first unit
+        auto fetch = [&](int s, int tl) {
+            const int u = (s - s0) * ctiles + tl;
+            if (u < nst) {
+                const uint32_t wo = UNITS_OFF + (uint32_t)u * kUnitBytes + 16u * (uint32_t)lane;
+                if (!EVA_BAD_S(wo) && !EVA_BAD_S(wo + 524u)) {
+                    nb0 = lds128(wo);
+                    nb1 = lds128(wo + 512u);
+                }
+            } else {
+                const uint8_t *up = p.wi + ((size_t)s * p.T + t0 + tl) * kUnitBytes + 16 * lane;
+                if (!EVA_BAD_G(BUF_WI, up, 16) && !EVA_BAD_G(BUF_WI, up + 512, 16)) ldg_unit(up, nb0, nb1);
+            }
+        };
+        for (int cb = cb_first; cb <= cb_last; ++cb) {
+            int i0, i1;
+            cb_tiles(cb, i0, i1);
+            if (GROUPED) {
                 if (cb != built_cb) {
                     __syncthreads();               // every warp is done with the previous table
                     build_codebook_table(p, cb, tid);
@@ -187,28 +215,30 @@ __global__ void __launch_bounds__(kThreads, (GROUPED && NTG == 2) ? 1 : 2) eva_d
                     units_ready = true;
                     if (!mbar_wait_bounded(bar, 0, p.wait_rounds) && tid == 0 && p.status) atomicOr(p.status, 1);
                 }
-                // Units [0, nst) of the CTA (slice-major) come from shared
-                // memory; the others stream from global memory one tile ahead.
-                const int ubase = (s - s0) * ctiles;
-                uint4 nb0 = make_uint4(0u, 0u, 0u, 0u), nb1 = nb0;
-                auto fetch = [&](int tl) {
-                    if (ubase + tl < nst) {
-                        const uint32_t wo = UNITS_OFF + (uint32_t)(ubase + tl) * kUnitBytes + 16u * (uint32_t)lane;
-                        if (!EVA_BAD_S(wo) && !EVA_BAD_S(wo + 524u)) {
-                            nb0 = lds128(wo);
-                            nb1 = lds128(wo + 512u);
-                        }
-                    } else {
-                        const uint8_t *up = p.wi + ((size_t)s * p.T + t0 + tl) * kUnitBytes + 16 * lane;
-                        if (!EVA_BAD_G(BUF_WI, up, 16) && !EVA_BAD_G(BUF_WI, up + 512, 16)) ldg_unit(up, nb0, nb1);
-                    }
-                };
-                if (i0 < i1) fetch(warp + kWarps * i0);
+                if (i0 < i1 && !have_next) fetch(s, warp + kWarps * i0);
+                have_next = false;
 #pragma unroll 1
                 for (int i = i0; i < i1; ++i) {
                     const int tl = warp + kWarps * i;
                     const uint32_t wv[8] = {nb0.x, nb0.y, nb0.z, nb0.w, nb1.x, nb1.y, nb1.z, nb1.w};
-                    if (i + 1 < i1) fetch(tl + kWarps);
+                    // One unit ahead, across slices and codebooks too: with
+                    // per-group codebooks a warp often has one tile per
+                    // (codebook, slice), and its next unit is then in the next one.
+                    if (i + 1 < i1) {
+                        fetch(s, tl + kWarps);
+                    } else if (DIRECT && !GROUPED) {
+                        // one slice, one codebook: nothing further ahead
+                    } else if (s + 1 < s1) {
+                        fetch(s + 1, warp + kWarps * i0);
+                        have_next = true;
+                    } else if (GROUPED && cb < cb_last) {
+                        int n0, n1;
+                        cb_tiles(cb + 1, n0, n1);
+                        if (n0 < n1) {
+                            fetch(s0, warp + kWarps * n0);
+                            have_next = true;
+                        }
+                    }
                     // rot[beta] = wv[(beta - g) mod 8]: the word holding sub-vectors 4 beta + q (+32).
                     uint32_t rot[8];
 #pragma unroll

@@ -447,11 +447,18 @@ void plan_dequant(eva_vq_linear *h, int ntg) {
     // none when the rest of the footprint already takes more than half
     // (measured: staging past that point costs the overlap, 6.1 -> 11.4 us
     // for 4096^2 at 4 tokens).
+    // With per-group codebooks the tile loop, not the prologue, sets the
+    // layer's time: the CTA takes the whole SM instead -- every unit that fits
+    // is staged, and at least half the SM's shared memory keeps a second CTA
+    // of the same layer off the SM (two on one SM stretched the slowest CTA's
+    // tile loop from 12.8 to 19.8 us for 8192^2 at one token).
     const size_t base = dequant_smem(nsl, tiles, pl.Gs, ntg);
     const size_t half = (size_t)h->smem_per_sm / 2 - (size_t)h->smem_reserved;
-    pl.staged = base < half ? (int)std::min<size_t>((size_t)nsl * tiles, (half - base) / kUnitBytes) : 0;
+    const size_t budget = h->tiles_per_cb ? (size_t)h->smem_optin : half;
+    pl.staged = base < budget ? (int)std::min<size_t>((size_t)nsl * tiles, (budget - base) / kUnitBytes) : 0;
     pl.smem = dequant_smem(nsl, tiles, pl.Gs, ntg, pl.staged);
     pl.smem_nostage = dequant_smem(nsl, tiles, pl.Gs, ntg);
+    if (h->tiles_per_cb) pl.smem = std::max(pl.smem, half + 1024);
     h->dq[ntg - 1] = pl;
 }
 

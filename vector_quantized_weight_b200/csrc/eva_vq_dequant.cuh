@@ -199,6 +199,112 @@ __global__ void __launch_bounds__(kThreads, (NTG == 2 && (GROUPED || !DIRECT)) ?
                     built_cb = cb;
                 }
             }
+            if constexpr (GROUPED) {
+                // Per-group codebooks: a warp has few tiles of a codebook (one
+                // when the codebook covers 8 tiles), so it takes each of them
+                // through all of the CTA's slices -- two slices in flight at a
+                // time where the registers allow -- and sums them in registers.
+                if (!units_ready) {
+                    // Bounded: a give-up is recorded; the CTA still finishes.
+                    units_ready = true;
+                    if (!mbar_wait_bounded(bar, 0, p.wait_rounds) && tid == 0 && p.status) atomicOr(p.status, 1);
+                }
+                auto load_unit = [&](int s, int tl, uint4 &a, uint4 &b) {
+                    const int u = (s - s0) * ctiles + tl;
+                    a = b = make_uint4(0u, 0u, 0u, 0u);
+                    if (u < nst) {
+                        const uint32_t wo = UNITS_OFF + (uint32_t)u * kUnitBytes + 16u * (uint32_t)lane;
+                        if (!EVA_BAD_S(wo) && !EVA_BAD_S(wo + 524u)) {
+                            a = lds128(wo);
+                            b = lds128(wo + 512u);
+                        }
+                    } else {
+                        const uint8_t *up = p.wi + ((size_t)s * p.T + t0 + tl) * kUnitBytes + 16 * lane;
+                        if (!EVA_BAD_G(BUF_WI, up, 16) && !EVA_BAD_G(BUF_WI, up + 512, 16)) ldg_unit(up, a, b);
+                    }
+                };
+                constexpr int kSliceUnroll = NTG == 1 ? 2 : 1;
+#pragma unroll 1
+                for (int i = i0; i < i1; ++i) {
+                    const int tl = warp + kWarps * i;
+                    float tacc[NTG][4];
+#pragma unroll
+                    for (int t = 0; t < NTG; ++t)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) tacc[t][e] = 0.f;
+#pragma unroll kSliceUnroll
+                    for (int s = s0; s < s1; ++s) {
+                        uint2 xs[NTG][16];
+#pragma unroll
+                        for (int t = 0; t < NTG; ++t)
+#pragma unroll
+                            for (int beta = 0; beta < 16; ++beta) {
+                                const uint32_t off = XS_OFF + (uint32_t)((s - s0) * TT + 8 * t + g) * kXTokStride +
+                                                     8u * (uint32_t)dq_subvec(beta, q);
+                                xs[t][beta] = EVA_BAD_S(off) ? make_uint2(0u, 0u) : lds64(off);
+                            }
+                        uint4 u0, u1;
+                        load_unit(s, tl, u0, u1);
+                        const uint32_t wv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+                        uint32_t rot[8];
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) rot[k] = wv[k];
+#pragma unroll
+                        for (int bit = 1; bit < 8; bit <<= 1) {
+                            uint32_t nr[8];
+#pragma unroll
+                            for (int k = 0; k < 8; ++k) nr[k] = (g & bit) ? rot[(k - bit) & 7] : rot[k];
+#pragma unroll
+                            for (int k = 0; k < 8; ++k) rot[k] = nr[k];
+                        }
+                        float acc[NTG][2][4];
+#pragma unroll
+                        for (int t = 0; t < NTG; ++t)
+#pragma unroll
+                            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) acc[t][h][e] = 0.f;
+#pragma unroll
+                        for (int beta = 0; beta < 16; ++beta) {
+                            const uint32_t w = rot[beta & 7];
+                            const uint32_t cg = beta < 8 ? (w & 0xFFu) : ((w >> 16) & 0xFFu);
+                            const uint32_t ch = beta < 8 ? ((w >> 8) & 0xFFu) : (w >> 24);
+                            const uint32_t og = TAB_OFF + (cg << 7) + lofs, oh = TAB_OFF + (ch << 7) + lofs;
+                            const uint2 ag = EVA_BAD_S(og) ? make_uint2(0u, 0u) : lds64(og);
+                            const uint2 ah = EVA_BAD_S(oh) ? make_uint2(0u, 0u) : lds64(oh);
+#pragma unroll
+                            for (int t = 0; t < NTG; ++t)
+                                mma_f16_k16(acc[t][beta & 1], ag.x, ah.x, ag.y, ah.y, xs[t][beta].x, xs[t][beta].y);
+                        }
+#pragma unroll
+                        for (int t = 0; t < NTG; ++t)
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) tacc[t][e] += acc[t][0][e] + acc[t][1][e];
+                    }
+                    // D: (row g, tokens 2q, 2q+1), (row g+8, tokens 2q, 2q+1) of each token group.
+                    if (direct) {
+                        const uint32_t off = (uint32_t)((tl / p.Gs) * p.Gs + ts) * BLK_S + 4u * (uint32_t)(g * RS + 2 * q);
+                        const uint32_t ra = dsmem_map(stage_addr + off, (uint32_t)(tl % p.Gs));
+#pragma unroll
+                        for (int t = 0; t < NTG; ++t)
+#pragma unroll
+                            for (int h = 0; h < 2; ++h) {
+                                const uint32_t o = 4u * (uint32_t)(8 * h * RS + 8 * t);
+                                if (!EVA_BAD_S(STAGE_OFF + off + o) && !EVA_BAD_S(STAGE_OFF + off + o + 4u))
+                                    st_dsmem_v2(ra + o, tacc[t][2 * h], tacc[t][2 * h + 1]);
+                            }
+                    } else {
+#pragma unroll
+                        for (int t = 0; t < NTG; ++t)
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int row = g + 8 * (e >> 1), tok = 8 * t + 2 * q + (e & 1);
+                                const int ai = (tl * kTileRows + row) * TT + tok;
+                                if (!EVA_BAD_S(ACC_OFF + 4u * (uint32_t)ai)) acc_s[ai] = tacc[t][e];
+                            }
+                    }
+                }
+            } else {
             for (int s = s0; s < s1; ++s) {
                 // B fragments of this slice: token 8t + g, sub-vector dq_subvec(beta, q).
                 uint2 xb[NTG][16];
@@ -301,6 +407,7 @@ __global__ void __launch_bounds__(kThreads, (NTG == 2 && (GROUPED || !DIRECT)) ?
                             }
                     }
                 }
+            }
             }
         }
 

@@ -202,8 +202,8 @@ __global__ void __launch_bounds__(kThreads, (NTG == 2 && (GROUPED || !DIRECT)) ?
             if constexpr (GROUPED) {
                 // Per-group codebooks: a warp has few tiles of a codebook (one
                 // when the codebook covers 8 tiles), so it takes each of them
-                // through all of the CTA's slices -- two slices in flight at a
-                // time where the registers allow -- and sums them in registers.
+                // through all of the CTA's slices (the slice loop unrolled by
+                // two at 8 tokens) and sums them in registers.
                 if (!units_ready) {
                     // Bounded: a give-up is recorded; the CTA still finishes.
                     units_ready = true;

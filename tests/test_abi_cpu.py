@@ -142,6 +142,7 @@ def test_kernels_do_not_spill():
     assert sum("eva_lookup_kernelI" in b[0] for b in blocks) == 32, out     # 16 for 8-bit + 16 for 4-bit indices
     assert sum("eva_lookup_kernel3I" in b[0] for b in blocks) == 4, out     # three CTAs per SM
     assert sum("eva_dequant_kernel" in b[0] for b in blocks) == 8, out      # per-group x tokens x direct push
+    assert sum("eva_dequant_group_kernel" in b[0] for b in blocks) == 4, out   # several layers per launch
     assert sum("eva_tc_kernel" in b[0] for b in blocks) == 2, out           # tcgen05 path, with / without residual
     assert sum("eva_kmeans_assign_kernel" in b[0] for b in blocks) == 2, out
     for name, stack, st, ld in blocks:

@@ -315,11 +315,13 @@ def test_four_bit_integer_exact():
         assert np.array_equal(y, oracle.layer_linear(layer, x))
 
 
-@pytest.mark.parametrize("B", [1, 2])
+@pytest.mark.parametrize("B", [1, 2, 4, 16])
 def test_grouped_call_matches_separate_calls(B):
     """eva_vq_linear_run_group: one launch for layers of one shape and format
-    (bitwise equal to separate calls with the same flag, plain or independent,
-    also with the residual), separate launches for a mixed group."""
+    (the lookup kernel at one or two tokens, the dequantize kernel from four
+    on; bitwise equal to separate calls with the same flag, plain or
+    independent, also with the residual), separate launches for a mixed
+    group."""
     import torch
     from vector_quantized_weight_b200 import eva_vq
     for shape in (synth.LayerShape("g", 4096, 4096), synth.LayerShape("gr", 512, 1024, residual_group=128)):
@@ -329,6 +331,8 @@ def test_grouped_call_matches_separate_calls(B):
             ref = [lin(x, independent=indep).clone() for lin, x in zip(lins, xs)]
             outs = eva_vq.run_group(lins, xs, independent=indep)
             torch.cuda.synchronize()
+            if shape.name == "g":
+                assert lins[0].info().path == (eva_vq.EVA_PATH_DEQUANT_MMA if B >= 4 else eva_vq.EVA_PATH_OC_LOOKUP)
             for a, b in zip(ref, outs):
                 assert torch.equal(a, b)
         for lin in lins:

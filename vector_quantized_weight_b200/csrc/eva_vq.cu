@@ -464,6 +464,16 @@ void plan_dequant(eva_vq_linear *h, int ntg) {
 
 cudaError_t set_smem_attrs(int smem_optin) {
     cudaError_t e;
+    for (int v = 0; v < 4; ++v) {
+        const void *fn = v == 0 ? (const void *)eva_dequant_group_kernel<1, false>
+                       : v == 1 ? (const void *)eva_dequant_group_kernel<2, false>
+                       : v == 2 ? (const void *)eva_dequant_group_kernel<1, true>
+                                : (const void *)eva_dequant_group_kernel<2, true>;
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_optin);
+        if (e != cudaSuccess) return e;
+    }
     for (int v = 0; v < 8; ++v) {
         const DequantFn fn = dequant_fn(v & 1, 1 + ((v >> 1) & 1), (v >> 2) & 1);
         e = cudaFuncSetAttribute((const void *)fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
@@ -521,8 +531,8 @@ void apply_injection(eva_vq_linear *h, LookupParams &p) {
 }
 
 // Launch the dequantize kernel for a call whose common parameters are in p.
-cudaError_t launch_dequant(eva_vq_linear *h, LookupParams p, int B, cudaStream_t s, size_t *smem_out,
-                           int *grid_out) {
+// The dequantize kernel's fields of a call's parameters (its plan for B).
+void dequant_params(eva_vq_linear *h, LookupParams &p, int B) {
     const int ntg = B > 8 ? 2 : 1;
     const eva_vq_linear::Plan &pl = h->dq[ntg - 1];
     p.Gs = pl.Gs;
@@ -531,14 +541,25 @@ cudaError_t launch_dequant(eva_vq_linear *h, LookupParams p, int B, cudaStream_t
     p.wi_staged = pl.staged;
     p.rot_b = 0;
     apply_injection(h, p);
-    *smem_out = pl.smem;
-    *grid_out = pl.Gs * pl.Gt;
 #ifdef EVA_DEVICE_CHECKS
     p.smem_bytes = (unsigned)pl.smem;
 #endif
-    const bool direct = (h->S + pl.Gs - 1) / pl.Gs == 1;   // the same rule as dequant_smem's
-    return launch_pdl(dequant_fn(h->tiles_per_cb != 0, ntg, direct), dim3(pl.Gs * pl.Gt), dim3(kThreads), pl.smem,
-                      s, pl.Gs, p);
+}
+
+bool dequant_direct(const eva_vq_linear *h, int B) {
+    const eva_vq_linear::Plan &pl = h->dq[B > 8 ? 1 : 0];
+    return (h->S + pl.Gs - 1) / pl.Gs == 1;   // the same rule as dequant_smem's
+}
+
+cudaError_t launch_dequant(eva_vq_linear *h, LookupParams p, int B, cudaStream_t s, size_t *smem_out,
+                           int *grid_out) {
+    const int ntg = B > 8 ? 2 : 1;
+    const eva_vq_linear::Plan &pl = h->dq[ntg - 1];
+    dequant_params(h, p, B);
+    *smem_out = pl.smem;
+    *grid_out = pl.Gs * pl.Gt;
+    return launch_pdl(dequant_fn(h->tiles_per_cb != 0, ntg, dequant_direct(h, B)), dim3(pl.Gs * pl.Gt),
+                      dim3(kThreads), pl.smem, s, pl.Gs, p);
 }
 
 bool use_three_per_sm(const eva_vq_linear *h, int B, int independent) {
@@ -1046,8 +1067,45 @@ eva_status_t eva_vq_linear_run_group(const eva_vq_linear_t *hs, const void *cons
         if (!h || !xs[i] || !ys[i] || !aligned16(xs[i]) || !aligned16(ys[i])) return EVA_ERR_INVALID_ARG;
         if (B < 1 || B > h->desc.max_batch || h->device != hs[0]->device) return EVA_ERR_INVALID_ARG;
     }
-    // One launch when every layer has the first one's shape and format.
     const eva_vq_desc &d0 = hs[0]->desc;
+    const int independent = (flags & EVA_RUN_INDEPENDENT) ? 1 : 0;
+    // Layers of one shape on the dequantize path (one shared codebook each):
+    // one launch of the dequantize kernel.
+    bool dq_one = use_dequant(hs[0], B) && !d0.codebook_rows && count > 1;
+    for (int i = 1; i < count && dq_one; ++i) {
+        const eva_vq_desc &d = hs[i]->desc;
+        dq_one = use_dequant(hs[i], B) && !d.codebook_rows && d.N == d0.N && d.K == d0.K &&
+                 d.out_dtype == d0.out_dtype && hs[i]->dq[B > 8 ? 1 : 0].Gs == hs[0]->dq[B > 8 ? 1 : 0].Gs &&
+                 hs[i]->dq[B > 8 ? 1 : 0].Gt == hs[0]->dq[B > 8 ? 1 : 0].Gt &&
+                 hs[i]->dq[B > 8 ? 1 : 0].smem == hs[0]->dq[B > 8 ? 1 : 0].smem;
+    }
+    if (dq_one) {
+        LookupGroup g;
+        std::memset(&g, 0, sizeof(g));
+        size_t smem = 0;
+        for (int i = 0; i < count; ++i) {
+            g.p[i] = call_params(hs[i], xs[i], B, ys[i], independent, &smem);
+            dequant_params(hs[i], g.p[i], B);
+        }
+        const int ntg = B > 8 ? 2 : 1;
+        const eva_vq_linear::Plan &pl = hs[0]->dq[ntg - 1];
+        g.count = count;
+        g.ctas_per_layer = pl.Gs * pl.Gt;
+        const bool direct = dequant_direct(hs[0], B);
+        using DqGroupFn = void (*)(LookupGroup);
+        const DqGroupFn fn = ntg == 2 ? (direct ? eva_dequant_group_kernel<2, true> : eva_dequant_group_kernel<2, false>)
+                                      : (direct ? eva_dequant_group_kernel<1, true> : eva_dequant_group_kernel<1, false>);
+        const cudaError_t e = launch_pdl(fn, dim3(count * pl.Gs * pl.Gt), dim3(kThreads), pl.smem,
+                                         reinterpret_cast<cudaStream_t>(stream), pl.Gs, g);
+        if (e != cudaSuccess) return cuda_status(e);
+        for (int i = 0; i < count; ++i) {
+            hs[i]->last_grid = pl.Gs * pl.Gt;
+            hs[i]->last_kernels = 1;
+            hs[i]->last_path = EVA_PATH_DEQUANT_MMA;
+        }
+        return EVA_OK;
+    }
+    // One launch when every layer has the first one's shape and format.
     bool one = groupable(hs[0], B);
     for (int i = 1; i < count && one; ++i) {
         const eva_vq_desc &d = hs[i]->desc;
@@ -1061,7 +1119,6 @@ eva_status_t eva_vq_linear_run_group(const eva_vq_linear_t *hs, const void *cons
         }
         return EVA_OK;
     }
-    const int independent = (flags & EVA_RUN_INDEPENDENT) ? 1 : 0;
     LookupGroup g;
     std::memset(&g, 0, sizeof(g));
     size_t smem = 0;

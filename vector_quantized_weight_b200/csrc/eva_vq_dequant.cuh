@@ -54,7 +54,11 @@ __device__ __forceinline__ void build_codebook_table(const LookupParams &p, int 
 // half the SM's shared memory anyway, so they keep one CTA per SM and the
 // registers that go with it.
 template <bool GROUPED, int NTG, bool DIRECT>
-__global__ void __launch_bounds__(kThreads, (NTG == 2 && (GROUPED || !DIRECT)) ? 1 : 2) eva_dequant_kernel(const LookupParams p) {
+constexpr int kDequantMinBlocks = (NTG == 2 && (GROUPED || !DIRECT)) ? 1 : 2;
+
+// The whole per-CTA program; eva_bid is the CTA's index within its layer.
+template <bool GROUPED, int NTG, bool DIRECT>
+__device__ __forceinline__ void dequant_body(const LookupParams &p, const int eva_bid) {
     constexpr int TT = 8 * NTG;                         // tokens per pass
     constexpr uint32_t BLK = kTileRows * TT * 4u;       // bytes of one tile's running sums
     // A tile's block in the reduction stage.  Sums pushed from registers (8
@@ -65,7 +69,6 @@ __global__ void __launch_bounds__(kThreads, (NTG == 2 && (GROUPED || !DIRECT)) ?
     constexpr uint32_t BLK_S = kTileRows * RS * 4u;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, q = lane & 3;
-    const int eva_bid = blockIdx.x;
     const int ts = eva_bid % p.Gs, tt = eva_bid / p.Gs;
     const int s0 = (int)((long long)p.S * ts / p.Gs), s1 = (int)((long long)p.S * (ts + 1) / p.Gs);
     const int t0 = (int)((long long)p.T * tt / p.Gt), t1 = (int)((long long)p.T * (tt + 1) / p.Gt);
@@ -472,6 +475,22 @@ __global__ void __launch_bounds__(kThreads, (NTG == 2 && (GROUPED || !DIRECT)) ?
         p.timeline[eva_bid * 8 + 7] = smid;
     }
 #endif
+}
+
+template <bool GROUPED, int NTG, bool DIRECT>
+__global__ void __launch_bounds__(kThreads, kDequantMinBlocks<GROUPED, NTG, DIRECT>)
+    eva_dequant_kernel(const LookupParams p) {
+    dequant_body<GROUPED, NTG, DIRECT>(p, blockIdx.x);
+}
+
+// Several layers of one shape (one shared codebook each) in one launch, as
+// eva_lookup_group_kernel: layer blockIdx.x / ctas_per_layer.
+template <int NTG, bool DIRECT>
+__global__ void __launch_bounds__(kThreads, kDequantMinBlocks<false, NTG, DIRECT>)
+    eva_dequant_group_kernel(const LookupGroup g) {
+    const int li = blockIdx.x / g.ctas_per_layer;
+    if (li >= g.count) return;
+    dequant_body<false, NTG, DIRECT>(g.p[li], blockIdx.x - li * g.ctas_per_layer);
 }
 
 }  // namespace eva

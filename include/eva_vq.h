@@ -159,7 +159,9 @@ EVA_API eva_status_t eva_vq_linear_run_ex(eva_vq_linear_t h, const void *x, int3
  * for the same B (1 <= count <= 16; all handles on the current device).  No
  * layer may read another's output.  When every layer has the first one's
  * N, K and format (8-bit indices, one shared codebook, no rotation, the same
- * residual setting and output type) and takes the lookup path at this B,
+ * residual setting and output type) and takes the lookup path at this B, or
+ * every layer has the first one's N, K, output type and dequantize-path plan
+ * (one shared codebook each, no residual, no rotation) and takes that path,
  * the layers run as ONE launch whose CTAs the hardware schedules as slots
  * free -- e.g. the q, k and v projections of a decoder block, which share
  * their input.  Otherwise it is one eva_vq_linear_run_ex per layer.  Results

@@ -240,6 +240,28 @@ def test_dequant_path_large_layers(N, K, cbr, B):
     assert np.all(err <= TOL), err.max()
 
 
+@pytest.mark.parametrize("N,K,cbr", [(4096, 4096, 0), (1040, 2048, 0), (2048, 4096, 128)])
+def test_dequant_path_ragged_batches(N, K, cbr):
+    """The dequantize path at batch sizes that leave token groups partly empty
+    (5, 9, 13 tokens) and a second pass partly empty (31): every row against
+    the oracle, for one-slice CTAs (4096 x 4096), several slices per CTA and a
+    ragged row count, and per-group codebooks."""
+    import torch
+    from vector_quantized_weight_b200 import eva_vq
+    shape = synth.LayerShape("rag", N, K, codebook_rows=cbr)
+    layer = synth.make_layer(shape, 4100 + N)
+    lin = eva_vq.from_layer(layer, max_batch=31, path=eva_vq.EVA_PATH_DEQUANT_MMA)
+    for B in (5, 9, 13, 31):
+        x = synth.make_x(K, B, 4200 + B)
+        y = lin(torch.from_numpy(x).cuda()).float().cpu().numpy()
+        torch.cuda.synchronize()
+        assert lin.info().path == eva_vq.EVA_PATH_DEQUANT_MMA
+        err = norm_rel_err(y, oracle.layer_linear(layer, x, nthreads=NTHREADS))
+        assert np.all(err <= TOL), (B, err.max())
+    assert eva_vq.eva_vq_sync_status(lin.handle) == eva_vq.EVA_OK
+    lin.close()
+
+
 def test_dequant_path_rejects_residual_layers():
     from vector_quantized_weight_b200 import eva_vq
     shape = synth.LayerShape("r", 64, 512, residual_group=128)

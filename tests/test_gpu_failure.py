@@ -66,7 +66,7 @@ def test_inject_rejects_bad_round_counts():
 
 
 def test_bounded_wait_gives_up_on_the_dequantize_path():
-    """The warp-level dequantize path (four tokens and more) stages its index
+    """The warp-level dequantize path (three tokens and more) stages its index
     units the same way: the hook makes its wait run out too."""
     import torch
     from vector_quantized_weight_b200 import eva_vq

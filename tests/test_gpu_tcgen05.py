@@ -79,21 +79,23 @@ def test_tcgen05_integer_inputs_exact():
 
 
 def test_auto_path_by_batch():
-    """AUTO: lookups below four tokens; from four on the warp-level dequantize
-    path where the layer allows it, the tcgen05 path past 32 tokens with one
-    shared codebook; a residual / rotated layer keeps the lookup path below
-    eight tokens and takes tcgen05 from there."""
+    """AUTO: lookups below three tokens (two with per-group codebooks); from
+    there on the warp-level dequantize path where the layer allows it, the
+    tcgen05 path past 32 tokens with one shared codebook; a residual / rotated
+    layer keeps the lookup path below eight tokens and takes tcgen05 from
+    there."""
     from vector_quantized_weight_b200 import eva_vq
     plain = synth.LayerShape("l7b", 4096, 4096)
     gemma = synth.LayerShape("gemma", 3584, 3584, residual_group=128, hadamard_block=512)
-    for shape, cases in ((plain, ((1, eva_vq.EVA_PATH_OC_LOOKUP), (3, eva_vq.EVA_PATH_OC_LOOKUP),
-                                  (4, eva_vq.EVA_PATH_DEQUANT_MMA), (16, eva_vq.EVA_PATH_DEQUANT_MMA),
+    for shape, cases in ((plain, ((1, eva_vq.EVA_PATH_OC_LOOKUP), (2, eva_vq.EVA_PATH_OC_LOOKUP),
+                                  (3, eva_vq.EVA_PATH_DEQUANT_MMA), (16, eva_vq.EVA_PATH_DEQUANT_MMA),
                                   (32, eva_vq.EVA_PATH_DEQUANT_MMA), (33, eva_vq.EVA_PATH_TCGEN05),
                                   (64, eva_vq.EVA_PATH_TCGEN05))),
                          (gemma, ((1, eva_vq.EVA_PATH_OC_LOOKUP), (4, eva_vq.EVA_PATH_OC_LOOKUP),
                                   (8, eva_vq.EVA_PATH_TCGEN05))),
                          (synth.LayerShape("l70b", 8192, 8192, codebook_rows=128),
-                          ((8, eva_vq.EVA_PATH_DEQUANT_MMA), (32, eva_vq.EVA_PATH_DEQUANT_MMA)))):
+                          ((1, eva_vq.EVA_PATH_OC_LOOKUP), (2, eva_vq.EVA_PATH_DEQUANT_MMA),
+                           (8, eva_vq.EVA_PATH_DEQUANT_MMA), (32, eva_vq.EVA_PATH_DEQUANT_MMA)))):
         layer = synth.make_layer(shape, 8)
         for B, path in cases:
             x = synth.make_x(shape.K, B, 9)

@@ -390,8 +390,16 @@ DequantFn dequant_fn(bool grouped, int ntg, bool direct) {
 }
 
 // Calls with at least this many tokens take the dequantize path (when the
-// layer allows it and the descriptor leaves the choice to the library).
-constexpr int kDequantMinBatch = 4;
+// layer allows it and the descriptor leaves the choice to the library); layers
+// with per-group codebooks from kDequantMinBatchGrouped on.  Measured on B200
+// (us per layer, each call waiting for the one before it, lookup against
+// dequantize path): 4096 x 4096 at 3 tokens 10.3 against 5.7, at 2 5.8 against
+// 5.7; 11008 x 4096 at 3 15.9 against 14.6, at 2 8.8 against 14.4; 4096 x
+// 11008 at 3 21.7 against 11.4; 8192 x 8192 with 128-row codebooks at 2 39.0
+// against 22.7, at 3 75.6 against 22.7.
+constexpr int kDequantMinBatch = 3;
+constexpr int kDequantMinBatchGrouped = 2;
+int dequant_min_batch(const eva_vq_desc &d) { return d.codebook_rows ? kDequantMinBatchGrouped : kDequantMinBatch; }
 
 // Dynamic shared memory of the dequantize kernel: the replicated codebook,
 // the x stage of up to nsl slices, the running sums, the reduction stage, the
@@ -582,9 +590,9 @@ bool use_three_per_sm(const eva_vq_linear *h, int B, int independent) {
 //    (3.125-bit 3584 x 3584: 15.4 against 22.0 us at 4 tokens), tcgen05 from
 //    there (24.7 against 55.5 us at 16).
 // A tcgen05.mma of M = 128 rows takes about as long for N = 16 tokens as for
-// N = 64 (about 100 cycles per instruction, measured), so the tensor-core
-// path pays off as the batch grows, while the warp-level MMA of 8 tokens
-// scales with the batch.
+// N = 64 (54-100 cycles per instruction in two single-thread probes), so the
+// tensor-core path pays off as the batch grows, while the warp-level MMA of 8
+// tokens scales with the batch.
 constexpr int kTcMinBatch = 33;
 constexpr int kTcResidMinBatch = 8;
 
@@ -598,7 +606,7 @@ bool use_tc(const eva_vq_linear *h, int B) {
 
 bool use_dequant(const eva_vq_linear *h, int B) {
     if (!h->dq_ok || use_tc(h, B)) return false;
-    return h->desc.path == EVA_PATH_DEQUANT_MMA || (h->desc.path == EVA_PATH_AUTO && B >= kDequantMinBatch);
+    return h->desc.path == EVA_PATH_DEQUANT_MMA || (h->desc.path == EVA_PATH_AUTO && B >= dequant_min_batch(h->desc));
 }
 
 // Tensor memory per tcgen05-path CTA (columns) and the dynamic shared memory
@@ -750,7 +758,8 @@ eva_status_t eva_vq_linear_create(eva_vq_linear_t *out, const eva_vq_desc *desc,
     if (desc->max_batch > 1) plan_grid(h, 1);
     int max_grid = std::max(h->plan[0].Gs * h->plan[0].Gt, h->plan[1].Gs * h->plan[1].Gt);
     if (!desc->residual_group && !desc->hadamard_block && desc->index_bits == 8 &&
-        (desc->path == EVA_PATH_DEQUANT_MMA || (desc->path == EVA_PATH_AUTO && desc->max_batch >= kDequantMinBatch))) {
+        (desc->path == EVA_PATH_DEQUANT_MMA ||
+         (desc->path == EVA_PATH_AUTO && desc->max_batch >= dequant_min_batch(*desc)))) {
         plan_dequant(h, 1);
         plan_dequant(h, 2);
         h->dq_ok = h->dq[0].Gs > 0 && h->dq[1].Gs > 0;

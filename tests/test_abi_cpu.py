@@ -58,6 +58,8 @@ def _create(desc, wc=0x1000, wi=0x2000, signs=None, alpha=None, hsign=None):
     (dict(d=3), eva_vq.EVA_ERR_UNSUPPORTED),
     (dict(index_bits=6), eva_vq.EVA_ERR_UNSUPPORTED),
     (dict(index_bits=4, path=2), eva_vq.EVA_ERR_UNSUPPORTED),   # 4-bit: the lookup path only
+    (dict(path=2, residual_group=128, codebook_rows=16), eva_vq.EVA_ERR_UNSUPPORTED),  # dequantize: residual,
+    (dict(path=2, K=520, hadamard_block=8), eva_vq.EVA_ERR_UNSUPPORTED),               # rotation need one codebook, K % 64 == 0
     (dict(index_bits=4, K=516), eva_vq.EVA_ERR_INVALID_ARG),
     (dict(N=0), eva_vq.EVA_ERR_INVALID_ARG),
     (dict(K=510), eva_vq.EVA_ERR_INVALID_ARG),
@@ -141,7 +143,7 @@ def test_kernels_do_not_spill():
                         r"(\d+) bytes spill stores, (\d+) bytes spill loads", out)
     assert sum("eva_lookup_kernelI" in b[0] for b in blocks) == 32, out     # 16 for 8-bit + 16 for 4-bit indices
     assert sum("eva_lookup_kernel3I" in b[0] for b in blocks) == 4, out     # three CTAs per SM
-    assert sum("eva_dequant_kernel" in b[0] for b in blocks) == 8, out      # per-group x tokens x direct push
+    assert sum("eva_dequant_kernel" in b[0] for b in blocks) == 12, out     # per-group x tokens x direct push, + residual
     assert sum("eva_dequant_group_kernel" in b[0] for b in blocks) == 4, out   # several layers per launch
     assert sum("eva_tc_kernel" in b[0] for b in blocks) == 2, out           # tcgen05 path, with / without residual
     assert sum("eva_kmeans_assign_kernel" in b[0] for b in blocks) == 2, out

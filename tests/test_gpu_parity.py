@@ -263,9 +263,36 @@ def test_dequant_path_ragged_batches(N, K, cbr):
     lin.close()
 
 
-def test_dequant_path_rejects_residual_layers():
+@pytest.mark.parametrize("shape,Bs", [
+    (synth.LayerShape("gemma", 3584, 3584, residual_group=128, hadamard_block=512), (4, 9)),
+    (synth.LayerShape("gemma_down", 3584, 14336, residual_group=128, hadamard_block=2048), (3,)),
+    (synth.LayerShape("gemma_rotK", 3584, 3584, residual_group=128, hadamard_block=3584), (2, 16)),
+    (synth.LayerShape("resid_only", 384, 1024, residual_group=128), (5, 17)),
+    (synth.LayerShape("ragged", 200, 1152, residual_group=128, hadamard_block=64), (6,)),
+])
+def test_dequant_path_with_residual_and_rotation(shape, Bs):
+    """The dequantize path carries the 1-bit sign residual (signed alpha
+    included) and reads the rotated input from the rotation kernel (Sylvester
+    and Paley blocks, a K range ending mid-slice): every row against the
+    oracle, the status word clean."""
+    import torch
     from vector_quantized_weight_b200 import eva_vq
-    shape = synth.LayerShape("r", 64, 512, residual_group=128)
+    layer = synth.make_layer(shape, 7100 + shape.N, alpha_signed=True)
+    lin = eva_vq.from_layer(layer, max_batch=max(Bs), path=eva_vq.EVA_PATH_DEQUANT_MMA)
+    for B in Bs:
+        x = synth.make_x(shape.K, B, 7200 + B)
+        y = lin(torch.from_numpy(x).cuda()).float().cpu().numpy()
+        torch.cuda.synchronize()
+        assert lin.info().path == eva_vq.EVA_PATH_DEQUANT_MMA
+        err = norm_rel_err(y, oracle.layer_linear(layer, x, nthreads=NTHREADS))
+        assert np.all(err <= TOL), (shape.name, B, err.max())
+    assert eva_vq.eva_vq_sync_status(lin.handle) == eva_vq.EVA_OK
+    lin.close()
+
+
+def test_dequant_path_rejects_residual_with_group_codebooks():
+    from vector_quantized_weight_b200 import eva_vq
+    shape = synth.LayerShape("r", 256, 512, residual_group=128, codebook_rows=128)
     layer = synth.make_layer(shape, 1)
     with pytest.raises(eva_vq.EvaError) as ei:
         eva_vq.from_layer(layer, max_batch=8, path=eva_vq.EVA_PATH_DEQUANT_MMA)

@@ -46,6 +46,28 @@ def test_noalloc_run_matches_regular_run(shape, B):
     lin.close()
 
 
+@pytest.mark.parametrize("shape,B", [
+    (synth.LayerShape("rot_3bit", 3584, 3584, residual_group=128, hadamard_block=512), 4),
+    (synth.LayerShape("rot_paley", 256, 3584, residual_group=128, hadamard_block=3584), 2),
+])
+def test_noalloc_dequantize_path_with_rotation(shape, B):
+    """The dequantize path of a rotated layer: the allocation-free call runs
+    the rotation kernel into the static scratch (Paley blocks too, which the
+    lookup path fuses) and matches the regular call bitwise."""
+    import torch
+    from vector_quantized_weight_b200 import eva_vq
+    layer = synth.make_layer(shape, 911)
+    lin = eva_vq.from_layer(layer, max_batch=B, path=eva_vq.EVA_PATH_DEQUANT_MMA)
+    x = torch.from_numpy(synth.make_x(shape.K, B, 912)).cuda()
+    ref = lin(x).clone()
+    y = torch.empty((B, shape.N), dtype=torch.float16, device="cuda")
+    eva_vq.eva_vq_linear_run_noalloc(lin.handle, x.data_ptr(), B, y.data_ptr(), eva_vq._stream_handle(None))
+    torch.cuda.synchronize()
+    assert lin.info().path == eva_vq.EVA_PATH_DEQUANT_MMA and lin.info().kernels_per_run == 2
+    assert torch.equal(y, ref)
+    lin.close()
+
+
 def test_noalloc_rejects_requests_beyond_the_static_scratch():
     import torch
     from vector_quantized_weight_b200 import eva_vq

@@ -162,7 +162,11 @@ eva_status_t validate_desc(const eva_vq_desc *d) {
     if (d->path != EVA_PATH_AUTO && d->path != EVA_PATH_OC_LOOKUP && d->path != EVA_PATH_DEQUANT_MMA &&
         d->path != EVA_PATH_TCGEN05)
         return EVA_ERR_INVALID_ARG;
-    if (d->path == EVA_PATH_DEQUANT_MMA && (d->residual_group || d->hadamard_block)) return EVA_ERR_UNSUPPORTED;
+    // The dequantize path takes a residual or a rotation with one shared
+    // codebook and the tcgen05 path's row-block data (K a multiple of 64).
+    if (d->path == EVA_PATH_DEQUANT_MMA && (d->residual_group || d->hadamard_block) &&
+        (d->codebook_rows || !tc_layer_ok(*d)))
+        return EVA_ERR_UNSUPPORTED;
     if (d->path == EVA_PATH_TCGEN05 && !tc_layer_ok(*d)) return EVA_ERR_UNSUPPORTED;
     return EVA_OK;
 }
@@ -379,8 +383,13 @@ cudaError_t launch_pdl(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_
 
 
 using DequantFn = void (*)(LookupParams);
-// `direct`: every CTA takes one K-slice (Gs = S), see eva_dequant_kernel.
-DequantFn dequant_fn(bool grouped, int ntg, bool direct) {
+// `direct`: every CTA takes one K-slice (Gs = S), see eva_dequant_kernel;
+// `resid`: the sign residual (one shared codebook only).
+DequantFn dequant_fn(bool grouped, int ntg, bool direct, bool resid = false) {
+    if (resid) {
+        if (direct) return ntg == 2 ? eva_dequant_kernel<false, 2, true, true> : eva_dequant_kernel<false, 1, true, true>;
+        return ntg == 2 ? eva_dequant_kernel<false, 2, false, true> : eva_dequant_kernel<false, 1, false, true>;
+    }
     if (direct) {
         if (grouped) return ntg == 2 ? eva_dequant_kernel<true, 2, true> : eva_dequant_kernel<true, 1, true>;
         return ntg == 2 ? eva_dequant_kernel<false, 2, true> : eva_dequant_kernel<false, 1, true>;
@@ -425,7 +434,7 @@ void plan_dequant(eva_vq_linear *h, int ntg) {
     pl.Gs = 0;
     for (int gs = 1; gs <= std::min(S, 16); ++gs) {
         const int nsl = (S + gs - 1) / gs;
-        const DequantFn fn = dequant_fn(h->tiles_per_cb != 0, ntg, nsl == 1);
+        const DequantFn fn = dequant_fn(h->tiles_per_cb != 0, ntg, nsl == 1, h->desc.residual_group != 0);
         const int gt_min = (T + kMaxCtaTiles - 1) / kMaxCtaTiles;
         const int clusters = max_active_clusters((LookupFn)fn, (size_t)h->smem_optin, gs);
         const int gt_max = std::min({T, std::max(clusters, gt_min), std::max(P / gs, gt_min)});
@@ -482,8 +491,9 @@ cudaError_t set_smem_attrs(int smem_optin) {
         e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_optin);
         if (e != cudaSuccess) return e;
     }
-    for (int v = 0; v < 8; ++v) {
-        const DequantFn fn = dequant_fn(v & 1, 1 + ((v >> 1) & 1), (v >> 2) & 1);
+    for (int v = 0; v < 12; ++v) {
+        const DequantFn fn = v < 8 ? dequant_fn(v & 1, 1 + ((v >> 1) & 1), (v >> 2) & 1)
+                                   : dequant_fn(false, 1 + (v & 1), (v >> 1) & 1, true);
         e = cudaFuncSetAttribute((const void *)fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute((const void *)fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_optin);
@@ -548,9 +558,21 @@ void dequant_params(eva_vq_linear *h, LookupParams &p, int B) {
     p.acc_tiles = (h->T + pl.Gt - 1) / pl.Gt;
     p.wi_staged = pl.staged;
     p.rot_b = 0;
+    p.sgb = h->sgb;
+    p.al_rm = h->al_rm;
+    p.KB = h->desc.K / kTcStageK;
     apply_injection(h, p);
 #ifdef EVA_DEVICE_CHECKS
     p.smem_bytes = (unsigned)pl.smem;
+    if (h->desc.residual_group) {
+        const int R128 = (h->desc.N + 127) / 128;
+        p.chk_base[BUF_SG] = h->sgb;
+        p.chk_bytes[BUF_SG] = (unsigned long long)R128 * 128 * (h->desc.K / 8);
+        p.chk_base[BUF_AL] = h->al_rm;
+        p.chk_bytes[BUF_AL] = (unsigned long long)h->desc.N * (h->desc.K / 128) * 2;
+    }
+    p.chk_base[BUF_X] = p.x;
+    p.chk_bytes[BUF_X] = (unsigned long long)B * h->desc.K * (p.x_f32 ? 4 : 2);
 #endif
 }
 
@@ -566,8 +588,8 @@ cudaError_t launch_dequant(eva_vq_linear *h, LookupParams p, int B, cudaStream_t
     dequant_params(h, p, B);
     *smem_out = pl.smem;
     *grid_out = pl.Gs * pl.Gt;
-    return launch_pdl(dequant_fn(h->tiles_per_cb != 0, ntg, dequant_direct(h, B)), dim3(pl.Gs * pl.Gt),
-                      dim3(kThreads), pl.smem, s, pl.Gs, p);
+    return launch_pdl(dequant_fn(h->tiles_per_cb != 0, ntg, dequant_direct(h, B), h->desc.residual_group != 0),
+                      dim3(pl.Gs * pl.Gt), dim3(kThreads), pl.smem, s, pl.Gs, p);
 }
 
 bool use_three_per_sm(const eva_vq_linear *h, int B, int independent) {
@@ -600,13 +622,17 @@ bool use_tc(const eva_vq_linear *h, int B) {
     if (!h->tc_ok) return false;
     if (h->desc.path == EVA_PATH_TCGEN05) return true;
     if (h->desc.path != EVA_PATH_AUTO || B < kDequantMinBatch) return false;
-    if (!h->dq_ok) return B >= kTcResidMinBatch;
+    if (!h->dq_ok || h->desc.residual_group || h->desc.hadamard_block) return B >= kTcResidMinBatch;
     return B >= kTcMinBatch && h->desc.codebook_rows == 0;
 }
 
 bool use_dequant(const eva_vq_linear *h, int B) {
     if (!h->dq_ok || use_tc(h, B)) return false;
-    return h->desc.path == EVA_PATH_DEQUANT_MMA || (h->desc.path == EVA_PATH_AUTO && B >= dequant_min_batch(h->desc));
+    if (h->desc.path == EVA_PATH_DEQUANT_MMA) return true;
+    // Residual / rotated layers: only when forced (AUTO keeps the lookup and
+    // tcgen05 paths for them).
+    if (h->desc.residual_group || h->desc.hadamard_block) return false;
+    return h->desc.path == EVA_PATH_AUTO && B >= dequant_min_batch(h->desc);
 }
 
 // Tensor memory per tcgen05-path CTA (columns) and the dynamic shared memory
@@ -757,7 +783,12 @@ eva_status_t eva_vq_linear_create(eva_vq_linear_t *out, const eva_vq_desc *desc,
     plan_grid(h, 0);
     if (desc->max_batch > 1) plan_grid(h, 1);
     int max_grid = std::max(h->plan[0].Gs * h->plan[0].Gt, h->plan[1].Gs * h->plan[1].Gt);
-    if (!desc->residual_group && !desc->hadamard_block && desc->index_bits == 8 &&
+    // Residual and rotated layers on the dequantize path read the row-block
+    // signs, the canonical alpha and the rotated x the tcgen05 path keeps.
+    const bool dq_resrot = desc->residual_group || desc->hadamard_block;
+    if (desc->index_bits == 8 &&
+        (!dq_resrot || (tc_layer_ok(*desc) && !desc->codebook_rows &&
+                        (!desc->residual_group || desc->residual_group == 128))) &&
         (desc->path == EVA_PATH_DEQUANT_MMA ||
          (desc->path == EVA_PATH_AUTO && desc->max_batch >= dequant_min_batch(*desc)))) {
         plan_dequant(h, 1);
@@ -786,7 +817,7 @@ eva_status_t eva_vq_linear_create(eva_vq_linear_t *out, const eva_vq_desc *desc,
     }
     chk(dalloc(&h->wi, (size_t)units * h->unit_bytes, nullptr));
     const int R128 = (N + kTcRows - 1) / kTcRows;
-    if (h->tc_ok) {
+    if (h->tc_ok || (h->dq_ok && dq_resrot)) {
         chk(dalloc(&h->wib, (size_t)R128 * kTcRows * h->J, nullptr));
         if (desc->residual_group) {
             chk(dalloc(&h->sgb, (size_t)R128 * kTcRows * (K / 8), nullptr));
@@ -832,7 +863,7 @@ eva_status_t eva_vq_linear_create(eva_vq_linear_t *out, const eva_vq_desc *desc,
             reinterpret_cast<const __half *>(alpha), h->al, N, K / desc->residual_group, h->T, ab);
         chk(cudaGetLastError());
     }
-    if (h->tc_ok) {
+    if (h->tc_ok || (h->dq_ok && dq_resrot)) {
         const long long nb = (long long)R128 * kTcRows * h->J;
         eva_repack_wi_rowblock_kernel<<<blocks_for(nb, thr), thr, 0, s>>>(wi, h->wib, N, h->J, nb);
         chk(cudaGetLastError());
@@ -953,6 +984,24 @@ GroupFn group_fn(bool pair_t, bool resid) {
 namespace {
 // One call on the tcgen05 path: for a rotated layer the standalone rotation
 // kernel first writes x~ (fp32) into `xrot`, then the tensor-core kernel.
+// x~ of a rotated layer into `xrot` (fp32 [B][K]) with the standalone
+// rotation kernel (Sylvester or Paley blocks).
+cudaError_t launch_rotation(const eva_vq_linear *h, const void *x, int B, cudaStream_t s, int independent,
+                            float *xrot) {
+    const eva_vq_desc &d = h->desc;
+    const int b = d.hadamard_block, m = paley_m(b), thr = std::min(b / 2, 1024);
+    const float scale = (float)(1.0 / std::sqrt((double)b));
+    if (m) {
+        // Launched in plain stream order (it reads x as soon as it starts).
+        eva_paley_rows_kernel<<<dim3(d.K / b, B), thr, (size_t)b * sizeof(float), s>>>(
+            reinterpret_cast<const __half *>(x), h->hsign, h->h28, xrot, d.K, b, m, scale);
+        return cudaGetLastError();
+    }
+    return launch_pdl(eva_hadamard_kernel, dim3(d.K / b, B), dim3(thr), (size_t)b * sizeof(float), s, 0,
+                      reinterpret_cast<const __half *>(x), (const int8_t *)h->hsign, xrot, d.K, b, scale,
+                      independent);
+}
+
 cudaError_t launch_tc(eva_vq_linear *h, const void *x, int B, void *y, cudaStream_t s, int independent,
                       float *xrot) {
     const eva_vq_desc &d = h->desc;
@@ -961,18 +1010,7 @@ cudaError_t launch_tc(eva_vq_linear *h, const void *x, int B, void *y, cudaStrea
     const void *xin = x;
     int x_f32 = 0;
     if (d.hadamard_block) {
-        const int b = d.hadamard_block, m = paley_m(b), thr = std::min(b / 2, 1024);
-        const float scale = (float)(1.0 / std::sqrt((double)b));
-        if (m) {
-            // Launched in plain stream order (it reads x as soon as it starts).
-            eva_paley_rows_kernel<<<dim3(d.K / b, B), thr, (size_t)b * sizeof(float), s>>>(
-                reinterpret_cast<const __half *>(x), h->hsign, h->h28, xrot, d.K, b, m, scale);
-            e = cudaGetLastError();
-        } else {
-            e = launch_pdl(eva_hadamard_kernel, dim3(d.K / b, B), dim3(thr), (size_t)b * sizeof(float), s, 0,
-                           reinterpret_cast<const __half *>(x), (const int8_t *)h->hsign, xrot, d.K, b, scale,
-                           independent);
-        }
+        e = launch_rotation(h, x, B, s, independent, xrot);
         if (e != cudaSuccess) return e;
         xin = xrot;
         x_f32 = 1;
@@ -1047,10 +1085,18 @@ eva_status_t eva_vq_linear_run_ex(eva_vq_linear_t h, const void *x, int32_t B, v
     if (use_dequant(h, B)) {
         size_t dsmem = 0;
         int dgrid = 0;
+        if (d.hadamard_block) {
+            // The dequantize kernel reads x~ (fp32) from the rotation kernel.
+            e = launch_rotation(h, x, B, s, independent, h->xrot);
+            if (e != cudaSuccess) return cuda_status(e);
+            p.x = h->xrot;
+            p.x_f32 = 1;
+            p.independent = 0;
+        }
         e = launch_dequant(h, p, B, s, &dsmem, &dgrid);
         if (e != cudaSuccess) return cuda_status(e);
         h->last_grid = dgrid;
-        h->last_kernels = 1;
+        h->last_kernels = d.hadamard_block ? 2 : 1;
         h->last_path = EVA_PATH_DEQUANT_MMA;
         return EVA_OK;
     }
@@ -1078,12 +1124,15 @@ eva_status_t eva_vq_linear_run_group(const eva_vq_linear_t *hs, const void *cons
     }
     const eva_vq_desc &d0 = hs[0]->desc;
     const int independent = (flags & EVA_RUN_INDEPENDENT) ? 1 : 0;
-    // Layers of one shape on the dequantize path (one shared codebook each):
-    // one launch of the dequantize kernel.
-    bool dq_one = use_dequant(hs[0], B) && !d0.codebook_rows && count > 1;
+    // Layers of one shape on the dequantize path (one shared codebook each, no
+    // residual, no rotation): one launch of the dequantize kernel.
+    const auto dq_plain = [](const eva_vq_desc &d) {
+        return !d.codebook_rows && !d.residual_group && !d.hadamard_block;
+    };
+    bool dq_one = use_dequant(hs[0], B) && dq_plain(d0) && count > 1;
     for (int i = 1; i < count && dq_one; ++i) {
         const eva_vq_desc &d = hs[i]->desc;
-        dq_one = use_dequant(hs[i], B) && !d.codebook_rows && d.N == d0.N && d.K == d0.K &&
+        dq_one = use_dequant(hs[i], B) && dq_plain(d) && d.N == d0.N && d.K == d0.K &&
                  d.out_dtype == d0.out_dtype && hs[i]->dq[B > 8 ? 1 : 0].Gs == hs[0]->dq[B > 8 ? 1 : 0].Gs &&
                  hs[i]->dq[B > 8 ? 1 : 0].Gt == hs[0]->dq[B > 8 ? 1 : 0].Gt &&
                  hs[i]->dq[B > 8 ? 1 : 0].smem == hs[0]->dq[B > 8 ? 1 : 0].smem;
@@ -1204,12 +1253,15 @@ eva_status_t eva_vq_linear_run_noalloc(eva_vq_linear_t h, const void *x, int32_t
     // A Paley rotation block has no standalone-kernel route that matches the
     // fused rotation bit for bit at every size, so it stays fused (no scratch).
     const bool fused_rot = paley_m(d.hadamard_block) != 0;
-    if (d.hadamard_block && !fused_rot && (size_t)B * d.K * sizeof(float) > kStaticScratchBytes)
-        return EVA_ERR_SCRATCH_TOO_SMALL;
+    // The dequantize path reads x~ from the standalone rotation kernel
+    // whatever the block; the lookup path fuses the Paley blocks.
+    const bool dq = use_dequant(h, B);
+    const bool rot_scratch = d.hadamard_block && (!fused_rot || dq);
+    if (rot_scratch && (size_t)B * d.K * sizeof(float) > kStaticScratchBytes) return EVA_ERR_SCRATCH_TOO_SMALL;
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev != h->device) return EVA_ERR_INVALID_ARG;
     float *scratch = nullptr;
-    if (d.hadamard_block && !fused_rot) {
+    if (rot_scratch) {
         const eva_status_t st = static_scratch(dev, &scratch);
         if (st != EVA_OK) return st;
     }
@@ -1248,7 +1300,12 @@ eva_status_t eva_vq_linear_run_noalloc(eva_vq_linear_t h, const void *x, int32_t
     return EVA_ERR_UNSUPPORTED;   // the checked build validates the handle path only
 #endif
     cudaError_t e;
-    if (fused_rot) {
+    if (dq && d.hadamard_block) {
+        e = launch_rotation(h, x, B, s, 0, scratch);
+        if (e != cudaSuccess) return cuda_status(e);
+        p.x = scratch;
+        p.x_f32 = 1;
+    } else if (fused_rot) {
         p.rot_b = d.hadamard_block;
         p.rot_m = paley_m(d.hadamard_block);
         p.h28 = h->h28;
@@ -1264,13 +1321,13 @@ eva_status_t eva_vq_linear_run_noalloc(eva_vq_linear_t h, const void *x, int32_t
         p.x = scratch;
         p.x_f32 = 1;
     }
-    if (use_dequant(h, B)) {   // no rotation on this path, so no scratch either
+    if (dq) {
         size_t dsmem = 0;
         int dgrid = 0;
         e = launch_dequant(h, p, B, s, &dsmem, &dgrid);
         if (e != cudaSuccess) return cuda_status(e);
         h->last_grid = dgrid;
-        h->last_kernels = 1;
+        h->last_kernels = d.hadamard_block ? 2 : 1;
         h->last_path = EVA_PATH_DEQUANT_MMA;
         return EVA_OK;
     }

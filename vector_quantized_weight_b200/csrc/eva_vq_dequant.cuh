@@ -53,12 +53,16 @@ __device__ __forceinline__ void build_codebook_table(const LookupParams &p, int 
 // The 16-token instances with running sums in shared memory take more than
 // half the SM's shared memory anyway, so they keep one CTA per SM and the
 // registers that go with it.
-template <bool GROUPED, int NTG, bool DIRECT>
-constexpr int kDequantMinBlocks = (NTG == 2 && (GROUPED || !DIRECT)) ? 1 : 2;
+template <bool GROUPED, int NTG, bool DIRECT, bool RESID = false>
+constexpr int kDequantMinBlocks = (RESID || (NTG == 2 && (GROUPED || !DIRECT))) ? 1 : 2;
 
 // The whole per-CTA program; eva_bid is the CTA's index within its layer.
-template <bool GROUPED, int NTG, bool DIRECT>
+// RESID: the 1-bit sign residual of the 3-bit SRAM-lookup article rides on
+// the rebuilt weights, w = WC[WI] + alpha sigma (one shared codebook); a
+// rotated layer's x~ comes in as fp32 (x_f32) from the rotation kernel.
+template <bool GROUPED, int NTG, bool DIRECT, bool RESID = false>
 __device__ __forceinline__ void dequant_body(const LookupParams &p, const int eva_bid) {
+    static_assert(!(RESID && GROUPED), "the residual rides on one shared codebook");
     constexpr int TT = 8 * NTG;                         // tokens per pass
     constexpr uint32_t BLK = kTileRows * TT * 4u;       // bytes of one tile's running sums
     // A tile's block in the reduction stage.  Sums pushed from registers (8
@@ -144,7 +148,24 @@ __device__ __forceinline__ void dequant_body(const LookupParams &p, const int ev
             const int chunk = i & 31, n = (i >> 5) % TT, sl = i / (32 * TT);
             const int tok = p0 + n, k0 = (s0 + sl) * kSliceK + 8 * chunk;
             uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (tok < p.B && k0 + 8 <= p.K && ((((size_t)tok * p.K + k0) & 7) == 0)) {
+            if (p.x_f32 && tok < p.B && k0 + 8 <= p.K) {
+                const float4 *xp = reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(p.x) +
+                                                                    (size_t)tok * p.K + k0);
+                if (!EVA_BAD_G(BUF_X, xp, 32)) {
+                    const float4 a = __ldcg(xp), b = __ldcg(xp + 1);
+                    v = make_uint4(pack_half2(a.x, a.y), pack_half2(a.z, a.w), pack_half2(b.x, b.y),
+                                   pack_half2(b.z, b.w));
+                }
+            } else if (p.x_f32 && tok < p.B && k0 < p.K) {
+                float f[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float *xp = reinterpret_cast<const float *>(p.x) + (size_t)tok * p.K + k0 + e;
+                    f[e] = (k0 + e < p.K && !EVA_BAD_G(BUF_X, xp, 4)) ? __ldcg(xp) : 0.f;
+                }
+                v = make_uint4(pack_half2(f[0], f[1]), pack_half2(f[2], f[3]), pack_half2(f[4], f[5]),
+                               pack_half2(f[6], f[7]));
+            } else if (tok < p.B && k0 + 8 <= p.K && ((((size_t)tok * p.K + k0) & 7) == 0)) {
                 const uint4 *xp = reinterpret_cast<const uint4 *>(reinterpret_cast<const __half *>(p.x) +
                                                                   (size_t)tok * p.K + k0);
                 if (!EVA_BAD_G(BUF_X, xp, 16)) v = __ldcg(xp);
@@ -360,6 +381,34 @@ __device__ __forceinline__ void dequant_body(const LookupParams &p, const int ev
 #pragma unroll
                         for (int k = 0; k < 8; ++k) rot[k] = nr[k];
                     }
+                    // Residual: the sign bits of rows g, g + 8 over this slice
+                    // (word w: slice inputs 32 w .. 32 w + 31, LSB first) and their
+                    // alpha for the slice's two 128-input groups.
+                    uint32_t sgw[2][8];
+                    __half alf[2][2];
+                    if constexpr (RESID) {
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int o = kTileRows * (t0 + tl) + g + 8 * h;
+                            const int rb = o >> 7, rr = o & 127;
+#pragma unroll
+                            for (int i4 = 0; i4 < 4; ++i4) {
+                                const int kb = 4 * s + i4;
+                                uint2 v2 = make_uint2(0u, 0u);
+                                const uint8_t *sp = p.sgb + (((size_t)rb * p.KB + kb) * 128 + rr) * 8;   // 128-row blocks
+                                if (kb < p.KB && !EVA_BAD_G(BUF_SG, sp, 8)) v2 = __ldg(reinterpret_cast<const uint2 *>(sp));
+                                sgw[h][2 * i4] = v2.x;
+                                sgw[h][2 * i4 + 1] = v2.y;
+                            }
+                            const int NG = p.K / 128;
+#pragma unroll
+                            for (int a = 0; a < 2; ++a) {
+                                const int gi = 2 * s + a;
+                                const __half *ap = p.al_rm + (size_t)o * NG + gi;
+                                alf[h][a] = (o < p.N && gi < NG && !EVA_BAD_G(BUF_AL, ap, 2)) ? __ldg(ap) : __float2half(0.f);
+                            }
+                        }
+                    }
                     // Two MMA accumulation chains per token group, one where the
                     // registers of two CTAs per SM would not hold two (16 tokens,
                     // sums pushed from registers).
@@ -377,8 +426,25 @@ __device__ __forceinline__ void dequant_body(const LookupParams &p, const int ev
                         const uint32_t cg = beta < 8 ? (w & 0xFFu) : ((w >> 16) & 0xFFu);
                         const uint32_t ch = beta < 8 ? ((w >> 8) & 0xFFu) : (w >> 24);
                         const uint32_t og = TAB_OFF + (cg << 7) + lofs, oh = TAB_OFF + (ch << 7) + lofs;
-                        const uint2 ag = EVA_BAD_S(og) ? make_uint2(0u, 0u) : lds64(og);
-                        const uint2 ah = EVA_BAD_S(oh) ? make_uint2(0u, 0u) : lds64(oh);
+                        uint2 ag = EVA_BAD_S(og) ? make_uint2(0u, 0u) : lds64(og);
+                        uint2 ah = EVA_BAD_S(oh) ? make_uint2(0u, 0u) : lds64(oh);
+                        if constexpr (RESID) {
+                            // Sub-vector 4 beta + q: sign nibble in word beta / 2 at bit
+                            // 16 (beta & 1) + 4 q; alpha of group beta / 8 of the slice.
+                            const int sh = 16 * (beta & 1) + 4 * q;
+                            auto add_resid = [&](uint2 &w, uint32_t nib, __half a) {
+                                const __half na = __hneg(a);
+                                const __half2 lo = __halves2half2((nib & 1u) ? a : na, (nib & 2u) ? a : na);
+                                const __half2 hi = __halves2half2((nib & 4u) ? a : na, (nib & 8u) ? a : na);
+                                __half2 x0 = *reinterpret_cast<const __half2 *>(&w.x), x1 = *reinterpret_cast<const __half2 *>(&w.y);
+                                x0 = __hadd2(x0, lo);
+                                x1 = __hadd2(x1, hi);
+                                w.x = *reinterpret_cast<const uint32_t *>(&x0);
+                                w.y = *reinterpret_cast<const uint32_t *>(&x1);
+                            };
+                            add_resid(ag, (sgw[0][beta >> 1] >> sh) & 0xFu, alf[0][beta >> 3]);
+                            add_resid(ah, (sgw[1][beta >> 1] >> sh) & 0xFu, alf[1][beta >> 3]);
+                        }
 #pragma unroll
                         for (int t = 0; t < NTG; ++t)
                             mma_f16_k16(acc[t][kChains == 1 ? 0 : (beta & 1)], ag.x, ah.x, ag.y, ah.y, xb[t][beta].x, xb[t][beta].y);
@@ -477,10 +543,10 @@ __device__ __forceinline__ void dequant_body(const LookupParams &p, const int ev
 #endif
 }
 
-template <bool GROUPED, int NTG, bool DIRECT>
-__global__ void __launch_bounds__(kThreads, kDequantMinBlocks<GROUPED, NTG, DIRECT>)
+template <bool GROUPED, int NTG, bool DIRECT, bool RESID = false>
+__global__ void __launch_bounds__(kThreads, kDequantMinBlocks<GROUPED, NTG, DIRECT, RESID>)
     eva_dequant_kernel(const LookupParams p) {
-    dequant_body<GROUPED, NTG, DIRECT>(p, blockIdx.x);
+    dequant_body<GROUPED, NTG, DIRECT, RESID>(p, blockIdx.x);
 }
 
 // Several layers of one shape (one shared codebook each) in one launch, as

@@ -46,6 +46,10 @@ struct LookupParams {
     int independent;         // neither x nor y is touched by the preceding kernel:
                              // run without waiting for it (wait only before exit)
     int acc_tiles;           // row tiles of the largest CTA (shared-memory layout)
+    const uint8_t *sgb;      // dequantize path with residual: signs in the row-block layout
+                             // [ceil(N/128)][KB][128][8] bytes (KB = K / 64 stages)
+    const __half *al_rm;     // dequantize path with residual: alpha [N][K/128]
+    int KB;
     int wi_staged;           // leading row tiles whose first-slice indices are copied
                              // into shared memory by one bulk copy in the prologue
     int *status;             // device error word (bit 0: the wait for the staged index

@@ -62,10 +62,11 @@ typedef enum {
     EVA_PATH_AUTO = 0,        /* pick per call from B and the codebook layout   */
     EVA_PATH_OC_LOOKUP = 1,   /* output codebook in shared memory + lookups     */
     EVA_PATH_DEQUANT_MMA = 2, /* codebook gather into warp-level tensor-core
-                                 operands (mma.sync; 8-bit indices, no residual,
-                                 no rotation); AUTO takes it for B >= 3 (B >= 2
-                                 with per-group codebooks) when the layer allows
-                                 it and EVA_PATH_TCGEN05 does not               */
+                                 operands (mma.sync; 8-bit indices; residual
+                                 and rotation with one shared codebook only);
+                                 AUTO takes it for B >= 3 (B >= 2 with
+                                 per-group codebooks) when the layer allows it
+                                 and EVA_PATH_TCGEN05 does not                  */
     EVA_PATH_TCGEN05 = 3      /* weights rebuilt from the codebook into tensor
                                  memory and multiplied by tcgen05.mma (fp32
                                  accumulation in tensor memory), residual and

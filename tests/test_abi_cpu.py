@@ -58,8 +58,8 @@ def _create(desc, wc=0x1000, wi=0x2000, signs=None, alpha=None, hsign=None):
     (dict(d=3), eva_vq.EVA_ERR_UNSUPPORTED),
     (dict(index_bits=6), eva_vq.EVA_ERR_UNSUPPORTED),
     (dict(index_bits=4, path=2), eva_vq.EVA_ERR_UNSUPPORTED),   # 4-bit: the lookup path only
-    (dict(path=2, residual_group=128, codebook_rows=16), eva_vq.EVA_ERR_UNSUPPORTED),  # dequantize: residual,
-    (dict(path=2, K=520, hadamard_block=8), eva_vq.EVA_ERR_UNSUPPORTED),               # rotation need one codebook, K % 64 == 0
+    (dict(path=2, residual_group=128, codebook_rows=16), eva_vq.EVA_ERR_UNSUPPORTED),  # dequantize: residual and
+    (dict(path=2, hadamard_block=128, codebook_rows=16), eva_vq.EVA_ERR_UNSUPPORTED),  # rotation need one codebook
     (dict(index_bits=4, K=516), eva_vq.EVA_ERR_INVALID_ARG),
     (dict(N=0), eva_vq.EVA_ERR_INVALID_ARG),
     (dict(K=510), eva_vq.EVA_ERR_INVALID_ARG),

@@ -269,11 +269,17 @@ def test_dequant_path_ragged_batches(N, K, cbr):
     (synth.LayerShape("gemma_rotK", 3584, 3584, residual_group=128, hadamard_block=3584), (2, 16)),
     (synth.LayerShape("resid_only", 384, 1024, residual_group=128), (5, 17)),
     (synth.LayerShape("ragged", 200, 1152, residual_group=128, hadamard_block=64), (6,)),
+    (synth.LayerShape("rot_only", 136, 520, hadamard_block=8), (3, 11)),
+    (synth.LayerShape("syl4096", 256, 8192, residual_group=128, hadamard_block=4096), (3, 12)),
+    (synth.LayerShape("syl1024", 512, 4096, residual_group=128, hadamard_block=1024), (5, 13)),
+    (synth.LayerShape("syl256", 128, 768, hadamard_block=256), (4,)),
 ])
 def test_dequant_path_with_residual_and_rotation(shape, Bs):
     """The dequantize path carries the 1-bit sign residual (signed alpha
-    included) and reads the rotated input from the rotation kernel (Sylvester
-    and Paley blocks, a K range ending mid-slice): every row against the
+    included) and the rotated input: Sylvester blocks of 64 to 4096 rotated
+    on chip with the residual where a CTA takes one slice, through the
+    rotation kernel otherwise, without the residual (8, 256) and for an
+    order-K Paley block; K ranges ending mid-slice; every row against the
     oracle, the status word clean."""
     import torch
     from vector_quantized_weight_b200 import eva_vq

@@ -80,10 +80,9 @@ def test_tcgen05_integer_inputs_exact():
 
 def test_auto_path_by_batch():
     """AUTO: lookups below three tokens (two with per-group codebooks); from
-    there on the warp-level dequantize path where the layer allows it, the
-    tcgen05 path past 32 tokens with one shared codebook; a residual / rotated
-    layer keeps the lookup path below eight tokens and takes tcgen05 from
-    there."""
+    there on the warp-level dequantize path, the tcgen05 path past 32 tokens
+    with one shared codebook -- 3.125-bit layers (rotation, residual)
+    included."""
     from vector_quantized_weight_b200 import eva_vq
     plain = synth.LayerShape("l7b", 4096, 4096)
     gemma = synth.LayerShape("gemma", 3584, 3584, residual_group=128, hadamard_block=512)
@@ -91,8 +90,9 @@ def test_auto_path_by_batch():
                                   (3, eva_vq.EVA_PATH_DEQUANT_MMA), (16, eva_vq.EVA_PATH_DEQUANT_MMA),
                                   (32, eva_vq.EVA_PATH_DEQUANT_MMA), (33, eva_vq.EVA_PATH_TCGEN05),
                                   (64, eva_vq.EVA_PATH_TCGEN05))),
-                         (gemma, ((1, eva_vq.EVA_PATH_OC_LOOKUP), (4, eva_vq.EVA_PATH_OC_LOOKUP),
-                                  (8, eva_vq.EVA_PATH_TCGEN05))),
+                         (gemma, ((1, eva_vq.EVA_PATH_OC_LOOKUP), (2, eva_vq.EVA_PATH_OC_LOOKUP),
+                                  (3, eva_vq.EVA_PATH_DEQUANT_MMA), (16, eva_vq.EVA_PATH_DEQUANT_MMA),
+                                  (32, eva_vq.EVA_PATH_DEQUANT_MMA), (33, eva_vq.EVA_PATH_TCGEN05))),
                          (synth.LayerShape("l70b", 8192, 8192, codebook_rows=128),
                           ((1, eva_vq.EVA_PATH_OC_LOOKUP), (2, eva_vq.EVA_PATH_DEQUANT_MMA),
                            (8, eva_vq.EVA_PATH_DEQUANT_MMA), (32, eva_vq.EVA_PATH_DEQUANT_MMA)))):

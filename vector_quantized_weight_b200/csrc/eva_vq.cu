@@ -52,7 +52,8 @@ struct eva_vq_linear {
     int tc_gs[4] = {0, 0, 0, 0};
     uint8_t *wib = nullptr, *sgb = nullptr;
     __half *al_rm = nullptr;
-    float *xrot = nullptr;
+    float *xrot = nullptr;              // also the dequantize path's x~
+    uint8_t *sgd = nullptr;             // dequantize path: sign units in its lane order
     uint8_t *wi = nullptr;              // repacked indices
     uint8_t *sg = nullptr;              // repacked signs
     __half *al = nullptr;               // repacked alpha
@@ -162,10 +163,8 @@ eva_status_t validate_desc(const eva_vq_desc *d) {
     if (d->path != EVA_PATH_AUTO && d->path != EVA_PATH_OC_LOOKUP && d->path != EVA_PATH_DEQUANT_MMA &&
         d->path != EVA_PATH_TCGEN05)
         return EVA_ERR_INVALID_ARG;
-    // The dequantize path takes a residual or a rotation with one shared
-    // codebook and the tcgen05 path's row-block data (K a multiple of 64).
-    if (d->path == EVA_PATH_DEQUANT_MMA && (d->residual_group || d->hadamard_block) &&
-        (d->codebook_rows || !tc_layer_ok(*d)))
+    // The dequantize path takes a residual or a rotation with one shared codebook.
+    if (d->path == EVA_PATH_DEQUANT_MMA && (d->residual_group || d->hadamard_block) && d->codebook_rows)
         return EVA_ERR_UNSUPPORTED;
     if (d->path == EVA_PATH_TCGEN05 && !tc_layer_ok(*d)) return EVA_ERR_UNSUPPORTED;
     return EVA_OK;
@@ -412,8 +411,9 @@ int dequant_min_batch(const eva_vq_desc &d) { return d.codebook_rows ? kDequantM
 
 // Dynamic shared memory of the dequantize kernel: the replicated codebook,
 // the x stage of up to nsl slices, the running sums, the reduction stage, the
-// staging mbarrier and `staged` index units.
-size_t dequant_smem(int nsl, int tiles, int gs, int ntg, int staged = 0) {
+// staging mbarrier and `staged` index units (with their sign and alpha units
+// when the layer has the residual).
+size_t dequant_smem(int nsl, int tiles, int gs, int ntg, int staged = 0, bool resid = false) {
     const size_t blk = (size_t)kTileRows * 8 * ntg * 4;
     const size_t xs = ((size_t)nsl * 8 * ntg * kXTokStride + 127) & ~(size_t)127;
     const size_t nslot = (size_t)(tiles + gs - 1) / gs;
@@ -422,7 +422,7 @@ size_t dequant_smem(int nsl, int tiles, int gs, int ntg, int staged = 0) {
     const size_t acc = nsl == 1 ? 0 : (size_t)tiles * blk;
     const size_t blk_s = nsl == 1 ? (size_t)kTileRows * (8 * ntg + 2) * 4 : blk;
     const size_t base = (size_t)kTabBytes + xs + acc + nslot * gs * blk_s;
-    return ((base + 127) & ~(size_t)127) + 128 + (size_t)staged * kUnitBytes;
+    return ((base + 127) & ~(size_t)127) + 128 + (size_t)staged * (kUnitBytes + (resid ? kDqResidUnitBytes : 0));
 }
 
 // Same search as plan_grid, for the dequantize kernel (one CTA per SM, every
@@ -469,11 +469,13 @@ void plan_dequant(eva_vq_linear *h, int ntg) {
     // is staged, and at least half the SM's shared memory keeps a second CTA
     // of the same layer off the SM (two on one SM stretched the slowest CTA's
     // tile loop from 12.8 to 19.8 us for 8192^2 at one token).
+    const bool resid = h->desc.residual_group != 0;
     const size_t base = dequant_smem(nsl, tiles, pl.Gs, ntg);
     const size_t half = (size_t)h->smem_per_sm / 2 - (size_t)h->smem_reserved;
     const size_t budget = h->tiles_per_cb ? (size_t)h->smem_optin : half;
-    pl.staged = base < budget ? (int)std::min<size_t>((size_t)nsl * tiles, (budget - base) / kUnitBytes) : 0;
-    pl.smem = dequant_smem(nsl, tiles, pl.Gs, ntg, pl.staged);
+    const size_t ubytes = kUnitBytes + (resid ? kDqResidUnitBytes : 0);
+    pl.staged = base < budget ? (int)std::min<size_t>((size_t)nsl * tiles, (budget - base) / ubytes) : 0;
+    pl.smem = dequant_smem(nsl, tiles, pl.Gs, ntg, pl.staged, resid);
     pl.smem_nostage = dequant_smem(nsl, tiles, pl.Gs, ntg);
     if (h->tiles_per_cb) pl.smem = std::max(pl.smem, half + 1024);
     h->dq[ntg - 1] = pl;
@@ -548,8 +550,30 @@ void apply_injection(eva_vq_linear *h, LookupParams &p) {
     }
 }
 
-// Launch the dequantize kernel for a call whose common parameters are in p.
-// The dequantize kernel's fields of a call's parameters (its plan for B).
+bool dequant_direct(const eva_vq_linear *h, int B) {
+    const eva_vq_linear::Plan &pl = h->dq[B > 8 ? 1 : 0];
+    return (h->S + pl.Gs - 1) / pl.Gs == 1;   // the same rule as dequant_smem's
+}
+
+// The dequantize kernel's residual instances rotate x on chip (the 3.125-bit
+// format has both) where that is cheap: a Sylvester block of at most 1024
+// inputs (one round of four sub-block loads per slice and token) and one
+// slice per CTA.  Measured on B200, 3.125-bit 3584 x 3584 (block 512), one
+// layer waiting for the previous one: 8.7 against 11.0 us at 4 tokens, 12.0
+// against 19.4 at 16.  Otherwise x~ comes from the standalone rotation
+// kernel: with several slices per CTA of a 2048 block the warps redo the
+// sub-block transforms one latency after the other (3584 x 14336 at 16
+// tokens: 64.0 on chip against 41.2 us); a Paley block's transform spans the
+// whole block; a rotated layer without the residual keeps the other
+// instances' registers as they are.
+bool dq_rotates_on_chip(const eva_vq_linear *h, int B) {
+    const eva_vq_desc &d = h->desc;
+    return d.hadamard_block && d.hadamard_block <= 1024 && !paley_m(d.hadamard_block) && d.residual_group &&
+           dequant_direct(h, B);
+}
+
+// The dequantize kernel's fields of a call's parameters (its plan for B);
+// p.x is fp16 x, or x~ in fp32 (x_f32) from the rotation kernel.
 void dequant_params(eva_vq_linear *h, LookupParams &p, int B) {
     const int ntg = B > 8 ? 2 : 1;
     const eva_vq_linear::Plan &pl = h->dq[ntg - 1];
@@ -558,27 +582,27 @@ void dequant_params(eva_vq_linear *h, LookupParams &p, int B) {
     p.acc_tiles = (h->T + pl.Gt - 1) / pl.Gt;
     p.wi_staged = pl.staged;
     p.rot_b = 0;
-    p.sgb = h->sgb;
-    p.al_rm = h->al_rm;
-    p.KB = h->desc.K / kTcStageK;
+    p.rot_m = 0;
+    if (dq_rotates_on_chip(h, B) && !p.x_f32) {
+        p.rot_b = h->desc.hadamard_block;
+        p.hs = h->hsign;
+        p.rot_scale = (float)(1.0 / std::sqrt((double)h->desc.hadamard_block));
+    }
+    p.sgd = h->sgd;
+    p.al = h->al;
     apply_injection(h, p);
 #ifdef EVA_DEVICE_CHECKS
     p.smem_bytes = (unsigned)pl.smem;
     if (h->desc.residual_group) {
-        const int R128 = (h->desc.N + 127) / 128;
-        p.chk_base[BUF_SG] = h->sgb;
-        p.chk_bytes[BUF_SG] = (unsigned long long)R128 * 128 * (h->desc.K / 8);
-        p.chk_base[BUF_AL] = h->al_rm;
-        p.chk_bytes[BUF_AL] = (unsigned long long)h->desc.N * (h->desc.K / 128) * 2;
+        const unsigned long long units = (unsigned long long)h->S * h->T;
+        p.chk_base[BUF_SG] = h->sgd;
+        p.chk_bytes[BUF_SG] = units * kDqSignUnitBytes;
+        p.chk_base[BUF_AL] = h->al;
+        p.chk_bytes[BUF_AL] = units * kAlphaUnitHalves * 2;
     }
     p.chk_base[BUF_X] = p.x;
     p.chk_bytes[BUF_X] = (unsigned long long)B * h->desc.K * (p.x_f32 ? 4 : 2);
 #endif
-}
-
-bool dequant_direct(const eva_vq_linear *h, int B) {
-    const eva_vq_linear::Plan &pl = h->dq[B > 8 ? 1 : 0];
-    return (h->S + pl.Gs - 1) / pl.Gs == 1;   // the same rule as dequant_smem's
 }
 
 cudaError_t launch_dequant(eva_vq_linear *h, LookupParams p, int B, cudaStream_t s, size_t *smem_out,
@@ -601,16 +625,20 @@ bool use_three_per_sm(const eva_vq_linear *h, int B, int independent) {
 
 // The tcgen05 path: forced, or AUTO from kDequantMinBatch tokens on.
 // AUTO (measured per batch on B200, one layer waiting for the previous one):
-//  - layers the warp-level dequantize path takes (no residual, no rotation):
-//    that path from kDequantMinBatch tokens on, except one shared codebook
-//    past two 16-token passes (kTcMinBatch), where tcgen05 wins (4096 x 4096:
-//    16.3 against 17.0 us at 32 tokens, 19.1 against 24.2 at 48, 21.3 against
-//    32.0 at 64; 11008 x 4096: 35.0 against 49.0 at 32, 62.0 against 65.1 at
-//    64); with per-group codebooks the warp-level path stays ahead (8192 x
-//    8192: 62.3 against 85.2 us at 32 tokens);
-//  - residual / rotated layers: the lookup path below kTcResidMinBatch tokens
-//    (3.125-bit 3584 x 3584: 15.4 against 22.0 us at 4 tokens), tcgen05 from
-//    there (24.7 against 55.5 us at 16).
+//  - the warp-level dequantize path from kDequantMinBatch tokens on, except
+//    with one shared codebook past two 16-token passes (kTcMinBatch), where
+//    tcgen05 wins (4096 x 4096: 16.3 against 17.0 us at 32 tokens, 19.1
+//    against 24.2 at 48, 21.3 against 32.0 at 64; 11008 x 4096: 35.0 against
+//    49.0 at 32, 62.0 against 65.1 at 64); with per-group codebooks the
+//    warp-level path stays ahead (8192 x 8192: 62.3 against 85.2 us at 32
+//    tokens).  The same split holds for 3.125-bit layers (Hadamard blocks,
+//    sign residual): 3584 x 3584 at 4 tokens 11.1 us against 16.0 (lookup)
+//    and 20.5 (tcgen05), at 16 19.4 against 24.1 (tcgen05), at 48 47.7
+//    against 30.6; 14336 x 3584 at 16 34.3 against 60.4, at 64 116.9 against
+//    110.6;
+//  - layers the warp-level path cannot take (residual or rotation with
+//    per-group codebooks): the lookup path below kTcResidMinBatch tokens,
+//    tcgen05 from there.
 // A tcgen05.mma of M = 128 rows takes about as long for N = 16 tokens as for
 // N = 64 (54-100 cycles per instruction in two single-thread probes), so the
 // tensor-core path pays off as the batch grows, while the warp-level MMA of 8
@@ -622,16 +650,13 @@ bool use_tc(const eva_vq_linear *h, int B) {
     if (!h->tc_ok) return false;
     if (h->desc.path == EVA_PATH_TCGEN05) return true;
     if (h->desc.path != EVA_PATH_AUTO || B < kDequantMinBatch) return false;
-    if (!h->dq_ok || h->desc.residual_group || h->desc.hadamard_block) return B >= kTcResidMinBatch;
+    if (!h->dq_ok) return B >= kTcResidMinBatch;
     return B >= kTcMinBatch && h->desc.codebook_rows == 0;
 }
 
 bool use_dequant(const eva_vq_linear *h, int B) {
     if (!h->dq_ok || use_tc(h, B)) return false;
     if (h->desc.path == EVA_PATH_DEQUANT_MMA) return true;
-    // Residual / rotated layers: only when forced (AUTO keeps the lookup and
-    // tcgen05 paths for them).
-    if (h->desc.residual_group || h->desc.hadamard_block) return false;
     return h->desc.path == EVA_PATH_AUTO && B >= dequant_min_batch(h->desc);
 }
 
@@ -694,7 +719,7 @@ void free_handle(eva_vq_linear *h) {
         if (hg.exec) cudaGraphExecDestroy(hg.exec);
     if (h->capture_stream) cudaStreamDestroy(h->capture_stream);
     void *ptrs[] = {h->wi, h->sg, h->al, h->wc, h->hsign, h->h28, h->status, h->x_stage,
-                    h->y_stage, h->timeline, h->wib, h->sgb, h->al_rm, h->xrot};
+                    h->y_stage, h->timeline, h->wib, h->sgb, h->al_rm, h->xrot, h->sgd};
     for (void *p : ptrs)
         if (p) cudaFree(p);
     delete h;
@@ -783,12 +808,11 @@ eva_status_t eva_vq_linear_create(eva_vq_linear_t *out, const eva_vq_desc *desc,
     plan_grid(h, 0);
     if (desc->max_batch > 1) plan_grid(h, 1);
     int max_grid = std::max(h->plan[0].Gs * h->plan[0].Gt, h->plan[1].Gs * h->plan[1].Gt);
-    // Residual and rotated layers on the dequantize path read the row-block
-    // signs, the canonical alpha and the rotated x the tcgen05 path keeps.
+    // Residual and rotated layers on the dequantize path (one shared codebook):
+    // its own sign units beside the lookup's alpha units, and the rotated x in
+    // the workspace the tcgen05 path uses too.
     const bool dq_resrot = desc->residual_group || desc->hadamard_block;
-    if (desc->index_bits == 8 &&
-        (!dq_resrot || (tc_layer_ok(*desc) && !desc->codebook_rows &&
-                        (!desc->residual_group || desc->residual_group == 128))) &&
+    if (desc->index_bits == 8 && (!dq_resrot || !desc->codebook_rows) &&
         (desc->path == EVA_PATH_DEQUANT_MMA ||
          (desc->path == EVA_PATH_AUTO && desc->max_batch >= dequant_min_batch(*desc)))) {
         plan_dequant(h, 1);
@@ -817,14 +841,16 @@ eva_status_t eva_vq_linear_create(eva_vq_linear_t *out, const eva_vq_desc *desc,
     }
     chk(dalloc(&h->wi, (size_t)units * h->unit_bytes, nullptr));
     const int R128 = (N + kTcRows - 1) / kTcRows;
-    if (h->tc_ok || (h->dq_ok && dq_resrot)) {
+    if (h->tc_ok) {
         chk(dalloc(&h->wib, (size_t)R128 * kTcRows * h->J, nullptr));
         if (desc->residual_group) {
             chk(dalloc(&h->sgb, (size_t)R128 * kTcRows * (K / 8), nullptr));
             chk(dalloc(&h->al_rm, (size_t)N * (K / desc->residual_group) * sizeof(__half), nullptr));
         }
-        if (desc->hadamard_block) chk(dalloc(&h->xrot, (size_t)desc->max_batch * K * sizeof(float), &ws));
     }
+    if ((h->tc_ok || h->dq_ok) && desc->hadamard_block)
+        chk(dalloc(&h->xrot, (size_t)desc->max_batch * K * sizeof(float), &ws));
+    if (h->dq_ok && desc->residual_group) chk(dalloc(&h->sgd, (size_t)units * kDqSignUnitBytes, nullptr));
     chk(dalloc(&h->wc, (size_t)h->G * h->ncent * kD * sizeof(__half), nullptr));
     if (desc->residual_group) {
         chk(dalloc(&h->sg, (size_t)units * kSignUnitBytes, nullptr));
@@ -863,7 +889,12 @@ eva_status_t eva_vq_linear_create(eva_vq_linear_t *out, const eva_vq_desc *desc,
             reinterpret_cast<const __half *>(alpha), h->al, N, K / desc->residual_group, h->T, ab);
         chk(cudaGetLastError());
     }
-    if (h->tc_ok || (h->dq_ok && dq_resrot)) {
+    if (h->dq_ok && desc->residual_group) {
+        const long long sb = units * kDqSignUnitBytes;
+        eva_repack_signs_dq_kernel<<<blocks_for(sb, thr), thr, 0, s>>>(signs, h->sgd, N, K, h->T, sb);
+        chk(cudaGetLastError());
+    }
+    if (h->tc_ok) {
         const long long nb = (long long)R128 * kTcRows * h->J;
         eva_repack_wi_rowblock_kernel<<<blocks_for(nb, thr), thr, 0, s>>>(wi, h->wib, N, h->J, nb);
         chk(cudaGetLastError());
@@ -991,12 +1022,10 @@ cudaError_t launch_rotation(const eva_vq_linear *h, const void *x, int B, cudaSt
     const eva_vq_desc &d = h->desc;
     const int b = d.hadamard_block, m = paley_m(b), thr = std::min(b / 2, 1024);
     const float scale = (float)(1.0 / std::sqrt((double)b));
-    if (m) {
-        // Launched in plain stream order (it reads x as soon as it starts).
-        eva_paley_rows_kernel<<<dim3(d.K / b, B), thr, (size_t)b * sizeof(float), s>>>(
-            reinterpret_cast<const __half *>(x), h->hsign, h->h28, xrot, d.K, b, m, scale);
-        return cudaGetLastError();
-    }
+    if (m)
+        return launch_pdl(eva_paley_x_kernel, dim3(28 * (d.K / b), B), dim3(m), (size_t)m * sizeof(float), s, 0,
+                          reinterpret_cast<const __half *>(x), (const int8_t *)h->hsign, (const int8_t *)h->h28,
+                          xrot, d.K, b, m, scale, independent);
     return launch_pdl(eva_hadamard_kernel, dim3(d.K / b, B), dim3(thr), (size_t)b * sizeof(float), s, 0,
                       reinterpret_cast<const __half *>(x), (const int8_t *)h->hsign, xrot, d.K, b, scale,
                       independent);
@@ -1085,7 +1114,8 @@ eva_status_t eva_vq_linear_run_ex(eva_vq_linear_t h, const void *x, int32_t B, v
     if (use_dequant(h, B)) {
         size_t dsmem = 0;
         int dgrid = 0;
-        if (d.hadamard_block) {
+        const bool rot_kernel = d.hadamard_block && !dq_rotates_on_chip(h, B);
+        if (rot_kernel) {
             // The dequantize kernel reads x~ (fp32) from the rotation kernel.
             e = launch_rotation(h, x, B, s, independent, h->xrot);
             if (e != cudaSuccess) return cuda_status(e);
@@ -1096,7 +1126,7 @@ eva_status_t eva_vq_linear_run_ex(eva_vq_linear_t h, const void *x, int32_t B, v
         e = launch_dequant(h, p, B, s, &dsmem, &dgrid);
         if (e != cudaSuccess) return cuda_status(e);
         h->last_grid = dgrid;
-        h->last_kernels = d.hadamard_block ? 2 : 1;
+        h->last_kernels = rot_kernel ? 2 : 1;
         h->last_path = EVA_PATH_DEQUANT_MMA;
         return EVA_OK;
     }
@@ -1253,10 +1283,11 @@ eva_status_t eva_vq_linear_run_noalloc(eva_vq_linear_t h, const void *x, int32_t
     // A Paley rotation block has no standalone-kernel route that matches the
     // fused rotation bit for bit at every size, so it stays fused (no scratch).
     const bool fused_rot = paley_m(d.hadamard_block) != 0;
-    // The dequantize path reads x~ from the standalone rotation kernel
-    // whatever the block; the lookup path fuses the Paley blocks.
+    // The dequantize path rotates Sylvester blocks on chip and reads a Paley
+    // block's x~ from the standalone rotation kernel; the lookup path the
+    // other way round.
     const bool dq = use_dequant(h, B);
-    const bool rot_scratch = d.hadamard_block && (!fused_rot || dq);
+    const bool rot_scratch = d.hadamard_block && (dq ? !dq_rotates_on_chip(h, B) : !fused_rot);
     if (rot_scratch && (size_t)B * d.K * sizeof(float) > kStaticScratchBytes) return EVA_ERR_SCRATCH_TOO_SMALL;
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev != h->device) return EVA_ERR_INVALID_ARG;
@@ -1300,11 +1331,13 @@ eva_status_t eva_vq_linear_run_noalloc(eva_vq_linear_t h, const void *x, int32_t
     return EVA_ERR_UNSUPPORTED;   // the checked build validates the handle path only
 #endif
     cudaError_t e;
-    if (dq && d.hadamard_block) {
-        e = launch_rotation(h, x, B, s, 0, scratch);
-        if (e != cudaSuccess) return cuda_status(e);
-        p.x = scratch;
-        p.x_f32 = 1;
+    if (dq) {
+        if (rot_scratch) {
+            e = launch_rotation(h, x, B, s, 0, scratch);
+            if (e != cudaSuccess) return cuda_status(e);
+            p.x = scratch;
+            p.x_f32 = 1;
+        }
     } else if (fused_rot) {
         p.rot_b = d.hadamard_block;
         p.rot_m = paley_m(d.hadamard_block);
@@ -1327,7 +1360,7 @@ eva_status_t eva_vq_linear_run_noalloc(eva_vq_linear_t h, const void *x, int32_t
         e = launch_dequant(h, p, B, s, &dsmem, &dgrid);
         if (e != cudaSuccess) return cuda_status(e);
         h->last_grid = dgrid;
-        h->last_kernels = d.hadamard_block ? 2 : 1;
+        h->last_kernels = rot_scratch ? 2 : 1;
         h->last_path = EVA_PATH_DEQUANT_MMA;
         return EVA_OK;
     }

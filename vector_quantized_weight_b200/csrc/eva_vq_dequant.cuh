@@ -6,8 +6,9 @@
 // from the codebook (WC[WI], one 8-byte read per index whatever the batch)
 // and let tensor-core MMAs (m16n8k16, f16 in, fp32 accumulate) multiply it
 // with up to 16 tokens at a time.  Layers with a shared codebook or one
-// codebook per group of rows; no sign residual, no rotation (those keep the
-// lookup path).
+// codebook per group of rows; with one shared codebook also the 1-bit sign
+// residual (w = WC[WI] + alpha sigma, added to the rebuilt pair before its
+// MMA) and a rotated input (x~ in fp32 from the rotation kernel).
 //
 // Same repacked index units and the same CTA grid as the lookup kernel
 // (clusters of Gs slice groups x Gt row groups, split-K sums combined in
@@ -32,6 +33,41 @@ __host__ __device__ __forceinline__ int dq_subvec(int beta, int q) {
     return beta < 8 ? 4 * beta + q : 4 * (beta - 8) + q + 32;
 }
 
+// Sign units of the residual (one per slice and row tile, like the index
+// units): 512 bytes, 16 per lane, so that one 128-bit read gives lane (g, q)
+// every sign bit it multiplies.  Word w of lane L = 4 g + q: row g + 8 (w >> 1)
+// of the tile; nibble n of the word: MMA block beta = 8 (w & 1) + n, whose bit
+// e is the sign of slice input 4 dq_subvec(beta, q) + e (set: + alpha).
+constexpr int kDqSignUnitBytes = 512;
+constexpr int kDqResidUnitBytes = kDqSignUnitBytes + kAlphaUnitHalves * 2;   // + the lookup's alpha unit
+
+// Sign byte b of a unit -> (row in tile, slice input) of its bit 0 (bits
+// 0..3: inputs i..i+3 of one sub-vector; bits 4..7: the next block's).
+__host__ __device__ __forceinline__ void dq_sign_pos(int b, int t, int &row, int &kin) {
+    const int lane = b >> 4, w = (b >> 2) & 3, n = 2 * (b & 3) + (t >> 2);
+    const int g = lane >> 2, q = lane & 3, beta = 8 * (w & 1) + n;
+    row = g + 8 * (w >> 1);
+    kin = 4 * dq_subvec(beta, q) + (t & 3);
+}
+
+// signs [N][K/8] (bit k % 8 of byte k / 8: input k, LSB first) -> sign units.
+__global__ void eva_repack_signs_dq_kernel(const uint8_t *__restrict__ sg, uint8_t *__restrict__ out, int N,
+                                           int K, int T, long long total) {
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= total) return;
+    const long long unit = idx / kDqSignUnitBytes;
+    const int b = (int)(idx % kDqSignUnitBytes);
+    const int s = (int)(unit / T), tile = (int)(unit % T);
+    uint32_t v = 0;
+    for (int t = 0; t < 8; ++t) {
+        int row, kin;
+        dq_sign_pos(b, t, row, kin);
+        const int o = kTileRows * tile + row, k = kSliceK * s + kin;
+        if (o < N && k < K) v |= (uint32_t)((sg[(size_t)o * (K / 8) + (k >> 3)] >> (k & 7)) & 1u) << t;
+    }
+    out[idx] = (uint8_t)v;
+}
+
 __device__ __forceinline__ uint2 lds64(uint32_t off) { return *reinterpret_cast<const uint2 *>(eva_smem + off); }
 
 // Codebook cb replicated: entry c, copy r at c * 128 + 8 r (r = lane mod 16).
@@ -45,6 +81,50 @@ __device__ __forceinline__ void build_codebook_table(const LookupParams &p, int 
     }
 }
 
+// x~[ks + 8 lane .. + 7] of token tok for a Sylvester rotation block b
+// (p.rot_b), x~ = s . (H_b x) / sqrt(b), computed by one warp from fp16 x:
+// b <= 256, the slice holds whole blocks (warp transform of stages < b);
+// b > 256, H_b = H_{b/256} (x) H_256, so the slice (sub-block a of its block)
+// is sum_sb (-1)^popc(sb & a) H_256 x_sb over the block's sub-blocks, four
+// sub-blocks' loads in flight at a time.  Zeros past B and past K.
+__device__ __forceinline__ void dq_rotated_x8(const LookupParams &p, int tok, int ks, int lane, float (&acc)[8]) {
+    const int b = p.rot_b;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+    if (tok >= p.B) return;
+    if (b <= kSliceK) {
+        load_x8_f16(p, tok, ks + 8 * lane, acc);
+        fwht_warp256(acc, lane, b);
+    } else {
+        const int nsb = b / kSliceK, blk0 = (ks / b) * b, a = (ks - blk0) / kSliceK;
+        for (int sb0 = 0; sb0 < nsb; sb0 += 4) {
+            float v[4][8];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                if (sb0 + u < nsb) {
+                    load_x8_f16(p, tok, blk0 + (sb0 + u) * kSliceK + 8 * lane, v[u]);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) v[u][j] = 0.f;
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                if (sb0 + u >= nsb) break;
+                fwht_warp256(v[u], lane, kSliceK);
+                const bool neg = (__popc((unsigned)((sb0 + u) & a)) & 1) != 0;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[j] = neg ? acc[j] - v[u][j] : acc[j] + v[u][j];
+            }
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int k = ks + 8 * lane + j;
+        acc[j] *= (k < p.K ? (float)p.hs[k] : 0.f) * p.rot_scale;
+    }
+}
+
 // DIRECT: launched only when every CTA takes one K-slice (Gs = S), so a
 // tile's sums are final when its MMAs end and go straight from registers to
 // the owning cluster CTA's stage (no running sums in shared memory).
@@ -54,7 +134,7 @@ __device__ __forceinline__ void build_codebook_table(const LookupParams &p, int 
 // half the SM's shared memory anyway, so they keep one CTA per SM and the
 // registers that go with it.
 template <bool GROUPED, int NTG, bool DIRECT, bool RESID = false>
-constexpr int kDequantMinBlocks = (RESID || (NTG == 2 && (GROUPED || !DIRECT))) ? 1 : 2;
+constexpr int kDequantMinBlocks = (NTG == 2 && (GROUPED || !DIRECT)) ? 1 : 2;
 
 // The whole per-CTA program; eva_bid is the CTA's index within its layer.
 // RESID: the 1-bit sign residual of the 3-bit SRAM-lookup article rides on
@@ -84,7 +164,8 @@ __device__ __forceinline__ void dequant_body(const LookupParams &p, const int ev
     // Shared memory: codebook table | x stage [slice][token] | running sums
     // [tile][16][TT] (only when a CTA takes several slices) | reduction stage
     // [ceil(acc_tiles / Gs)][Gs][16][TT] | the staging mbarrier (128 bytes) |
-    // the staged index units (slice-major: unit sl * ctiles + tl).
+    // the staged index units (slice-major: unit sl * ctiles + tl) | with the
+    // residual, the same units' signs, then their alphas.
     constexpr uint32_t TAB_OFF = 0, XS_OFF = kTabBytes;
     // The layout must be the same in every CTA of a cluster (peers write into
     // the reduction stage at this CTA's offsets): size the x stage for the
@@ -99,6 +180,9 @@ __device__ __forceinline__ void dequant_body(const LookupParams &p, const int ev
     const uint32_t BAR_OFF = (STAGE_OFF + (uint32_t)((p.acc_tiles + p.Gs - 1) / p.Gs) * p.Gs * BLK_S + 127u) & ~127u;
     const uint32_t UNITS_OFF = BAR_OFF + 128u;
     const int nst = min(nsl * ctiles, p.wi_staged);   // units copied into shared memory
+    const uint32_t SG_OFF = UNITS_OFF + (uint32_t)nst * kUnitBytes;
+    const uint32_t AL_OFF = SG_OFF + (uint32_t)nst * kDqSignUnitBytes;
+    constexpr uint32_t kStagedUnitBytes = kUnitBytes + (RESID ? kDqResidUnitBytes : 0);
     const uint32_t bar = (uint32_t)__cvta_generic_to_shared(eva_smem + BAR_OFF);
 
     // ---- prologue: weights only ----
@@ -109,17 +193,27 @@ __device__ __forceinline__ void dequant_body(const LookupParams &p, const int ev
     // slice (a slice's units of this CTA are contiguous), on one mbarrier.
     if (tid == 0 && nst > 0) {
         mbar_init(bar, 1);
-        if (!p.skip_stage_copy && !EVA_BAD_S(UNITS_OFF) && !EVA_BAD_S(UNITS_OFF + (uint32_t)nst * kUnitBytes - 4u)) {
-            mbar_arrive_expect_tx(bar, (uint32_t)nst * kUnitBytes);
-            for (int sl = 0; sl < nsl; ++sl) {
-                const int cnt = min(ctiles, nst - sl * ctiles);
-                if (cnt <= 0) break;
-                const uint8_t *src = p.wi + ((size_t)(s0 + sl) * p.T + t0) * kUnitBytes;
-                const uint32_t dst = (uint32_t)__cvta_generic_to_shared(eva_smem + UNITS_OFF) +
-                                     (uint32_t)(sl * ctiles) * kUnitBytes;
-                const uint32_t bytes = (uint32_t)cnt * kUnitBytes;
-                for (uint32_t off = 0; off < bytes; off += 32768u)
-                    bulk_copy_g2s(dst + off, src + off, min(32768u, bytes - off), bar);
+        if (!p.skip_stage_copy && !EVA_BAD_S(UNITS_OFF) &&
+            !EVA_BAD_S(UNITS_OFF + (uint32_t)nst * kStagedUnitBytes - 4u)) {
+            mbar_arrive_expect_tx(bar, (uint32_t)nst * kStagedUnitBytes);
+            const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(eva_smem);
+            // One array's units [s][t0, t0 + cnt) of every slice: contiguous in
+            // global memory, placed slice-major in shared memory.
+            auto copy_units = [&](const uint8_t *base, uint32_t ubytes, uint32_t region) {
+                for (int sl = 0; sl < nsl; ++sl) {
+                    const int cnt = min(ctiles, nst - sl * ctiles);
+                    if (cnt <= 0) break;
+                    const uint8_t *src = base + ((size_t)(s0 + sl) * p.T + t0) * ubytes;
+                    const uint32_t dst = sbase + region + (uint32_t)(sl * ctiles) * ubytes;
+                    const uint32_t bytes = (uint32_t)cnt * ubytes;
+                    for (uint32_t off = 0; off < bytes; off += 32768u)
+                        bulk_copy_g2s(dst + off, src + off, min(32768u, bytes - off), bar);
+                }
+            };
+            copy_units(p.wi, kUnitBytes, UNITS_OFF);
+            if constexpr (RESID) {
+                copy_units(p.sgd, kDqSignUnitBytes, SG_OFF);
+                copy_units(reinterpret_cast<const uint8_t *>(p.al), kAlphaUnitHalves * 2, AL_OFF);
             }
         } else if (!p.skip_stage_copy) {
             mbar_arrive(bar);
@@ -132,6 +226,12 @@ __device__ __forceinline__ void dequant_body(const LookupParams &p, const int ev
         const uint32_t nt = (uint32_t)(ctiles - first);
         if (nt > 0 && !EVA_BAD_G(BUF_WI, p.wi + u * kUnitBytes, nt * kUnitBytes))
             prefetch_l2_bulk(p.wi + u * kUnitBytes, nt * kUnitBytes);
+        if constexpr (RESID) {
+            if (nt > 0 && !EVA_BAD_G(BUF_SG, p.sgd + u * kDqSignUnitBytes, nt * kDqSignUnitBytes))
+                prefetch_l2_bulk(p.sgd + u * kDqSignUnitBytes, nt * kDqSignUnitBytes);
+            if (nt > 0 && !EVA_BAD_G(BUF_AL, p.al + u * kAlphaUnitHalves, nt * kAlphaUnitHalves * 2))
+                prefetch_l2_bulk(p.al + u * kAlphaUnitHalves, nt * kAlphaUnitHalves * 2);
+        }
     }
     bool units_ready = nst == 0;
     build_codebook_table(p, cb_first, tid);
@@ -144,7 +244,22 @@ __device__ __forceinline__ void dequant_body(const LookupParams &p, const int ev
     const uint32_t lofs = 8u * (uint32_t)(lane & 15);   // this lane's copy in the table
     for (int p0 = 0; p0 < p.B; p0 += TT) {
         // x of this pass's tokens for all the CTA's slices, fp16, zeros past B / K.
-        for (int i = tid; i < nsl * TT * 32; i += kThreads) {
+        // The residual instances rotate on chip (Sylvester blocks, p.rot_b):
+        // one warp per (slice, token).
+        const bool rot_x = RESID && p.rot_b != 0;
+        if (rot_x) {
+            for (int it = warp; it < nsl * TT; it += kWarps) {
+                const int sl = it / TT, n = it - sl * TT;
+                float v[8];
+                dq_rotated_x8(p, p0 + n, (s0 + sl) * kSliceK, lane, v);
+                const uint32_t off = XS_OFF + (uint32_t)(sl * TT + n) * kXTokStride + 16u * (uint32_t)lane;
+                if (!EVA_BAD_S(off) && !EVA_BAD_S(off + 12u))
+                    *reinterpret_cast<uint4 *>(eva_smem + off) =
+                        make_uint4(pack_half2(v[0], v[1]), pack_half2(v[2], v[3]), pack_half2(v[4], v[5]),
+                                   pack_half2(v[6], v[7]));
+            }
+        }
+        for (int i = tid; i < (rot_x ? 0 : nsl * TT * 32); i += kThreads) {
             const int chunk = i & 31, n = (i >> 5) % TT, sl = i / (32 * TT);
             const int tok = p0 + n, k0 = (s0 + sl) * kSliceK + 8 * chunk;
             uint4 v = make_uint4(0u, 0u, 0u, 0u);
@@ -198,6 +313,8 @@ __device__ __forceinline__ void dequant_body(const LookupParams &p, const int ev
         // Units [0, nst) of the CTA (slice-major) come from shared memory; the
         // others stream from global memory one unit ahead (nb0, nb1).
         uint4 nb0 = make_uint4(0u, 0u, 0u, 0u), nb1 = nb0;
+        uint4 nsv = nb0;                  // residual: the unit's sign words for this lane
+        uint2 nav = make_uint2(0u, 0u);   // and the alphas of rows g, g + 8 (groups 0, 1)
         bool have_next = false;   // nb0, nb1 already hold the next (codebook, slice)'s first unit
         auto fetch = [&](int s, int tl) {
             const int u = (s - s0) * ctiles + tl;
@@ -207,9 +324,22 @@ __device__ __forceinline__ void dequant_body(const LookupParams &p, const int ev
                     nb0 = lds128(wo);
                     nb1 = lds128(wo + 512u);
                 }
+                if constexpr (RESID) {
+                    const uint32_t so = SG_OFF + (uint32_t)u * kDqSignUnitBytes + 16u * (uint32_t)lane;
+                    const uint32_t ao = AL_OFF + (uint32_t)u * (kAlphaUnitHalves * 2) + 8u * (uint32_t)g;
+                    if (!EVA_BAD_S(so) && !EVA_BAD_S(so + 12u)) nsv = lds128(so);
+                    if (!EVA_BAD_S(ao) && !EVA_BAD_S(ao + 4u)) nav = lds64(ao);
+                }
             } else {
-                const uint8_t *up = p.wi + ((size_t)s * p.T + t0 + tl) * kUnitBytes + 16 * lane;
+                const size_t un = (size_t)s * p.T + t0 + tl;
+                const uint8_t *up = p.wi + un * kUnitBytes + 16 * lane;
                 if (!EVA_BAD_G(BUF_WI, up, 16) && !EVA_BAD_G(BUF_WI, up + 512, 16)) ldg_unit(up, nb0, nb1);
+                if constexpr (RESID) {
+                    const uint8_t *sp = p.sgd + un * kDqSignUnitBytes + 16 * lane;
+                    const __half *ap = p.al + un * kAlphaUnitHalves + 4 * g;
+                    if (!EVA_BAD_G(BUF_SG, sp, 16)) nsv = ldg_stream(sp);
+                    if (!EVA_BAD_G(BUF_AL, ap, 8)) nav = __ldg(reinterpret_cast<const uint2 *>(ap));
+                }
             }
         };
         for (int cb = cb_first; cb <= cb_last; ++cb) {
@@ -351,6 +481,8 @@ __device__ __forceinline__ void dequant_body(const LookupParams &p, const int ev
                 for (int i = i0; i < i1; ++i) {
                     const int tl = warp + kWarps * i;
                     const uint32_t wv[8] = {nb0.x, nb0.y, nb0.z, nb0.w, nb1.x, nb1.y, nb1.z, nb1.w};
+                    const uint4 sv = nsv;
+                    const uint2 av = nav;
                     // One unit ahead, across slices and codebooks too: with
                     // per-group codebooks a warp often has one tile per
                     // (codebook, slice), and its next unit is then in the next one.
@@ -381,34 +513,6 @@ __device__ __forceinline__ void dequant_body(const LookupParams &p, const int ev
 #pragma unroll
                         for (int k = 0; k < 8; ++k) rot[k] = nr[k];
                     }
-                    // Residual: the sign bits of rows g, g + 8 over this slice
-                    // (word w: slice inputs 32 w .. 32 w + 31, LSB first) and their
-                    // alpha for the slice's two 128-input groups.
-                    uint32_t sgw[2][8];
-                    __half alf[2][2];
-                    if constexpr (RESID) {
-#pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            const int o = kTileRows * (t0 + tl) + g + 8 * h;
-                            const int rb = o >> 7, rr = o & 127;
-#pragma unroll
-                            for (int i4 = 0; i4 < 4; ++i4) {
-                                const int kb = 4 * s + i4;
-                                uint2 v2 = make_uint2(0u, 0u);
-                                const uint8_t *sp = p.sgb + (((size_t)rb * p.KB + kb) * 128 + rr) * 8;   // 128-row blocks
-                                if (kb < p.KB && !EVA_BAD_G(BUF_SG, sp, 8)) v2 = __ldg(reinterpret_cast<const uint2 *>(sp));
-                                sgw[h][2 * i4] = v2.x;
-                                sgw[h][2 * i4 + 1] = v2.y;
-                            }
-                            const int NG = p.K / 128;
-#pragma unroll
-                            for (int a = 0; a < 2; ++a) {
-                                const int gi = 2 * s + a;
-                                const __half *ap = p.al_rm + (size_t)o * NG + gi;
-                                alf[h][a] = (o < p.N && gi < NG && !EVA_BAD_G(BUF_AL, ap, 2)) ? __ldg(ap) : __float2half(0.f);
-                            }
-                        }
-                    }
                     // Two MMA accumulation chains per token group, one where the
                     // registers of two CTAs per SM would not hold two (16 tokens,
                     // sums pushed from registers).
@@ -429,9 +533,14 @@ __device__ __forceinline__ void dequant_body(const LookupParams &p, const int ev
                         uint2 ag = EVA_BAD_S(og) ? make_uint2(0u, 0u) : lds64(og);
                         uint2 ah = EVA_BAD_S(oh) ? make_uint2(0u, 0u) : lds64(oh);
                         if constexpr (RESID) {
-                            // Sub-vector 4 beta + q: sign nibble in word beta / 2 at bit
-                            // 16 (beta & 1) + 4 q; alpha of group beta / 8 of the slice.
-                            const int sh = 16 * (beta & 1) + 4 * q;
+                            // Sign nibble beta % 8 of word beta / 8 (row g) or 2 + beta / 8
+                            // (row g + 8); alpha of the slice's group beta / 8.
+                            const int sh = 4 * (beta & 7);
+                            const uint32_t alw[2] = {av.x, av.y};
+                            auto alpha_of = [&](int h) {
+                                const uint32_t w2 = alw[h] >> (16 * (beta >> 3));
+                                return __ushort_as_half((unsigned short)(w2 & 0xFFFFu));
+                            };
                             auto add_resid = [&](uint2 &w, uint32_t nib, __half a) {
                                 const __half na = __hneg(a);
                                 const __half2 lo = __halves2half2((nib & 1u) ? a : na, (nib & 2u) ? a : na);
@@ -442,8 +551,8 @@ __device__ __forceinline__ void dequant_body(const LookupParams &p, const int ev
                                 w.x = *reinterpret_cast<const uint32_t *>(&x0);
                                 w.y = *reinterpret_cast<const uint32_t *>(&x1);
                             };
-                            add_resid(ag, (sgw[0][beta >> 1] >> sh) & 0xFu, alf[0][beta >> 3]);
-                            add_resid(ah, (sgw[1][beta >> 1] >> sh) & 0xFu, alf[1][beta >> 3]);
+                            add_resid(ag, ((beta < 8 ? sv.x : sv.y) >> sh) & 0xFu, alpha_of(0));
+                            add_resid(ah, ((beta < 8 ? sv.z : sv.w) >> sh) & 0xFu, alpha_of(1));
                         }
 #pragma unroll
                         for (int t = 0; t < NTG; ++t)

@@ -46,10 +46,8 @@ struct LookupParams {
     int independent;         // neither x nor y is touched by the preceding kernel:
                              // run without waiting for it (wait only before exit)
     int acc_tiles;           // row tiles of the largest CTA (shared-memory layout)
-    const uint8_t *sgb;      // dequantize path with residual: signs in the row-block layout
-                             // [ceil(N/128)][KB][128][8] bytes (KB = K / 64 stages)
-    const __half *al_rm;     // dequantize path with residual: alpha [N][K/128]
-    int KB;
+    const uint8_t *sgd;      // dequantize path with residual: sign units in its own lane
+                             // order, [S][T][512] bytes (alpha: the lookup's units, al)
     int wi_staged;           // leading row tiles whose first-slice indices are copied
                              // into shared memory by one bulk copy in the prologue
     int *status;             // device error word (bit 0: the wait for the staged index
@@ -1322,8 +1320,7 @@ __global__ void __launch_bounds__(1024) eva_hadamard_kernel(const __half *__rest
     }
 }
 
-// The Paley-block rotation of rows (weights in the quantizer; inputs in the
-// two-kernel route): grid (K / b, rows), b / 2 threads at most 1024, b floats
+// The Paley-block rotation of weight rows in the quantizer: grid (K / b, rows), b / 2 threads at most 1024, b floats
 // of shared memory.  Stages h < m of the fast transform inside every
 // m-sub-block, then out[a m + c] = sum_a' H28[a'][a] y[a' m + c] in order
 // a' = 0..27, times s / sqrt(b).
@@ -1356,6 +1353,51 @@ __global__ void __launch_bounds__(1024) eva_paley_rows_kernel(const __half *__re
         }
         const int k = blk * b + i;
         xt[(size_t)tok * K + k] = (float)hs[k] * acc * scale;
+    }
+}
+
+// The Paley-block rotation of the input for the two-kernel routes (tcgen05
+// and dequantize paths): x~ = s (.) (H28 (x) H_m) x / sqrt(b) per block of
+// b = 28 m inputs.  The two Kronecker factors commute, so CTA (block, a)
+// first mixes the block's 28 sub-blocks into its own one,
+// z[c] = sum_a' H28[a'][a] x[a' m + c] (a' = 0..27, fp32), then runs the
+// m-point fast transform on z in shared memory and writes x~[a m + c]:
+// 28 CTAs per block and token and no step done twice.  Grid (28 K / b, B),
+// m threads (64..1024), m floats of shared memory.
+__global__ void __launch_bounds__(1024) eva_paley_x_kernel(const __half *__restrict__ x,
+                                                           const int8_t *__restrict__ hs,
+                                                           const int8_t *__restrict__ h28,
+                                                           float *__restrict__ xt, int K, int b, int m,
+                                                           float scale, int independent) {
+    float *sb = reinterpret_cast<float *>(eva_smem);
+    const int blk = blockIdx.x / 28, a = blockIdx.x % 28, tok = blockIdx.y;
+    pdl_launch();
+    if (!independent) pdl_wait();  // x may be the output of the preceding kernel
+    const unsigned short *xb =
+        reinterpret_cast<const unsigned short *>(x) + (size_t)tok * K + (size_t)blk * b;
+    for (int c = threadIdx.x; c < m; c += blockDim.x) {
+        float acc = 0.f;
+#pragma unroll 4
+        for (int a2 = 0; a2 < 28; ++a2) {
+            const float v = __half2float(__ushort_as_half(__ldcg(xb + a2 * m + c)));
+            acc = __ldg(h28 + a2 * 28 + a) > 0 ? acc + v : acc - v;
+        }
+        sb[c] = acc;
+    }
+    for (int h = 1; h < m; h <<= 1) {
+        __syncthreads();
+        for (int i = threadIdx.x; i < m / 2; i += blockDim.x) {
+            const int lo = (i / h) * 2 * h + (i % h);
+            const float u = sb[lo], w = sb[lo + h];
+            sb[lo] = u + w;
+            sb[lo + h] = u - w;
+        }
+    }
+    __syncthreads();
+    if (independent) pdl_wait();  // the rotated input is this handle's workspace
+    for (int c = threadIdx.x; c < m; c += blockDim.x) {
+        const int k = blk * b + a * m + c;
+        xt[(size_t)tok * K + k] = (float)hs[k] * sb[c] * scale;
     }
 }
 

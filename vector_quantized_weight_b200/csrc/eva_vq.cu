@@ -557,19 +557,24 @@ bool dequant_direct(const eva_vq_linear *h, int B) {
 
 // The dequantize kernel's residual instances rotate x on chip (the 3.125-bit
 // format has both) where that is cheap: a Sylvester block of at most 1024
-// inputs (one round of four sub-block loads per slice and token) and one
-// slice per CTA.  Measured on B200, 3.125-bit 3584 x 3584 (block 512), one
-// layer waiting for the previous one: 8.7 against 11.0 us at 4 tokens, 12.0
-// against 19.4 at 16.  Otherwise x~ comes from the standalone rotation
-// kernel: with several slices per CTA of a 2048 block the warps redo the
-// sub-block transforms one latency after the other (3584 x 14336 at 16
-// tokens: 64.0 on chip against 41.2 us); a Paley block's transform spans the
-// whole block; a rotated layer without the residual keeps the other
-// instances' registers as they are.
+// inputs (one round of four sub-block loads per slice and token), one slice
+// per CTA and at most kOnChipRotMaxTiles row tiles per CTA.  Measured on
+// B200, 3.125-bit layers (block 512), one layer waiting for the previous
+// one: 3584 x 3584 (32 tiles a CTA) 8.7 against 11.0 us at 4 tokens, 12.0
+// against 19.4 at 16; 14336 x 3584 (128 tiles a CTA) 29.0 against 27.7 at 4,
+// 35.7 against 33.5 at 16 -- with long tile loops the rotation kernel's
+// launch costs less than the rotation on the CTAs' critical path.  Otherwise
+// x~ comes from the standalone rotation kernel: with several slices per CTA
+// of a 2048 block the warps redo the sub-block transforms one latency after
+// the other (3584 x 14336 at 16 tokens: 64.0 on chip against 41.2 us); a
+// Paley block's transform spans the whole block; a rotated layer without the
+// residual keeps the other instances' registers as they are.
+constexpr int kOnChipRotMaxTiles = 64;
 bool dq_rotates_on_chip(const eva_vq_linear *h, int B) {
     const eva_vq_desc &d = h->desc;
-    return d.hadamard_block && d.hadamard_block <= 1024 && !paley_m(d.hadamard_block) && d.residual_group &&
-           dequant_direct(h, B);
+    if (!d.hadamard_block || d.hadamard_block > 1024 || paley_m(d.hadamard_block) || !d.residual_group) return false;
+    const eva_vq_linear::Plan &pl = h->dq[B > 8 ? 1 : 0];
+    return dequant_direct(h, B) && (h->T + pl.Gt - 1) / pl.Gt <= kOnChipRotMaxTiles;
 }
 
 // The dequantize kernel's fields of a call's parameters (its plan for B);

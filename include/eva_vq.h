@@ -73,9 +73,10 @@ typedef enum {
                                  rotation included; 8-bit indices, K a multiple
                                  of 64, codebook_rows 0 or a multiple of 128;
                                  AUTO takes it for B > 32 on a layer with one
-                                 shared codebook and no residual or rotation,
-                                 for B >= 8 on a residual or rotated layer, and
-                                 otherwise not.  A rotated layer runs the standalone
+                                 shared codebook (residual and rotation
+                                 included), for B >= 8 on a residual or rotated
+                                 layer with per-group codebooks, and otherwise
+                                 not.  A rotated layer runs the standalone
                                  rotation kernel first (x~ in a handle
                                  workspace of max_batch * K * 4 bytes); the
                                  handle keeps a second copy of the indices (and

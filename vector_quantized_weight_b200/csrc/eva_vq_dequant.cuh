@@ -132,7 +132,8 @@ __device__ __forceinline__ void dq_rotated_x8(const LookupParams &p, int tok, in
 // a thread): then the next layer's CTA runs its prologue beside this one.
 // The 16-token instances with running sums in shared memory take more than
 // half the SM's shared memory anyway, so they keep one CTA per SM and the
-// registers that go with it.
+// registers that go with it.  The residual instances follow the same rule
+// (124-128 registers where it asks for two CTAs per SM, no spills).
 template <bool GROUPED, int NTG, bool DIRECT, bool RESID = false>
 constexpr int kDequantMinBlocks = (NTG == 2 && (GROUPED || !DIRECT)) ? 1 : 2;
 

@@ -204,7 +204,10 @@ def test_create_accepts_order_k_rotation_descriptor():
 def test_unit_layouts_are_bijections():
     """The repack layouts (host-compilable header): every (row, sub-vector) of
     a unit appears exactly once, for byte indices and for 4-bit indices, and
-    the 4-bit inverse undoes the forward map."""
+    the 4-bit inverse undoes the forward map; every (row, input) of a
+    dequantize-path sign unit has exactly one bit, and lane (g, q)'s 16 bytes
+    hold rows g and g + 8 only, at the inputs of the sub-vectors it reads
+    (dq_subvec)."""
     src = r"""
 #include <cstdio>
 #define __host__
@@ -220,6 +223,20 @@ int main() {
         if (wi4_unit_nibble(r, j) != n) ++bad;
     }
     for (int r = 0; r < 16; ++r) for (int j = 0; j < 64; ++j) bad += (seen8[r][j] != 1) + (seen4[r][j] != 1);
+    static int seen_s[16][256];
+    for (int b = 0; b < kDqSignUnitBytes; ++b)
+        for (int t = 0; t < 8; ++t) {
+            int r, k;
+            dq_sign_pos(b, t, r, k);
+            if (r < 0 || r >= 16 || k < 0 || k >= 256) { ++bad; continue; }
+            seen_s[r][k]++;
+            const int lane = b >> 4, g = lane >> 2, q = lane & 3;
+            if ((r & 7) != g) ++bad;
+            bool read = false;
+            for (int beta = 0; beta < 16; ++beta) read |= (k >> 2) == dq_subvec(beta, q);
+            if (!read) ++bad;
+        }
+    for (int r = 0; r < 16; ++r) for (int k = 0; k < 256; ++k) bad += seen_s[r][k] != 1;
     std::printf("%d\n", bad);
     return 0;
 }

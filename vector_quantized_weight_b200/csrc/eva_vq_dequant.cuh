@@ -28,27 +28,6 @@ namespace eva {
 constexpr uint32_t kTabBytes = kCent * 16u * 8u;      // 256 centroids x 16 copies x 8 bytes
 constexpr uint32_t kXTokStride = 544u;                // bytes per staged token (512 + 32: conflict-free)
 
-// Sub-vector (within the slice) that lane quarter q reads in MMA block beta.
-__host__ __device__ __forceinline__ int dq_subvec(int beta, int q) {
-    return beta < 8 ? 4 * beta + q : 4 * (beta - 8) + q + 32;
-}
-
-// Sign units of the residual (one per slice and row tile, like the index
-// units): 512 bytes, 16 per lane, so that one 128-bit read gives lane (g, q)
-// every sign bit it multiplies.  Word w of lane L = 4 g + q: row g + 8 (w >> 1)
-// of the tile; nibble n of the word: MMA block beta = 8 (w & 1) + n, whose bit
-// e is the sign of slice input 4 dq_subvec(beta, q) + e (set: + alpha).
-constexpr int kDqSignUnitBytes = 512;
-constexpr int kDqResidUnitBytes = kDqSignUnitBytes + kAlphaUnitHalves * 2;   // + the lookup's alpha unit
-
-// Sign byte b of a unit -> (row in tile, slice input) of its bit 0 (bits
-// 0..3: inputs i..i+3 of one sub-vector; bits 4..7: the next block's).
-__host__ __device__ __forceinline__ void dq_sign_pos(int b, int t, int &row, int &kin) {
-    const int lane = b >> 4, w = (b >> 2) & 3, n = 2 * (b & 3) + (t >> 2);
-    const int g = lane >> 2, q = lane & 3, beta = 8 * (w & 1) + n;
-    row = g + 8 * (w >> 1);
-    kin = 4 * dq_subvec(beta, q) + (t & 3);
-}
 
 // signs [N][K/8] (bit k % 8 of byte k / 8: input k, LSB first) -> sign units.
 __global__ void eva_repack_signs_dq_kernel(const uint8_t *__restrict__ sg, uint8_t *__restrict__ out, int N,

@@ -97,4 +97,29 @@ __host__ __device__ __forceinline__ void alpha_unit_pos(int e, int &row, int &gr
     grp = e & 1;
 }
 
+// ------------------------------------------------ dequantize-path layouts
+//
+// Sub-vector (within the slice) that lane quarter q reads in MMA block beta of
+// the dequantize kernel (16 inputs = 4 sub-vectors per block).
+__host__ __device__ __forceinline__ int dq_subvec(int beta, int q) {
+    return beta < 8 ? 4 * beta + q : 4 * (beta - 8) + q + 32;
+}
+
+// Sign units of the residual on the dequantize path (one per slice and row
+// tile, like the index units): 512 bytes, 16 per lane, so that one 128-bit
+// read gives lane (g, q) every sign bit it multiplies.  Word w of lane
+// L = 4 g + q: row g + 8 (w >> 1) of the tile; nibble n of the word: MMA block
+// beta = 8 (w & 1) + n, whose bit e is the sign of slice input
+// 4 dq_subvec(beta, q) + e (set: + alpha).
+constexpr int kDqSignUnitBytes = 512;
+constexpr int kDqResidUnitBytes = kDqSignUnitBytes + kAlphaUnitHalves * 2;   // + the lookup's alpha unit
+
+// Bit t of sign byte b of a unit -> (row in tile, slice input).
+__host__ __device__ __forceinline__ void dq_sign_pos(int b, int t, int &row, int &kin) {
+    const int lane = b >> 4, w = (b >> 2) & 3, n = 2 * (b & 3) + (t >> 2);
+    const int g = lane >> 2, q = lane & 3, beta = 8 * (w & 1) + n;
+    row = g + 8 * (w >> 1);
+    kin = 4 * dq_subvec(beta, q) + (t & 3);
+}
+
 }  // namespace eva

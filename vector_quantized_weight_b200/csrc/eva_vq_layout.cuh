@@ -1,6 +1,7 @@
 // eva_vq_layout.cuh -- data layout of the repacked weights and the shared-memory
 // output-codebook image, shared by the create-time repack, the unpack test hook
-// and the lookup kernels.
+// and the lookup kernels; at the end, the dequantize kernel's lane order of
+// sub-vectors and residual sign units.
 //
 // Work unit: one tile of 16 output rows (the M of one tensor-core MMA) times one
 // K-slice of 64 sub-vectors (256 inputs).  A unit holds 1024 index bytes.

@@ -78,9 +78,11 @@ typedef enum {
                                  layer with per-group codebooks, and otherwise
                                  not.  A rotated layer runs the standalone
                                  rotation kernel first (x~ in a handle
-                                 workspace of max_batch * K * 4 bytes); the
-                                 handle keeps a second copy of the indices (and
-                                 signs) in 128-row blocks for this path.         */
+                                 workspace of max_batch * K * 4 bytes); a
+                                 handle that may take this path (forced, or
+                                 AUTO with a max_batch it applies to) keeps a
+                                 second copy of the indices (and signs) in
+                                 128-row blocks for it.                          */
 } eva_path_t;
 
 typedef struct {

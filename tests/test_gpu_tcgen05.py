@@ -110,3 +110,31 @@ def test_tcgen05_rejects_layers_it_cannot_take():
         with pytest.raises(eva_vq.EvaError) as ei:
             eva_vq.from_layer(synth.make_layer(shape, 1), max_batch=8, path=eva_vq.EVA_PATH_TCGEN05)
         assert ei.value.status == eva_vq.EVA_ERR_UNSUPPORTED
+
+
+def test_row_block_copy_only_where_the_path_can_run():
+    """A handle keeps the tcgen05 path's row-block copy of the indices only
+    where that path can run: AUTO with max_batch past 32 and one shared
+    codebook (4096 x 4096: about 4 MB more than at 32), never for per-group
+    codebooks, whose batches the warp-level path takes."""
+    import torch
+    from vector_quantized_weight_b200 import eva_vq
+
+    def footprint(shape, **kw):
+        layer = synth.make_layer(shape, 12)
+        wc = torch.from_numpy(layer.wc).cuda()
+        wi = torch.from_numpy(layer.wi).cuda()
+        torch.cuda.synchronize()
+        free0 = torch.cuda.mem_get_info()[0]
+        lin = eva_vq.VQLinear(wc, wi, codebook_rows=shape.codebook_rows, **kw)
+        torch.cuda.synchronize()
+        used = free0 - torch.cuda.mem_get_info()[0]
+        lin.close()
+        torch.cuda.synchronize()
+        return used
+
+    plain = synth.LayerShape("l7b", 4096, 4096)
+    copy = plain.N * plain.K // 4
+    assert footprint(plain, max_batch=33) - footprint(plain, max_batch=32) >= 0.9 * copy
+    grouped = synth.LayerShape("l70b_part", 4096, 4096, codebook_rows=128)
+    assert footprint(grouped, max_batch=64) - footprint(grouped, max_batch=32) < 0.75 * copy

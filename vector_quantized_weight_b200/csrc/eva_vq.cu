@@ -651,6 +651,14 @@ bool use_three_per_sm(const eva_vq_linear *h, int B, int independent) {
 constexpr int kTcMinBatch = 33;
 constexpr int kTcResidMinBatch = 8;
 
+// Whether AUTO can ever pick the tcgen05 path for this handle (the rule of
+// use_tc at the handle's largest batch): only then does create plan it and
+// keep its row-block copies of the indices and signs.
+bool auto_may_use_tc(const eva_vq_linear *h) {
+    if (h->dq_ok) return h->desc.codebook_rows == 0 && h->desc.max_batch >= kTcMinBatch;
+    return h->desc.max_batch >= kTcResidMinBatch;
+}
+
 bool use_tc(const eva_vq_linear *h, int B) {
     if (!h->tc_ok) return false;
     if (h->desc.path == EVA_PATH_TCGEN05) return true;
@@ -829,8 +837,7 @@ eva_status_t eva_vq_linear_create(eva_vq_linear_t *out, const eva_vq_desc *desc,
             return EVA_ERR_UNSUPPORTED;
         }
     }
-    if (tc_layer_ok(*desc) &&
-        (desc->path == EVA_PATH_TCGEN05 || (desc->path == EVA_PATH_AUTO && desc->max_batch >= kDequantMinBatch))) {
+    if (tc_layer_ok(*desc) && (desc->path == EVA_PATH_TCGEN05 || (desc->path == EVA_PATH_AUTO && auto_may_use_tc(h)))) {
         // Plans for the padded batches up to max_batch; a batch whose padded
         // size has no plan (its x range does not fit in shared memory) runs
         // as several launches of the largest size that has one.
